@@ -1,0 +1,209 @@
+"""Thin ctypes binding of libcce.so and the autograd wrapper ``linear_cross_entropy``.
+
+Argument marshalling only: every step of the forward and the backward runs in the
+library's CUDA kernels. torch provides device memory and the current stream.
+The library is loaded on first use; a missing library or a machine without a
+CUDA device raises ``CCEError`` (there is no fallback of any kind).
+
+API shape follows the mlx-cross-entropy README ("API" table and "Usage"):
+``linear_cross_entropy(e, c, targets, reduction="mean", ignore_index=-100)`` with
+``[..., D]`` hidden states flattened to ``[N, D]`` and, for ``reduction="none"``,
+the per-token loss returned in the targets' shape.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcce.so")
+
+REDUCTION_CODES = {"none": 0, "mean": 1, "sum": 2}
+STATUS_NAMES = {
+    0: "CCE_OK",
+    1: "CCE_ERR_INVALID_ARG",
+    2: "CCE_ERR_UNSUPPORTED",
+    3: "CCE_ERR_WORKSPACE",
+    4: "CCE_ERR_TARGET_RANGE",
+    5: "CCE_ERR_DEVICE_TIMEOUT",
+    6: "CCE_ERR_CUDA",
+}
+DEFAULT_FILTER_EPS = 2.0 ** -12
+
+
+class CCEError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int64),
+        ("D", ctypes.c_int64),
+        ("V", ctypes.c_int64),
+        ("ignore_index", ctypes.c_int64),
+        ("reduction", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
+# Every symbol include/cce.h declares, with its ctypes signature.
+_VP, _SZ, _I32, _I64, _F32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+_PP = ctypes.POINTER(Problem)
+SIGNATURES = {
+    "cce_tile_max_len": (_I64, [_PP]),
+    "cce_backward_tile_shape": (None, [ctypes.POINTER(_I32), ctypes.POINTER(_I32)]),
+    "cce_forward_workspace_size": (_SZ, [_PP]),
+    "cce_backward_workspace_size": (_SZ, [_PP, _I32]),
+    "cce_forward": (_I32, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "cce_backward": (_I32, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _F32, _VP, _VP, _I32, _VP, _VP, _SZ, _VP]),
+    "cce_check_device_error": (_I32, [_VP, _VP]),
+    "cce_status_string": (ctypes.c_char_p, [_I32]),
+    "cce_last_error_message": (ctypes.c_char_p, []),
+    "cce_version": (_I32, []),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libcce.so (once) and declare its signatures. Raises CCEError if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise CCEError(6, f"{path} not found: build it with `python -m linear_cross_entropy_06_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        msg = _lib.cce_last_error_message().decode() if _lib is not None else ""
+        raise CCEError(status, msg)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _problem(N: int, D: int, V: int, ignore_index: int, reduction: str) -> Problem:
+    if reduction not in REDUCTION_CODES:
+        raise ValueError(f"reduction must be one of {tuple(REDUCTION_CODES)}, got {reduction!r}")
+    return Problem(N, D, V, ignore_index, REDUCTION_CODES[reduction], 0)
+
+
+def _require_cuda(*tensors: torch.Tensor) -> torch.device:
+    dev = tensors[0].device
+    if dev.type != "cuda":
+        raise CCEError(1, "inputs must be CUDA tensors: there is no CPU path")
+    for t in tensors:
+        if t.device != dev:
+            raise CCEError(1, "all inputs must be on the same device")
+    return dev
+
+
+def backward_tile_shape() -> Tuple[int, int]:
+    lib = load_library()
+    r, c = _I32(), _I32()
+    lib.cce_backward_tile_shape(ctypes.byref(r), ctypes.byref(c))
+    return r.value, c.value
+
+
+def cce_forward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, ignore_index: int = -100,
+                reduction: str = "mean", check: bool = False):
+    """Run the forward. Returns (loss, lse, tile_max, count) as device tensors."""
+    lib = load_library()
+    dev = _require_cuda(E, C, targets)
+    E, C, targets = E.contiguous(), C.contiguous(), targets.contiguous()
+    N, D = E.shape
+    V = C.shape[0]
+    p = _problem(N, D, V, ignore_index, reduction)
+    loss = torch.empty(N if reduction == "none" else 1, device=dev, dtype=torch.float32)
+    lse = torch.empty(N, device=dev, dtype=torch.float32)
+    tm_len = lib.cce_tile_max_len(ctypes.byref(p))
+    if tm_len < 0:
+        raise CCEError(1, f"bad problem N={N} D={D} V={V}")
+    tile_max = torch.empty(max(tm_len, 1), device=dev, dtype=torch.float32)
+    count = torch.empty(1, device=dev, dtype=torch.int64)
+    ws_bytes = lib.cce_forward_workspace_size(ctypes.byref(p))
+    ws = torch.empty(max(ws_bytes, 1), device=dev, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        _check(lib.cce_forward(ctypes.byref(p), _ptr(E), _ptr(C), _ptr(targets), _ptr(loss), _ptr(lse),
+                               _ptr(tile_max), _ptr(count), _ptr(ws), ws_bytes, _stream(dev)))
+        if check:
+            _check(lib.cce_check_device_error(_ptr(ws), _stream(dev)))
+    return loss, lse, tile_max, count
+
+
+def cce_backward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, lse: torch.Tensor,
+                 tile_max: torch.Tensor, count: torch.Tensor, grad_out: torch.Tensor,
+                 filter_eps: float = DEFAULT_FILTER_EPS, ignore_index: int = -100,
+                 reduction: str = "mean", out_fp32: bool = False, check: bool = False):
+    """Run the backward. Returns (dE, dC, filtered_tiles) as device tensors."""
+    lib = load_library()
+    dev = _require_cuda(E, C, targets, lse, tile_max, count)
+    E, C, targets = E.contiguous(), C.contiguous(), targets.contiguous()
+    N, D = E.shape
+    V = C.shape[0]
+    p = _problem(N, D, V, ignore_index, reduction)
+    g = grad_out.to(device=dev, dtype=torch.float32).reshape(-1).contiguous()
+    out_dtype = torch.float32 if out_fp32 else torch.bfloat16
+    dE = torch.empty(N, D, device=dev, dtype=out_dtype)
+    dC = torch.empty(V, D, device=dev, dtype=out_dtype)
+    filtered = torch.empty(1, device=dev, dtype=torch.int64)
+    ws_bytes = lib.cce_backward_workspace_size(ctypes.byref(p), int(out_fp32))
+    ws = torch.empty(max(ws_bytes, 1), device=dev, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        _check(lib.cce_backward(ctypes.byref(p), _ptr(E), _ptr(C), _ptr(targets), _ptr(lse), _ptr(tile_max),
+                                _ptr(count), _ptr(g), float(filter_eps), _ptr(dE), _ptr(dC), int(out_fp32),
+                                _ptr(filtered), _ptr(ws), ws_bytes, _stream(dev)))
+        if check:
+            _check(lib.cce_check_device_error(_ptr(ws), _stream(dev)))
+    return dE, dC, filtered
+
+
+class _LinearCrossEntropy(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, E, C, targets, ignore_index, reduction, filter_eps):
+        loss, lse, tile_max, count = cce_forward(E, C, targets, ignore_index, reduction)
+        ctx.save_for_backward(E, C, targets, lse, tile_max, count)
+        ctx.cfg = (ignore_index, reduction, filter_eps)
+        return loss if reduction == "none" else loss.reshape(())
+
+    @staticmethod
+    def backward(ctx, grad_loss):
+        E, C, targets, lse, tile_max, count = ctx.saved_tensors
+        ignore_index, reduction, filter_eps = ctx.cfg
+        dE, dC, _ = cce_backward(E, C, targets, lse, tile_max, count, grad_loss, filter_eps,
+                                 ignore_index, reduction, out_fp32=False)
+        return dE.to(E.dtype), dC.to(C.dtype), None, None, None, None
+
+
+def linear_cross_entropy(e: torch.Tensor, c: torch.Tensor, targets: torch.Tensor, reduction: str = "mean",
+                         ignore_index: int = -100, filter_eps: float = DEFAULT_FILTER_EPS) -> torch.Tensor:
+    """Cross-entropy of softmax(e @ c.T) at ``targets`` without materialising the logits.
+
+    e: [..., D] bf16 hidden states; c: [V, D] bf16 classifier; targets: [...] int64.
+    Returns a scalar (mean/sum) or the per-token loss in the shape of ``targets`` (none).
+    """
+    if e.shape[:-1] != targets.shape:
+        raise ValueError(f"targets shape {tuple(targets.shape)} must equal e.shape[:-1] {tuple(e.shape[:-1])}")
+    lead = targets.shape
+    E = e.reshape(-1, e.shape[-1])
+    t = targets.reshape(-1).to(torch.int64)
+    out = _LinearCrossEntropy.apply(E, c, t, ignore_index, reduction, filter_eps)
+    return out.reshape(lead) if reduction == "none" else out
