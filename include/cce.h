@@ -27,6 +27,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define CCE_API __attribute__((visibility("default")))
+#else
+#define CCE_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -65,18 +71,18 @@ typedef struct {
 
 /* Number of floats in the saved tile-max buffer: ceil(V / 128) * N. Layout [ceil(V/128), N]:
  * entry (j, r) is max_{v in [128 j, 128 j + 128) and v < V} z[r, v]. -1 for a bad problem. */
-int64_t cce_tile_max_len(const cce_problem* p);
+CCE_API int64_t cce_tile_max_len(const cce_problem* p);
 
 /* Rows and vocabulary columns of one backward tile. The skip rule of the backward decides per
  * tile of this size (mlx-cross-entropy README, "How it works" item 2). */
-void cce_backward_tile_shape(int32_t* tile_rows, int32_t* tile_cols);
+CCE_API void cce_backward_tile_shape(int32_t* tile_rows, int32_t* tile_cols);
 
 /* Bytes of device workspace cce_forward() needs (0 for a bad problem). */
-size_t cce_forward_workspace_size(const cce_problem* p);
+CCE_API size_t cce_forward_workspace_size(const cce_problem* p);
 
 /* Bytes of device workspace cce_backward() needs. With out_fp32 = 0 it holds the fp32
  * accumulators of dE and dC, (N + V) * D * 4 bytes; never anything of size N * V. */
-size_t cce_backward_workspace_size(const cce_problem* p, int32_t out_fp32);
+CCE_API size_t cce_backward_workspace_size(const cce_problem* p, int32_t out_fp32);
 
 /*
  * Forward: loss and per-row LSE without materialising the logits.
@@ -95,7 +101,7 @@ size_t cce_backward_workspace_size(const cce_problem* p, int32_t out_fp32);
  *           it also holds the device error word read by cce_check_device_error().
  * N = 0 is allowed (loss 0, count 0).
  */
-cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
+CCE_API cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
                        float* loss, float* lse, float* tile_max, int64_t* count, void* workspace,
                        size_t workspace_bytes, cce_stream_t stream);
 
@@ -116,7 +122,7 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
  *  filtered_tiles device int64 [1]: number of skipped tiles
  *  workspace: device scratch of at least cce_backward_workspace_size(p, out_fp32) bytes.
  */
-cce_status cce_backward(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
+CCE_API cce_status cce_backward(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
                         const float* lse, const float* tile_max, const int64_t* count,
                         const float* grad_out, float filter_eps, void* dE, void* dC, int32_t out_fp32,
                         int64_t* filtered_tiles, void* workspace, size_t workspace_bytes,
@@ -125,16 +131,16 @@ cce_status cce_backward(const cce_problem* p, const void* E, const void* C, cons
 /* Synchronises `stream`, then reads and clears the device error word kept at the start of
  * `workspace` (a forward or backward workspace passed to an earlier call on that stream).
  * Returns CCE_OK, CCE_ERR_TARGET_RANGE, CCE_ERR_DEVICE_TIMEOUT or CCE_ERR_CUDA. */
-cce_status cce_check_device_error(void* workspace, cce_stream_t stream);
+CCE_API cce_status cce_check_device_error(void* workspace, cce_stream_t stream);
 
 /* Static description of a status code. */
-const char* cce_status_string(cce_status s);
+CCE_API const char* cce_status_string(cce_status s);
 
 /* Detail of the last failing call on the calling thread ("" if none). */
-const char* cce_last_error_message(void);
+CCE_API const char* cce_last_error_message(void);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
-int32_t cce_version(void);
+CCE_API int32_t cce_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,352 @@
+// The C ABI of libcce.so (declared in include/cce.h): argument checks, workspace carving, TMA
+// descriptor encoding and the launch sequence of each call. Host code only.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+#include <string>
+
+#include "cce.h"
+#include "cce_internal.h"
+
+namespace {
+
+constexpr int32_t kVersion = 100;  // 0.1.0
+constexpr size_t kHeaderBytes = 256;
+constexpr size_t kAlign = 256;
+
+thread_local std::string g_last_error;
+
+cce_status fail(cce_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+cce_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(CCE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Layout of the error word area at the start of every workspace.
+struct WsHeader {
+  int err;
+  int num_tiles;
+};
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+bool problem_ok(const cce_problem* p, bool set_error) {
+  auto bad = [&](const char* msg) {
+    if (set_error) fail(CCE_ERR_INVALID_ARG, "%s", msg);
+    return false;
+  };
+  if (p == nullptr) return bad("problem is NULL");
+  if (p->N < 0) return bad("N must be >= 0");
+  if (p->D < 8 || p->D % 8 != 0) return bad("D must be a positive multiple of 8");
+  if (p->V < 1) return bad("V must be >= 1");
+  if (p->reduction < 0 || p->reduction > 2) return bad("reduction must be 0 (none), 1 (mean) or 2 (sum)");
+  if (p->reserved != 0) return bad("reserved must be 0");
+  // Kernel indices are 32-bit for rows and tiles; keep every count well inside that.
+  if (p->N >= (int64_t(1) << 31) - 256 || p->V >= (int64_t(1) << 31) - 256 || p->D >= (int64_t(1) << 24))
+    return bad("N, V or D too large");
+  if (ceil_div(p->N, cce::kBwdBM) * ceil_div(p->V, cce::kBwdBN) >= (int64_t(1) << 31))
+    return bad("too many backward tiles");
+  return true;
+}
+
+struct FwdWs {
+  WsHeader* hdr;
+  float* tile_sum;
+  float* z_target;
+  float* loss_rows;
+  size_t bytes;
+};
+
+FwdWs carve_fwd(const cce_problem* p, void* base) {
+  const int64_t T = ceil_div(p->V, cce::kSubTile);
+  FwdWs w{};
+  size_t off = kHeaderBytes;
+  char* b = static_cast<char*>(base);
+  w.hdr = reinterpret_cast<WsHeader*>(b);
+  w.tile_sum = reinterpret_cast<float*>(b + off);
+  off = align_up(off + sizeof(float) * static_cast<size_t>(T * p->N));
+  w.z_target = reinterpret_cast<float*>(b + off);
+  off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
+  w.loss_rows = reinterpret_cast<float*>(b + off);
+  off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
+  w.bytes = off;
+  return w;
+}
+
+struct BwdWs {
+  WsHeader* hdr;
+  float* scale;
+  int2* tiles;
+  float* dE_acc;
+  float* dC_acc;
+  size_t bytes;
+};
+
+BwdWs carve_bwd(const cce_problem* p, int32_t out_fp32, void* base) {
+  const int64_t nb = ceil_div(p->N, cce::kBwdBM), nt = ceil_div(p->V, cce::kBwdBN);
+  BwdWs w{};
+  size_t off = kHeaderBytes;
+  char* b = static_cast<char*>(base);
+  w.hdr = reinterpret_cast<WsHeader*>(b);
+  w.scale = reinterpret_cast<float*>(b + off);
+  off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
+  w.tiles = reinterpret_cast<int2*>(b + off);
+  off = align_up(off + sizeof(int2) * static_cast<size_t>(nb * nt));
+  if (!out_fp32) {
+    w.dE_acc = reinterpret_cast<float*>(b + off);
+    off = align_up(off + sizeof(float) * static_cast<size_t>(p->N * p->D));
+    w.dC_acc = reinterpret_cast<float*>(b + off);
+    off = align_up(off + sizeof(float) * static_cast<size_t>(p->V * p->D));
+  }
+  w.bytes = off;
+  return w;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+// ---------------------------------------------------------------------------------------------
+// Device checks and TMA descriptors
+// ---------------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+cce_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (g_encode == nullptr) return fail(CCE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  return CCE_OK;
+}
+
+cce_status check_device(int* num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(CCE_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a (B200)", dev, major,
+                minor);
+  e = cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  return CCE_OK;
+}
+
+// 2-D row-major tensor [rows, cols] with contiguous rows, box [box_rows, box_cols], 128B swizzle.
+cce_status make_map(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem, const void* ptr, int64_t rows,
+                    int64_t cols, uint32_t box_cols, uint32_t box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * elem};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, dtype, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CCE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return CCE_OK;
+}
+
+uint64_t wait_timeout_ns() {
+  const char* s = std::getenv("CCE_WAIT_TIMEOUT_MS");
+  double ms = s ? std::atof(s) : 4000.0;
+  if (!(ms > 0)) ms = 4000.0;
+  return static_cast<uint64_t>(ms * 1e6);
+}
+
+#define CCE_TRY(expr)                                \
+  do {                                               \
+    cudaError_t e_ = (expr);                         \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #expr); \
+  } while (0)
+
+#define CCE_CHECK(expr)            \
+  do {                             \
+    cce_status s_ = (expr);        \
+    if (s_ != CCE_OK) return s_;   \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int32_t cce_version(void) { return kVersion; }
+
+const char* cce_status_string(cce_status s) {
+  switch (s) {
+    case CCE_OK: return "ok";
+    case CCE_ERR_INVALID_ARG: return "invalid argument";
+    case CCE_ERR_UNSUPPORTED: return "unsupported device or size";
+    case CCE_ERR_WORKSPACE: return "workspace too small";
+    case CCE_ERR_TARGET_RANGE: return "target outside [0, V) and not ignore_index";
+    case CCE_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case CCE_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* cce_last_error_message(void) { return g_last_error.c_str(); }
+
+int64_t cce_tile_max_len(const cce_problem* p) {
+  if (!problem_ok(p, false)) return -1;
+  return ceil_div(p->V, cce::kSubTile) * p->N;
+}
+
+void cce_backward_tile_shape(int32_t* tile_rows, int32_t* tile_cols) {
+  if (tile_rows) *tile_rows = cce::kBwdBM;
+  if (tile_cols) *tile_cols = cce::kBwdBN;
+}
+
+size_t cce_forward_workspace_size(const cce_problem* p) {
+  if (!problem_ok(p, false)) return 0;
+  return carve_fwd(p, nullptr).bytes;
+}
+
+size_t cce_backward_workspace_size(const cce_problem* p, int32_t out_fp32) {
+  if (!problem_ok(p, false)) return 0;
+  return carve_bwd(p, out_fp32 ? 1 : 0, nullptr).bytes;
+}
+
+cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const int64_t* targets, float* loss,
+                       float* lse, float* tile_max, int64_t* count, void* workspace, size_t workspace_bytes,
+                       cce_stream_t stream) {
+  g_last_error.clear();
+  if (!problem_ok(p, true)) return CCE_ERR_INVALID_ARG;
+  const bool has_rows = p->N > 0;
+  if (C == nullptr || loss == nullptr || count == nullptr || workspace == nullptr ||
+      (has_rows && (E == nullptr || targets == nullptr || lse == nullptr || tile_max == nullptr)))
+    return fail(CCE_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(E) || !aligned16(C) || !aligned16(workspace))
+    return fail(CCE_ERR_INVALID_ARG, "E, C and workspace must be 16-byte aligned");
+  const FwdWs w = carve_fwd(p, workspace);
+  if (workspace_bytes < w.bytes)
+    return fail(CCE_ERR_WORKSPACE, "forward workspace is %zu bytes, needs %zu", workspace_bytes, w.bytes);
+  int num_sms = 0;
+  CCE_CHECK(check_device(&num_sms));
+  CCE_CHECK(get_encoder());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t N = p->N, D = p->D, V = p->V, T = ceil_div(V, cce::kSubTile);
+  const auto* Eb = static_cast<const __nv_bfloat16*>(E);
+  const auto* Cb = static_cast<const __nv_bfloat16*>(C);
+
+  CCE_TRY(cudaMemsetAsync(w.hdr, 0, sizeof(WsHeader), s));
+  if (has_rows) {
+    cce::FwdLaunch L{};
+    CCE_CHECK(make_map(&L.tmE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kFwdBM));
+    CCE_CHECK(make_map(&L.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, cce::kFwdBN));
+    L.N = static_cast<int>(N);
+    L.D = static_cast<int>(D);
+    L.V = static_cast<int>(V);
+    L.T = static_cast<int>(T);
+    L.tile_max = tile_max;
+    L.tile_sum = w.tile_sum;
+    L.err = &w.hdr->err;
+    L.timeout_ns = wait_timeout_ns();
+    L.num_sms = num_sms;
+    CCE_TRY(cce::launch_target_logit(Eb, Cb, targets, N, D, V, p->ignore_index, w.z_target, &w.hdr->err, s));
+    CCE_TRY(cce::launch_fwd_lse(L, s));
+    float* rows_out = p->reduction == CCE_REDUCTION_NONE ? loss : w.loss_rows;
+    CCE_TRY(cce::launch_lse_loss(tile_max, w.tile_sum, w.z_target, targets, N, T, p->ignore_index, V, lse, rows_out,
+                                 s));
+  }
+  CCE_TRY(cce::launch_loss_reduce(w.loss_rows, targets, N, p->ignore_index, p->reduction, loss, count, s));
+  return CCE_OK;
+}
+
+cce_status cce_backward(const cce_problem* p, const void* E, const void* C, const int64_t* targets, const float* lse,
+                        const float* tile_max, const int64_t* count, const float* grad_out, float filter_eps,
+                        void* dE, void* dC, int32_t out_fp32, int64_t* filtered_tiles, void* workspace,
+                        size_t workspace_bytes, cce_stream_t stream) {
+  g_last_error.clear();
+  if (!problem_ok(p, true)) return CCE_ERR_INVALID_ARG;
+  const bool has_rows = p->N > 0;
+  if (C == nullptr || dC == nullptr || count == nullptr || filtered_tiles == nullptr || workspace == nullptr ||
+      (has_rows && (E == nullptr || targets == nullptr || lse == nullptr || tile_max == nullptr || dE == nullptr ||
+                    grad_out == nullptr)))
+    return fail(CCE_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(E) || !aligned16(C) || !aligned16(dE) || !aligned16(dC) || !aligned16(workspace))
+    return fail(CCE_ERR_INVALID_ARG, "E, C, dE, dC and workspace must be 16-byte aligned");
+  if (std::isnan(filter_eps)) return fail(CCE_ERR_INVALID_ARG, "filter_eps is NaN");
+  out_fp32 = out_fp32 ? 1 : 0;
+  const BwdWs w = carve_bwd(p, out_fp32, workspace);
+  if (workspace_bytes < w.bytes)
+    return fail(CCE_ERR_WORKSPACE, "backward workspace is %zu bytes, needs %zu", workspace_bytes, w.bytes);
+  int num_sms = 0;
+  CCE_CHECK(check_device(&num_sms));
+  CCE_CHECK(get_encoder());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t N = p->N, D = p->D, V = p->V, T = ceil_div(V, cce::kSubTile);
+  const auto* Eb = static_cast<const __nv_bfloat16*>(E);
+  const auto* Cb = static_cast<const __nv_bfloat16*>(C);
+  float* dE_acc = out_fp32 ? static_cast<float*>(dE) : w.dE_acc;
+  float* dC_acc = out_fp32 ? static_cast<float*>(dC) : w.dC_acc;
+
+  CCE_TRY(cudaMemsetAsync(w.hdr, 0, sizeof(WsHeader), s));
+  CCE_TRY(cce::launch_row_scale(targets, count, grad_out, N, p->ignore_index, p->reduction, w.scale,
+                                &w.hdr->num_tiles, s));
+  CCE_TRY(cce::launch_tile_mask(tile_max, lse, targets, N, V, T, p->ignore_index, filter_eps, w.tiles,
+                                &w.hdr->num_tiles, filtered_tiles, s));
+  CCE_TRY(cce::launch_grad_init(Eb, Cb, targets, w.scale, N, D, V, p->ignore_index, dE_acc, dC_acc, s));
+  if (has_rows) {
+    cce::BwdLaunch L{};
+    CCE_CHECK(make_map(&L.tmE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kBwdBM));
+    CCE_CHECK(make_map(&L.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, cce::kBwdBN));
+    CCE_CHECK(make_map(&L.tmdE, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dE_acc, N, D, 32, 32));
+    CCE_CHECK(make_map(&L.tmdC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dC_acc, V, D, 32, 32));
+    L.N = static_cast<int>(N);
+    L.D = static_cast<int>(D);
+    L.V = static_cast<int>(V);
+    L.lse = lse;
+    L.scale = w.scale;
+    L.tiles = w.tiles;
+    L.num_tiles = &w.hdr->num_tiles;
+    L.err = &w.hdr->err;
+    L.timeout_ns = wait_timeout_ns();
+    L.num_sms = num_sms;
+    CCE_TRY(cce::launch_bwd_grad(L, s));
+  }
+  if (!out_fp32) {
+    CCE_TRY(cce::launch_to_bf16(dE_acc, static_cast<__nv_bfloat16*>(dE), N * D, s));
+    CCE_TRY(cce::launch_to_bf16(dC_acc, static_cast<__nv_bfloat16*>(dC), V * D, s));
+  }
+  return CCE_OK;
+}
+
+cce_status cce_check_device_error(void* workspace, cce_stream_t stream) {
+  if (workspace == nullptr) return fail(CCE_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int err = 0;
+  e = cudaMemcpy(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+  if (err != 0) {
+    const int zero = 0;
+    cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    const cce_status st = static_cast<cce_status>(err);
+    return fail(st, "device reported: %s", cce_status_string(st));
+  }
+  return CCE_OK;
+}
+
+}  // extern "C"

@@ -36,9 +36,9 @@ IGNORE_INDEX = -100
 
 # Peaking factor per (D, V, target law), from oracle/calibrate_alpha.py.
 ALPHA = {
-    (2048, 128256, "uniform"): 11.45,
-    (2304, 256000, "uniform"): 12.15,
-    (4096, 128256, "zipf"): 11.45,
+    (2048, 128256, "uniform"): 11.2,  # mean p_target 0.301
+    (2304, 256000, "uniform"): 11.98,  # mean p_target 0.298
+    (4096, 128256, "zipf"): 11.27,  # mean p_target 0.300
 }
 
 
@@ -104,7 +104,7 @@ def make_inputs(name_or_workload, *, N: Optional[int] = None, D: Optional[int] =
     seed = w.seed if seed is None else seed
     ignore_frac = w.ignore_frac if ignore_frac is None else ignore_frac
     if alpha is None:
-        alpha = ALPHA.get((D, V, w.targets), 11.45) if w.peaked else 0.0
+        alpha = ALPHA.get((D, V, w.targets), 11.27) if w.peaked else 0.0
     keep_fp32 = (w.name == "tiny") if keep_fp32 is None else keep_fp32
     rng = np.random.default_rng(seed)
 

@@ -341,3 +341,58 @@ def sampled(E, C, targets, rows: Sequence[int], cols: Sequence[int], grad_out=1.
     borderline = int((np.abs(margin - ln_eps) < window).sum()) if filter_eps > 0 else 0
     return SampledResult(lse, nll, count, reduce_loss(nll, count, reduction), margin,
                          int(skip_all.sum()), borderline, rows, dE_rows, cols, dC_cols)
+
+
+@dataclass
+class RowBlockResult:
+    rows: np.ndarray  # every row of the chosen blocks, ascending
+    lse: np.ndarray
+    nll: np.ndarray
+    margin: np.ndarray  # [len(blocks), ceil(V/tile_n)]
+    filtered: int  # skipped tiles among the chosen blocks
+    dE: np.ndarray  # [len(rows), D]
+
+
+def row_blocks(E, C, targets, blocks: Sequence[int], grad_out=1.0, ignore_index: int = -100,
+               reduction: str = "mean", filter_eps: float = 2.0 ** -12, tile_m: int = 128,
+               tile_n: int = 256) -> RowBlockResult:
+    """Exact results for whole row blocks of the tile grid.
+
+    A tile's skip decision depends only on the rows of its own row block, and a
+    row's dE depends only on its own logits and those decisions, so evaluating
+    complete blocks gives their LSE, loss, decisions and dE exactly. The row
+    count used by ``mean`` comes from all targets.
+    """
+    E64, C64, t = _f64(E), _f64(C), _i64(targets)
+    N, V = E64.shape[0], C64.shape[0]
+    validate_targets(t, V, ignore_index)
+    count = int((t != ignore_index).sum())
+    scale_all = row_scale(t, ignore_index, reduction, grad_out, count)
+    rows = np.concatenate([np.arange(b * tile_m, min((b + 1) * tile_m, N)) for b in sorted(blocks)])
+    lse = np.empty(len(rows))
+    nll = np.empty(len(rows))
+    margins = []
+    dE = np.zeros((len(rows), E64.shape[1]))
+    filtered = 0
+    pos = 0
+    for b in sorted(blocks):
+        rr = np.arange(b * tile_m, min((b + 1) * tile_m, N))
+        z = E64[rr] @ C64.T
+        l = log_sum_exp_rows(z)
+        tb = t[rr]
+        vb = tb != ignore_index
+        m = tile_log_margin(z - l[:, None], vb, tile_m, tile_n)
+        skip = filtered_tiles(m, filter_eps)
+        filtered += int(skip.sum())
+        p = softmax_rows(z, l)
+        for tt in np.flatnonzero(skip[0]):
+            p[:, tt * tile_n:(tt + 1) * tile_n] = 0.0
+        G = scale_all[rr][:, None] * p
+        G[np.flatnonzero(vb), tb[vb]] -= scale_all[rr][vb]
+        zt = np.where(vb, z[np.arange(len(rr)), np.where(vb, tb, 0)], 0.0)
+        lse[pos:pos + len(rr)] = l
+        nll[pos:pos + len(rr)] = np.where(vb, l - zt, 0.0)
+        dE[pos:pos + len(rr)] = G @ C64
+        margins.append(m[0])
+        pos += len(rr)
+    return RowBlockResult(rows, lse, nll, np.array(margins), filtered, dE)

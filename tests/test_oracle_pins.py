@@ -309,3 +309,17 @@ def test_sampled_evaluation_agrees_with_full(monkeypatch):
         assert s.filtered == full_b.filtered
         np.testing.assert_allclose(s.dE_rows, full_b.dE[rows], rtol=1e-11, atol=1e-14)
         np.testing.assert_allclose(s.dC_cols, full_b.dC[cols], rtol=1e-11, atol=1e-14)
+
+
+def test_row_block_evaluation_agrees_with_full():
+    E, C, t = _rand_problem(N=40, D=12, V=300, seed=15, ignore=(0, 17, 18))
+    E = E * 2.0
+    full = O.backward(E, C, t, grad_out=0.5, reduction="mean", filter_eps=2.0 ** -8, tile_m=8, tile_n=64)
+    f = O.forward(E, C, t)
+    rb = O.row_blocks(E, C, t, [4, 1], grad_out=0.5, reduction="mean", filter_eps=2.0 ** -8, tile_m=8, tile_n=64)
+    assert list(rb.rows) == list(range(8, 16)) + list(range(32, 40))
+    np.testing.assert_allclose(rb.lse, f.lse[rb.rows], rtol=1e-13)
+    np.testing.assert_allclose(rb.nll, f.nll[rb.rows], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(rb.dE, full.dE[rb.rows], rtol=1e-11, atol=1e-14)
+    margin = O.tile_log_margin(O.logits(E, C) - f.lse[:, None], t != -100, 8, 64)
+    assert rb.filtered == int(O.filtered_tiles(margin[[1, 4]], 2.0 ** -8).sum())
