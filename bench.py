@@ -1,0 +1,372 @@
+"""Benchmark of the Cut Cross-Entropy hot path: forward + backward tokens/s on one B200 per rank.
+
+A step is one forward (loss and LSE) and one backward (dE and dC, tile skipping at 2^-12) over
+one batch of the workload, through the library's C ABI. With no flags: 1 GPU, the Llama-3.1-8B
+head shape (N = 4096 tokens, D = 4096, V = 128256, peaked Zipf(1.1) targets, 5% ignored,
+reduction mean), synthetic seeded data.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Under torchrun (N > 1) every rank runs its own batch (independent replicas: the method shards by
+tokens with no exchange in the loss), the step time is the max over ranks, and rank 0 prints one
+JSON line. ``--impl reference`` times the fp64 CPU oracle on a bounded row sample of the same
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+EPS = 2.0 ** -12
+L2_FLUSH_BYTES = 512 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        busy = [s for s in sm if s > 0.5 * (max(sm) if sm else 0)]
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def algorithmic_flops(N: int, D: int, V: int, kept_tiles: int, tile: tuple) -> tuple:
+    """2NVD forward; 6 * rows * cols * D per kept backward tile (all tiles full at the bench shape)."""
+    tm, tn = tile
+    fwd = 2.0 * N * V * D
+    if N % tm == 0 and V % tn == 0:
+        bwd = 6.0 * tm * tn * D * kept_tiles
+    else:  # bound: kept tiles counted at full size
+        bwd = 6.0 * tm * tn * D * kept_tiles
+    return fwd, bwd
+
+
+def oracle_sample_seconds(inp, rows: int):
+    """fp64 oracle forward + backward on the first `rows` tokens of the workload (full vocabulary)."""
+    from oracle import cce_oracle as O
+
+    from linear_cross_entropy_06_b200.ops import backward_tile_shape
+
+    tm, tn = 128, 128
+    try:
+        tm, tn = backward_tile_shape()
+    except Exception:
+        pass
+    w = inp.workload
+    E, t = inp.E[:rows], inp.targets[:rows]
+    g = inp.grad_out[:rows] if w.reduction == "none" else inp.grad_out
+    gv = g.numpy() if w.reduction == "none" else float(g.reshape(-1)[0])
+    t0 = time.perf_counter()
+    O.forward(E, inp.C, t, -100, w.reduction)
+    O.backward(E, inp.C, t, gv, -100, w.reduction, EPS, tm, tn)
+    return time.perf_counter() - t0
+
+
+def run_reference(args, world, rank):
+    """--impl reference: the fp64 CPU oracle, as it stands, on a bounded row sample per step."""
+    if rank != 0:
+        return
+    from linear_cross_entropy_06_b200.inputs import make_inputs
+
+    inp = make_inputs(args.workload)
+    w = inp.workload
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample_seconds(inp, rows)
+    secs = [oracle_sample_seconds(inp, rows) for _ in range(args.steps)]
+    total = sum(secs)
+    value = rows * args.steps / total
+    cores = torch.get_num_threads()
+    line = {
+        "impl": "reference", "metric": "fwd+bwd tokens/s", "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {rows} of {w.N} tokens per step, full V={w.V} and D={w.D}, fp64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, gpus, shape=None):
+    N, D, V = shape or (w.N, w.D, w.V)
+    return {"workload": w.name, "tokens_per_gpu": N, "hidden": D, "vocab": V, "targets": w.targets,
+            "ignore_frac": w.ignore_frac, "reduction": w.reduction, "filter_eps": EPS,
+            "parallelism": f"replicas x{gpus} (tokens sharded, no collective)",
+            "l2": "512 MiB written between timed steps; C (up to 2 GB) is larger than L2"}
+
+
+def run_ours(args, world, rank, local):
+    from linear_cross_entropy_06_b200 import ops
+    from linear_cross_entropy_06_b200.inputs import make_inputs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    lib = ops.load_library()
+    over = dict(zip("NDV", map(int, args.shape.split(",")))) if args.shape else {}
+    inp = make_inputs(args.workload, seed=None if world == 1 else 1238 + 1000 * rank, **over)
+    w = inp.workload
+    N, D, V = inp.E.shape[0], inp.E.shape[1], inp.C.shape[0]
+    E, C, t = inp.E.to(dev), inp.C.to(dev), inp.targets.to(dev)
+    g = inp.grad_out.to(dev)
+    if w.reduction != "none":
+        g = g[:1]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    tile = ops.backward_tile_shape()
+
+    def step():
+        loss, lse, tmax, count = ops.cce_forward(E, C, t, -100, w.reduction)
+        dE, dC, filt = ops.cce_backward(E, C, t, lse, tmax, count, g, EPS, -100, w.reduction, out_fp32=False)
+        return loss, filt
+
+    # check once that nothing was reported on the device
+    loss0, lse0, tmax0, count0 = ops.cce_forward(E, C, t, -100, w.reduction, check=True)
+    ops.cce_backward(E, C, t, lse0, tmax0, count0, g, EPS, -100, w.reduction, check=True)
+    del loss0, lse0, tmax0, count0
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for e6 in ev:  # materialise the raw handles
+        for e in e6:
+            e.record()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    launches0 = lib.cce_kernel_launch_count()
+    filt_last = None
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        s0, s1, f0, f1, b0, b1 = ev[k]
+        lib.cce_set_kernel_events(f0.cuda_event, f1.cuda_event, b0.cuda_event, b1.cuda_event)
+        s0.record()
+        loss, filt_last = step()
+        s1.record()
+    lib.cce_set_kernel_events(None, None, None, None)
+    torch.cuda.synchronize()
+    launches = lib.cce_kernel_launch_count() - launches0
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+
+    step_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    fwd_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    bwd_ms = [e[4].elapsed_time(e[5]) for e in ev]
+    total_s = max_over_ranks(sum(step_ms) / 1e3, world, dev)
+    value = world * N * args.steps / total_s
+    filtered = int(filt_last.item())
+    nb, nt = -(-N // tile[0]), -(-V // tile[1])
+    kept = nb * nt - filtered
+    fwd_flop, bwd_flop = algorithmic_flops(N, D, V, kept, tile)
+    peaks, peak_kind = load_peaks()
+    peak_tf = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    fwd_avg, bwd_avg = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    kernels = {
+        "fwd_lse": {"ms": fwd_avg, "tflops": fwd_flop / fwd_avg / 1e9, "frac": fwd_flop / fwd_avg / 1e9 / peak_tf},
+        "bwd_grad": {"ms": bwd_avg, "tflops": bwd_flop / bwd_avg / 1e9, "frac": bwd_flop / bwd_avg / 1e9 / peak_tf},
+    }
+    dom = "bwd_grad" if bwd_avg >= fwd_avg else "fwd_lse"
+    dom_flop = bwd_flop if dom == "bwd_grad" else fwd_flop
+    dom_ms = kernels[dom]["ms"]
+    ms_step = 1e3 * total_s / args.steps
+    path_tflops = (fwd_flop + bwd_flop) / (ms_step / 1e3) / 1e12
+
+    # end to end through the public API: inputs copied from pinned host memory every step and the
+    # loss read back to the host
+    e2e = None
+    if not args.no_e2e:
+        hE, hC, ht = inp.E.pin_memory(), inp.C.pin_memory(), inp.targets.pin_memory()
+        dE_in = torch.empty_like(E)
+        dC_in = torch.empty_like(C)
+        dt = torch.empty_like(t)
+        h2d = hE.numel() * 2 + hC.numel() * 2 + ht.numel() * 8
+        d2h = 4
+        for _ in range(2):
+            dE_in.copy_(hE, non_blocking=True)
+            dC_in.copy_(hC, non_blocking=True)
+            dt.copy_(ht, non_blocking=True)
+            e_ = dE_in.detach().requires_grad_(True)
+            c_ = dC_in.detach().requires_grad_(True)
+            out = ops.linear_cross_entropy(e_, c_, dt, reduction=w.reduction)
+            out.backward(torch.ones_like(out) if w.reduction == "none" else None)
+            float(out.sum().item())
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.e2e_steps):
+            dE_in.copy_(hE, non_blocking=True)
+            dC_in.copy_(hC, non_blocking=True)
+            dt.copy_(ht, non_blocking=True)
+            e_ = dE_in.detach().requires_grad_(True)
+            c_ = dC_in.detach().requires_grad_(True)
+            out = ops.linear_cross_entropy(e_, c_, dt, reduction=w.reduction)
+            out.backward(torch.ones_like(out) if w.reduction == "none" else None)
+            _ = out.sum().item()  # device -> host read of the step's result
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+        e2e = {"value": world * N * args.e2e_steps / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "path": "linear_cross_entropy(e, c, targets) + backward, inputs copied from pinned host memory"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rows = args.cpu_rows
+        secs = oracle_sample_seconds(inp, rows)
+        cpu = {"value": rows / secs, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
+               "sample": f"first {rows} of {N} tokens, full V={V} and D={D}, fp64 forward + backward, {secs:.1f} s"}
+
+    if rank != 0:
+        return
+    line = {
+        "metric": "fwd+bwd tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w, world, (N, D, V)),
+        "tensor_peak_frac": {"achieved_tflops": path_tflops, "peak": peak_tf, "frac": path_tflops / peak_tf,
+                             "peak_kind": f"bf16_tflops ({peak_kind})",
+                             "flops_per_step": fwd_flop + bwd_flop, "kept_tiles": kept, "filtered_tiles": filtered},
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_flop / dom_ms / 1e9, "peak": peak_tf,
+                     "unit": "TFLOP/s", "frac": dom_flop / dom_ms / 1e9 / peak_tf, "traffic": None,
+                     "peak_kind": f"bf16_tflops ({peak_kind})"},
+        "kernels": kernels,
+        "clocks": clocks,
+        "gpu_launches": launches,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=int(os.environ.get("WORLD_SIZE", "1")))
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama3.1-8b-head")
+    ap.add_argument("--shape", default=None,
+                    help="N,D,V override of the workload's sizes (profiling captures on a smaller case)")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-rows", type=int, default=384)
+    ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

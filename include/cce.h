@@ -139,6 +139,16 @@ CCE_API const char* cce_status_string(cce_status s);
 /* Detail of the last failing call on the calling thread ("" if none). */
 CCE_API const char* cce_last_error_message(void);
 
+/* Optional instrumentation, off by default and per calling thread. When an event pair is set
+ * (cudaEvent_t handles created by the caller; NULL clears), cce_forward() records fwd_start and
+ * fwd_stop on its stream immediately before and after launching its tensor-core kernel, and
+ * cce_backward() does the same with bwd_start and bwd_stop, so the caller can time that kernel
+ * alone. */
+CCE_API void cce_set_kernel_events(void* fwd_start, void* fwd_stop, void* bwd_start, void* bwd_stop);
+
+/* Number of kernels this library has launched from the calling thread since it was loaded. */
+CCE_API int64_t cce_kernel_launch_count(void);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 CCE_API int32_t cce_version(void);
 

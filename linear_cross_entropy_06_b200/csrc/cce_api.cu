@@ -21,6 +21,9 @@ constexpr size_t kHeaderBytes = 256;
 constexpr size_t kAlign = 256;
 
 thread_local std::string g_last_error;
+thread_local int64_t g_launches = 0;
+thread_local cudaEvent_t g_fwd_ev[2] = {nullptr, nullptr};
+thread_local cudaEvent_t g_bwd_ev[2] = {nullptr, nullptr};
 
 cce_status fail(cce_status s, const char* fmt, ...) {
   char buf[512];
@@ -93,6 +96,7 @@ struct BwdWs {
   WsHeader* hdr;
   float* scale;
   int2* tiles;
+  uint8_t* keep;
   float* dE_acc;
   float* dC_acc;
   size_t bytes;
@@ -108,6 +112,8 @@ BwdWs carve_bwd(const cce_problem* p, int32_t out_fp32, void* base) {
   off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
   w.tiles = reinterpret_cast<int2*>(b + off);
   off = align_up(off + sizeof(int2) * static_cast<size_t>(nb * nt));
+  w.keep = reinterpret_cast<uint8_t*>(b + off);
+  off = align_up(off + static_cast<size_t>(nb * nt));
   if (!out_fp32) {
     w.dE_acc = reinterpret_cast<float*>(b + off);
     off = align_up(off + sizeof(float) * static_cast<size_t>(p->N * p->D));
@@ -188,7 +194,21 @@ uint64_t wait_timeout_ns() {
 
 }  // namespace
 
+namespace cce {
+void note_launches(int n) { g_launches += n; }
+}  // namespace cce
+
 extern "C" {
+
+void cce_set_kernel_events(void* fwd_start, void* fwd_stop, void* bwd_start, void* bwd_stop) {
+  g_fwd_ev[0] = static_cast<cudaEvent_t>(fwd_start);
+  g_fwd_ev[1] = static_cast<cudaEvent_t>(fwd_stop);
+  g_bwd_ev[0] = static_cast<cudaEvent_t>(bwd_start);
+  g_bwd_ev[1] = static_cast<cudaEvent_t>(bwd_stop);
+}
+
+int64_t cce_kernel_launch_count(void) { return g_launches; }
+
 
 int32_t cce_version(void) { return kVersion; }
 
@@ -264,7 +284,9 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
     L.timeout_ns = wait_timeout_ns();
     L.num_sms = num_sms;
     CCE_TRY(cce::launch_target_logit(Eb, Cb, targets, N, D, V, p->ignore_index, w.z_target, &w.hdr->err, s));
+    if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[0], s));
     CCE_TRY(cce::launch_fwd_lse(L, s));
+    if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[1], s));
     float* rows_out = p->reduction == CCE_REDUCTION_NONE ? loss : w.loss_rows;
     CCE_TRY(cce::launch_lse_loss(tile_max, w.tile_sum, w.z_target, targets, N, T, p->ignore_index, V, lse, rows_out,
                                  s));
@@ -304,9 +326,10 @@ cce_status cce_backward(const cce_problem* p, const void* E, const void* C, cons
   CCE_TRY(cudaMemsetAsync(w.hdr, 0, sizeof(WsHeader), s));
   CCE_TRY(cce::launch_row_scale(targets, count, grad_out, N, p->ignore_index, p->reduction, w.scale,
                                 &w.hdr->num_tiles, s));
-  CCE_TRY(cce::launch_tile_mask(tile_max, lse, targets, N, V, T, p->ignore_index, filter_eps, w.tiles,
+  CCE_TRY(cce::launch_tile_mask(tile_max, lse, targets, N, V, T, p->ignore_index, filter_eps, w.tiles, w.keep,
                                 &w.hdr->num_tiles, filtered_tiles, s));
-  CCE_TRY(cce::launch_grad_init(Eb, Cb, targets, w.scale, N, D, V, p->ignore_index, dE_acc, dC_acc, s));
+  CCE_TRY(cce::launch_grad_init(Eb, Cb, targets, w.scale, w.keep, N, D, V, p->ignore_index, dE_acc, dC_acc,
+                                &w.hdr->err, s));
   if (has_rows) {
     cce::BwdLaunch L{};
     CCE_CHECK(make_map(&L.tmE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kBwdBM));
@@ -318,12 +341,16 @@ cce_status cce_backward(const cce_problem* p, const void* E, const void* C, cons
     L.V = static_cast<int>(V);
     L.lse = lse;
     L.scale = w.scale;
+    L.targets = targets;
+    L.ignore_index = p->ignore_index;
     L.tiles = w.tiles;
     L.num_tiles = &w.hdr->num_tiles;
     L.err = &w.hdr->err;
     L.timeout_ns = wait_timeout_ns();
     L.num_sms = num_sms;
+    if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
     CCE_TRY(cce::launch_bwd_grad(L, s));
+    if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
   }
   if (!out_fp32) {
     CCE_TRY(cce::launch_to_bf16(dE_acc, static_cast<__nv_bfloat16*>(dE), N * D, s));

@@ -10,8 +10,11 @@
 //  row_scale      per-row factor of the gradient: g/max(count,1), g or g[r]; 0 for ignored rows.
 //  tile_mask      keep/skip decision per backward tile from the saved maxima and LSE, compacted
 //                 into a list. mlx-cross-entropy README, "How it works" item 2.
-//  grad_init      dE_acc[r] = -scale_r C[t_r] (the onehot part of p - y; ignored rows +0),
-//                 dC_acc = 0; onehot_dC then adds -scale_r E[r] into dC_acc[t_r].
+//  grad_init      dC_acc = 0 and dE_acc[r] = -scale_r C[t_r] when the tile holding (r, t_r) is
+//                 skipped, else +0; onehot_dC adds -scale_r E[r] into dC_acc[t_r] for the same
+//                 rows. The onehot part of p - y of a kept tile is folded into the gradient tile
+//                 by the backward kernel (before rounding to bf16), so it is never skipped and
+//                 never cancels against a rounded p.
 //  to_bf16        fp32 accumulators -> bf16 outputs (round to nearest even).
 #include <cuda_bf16.h>
 
@@ -159,8 +162,8 @@ __global__ void row_scale_kernel(const int64_t* __restrict__ targets, const int6
 // so each vocabulary tile's row blocks are adjacent in the list.
 __global__ void tile_mask_kernel(const float* __restrict__ tile_max, const float* __restrict__ lse,
                                  const int64_t* __restrict__ targets, int64_t N, int64_t V, int64_t T,
-                                 int64_t ignore_index,
-                                 float ln_eps, int filter_on, int2* __restrict__ tiles, int* num_tiles) {
+                                 int64_t ignore_index, float ln_eps, int filter_on, int2* __restrict__ tiles,
+                                 uint8_t* __restrict__ keep, int* num_tiles) {
   __shared__ float wmax[4];
   __shared__ int base;
   const int t = blockIdx.x;
@@ -169,7 +172,7 @@ __global__ void tile_mask_kernel(const float* __restrict__ tile_max, const float
   for (int pass = 0; pass < 2; ++pass) {
     int k = 0;
     for (int b = 0; b < nb; ++b) {
-      bool keep = true;
+      bool keep_tile = true;
       if (filter_on) {
         const int64_t r = static_cast<int64_t>(b) * kBwdBM + threadIdx.x;
         float m = -INFINITY;
@@ -184,9 +187,10 @@ __global__ void tile_mask_kernel(const float* __restrict__ tile_max, const float
         __syncthreads();
         const float bm = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
         __syncthreads();
-        keep = bm >= ln_eps;
+        keep_tile = bm >= ln_eps;
       }
-      if (keep) {
+      if (pass == 0 && threadIdx.x == 0) keep[static_cast<int64_t>(b) * gridDim.x + t] = keep_tile ? 1 : 0;
+      if (keep_tile) {
         if (pass == 1 && threadIdx.x == 0) tiles[base + k] = make_int2(b, t);
         ++k;
       }
@@ -203,17 +207,27 @@ __global__ void mask_finish_kernel(const int* __restrict__ num_tiles, int64_t to
   *filtered = total - static_cast<int64_t>(*num_tiles);
 }
 
-// dE_acc[r, :] = -scale_r * C[t_r, :] for non-ignored rows, +0 otherwise. One warp per row, 8
-// elements per lane per step.
+// True when row r has a valid target whose tile (r's row block, t_r's vocabulary tile) was skipped:
+// then the onehot term of that row is added here instead of inside the backward kernel.
+__device__ __forceinline__ bool onehot_outside(int64_t r, int64_t t, int64_t V, int64_t ignore_index,
+                                               const uint8_t* keep, int64_t nt) {
+  return valid_target(t, V, ignore_index) && keep[(r / kBwdBM) * nt + t / kBwdBN] == 0;
+}
+
+// dE_acc[r, :] = -scale_r * C[t_r, :] for rows whose target tile is skipped, +0 otherwise. One warp
+// per row, 8 elements per lane per step.
 __global__ void grad_init_dE_kernel(const __nv_bfloat16* __restrict__ C, const int64_t* __restrict__ targets,
-                                    const float* __restrict__ scale, int64_t N, int64_t D, int64_t V,
-                                    int64_t ignore_index, float* __restrict__ dE_acc) {
+                                    const float* __restrict__ scale, const uint8_t* __restrict__ keep, int64_t N,
+                                    int64_t D, int64_t V, int64_t ignore_index, float* __restrict__ dE_acc,
+                                    int* err) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= N) return;
   const int64_t t = targets[row];
   float* out = dE_acc + row * D;
-  if (!valid_target(t, V, ignore_index)) {
+  if (lane == 0 && t != ignore_index && !valid_target(t, V, ignore_index)) record_error(err, kErrTargetRange);
+  const int64_t nt = (V + kBwdBN - 1) / kBwdBN;
+  if (!onehot_outside(row, t, V, ignore_index, keep, nt)) {
     for (int64_t d = static_cast<int64_t>(lane) * 4; d < D; d += 128)
       *reinterpret_cast<float4*>(out + d) = make_float4(0.f, 0.f, 0.f, 0.f);
     return;
@@ -237,13 +251,13 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 
 // dC_acc[t_r, :] += -scale_r * E[r, :] for non-ignored rows (targets repeat, hence atomics).
 __global__ void onehot_dC_kernel(const __nv_bfloat16* __restrict__ E, const int64_t* __restrict__ targets,
-                                 const float* __restrict__ scale, int64_t N, int64_t D, int64_t V,
-                                 int64_t ignore_index, float* __restrict__ dC_acc) {
+                                 const float* __restrict__ scale, const uint8_t* __restrict__ keep, int64_t N,
+                                 int64_t D, int64_t V, int64_t ignore_index, float* __restrict__ dC_acc) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= N) return;
   const int64_t t = targets[row];
-  if (!valid_target(t, V, ignore_index)) return;
+  if (!onehot_outside(row, t, V, ignore_index, keep, (V + kBwdBN - 1) / kBwdBN)) return;
   const float s = -scale[row];
   const __nv_bfloat16* e = E + row * D;
   float* out = dC_acc + t * D;
@@ -290,6 +304,7 @@ cudaError_t launch_target_logit(const __nv_bfloat16* E, const __nv_bfloat16* C, 
   if (N == 0) return cudaSuccess;
   const int grid = static_cast<int>((N + 7) / 8);
   target_logit_kernel<<<grid, 256, 0, s>>>(E, C, targets, N, D, V, ignore_index, z_target, err);
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -299,12 +314,14 @@ cudaError_t launch_lse_loss(const float* tile_max, const float* tile_sum, const 
   if (N == 0) return cudaSuccess;
   const int grid = static_cast<int>((N + 31) / 32);
   lse_loss_kernel<<<grid, 256, 0, s>>>(tile_max, tile_sum, z_target, targets, N, T, ignore_index, V, lse, loss_rows);
+  note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_loss_reduce(const float* loss_rows, const int64_t* targets, int64_t N, int64_t ignore_index,
                                int reduction, float* loss, int64_t* count, cudaStream_t s) {
   loss_reduce_kernel<<<1, kReduceThreads, 0, s>>>(loss_rows, targets, N, ignore_index, reduction, loss, count);
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -312,37 +329,42 @@ cudaError_t launch_row_scale(const int64_t* targets, const int64_t* count, const
                              int64_t ignore_index, int reduction, float* scale, int* num_tiles, cudaStream_t s) {
   const int grid = static_cast<int>(N > 0 ? (N + 255) / 256 : 1);
   row_scale_kernel<<<grid, 256, 0, s>>>(targets, count, grad_out, N, ignore_index, reduction, scale, num_tiles);
+  note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_tile_mask(const float* tile_max, const float* lse, const int64_t* targets, int64_t N, int64_t V,
-                             int64_t T, int64_t ignore_index, float filter_eps, int2* tiles, int* num_tiles,
-                             int64_t* filtered_tiles, cudaStream_t s) {
+                             int64_t T, int64_t ignore_index, float filter_eps, int2* tiles, uint8_t* keep,
+                             int* num_tiles, int64_t* filtered_tiles, cudaStream_t s) {
   const int64_t nb = (N + kBwdBM - 1) / kBwdBM;
   const int64_t nt = (V + kBwdBN - 1) / kBwdBN;
   const int filter_on = filter_eps > 0.f ? 1 : 0;
   const float ln_eps = filter_on ? logf(filter_eps) : -INFINITY;
   if (nb > 0) {
     tile_mask_kernel<<<static_cast<int>(nt), kBwdBM, 0, s>>>(tile_max, lse, targets, N, V, T, ignore_index, ln_eps,
-                                                             filter_on, tiles, num_tiles);
+                                                             filter_on, tiles, keep, num_tiles);
+    note_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   mask_finish_kernel<<<1, 1, 0, s>>>(num_tiles, nb * nt, filtered_tiles);
+  note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_grad_init(const __nv_bfloat16* E, const __nv_bfloat16* C, const int64_t* targets,
-                             const float* scale, int64_t N, int64_t D, int64_t V, int64_t ignore_index,
-                             float* dE_acc, float* dC_acc, cudaStream_t s) {
+                             const float* scale, const uint8_t* keep, int64_t N, int64_t D, int64_t V,
+                             int64_t ignore_index, float* dE_acc, float* dC_acc, int* err, cudaStream_t s) {
   cudaError_t e = launch_fill_zero(dC_acc, V * D * 4, s);
   if (e != cudaSuccess) return e;
   if (N == 0) return cudaSuccess;
   const int grid = static_cast<int>((N + 7) / 8);
-  grad_init_dE_kernel<<<grid, 256, 0, s>>>(C, targets, scale, N, D, V, ignore_index, dE_acc);
+  grad_init_dE_kernel<<<grid, 256, 0, s>>>(C, targets, scale, keep, N, D, V, ignore_index, dE_acc, err);
+  note_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  onehot_dC_kernel<<<grid, 256, 0, s>>>(E, targets, scale, N, D, V, ignore_index, dC_acc);
+  onehot_dC_kernel<<<grid, 256, 0, s>>>(E, targets, scale, keep, N, D, V, ignore_index, dC_acc);
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -350,6 +372,7 @@ cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, int64_t n, cuda
   if (n == 0) return cudaSuccess;
   const int64_t n8 = n / 8;  // n is a multiple of 8 (D is)
   to_bf16_kernel<<<grid_for(n8, 256, 148 * 16), 256, 0, s>>>(src, dst, n8);
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -357,6 +380,7 @@ cudaError_t launch_fill_zero(void* dst, int64_t bytes, cudaStream_t s) {
   if (bytes == 0) return cudaSuccess;
   const int64_t n16 = bytes / 16;  // callers pass multiples of 16 bytes
   fill_zero_kernel<<<grid_for(n16, 256, 148 * 16), 256, 0, s>>>(static_cast<uint4*>(dst), n16);
+  note_launches(1);
   return cudaGetLastError();
 }
 

@@ -5,9 +5,10 @@
 //
 // mlx-cross-entropy README, "How it works" items 2 and 3 (recompute, skip tiles below 2^-12 using
 // the forward's saved maxima, accumulate with atomics instead of [batch, tiles, D] buffers); Loss
-// functions explainer, "How it works" item 2 (the logit gradient is p - y; the "- y" onehot part
-// is added by a separate kernel and is never skipped). Cut Your Losses abstract (skip gradient
-// elements below numerical precision).
+// functions explainer, "How it works" item 2 (the logit gradient is p - y). The onehot "- y" of a
+// kept tile is folded into G in fp32 before the bf16 rounding; for a skipped tile that holds a
+// target it is added by a separate kernel, so it is never skipped. Cut Your Losses abstract (skip
+// gradient elements below numerical precision).
 //
 // Design (B200): one persistent CTA per SM, 6 warps, walking the compacted list of kept tiles.
 //   warp 0      TMA producer into a 3-stage ring of 32 KB stages: first the D/64 k-blocks of
@@ -76,8 +77,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_grad_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC,
                     const __grid_constant__ CUtensorMap tmdE, const __grid_constant__ CUtensorMap tmdC, int N,
                     int D, int V, const float* __restrict__ lse, const float* __restrict__ scale,
-                    const int2* __restrict__ tiles, const int* __restrict__ num_tiles_ptr, int* err,
-                    uint64_t timeout_ns) {
+                    const int64_t* __restrict__ targets, int64_t ignore_index, const int2* __restrict__ tiles,
+                    const int* __restrict__ num_tiles_ptr, int* err, uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm = carve(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -247,6 +248,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int r = bt.x * BM + row;
       const float lse_l2 = (r < N) ? lse[r] * kLog2e : 0.f;
       const float sc = (r < N) ? scale[r] : 0.f;
+      // Column of this row's target inside the tile, or -1: there G gets the onehot term -scale_r
+      // in fp32, before rounding, so p_t - 1 does not lose its digits when p_t is close to 1.
+      int tcol = -1;
+      if (r < N) {
+        const int64_t tg = targets[r];
+        const int64_t rel = tg - static_cast<int64_t>(bt.y) * BN;
+        if (tg != ignore_index && tg >= 0 && tg < V && rel >= 0 && rel < BN) tcol = static_cast<int>(rel);
+      }
       if (!mbar_wait(sfull_bar, tile_iter & 1u, wc)) break;
       tc_fence_after();
       // G[row, :] = scale_r * exp(S[row, :] - LSE_r), bf16, 128B-swizzled, two 64-column blocks.
@@ -257,7 +266,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int col0 = bt.y * BN + c * 32;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float gval = sc * exp2f(fmaf(v[j], kLog2e, -lse_l2));
+          float gval = sc * exp2f(fmaf(v[j], kLog2e, -lse_l2));
+          if (c * 32 + j == tcol) gval -= sc;
           v[j] = (col0 + j < V) ? gval : 0.f;
         }
         const uint32_t blk = g0 + static_cast<uint32_t>((c >> 1) * HALF);
@@ -345,7 +355,9 @@ cudaError_t launch_bwd_grad(const BwdLaunch& L, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(max_tiles < L.num_sms ? max_tiles : L.num_sms);
   bwd_grad_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmC, L.tmdE, L.tmdC, L.N, L.D, L.V, L.lse, L.scale,
-                                                        L.tiles, L.num_tiles, L.err, L.timeout_ns);
+                                                        L.targets, L.ignore_index, L.tiles, L.num_tiles, L.err,
+                                                        L.timeout_ns);
+  note_launches(1);
   return cudaGetLastError();
 }
 

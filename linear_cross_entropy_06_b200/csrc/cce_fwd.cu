@@ -244,6 +244,7 @@ cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s) {
   const int grid = static_cast<int>(total < L.num_sms ? total : L.num_sms);
   fwd_lse_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmC, L.N, L.D, L.V, L.T, L.tile_max, L.tile_sum,
                                                        L.err, L.timeout_ns);
+  note_launches(1);
   return cudaGetLastError();
 }
 

@@ -36,12 +36,17 @@ struct BwdLaunch {
   int N, D, V;
   const float* lse;     // [N]
   const float* scale;   // [N]: per-row gradient factor, 0 for ignored rows
+  const int64_t* targets;  // [N]: the onehot term of a kept tile is applied inside the kernel
+  int64_t ignore_index;
   const int2* tiles;    // kept tiles (row block, vocab tile)
   const int* num_tiles; // device count of kept tiles
   int* err;
   uint64_t timeout_ns;
   int num_sms;
 };
+
+// Counts every kernel launch of the calling thread (instrumentation for benchmarks).
+void note_launches(int n);
 
 cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
 cudaError_t launch_bwd_grad(const BwdLaunch& L, cudaStream_t s);
@@ -58,11 +63,11 @@ cudaError_t launch_loss_reduce(const float* loss_rows, const int64_t* targets, i
 cudaError_t launch_row_scale(const int64_t* targets, const int64_t* count, const float* grad_out, int64_t N,
                              int64_t ignore_index, int reduction, float* scale, int* num_tiles, cudaStream_t s);
 cudaError_t launch_tile_mask(const float* tile_max, const float* lse, const int64_t* targets, int64_t N, int64_t V,
-                             int64_t T, int64_t ignore_index, float filter_eps, int2* tiles, int* num_tiles,
-                             int64_t* filtered_tiles, cudaStream_t s);
+                             int64_t T, int64_t ignore_index, float filter_eps, int2* tiles, uint8_t* keep,
+                             int* num_tiles, int64_t* filtered_tiles, cudaStream_t s);
 cudaError_t launch_grad_init(const __nv_bfloat16* E, const __nv_bfloat16* C, const int64_t* targets,
-                             const float* scale, int64_t N, int64_t D, int64_t V, int64_t ignore_index,
-                             float* dE_acc, float* dC_acc, cudaStream_t s);
+                             const float* scale, const uint8_t* keep, int64_t N, int64_t D, int64_t V,
+                             int64_t ignore_index, float* dE_acc, float* dC_acc, int* err, cudaStream_t s);
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, int64_t n, cudaStream_t s);
 cudaError_t launch_fill_zero(void* dst, int64_t bytes, cudaStream_t s);
 

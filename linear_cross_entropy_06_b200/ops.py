@@ -65,6 +65,8 @@ SIGNATURES = {
     "cce_status_string": (ctypes.c_char_p, [_I32]),
     "cce_last_error_message": (ctypes.c_char_p, []),
     "cce_version": (_I32, []),
+    "cce_set_kernel_events": (None, [_VP, _VP, _VP, _VP]),
+    "cce_kernel_launch_count": (_I64, []),
 }
 
 _lib: Optional[ctypes.CDLL] = None
