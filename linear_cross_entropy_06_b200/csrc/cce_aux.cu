@@ -79,26 +79,38 @@ __device__ __forceinline__ void lse_merge(float& M, float& S, float m, float s) 
   }
 }
 
-// Block = 8 warps x 32 rows. Warp w merges sub-tiles j = w, w + 8, ... of its 32 rows (lane = row,
-// so each load is 128 contiguous bytes); the 8 partial results merge in shared memory.
-__global__ void lse_loss_kernel(const float* __restrict__ tile_max, const float* __restrict__ tile_sum,
-                                const float* __restrict__ z_target, const int64_t* __restrict__ targets, int64_t N,
-                                int64_t T, int64_t ignore_index, int64_t V, float* __restrict__ lse,
-                                float* __restrict__ loss_rows) {
-  __shared__ float sm_m[8][32], sm_s[8][32];
+constexpr int kLseWarps = 32;
+
+// Block = 32 warps x 32 rows. Warp w merges sub-tiles j = w, w + 32, ... of its 32 rows (lane = row,
+// so each load is 128 contiguous bytes), four sub-tiles per step so that eight loads are in flight;
+// the 32 partial results merge in shared memory.
+__global__ void __launch_bounds__(kLseWarps * 32)
+    lse_loss_kernel(const float* __restrict__ tile_max, const float* __restrict__ tile_sum,
+                    const float* __restrict__ z_target, const int64_t* __restrict__ targets, int64_t N, int64_t T,
+                    int64_t ignore_index, int64_t V, float* __restrict__ lse, float* __restrict__ loss_rows) {
+  __shared__ float sm_m[kLseWarps][32], sm_s[kLseWarps][32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * 32 + lane;
   float M = -INFINITY, S = 0.f;
   if (r < N) {
-    for (int64_t j = w; j < T; j += 8) lse_merge(M, S, tile_max[j * N + r], tile_sum[j * N + r]);
+    for (int64_t j = w; j < T; j += 4 * kLseWarps) {
+      float m[4], s[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t jj = j + u * kLseWarps;
+        m[u] = jj < T ? tile_max[jj * N + r] : -INFINITY;
+        s[u] = jj < T ? tile_sum[jj * N + r] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) lse_merge(M, S, m[u], s[u]);
+    }
   }
   sm_m[w][lane] = M;
   sm_s[w][lane] = S;
   __syncthreads();
   if (w == 0 && r < N) {
     float Mt = -INFINITY, St = 0.f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) lse_merge(Mt, St, sm_m[k][lane], sm_s[k][lane]);
+    for (int k = 0; k < kLseWarps; ++k) lse_merge(Mt, St, sm_m[k][lane], sm_s[k][lane]);
     const float L = Mt + logf(St);
     lse[r] = L;
     const int64_t t = targets[r];
@@ -313,7 +325,8 @@ cudaError_t launch_lse_loss(const float* tile_max, const float* tile_sum, const 
                             float* lse, float* loss_rows, cudaStream_t s) {
   if (N == 0) return cudaSuccess;
   const int grid = static_cast<int>((N + 31) / 32);
-  lse_loss_kernel<<<grid, 256, 0, s>>>(tile_max, tile_sum, z_target, targets, N, T, ignore_index, V, lse, loss_rows);
+  lse_loss_kernel<<<grid, kLseWarps * 32, 0, s>>>(tile_max, tile_sum, z_target, targets, N, T, ignore_index, V, lse,
+                                                  loss_rows);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -3,7 +3,7 @@
 Tolerances: the loss and per-row LSE within 2e-3 absolute; dE and dC within a relative
 Frobenius error of 1e-2 when nothing is skipped. With skipping, dE and dC are within 2e-2 of
 the unskipped oracle and within 1e-2 of the oracle that applies the same tile rule.
-Elementwise: |gpu - oracle| <= 3e-2 * rms(oracle) + 3e-2 * |oracle|. Rows of ignored tokens
+Elementwise: |gpu - oracle| <= 3e-2 * rms(that row of the oracle) + 3e-2 * |oracle|. Rows of ignored tokens
 in dE are exactly +0 and skipped-tile counts equal the oracle's (unless the oracle reports a
 tile whose margin lies within 2e-3 of ln eps, in which case the difference is bounded by that
 number).
@@ -44,7 +44,9 @@ def rel_frob(a, b):
 
 
 def assert_close_elementwise(a, b, what):
-    rms = math.sqrt(float(np.mean(b * b))) if b.size else 0.0
+    # Row-wise scale: a row of dE or dC is one column of G times E or C, so its rounding error
+    # grows with that row's own magnitude (rows of popular targets are far larger than the rest).
+    rms = np.sqrt(np.mean(b * b, axis=1, keepdims=True)) if b.size else 0.0
     bad = np.abs(a - b) > 3e-2 * rms + 3e-2 * np.abs(b) + 1e-30
     assert not bad.any(), f"{what}: {int(bad.sum())} elements outside tolerance, worst {np.abs(a - b).max():.3e}"
 
@@ -184,7 +186,7 @@ def test_autograd_wrapper(device):
     f = O.forward(inp.E, inp.C, inp.targets)
     tm, tn = tile_shape()
     b = O.backward(inp.E, inp.C, inp.targets, 1.0, -100, "mean", EPS, tm, tn)
-    assert abs(float(loss) - float(f.loss)) <= LOSS_TOL
+    assert abs(float(loss.detach()) - float(f.loss)) <= LOSS_TOL
     assert rel_frob(e.grad.reshape(96, 128).double().cpu().numpy(), b.dE) <= 1e-2
     assert rel_frob(c.grad.double().cpu().numpy(), b.dC) <= 1e-2
     nll = ops.linear_cross_entropy(e, c, t, reduction="none")
