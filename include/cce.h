@@ -139,6 +139,29 @@ CCE_API const char* cce_status_string(cce_status s);
 /* Detail of the last failing call on the calling thread ("" if none). */
 CCE_API const char* cce_last_error_message(void);
 
+/* Bytes of device scratch the library holds, per GPU that loads it, for cce_forward_noalloc(). */
+#define CCE_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * Forward that allocates nothing and takes no workspace, for callers that cannot allocate device
+ * memory where they compute the loss (for example code running during CUDA graph capture, or an
+ * embedding that only hands the library fixed buffers for inputs and outputs). The pages have no
+ * counterpart; it is an addition for such callers. Arguments and results are those of
+ * cce_forward() without the workspace.
+ *  - Scratch lives in one device array of CCE_NOALLOC_SCRATCH_BYTES that every GPU loading the
+ *    library holds until exit. Problems needing more (about ceil(V/128) * N * 4 + 8 N bytes; at
+ *    V = 128256 up to N of about 8000) are rejected with CCE_ERR_UNSUPPORTED before anything runs.
+ *  - The first call on each device looks up the array's device address; make that first call
+ *    before any stream capture.
+ *  - Every call shares the array, so calls whose work overlaps on the GPU (other streams, other
+ *    threads) race and give undefined results; serialise them.
+ *  - Device-side errors (a target outside [0, V)) are not reported by this variant; use
+ *    cce_forward() and cce_check_device_error() to diagnose them.
+ */
+CCE_API cce_status cce_forward_noalloc(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
+                                       float* loss, float* lse, float* tile_max, int64_t* count,
+                                       cce_stream_t stream);
+
 /* Optional instrumentation, off by default and per calling thread. When an event pair is set
  * (cudaEvent_t handles created by the caller; NULL clears), cce_forward() records fwd_start and
  * fwd_stop on its stream immediately before and after launching its tensor-core kernel, and

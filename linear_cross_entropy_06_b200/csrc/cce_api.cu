@@ -196,6 +196,7 @@ uint64_t wait_timeout_ns() {
 
 namespace cce {
 void note_launches(int n) { g_launches += n; }
+void set_last_error(const char* msg) { g_last_error = msg; }
 }  // namespace cce
 
 extern "C" {

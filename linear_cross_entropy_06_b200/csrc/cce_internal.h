@@ -48,6 +48,9 @@ struct BwdLaunch {
 // Counts every kernel launch of the calling thread (instrumentation for benchmarks).
 void note_launches(int n);
 
+// Sets the message cce_last_error_message() returns on the calling thread.
+void set_last_error(const char* msg);
+
 cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
 cudaError_t launch_bwd_grad(const BwdLaunch& L, cudaStream_t s);
 

@@ -1,0 +1,155 @@
+// cce_forward_noalloc: the forward for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc or an allocator of their own at the point where they
+// compute the loss: code running while a CUDA graph is being captured, an embedding that
+// hands this library only fixed, pre-registered buffers for inputs and outputs, or a runtime
+// whose allocator must not be re-entered from inside a loss callback. For them this entry point
+// keeps its scratch (per-sub-tile exp sums, target logits, per-row losses and the device error
+// word) in one file-scope device array of kNoAllocScratchBytes, which every GPU that loads the
+// library holds until the process exits. The caller passes inputs and outputs only.
+//
+// It launches the same kernels as cce_forward(); only where the scratch lives differs.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "cce.h"
+#include "cce_internal.h"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = CCE_NOALLOC_SCRATCH_BYTES;
+constexpr size_t kHeader = 256;
+constexpr size_t kAlign = 256;
+constexpr int kMaxDevices = 64;
+
+// Shared by every call on a device; keeps the last call's contents.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_fn = nullptr;
+
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+cce_status fail(cce_status s, const char* msg) {
+  cce::set_last_error(msg);
+  return s;
+}
+
+// Device address of the scratch array for the current device. The first call on a device looks
+// it up (with that device current) and caches it.
+cce_status scratch_for_current_device(void** out, int* num_sms) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return fail(CCE_ERR_CUDA, "cce_forward_noalloc: no usable current CUDA device");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) return fail(CCE_ERR_UNSUPPORTED, "cce_forward_noalloc: device is not sm_100 (B200)");
+  if (cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return fail(CCE_ERR_CUDA, "cce_forward_noalloc: cudaDeviceGetAttribute failed");
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr) return fail(CCE_ERR_CUDA, "cce_forward_noalloc: cudaGetSymbolAddress failed");
+    g_scratch_addr[dev] = ptr;
+  }
+  if (g_encode_fn == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return fail(CCE_ERR_CUDA, "cce_forward_noalloc: cuTensorMapEncodeTiled unavailable");
+    g_encode_fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  *out = g_scratch_addr[dev];
+  return CCE_OK;
+}
+
+cce_status encode(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, uint32_t box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  if (g_encode_fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return fail(CCE_ERR_CUDA, "cce_forward_noalloc: cuTensorMapEncodeTiled failed");
+  return CCE_OK;
+}
+
+}  // namespace
+
+extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
+                                          float* loss, float* lse, float* tile_max, int64_t* count,
+                                          cce_stream_t stream) {
+  cce::set_last_error("");
+  if (p == nullptr || p->N < 0 || p->D < 8 || p->D % 8 != 0 || p->V < 1 || p->reduction < 0 || p->reduction > 2 ||
+      p->reserved != 0 || p->N >= (int64_t(1) << 31) - 256 || p->V >= (int64_t(1) << 31) - 256 ||
+      p->D >= (int64_t(1) << 24))
+    return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: invalid problem");
+  const int64_t N = p->N, D = p->D, V = p->V;
+  const int64_t T = (V + cce::kSubTile - 1) / cce::kSubTile;
+  if (C == nullptr || loss == nullptr || count == nullptr ||
+      (N > 0 && (E == nullptr || targets == nullptr || lse == nullptr || tile_max == nullptr)))
+    return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: a required pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(E) | reinterpret_cast<uintptr_t>(C)) & 15u)
+    return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: E and C must be 16-byte aligned");
+  // Same layout as the forward workspace: header | tile_sum [T, N] | z_target [N] | loss_rows [N].
+  const size_t off_sum = kHeader;
+  const size_t off_zt = up(off_sum + sizeof(float) * static_cast<size_t>(T * N));
+  const size_t off_rows = up(off_zt + sizeof(float) * static_cast<size_t>(N));
+  const size_t need = up(off_rows + sizeof(float) * static_cast<size_t>(N));
+  if (need > kNoAllocScratchBytes) {
+    char msg[256];
+    snprintf(msg, sizeof(msg),
+             "cce_forward_noalloc: this problem needs %zu bytes of scratch, more than the %zu bytes the library "
+             "holds for allocation-free calls (about ceil(V/128) * N * 4 bytes); use cce_forward with a workspace",
+             need, kNoAllocScratchBytes);
+    return fail(CCE_ERR_UNSUPPORTED, msg);
+  }
+  void* base = nullptr;
+  int num_sms = 0;
+  cce_status st = scratch_for_current_device(&base, &num_sms);
+  if (st != CCE_OK) return st;
+  char* b = static_cast<char*>(base);
+  int* err = reinterpret_cast<int*>(b);
+  float* tile_sum = reinterpret_cast<float*>(b + off_sum);
+  float* z_target = reinterpret_cast<float*>(b + off_zt);
+  float* loss_rows = reinterpret_cast<float*>(b + off_rows);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const auto* Eb = static_cast<const __nv_bfloat16*>(E);
+  const auto* Cb = static_cast<const __nv_bfloat16*>(C);
+
+  // The array keeps the previous call's contents: the error word must start at zero; every other
+  // scratch value is written before it is read.
+  if (cudaMemsetAsync(err, 0, kHeader, s) != cudaSuccess) return fail(CCE_ERR_CUDA, "cce_forward_noalloc: memset");
+  if (N > 0) {
+    cce::FwdLaunch L{};
+    if ((st = encode(&L.tmE, E, N, D, cce::kFwdBM)) != CCE_OK) return st;
+    if ((st = encode(&L.tmC, C, V, D, cce::kFwdBN)) != CCE_OK) return st;
+    L.N = static_cast<int>(N);
+    L.D = static_cast<int>(D);
+    L.V = static_cast<int>(V);
+    L.T = static_cast<int>(T);
+    L.tile_max = tile_max;
+    L.tile_sum = tile_sum;
+    L.err = err;
+    L.timeout_ns = 4000000000ull;
+    L.num_sms = num_sms;
+    if (cce::launch_target_logit(Eb, Cb, targets, N, D, V, p->ignore_index, z_target, err, s) != cudaSuccess ||
+        cce::launch_fwd_lse(L, s) != cudaSuccess ||
+        cce::launch_lse_loss(tile_max, tile_sum, z_target, targets, N, T, p->ignore_index, V, lse,
+                             p->reduction == CCE_REDUCTION_NONE ? loss : loss_rows, s) != cudaSuccess)
+      return fail(CCE_ERR_CUDA, "cce_forward_noalloc: kernel launch failed");
+  }
+  if (cce::launch_loss_reduce(loss_rows, targets, N, p->ignore_index, p->reduction, loss, count, s) != cudaSuccess)
+    return fail(CCE_ERR_CUDA, "cce_forward_noalloc: kernel launch failed");
+  return CCE_OK;
+}

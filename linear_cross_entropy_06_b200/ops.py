@@ -67,6 +67,7 @@ SIGNATURES = {
     "cce_version": (_I32, []),
     "cce_set_kernel_events": (None, [_VP, _VP, _VP, _VP]),
     "cce_kernel_launch_count": (_I64, []),
+    "cce_forward_noalloc": (_I32, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
