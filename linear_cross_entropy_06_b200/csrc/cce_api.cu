@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -124,6 +125,60 @@ BwdWs carve_bwd(const cce_problem* p, int32_t out_fp32, void* base) {
   return w;
 }
 
+// Workspace of the split backward: the tile plan, the gradient tiles of one vocabulary chunk and
+// the fp32 dE accumulator. dC needs no accumulator: each vocabulary tile's rows are summed in TMEM
+// and written once.
+struct SplitWs {
+  WsHeader* hdr;
+  float* scale;
+  cce::BwdPlan plan;
+  uint8_t* gscratch;
+  float* dE_acc;
+  int64_t chunk_tiles;  // vocabulary tiles per chunk
+  size_t bytes;
+};
+
+SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
+  const int64_t nb = ceil_div(p->N, cce::kBwdBM), nt = ceil_div(p->V, cce::kBwdBN);
+  const int64_t tiles = nb * nt;
+  SplitWs w{};
+  char* b = static_cast<char*>(base);
+  size_t off = kHeaderBytes;
+  auto take = [&](size_t bytes) {
+    char* ptr = b + off;
+    off = align_up(off + bytes);
+    return ptr;
+  };
+  w.hdr = reinterpret_cast<WsHeader*>(b);
+  w.scale = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N)));
+  w.plan.nb = static_cast<int>(nb);
+  w.plan.nt = static_cast<int>(nt);
+  w.plan.flags = reinterpret_cast<uint8_t*>(take(static_cast<size_t>(tiles)));
+  w.plan.rank = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(tiles)));
+  w.plan.cnt_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt)));
+  w.plan.offsets_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt + 1)));
+  w.plan.entries_t = reinterpret_cast<int2*>(take(sizeof(int2) * static_cast<size_t>(tiles)));
+  w.plan.cnt_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nb)));
+  w.plan.offsets_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nb + 1)));
+  w.plan.entries_b = reinterpret_cast<int2*>(take(sizeof(int2) * static_cast<size_t>(tiles)));
+  w.plan.kept_total = reinterpret_cast<int*>(take(sizeof(int)));
+  // Vocabulary tiles per chunk: the chunk's gradient tiles (at most nb of them per vocabulary
+  // tile) fit in the scratch budget; at least one vocabulary tile per chunk.
+  const int64_t per_vtile = std::max<int64_t>(nb, 1) * cce::kGradTileBytes;
+  w.chunk_tiles = std::max<int64_t>(1, std::min<int64_t>(nt, cce::kGradScratchBudget / per_vtile));
+  w.gscratch = reinterpret_cast<uint8_t*>(take(static_cast<size_t>(per_vtile * w.chunk_tiles)));
+  if (!out_fp32) w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
+  w.bytes = off;
+  return w;
+}
+
+// The fused per-tile backward (reduce-add of every tile's dE and dC partials) is kept only as the
+// measured comparison for the split design; CCE_BWD=fused selects it.
+bool use_fused_backward() {
+  const char* s = std::getenv("CCE_BWD");
+  return s != nullptr && s[0] == 'f';
+}
+
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 // ---------------------------------------------------------------------------------------------
@@ -173,6 +228,17 @@ cce_status make_map(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem, co
   return CCE_OK;
 }
 
+// L2 eviction hints of the backward kernel. By default E and the dE accumulator are kept (they are
+// re-read or re-added by every vocabulary tile) when together they leave room in the 126 MB L2 for
+// the C and dC tiles in flight. CCE_L2_HINTS=<bits> overrides (0 = no hints).
+uint32_t backward_l2_hints(int64_t N, int64_t D) {
+  if (const char* s = std::getenv("CCE_L2_HINTS")) return static_cast<uint32_t>(std::strtoul(s, nullptr, 0)) & 15u;
+  const double e_bytes = 2.0 * N * D, de_bytes = 4.0 * N * D;
+  uint32_t h = 0;
+  if (e_bytes + de_bytes <= 100.0 * (1 << 20)) h |= cce::kL2KeepE | cce::kL2KeepdE;
+  return h;
+}
+
 uint64_t wait_timeout_ns() {
   const char* s = std::getenv("CCE_WAIT_TIMEOUT_MS");
   double ms = s ? std::atof(s) : 4000.0;
@@ -191,6 +257,84 @@ uint64_t wait_timeout_ns() {
     cce_status s_ = (expr);        \
     if (s_ != CCE_OK) return s_;   \
   } while (0)
+
+// The split backward (see cce_bwd_g.cu and cce_bwd_gemm.cu): plan the tiles, then per vocabulary
+// chunk form the gradient tiles and run the dC and dE MMAs from them.
+cce_status backward_split(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
+                          const float* lse, const float* tile_max, const int64_t* count, const float* grad_out,
+                          float filter_eps, void* dE, void* dC, int32_t out_fp32, int64_t* filtered_tiles,
+                          void* workspace, size_t workspace_bytes, cudaStream_t s) {
+  const SplitWs w = carve_split(p, out_fp32, workspace);
+  if (workspace_bytes < w.bytes)
+    return fail(CCE_ERR_WORKSPACE, "backward workspace is %zu bytes, needs %zu", workspace_bytes, w.bytes);
+  int num_sms = 0;
+  CCE_CHECK(check_device(&num_sms));
+  CCE_CHECK(get_encoder());
+  const int64_t N = p->N, D = p->D, V = p->V, T = ceil_div(V, cce::kSubTile);
+  float* dE_acc = out_fp32 ? static_cast<float*>(dE) : w.dE_acc;
+
+  CCE_TRY(cudaMemsetAsync(w.hdr, 0, sizeof(WsHeader), s));
+  if (N == 0) {  // no rows: dC = 0
+    CCE_TRY(cce::launch_fill_zero(dC, V * D * (out_fp32 ? 4 : 2), s));
+    return cudaMemsetAsync(filtered_tiles, 0, sizeof(int64_t), s) == cudaSuccess ? CCE_OK
+                                                                                  : fail(CCE_ERR_CUDA, "memset");
+  }
+  CCE_TRY(cce::launch_row_scale(targets, count, grad_out, N, p->ignore_index, p->reduction, w.scale,
+                                &w.hdr->num_tiles, s));
+  CCE_TRY(cce::launch_bwd_plan(w.plan, tile_max, lse, targets, N, V, T, p->ignore_index, filter_eps, filtered_tiles,
+                               s));
+  CCE_TRY(cce::launch_fill_zero(dE_acc, N * D * 4, s));
+
+  cce::BwdGradTiles G{};
+  CCE_CHECK(make_map(&G.tmE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kBwdBM));
+  CCE_CHECK(make_map(&G.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, cce::kBwdBN));
+  G.N = static_cast<int>(N);
+  G.D = static_cast<int>(D);
+  G.V = static_cast<int>(V);
+  G.lse = lse;
+  G.scale = w.scale;
+  G.targets = targets;
+  G.ignore_index = p->ignore_index;
+  G.entries_t = w.plan.entries_t;
+  G.offsets_t = w.plan.offsets_t;
+  G.gscratch = w.gscratch;
+  G.max_entries_per_chunk = static_cast<int>(std::min<int64_t>(int64_t(w.plan.nb) * w.chunk_tiles, 1 << 30));
+  G.num_sms = num_sms;
+  G.err = &w.hdr->err;
+  G.timeout_ns = wait_timeout_ns();
+
+  cce::BwdGemm M{};
+  M.tmE = G.tmE;
+  M.tmC = G.tmC;
+  CCE_CHECK(make_map(&M.tmdE, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dE_acc, N, D, 32, 32));
+  if (out_fp32) CCE_CHECK(make_map(&M.tmdC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dC, V, D, 32, 32));
+  else CCE_CHECK(make_map(&M.tmdC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dC, V, D, 64, 32));
+  M.N = G.N;
+  M.D = G.D;
+  M.V = G.V;
+  M.nb = w.plan.nb;
+  M.entries_t = w.plan.entries_t;
+  M.offsets_t = w.plan.offsets_t;
+  M.entries_b = w.plan.entries_b;
+  M.offsets_b = w.plan.offsets_b;
+  M.gscratch = w.gscratch;
+  M.dC_bf16 = out_fp32 ? 0 : 1;
+  M.num_sms = num_sms;
+  M.err = G.err;
+  M.timeout_ns = G.timeout_ns;
+
+  if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
+  const int nt = w.plan.nt;
+  for (int64_t t0 = 0; t0 < nt; t0 += w.chunk_tiles) {
+    const int c0 = static_cast<int>(t0), c1 = static_cast<int>(std::min<int64_t>(nt, t0 + w.chunk_tiles));
+    CCE_TRY(cce::launch_bwd_g(G, c0, c1, s));
+    CCE_TRY(cce::launch_bwd_gemm(M, false, c0, c1, s));
+    CCE_TRY(cce::launch_bwd_gemm(M, true, c0, c1, s));
+  }
+  if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
+  if (!out_fp32) CCE_TRY(cce::launch_to_bf16(dE_acc, static_cast<__nv_bfloat16*>(dE), N * D, s));
+  return CCE_OK;
+}
 
 }  // namespace
 
@@ -245,7 +389,8 @@ size_t cce_forward_workspace_size(const cce_problem* p) {
 
 size_t cce_backward_workspace_size(const cce_problem* p, int32_t out_fp32) {
   if (!problem_ok(p, false)) return 0;
-  return carve_bwd(p, out_fp32 ? 1 : 0, nullptr).bytes;
+  if (use_fused_backward()) return carve_bwd(p, out_fp32 ? 1 : 0, nullptr).bytes;
+  return carve_split(p, out_fp32 ? 1 : 0, nullptr).bytes;
 }
 
 cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const int64_t* targets, float* loss,
@@ -284,6 +429,10 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
     L.err = &w.hdr->err;
     L.timeout_ns = wait_timeout_ns();
     L.num_sms = num_sms;
+    // Failure-detection test hook: CCE_TEST_INJECT_STALL=1 makes the forward's bounded wait run out
+    // (reported as CCE_ERR_DEVICE_TIMEOUT by cce_check_device_error; the outputs are undefined).
+    const char* stall = std::getenv("CCE_TEST_INJECT_STALL");
+    L.inject_stall = (stall != nullptr && stall[0] == '1') ? 1 : 0;
     CCE_TRY(cce::launch_target_logit(Eb, Cb, targets, N, D, V, p->ignore_index, w.z_target, &w.hdr->err, s));
     if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[0], s));
     CCE_TRY(cce::launch_fwd_lse(L, s));
@@ -311,6 +460,9 @@ cce_status cce_backward(const cce_problem* p, const void* E, const void* C, cons
     return fail(CCE_ERR_INVALID_ARG, "E, C, dE, dC and workspace must be 16-byte aligned");
   if (std::isnan(filter_eps)) return fail(CCE_ERR_INVALID_ARG, "filter_eps is NaN");
   out_fp32 = out_fp32 ? 1 : 0;
+  if (!use_fused_backward())
+    return backward_split(p, E, C, targets, lse, tile_max, count, grad_out, filter_eps, dE, dC, out_fp32,
+                          filtered_tiles, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
   const BwdWs w = carve_bwd(p, out_fp32, workspace);
   if (workspace_bytes < w.bytes)
     return fail(CCE_ERR_WORKSPACE, "backward workspace is %zu bytes, needs %zu", workspace_bytes, w.bytes);
@@ -346,6 +498,11 @@ cce_status cce_backward(const cce_problem* p, const void* E, const void* C, cons
     L.ignore_index = p->ignore_index;
     L.tiles = w.tiles;
     L.num_tiles = &w.hdr->num_tiles;
+    L.l2_hints = backward_l2_hints(N, D);
+    L.dE_acc = dE_acc;
+    L.dC_acc = dC_acc;
+    const char* flush = std::getenv("CCE_FLUSH");
+    L.direct_red = (flush != nullptr && flush[0] == 'r') ? 1 : 0;
     L.err = &w.hdr->err;
     L.timeout_ns = wait_timeout_ns();
     L.num_sms = num_sms;

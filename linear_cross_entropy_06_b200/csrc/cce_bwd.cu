@@ -73,12 +73,14 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+template <bool kDirectRed>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_grad_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC,
                     const __grid_constant__ CUtensorMap tmdE, const __grid_constant__ CUtensorMap tmdC, int N,
                     int D, int V, const float* __restrict__ lse, const float* __restrict__ scale,
                     const int64_t* __restrict__ targets, int64_t ignore_index, const int2* __restrict__ tiles,
-                    const int* __restrict__ num_tiles_ptr, int* err, uint64_t timeout_ns) {
+                    const int* __restrict__ num_tiles_ptr, uint32_t l2_hints, float* __restrict__ dE_acc,
+                    float* __restrict__ dC_acc, int* err, uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm = carve(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -131,6 +133,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued[STAGES] = {0, 0, 0};
       bool ok = true;
+      const uint64_t pol_last = policy_evict_last(), pol_first = policy_evict_first();
+      const bool keepE = (l2_hints & kL2KeepE) != 0, streamC = (l2_hints & kL2StreamC) != 0;
+      auto load_E = [&](uint32_t dst, uint32_t bar, int x, int y) {
+        if (keepE) tma_load_2d_hint(dst, &tmE, bar, x, y, pol_last);
+        else tma_load_2d(dst, &tmE, bar, x, y);
+      };
+      auto load_C = [&](uint32_t dst, uint32_t bar, int x, int y) {
+        if (streamC) tma_load_2d_hint(dst, &tmC, bar, x, y, pol_first);
+        else tma_load_2d(dst, &tmC, bar, x, y);
+      };
       for (int i = blockIdx.x; i < num_tiles && ok; i += gridDim.x) {
         const int2 bt = tiles[i];
         const int rb = bt.x * BM, vb = bt.y * BN;
@@ -142,12 +154,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t dst = smem_u32(sm.stage + stage * STAGE_BYTES);
           mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
           if (step < num_kb) {  // recompute operands: E_b | C_t, K block `step`
-            tma_load_2d(dst, &tmE, full_bar(stage), step * BK, rb);
-            tma_load_2d(dst + HALF, &tmC, full_bar(stage), step * BK, vb);
+            load_E(dst, full_bar(stage), step * BK, rb);
+            load_C(dst + HALF, full_bar(stage), step * BK, vb);
           } else {  // gradient operands: C_t | E_b, D chunk `c`
             const int c = step - num_kb;
-            tma_load_2d(dst, &tmC, full_bar(stage), c * DC, vb);
-            tma_load_2d(dst + HALF, &tmE, full_bar(stage), c * DC, rb);
+            load_C(dst, full_bar(stage), c * DC, vb);
+            load_E(dst + HALF, full_bar(stage), c * DC, rb);
           }
           ++issued[stage];
           if (++stage == STAGES) {
@@ -241,6 +253,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t g0 = smem_u32(sm.g);
     const uint32_t stg = smem_u32(sm.stg + q * STG_WARP);
+    const uint64_t pol_last = policy_evict_last(), pol_first = policy_evict_first();
+    const bool keep_dE = (l2_hints & kL2KeepdE) != 0, stream_dC = (l2_hints & kL2StreamdC) != 0;
+    auto add_dE = [&](uint32_t src, int x, int y) {
+      if (keep_dE) tma_reduce_add_2d_hint(&tmdE, src, x, y, pol_last);
+      else tma_reduce_add_2d(&tmdE, src, x, y);
+    };
+    auto add_dC = [&](uint32_t src, int x, int y) {
+      if (stream_dC) tma_reduce_add_2d_hint(&tmdC, src, x, y, pol_first);
+      else tma_reduce_add_2d(&tmdC, src, x, y);
+    };
     uint32_t tile_iter = 0, gc = 0;
     bool ok = true;
     for (int i = blockIdx.x; i < num_tiles && ok; i += gridDim.x, ++tile_iter) {
@@ -290,8 +312,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         }
         tc_fence_after();
-        float e0[32], e1[32], c0[32], c1[32];
         const uint32_t t_de = tmem_base + lane_off + 128u + 128u * u;
+        if constexpr (kDirectRed) {
+          // Registers -> L2 with red.global.add.v2.f32: the 16x256b load shape gives four threads
+          // 8 consecutive columns of one row, so every warp instruction adds whole 32-byte sectors.
+          float a0[32], a1[32], b0[32], b1[32];
+          tmem_ld16x256b_x8(t_de, a0);
+          tmem_ld16x256b_x8(t_de + (16u << 16), a1);
+          tmem_ld16x256b_x8(t_de + 64u, b0);
+          tmem_ld16x256b_x8(t_de + 64u + (16u << 16), b1);
+          tc_fence_before();
+          mbar_arrive(gradempty_bar(u));
+          const int t0 = lane & 3, t1 = lane >> 2;
+          const int rE = bt.x * BM + q * 32 + t1, rC = bt.y * BN + q * 32 + t1;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int col = c * DC + 8 * k + 2 * t0;
+            if (col >= D) continue;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {  // rows +0, +8 (first 16 lanes), +16, +24 (second 16 lanes)
+              const float* src_e = g < 2 ? a0 : a1;
+              const float* src_c = g < 2 ? b0 : b1;
+              const int reg = 4 * k + 2 * (g & 1);
+              const int roff = (g >> 1) * 16 + (g & 1) * 8;
+              if (rE + roff < N)
+                red_add_v2(dE_acc + static_cast<size_t>(rE + roff) * D + col, src_e[reg], src_e[reg + 1]);
+              if (rC + roff < V)
+                red_add_v2(dC_acc + static_cast<size_t>(rC + roff) * D + col, src_c[reg], src_c[reg + 1]);
+            }
+          }
+          continue;
+        }
+        float e0[32], e1[32], c0[32], c1[32];
         tmem_ld32(t_de, e0);
         tmem_ld32(t_de + 32u, e1);
         tmem_ld32(t_de + 64u, c0);
@@ -319,12 +371,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int x = c * DC;
           const int ye = bt.x * BM + q * 32, yc = bt.y * BN + q * 32;
           if (ye < N) {
-            tma_reduce_add_2d(&tmdE, stg, x, ye);
-            if (x + 32 < D) tma_reduce_add_2d(&tmdE, stg + 4096u, x + 32, ye);
+            add_dE(stg, x, ye);
+            if (x + 32 < D) add_dE(stg + 4096u, x + 32, ye);
           }
           if (yc < V) {
-            tma_reduce_add_2d(&tmdC, stg + 8192u, x, yc);
-            if (x + 32 < D) tma_reduce_add_2d(&tmdC, stg + 12288u, x + 32, yc);
+            add_dC(stg + 8192u, x, yc);
+            if (x + 32 < D) add_dC(stg + 12288u, x + 32, yc);
           }
           bulk_commit_group();
         }
@@ -351,12 +403,13 @@ cudaError_t launch_bwd_grad(const BwdLaunch& L, cudaStream_t s) {
   const long long nt = (L.V + BN - 1) / BN;
   const long long max_tiles = nb * nt;
   if (max_tiles == 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  auto kernel = L.direct_red ? bwd_grad_kernel<true> : bwd_grad_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(max_tiles < L.num_sms ? max_tiles : L.num_sms);
-  bwd_grad_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmC, L.tmdE, L.tmdC, L.N, L.D, L.V, L.lse, L.scale,
-                                                        L.targets, L.ignore_index, L.tiles, L.num_tiles, L.err,
-                                                        L.timeout_ns);
+  kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmC, L.tmdE, L.tmdC, L.N, L.D, L.V, L.lse, L.scale, L.targets,
+                                               L.ignore_index, L.tiles, L.num_tiles, L.l2_hints, L.dE_acc, L.dC_acc,
+                                               L.err, L.timeout_ns);
   note_launches(1);
   return cudaGetLastError();
 }

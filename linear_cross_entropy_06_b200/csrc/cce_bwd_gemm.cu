@@ -1,0 +1,385 @@
+// Backward, steps 2 and 3 of 3 per vocabulary chunk: the gradient MMAs, from bf16 gradient tiles
+// in shared memory, with fp32 accumulation in TMEM.
+//
+//   dC mode  work item (vocabulary tile t, 256-column slice s of D):
+//            dC[t rows, s cols] = sum over listed b of G_bt^T E_b[:, s]     (written directly; every
+//            listed tile of t is in this chunk, so no reduction is needed)
+//   dE mode  work item (row block b, slice s):
+//            dE[b rows, s cols] += sum over listed t in the chunk of G_bt C_t[:, s]
+//            (one fp32 TMA reduce-add per item and chunk: split-reduce over vocabulary chunks)
+//
+// mlx-cross-entropy README, "How it works" item 3 (gradients accumulated without intermediate
+// [batch, tiles, D] buffers); Loss functions explainer, "How it works" item 2 (dE = G C and
+// dC = G^T E with G = p - y). The gradient tiles come from the recompute kernel (cce_bwd_g.cu).
+//
+// Design (B200): one persistent CTA per SM, 6 warps.
+//   warp 0      producer: per listed tile, the 32 KB gradient tile (bulk copy from the chunk
+//               scratch) and the 128 x 256 operand slice (TMA, 128B swizzle, two 32 KB halves)
+//               into a ring of six 32 KB units.
+//   warp 1      TMEM: two 256-column fp32 accumulators; one lane issues tcgen05.mma M=128 N=128
+//               per half slice (dC: A = G read MN-major as G^T; dE: A = G K-major; B = the slice,
+//               MN-major).
+//   warps 2..5  write-out: TMEM -> registers -> swizzled staging -> TMA store (dC, bf16 or fp32)
+//               or TMA reduce-add (dE, fp32), while the MMA fills the other accumulator.
+#include "cce_device.cuh"
+#include "cce_internal.h"
+
+namespace cce {
+namespace {
+
+constexpr int BM = kBwdBM;
+constexpr int BN = kBwdBN;
+constexpr int SLICE = kGemmSlice;  // 256 columns of D per work item
+constexpr int UNITS = 6;
+constexpr int UNIT_BYTES = 32768;
+constexpr int BOX_BYTES = 16384;  // 128 rows x 64 bf16
+constexpr int STG_WARP = 8192;    // per epilogue warp: 32 rows x 64 columns of fp32 (or bf16 + unused)
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 512;
+constexpr int NUM_BARRIERS = 2 * UNITS + 4 + 1;
+constexpr int SMEM_BYTES = 1024 + UNITS * UNIT_BYTES + 4 * STG_WARP + NUM_BARRIERS * 8 + 16;
+
+constexpr uint32_t IDESC_DC = idesc_bf16(BN, 128, true, true);   // M = vocab (G^T, MN-major), N = 128 of D
+constexpr uint32_t IDESC_DE = idesc_bf16(BM, 128, false, true);  // M = rows (G, K-major), N = 128 of D
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map), "r"(src),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
+struct ItemRange {
+  int key, s, begin, end;  // entries [begin, end) of the key's list
+};
+
+// The work item's key tile, slice, and the range of its list entries inside this chunk.
+template <bool kDE>
+__device__ __forceinline__ ItemRange item_range(int w, int S, int chunk_t0, int chunk_t1, const int* offsets) {
+  ItemRange it;
+  it.s = w % S;
+  if (!kDE) {
+    it.key = chunk_t0 + w / S;
+    it.begin = offsets[it.key];
+    it.end = offsets[it.key + 1];
+    return it;
+  }
+  it.key = w / S;
+  // entries_b of row block b are sorted by vocabulary tile; the caller narrows to the chunk.
+  it.begin = offsets[it.key];
+  it.end = offsets[it.key + 1];
+  return it;
+}
+
+__device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int t) {
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (e[mid].x < t) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+template <bool kDE>
+__device__ __forceinline__ ItemRange item_in_chunk(int w, int S, int chunk_t0, int chunk_t1, const int* offsets,
+                                                   const int2* entries) {
+  ItemRange it = item_range<kDE>(w, S, chunk_t0, chunk_t1, offsets);
+  if (kDE) {
+    const int lo = lower_bound_t(entries, it.begin, it.end, chunk_t0);
+    const int hi = lower_bound_t(entries, lo, it.end, chunk_t1);
+    it.begin = lo;
+    it.end = hi;
+  }
+  return it;
+}
+
+// Entry i of a list -> (tile index of the "other" operand, slot of its gradient tile in the chunk).
+template <bool kDE>
+__device__ __forceinline__ int2 entry_of(const int2* entries, int i, int slot_base) {
+  const int2 en = entries[i];
+  if (!kDE) return make_int2(en.x >> 2, i - slot_base);  // (row block b, slot)
+  return make_int2(en.x, en.y - slot_base);              // (vocabulary tile t, slot)
+}
+
+template <bool kDE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmOut, int N, int D,
+                    int V, const int2* __restrict__ entries, const int* __restrict__ offsets,
+                    const int* __restrict__ offsets_t, int chunk_t0, int chunk_t1, int num_keys,
+                    const uint8_t* __restrict__ gscratch, int out_bf16, int* err, uint64_t timeout_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* units = base;
+  uint8_t* stg_all = base + UNITS * UNIT_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg_all + 4 * STG_WARP);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NUM_BARRIERS);
+  int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int u) { return bar0 + 8u * u; };
+  auto empty_bar = [&](int u) { return bar0 + 8u * (UNITS + u); };
+  auto accfull_bar = [&](int a) { return bar0 + 8u * (2 * UNITS + a); };
+  auto accempty_bar = [&](int a) { return bar0 + 8u * (2 * UNITS + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * UNITS + 4);
+
+  const int S = (D + SLICE - 1) / SLICE;
+  const int num_items = num_keys * S;
+  if (num_items <= static_cast<int>(blockIdx.x)) return;
+  const int slot_base = offsets_t[chunk_t0];
+
+  if (threadIdx.x == 0) {
+    for (int u = 0; u < UNITS; ++u) {
+      mbar_init(full_bar(u), 1);
+      mbar_init(empty_bar(u), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accfull_bar(a), 1);
+      mbar_init(accempty_bar(a), 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const WaitCtl wc{abort_flag, err, timeout_ns};
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      int unit = 0;
+      uint32_t phase = 0;
+      uint32_t issued[UNITS] = {0, 0, 0, 0, 0, 0};
+      bool ok = true;
+      auto acquire = [&](uint32_t bytes) -> uint32_t {
+        if (!mbar_wait(empty_bar(unit), phase ^ 1u, wc)) return 0xffffffffu;
+        mbar_arrive_expect_tx(full_bar(unit), bytes);
+        ++issued[unit];
+        return static_cast<uint32_t>(unit);
+      };
+      auto advance = [&]() {
+        if (++unit == UNITS) {
+          unit = 0;
+          phase ^= 1u;
+        }
+      };
+      for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
+        const ItemRange it = item_in_chunk<kDE>(w, S, chunk_t0, chunk_t1, offsets, entries);
+        const int x0 = it.s * SLICE;
+        const int halves = (D - x0 > 128) ? 2 : 1;
+        for (int i = it.begin; i < it.end && ok; ++i) {
+          const int2 os = entry_of<kDE>(entries, i, slot_base);
+          // gradient tile
+          uint32_t u = acquire(UNIT_BYTES);
+          if (u == 0xffffffffu) {
+            ok = false;
+            break;
+          }
+          bulk_load(smem_u32(units + u * UNIT_BYTES), gscratch + static_cast<size_t>(os.y) * UNIT_BYTES, UNIT_BYTES,
+                    full_bar(u));
+          advance();
+          // operand slice halves: rows of E_b (dC) or C_t (dE), columns x0 .. x0 + 255
+          for (int h = 0; h < halves; ++h) {
+            u = acquire(UNIT_BYTES);
+            if (u == 0xffffffffu) {
+              ok = false;
+              break;
+            }
+            const uint32_t dst = smem_u32(units + u * UNIT_BYTES);
+            const int y = os.x * BM;
+            tma_load_2d(dst, &tmX, full_bar(u), x0 + 128 * h, y);
+            tma_load_2d(dst + BOX_BYTES, &tmX, full_bar(u), x0 + 128 * h + 64, y);
+            advance();
+          }
+        }
+      }
+      if (!ok) {
+        for (int u = 0; u < UNITS; ++u)
+          if (issued[u]) mbar_wait_drain(full_bar(u), (issued[u] - 1u) & 1u, 200000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int unit = 0;
+      uint32_t phase = 0;
+      uint32_t acc_iter = 0;
+      bool ok = true, issued_any = false;
+      auto wait_unit = [&]() -> int {
+        if (!mbar_wait(full_bar(unit), phase, wc)) return -1;
+        tc_fence_after();
+        const int u = unit;
+        if (++unit == UNITS) {
+          unit = 0;
+          phase ^= 1u;
+        }
+        return u;
+      };
+      for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
+        const ItemRange it = item_in_chunk<kDE>(w, S, chunk_t0, chunk_t1, offsets, entries);
+        if (it.begin == it.end) continue;  // nothing to accumulate (dC writes zeros without TMEM)
+        const int halves = (D - it.s * SLICE > 128) ? 2 : 1;
+        const int a = acc_iter & 1;
+        if (!mbar_wait(accempty_bar(a), ((acc_iter >> 1) & 1u) ^ 1u, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int i = it.begin; i < it.end && ok; ++i) {
+          const int ug = wait_unit();
+          if (ug < 0) {
+            ok = false;
+            break;
+          }
+          const uint32_t g0 = smem_u32(units + ug * UNIT_BYTES);
+          for (int h = 0; h < halves; ++h) {
+            const int ux = wait_unit();
+            if (ux < 0) {
+              ok = false;
+              break;
+            }
+            const uint32_t x0 = smem_u32(units + ux * UNIT_BYTES);
+            const uint32_t d = tmem_base + static_cast<uint32_t>(a * SLICE + h * 128);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {  // K = 128 (rows for dC, vocabulary for dE), 16 per MMA
+              uint64_t adesc;
+              if (kDE) adesc = sdesc_sw128(g0 + (k >> 2) * BOX_BYTES + 32u * (k & 3), 16, 1024);
+              else adesc = sdesc_sw128(g0 + 2048u * k, BOX_BYTES, 1024);
+              const uint64_t bdesc = sdesc_sw128(x0 + 2048u * k, BOX_BYTES, 1024);
+              tc_mma_bf16(d, adesc, bdesc, kDE ? IDESC_DE : IDESC_DC, (i > it.begin || k > 0) ? 1u : 0u);
+            }
+            issued_any = true;
+            tc_commit(empty_bar(ux));
+          }
+          if (!ok) break;
+          tc_commit(empty_bar(ug));
+        }
+        if (!ok) break;
+        tc_commit(accfull_bar(a));
+        ++acc_iter;
+      }
+      if (!ok && issued_any) {
+        tc_commit(drain_bar);
+        mbar_wait_drain(drain_bar, 0, 200000000ull);
+      }
+    }
+  } else {
+    // ---------------- write-out ----------------
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t stg = smem_u32(stg_all + q * STG_WARP);
+    const int rows_limit = kDE ? N : V;
+    uint32_t acc_iter = 0;
+    for (int w = blockIdx.x; w < num_items; w += gridDim.x) {
+      const ItemRange it = item_in_chunk<kDE>(w, S, chunk_t0, chunk_t1, offsets, entries);
+      const bool has = it.begin < it.end;
+      if (kDE && !has) continue;  // nothing to add for this row block in this chunk
+      const int a = acc_iter & 1;
+      if (has) {
+        if (!mbar_wait(accfull_bar(a), (acc_iter >> 1) & 1u, wc)) break;
+        tc_fence_after();
+      }
+      const int y = it.key * BM + q * 32;
+      for (int p = 0; p < SLICE / 64; ++p) {
+        const int x = it.s * SLICE + 64 * p;
+        if (x >= D) break;
+        float v0[32], v1[32];
+        if (has) {
+          tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * SLICE + 64 * p), v0);
+          tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * SLICE + 64 * p + 32), v1);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v0[k] = v1[k] = 0.f;
+        }
+        // This warp's staging is free once its previous TMA op has read it.
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+        if (!kDE && out_bf16) {
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            const float* src = h < 4 ? v0 + 8 * h : v1 + 8 * (h - 4);
+            st_shared_v4(stg + swz(lane, h), pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                         pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            st_shared_v4(stg + swz(lane, h), __float_as_uint(v0[4 * h]), __float_as_uint(v0[4 * h + 1]),
+                         __float_as_uint(v0[4 * h + 2]), __float_as_uint(v0[4 * h + 3]));
+            st_shared_v4(stg + 4096u + swz(lane, h), __float_as_uint(v1[4 * h]), __float_as_uint(v1[4 * h + 1]),
+                         __float_as_uint(v1[4 * h + 2]), __float_as_uint(v1[4 * h + 3]));
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && y < rows_limit) {
+          if (!kDE && out_bf16) {
+            tma_store_2d(&tmOut, stg, x, y);
+          } else if (!kDE) {
+            tma_store_2d(&tmOut, stg, x, y);
+            if (x + 32 < D) tma_store_2d(&tmOut, stg + 4096u, x + 32, y);
+          } else {
+            tma_reduce_add_2d(&tmOut, stg, x, y);
+            if (x + 32 < D) tma_reduce_add_2d(&tmOut, stg + 4096u, x + 32, y);
+          }
+          bulk_commit_group();
+        }
+      }
+      if (has) {
+        tc_fence_before();
+        mbar_arrive(accempty_bar(a));
+        ++acc_iter;
+      }
+    }
+    if (lane == 0) bulk_wait_group0();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_gemm(const BwdGemm& L, bool dE_mode, int chunk_t0, int chunk_t1, cudaStream_t s) {
+  const int S = (L.D + SLICE - 1) / SLICE;
+  const int num_keys = dE_mode ? L.nb : (chunk_t1 - chunk_t0);
+  const long long items = static_cast<long long>(num_keys) * S;
+  if (items <= 0) return cudaSuccess;
+  auto kernel = dE_mode ? bwd_gemm_kernel<true> : bwd_gemm_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int grid = static_cast<int>(items < L.num_sms ? items : L.num_sms);
+  if (dE_mode)
+    kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmC, L.tmdE, L.N, L.D, L.V, L.entries_b, L.offsets_b, L.offsets_t,
+                                                 chunk_t0, chunk_t1, num_keys, L.gscratch, 0, L.err, L.timeout_ns);
+  else
+    kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmdC, L.N, L.D, L.V, L.entries_t, L.offsets_t, L.offsets_t,
+                                                 chunk_t0, chunk_t1, num_keys, L.gscratch, L.dC_bf16, L.err,
+                                                 L.timeout_ns);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace cce

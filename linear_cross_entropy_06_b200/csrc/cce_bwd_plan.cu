@@ -1,0 +1,173 @@
+// Planning of the backward: which (row block b, vocabulary tile t) tiles carry gradient, and two
+// compact lists of them.
+//
+// A tile of 128 rows x 128 vocabulary columns is kept when some non-ignored row r of block b has
+// max over the tile of z[r, v] - LSE_r >= ln(eps) (mlx-cross-entropy README, "How it works" item 2:
+// skip tiles whose softmax is below 2^-12), judged from the forward's saved per-sub-tile maxima.
+// A skipped tile that holds the target of one of its rows still carries the onehot term of
+// p - y (Loss functions explainer, "How it works" item 2), which is never skipped; it is listed as
+// "onehot only" (its gradient tile is -scale_r at (r, t_r) and zero elsewhere, no recompute).
+//
+// flags[b * nt + t]: 0 = no gradient, 1 = kept, 2 = onehot only.
+// By vocabulary tile (recompute and dC kernels): offsets_t[t] .. offsets_t[t+1] index entries_t,
+//   each (b * 4 + flag, t), row blocks ascending. An entry's position is also its gradient-tile slot.
+// By row block (dE kernel): offsets_b[b] .. offsets_b[b+1] index entries_b, each (t, slot),
+//   vocabulary tiles ascending.
+#include "cce_device.cuh"
+#include "cce_internal.h"
+
+namespace cce {
+namespace {
+
+__device__ __forceinline__ bool valid_target(int64_t t, int64_t V, int64_t ignore_index) {
+  return t != ignore_index && t >= 0 && t < V;
+}
+
+// One block (128 threads, one per tile row) per vocabulary tile, walking the row blocks in order.
+__global__ void tile_flags_kernel(const float* __restrict__ tile_max, const float* __restrict__ lse,
+                                  const int64_t* __restrict__ targets, int64_t N, int64_t V, int64_t T,
+                                  int64_t ignore_index, float ln_eps, int filter_on, int nb, uint8_t* __restrict__ flags,
+                                  int* __restrict__ rank, int* __restrict__ cnt_t, int* __restrict__ kept_total) {
+  __shared__ float wmax[4];
+  const int t = blockIdx.x;
+  const int nt = gridDim.x;
+  const int64_t v0 = static_cast<int64_t>(t) * kBwdBN;
+  int listed = 0, kept = 0;
+  for (int b = 0; b < nb; ++b) {
+    const int64_t r = static_cast<int64_t>(b) * kBwdBM + threadIdx.x;
+    float m = -INFINITY;
+    bool has_target = false;
+    if (r < N) {
+      const int64_t tr = targets[r];
+      if (valid_target(tr, V, ignore_index)) {
+        has_target = tr >= v0 && tr < v0 + kBwdBN;
+        if (filter_on) {
+          const int64_t j0 = static_cast<int64_t>(t) * (kBwdBN / kSubTile);
+          const int64_t j1 = j0 + kBwdBN / kSubTile < T ? j0 + kBwdBN / kSubTile : T;
+          for (int64_t j = j0; j < j1; ++j) m = fmaxf(m, tile_max[j * N + r]);
+          m -= lse[r];
+        }
+      }
+    }
+    bool keep = true;
+    if (filter_on) {
+      m = warp_max(m);
+      if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+    }
+    const int any_target = __syncthreads_or(has_target ? 1 : 0);
+    if (filter_on) {
+      const float bm = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+      keep = bm >= ln_eps;
+    }
+    const uint8_t f = keep ? 1 : (any_target ? 2 : 0);
+    if (threadIdx.x == 0) {
+      flags[static_cast<int64_t>(b) * nt + t] = f;
+      rank[static_cast<int64_t>(b) * nt + t] = listed;
+    }
+    listed += f != 0;
+    kept += f == 1;
+    __syncthreads();  // wmax is rewritten for the next row block
+  }
+  if (threadIdx.x == 0) {
+    cnt_t[t] = listed;
+    atomicAdd(kept_total, kept);
+  }
+}
+
+// Exclusive scan of cnt[0..n) into off[0..n]; one block of 1024 threads, in chunks.
+__global__ void scan_kernel(const int* __restrict__ cnt, int n, int* __restrict__ off) {
+  __shared__ int buf[1024];
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < n; base += 1024) {
+    const int i = base + threadIdx.x;
+    const int v = i < n ? cnt[i] : 0;
+    buf[threadIdx.x] = v;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+      const int add = threadIdx.x >= o ? buf[threadIdx.x - o] : 0;
+      __syncthreads();
+      buf[threadIdx.x] += add;
+      __syncthreads();
+    }
+    if (i < n) off[i] = carry + buf[threadIdx.x] - v;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry += buf[1023];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) off[n] = carry;
+}
+
+__global__ void fill_col_kernel(const uint8_t* __restrict__ flags, const int* __restrict__ rank,
+                                const int* __restrict__ offsets_t, int nb, int nt, int2* __restrict__ entries_t) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<int64_t>(nb) * nt) return;
+  const uint8_t f = flags[i];
+  if (f == 0) return;
+  const int b = static_cast<int>(i / nt), t = static_cast<int>(i % nt);
+  entries_t[offsets_t[t] + rank[i]] = make_int2(b * 4 + f, t);
+}
+
+// One warp per row block: counts (pass 0) or writes (pass 1) its listed tiles in vocabulary order.
+__global__ void row_list_kernel(const uint8_t* __restrict__ flags, const int* __restrict__ rank,
+                                const int* __restrict__ offsets_t, int nb, int nt, int* __restrict__ cnt_b,
+                                const int* __restrict__ offsets_b, int2* __restrict__ entries_b, int pass) {
+  const int b = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (b >= nb) return;
+  const uint8_t* row = flags + static_cast<int64_t>(b) * nt;
+  int k = 0;
+  for (int t0 = 0; t0 < nt; t0 += 32) {
+    const int t = t0 + lane;
+    const bool on = t < nt && row[t] != 0;
+    const unsigned mask = __ballot_sync(0xffffffffu, on);
+    if (pass == 1 && on) {
+      const int pos = offsets_b[b] + k + __popc(mask & ((1u << lane) - 1u));
+      entries_b[pos] = make_int2(t, offsets_t[t] + rank[static_cast<int64_t>(b) * nt + t]);
+    }
+    k += __popc(mask);
+  }
+  if (pass == 0 && lane == 0) cnt_b[b] = k;
+}
+
+__global__ void plan_finish_kernel(const int* __restrict__ kept_total, int64_t total, int64_t* __restrict__ filtered) {
+  *filtered = total - static_cast<int64_t>(*kept_total);
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float* lse, const int64_t* targets,
+                            int64_t N, int64_t V, int64_t T, int64_t ignore_index, float filter_eps,
+                            int64_t* filtered_tiles, cudaStream_t s) {
+  const int nb = P.nb, nt = P.nt;
+  const int filter_on = filter_eps > 0.f ? 1 : 0;
+  const float ln_eps = filter_on ? logf(filter_eps) : -INFINITY;
+  cudaError_t e = cudaMemsetAsync(P.kept_total, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  if (nb > 0) {
+    tile_flags_kernel<<<nt, kBwdBM, 0, s>>>(tile_max, lse, targets, N, V, T, ignore_index, ln_eps, filter_on, nb,
+                                            P.flags, P.rank, P.cnt_t, P.kept_total);
+    note_launches(1);
+    scan_kernel<<<1, 1024, 0, s>>>(P.cnt_t, nt, P.offsets_t);
+    note_launches(1);
+    const int64_t tiles = static_cast<int64_t>(nb) * nt;
+    fill_col_kernel<<<static_cast<int>((tiles + 255) / 256), 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt,
+                                                                          P.entries_t);
+    note_launches(1);
+    const int grid_b = (nb * 32 + 255) / 256;
+    row_list_kernel<<<grid_b, 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt, P.cnt_b, P.offsets_b, P.entries_b,
+                                           0);
+    note_launches(1);
+    scan_kernel<<<1, 1024, 0, s>>>(P.cnt_b, nb, P.offsets_b);
+    note_launches(1);
+    row_list_kernel<<<grid_b, 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt, P.cnt_b, P.offsets_b, P.entries_b,
+                                           1);
+    note_launches(1);
+  }
+  plan_finish_kernel<<<1, 1, 0, s>>>(P.kept_total, static_cast<int64_t>(nb) * nt, filtered_tiles);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace cce

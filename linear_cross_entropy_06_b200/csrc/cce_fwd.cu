@@ -54,7 +54,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_lse_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC, int N, int D,
                    int V, int T, float* __restrict__ tile_max, float* __restrict__ tile_sum, int* err,
-                   uint64_t timeout_ns) {
+                   uint64_t timeout_ns, int inject_stall) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm = carve(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -97,7 +97,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
-    if (lane == 0) {
+    // inject_stall (test hook): issue no loads at all, so the MMA warp's first bounded wait runs
+    // out and the kernel reports kErrDeviceTimeout. Nothing is left in flight in that case.
+    if (lane == 0 && !inject_stall) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued[STAGES] = {0, 0, 0, 0};
@@ -243,7 +245,7 @@ cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(total < L.num_sms ? total : L.num_sms);
   fwd_lse_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmC, L.N, L.D, L.V, L.T, L.tile_max, L.tile_sum,
-                                                       L.err, L.timeout_ns);
+                                                       L.err, L.timeout_ns, L.inject_stall);
   note_launches(1);
   return cudaGetLastError();
 }

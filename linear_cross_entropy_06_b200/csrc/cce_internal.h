@@ -17,6 +17,12 @@ constexpr int kSubTile = 128;  // vocabulary width of one saved tile max
 constexpr int kBwdBM = 128;
 constexpr int kBwdBN = 128;
 
+// L2 eviction hints of the backward kernel (bits of BwdLaunch::l2_hints).
+constexpr uint32_t kL2KeepE = 1;        // E tile loads: evict_last (E is re-read by every vocab tile)
+constexpr uint32_t kL2KeepdE = 2;       // dE reduce-adds: evict_last (every vocab tile adds into dE)
+constexpr uint32_t kL2StreamC = 4;      // C tile loads: evict_first
+constexpr uint32_t kL2StreamdC = 8;     // dC reduce-adds: evict_first
+
 struct FwdLaunch {
   CUtensorMap tmE;  // bf16 [N, D], box 64 x 128, 128B swizzle
   CUtensorMap tmC;  // bf16 [V, D], box 64 x 256, 128B swizzle
@@ -26,6 +32,7 @@ struct FwdLaunch {
   int* err;
   uint64_t timeout_ns;
   int num_sms;
+  int inject_stall;  // test hook: the producer issues nothing, so a bounded wait runs out
 };
 
 struct BwdLaunch {
@@ -40,6 +47,10 @@ struct BwdLaunch {
   int64_t ignore_index;
   const int2* tiles;    // kept tiles (row block, vocab tile)
   const int* num_tiles; // device count of kept tiles
+  uint32_t l2_hints;    // kL2* bits: which streams get an L2 eviction-priority hint
+  float* dE_acc;        // fp32 accumulators (the direct-red flush adds into them by address)
+  float* dC_acc;
+  int direct_red;       // 1: flush with red.global.add from registers; 0: smem staging + TMA reduce
   int* err;
   uint64_t timeout_ns;
   int num_sms;
@@ -50,6 +61,62 @@ void note_launches(int n);
 
 // Sets the message cce_last_error_message() returns on the calling thread.
 void set_last_error(const char* msg);
+
+// Split backward (cce_bwd_plan.cu, cce_bwd_g.cu, cce_bwd_gemm.cu).
+constexpr int kGradTileBytes = kBwdBM * kBwdBN * 2;      // one bf16 gradient tile, 128B-swizzled
+constexpr int kGemmSlice = 256;                           // columns of D per dC/dE work item
+constexpr int64_t kGradScratchBudget = int64_t(128) << 20;  // gradient tiles of one vocabulary chunk
+
+struct BwdPlan {
+  int nb, nt;
+  uint8_t* flags;   // [nb * nt]: 0 none, 1 kept, 2 onehot only
+  int* rank;        // [nb * nt]: position of (b, t) among the listed row blocks of t
+  int* cnt_t;       // [nt]
+  int* offsets_t;   // [nt + 1]
+  int2* entries_t;  // [nb * nt]: (b * 4 + flag, t), by vocabulary tile then row block
+  int* cnt_b;       // [nb]
+  int* offsets_b;   // [nb + 1]
+  int2* entries_b;  // [nb * nt]: (t, slot in entries_t), by row block then vocabulary tile
+  int* kept_total;
+};
+
+struct BwdGradTiles {
+  CUtensorMap tmE, tmC;  // bf16, box 64 x 128
+  int N, D, V;
+  const float* lse;
+  const float* scale;
+  const int64_t* targets;
+  int64_t ignore_index;
+  const int2* entries_t;
+  const int* offsets_t;
+  uint8_t* gscratch;
+  int max_entries_per_chunk;
+  int num_sms;
+  int* err;
+  uint64_t timeout_ns;
+};
+
+struct BwdGemm {
+  CUtensorMap tmE, tmC;  // bf16, box 64 x 128 (operand slices)
+  CUtensorMap tmdE;      // fp32 dE accumulator, box 32 x 32 (reduce-add)
+  CUtensorMap tmdC;      // dC output: bf16 box 64 x 32, or fp32 box 32 x 32
+  int N, D, V, nb;
+  const int2* entries_t;
+  const int* offsets_t;
+  const int2* entries_b;
+  const int* offsets_b;
+  const uint8_t* gscratch;
+  int dC_bf16;
+  int num_sms;
+  int* err;
+  uint64_t timeout_ns;
+};
+
+cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float* lse, const int64_t* targets,
+                            int64_t N, int64_t V, int64_t T, int64_t ignore_index, float filter_eps,
+                            int64_t* filtered_tiles, cudaStream_t s);
+cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk_t0, int chunk_t1, cudaStream_t s);
+cudaError_t launch_bwd_gemm(const BwdGemm& L, bool dE_mode, int chunk_t0, int chunk_t1, cudaStream_t s);
 
 cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
 cudaError_t launch_bwd_grad(const BwdLaunch& L, cudaStream_t s);

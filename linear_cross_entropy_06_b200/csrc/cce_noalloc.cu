@@ -143,6 +143,7 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
     L.err = err;
     L.timeout_ns = 4000000000ull;
     L.num_sms = num_sms;
+    L.inject_stall = 0;
     if (cce::launch_target_logit(Eb, Cb, targets, N, D, V, p->ignore_index, z_target, err, s) != cudaSuccess ||
         cce::launch_fwd_lse(L, s) != cudaSuccess ||
         cce::launch_lse_loss(tile_max, tile_sum, z_target, targets, N, T, p->ignore_index, V, lse,

@@ -56,7 +56,7 @@ def test_sizes(lib):
     assert 0 < fw < 256 + 4 * (T * 300 + 600) + 4 * 256
     bw32 = lib.cce_backward_workspace_size(ctypes.byref(p), 1)
     bw16 = lib.cce_backward_workspace_size(ctypes.byref(p), 0)
-    assert bw16 - bw32 >= 4 * (300 + 1000) * 136  # the fp32 accumulators
+    assert bw16 - bw32 >= 4 * 300 * 136  # the fp32 dE accumulator (dC is summed on chip)
     # nothing of size N*V: the workspaces of a Llama-3 head are far below N*V*2 bytes
     big = _p(N=32768, D=4096, V=128256, red=0)
     assert lib.cce_forward_workspace_size(ctypes.byref(big)) < 32768 * 128256 * 2 // 8
