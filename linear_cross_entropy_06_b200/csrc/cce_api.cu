@@ -43,7 +43,6 @@ cce_status cuda_fail(cudaError_t e, const char* what) {
 // Layout of the error word area at the start of every workspace.
 struct WsHeader {
   int err;
-  int num_tiles;
 };
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -89,38 +88,6 @@ FwdWs carve_fwd(const cce_problem* p, void* base) {
   off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
   w.loss_rows = reinterpret_cast<float*>(b + off);
   off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
-  w.bytes = off;
-  return w;
-}
-
-struct BwdWs {
-  WsHeader* hdr;
-  float* scale;
-  int2* tiles;
-  uint8_t* keep;
-  float* dE_acc;
-  float* dC_acc;
-  size_t bytes;
-};
-
-BwdWs carve_bwd(const cce_problem* p, int32_t out_fp32, void* base) {
-  const int64_t nb = ceil_div(p->N, cce::kBwdBM), nt = ceil_div(p->V, cce::kBwdBN);
-  BwdWs w{};
-  size_t off = kHeaderBytes;
-  char* b = static_cast<char*>(base);
-  w.hdr = reinterpret_cast<WsHeader*>(b);
-  w.scale = reinterpret_cast<float*>(b + off);
-  off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
-  w.tiles = reinterpret_cast<int2*>(b + off);
-  off = align_up(off + sizeof(int2) * static_cast<size_t>(nb * nt));
-  w.keep = reinterpret_cast<uint8_t*>(b + off);
-  off = align_up(off + static_cast<size_t>(nb * nt));
-  if (!out_fp32) {
-    w.dE_acc = reinterpret_cast<float*>(b + off);
-    off = align_up(off + sizeof(float) * static_cast<size_t>(p->N * p->D));
-    w.dC_acc = reinterpret_cast<float*>(b + off);
-    off = align_up(off + sizeof(float) * static_cast<size_t>(p->V * p->D));
-  }
   w.bytes = off;
   return w;
 }
@@ -172,13 +139,6 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   return w;
 }
 
-// The fused per-tile backward (reduce-add of every tile's dE and dC partials) is kept only as the
-// measured comparison for the split design; CCE_BWD=fused selects it.
-bool use_fused_backward() {
-  const char* s = std::getenv("CCE_BWD");
-  return s != nullptr && s[0] == 'f';
-}
-
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 // ---------------------------------------------------------------------------------------------
@@ -228,17 +188,6 @@ cce_status make_map(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem, co
   return CCE_OK;
 }
 
-// L2 eviction hints of the backward kernel. By default E and the dE accumulator are kept (they are
-// re-read or re-added by every vocabulary tile) when together they leave room in the 126 MB L2 for
-// the C and dC tiles in flight. CCE_L2_HINTS=<bits> overrides (0 = no hints).
-uint32_t backward_l2_hints(int64_t N, int64_t D) {
-  if (const char* s = std::getenv("CCE_L2_HINTS")) return static_cast<uint32_t>(std::strtoul(s, nullptr, 0)) & 15u;
-  const double e_bytes = 2.0 * N * D, de_bytes = 4.0 * N * D;
-  uint32_t h = 0;
-  if (e_bytes + de_bytes <= 100.0 * (1 << 20)) h |= cce::kL2KeepE | cce::kL2KeepdE;
-  return h;
-}
-
 uint64_t wait_timeout_ns() {
   const char* s = std::getenv("CCE_WAIT_TIMEOUT_MS");
   double ms = s ? std::atof(s) : 4000.0;
@@ -279,8 +228,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
     return cudaMemsetAsync(filtered_tiles, 0, sizeof(int64_t), s) == cudaSuccess ? CCE_OK
                                                                                   : fail(CCE_ERR_CUDA, "memset");
   }
-  CCE_TRY(cce::launch_row_scale(targets, count, grad_out, N, p->ignore_index, p->reduction, w.scale,
-                                &w.hdr->num_tiles, s));
+  CCE_TRY(cce::launch_row_scale(targets, count, grad_out, N, p->ignore_index, p->reduction, w.scale, s));
   CCE_TRY(cce::launch_bwd_plan(w.plan, tile_max, lse, targets, N, V, T, p->ignore_index, filter_eps, filtered_tiles,
                                s));
   CCE_TRY(cce::launch_fill_zero(dE_acc, N * D * 4, s));
@@ -389,7 +337,6 @@ size_t cce_forward_workspace_size(const cce_problem* p) {
 
 size_t cce_backward_workspace_size(const cce_problem* p, int32_t out_fp32) {
   if (!problem_ok(p, false)) return 0;
-  if (use_fused_backward()) return carve_bwd(p, out_fp32 ? 1 : 0, nullptr).bytes;
   return carve_split(p, out_fp32 ? 1 : 0, nullptr).bytes;
 }
 
@@ -460,61 +407,8 @@ cce_status cce_backward(const cce_problem* p, const void* E, const void* C, cons
     return fail(CCE_ERR_INVALID_ARG, "E, C, dE, dC and workspace must be 16-byte aligned");
   if (std::isnan(filter_eps)) return fail(CCE_ERR_INVALID_ARG, "filter_eps is NaN");
   out_fp32 = out_fp32 ? 1 : 0;
-  if (!use_fused_backward())
-    return backward_split(p, E, C, targets, lse, tile_max, count, grad_out, filter_eps, dE, dC, out_fp32,
-                          filtered_tiles, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
-  const BwdWs w = carve_bwd(p, out_fp32, workspace);
-  if (workspace_bytes < w.bytes)
-    return fail(CCE_ERR_WORKSPACE, "backward workspace is %zu bytes, needs %zu", workspace_bytes, w.bytes);
-  int num_sms = 0;
-  CCE_CHECK(check_device(&num_sms));
-  CCE_CHECK(get_encoder());
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t N = p->N, D = p->D, V = p->V, T = ceil_div(V, cce::kSubTile);
-  const auto* Eb = static_cast<const __nv_bfloat16*>(E);
-  const auto* Cb = static_cast<const __nv_bfloat16*>(C);
-  float* dE_acc = out_fp32 ? static_cast<float*>(dE) : w.dE_acc;
-  float* dC_acc = out_fp32 ? static_cast<float*>(dC) : w.dC_acc;
-
-  CCE_TRY(cudaMemsetAsync(w.hdr, 0, sizeof(WsHeader), s));
-  CCE_TRY(cce::launch_row_scale(targets, count, grad_out, N, p->ignore_index, p->reduction, w.scale,
-                                &w.hdr->num_tiles, s));
-  CCE_TRY(cce::launch_tile_mask(tile_max, lse, targets, N, V, T, p->ignore_index, filter_eps, w.tiles, w.keep,
-                                &w.hdr->num_tiles, filtered_tiles, s));
-  CCE_TRY(cce::launch_grad_init(Eb, Cb, targets, w.scale, w.keep, N, D, V, p->ignore_index, dE_acc, dC_acc,
-                                &w.hdr->err, s));
-  if (has_rows) {
-    cce::BwdLaunch L{};
-    CCE_CHECK(make_map(&L.tmE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kBwdBM));
-    CCE_CHECK(make_map(&L.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, cce::kBwdBN));
-    CCE_CHECK(make_map(&L.tmdE, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dE_acc, N, D, 32, 32));
-    CCE_CHECK(make_map(&L.tmdC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dC_acc, V, D, 32, 32));
-    L.N = static_cast<int>(N);
-    L.D = static_cast<int>(D);
-    L.V = static_cast<int>(V);
-    L.lse = lse;
-    L.scale = w.scale;
-    L.targets = targets;
-    L.ignore_index = p->ignore_index;
-    L.tiles = w.tiles;
-    L.num_tiles = &w.hdr->num_tiles;
-    L.l2_hints = backward_l2_hints(N, D);
-    L.dE_acc = dE_acc;
-    L.dC_acc = dC_acc;
-    const char* flush = std::getenv("CCE_FLUSH");
-    L.direct_red = (flush != nullptr && flush[0] == 'r') ? 1 : 0;
-    L.err = &w.hdr->err;
-    L.timeout_ns = wait_timeout_ns();
-    L.num_sms = num_sms;
-    if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
-    CCE_TRY(cce::launch_bwd_grad(L, s));
-    if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
-  }
-  if (!out_fp32) {
-    CCE_TRY(cce::launch_to_bf16(dE_acc, static_cast<__nv_bfloat16*>(dE), N * D, s));
-    CCE_TRY(cce::launch_to_bf16(dC_acc, static_cast<__nv_bfloat16*>(dC), V * D, s));
-  }
-  return CCE_OK;
+  return backward_split(p, E, C, targets, lse, tile_max, count, grad_out, filter_eps, dE, dC, out_fp32,
+                        filtered_tiles, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 cce_status cce_check_device_error(void* workspace, cce_stream_t stream) {

@@ -1,4 +1,4 @@
-// The bandwidth-bound and bookkeeping kernels around the two tensor-core kernels:
+// The bandwidth-bound and bookkeeping kernels around the tensor-core kernels:
 //  target_logit   z_t[r] = E[r] . C[t_r] (fp32 accumulation of bf16 products), target validation.
 //                 Cut Your Losses abstract: only the correct token's logit is computed.
 //  lse_loss       LSE_r = M + ln sum_j s_j exp(m_j - M) over the saved sub-tile (max, sum-exp)
@@ -8,14 +8,7 @@
 //                 mlx-cross-entropy README, "API" (reduction); explainer item 4 (mean over
 //                 non-ignored tokens).
 //  row_scale      per-row factor of the gradient: g/max(count,1), g or g[r]; 0 for ignored rows.
-//  tile_mask      keep/skip decision per backward tile from the saved maxima and LSE, compacted
-//                 into a list. mlx-cross-entropy README, "How it works" item 2.
-//  grad_init      dC_acc = 0 and dE_acc[r] = -scale_r C[t_r] when the tile holding (r, t_r) is
-//                 skipped, else +0; onehot_dC adds -scale_r E[r] into dC_acc[t_r] for the same
-//                 rows. The onehot part of p - y of a kept tile is folded into the gradient tile
-//                 by the backward kernel (before rounding to bf16), so it is never skipped and
-//                 never cancels against a rounded p.
-//  to_bf16        fp32 accumulators -> bf16 outputs (round to nearest even).
+//  to_bf16        fp32 dE accumulator -> bf16 output (round to nearest even).
 #include <cuda_bf16.h>
 
 #include "cce_device.cuh"
@@ -152,9 +145,8 @@ __global__ void loss_reduce_kernel(const float* __restrict__ loss_rows, const in
 
 __global__ void row_scale_kernel(const int64_t* __restrict__ targets, const int64_t* __restrict__ count,
                                  const float* __restrict__ grad_out, int64_t N, int64_t ignore_index, int reduction,
-                                 float* __restrict__ scale, int* num_tiles) {
+                                 float* __restrict__ scale) {
   const int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (r == 0) *num_tiles = 0;
   if (r >= N) return;
   float s;
   if (reduction == 1) {
@@ -166,121 +158,6 @@ __global__ void row_scale_kernel(const int64_t* __restrict__ targets, const int6
     s = grad_out[r];
   }
   scale[r] = (targets[r] != ignore_index) ? s : 0.f;
-}
-
-// One block (128 threads, one per tile row) per vocabulary tile. Tile (b, t) is kept iff some
-// non-ignored row r of block b has tile_max[t, r] - LSE_r >= ln(eps), or eps <= 0. The block
-// counts its kept tiles, reserves a contiguous range with one atomic, then writes (b, t) in b order,
-// so each vocabulary tile's row blocks are adjacent in the list.
-__global__ void tile_mask_kernel(const float* __restrict__ tile_max, const float* __restrict__ lse,
-                                 const int64_t* __restrict__ targets, int64_t N, int64_t V, int64_t T,
-                                 int64_t ignore_index, float ln_eps, int filter_on, int2* __restrict__ tiles,
-                                 uint8_t* __restrict__ keep, int* num_tiles) {
-  __shared__ float wmax[4];
-  __shared__ int base;
-  const int t = blockIdx.x;
-  const int nb = static_cast<int>((N + kBwdBM - 1) / kBwdBM);
-  int kept_count = 0;
-  for (int pass = 0; pass < 2; ++pass) {
-    int k = 0;
-    for (int b = 0; b < nb; ++b) {
-      bool keep_tile = true;
-      if (filter_on) {
-        const int64_t r = static_cast<int64_t>(b) * kBwdBM + threadIdx.x;
-        float m = -INFINITY;
-        if (r < N && valid_target(targets[r], V, ignore_index)) {
-          const int64_t j0 = static_cast<int64_t>(t) * (kBwdBN / kSubTile);
-          const int64_t j1 = j0 + kBwdBN / kSubTile < T ? j0 + kBwdBN / kSubTile : T;
-          for (int64_t j = j0; j < j1; ++j) m = fmaxf(m, tile_max[j * N + r]);
-          m -= lse[r];
-        }
-        m = warp_max(m);
-        if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
-        __syncthreads();
-        const float bm = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
-        __syncthreads();
-        keep_tile = bm >= ln_eps;
-      }
-      if (pass == 0 && threadIdx.x == 0) keep[static_cast<int64_t>(b) * gridDim.x + t] = keep_tile ? 1 : 0;
-      if (keep_tile) {
-        if (pass == 1 && threadIdx.x == 0) tiles[base + k] = make_int2(b, t);
-        ++k;
-      }
-    }
-    if (pass == 0) {
-      kept_count = k;
-      if (threadIdx.x == 0) base = atomicAdd(num_tiles, kept_count);
-      __syncthreads();
-    }
-  }
-}
-
-__global__ void mask_finish_kernel(const int* __restrict__ num_tiles, int64_t total, int64_t* __restrict__ filtered) {
-  *filtered = total - static_cast<int64_t>(*num_tiles);
-}
-
-// True when row r has a valid target whose tile (r's row block, t_r's vocabulary tile) was skipped:
-// then the onehot term of that row is added here instead of inside the backward kernel.
-__device__ __forceinline__ bool onehot_outside(int64_t r, int64_t t, int64_t V, int64_t ignore_index,
-                                               const uint8_t* keep, int64_t nt) {
-  return valid_target(t, V, ignore_index) && keep[(r / kBwdBM) * nt + t / kBwdBN] == 0;
-}
-
-// dE_acc[r, :] = -scale_r * C[t_r, :] for rows whose target tile is skipped, +0 otherwise. One warp
-// per row, 8 elements per lane per step.
-__global__ void grad_init_dE_kernel(const __nv_bfloat16* __restrict__ C, const int64_t* __restrict__ targets,
-                                    const float* __restrict__ scale, const uint8_t* __restrict__ keep, int64_t N,
-                                    int64_t D, int64_t V, int64_t ignore_index, float* __restrict__ dE_acc,
-                                    int* err) {
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= N) return;
-  const int64_t t = targets[row];
-  float* out = dE_acc + row * D;
-  if (lane == 0 && t != ignore_index && !valid_target(t, V, ignore_index)) record_error(err, kErrTargetRange);
-  const int64_t nt = (V + kBwdBN - 1) / kBwdBN;
-  if (!onehot_outside(row, t, V, ignore_index, keep, nt)) {
-    for (int64_t d = static_cast<int64_t>(lane) * 4; d < D; d += 128)
-      *reinterpret_cast<float4*>(out + d) = make_float4(0.f, 0.f, 0.f, 0.f);
-    return;
-  }
-  const float s = -scale[row];
-  const __nv_bfloat16* c = C + t * D;
-  for (int64_t d = static_cast<int64_t>(lane) * 8; d < D; d += 256) {
-    const uint4 raw = ld_global_nc_v4(c + d);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-    const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-    const float2 cc = __bfloat1622float2(h[2]), dd = __bfloat1622float2(h[3]);
-    *reinterpret_cast<float4*>(out + d) = make_float4(s * a.x, s * a.y, s * b.x, s * b.y);
-    *reinterpret_cast<float4*>(out + d + 4) = make_float4(s * cc.x, s * cc.y, s * dd.x, s * dd.y);
-  }
-}
-
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
-// dC_acc[t_r, :] += -scale_r * E[r, :] for non-ignored rows (targets repeat, hence atomics).
-__global__ void onehot_dC_kernel(const __nv_bfloat16* __restrict__ E, const int64_t* __restrict__ targets,
-                                 const float* __restrict__ scale, const uint8_t* __restrict__ keep, int64_t N,
-                                 int64_t D, int64_t V, int64_t ignore_index, float* __restrict__ dC_acc) {
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= N) return;
-  const int64_t t = targets[row];
-  if (!onehot_outside(row, t, V, ignore_index, keep, (V + kBwdBN - 1) / kBwdBN)) return;
-  const float s = -scale[row];
-  const __nv_bfloat16* e = E + row * D;
-  float* out = dC_acc + t * D;
-  for (int64_t d = static_cast<int64_t>(lane) * 8; d < D; d += 256) {
-    const uint4 raw = ld_global_nc_v4(e + d);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-    const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-    const float2 cc = __bfloat1622float2(h[2]), dd = __bfloat1622float2(h[3]);
-    red_add_v4(out + d, s * a.x, s * a.y, s * b.x, s * b.y);
-    red_add_v4(out + d + 4, s * cc.x, s * cc.y, s * dd.x, s * dd.y);
-  }
 }
 
 __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t n8) {
@@ -339,44 +216,10 @@ cudaError_t launch_loss_reduce(const float* loss_rows, const int64_t* targets, i
 }
 
 cudaError_t launch_row_scale(const int64_t* targets, const int64_t* count, const float* grad_out, int64_t N,
-                             int64_t ignore_index, int reduction, float* scale, int* num_tiles, cudaStream_t s) {
-  const int grid = static_cast<int>(N > 0 ? (N + 255) / 256 : 1);
-  row_scale_kernel<<<grid, 256, 0, s>>>(targets, count, grad_out, N, ignore_index, reduction, scale, num_tiles);
-  note_launches(1);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_tile_mask(const float* tile_max, const float* lse, const int64_t* targets, int64_t N, int64_t V,
-                             int64_t T, int64_t ignore_index, float filter_eps, int2* tiles, uint8_t* keep,
-                             int* num_tiles, int64_t* filtered_tiles, cudaStream_t s) {
-  const int64_t nb = (N + kBwdBM - 1) / kBwdBM;
-  const int64_t nt = (V + kBwdBN - 1) / kBwdBN;
-  const int filter_on = filter_eps > 0.f ? 1 : 0;
-  const float ln_eps = filter_on ? logf(filter_eps) : -INFINITY;
-  if (nb > 0) {
-    tile_mask_kernel<<<static_cast<int>(nt), kBwdBM, 0, s>>>(tile_max, lse, targets, N, V, T, ignore_index, ln_eps,
-                                                             filter_on, tiles, keep, num_tiles);
-    note_launches(1);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  mask_finish_kernel<<<1, 1, 0, s>>>(num_tiles, nb * nt, filtered_tiles);
-  note_launches(1);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_grad_init(const __nv_bfloat16* E, const __nv_bfloat16* C, const int64_t* targets,
-                             const float* scale, const uint8_t* keep, int64_t N, int64_t D, int64_t V,
-                             int64_t ignore_index, float* dE_acc, float* dC_acc, int* err, cudaStream_t s) {
-  cudaError_t e = launch_fill_zero(dC_acc, V * D * 4, s);
-  if (e != cudaSuccess) return e;
+                             int64_t ignore_index, int reduction, float* scale, cudaStream_t s) {
   if (N == 0) return cudaSuccess;
-  const int grid = static_cast<int>((N + 7) / 8);
-  grad_init_dE_kernel<<<grid, 256, 0, s>>>(C, targets, scale, keep, N, D, V, ignore_index, dE_acc, err);
-  note_launches(1);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  onehot_dC_kernel<<<grid, 256, 0, s>>>(E, targets, scale, keep, N, D, V, ignore_index, dC_acc);
+  const int grid = static_cast<int>((N + 255) / 256);
+  row_scale_kernel<<<grid, 256, 0, s>>>(targets, count, grad_out, N, ignore_index, reduction, scale);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -13,15 +13,9 @@ constexpr int kFwdBM = 128;
 constexpr int kFwdBN = 256;
 constexpr int kSubTile = 128;  // vocabulary width of one saved tile max
 
-// Backward tile: 128 rows x 128 vocabulary columns; gradients in D-chunks of 64 columns.
+// Backward tile: 128 rows x 128 vocabulary columns (the unit of the skip rule and of a gradient tile).
 constexpr int kBwdBM = 128;
 constexpr int kBwdBN = 128;
-
-// L2 eviction hints of the backward kernel (bits of BwdLaunch::l2_hints).
-constexpr uint32_t kL2KeepE = 1;        // E tile loads: evict_last (E is re-read by every vocab tile)
-constexpr uint32_t kL2KeepdE = 2;       // dE reduce-adds: evict_last (every vocab tile adds into dE)
-constexpr uint32_t kL2StreamC = 4;      // C tile loads: evict_first
-constexpr uint32_t kL2StreamdC = 8;     // dC reduce-adds: evict_first
 
 struct FwdLaunch {
   CUtensorMap tmE;  // bf16 [N, D], box 64 x 128, 128B swizzle
@@ -33,27 +27,6 @@ struct FwdLaunch {
   uint64_t timeout_ns;
   int num_sms;
   int inject_stall;  // test hook: the producer issues nothing, so a bounded wait runs out
-};
-
-struct BwdLaunch {
-  CUtensorMap tmE;      // bf16 [N, D], box 64 x 128, 128B swizzle
-  CUtensorMap tmC;      // bf16 [V, D], box 64 x 128, 128B swizzle
-  CUtensorMap tmdE;     // fp32 [N, D] accumulator, box 32 x 32, 128B swizzle (reduce-add)
-  CUtensorMap tmdC;     // fp32 [V, D] accumulator, box 32 x 32, 128B swizzle (reduce-add)
-  int N, D, V;
-  const float* lse;     // [N]
-  const float* scale;   // [N]: per-row gradient factor, 0 for ignored rows
-  const int64_t* targets;  // [N]: the onehot term of a kept tile is applied inside the kernel
-  int64_t ignore_index;
-  const int2* tiles;    // kept tiles (row block, vocab tile)
-  const int* num_tiles; // device count of kept tiles
-  uint32_t l2_hints;    // kL2* bits: which streams get an L2 eviction-priority hint
-  float* dE_acc;        // fp32 accumulators (the direct-red flush adds into them by address)
-  float* dC_acc;
-  int direct_red;       // 1: flush with red.global.add from registers; 0: smem staging + TMA reduce
-  int* err;
-  uint64_t timeout_ns;
-  int num_sms;
 };
 
 // Counts every kernel launch of the calling thread (instrumentation for benchmarks).
@@ -119,7 +92,6 @@ cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk_t0, int chunk_t1, cuda
 cudaError_t launch_bwd_gemm(const BwdGemm& L, bool dE_mode, int chunk_t0, int chunk_t1, cudaStream_t s);
 
 cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
-cudaError_t launch_bwd_grad(const BwdLaunch& L, cudaStream_t s);
 
 // Small kernels (cce_aux.cu).
 cudaError_t launch_target_logit(const __nv_bfloat16* E, const __nv_bfloat16* C, const int64_t* targets, int64_t N,
@@ -131,13 +103,7 @@ cudaError_t launch_lse_loss(const float* tile_max, const float* tile_sum, const 
 cudaError_t launch_loss_reduce(const float* loss_rows, const int64_t* targets, int64_t N, int64_t ignore_index,
                                int reduction, float* loss, int64_t* count, cudaStream_t s);
 cudaError_t launch_row_scale(const int64_t* targets, const int64_t* count, const float* grad_out, int64_t N,
-                             int64_t ignore_index, int reduction, float* scale, int* num_tiles, cudaStream_t s);
-cudaError_t launch_tile_mask(const float* tile_max, const float* lse, const int64_t* targets, int64_t N, int64_t V,
-                             int64_t T, int64_t ignore_index, float filter_eps, int2* tiles, uint8_t* keep,
-                             int* num_tiles, int64_t* filtered_tiles, cudaStream_t s);
-cudaError_t launch_grad_init(const __nv_bfloat16* E, const __nv_bfloat16* C, const int64_t* targets,
-                             const float* scale, const uint8_t* keep, int64_t N, int64_t D, int64_t V,
-                             int64_t ignore_index, float* dE_acc, float* dC_acc, int* err, cudaStream_t s);
+                             int64_t ignore_index, int reduction, float* scale, cudaStream_t s);
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, int64_t n, cudaStream_t s);
 cudaError_t launch_fill_zero(void* dst, int64_t bytes, cudaStream_t s);
 
