@@ -133,6 +133,9 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   // tile) fit in the scratch budget; at least one vocabulary tile per chunk.
   const int64_t per_vtile = std::max<int64_t>(nb, 1) * cce::kGradTileBytes;
   w.chunk_tiles = std::max<int64_t>(1, std::min<int64_t>(nt, cce::kGradScratchBudget / per_vtile));
+  w.plan.chunk_tiles = static_cast<int>(w.chunk_tiles);
+  w.plan.nchunks = static_cast<int>(ceil_div(nt, w.chunk_tiles));
+  w.plan.pair_off = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks * (nb + 1))));
   w.gscratch = reinterpret_cast<uint8_t*>(take(static_cast<size_t>(per_vtile * w.chunk_tiles)));
   if (!out_fp32) w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
   w.bytes = off;
@@ -243,17 +246,21 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   G.scale = w.scale;
   G.targets = targets;
   G.ignore_index = p->ignore_index;
-  G.entries_t = w.plan.entries_t;
+  G.nb = w.plan.nb;
+  G.nt = w.plan.nt;
+  G.flags = w.plan.flags;
+  G.entries_b = w.plan.entries_b;
+  G.offsets_b = w.plan.offsets_b;
+  G.pair_off = w.plan.pair_off;
   G.offsets_t = w.plan.offsets_t;
   G.gscratch = w.gscratch;
-  G.max_entries_per_chunk = static_cast<int>(std::min<int64_t>(int64_t(w.plan.nb) * w.chunk_tiles, 1 << 30));
   G.num_sms = num_sms;
   G.err = &w.hdr->err;
   G.timeout_ns = wait_timeout_ns();
 
   cce::BwdGemm M{};
-  M.tmE = G.tmE;
-  M.tmC = G.tmC;
+  CCE_CHECK(make_map(&M.tmE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, 64));
+  CCE_CHECK(make_map(&M.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, 64));
   CCE_CHECK(make_map(&M.tmdE, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dE_acc, N, D, 32, 32));
   if (out_fp32) CCE_CHECK(make_map(&M.tmdC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dC, V, D, 32, 32));
   else CCE_CHECK(make_map(&M.tmdC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dC, V, D, 64, 32));
@@ -273,9 +280,10 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
 
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
   const int nt = w.plan.nt;
-  for (int64_t t0 = 0; t0 < nt; t0 += w.chunk_tiles) {
-    const int c0 = static_cast<int>(t0), c1 = static_cast<int>(std::min<int64_t>(nt, t0 + w.chunk_tiles));
-    CCE_TRY(cce::launch_bwd_g(G, c0, c1, s));
+  for (int c = 0; c < w.plan.nchunks; ++c) {
+    const int c0 = static_cast<int>(c * w.chunk_tiles);
+    const int c1 = static_cast<int>(std::min<int64_t>(nt, c0 + w.chunk_tiles));
+    CCE_TRY(cce::launch_bwd_g(G, c, c0, c1, s));
     CCE_TRY(cce::launch_bwd_gemm(M, false, c0, c1, s));
     CCE_TRY(cce::launch_bwd_gemm(M, true, c0, c1, s));
   }

@@ -10,11 +10,15 @@
 // 2^-12); Loss functions explainer, "How it works" item 2 (gradient p - y); Cut Your Losses
 // abstract (logits are recomputed blockwise, never stored).
 //
-// Design (B200): one persistent CTA per SM, 6 warps.
-//   warp 0      TMA producer: E_b and C_t K-blocks (bf16, 128B swizzle) into a 4-stage ring.
-//   warp 1      TMEM (256 columns = two S buffers of 128); one lane issues tcgen05.mma M=128 N=128.
-//   warps 2..5  G formation (TMEM -> exp -> bf16 -> swizzled smem), one bulk store per tile; the
-//               two smem G buffers let the store of one tile overlap the formation of the next.
+// Two listed tiles of the same row block are recomputed together, as one 128 x 256 logit tile:
+// E_b is loaded once for both vocabulary tiles and each MMA is M=128 x N=256, the forward's shape.
+//
+// Design (B200): one persistent CTA per SM, 6 warps, over pairs of consecutive listed tiles of a row
+// block inside the chunk (the row-block lists are ordered by vocabulary tile).
+//   warp 0      TMA producer: E_b, C_t1 and C_t2 K-blocks (bf16, 128B swizzle), 48 KB stages, 4 deep.
+//   warp 1      TMEM (512 columns = two 256-column S buffers); one lane issues tcgen05.mma M=128 N=256.
+//   warps 2..5  G formation (TMEM -> exp -> bf16 -> swizzled smem) and one bulk store per tile, while
+//               the MMA recomputes the next pair into the other S buffer.
 #include "cce_device.cuh"
 #include "cce_internal.h"
 
@@ -26,13 +30,13 @@ constexpr int BN = kBwdBN;
 constexpr int BK = 64;
 constexpr int STAGES = 4;
 constexpr int HALF = 16384;            // 128 x 64 bf16
-constexpr int STAGE_BYTES = 2 * HALF;  // E_b K-block | C_t K-block
+constexpr int STAGE_BYTES = 3 * HALF;  // E_b K-block | C_t1 K-block | C_t2 K-block
 constexpr int G_BYTES = kGradTileBytes;
 constexpr int NUM_THREADS = 192;
-constexpr int TMEM_COLS = 256;
+constexpr int TMEM_COLS = 512;
 constexpr int NUM_BARRIERS = 2 * STAGES + 4 + 3;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 2 * G_BYTES + NUM_BARRIERS * 8 + 16;
-constexpr uint32_t IDESC_S = idesc_bf16(BM, BN, false, false);
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + G_BYTES + NUM_BARRIERS * 8 + 16;
+constexpr uint32_t IDESC_S = idesc_bf16(BM, 2 * BN, false, false);
 
 static_assert(G_BYTES == BM * BN * 2, "gradient tile is 128 x 128 bf16");
 
@@ -45,16 +49,60 @@ __device__ __forceinline__ void bulk_store_32k(void* gdst, uint32_t src) {
                : "memory");
 }
 
+__device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int t) {
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (e[mid].x < t) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// Pair w of this chunk: its row block, and its one or two tiles (vocabulary tile, slot, kept?).
+struct Pair {
+  int b;
+  int t[2], slot[2];
+  bool kept[2], present[2];
+  __device__ bool any_kept() const { return kept[0] || kept[1]; }
+};
+
+__device__ __forceinline__ Pair pair_at(int w, const int* pair_off, int nb, const int2* entries_b,
+                                        const int* offsets_b, const uint8_t* flags, int nt, int chunk_t0,
+                                        int chunk_t1, int slot_base) {
+  int lo = 0, hi = nb;  // largest b with pair_off[b] <= w
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (pair_off[mid] <= w) lo = mid;
+    else hi = mid;
+  }
+  Pair p;
+  p.b = lo;
+  const int first = lower_bound_t(entries_b, offsets_b[lo], offsets_b[lo + 1], chunk_t0);
+  const int last = lower_bound_t(entries_b, first, offsets_b[lo + 1], chunk_t1);
+  const int i0 = first + 2 * (w - pair_off[lo]);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    p.present[k] = i0 + k < last;
+    const int2 en = entries_b[p.present[k] ? i0 + k : i0];
+    p.t[k] = en.x;
+    p.slot[k] = en.y - slot_base;
+    p.kept[k] = p.present[k] && flags[static_cast<int64_t>(lo) * nt + en.x] == 1;
+  }
+  return p;
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_g_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC, int N, int D, int V,
                  const float* __restrict__ lse, const float* __restrict__ scale, const int64_t* __restrict__ targets,
-                 int64_t ignore_index, const int2* __restrict__ entries_t, const int* __restrict__ offsets_t,
-                 int chunk_t0, int chunk_t1, uint8_t* __restrict__ gscratch, int* err, uint64_t timeout_ns) {
+                 int64_t ignore_index, const int* __restrict__ offsets_t, const uint8_t* __restrict__ flags, int nb,
+                 int nt, const int2* __restrict__ entries_b, const int* __restrict__ offsets_b,
+                 const int* __restrict__ pair_off, int chunk_t0, int chunk_t1, uint8_t* __restrict__ gscratch,
+                 int* err, uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
   uint8_t* gbuf = base + STAGES * STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gbuf + 2 * G_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gbuf + G_BYTES);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NUM_BARRIERS);
   int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
 
@@ -68,8 +116,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t gfree_bar = bar0 + 8u * (2 * STAGES + 5);   // leader: the smem G buffer may be rewritten
   const uint32_t gready_bar = bar0 + 8u * (2 * STAGES + 6);  // all 128 rows of G are in smem
 
-  const int e0 = offsets_t[chunk_t0], e1 = offsets_t[chunk_t1];
-  if (e1 - e0 <= static_cast<int>(blockIdx.x)) return;  // uniform across the CTA, before any sync
+  const int num_pairs = pair_off[nb];
+  if (num_pairs <= static_cast<int>(blockIdx.x)) return;  // uniform across the CTA, before any sync
+  const int slot_base = offsets_t[chunk_t0];
+  auto get_pair = [&](int w) {
+    return pair_at(w, pair_off, nb, entries_b, offsets_b, flags, nt, chunk_t0, chunk_t1, slot_base);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -103,10 +155,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued[STAGES] = {0, 0, 0, 0};
       bool ok = true;
-      for (int i = e0 + blockIdx.x; i < e1 && ok; i += gridDim.x) {
-        const int2 en = entries_t[i];
-        if ((en.x & 3) != 1) continue;  // onehot-only tiles need no recompute
-        const int rb = (en.x >> 2) * BM, vb = en.y * BN;
+      for (int w = blockIdx.x; w < num_pairs && ok; w += gridDim.x) {
+        const Pair p = get_pair(w);
+        if (!p.any_kept()) continue;  // onehot-only tiles need no recompute
+        const int rb = p.b * BM;
+        const int vb0 = p.t[0] * BN, vb1 = (p.present[1] ? p.t[1] : p.t[0]) * BN;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, wc)) {
             ok = false;
@@ -115,7 +168,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t dst = smem_u32(stages + stage * STAGE_BYTES);
           mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
           tma_load_2d(dst, &tmE, full_bar(stage), kb * BK, rb);
-          tma_load_2d(dst + HALF, &tmC, full_bar(stage), kb * BK, vb);
+          tma_load_2d(dst + HALF, &tmC, full_bar(stage), kb * BK, vb0);
+          tma_load_2d(dst + 2 * HALF, &tmC, full_bar(stage), kb * BK, vb1);
           ++issued[stage];
           if (++stage == STAGES) {
             stage = 0;
@@ -134,16 +188,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t sidx = 0;
       bool ok = true, issued_any = false;
-      for (int i = e0 + blockIdx.x; i < e1 && ok; i += gridDim.x) {
-        const int2 en = entries_t[i];
-        if ((en.x & 3) != 1) continue;
+      for (int w = blockIdx.x; w < num_pairs && ok; w += gridDim.x) {
+        const Pair p = get_pair(w);
+        if (!p.any_kept()) continue;
         const int a = sidx & 1;
         if (!mbar_wait(sempty_bar(a), ((sidx >> 1) & 1u) ^ 1u, wc)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * 2 * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, wc)) {
             ok = false;
@@ -152,7 +206,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           const uint32_t a0 = smem_u32(stages + stage * STAGE_BYTES);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
+          for (int k = 0; k < BK / 16; ++k)  // B = C_t1 and C_t2 rows: 256 rows of 128 bytes, contiguous
             tc_mma_bf16(d_tmem, sdesc_sw128(a0 + 32u * k, 16, 1024), sdesc_sw128(a0 + HALF + 32u * k, 16, 1024),
                         IDESC_S, (kb | k) != 0 ? 1u : 0u);
           issued_any = true;
@@ -177,70 +231,78 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const bool leader = (warp == 2 && lane == 0);
+    const uint32_t g0 = smem_u32(gbuf);
     uint32_t sidx = 0, j = 0;
-    for (int i = e0 + blockIdx.x; i < e1; i += gridDim.x, ++j) {
-      const int2 en = entries_t[i];
-      const bool full = (en.x & 3) == 1;
-      const int rb = (en.x >> 2) * BM, vb = en.y * BN;
-      const int r = rb + row;
+    bool ok = true;
+    for (int w = blockIdx.x; w < num_pairs && ok; w += gridDim.x) {
+      const Pair p = get_pair(w);
+      const int r = p.b * BM + row;
       const float lse_l2 = (r < N) ? lse[r] * kLog2e : 0.f;
       const float sc = (r < N) ? scale[r] : 0.f;
-      int tcol = -1;  // target column inside this tile: G gets -scale_r there, in fp32, before rounding
-      if (r < N) {
-        const int64_t tg = targets[r];
-        const int64_t rel = tg - vb;
-        if (tg != ignore_index && tg >= 0 && tg < V && rel >= 0 && rel < BN) tcol = static_cast<int>(rel);
-      }
-      // The smem buffer of tile j was last stored two tiles ago: that store must have read it.
-      // (mbarriers with bounded waits, not a named barrier, so that an abort cannot hang here.)
-      if (leader) {
-        asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-        mbar_arrive(gfree_bar);
-      }
-      if (!mbar_wait(gfree_bar, j & 1u, wc)) break;
-      const uint32_t g0 = smem_u32(gbuf + (j & 1) * G_BYTES);
+      const int64_t tg = (r < N) ? targets[r] : ignore_index;
+      const bool tvalid = tg != ignore_index && tg >= 0 && tg < V;
       const int a = sidx & 1;
-      if (full) {
+      if (p.any_kept()) {
         if (!mbar_wait(sfull_bar(a), (sidx >> 1) & 1u, wc)) break;
         tc_fence_after();
       }
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        if (full) {
-          tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * BN + c * 32), v);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = sc * exp2f(fmaf(v[k], kLog2e, -lse_l2));
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = 0.f;
+      for (int k = 0; k < 2 && ok; ++k) {
+        if (!p.present[k]) break;
+        const int vb = p.t[k] * BN;
+        const int64_t rel = tg - vb;
+        const int tcol = (tvalid && rel >= 0 && rel < BN) ? static_cast<int>(rel) : -1;  // -scale_r goes here
+        // The G buffer is free once the previous tile's store has read it (bounded mbarrier waits,
+        // not a named barrier, so that an abort cannot hang here).
+        if (leader) {
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          mbar_arrive(gfree_bar);
         }
-        const int col0 = vb + c * 32;
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          if (c * 32 + k == tcol) v[k] -= sc;
-          if (col0 + k >= V) v[k] = 0.f;
+        if (!mbar_wait(gfree_bar, j & 1u, wc)) {
+          ok = false;
+          break;
         }
-        const uint32_t blk = g0 + static_cast<uint32_t>((c >> 1) * HALF);
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const int chunk = (c & 1) * 4 + h;
-          st_shared_v4(blk + swz(row, chunk), pack_bf16x2(v[8 * h + 0], v[8 * h + 1]),
-                       pack_bf16x2(v[8 * h + 2], v[8 * h + 3]), pack_bf16x2(v[8 * h + 4], v[8 * h + 5]),
-                       pack_bf16x2(v[8 * h + 6], v[8 * h + 7]));
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          if (p.kept[k]) {
+            tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * 2 * BN + k * BN + c * 32), v);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = sc * exp2f(fmaf(v[e], kLog2e, -lse_l2));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0.f;
+          }
+          const int col0 = vb + c * 32;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (c * 32 + e == tcol) v[e] -= sc;
+            if (col0 + e >= V) v[e] = 0.f;
+          }
+          const uint32_t blk = g0 + static_cast<uint32_t>((c >> 1) * HALF);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int chunk = (c & 1) * 4 + h;
+            st_shared_v4(blk + swz(row, chunk), pack_bf16x2(v[8 * h + 0], v[8 * h + 1]),
+                         pack_bf16x2(v[8 * h + 2], v[8 * h + 3]), pack_bf16x2(v[8 * h + 4], v[8 * h + 5]),
+                         pack_bf16x2(v[8 * h + 6], v[8 * h + 7]));
+          }
         }
+        fence_proxy_async_smem();
+        mbar_arrive(gready_bar);
+        if (leader) {
+          if (!mbar_wait(gready_bar, j & 1u, wc)) {
+            ok = false;
+            break;
+          }
+          bulk_store_32k(gscratch + static_cast<size_t>(p.slot[k]) * G_BYTES, g0);
+          bulk_commit_group();
+        }
+        ++j;  // one gfree / gready phase per tile
       }
-      if (full) {
+      if (p.any_kept()) {
         tc_fence_before();
         mbar_arrive(sempty_bar(a));
         ++sidx;
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(gready_bar);
-      if (leader) {
-        if (!mbar_wait(gready_bar, j & 1u, wc)) break;
-        bulk_store_32k(gscratch + static_cast<size_t>(i - e0) * G_BYTES, g0);
-        bulk_commit_group();
       }
     }
     // Every tile must be in global memory before the kernel ends (the next kernels read them).
@@ -258,14 +320,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 }  // namespace
 
-cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk_t0, int chunk_t1, cudaStream_t s) {
+cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk, int chunk_t0, int chunk_t1, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(bwd_g_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int grid = L.max_entries_per_chunk < L.num_sms ? L.max_entries_per_chunk : L.num_sms;
+  // At most one pair per two listed tiles of a row block, plus one per row block for an odd count.
+  const long long bound = static_cast<long long>(L.nb) * ((chunk_t1 - chunk_t0 + 1) / 2 + 1);
+  const int grid = static_cast<int>(bound < L.num_sms ? bound : L.num_sms);
   if (grid <= 0) return cudaSuccess;
-  bwd_g_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmC, L.N, L.D, L.V, L.lse, L.scale, L.targets,
-                                                     L.ignore_index, L.entries_t, L.offsets_t, chunk_t0, chunk_t1,
-                                                     L.gscratch, L.err, L.timeout_ns);
+  bwd_g_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(
+      L.tmE, L.tmC, L.N, L.D, L.V, L.lse, L.scale, L.targets, L.ignore_index, L.offsets_t, L.flags, L.nb, L.nt,
+      L.entries_b, L.offsets_b, L.pair_off + static_cast<int64_t>(chunk) * (L.nb + 1), chunk_t0, chunk_t1,
+      L.gscratch, L.err, L.timeout_ns);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -13,12 +13,12 @@
 // dC = G^T E with G = p - y). The gradient tiles come from the recompute kernel (cce_bwd_g.cu).
 //
 // Design (B200): one persistent CTA per SM, 6 warps.
-//   warp 0      producer: per listed tile, the 32 KB gradient tile (bulk copy from the chunk
-//               scratch) and the 128 x 256 operand slice (TMA, 128B swizzle, two 32 KB halves)
-//               into a ring of six 32 KB units.
-//   warp 1      TMEM: two 256-column fp32 accumulators; one lane issues tcgen05.mma M=128 N=128
-//               per half slice (dC: A = G read MN-major as G^T; dE: A = G K-major; B = the slice,
-//               MN-major).
+//   warp 0      producer: per listed tile, two 48 KB stages, one per 64-wide half of the MMA's K:
+//               16 KB of the gradient tile (bulk copy from the chunk scratch) and the 64 x 256
+//               operand slice (four TMA boxes of 64 x 64, 128B swizzle) into a 4-stage ring.
+//   warp 1      TMEM: two 256-column fp32 accumulators; one lane issues tcgen05.mma M=128 N=256
+//               K=16, four per stage (dC: A = G read MN-major as G^T; dE: A = G K-major; B = the
+//               slice, MN-major). The shape and the 48 KB per 512 cycles match the forward kernel.
 //   warps 2..5  write-out: TMEM -> registers -> swizzled staging -> TMA store (dC, bf16 or fp32)
 //               or TMA reduce-add (dE, fp32), while the MMA fills the other accumulator.
 #include "cce_device.cuh"
@@ -30,17 +30,19 @@ namespace {
 constexpr int BM = kBwdBM;
 constexpr int BN = kBwdBN;
 constexpr int SLICE = kGemmSlice;  // 256 columns of D per work item
-constexpr int UNITS = 6;
-constexpr int UNIT_BYTES = 32768;
-constexpr int BOX_BYTES = 16384;  // 128 rows x 64 bf16
+constexpr int STAGES = 4;
+constexpr int G_PART = 16384;       // one K-half of the gradient tile
+constexpr int X_BOX = 8192;         // 64 rows x 64 bf16
+constexpr int STAGE_BYTES = G_PART + 4 * X_BOX;
+constexpr int TILE_BYTES = kGradTileBytes;
 constexpr int STG_WARP = 8192;    // per epilogue warp: 32 rows x 64 columns of fp32 (or bf16 + unused)
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
-constexpr int NUM_BARRIERS = 2 * UNITS + 4 + 1;
-constexpr int SMEM_BYTES = 1024 + UNITS * UNIT_BYTES + 4 * STG_WARP + NUM_BARRIERS * 8 + 16;
+constexpr int NUM_BARRIERS = 2 * STAGES + 4 + 1;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 4 * STG_WARP + NUM_BARRIERS * 8 + 16;
 
-constexpr uint32_t IDESC_DC = idesc_bf16(BN, 128, true, true);   // M = vocab (G^T, MN-major), N = 128 of D
-constexpr uint32_t IDESC_DE = idesc_bf16(BM, 128, false, true);  // M = rows (G, K-major), N = 128 of D
+constexpr uint32_t IDESC_DC = idesc_bf16(BN, SLICE, true, true);   // M = vocab (G^T, MN-major), N = 256 of D
+constexpr uint32_t IDESC_DE = idesc_bf16(BM, SLICE, false, true);  // M = rows (G, K-major), N = 256 of D
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
@@ -118,8 +120,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint8_t* __restrict__ gscratch, int out_bf16, int* err, uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* units = base;
-  uint8_t* stg_all = base + UNITS * UNIT_BYTES;
+  uint8_t* stages = base;
+  uint8_t* stg_all = base + STAGES * STAGE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(stg_all + 4 * STG_WARP);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NUM_BARRIERS);
   int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
@@ -127,10 +129,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int u) { return bar0 + 8u * u; };
-  auto empty_bar = [&](int u) { return bar0 + 8u * (UNITS + u); };
-  auto accfull_bar = [&](int a) { return bar0 + 8u * (2 * UNITS + a); };
-  auto accempty_bar = [&](int a) { return bar0 + 8u * (2 * UNITS + 2 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * UNITS + 4);
+  auto empty_bar = [&](int u) { return bar0 + 8u * (STAGES + u); };
+  auto accfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto accempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
 
   const int S = (D + SLICE - 1) / SLICE;
   const int num_items = num_keys * S;
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int slot_base = offsets_t[chunk_t0];
 
   if (threadIdx.x == 0) {
-    for (int u = 0; u < UNITS; ++u) {
+    for (int u = 0; u < STAGES; ++u) {
       mbar_init(full_bar(u), 1);
       mbar_init(empty_bar(u), 1);
     }
@@ -163,112 +165,85 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     // ---------------- producer ----------------
     if (lane == 0) {
-      int unit = 0;
+      int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued[UNITS] = {0, 0, 0, 0, 0, 0};
+      uint32_t issued[STAGES] = {0, 0, 0, 0};
       bool ok = true;
-      auto acquire = [&](uint32_t bytes) -> uint32_t {
-        if (!mbar_wait(empty_bar(unit), phase ^ 1u, wc)) return 0xffffffffu;
-        mbar_arrive_expect_tx(full_bar(unit), bytes);
-        ++issued[unit];
-        return static_cast<uint32_t>(unit);
-      };
-      auto advance = [&]() {
-        if (++unit == UNITS) {
-          unit = 0;
-          phase ^= 1u;
-        }
-      };
       for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
         const ItemRange it = item_in_chunk<kDE>(w, S, chunk_t0, chunk_t1, offsets, entries);
         const int x0 = it.s * SLICE;
-        const int halves = (D - x0 > 128) ? 2 : 1;
         for (int i = it.begin; i < it.end && ok; ++i) {
           const int2 os = entry_of<kDE>(entries, i, slot_base);
-          // gradient tile
-          uint32_t u = acquire(UNIT_BYTES);
-          if (u == 0xffffffffu) {
-            ok = false;
-            break;
-          }
-          bulk_load(smem_u32(units + u * UNIT_BYTES), gscratch + static_cast<size_t>(os.y) * UNIT_BYTES, UNIT_BYTES,
-                    full_bar(u));
-          advance();
-          // operand slice halves: rows of E_b (dC) or C_t (dE), columns x0 .. x0 + 255
-          for (int h = 0; h < halves; ++h) {
-            u = acquire(UNIT_BYTES);
-            if (u == 0xffffffffu) {
+          const uint8_t* tile = gscratch + static_cast<size_t>(os.y) * TILE_BYTES;
+          for (int h = 0; h < 2; ++h) {  // K-halves: 64 rows (dC) or 64 vocabulary columns (dE)
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, wc)) {
               ok = false;
               break;
             }
-            const uint32_t dst = smem_u32(units + u * UNIT_BYTES);
-            const int y = os.x * BM;
-            tma_load_2d(dst, &tmX, full_bar(u), x0 + 128 * h, y);
-            tma_load_2d(dst + BOX_BYTES, &tmX, full_bar(u), x0 + 128 * h + 64, y);
-            advance();
+            const uint32_t dst = smem_u32(stages + stage * STAGE_BYTES);
+            mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
+            if (kDE) {  // G block h: rows 0..127, vocabulary 64h .. 64h + 63 (K-major A)
+              bulk_load(dst, tile + h * G_PART, G_PART, full_bar(stage));
+            } else {  // rows 64h .. 64h + 63 of both 64-column vocabulary blocks (MN-major A = G^T)
+              bulk_load(dst, tile + h * (G_PART / 2), G_PART / 2, full_bar(stage));
+              bulk_load(dst + G_PART / 2, tile + G_PART + h * (G_PART / 2), G_PART / 2, full_bar(stage));
+            }
+            const int y = os.x * BM + 64 * h;  // K rows of the operand: E_b rows (dC), C_t rows (dE)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tma_load_2d(dst + G_PART + c * X_BOX, &tmX, full_bar(stage), x0 + 64 * c, y);
+            ++issued[stage];
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
       }
       if (!ok) {
-        for (int u = 0; u < UNITS; ++u)
+        for (int u = 0; u < STAGES; ++u)
           if (issued[u]) mbar_wait_drain(full_bar(u), (issued[u] - 1u) & 1u, 200000000ull);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      int unit = 0;
+      int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_iter = 0;
       bool ok = true, issued_any = false;
-      auto wait_unit = [&]() -> int {
-        if (!mbar_wait(full_bar(unit), phase, wc)) return -1;
-        tc_fence_after();
-        const int u = unit;
-        if (++unit == UNITS) {
-          unit = 0;
-          phase ^= 1u;
-        }
-        return u;
-      };
       for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
         const ItemRange it = item_in_chunk<kDE>(w, S, chunk_t0, chunk_t1, offsets, entries);
         if (it.begin == it.end) continue;  // nothing to accumulate (dC writes zeros without TMEM)
-        const int halves = (D - it.s * SLICE > 128) ? 2 : 1;
         const int a = acc_iter & 1;
         if (!mbar_wait(accempty_bar(a), ((acc_iter >> 1) & 1u) ^ 1u, wc)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(a * SLICE);
         for (int i = it.begin; i < it.end && ok; ++i) {
-          const int ug = wait_unit();
-          if (ug < 0) {
-            ok = false;
-            break;
-          }
-          const uint32_t g0 = smem_u32(units + ug * UNIT_BYTES);
-          for (int h = 0; h < halves; ++h) {
-            const int ux = wait_unit();
-            if (ux < 0) {
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait(full_bar(stage), phase, wc)) {
               ok = false;
               break;
             }
-            const uint32_t x0 = smem_u32(units + ux * UNIT_BYTES);
-            const uint32_t d = tmem_base + static_cast<uint32_t>(a * SLICE + h * 128);
+            tc_fence_after();
+            const uint32_t g0 = smem_u32(stages + stage * STAGE_BYTES);
+            const uint32_t x0 = g0 + G_PART;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {  // K = 128 (rows for dC, vocabulary for dE), 16 per MMA
-              uint64_t adesc;
-              if (kDE) adesc = sdesc_sw128(g0 + (k >> 2) * BOX_BYTES + 32u * (k & 3), 16, 1024);
-              else adesc = sdesc_sw128(g0 + 2048u * k, BOX_BYTES, 1024);
-              const uint64_t bdesc = sdesc_sw128(x0 + 2048u * k, BOX_BYTES, 1024);
-              tc_mma_bf16(d, adesc, bdesc, kDE ? IDESC_DE : IDESC_DC, (i > it.begin || k > 0) ? 1u : 0u);
+            for (int k = 0; k < 4; ++k) {  // 16 of the 64 K values per MMA
+              const uint64_t adesc = kDE ? sdesc_sw128(g0 + 32u * k, 16, 1024)
+                                         : sdesc_sw128(g0 + 2048u * k, G_PART / 2, 1024);
+              const uint64_t bdesc = sdesc_sw128(x0 + 2048u * k, X_BOX, 1024);
+              tc_mma_bf16(d, adesc, bdesc, kDE ? IDESC_DE : IDESC_DC, (i > it.begin || h > 0 || k > 0) ? 1u : 0u);
             }
             issued_any = true;
-            tc_commit(empty_bar(ux));
+            tc_commit(empty_bar(stage));
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          if (!ok) break;
-          tc_commit(empty_bar(ug));
         }
         if (!ok) break;
         tc_commit(accfull_bar(a));

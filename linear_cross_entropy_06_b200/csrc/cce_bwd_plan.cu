@@ -131,6 +131,51 @@ __global__ void row_list_kernel(const uint8_t* __restrict__ flags, const int* __
   if (pass == 0 && lane == 0) cnt_b[b] = k;
 }
 
+__device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int t) {
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (e[mid].x < t) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// One block per vocabulary chunk: for every row block, the number of pairs of its consecutive
+// listed tiles inside the chunk (the gradient-tile kernel recomputes two vocabulary tiles of one
+// row block at once), and the exclusive prefix sums of those counts.
+__global__ void pair_plan_kernel(const int2* __restrict__ entries_b, const int* __restrict__ offsets_b, int nb,
+                                 int chunk_tiles, int nt, int* __restrict__ pair_off) {
+  __shared__ int buf[1024];
+  __shared__ int carry;
+  const int c = blockIdx.x;
+  const int t0 = c * chunk_tiles, t1 = min(nt, t0 + chunk_tiles);
+  int* out = pair_off + static_cast<int64_t>(c) * (nb + 1);
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < nb; base += 1024) {
+    const int b = base + threadIdx.x;
+    int v = 0;
+    if (b < nb) {
+      const int lo = lower_bound_t(entries_b, offsets_b[b], offsets_b[b + 1], t0);
+      const int hi = lower_bound_t(entries_b, lo, offsets_b[b + 1], t1);
+      v = (hi - lo + 1) / 2;
+    }
+    buf[threadIdx.x] = v;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+      const int add = threadIdx.x >= o ? buf[threadIdx.x - o] : 0;
+      __syncthreads();
+      buf[threadIdx.x] += add;
+      __syncthreads();
+    }
+    if (b < nb) out[b] = carry + buf[threadIdx.x] - v;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry += buf[1023];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out[nb] = carry;
+}
+
 __global__ void plan_finish_kernel(const int* __restrict__ kept_total, int64_t total, int64_t* __restrict__ filtered) {
   *filtered = total - static_cast<int64_t>(*kept_total);
 }
@@ -163,6 +208,8 @@ cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float
     note_launches(1);
     row_list_kernel<<<grid_b, 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt, P.cnt_b, P.offsets_b, P.entries_b,
                                            1);
+    note_launches(1);
+    pair_plan_kernel<<<P.nchunks, 1024, 0, s>>>(P.entries_b, P.offsets_b, nb, P.chunk_tiles, nt, P.pair_off);
     note_launches(1);
   }
   plan_finish_kernel<<<1, 1, 0, s>>>(P.kept_total, static_cast<int64_t>(nb) * nt, filtered_tiles);

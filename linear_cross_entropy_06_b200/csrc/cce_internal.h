@@ -51,26 +51,33 @@ struct BwdPlan {
   int* offsets_b;   // [nb + 1]
   int2* entries_b;  // [nb * nt]: (t, slot in entries_t), by row block then vocabulary tile
   int* kept_total;
+  int chunk_tiles;  // vocabulary tiles per chunk
+  int nchunks;
+  int* pair_off;    // [nchunks * (nb + 1)]: per chunk, prefix sums over row blocks of the number of
+                    // pairs of consecutive listed tiles of that row block inside the chunk
 };
 
 struct BwdGradTiles {
   CUtensorMap tmE, tmC;  // bf16, box 64 x 128
+  int nb, nt;
+  const uint8_t* flags;
+  const int2* entries_b;
+  const int* offsets_b;
+  const int* pair_off;   // of this chunk: [nb + 1]
   int N, D, V;
   const float* lse;
   const float* scale;
   const int64_t* targets;
   int64_t ignore_index;
-  const int2* entries_t;
   const int* offsets_t;
   uint8_t* gscratch;
-  int max_entries_per_chunk;
   int num_sms;
   int* err;
   uint64_t timeout_ns;
 };
 
 struct BwdGemm {
-  CUtensorMap tmE, tmC;  // bf16, box 64 x 128 (operand slices)
+  CUtensorMap tmE, tmC;  // bf16, box 64 x 64 (operand slices, one K-half of 64 rows per stage)
   CUtensorMap tmdE;      // fp32 dE accumulator, box 32 x 32 (reduce-add)
   CUtensorMap tmdC;      // dC output: bf16 box 64 x 32, or fp32 box 32 x 32
   int N, D, V, nb;
@@ -88,7 +95,7 @@ struct BwdGemm {
 cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float* lse, const int64_t* targets,
                             int64_t N, int64_t V, int64_t T, int64_t ignore_index, float filter_eps,
                             int64_t* filtered_tiles, cudaStream_t s);
-cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk_t0, int chunk_t1, cudaStream_t s);
+cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk, int chunk_t0, int chunk_t1, cudaStream_t s);
 cudaError_t launch_bwd_gemm(const BwdGemm& L, bool dE_mode, int chunk_t0, int chunk_t1, cudaStream_t s);
 
 cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
