@@ -101,7 +101,6 @@ struct SplitWs {
   cce::BwdPlan plan;
   uint8_t* gscratch;
   float* dE_acc;
-  int64_t chunk_tiles;  // vocabulary tiles per chunk
   size_t bytes;
 };
 
@@ -129,14 +128,18 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.offsets_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nb + 1)));
   w.plan.entries_b = reinterpret_cast<int2*>(take(sizeof(int2) * static_cast<size_t>(tiles)));
   w.plan.kept_total = reinterpret_cast<int*>(take(sizeof(int)));
-  // Vocabulary tiles per chunk: the chunk's gradient tiles (at most nb of them per vocabulary
-  // tile) fit in the scratch budget; at least one vocabulary tile per chunk.
+  // A chunk spans at most kChunkCBytes of C (its C rows stay in L2 while they are re-read for
+  // every listed row block), and its gradient tiles, at most nb per vocabulary tile, fit in
+  // kGradScratchBudget; at least one vocabulary tile per chunk.
+  const int64_t vt_bytes = static_cast<int64_t>(cce::kBwdBN) * p->D * 2;
   const int64_t per_vtile = std::max<int64_t>(nb, 1) * cce::kGradTileBytes;
-  w.chunk_tiles = std::max<int64_t>(1, std::min<int64_t>(nt, cce::kGradScratchBudget / per_vtile));
-  w.plan.chunk_tiles = static_cast<int>(w.chunk_tiles);
-  w.plan.nchunks = static_cast<int>(ceil_div(nt, w.chunk_tiles));
-  w.plan.pair_off = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks * (nb + 1))));
-  w.gscratch = reinterpret_cast<uint8_t*>(take(static_cast<size_t>(per_vtile * w.chunk_tiles)));
+  const int64_t chunk_vt = std::max<int64_t>(
+      1, std::min({nt, cce::kChunkCBytes / vt_bytes, cce::kGradScratchBudget / per_vtile}));
+  w.plan.chunk_vt = static_cast<int>(chunk_vt);
+  w.plan.nchunks = static_cast<int>(ceil_div(nt, chunk_vt));
+  w.plan.chunk_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks + 1)));
+  w.plan.pair_off = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks) * (nb + 1)));
+  w.gscratch = reinterpret_cast<uint8_t*>(take(static_cast<size_t>(nb * chunk_vt) * cce::kGradTileBytes));
   if (!out_fp32) w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
   w.bytes = off;
   return w;
@@ -252,6 +255,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   G.entries_b = w.plan.entries_b;
   G.offsets_b = w.plan.offsets_b;
   G.pair_off = w.plan.pair_off;
+  G.chunk_t = w.plan.chunk_t;
   G.offsets_t = w.plan.offsets_t;
   G.gscratch = w.gscratch;
   G.num_sms = num_sms;
@@ -273,19 +277,16 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   M.entries_b = w.plan.entries_b;
   M.offsets_b = w.plan.offsets_b;
   M.gscratch = w.gscratch;
+  M.chunk_t = w.plan.chunk_t;
   M.dC_bf16 = out_fp32 ? 0 : 1;
   M.num_sms = num_sms;
   M.err = G.err;
   M.timeout_ns = G.timeout_ns;
 
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
-  const int nt = w.plan.nt;
   for (int c = 0; c < w.plan.nchunks; ++c) {
-    const int c0 = static_cast<int>(c * w.chunk_tiles);
-    const int c1 = static_cast<int>(std::min<int64_t>(nt, c0 + w.chunk_tiles));
-    CCE_TRY(cce::launch_bwd_g(G, c, c0, c1, s));
-    CCE_TRY(cce::launch_bwd_gemm(M, false, c0, c1, s));
-    CCE_TRY(cce::launch_bwd_gemm(M, true, c0, c1, s));
+    CCE_TRY(cce::launch_bwd_g(G, c, s));
+    CCE_TRY(cce::launch_bwd_gemm(M, c, s));
   }
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
   if (!out_fp32) CCE_TRY(cce::launch_to_bf16(dE_acc, static_cast<__nv_bfloat16*>(dE), N * D, s));

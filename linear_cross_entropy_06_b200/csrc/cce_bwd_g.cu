@@ -96,8 +96,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                  const float* __restrict__ lse, const float* __restrict__ scale, const int64_t* __restrict__ targets,
                  int64_t ignore_index, const int* __restrict__ offsets_t, const uint8_t* __restrict__ flags, int nb,
                  int nt, const int2* __restrict__ entries_b, const int* __restrict__ offsets_b,
-                 const int* __restrict__ pair_off, int chunk_t0, int chunk_t1, uint8_t* __restrict__ gscratch,
-                 int* err, uint64_t timeout_ns) {
+                 const int* __restrict__ pair_off, const int* __restrict__ chunk_t, int chunk,
+                 uint8_t* __restrict__ gscratch, int* err, uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int num_pairs = pair_off[nb];
   if (num_pairs <= static_cast<int>(blockIdx.x)) return;  // uniform across the CTA, before any sync
+  const int chunk_t0 = chunk_t[chunk], chunk_t1 = chunk_t[chunk + 1];
   const int slot_base = offsets_t[chunk_t0];
   auto get_pair = [&](int w) {
     return pair_at(w, pair_off, nb, entries_b, offsets_b, flags, nt, chunk_t0, chunk_t1, slot_base);
@@ -320,16 +321,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 }  // namespace
 
-cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk, int chunk_t0, int chunk_t1, cudaStream_t s) {
+cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(bwd_g_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  // At most one pair per two listed tiles of a row block, plus one per row block for an odd count.
-  const long long bound = static_cast<long long>(L.nb) * ((chunk_t1 - chunk_t0 + 1) / 2 + 1);
-  const int grid = static_cast<int>(bound < L.num_sms ? bound : L.num_sms);
-  if (grid <= 0) return cudaSuccess;
+  const int grid = L.num_sms;  // CTAs past the chunk's pair count exit at once
   bwd_g_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(
       L.tmE, L.tmC, L.N, L.D, L.V, L.lse, L.scale, L.targets, L.ignore_index, L.offsets_t, L.flags, L.nb, L.nt,
-      L.entries_b, L.offsets_b, L.pair_off + static_cast<int64_t>(chunk) * (L.nb + 1), chunk_t0, chunk_t1,
+      L.entries_b, L.offsets_b, L.pair_off + static_cast<int64_t>(chunk) * (L.nb + 1), L.chunk_t, chunk,
       L.gscratch, L.err, L.timeout_ns);
   note_launches(1);
   return cudaGetLastError();

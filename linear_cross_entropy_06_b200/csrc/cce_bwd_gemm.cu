@@ -1,5 +1,6 @@
-// Backward, steps 2 and 3 of 3 per vocabulary chunk: the gradient MMAs, from bf16 gradient tiles
-// in shared memory, with fp32 accumulation in TMEM.
+// Backward, step 2 of 2 per vocabulary chunk: the gradient MMAs, from bf16 gradient tiles in shared
+// memory, with fp32 accumulation in TMEM. One launch per chunk runs both kinds of work item (dE
+// items first: they are the longer ones), so the chunk has a single tail.
 //
 //   dC mode  work item (vocabulary tile t, 256-column slice s of D):
 //            dC[t rows, s cols] = sum over listed b of G_bt^T E_b[:, s]     (written directly; every
@@ -61,26 +62,9 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
 }
 
 struct ItemRange {
+  bool de;                 // dE item (row block key) or dC item (vocabulary tile key)
   int key, s, begin, end;  // entries [begin, end) of the key's list
 };
-
-// The work item's key tile, slice, and the range of its list entries inside this chunk.
-template <bool kDE>
-__device__ __forceinline__ ItemRange item_range(int w, int S, int chunk_t0, int chunk_t1, const int* offsets) {
-  ItemRange it;
-  it.s = w % S;
-  if (!kDE) {
-    it.key = chunk_t0 + w / S;
-    it.begin = offsets[it.key];
-    it.end = offsets[it.key + 1];
-    return it;
-  }
-  it.key = w / S;
-  // entries_b of row block b are sorted by vocabulary tile; the caller narrows to the chunk.
-  it.begin = offsets[it.key];
-  it.end = offsets[it.key + 1];
-  return it;
-}
 
 __device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int t) {
   while (lo < hi) {
@@ -91,33 +75,49 @@ __device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int 
   return lo;
 }
 
-template <bool kDE>
-__device__ __forceinline__ ItemRange item_in_chunk(int w, int S, int chunk_t0, int chunk_t1, const int* offsets,
-                                                   const int2* entries) {
-  ItemRange it = item_range<kDE>(w, S, chunk_t0, chunk_t1, offsets);
-  if (kDE) {
-    const int lo = lower_bound_t(entries, it.begin, it.end, chunk_t0);
-    const int hi = lower_bound_t(entries, lo, it.end, chunk_t1);
+// Items [0, nb * S) are dE items (row block w / S, slice w % S); the rest are dC items (vocabulary
+// tile chunk_t0 + (w - nb S) / S). Each gets the range of its list entries inside this chunk:
+// entries_b of a row block are sorted by vocabulary tile, entries_t of a vocabulary tile are all
+// inside the chunk.
+__device__ __forceinline__ ItemRange item_in_chunk(int w, int S, int nb, int chunk_t0, int chunk_t1,
+                                                   const int* offsets_b, const int2* entries_b,
+                                                   const int* offsets_t) {
+  ItemRange it;
+  it.de = w < nb * S;
+  if (it.de) {
+    it.key = w / S;
+    it.s = w % S;
+    const int lo = lower_bound_t(entries_b, offsets_b[it.key], offsets_b[it.key + 1], chunk_t0);
     it.begin = lo;
-    it.end = hi;
+    it.end = lower_bound_t(entries_b, lo, offsets_b[it.key + 1], chunk_t1);
+  } else {
+    const int v = w - nb * S;
+    it.key = chunk_t0 + v / S;
+    it.s = v % S;
+    it.begin = offsets_t[it.key];
+    it.end = offsets_t[it.key + 1];
   }
   return it;
 }
 
-// Entry i of a list -> (tile index of the "other" operand, slot of its gradient tile in the chunk).
-template <bool kDE>
-__device__ __forceinline__ int2 entry_of(const int2* entries, int i, int slot_base) {
-  const int2 en = entries[i];
-  if (!kDE) return make_int2(en.x >> 2, i - slot_base);  // (row block b, slot)
-  return make_int2(en.x, en.y - slot_base);              // (vocabulary tile t, slot)
+// Entry i of the item's list -> (tile index of the "other" operand, slot of its gradient tile).
+__device__ __forceinline__ int2 entry_of(bool de, const int2* entries_b, const int2* entries_t, int i,
+                                         int slot_base) {
+  if (de) {
+    const int2 en = entries_b[i];
+    return make_int2(en.x, en.y - slot_base);  // (vocabulary tile t, slot)
+  }
+  const int2 en = entries_t[i];
+  return make_int2(en.x >> 2, i - slot_base);  // (row block b, slot)
 }
 
-template <bool kDE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmOut, int N, int D,
-                    int V, const int2* __restrict__ entries, const int* __restrict__ offsets,
-                    const int* __restrict__ offsets_t, int chunk_t0, int chunk_t1, int num_keys,
-                    const uint8_t* __restrict__ gscratch, int out_bf16, int* err, uint64_t timeout_ns) {
+    bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC,
+                    const __grid_constant__ CUtensorMap tmdC, const __grid_constant__ CUtensorMap tmdE, int N, int D,
+                    int V, const int2* __restrict__ entries_t, const int* __restrict__ offsets_t,
+                    const int2* __restrict__ entries_b, const int* __restrict__ offsets_b,
+                    const int* __restrict__ chunk_t, int chunk, int nb, const uint8_t* __restrict__ gscratch,
+                    int out_bf16, int* err, uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
@@ -135,8 +135,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
 
   const int S = (D + SLICE - 1) / SLICE;
-  const int num_items = num_keys * S;
+  const int chunk_t0 = chunk_t[chunk], chunk_t1 = chunk_t[chunk + 1];
+  if (chunk_t0 >= chunk_t1) return;  // empty chunk
+  const int num_items = (nb + chunk_t1 - chunk_t0) * S;
   if (num_items <= static_cast<int>(blockIdx.x)) return;
+  auto item = [&](int w) {
+    return item_in_chunk(w, S, nb, chunk_t0, chunk_t1, offsets_b, entries_b, offsets_t);
+  };
   const int slot_base = offsets_t[chunk_t0];
 
   if (threadIdx.x == 0) {
@@ -170,10 +175,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t issued[STAGES] = {0, 0, 0, 0};
       bool ok = true;
       for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
-        const ItemRange it = item_in_chunk<kDE>(w, S, chunk_t0, chunk_t1, offsets, entries);
+        const ItemRange it = item(w);
         const int x0 = it.s * SLICE;
         for (int i = it.begin; i < it.end && ok; ++i) {
-          const int2 os = entry_of<kDE>(entries, i, slot_base);
+          const int2 os = entry_of(it.de, entries_b, entries_t, i, slot_base);
           const uint8_t* tile = gscratch + static_cast<size_t>(os.y) * TILE_BYTES;
           for (int h = 0; h < 2; ++h) {  // K-halves: 64 rows (dC) or 64 vocabulary columns (dE)
             if (!mbar_wait(empty_bar(stage), phase ^ 1u, wc)) {
@@ -182,7 +187,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             const uint32_t dst = smem_u32(stages + stage * STAGE_BYTES);
             mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
-            if (kDE) {  // G block h: rows 0..127, vocabulary 64h .. 64h + 63 (K-major A)
+            if (it.de) {  // G block h: rows 0..127, vocabulary 64h .. 64h + 63 (K-major A)
               bulk_load(dst, tile + h * G_PART, G_PART, full_bar(stage));
             } else {  // rows 64h .. 64h + 63 of both 64-column vocabulary blocks (MN-major A = G^T)
               bulk_load(dst, tile + h * (G_PART / 2), G_PART / 2, full_bar(stage));
@@ -190,7 +195,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             const int y = os.x * BM + 64 * h;  // K rows of the operand: E_b rows (dC), C_t rows (dE)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tma_load_2d(dst + G_PART + c * X_BOX, &tmX, full_bar(stage), x0 + 64 * c, y);
+            for (int c = 0; c < 4; ++c)
+              tma_load_2d(dst + G_PART + c * X_BOX, it.de ? &tmC : &tmE, full_bar(stage), x0 + 64 * c, y);
             ++issued[stage];
             if (++stage == STAGES) {
               stage = 0;
@@ -212,7 +218,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t acc_iter = 0;
       bool ok = true, issued_any = false;
       for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
-        const ItemRange it = item_in_chunk<kDE>(w, S, chunk_t0, chunk_t1, offsets, entries);
+        const ItemRange it = item(w);
         if (it.begin == it.end) continue;  // nothing to accumulate (dC writes zeros without TMEM)
         const int a = acc_iter & 1;
         if (!mbar_wait(accempty_bar(a), ((acc_iter >> 1) & 1u) ^ 1u, wc)) {
@@ -232,10 +238,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t x0 = g0 + G_PART;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {  // 16 of the 64 K values per MMA
-              const uint64_t adesc = kDE ? sdesc_sw128(g0 + 32u * k, 16, 1024)
-                                         : sdesc_sw128(g0 + 2048u * k, G_PART / 2, 1024);
+              const uint64_t adesc = it.de ? sdesc_sw128(g0 + 32u * k, 16, 1024)
+                                           : sdesc_sw128(g0 + 2048u * k, G_PART / 2, 1024);
               const uint64_t bdesc = sdesc_sw128(x0 + 2048u * k, X_BOX, 1024);
-              tc_mma_bf16(d, adesc, bdesc, kDE ? IDESC_DE : IDESC_DC, (i > it.begin || h > 0 || k > 0) ? 1u : 0u);
+              tc_mma_bf16(d, adesc, bdesc, it.de ? IDESC_DE : IDESC_DC, (i > it.begin || h > 0 || k > 0) ? 1u : 0u);
             }
             issued_any = true;
             tc_commit(empty_bar(stage));
@@ -259,12 +265,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t stg = smem_u32(stg_all + q * STG_WARP);
-    const int rows_limit = kDE ? N : V;
     uint32_t acc_iter = 0;
     for (int w = blockIdx.x; w < num_items; w += gridDim.x) {
-      const ItemRange it = item_in_chunk<kDE>(w, S, chunk_t0, chunk_t1, offsets, entries);
+      const ItemRange it = item(w);
       const bool has = it.begin < it.end;
-      if (kDE && !has) continue;  // nothing to add for this row block in this chunk
+      if (it.de && !has) continue;  // nothing to add for this row block in this chunk
+      const int rows_limit = it.de ? N : V;
       const int a = acc_iter & 1;
       if (has) {
         if (!mbar_wait(accfull_bar(a), (acc_iter >> 1) & 1u, wc)) break;
@@ -285,7 +291,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // This warp's staging is free once its previous TMA op has read it.
         if (lane == 0) bulk_wait_group_read0();
         __syncwarp();
-        if (!kDE && out_bf16) {
+        if (!it.de && out_bf16) {
 #pragma unroll
           for (int h = 0; h < 8; ++h) {
             const float* src = h < 4 ? v0 + 8 * h : v1 + 8 * (h - 4);
@@ -304,14 +310,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && y < rows_limit) {
-          if (!kDE && out_bf16) {
-            tma_store_2d(&tmOut, stg, x, y);
-          } else if (!kDE) {
-            tma_store_2d(&tmOut, stg, x, y);
-            if (x + 32 < D) tma_store_2d(&tmOut, stg + 4096u, x + 32, y);
+          if (!it.de && out_bf16) {
+            tma_store_2d(&tmdC, stg, x, y);
+          } else if (!it.de) {
+            tma_store_2d(&tmdC, stg, x, y);
+            if (x + 32 < D) tma_store_2d(&tmdC, stg + 4096u, x + 32, y);
           } else {
-            tma_reduce_add_2d(&tmOut, stg, x, y);
-            if (x + 32 < D) tma_reduce_add_2d(&tmOut, stg + 4096u, x + 32, y);
+            tma_reduce_add_2d(&tmdE, stg, x, y);
+            if (x + 32 < D) tma_reduce_add_2d(&tmdE, stg + 4096u, x + 32, y);
           }
           bulk_commit_group();
         }
@@ -337,22 +343,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 }  // namespace
 
-cudaError_t launch_bwd_gemm(const BwdGemm& L, bool dE_mode, int chunk_t0, int chunk_t1, cudaStream_t s) {
-  const int S = (L.D + SLICE - 1) / SLICE;
-  const int num_keys = dE_mode ? L.nb : (chunk_t1 - chunk_t0);
-  const long long items = static_cast<long long>(num_keys) * S;
-  if (items <= 0) return cudaSuccess;
-  auto kernel = dE_mode ? bwd_gemm_kernel<true> : bwd_gemm_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+cudaError_t launch_bwd_gemm(const BwdGemm& L, int chunk, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int grid = static_cast<int>(items < L.num_sms ? items : L.num_sms);
-  if (dE_mode)
-    kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmC, L.tmdE, L.N, L.D, L.V, L.entries_b, L.offsets_b, L.offsets_t,
-                                                 chunk_t0, chunk_t1, num_keys, L.gscratch, 0, L.err, L.timeout_ns);
-  else
-    kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmdC, L.N, L.D, L.V, L.entries_t, L.offsets_t, L.offsets_t,
-                                                 chunk_t0, chunk_t1, num_keys, L.gscratch, L.dC_bf16, L.err,
-                                                 L.timeout_ns);
+  const int grid = L.num_sms;  // CTAs past the chunk's item count exit at once
+  bwd_gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmC, L.tmdC, L.tmdE, L.N, L.D, L.V, L.entries_t,
+                                                        L.offsets_t, L.entries_b, L.offsets_b, L.chunk_t, chunk, L.nb,
+                                                        L.gscratch, L.dC_bf16, L.err, L.timeout_ns);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -140,15 +140,21 @@ __device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int 
   return lo;
 }
 
+// Chunk boundaries: chunk c covers vocabulary tiles [c * chunk_vt, min(nt, (c + 1) * chunk_vt)).
+__global__ void chunk_plan_kernel(int nt, int chunk_vt, int nchunks, int* __restrict__ chunk_t) {
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c <= nchunks; c += gridDim.x * blockDim.x)
+    chunk_t[c] = min(nt, c * chunk_vt);
+}
+
 // One block per vocabulary chunk: for every row block, the number of pairs of its consecutive
 // listed tiles inside the chunk (the gradient-tile kernel recomputes two vocabulary tiles of one
 // row block at once), and the exclusive prefix sums of those counts.
 __global__ void pair_plan_kernel(const int2* __restrict__ entries_b, const int* __restrict__ offsets_b, int nb,
-                                 int chunk_tiles, int nt, int* __restrict__ pair_off) {
+                                 const int* __restrict__ chunk_t, int* __restrict__ pair_off) {
   __shared__ int buf[1024];
   __shared__ int carry;
   const int c = blockIdx.x;
-  const int t0 = c * chunk_tiles, t1 = min(nt, t0 + chunk_tiles);
+  const int t0 = chunk_t[c], t1 = chunk_t[c + 1];
   int* out = pair_off + static_cast<int64_t>(c) * (nb + 1);
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
@@ -209,7 +215,9 @@ cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float
     row_list_kernel<<<grid_b, 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt, P.cnt_b, P.offsets_b, P.entries_b,
                                            1);
     note_launches(1);
-    pair_plan_kernel<<<P.nchunks, 1024, 0, s>>>(P.entries_b, P.offsets_b, nb, P.chunk_tiles, nt, P.pair_off);
+    chunk_plan_kernel<<<(P.nchunks + 256) / 256, 256, 0, s>>>(nt, P.chunk_vt, P.nchunks, P.chunk_t);
+    note_launches(1);
+    pair_plan_kernel<<<P.nchunks, 1024, 0, s>>>(P.entries_b, P.offsets_b, nb, P.chunk_t, P.pair_off);
     note_launches(1);
   }
   plan_finish_kernel<<<1, 1, 0, s>>>(P.kept_total, static_cast<int64_t>(nb) * nt, filtered_tiles);

@@ -38,7 +38,12 @@ void set_last_error(const char* msg);
 // Split backward (cce_bwd_plan.cu, cce_bwd_g.cu, cce_bwd_gemm.cu).
 constexpr int kGradTileBytes = kBwdBM * kBwdBN * 2;      // one bf16 gradient tile, 128B-swizzled
 constexpr int kGemmSlice = 256;                           // columns of D per dC/dE work item
-constexpr int64_t kGradScratchBudget = int64_t(128) << 20;  // gradient tiles of one vocabulary chunk
+// A vocabulary chunk spans at most kChunkCBytes of C, so that the C rows of a chunk stay in L2
+// while the gradient-tile and dE kernels re-read them for every row block that lists them.
+constexpr int64_t kChunkCBytes = int64_t(128) << 20;
+// ... and its gradient tiles (at most one per listed row block and vocabulary tile) fit in a
+// fixed scratch of kGradScratchBudget.
+constexpr int64_t kGradScratchBudget = int64_t(128) << 20;
 
 struct BwdPlan {
   int nb, nt;
@@ -51,8 +56,9 @@ struct BwdPlan {
   int* offsets_b;   // [nb + 1]
   int2* entries_b;  // [nb * nt]: (t, slot in entries_t), by row block then vocabulary tile
   int* kept_total;
-  int chunk_tiles;  // vocabulary tiles per chunk
+  int chunk_vt;     // vocabulary tiles per chunk
   int nchunks;
+  int* chunk_t;     // [nchunks + 1]: first vocabulary tile of each chunk
   int* pair_off;    // [nchunks * (nb + 1)]: per chunk, prefix sums over row blocks of the number of
                     // pairs of consecutive listed tiles of that row block inside the chunk
 };
@@ -64,6 +70,7 @@ struct BwdGradTiles {
   const int2* entries_b;
   const int* offsets_b;
   const int* pair_off;   // of this chunk: [nb + 1]
+  const int* chunk_t;
   int N, D, V;
   const float* lse;
   const float* scale;
@@ -86,6 +93,7 @@ struct BwdGemm {
   const int2* entries_b;
   const int* offsets_b;
   const uint8_t* gscratch;
+  const int* chunk_t;
   int dC_bf16;
   int num_sms;
   int* err;
@@ -95,8 +103,8 @@ struct BwdGemm {
 cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float* lse, const int64_t* targets,
                             int64_t N, int64_t V, int64_t T, int64_t ignore_index, float filter_eps,
                             int64_t* filtered_tiles, cudaStream_t s);
-cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk, int chunk_t0, int chunk_t1, cudaStream_t s);
-cudaError_t launch_bwd_gemm(const BwdGemm& L, bool dE_mode, int chunk_t0, int chunk_t1, cudaStream_t s);
+cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk, cudaStream_t s);
+cudaError_t launch_bwd_gemm(const BwdGemm& L, int chunk, cudaStream_t s);
 
 cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
 
