@@ -139,6 +139,11 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.nchunks = static_cast<int>(ceil_div(nt, chunk_vt));
   w.plan.chunk_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks + 1)));
   w.plan.pair_off = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks) * (nb + 1)));
+  w.plan.rb_range = reinterpret_cast<int2*>(take(sizeof(int2) * static_cast<size_t>(w.plan.nchunks) * nb));
+  w.plan.pair_cap = nb * ((chunk_vt + 1) / 2);
+  const size_t pairs = static_cast<size_t>(w.plan.nchunks) * static_cast<size_t>(w.plan.pair_cap);
+  w.plan.pair_desc = reinterpret_cast<int4*>(take(sizeof(int4) * pairs));
+  w.plan.pair_slot = reinterpret_cast<int2*>(take(sizeof(int2) * pairs));
   w.gscratch = reinterpret_cast<uint8_t*>(take(static_cast<size_t>(nb * chunk_vt) * cce::kGradTileBytes));
   if (!out_fp32) w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
   w.bytes = off;
@@ -250,13 +255,10 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   G.targets = targets;
   G.ignore_index = p->ignore_index;
   G.nb = w.plan.nb;
-  G.nt = w.plan.nt;
-  G.flags = w.plan.flags;
-  G.entries_b = w.plan.entries_b;
-  G.offsets_b = w.plan.offsets_b;
   G.pair_off = w.plan.pair_off;
-  G.chunk_t = w.plan.chunk_t;
-  G.offsets_t = w.plan.offsets_t;
+  G.pair_cap = w.plan.pair_cap;
+  G.pair_desc = w.plan.pair_desc;
+  G.pair_slot = w.plan.pair_slot;
   G.gscratch = w.gscratch;
   G.num_sms = num_sms;
   G.err = &w.hdr->err;
@@ -275,7 +277,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   M.entries_t = w.plan.entries_t;
   M.offsets_t = w.plan.offsets_t;
   M.entries_b = w.plan.entries_b;
-  M.offsets_b = w.plan.offsets_b;
+  M.rb_range = w.plan.rb_range;
   M.gscratch = w.gscratch;
   M.chunk_t = w.plan.chunk_t;
   M.dC_bf16 = out_fp32 ? 0 : 1;

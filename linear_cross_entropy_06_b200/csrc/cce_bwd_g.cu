@@ -49,16 +49,8 @@ __device__ __forceinline__ void bulk_store_32k(void* gdst, uint32_t src) {
                : "memory");
 }
 
-__device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int t) {
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (e[mid].x < t) lo = mid + 1;
-    else hi = mid;
-  }
-  return lo;
-}
-
-// Pair w of this chunk: its row block, and its one or two tiles (vocabulary tile, slot, kept?).
+// Pair w of this chunk: its row block, and its one or two tiles (vocabulary tile, slot, kept?),
+// from the plan's flat pair list (one 16-byte and one 8-byte load).
 struct Pair {
   int b;
   int t[2], slot[2];
@@ -66,38 +58,27 @@ struct Pair {
   __device__ bool any_kept() const { return kept[0] || kept[1]; }
 };
 
-__device__ __forceinline__ Pair pair_at(int w, const int* pair_off, int nb, const int2* entries_b,
-                                        const int* offsets_b, const uint8_t* flags, int nt, int chunk_t0,
-                                        int chunk_t1, int slot_base) {
-  int lo = 0, hi = nb;  // largest b with pair_off[b] <= w
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (pair_off[mid] <= w) lo = mid;
-    else hi = mid;
-  }
+__device__ __forceinline__ Pair pair_at(int w, const int4* pair_desc, const int2* pair_slot) {
+  const int4 d = pair_desc[w];
+  const int2 sl = pair_slot[w];
   Pair p;
-  p.b = lo;
-  const int first = lower_bound_t(entries_b, offsets_b[lo], offsets_b[lo + 1], chunk_t0);
-  const int last = lower_bound_t(entries_b, first, offsets_b[lo + 1], chunk_t1);
-  const int i0 = first + 2 * (w - pair_off[lo]);
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    p.present[k] = i0 + k < last;
-    const int2 en = entries_b[p.present[k] ? i0 + k : i0];
-    p.t[k] = en.x;
-    p.slot[k] = en.y - slot_base;
-    p.kept[k] = p.present[k] && flags[static_cast<int64_t>(lo) * nt + en.x] == 1;
-  }
+  p.b = d.x;
+  p.t[0] = d.y;
+  p.t[1] = d.z >= 0 ? d.z : d.y;
+  p.present[0] = true;
+  p.present[1] = d.z >= 0;
+  p.kept[0] = (d.w & 1) != 0;
+  p.kept[1] = (d.w & 2) != 0;
+  p.slot[0] = sl.x;
+  p.slot[1] = sl.y;
   return p;
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_g_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC, int N, int D, int V,
                  const float* __restrict__ lse, const float* __restrict__ scale, const int64_t* __restrict__ targets,
-                 int64_t ignore_index, const int* __restrict__ offsets_t, const uint8_t* __restrict__ flags, int nb,
-                 int nt, const int2* __restrict__ entries_b, const int* __restrict__ offsets_b,
-                 const int* __restrict__ pair_off, const int* __restrict__ chunk_t, int chunk,
-                 uint8_t* __restrict__ gscratch, int* err, uint64_t timeout_ns) {
+                 int64_t ignore_index, const int* __restrict__ num_pairs_p, const int4* __restrict__ pair_desc,
+                 const int2* __restrict__ pair_slot, uint8_t* __restrict__ gscratch, int* err, uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
@@ -116,13 +97,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t gfree_bar = bar0 + 8u * (2 * STAGES + 5);   // leader: the smem G buffer may be rewritten
   const uint32_t gready_bar = bar0 + 8u * (2 * STAGES + 6);  // all 128 rows of G are in smem
 
-  const int num_pairs = pair_off[nb];
+  const int num_pairs = *num_pairs_p;
   if (num_pairs <= static_cast<int>(blockIdx.x)) return;  // uniform across the CTA, before any sync
-  const int chunk_t0 = chunk_t[chunk], chunk_t1 = chunk_t[chunk + 1];
-  const int slot_base = offsets_t[chunk_t0];
-  auto get_pair = [&](int w) {
-    return pair_at(w, pair_off, nb, entries_b, offsets_b, flags, nt, chunk_t0, chunk_t1, slot_base);
-  };
+  // Each role loads the next pair's descriptor before working on the current one.
+  auto get_pair = [&](int w) { return pair_at(w < num_pairs ? w : static_cast<int>(blockIdx.x), pair_desc, pair_slot); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -156,8 +134,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued[STAGES] = {0, 0, 0, 0};
       bool ok = true;
+      Pair nx = get_pair(blockIdx.x);
       for (int w = blockIdx.x; w < num_pairs && ok; w += gridDim.x) {
-        const Pair p = get_pair(w);
+        const Pair p = nx;
+        nx = get_pair(w + gridDim.x);
         if (!p.any_kept()) continue;  // onehot-only tiles need no recompute
         const int rb = p.b * BM;
         const int vb0 = p.t[0] * BN, vb1 = (p.present[1] ? p.t[1] : p.t[0]) * BN;
@@ -189,8 +169,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t sidx = 0;
       bool ok = true, issued_any = false;
+      Pair nx = get_pair(blockIdx.x);
       for (int w = blockIdx.x; w < num_pairs && ok; w += gridDim.x) {
-        const Pair p = get_pair(w);
+        const Pair p = nx;
+        nx = get_pair(w + gridDim.x);
         if (!p.any_kept()) continue;
         const int a = sidx & 1;
         if (!mbar_wait(sempty_bar(a), ((sidx >> 1) & 1u) ^ 1u, wc)) {
@@ -325,9 +307,10 @@ cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(bwd_g_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = L.num_sms;  // CTAs past the chunk's pair count exit at once
+  const int64_t first = static_cast<int64_t>(chunk) * L.pair_cap;
   bwd_g_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(
-      L.tmE, L.tmC, L.N, L.D, L.V, L.lse, L.scale, L.targets, L.ignore_index, L.offsets_t, L.flags, L.nb, L.nt,
-      L.entries_b, L.offsets_b, L.pair_off + static_cast<int64_t>(chunk) * (L.nb + 1), L.chunk_t, chunk,
+      L.tmE, L.tmC, L.N, L.D, L.V, L.lse, L.scale, L.targets, L.ignore_index,
+      L.pair_off + static_cast<int64_t>(chunk) * (L.nb + 1) + L.nb, L.pair_desc + first, L.pair_slot + first,
       L.gscratch, L.err, L.timeout_ns);
   note_launches(1);
   return cudaGetLastError();

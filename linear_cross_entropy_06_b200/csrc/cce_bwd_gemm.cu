@@ -66,30 +66,20 @@ struct ItemRange {
   int key, s, begin, end;  // entries [begin, end) of the key's list
 };
 
-__device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int t) {
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (e[mid].x < t) lo = mid + 1;
-    else hi = mid;
-  }
-  return lo;
-}
-
 // Items [0, nb * S) are dE items (row block w / S, slice w % S); the rest are dC items (vocabulary
-// tile chunk_t0 + (w - nb S) / S). Each gets the range of its list entries inside this chunk:
-// entries_b of a row block are sorted by vocabulary tile, entries_t of a vocabulary tile are all
-// inside the chunk.
-__device__ __forceinline__ ItemRange item_in_chunk(int w, int S, int nb, int chunk_t0, int chunk_t1,
-                                                   const int* offsets_b, const int2* entries_b,
+// tile chunk_t0 + (w - nb S) / S). Each gets the range of its list entries inside this chunk: for
+// a row block, the plan's range of its entries_b inside the chunk; for a vocabulary tile, all of
+// its entries_t (every listed tile of a vocabulary tile lies in the tile's chunk).
+__device__ __forceinline__ ItemRange item_in_chunk(int w, int S, int nb, int chunk_t0, const int2* rb_range,
                                                    const int* offsets_t) {
   ItemRange it;
   it.de = w < nb * S;
   if (it.de) {
     it.key = w / S;
     it.s = w % S;
-    const int lo = lower_bound_t(entries_b, offsets_b[it.key], offsets_b[it.key + 1], chunk_t0);
-    it.begin = lo;
-    it.end = lower_bound_t(entries_b, lo, offsets_b[it.key + 1], chunk_t1);
+    const int2 r = rb_range[it.key];
+    it.begin = r.x;
+    it.end = r.y;
   } else {
     const int v = w - nb * S;
     it.key = chunk_t0 + v / S;
@@ -115,7 +105,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC,
                     const __grid_constant__ CUtensorMap tmdC, const __grid_constant__ CUtensorMap tmdE, int N, int D,
                     int V, const int2* __restrict__ entries_t, const int* __restrict__ offsets_t,
-                    const int2* __restrict__ entries_b, const int* __restrict__ offsets_b,
+                    const int2* __restrict__ entries_b, const int2* __restrict__ rb_range,
                     const int* __restrict__ chunk_t, int chunk, int nb, const uint8_t* __restrict__ gscratch,
                     int out_bf16, int* err, uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
@@ -139,8 +129,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (chunk_t0 >= chunk_t1) return;  // empty chunk
   const int num_items = (nb + chunk_t1 - chunk_t0) * S;
   if (num_items <= static_cast<int>(blockIdx.x)) return;
+  // Each role loads the next item's range before working on the current one.
   auto item = [&](int w) {
-    return item_in_chunk(w, S, nb, chunk_t0, chunk_t1, offsets_b, entries_b, offsets_t);
+    return item_in_chunk(w < num_items ? w : static_cast<int>(blockIdx.x), S, nb, chunk_t0, rb_range, offsets_t);
   };
   const int slot_base = offsets_t[chunk_t0];
 
@@ -174,11 +165,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued[STAGES] = {0, 0, 0, 0};
       bool ok = true;
+      ItemRange nx = item(blockIdx.x);
       for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
-        const ItemRange it = item(w);
+        const ItemRange it = nx;
+        nx = item(w + gridDim.x);
         const int x0 = it.s * SLICE;
+        int2 os_next = it.begin < it.end ? entry_of(it.de, entries_b, entries_t, it.begin, slot_base) : make_int2(0, 0);
         for (int i = it.begin; i < it.end && ok; ++i) {
-          const int2 os = entry_of(it.de, entries_b, entries_t, i, slot_base);
+          const int2 os = os_next;
+          if (i + 1 < it.end) os_next = entry_of(it.de, entries_b, entries_t, i + 1, slot_base);
           const uint8_t* tile = gscratch + static_cast<size_t>(os.y) * TILE_BYTES;
           for (int h = 0; h < 2; ++h) {  // K-halves: 64 rows (dC) or 64 vocabulary columns (dE)
             if (!mbar_wait(empty_bar(stage), phase ^ 1u, wc)) {
@@ -217,8 +212,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t acc_iter = 0;
       bool ok = true, issued_any = false;
+      ItemRange nx = item(blockIdx.x);
       for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
-        const ItemRange it = item(w);
+        const ItemRange it = nx;
+        nx = item(w + gridDim.x);
         if (it.begin == it.end) continue;  // nothing to accumulate (dC writes zeros without TMEM)
         const int a = acc_iter & 1;
         if (!mbar_wait(accempty_bar(a), ((acc_iter >> 1) & 1u) ^ 1u, wc)) {
@@ -347,9 +344,10 @@ cudaError_t launch_bwd_gemm(const BwdGemm& L, int chunk, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = L.num_sms;  // CTAs past the chunk's item count exit at once
-  bwd_gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmC, L.tmdC, L.tmdE, L.N, L.D, L.V, L.entries_t,
-                                                        L.offsets_t, L.entries_b, L.offsets_b, L.chunk_t, chunk, L.nb,
-                                                        L.gscratch, L.dC_bf16, L.err, L.timeout_ns);
+  bwd_gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(
+      L.tmE, L.tmC, L.tmdC, L.tmdE, L.N, L.D, L.V, L.entries_t, L.offsets_t, L.entries_b,
+      L.rb_range + static_cast<int64_t>(chunk) * L.nb, L.chunk_t, chunk, L.nb, L.gscratch, L.dC_bf16, L.err,
+      L.timeout_ns);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -13,6 +13,10 @@
 //   each (b * 4 + flag, t), row blocks ascending. An entry's position is also its gradient-tile slot.
 // By row block (dE kernel): offsets_b[b] .. offsets_b[b+1] index entries_b, each (t, slot),
 //   vocabulary tiles ascending.
+// Per vocabulary chunk c, flat work lists the backward kernels read with one load per item:
+//   rb_range[c * nb + b]   the entries [lo, hi) of row block b inside the chunk;
+//   pair_desc/pair_slot    from c * pair_cap: the pairs of consecutive listed tiles of a row block
+//                          inside the chunk, row blocks ascending (pair_off[c] holds their prefix sums).
 #include "cce_device.cuh"
 #include "cce_internal.h"
 
@@ -150,7 +154,8 @@ __global__ void chunk_plan_kernel(int nt, int chunk_vt, int nchunks, int* __rest
 // listed tiles inside the chunk (the gradient-tile kernel recomputes two vocabulary tiles of one
 // row block at once), and the exclusive prefix sums of those counts.
 __global__ void pair_plan_kernel(const int2* __restrict__ entries_b, const int* __restrict__ offsets_b, int nb,
-                                 const int* __restrict__ chunk_t, int* __restrict__ pair_off) {
+                                 const int* __restrict__ chunk_t, int* __restrict__ pair_off,
+                                 int2* __restrict__ rb_range) {
   __shared__ int buf[1024];
   __shared__ int carry;
   const int c = blockIdx.x;
@@ -165,6 +170,7 @@ __global__ void pair_plan_kernel(const int2* __restrict__ entries_b, const int* 
       const int lo = lower_bound_t(entries_b, offsets_b[b], offsets_b[b + 1], t0);
       const int hi = lower_bound_t(entries_b, lo, offsets_b[b + 1], t1);
       v = (hi - lo + 1) / 2;
+      rb_range[static_cast<int64_t>(c) * nb + b] = make_int2(lo, hi);
     }
     buf[threadIdx.x] = v;
     __syncthreads();
@@ -180,6 +186,33 @@ __global__ void pair_plan_kernel(const int2* __restrict__ entries_b, const int* 
     __syncthreads();
   }
   if (threadIdx.x == 0) out[nb] = carry;
+}
+
+// One warp per (chunk, row block): writes that row block's pairs into the chunk's pair list.
+// pair_desc = (b, t of the first tile, t of the second tile or -1, kept bits: 1 first, 2 second);
+// pair_slot = the two tiles' gradient-tile slots relative to the chunk's first slot.
+__global__ void pair_fill_kernel(const int2* __restrict__ entries_b, const uint8_t* __restrict__ flags, int nb, int nt,
+                                 int nchunks, const int* __restrict__ chunk_t, const int* __restrict__ offsets_t,
+                                 const int2* __restrict__ rb_range, const int* __restrict__ pair_off,
+                                 int64_t pair_cap, int4* __restrict__ pair_desc, int2* __restrict__ pair_slot) {
+  const int64_t total = static_cast<int64_t>(nb) * nchunks;
+  for (int64_t cb = blockIdx.x; cb < total; cb += gridDim.x) {
+    const int c = static_cast<int>(cb / nb), b = static_cast<int>(cb % nb);
+    const int2 r = rb_range[cb];
+    const int slot_base = offsets_t[chunk_t[c]];
+    const int64_t out0 = static_cast<int64_t>(c) * pair_cap + pair_off[static_cast<int64_t>(c) * (nb + 1) + b];
+    const int np = (r.y - r.x + 1) / 2;
+    for (int k = threadIdx.x; k < np; k += blockDim.x) {
+      const int i0 = r.x + 2 * k;
+      const bool two = i0 + 1 < r.y;
+      const int2 e0 = entries_b[i0];
+      const int2 e1 = two ? entries_b[i0 + 1] : make_int2(-1, e0.y);
+      const uint8_t* row = flags + static_cast<int64_t>(b) * nt;
+      const int kept = (row[e0.x] == 1 ? 1 : 0) | (two && row[e1.x] == 1 ? 2 : 0);
+      pair_desc[out0 + k] = make_int4(b, e0.x, e1.x, kept);
+      pair_slot[out0 + k] = make_int2(e0.y - slot_base, e1.y - slot_base);
+    }
+  }
 }
 
 __global__ void plan_finish_kernel(const int* __restrict__ kept_total, int64_t total, int64_t* __restrict__ filtered) {
@@ -217,7 +250,12 @@ cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float
     note_launches(1);
     chunk_plan_kernel<<<(P.nchunks + 256) / 256, 256, 0, s>>>(nt, P.chunk_vt, P.nchunks, P.chunk_t);
     note_launches(1);
-    pair_plan_kernel<<<P.nchunks, 1024, 0, s>>>(P.entries_b, P.offsets_b, nb, P.chunk_t, P.pair_off);
+    pair_plan_kernel<<<P.nchunks, 1024, 0, s>>>(P.entries_b, P.offsets_b, nb, P.chunk_t, P.pair_off, P.rb_range);
+    note_launches(1);
+    const int64_t cbs = static_cast<int64_t>(nb) * P.nchunks;
+    const int grid_p = static_cast<int>(cbs < (int64_t(1) << 20) ? cbs : (int64_t(1) << 20));
+    pair_fill_kernel<<<grid_p, 32, 0, s>>>(P.entries_b, P.flags, nb, nt, P.nchunks, P.chunk_t, P.offsets_t,
+                                           P.rb_range, P.pair_off, P.pair_cap, P.pair_desc, P.pair_slot);
     note_launches(1);
   }
   plan_finish_kernel<<<1, 1, 0, s>>>(P.kept_total, static_cast<int64_t>(nb) * nt, filtered_tiles);

@@ -61,22 +61,24 @@ struct BwdPlan {
   int* chunk_t;     // [nchunks + 1]: first vocabulary tile of each chunk
   int* pair_off;    // [nchunks * (nb + 1)]: per chunk, prefix sums over row blocks of the number of
                     // pairs of consecutive listed tiles of that row block inside the chunk
+  int2* rb_range;   // [nchunks * nb]: entries [lo, hi) of each row block inside each chunk
+  int64_t pair_cap; // pairs a chunk can hold: nb * ceil(chunk_vt / 2)
+  int4* pair_desc;  // [nchunks * pair_cap]: (b, t0, t1 or -1, kept bits)
+  int2* pair_slot;  // [nchunks * pair_cap]: gradient-tile slots of t0 and t1, relative to the chunk
 };
 
 struct BwdGradTiles {
   CUtensorMap tmE, tmC;  // bf16, box 64 x 128
-  int nb, nt;
-  const uint8_t* flags;
-  const int2* entries_b;
-  const int* offsets_b;
-  const int* pair_off;   // of this chunk: [nb + 1]
-  const int* chunk_t;
+  int nb;
+  const int* pair_off;    // [nchunks * (nb + 1)]; entry nb of a chunk is its number of pairs
+  int64_t pair_cap;
+  const int4* pair_desc;  // [nchunks * pair_cap]
+  const int2* pair_slot;  // [nchunks * pair_cap]
   int N, D, V;
   const float* lse;
   const float* scale;
   const int64_t* targets;
   int64_t ignore_index;
-  const int* offsets_t;
   uint8_t* gscratch;
   int num_sms;
   int* err;
@@ -91,7 +93,7 @@ struct BwdGemm {
   const int2* entries_t;
   const int* offsets_t;
   const int2* entries_b;
-  const int* offsets_b;
+  const int2* rb_range;  // [nchunks * nb]
   const uint8_t* gscratch;
   const int* chunk_t;
   int dC_bf16;
