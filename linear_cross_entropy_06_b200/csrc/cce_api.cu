@@ -92,14 +92,17 @@ FwdWs carve_fwd(const cce_problem* p, void* base) {
   return w;
 }
 
-// Workspace of the split backward: the tile plan, the gradient tiles of one vocabulary chunk and
-// the fp32 dE accumulator. dC needs no accumulator: each vocabulary tile's rows are summed in TMEM
-// and written once.
+// Workspace of the backward: the tile plan and work lists, the queue counters, two gradient-tile
+// buffers (one vocabulary chunk each) and the fp32 dE accumulator. dC needs no accumulator: each
+// vocabulary tile's rows are summed in TMEM and written once.
 struct SplitWs {
   WsHeader* hdr;
   float* scale;
   cce::BwdPlan plan;
-  uint8_t* gscratch;
+  int* sync;         // [1 + nchunks * nb + nt + nchunks]: queue position, then the counters
+  size_t sync_bytes;
+  uint8_t* gscratch; // 2 * buf_bytes
+  size_t buf_bytes;
   float* dE_acc;
   size_t bytes;
 };
@@ -129,12 +132,12 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.entries_b = reinterpret_cast<int2*>(take(sizeof(int2) * static_cast<size_t>(tiles)));
   w.plan.kept_total = reinterpret_cast<int*>(take(sizeof(int)));
   // A chunk spans at most kChunkCBytes of C (its C rows stay in L2 while they are re-read for
-  // every listed row block), and its gradient tiles, at most nb per vocabulary tile, fit in
-  // kGradScratchBudget; at least one vocabulary tile per chunk.
+  // every listed row block), and the gradient tiles of two chunks, at most nb per vocabulary tile,
+  // fit in kGradScratchBudget; at least one vocabulary tile per chunk.
   const int64_t vt_bytes = static_cast<int64_t>(cce::kBwdBN) * p->D * 2;
   const int64_t per_vtile = std::max<int64_t>(nb, 1) * cce::kGradTileBytes;
   const int64_t chunk_vt = std::max<int64_t>(
-      1, std::min({nt, cce::kChunkCBytes / vt_bytes, cce::kGradScratchBudget / per_vtile}));
+      1, std::min({nt, cce::kChunkCBytes / vt_bytes, cce::kGradScratchBudget / 2 / per_vtile}));
   w.plan.chunk_vt = static_cast<int>(chunk_vt);
   w.plan.nchunks = static_cast<int>(ceil_div(nt, chunk_vt));
   w.plan.chunk_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks + 1)));
@@ -144,7 +147,13 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   const size_t pairs = static_cast<size_t>(w.plan.nchunks) * static_cast<size_t>(w.plan.pair_cap);
   w.plan.pair_desc = reinterpret_cast<int4*>(take(sizeof(int4) * pairs));
   w.plan.pair_slot = reinterpret_cast<int2*>(take(sizeof(int2) * pairs));
-  w.gscratch = reinterpret_cast<uint8_t*>(take(static_cast<size_t>(nb * chunk_vt) * cce::kGradTileBytes));
+  w.plan.S = static_cast<int>(ceil_div(p->D, cce::kGemmSlice));
+  w.plan.grp_size = reinterpret_cast<int*>(take(sizeof(int) * 2 * static_cast<size_t>(w.plan.nchunks)));
+  w.plan.grp_start = reinterpret_cast<int*>(take(sizeof(int) * (2 * static_cast<size_t>(w.plan.nchunks) + 1)));
+  w.sync_bytes = sizeof(int) * static_cast<size_t>(1 + w.plan.nchunks * nb + nt + w.plan.nchunks);
+  w.sync = reinterpret_cast<int*>(take(w.sync_bytes));
+  w.buf_bytes = static_cast<size_t>(nb * chunk_vt) * cce::kGradTileBytes;
+  w.gscratch = reinterpret_cast<uint8_t*>(take(2 * w.buf_bytes));
   if (!out_fp32) w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
   w.bytes = off;
   return w;
@@ -218,8 +227,8 @@ uint64_t wait_timeout_ns() {
     if (s_ != CCE_OK) return s_;   \
   } while (0)
 
-// The split backward (see cce_bwd_g.cu and cce_bwd_gemm.cu): plan the tiles, then per vocabulary
-// chunk form the gradient tiles and run the dC and dE MMAs from them.
+// The backward: plan the tiles and work lists, then one persistent launch (cce_bwd.cu) forms the
+// gradient tiles chunk by chunk and runs the dC and dE MMAs from them.
 cce_status backward_split(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
                           const float* lse, const float* tile_max, const int64_t* count, const float* grad_out,
                           float filter_eps, void* dE, void* dC, int32_t out_fp32, int64_t* filtered_tiles,
@@ -243,53 +252,51 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   CCE_TRY(cce::launch_bwd_plan(w.plan, tile_max, lse, targets, N, V, T, p->ignore_index, filter_eps, filtered_tiles,
                                s));
   CCE_TRY(cce::launch_fill_zero(dE_acc, N * D * 4, s));
+  CCE_TRY(cudaMemsetAsync(w.sync, 0, w.sync_bytes, s));
 
-  cce::BwdGradTiles G{};
-  CCE_CHECK(make_map(&G.tmE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kBwdBM));
-  CCE_CHECK(make_map(&G.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, cce::kBwdBN));
-  G.N = static_cast<int>(N);
-  G.D = static_cast<int>(D);
-  G.V = static_cast<int>(V);
-  G.lse = lse;
-  G.scale = w.scale;
-  G.targets = targets;
-  G.ignore_index = p->ignore_index;
-  G.nb = w.plan.nb;
-  G.pair_off = w.plan.pair_off;
-  G.pair_cap = w.plan.pair_cap;
-  G.pair_desc = w.plan.pair_desc;
-  G.pair_slot = w.plan.pair_slot;
-  G.gscratch = w.gscratch;
-  G.num_sms = num_sms;
-  G.err = &w.hdr->err;
-  G.timeout_ns = wait_timeout_ns();
-
-  cce::BwdGemm M{};
-  CCE_CHECK(make_map(&M.tmE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, 64));
-  CCE_CHECK(make_map(&M.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, 64));
-  CCE_CHECK(make_map(&M.tmdE, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dE_acc, N, D, 32, 32));
-  if (out_fp32) CCE_CHECK(make_map(&M.tmdC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dC, V, D, 32, 32));
-  else CCE_CHECK(make_map(&M.tmdC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dC, V, D, 64, 32));
-  M.N = G.N;
-  M.D = G.D;
-  M.V = G.V;
-  M.nb = w.plan.nb;
-  M.entries_t = w.plan.entries_t;
-  M.offsets_t = w.plan.offsets_t;
-  M.entries_b = w.plan.entries_b;
-  M.rb_range = w.plan.rb_range;
-  M.gscratch = w.gscratch;
-  M.chunk_t = w.plan.chunk_t;
-  M.dC_bf16 = out_fp32 ? 0 : 1;
-  M.num_sms = num_sms;
-  M.err = G.err;
-  M.timeout_ns = G.timeout_ns;
+  cce::BwdLaunch L{};
+  CCE_CHECK(make_map(&L.tmE128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kBwdBM));
+  CCE_CHECK(make_map(&L.tmC128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, cce::kBwdBN));
+  CCE_CHECK(make_map(&L.tmE64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, 64));
+  CCE_CHECK(make_map(&L.tmC64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, 64));
+  CCE_CHECK(make_map(&L.tmdE, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dE_acc, N, D, 32, 32));
+  if (out_fp32) CCE_CHECK(make_map(&L.tmdC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dC, V, D, 32, 32));
+  else CCE_CHECK(make_map(&L.tmdC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dC, V, D, 64, 32));
+  cce::BwdArgs& A = L.args;
+  A.N = static_cast<int>(N);
+  A.D = static_cast<int>(D);
+  A.V = static_cast<int>(V);
+  A.nb = w.plan.nb;
+  A.nt = w.plan.nt;
+  A.S = w.plan.S;
+  A.nchunks = w.plan.nchunks;
+  A.out_bf16 = out_fp32 ? 0 : 1;
+  A.ignore_index = p->ignore_index;
+  A.pair_cap = w.plan.pair_cap;
+  A.buf_bytes = w.buf_bytes;
+  A.lse = lse;
+  A.scale = w.scale;
+  A.targets = targets;
+  A.grp_start = w.plan.grp_start;
+  A.chunk_t = w.plan.chunk_t;
+  A.pair_desc = w.plan.pair_desc;
+  A.pair_slot = w.plan.pair_slot;
+  A.rb_range = w.plan.rb_range;
+  A.offsets_t = w.plan.offsets_t;
+  A.entries_t = w.plan.entries_t;
+  A.entries_b = w.plan.entries_b;
+  A.gscratch = w.gscratch;
+  A.qctr = w.sync;
+  A.counters = w.sync + 1;
+  A.ctr_g_b = 0;
+  A.ctr_g_t = w.plan.nchunks * w.plan.nb;
+  A.ctr_b_done = A.ctr_g_t + w.plan.nt;
+  A.err = &w.hdr->err;
+  A.timeout_ns = wait_timeout_ns();
+  L.num_sms = num_sms;
 
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
-  for (int c = 0; c < w.plan.nchunks; ++c) {
-    CCE_TRY(cce::launch_bwd_g(G, c, s));
-    CCE_TRY(cce::launch_bwd_gemm(M, c, s));
-  }
+  CCE_TRY(cce::launch_bwd(L, s));
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
   if (!out_fp32) CCE_TRY(cce::launch_to_bf16(dE_acc, static_cast<__nv_bfloat16*>(dE), N * D, s));
   return CCE_OK;

@@ -1,0 +1,617 @@
+// Backward: one persistent launch that recomputes the kept logit tiles, forms their bf16 gradient
+// tiles, and runs the dC and dE MMAs on them, chunk by chunk of the vocabulary.
+//
+// mlx-cross-entropy README, "How it works" items 2 and 3 (recompute from the saved LSE, skip tiles
+// whose softmax is below 2^-12, accumulate the gradients without [batch, tiles, D] buffers); Loss
+// functions explainer, "How it works" item 2 (G = p - y, dE = G C, dC = G^T E); Cut Your Losses
+// abstract (logits are recomputed blockwise and never stored).
+//
+// Work items, per vocabulary chunk c (its gradient tiles live in scratch buffer c mod 2):
+//   pair   two consecutive listed 128 x 128 tiles (b, t0), (b, t1) of row block b in the chunk:
+//          S = E_b [C_t0; C_t1]^T (tcgen05 M=128 N=256 K=D; skipped for onehot-only tiles), then
+//          G = scale_r * exp(S - LSE_r) - scale_r * [v = t_r] in fp32, rounded to bf16 into a
+//          128B-swizzled shared tile, one 32 KB bulk store per tile into the scratch buffer.
+//   dE     (row block b, 256-column slice s of D): sum over the chunk's listed t of G_bt C_t[:, s]
+//          in TMEM, then one fp32 TMA reduce-add into dE_acc (split-reduce over chunks).
+//   dC     (vocabulary tile t, slice s): sum over the listed b of G_bt^T E_b[:, s] in TMEM (A = the
+//          same G tile read MN-major), written once by TMA store: every listed tile of t lies in
+//          t's chunk, so dC needs no reduction.
+//
+// Scheduling: a global queue holds the items in the order pairs(0), dE/dC(0), pairs(1), dE/dC(1),
+// ...; CTAs claim them one at a time with an atomic counter, so a claimed item always belongs to a
+// running CTA. Dependencies point only to earlier items:
+//   a dE item waits until every gradient tile of its row block in the chunk is stored, a dC item
+//   until every gradient tile of its vocabulary tile is, and a pair of chunk c waits, before it
+//   stores, until every dE/dC item of chunk c - 2 (the previous user of the buffer) has read it.
+// Every such wait is bounded. Because items are claimed in order and the smallest unfinished item
+// has no unfinished dependency, the queue always drains; and with no boundary between chunks the
+// machine has a single tail per backward instead of one per chunk and kernel.
+//
+// Design (B200): one CTA per SM, 7 warps, 224 KB of shared memory.
+//   warp 0      producer: per stage (48 KB, 4 deep) either E_b, C_t0, C_t1 K-blocks of 64 (pair), or
+//               one K-half of a gradient tile (16 KB bulk copy) and the 64 x 256 operand slice
+//               (four TMA boxes of 64 x 64) (dE, dC).
+//   warp 1      TMEM owner (two 256-column fp32 buffers); one lane issues tcgen05.mma M=128 N=256.
+//   warps 2..5  write-out: G formation and bulk stores (pair), or TMEM -> swizzled staging -> TMA
+//               store / reduce-add (dC / dE), while the MMA fills the other TMEM buffer.
+//   warp 6      scheduler: claims and decodes items into an 8-deep shared ring.
+#include "cce_device.cuh"
+#include "cce_internal.h"
+
+namespace cce {
+namespace {
+
+constexpr int BM = kBwdBM;
+constexpr int BN = kBwdBN;
+constexpr int BK = 64;
+constexpr int SLICE = kGemmSlice;
+constexpr int STAGES = 4;
+constexpr int PART = 16384;              // 128 x 64 bf16: one K-block of 128 rows, or half a G tile
+constexpr int X_BOX = 8192;              // 64 x 64 bf16
+constexpr int STAGE_BYTES = 3 * PART;    // 48 KB
+constexpr int TILE_BYTES = kGradTileBytes;
+constexpr int REGION_BYTES = TILE_BYTES;  // one G tile (pair) or 4 x 8 KB staging (dE / dC)
+constexpr int STG_WARP = 8192;
+constexpr int RING = 8;
+constexpr int NUM_THREADS = 224;
+constexpr int TMEM_COLS = 512;
+
+enum Kind : int { kPair = 0, kDE = 1, kDC = 2, kEnd = 3 };
+
+// A decoded work item, written by the scheduler into the shared ring (16-byte aligned: it is
+// copied as int4).
+struct alignas(16) WorkItem {
+  int kind;
+  int chunk;
+  int key;         // pair, dE: row block b; dC: vocabulary tile t
+  int s;           // dE, dC: slice of D; pair: kept bits (1 first tile, 2 second tile)
+  int begin, end;  // dE, dC: list entries; pair: vocabulary tiles t0 and t1 (-1 when absent)
+  int slot0;       // pair: slot of t0 in the chunk's buffer; dE, dC: the chunk's first slot
+  int slot1;       // pair: slot of t1
+  int dep_idx;     // counter this item waits on (-1: none): before its loads (dE, dC) or stores (pair)
+  int dep_val;     // value the counter must reach
+  int pad[6];
+};
+static_assert(sizeof(WorkItem) == 64, "ring entries are 64 bytes");
+
+enum Bar : int {
+  kFull = 0,
+  kEmpty = kFull + STAGES,
+  kAccFull = kEmpty + STAGES,
+  kAccEmpty = kAccFull + 2,
+  kDrain = kAccEmpty + 2,
+  kRegion = kDrain + 1,  // the shared write-out region is free (one arrival per write-out warp)
+  kGReady = kRegion + 1, // all 128 rows of a G tile are in the region
+  kItemFull = kGReady + 1,
+  kItemEmpty = kItemFull + RING,
+  kItemTaken = kItemEmpty + RING,  // the producer has started the entry's item
+  kNumBars = kItemTaken + RING
+};
+
+// The scheduler claims item k only once the producer has started item k - LOOKAHEAD: enough to
+// hide the claim and decode latency, few enough that no CTA hoards claimed items at the end.
+constexpr uint32_t LOOKAHEAD = 2;
+
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + REGION_BYTES + kNumBars * 8 + RING * 64 + 16;
+static_assert(SMEM_BYTES <= 232448, "fits the 227 KB opt-in shared memory of an SM");
+
+constexpr uint32_t IDESC_S = idesc_bf16(BM, 2 * BN, false, false);  // S = E_b [C_t0; C_t1]^T
+constexpr uint32_t IDESC_DC = idesc_bf16(BN, SLICE, true, true);    // M = vocabulary (G^T, MN-major)
+constexpr uint32_t IDESC_DE = idesc_bf16(BM, SLICE, false, true);   // M = rows (G, K-major)
+
+// Consumers of one ring entry: producer lane, MMA lane, one lane per write-out warp.
+constexpr uint32_t kRingConsumers = 1 + 1 + 4;
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(src), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map), "r"(src),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
+__device__ __forceinline__ void read_item(const WorkItem* ring, int idx, WorkItem& it) {
+  const int4* src = reinterpret_cast<const int4*>(ring + idx);
+  int4* dst = reinterpret_cast<int4*>(&it);
+#pragma unroll
+  for (int i = 0; i < 3; ++i) dst[i] = src[i];
+}
+
+// Item w of the queue, in group g (2c: pairs of chunk c; 2c + 1: dE / dC items of chunk c) that
+// starts at item g_begin -> its decoded form (the scheduler's only global reads).
+__device__ __forceinline__ void decode_item(int w, int g, int g_begin, const BwdArgs& A, WorkItem& it) {
+  const int c = g >> 1, local = w - g_begin;
+  const int t_begin = A.chunk_t[c];
+  it.chunk = c;
+  if ((g & 1) == 0) {
+    const int64_t pi = static_cast<int64_t>(c) * A.pair_cap + local;
+    const int4 d = A.pair_desc[pi];
+    const int2 sl = A.pair_slot[pi];
+    it.kind = kPair;
+    it.key = d.x;
+    it.begin = d.y;
+    it.end = d.z;
+    it.s = d.w;
+    it.slot0 = sl.x;
+    it.slot1 = sl.y;
+    if (c >= 2) {  // the buffer's previous chunk must have been read by all of its dE / dC items
+      it.dep_idx = A.ctr_b_done + (c - 2);
+      it.dep_val = A.grp_start[2 * (c - 2) + 2] - A.grp_start[2 * (c - 2) + 1];
+    } else {
+      it.dep_idx = -1;
+      it.dep_val = 0;
+    }
+  } else {
+    const int S = A.S;
+    it.slot0 = A.offsets_t[t_begin];
+    it.slot1 = 0;
+    if (local < A.nb * S) {
+      it.kind = kDE;
+      it.key = local / S;
+      it.s = local % S;
+      const int2 r = A.rb_range[static_cast<int64_t>(c) * A.nb + it.key];
+      it.begin = r.x;
+      it.end = r.y;
+      it.dep_idx = A.ctr_g_b + c * A.nb + it.key;
+    } else {
+      const int v = local - A.nb * S;
+      it.kind = kDC;
+      it.key = t_begin + v / S;
+      it.s = v % S;
+      it.begin = A.offsets_t[it.key];
+      it.end = A.offsets_t[it.key + 1];
+      it.dep_idx = A.ctr_g_t + it.key;
+    }
+    it.dep_val = it.end - it.begin;
+  }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmE128, const __grid_constant__ CUtensorMap tmC128,
+               const __grid_constant__ CUtensorMap tmE64, const __grid_constant__ CUtensorMap tmC64,
+               const __grid_constant__ CUtensorMap tmdC, const __grid_constant__ CUtensorMap tmdE,
+               const __grid_constant__ BwdArgs A) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = base;
+  uint8_t* region = base + STAGES * STAGE_BYTES;
+  WorkItem* ring = reinterpret_cast<WorkItem*>(region + REGION_BYTES);  // 1024-byte aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + RING);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar0 = smem_u32(bars);
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+
+  if (threadIdx.x == 0) {
+    for (int u = 0; u < STAGES; ++u) {
+      mbar_init(bar(kFull + u), 1);
+      mbar_init(bar(kEmpty + u), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar(kAccFull + a), 1);
+      mbar_init(bar(kAccEmpty + a), 128);
+    }
+    mbar_init(bar(kDrain), 1);
+    mbar_init(bar(kRegion), 4);
+    mbar_init(bar(kGReady), 128);
+    for (int i = 0; i < RING; ++i) {
+      mbar_init(bar(kItemFull + i), 1);
+      mbar_init(bar(kItemEmpty + i), kRingConsumers);
+      mbar_init(bar(kItemTaken + i), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const WaitCtl wc{abort_flag, A.err, A.timeout_ns};
+  const int num_kb = (A.D + BK - 1) / BK;
+  auto buffer = [&](int chunk) { return A.gscratch + static_cast<size_t>(chunk & 1) * A.buf_bytes; };
+
+  if (warp == 6) {
+    // ---------------- scheduler ----------------
+    if (lane == 0) {
+      const int total = A.grp_start[2 * A.nchunks];
+      int g = 0, g_begin = 0, g_end = A.grp_start[1];  // this CTA's claims only increase
+      for (uint32_t k = 0;; ++k) {
+        const int idx = static_cast<int>(k % RING);
+        if (!mbar_wait(bar(kItemEmpty + idx), ((k / RING) & 1u) ^ 1u, wc)) break;
+        if (k >= LOOKAHEAD) {
+          const uint32_t j = k - LOOKAHEAD;
+          if (!mbar_wait(bar(kItemTaken + j % RING), (j / RING) & 1u, wc)) break;
+        }
+        const int w = atomicAdd(A.qctr, 1);
+        WorkItem it;
+        if (w >= total) {
+          it.kind = kEnd;
+        } else {
+          while (w >= g_end) {
+            ++g;
+            g_begin = g_end;
+            g_end = A.grp_start[g + 1];
+          }
+          decode_item(w, g, g_begin, A, it);
+        }
+        int4* dst = reinterpret_cast<int4*>(ring + idx);
+        const int4* src = reinterpret_cast<const int4*>(&it);
+#pragma unroll
+        for (int i = 0; i < 3; ++i) dst[i] = src[i];
+        mbar_arrive(bar(kItemFull + idx));  // release: the entry is visible to the waiters
+        if (it.kind == kEnd) break;
+      }
+    }
+  } else if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued[STAGES] = {0, 0, 0, 0};
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int idx = static_cast<int>(k % RING);
+        if (!mbar_wait(bar(kItemFull + idx), (k / RING) & 1u, wc)) break;
+        WorkItem it;
+        read_item(ring, idx, it);
+        mbar_arrive(bar(kItemEmpty + idx));
+        mbar_arrive(bar(kItemTaken + idx));
+        if (it.kind == kEnd) break;
+        if (it.kind == kPair) {
+          if (it.s == 0) continue;  // onehot-only tiles need no recompute
+          const int rb = it.key * BM;
+          const int vb0 = it.begin * BN, vb1 = (it.end >= 0 ? it.end : it.begin) * BN;
+          for (int kb = 0; kb < num_kb; ++kb) {
+            if (!mbar_wait(bar(kEmpty + stage), phase ^ 1u, wc)) {
+              ok = false;
+              break;
+            }
+            const uint32_t dst = smem_u32(stages + stage * STAGE_BYTES);
+            mbar_arrive_expect_tx(bar(kFull + stage), STAGE_BYTES);
+            tma_load_2d(dst, &tmE128, bar(kFull + stage), kb * BK, rb);
+            tma_load_2d(dst + PART, &tmC128, bar(kFull + stage), kb * BK, vb0);
+            tma_load_2d(dst + 2 * PART, &tmC128, bar(kFull + stage), kb * BK, vb1);
+            ++issued[stage];
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          continue;
+        }
+        // dE / dC: every gradient tile this item reads must be stored
+        if (it.begin < it.end && !wait_counter(A.counters + it.dep_idx, it.dep_val, wc)) break;
+        const bool de = it.kind == kDE;
+        const uint8_t* buf = buffer(it.chunk);
+        const int x0 = it.s * SLICE;
+        auto entry = [&](int i) {  // (tile index of the other operand, slot in the chunk's buffer)
+          if (de) {
+            const int2 en = A.entries_b[i];
+            return make_int2(en.x, en.y - it.slot0);
+          }
+          return make_int2(A.entries_t[i].x >> 2, i - it.slot0);
+        };
+        int2 os_next = it.begin < it.end ? entry(it.begin) : make_int2(0, 0);
+        for (int i = it.begin; i < it.end && ok; ++i) {
+          const int2 os = os_next;
+          if (i + 1 < it.end) os_next = entry(i + 1);
+          const uint8_t* tile = buf + static_cast<size_t>(os.y) * TILE_BYTES;
+          for (int h = 0; h < 2; ++h) {  // K-halves: 64 vocabulary columns (dE) or 64 rows (dC)
+            if (!mbar_wait(bar(kEmpty + stage), phase ^ 1u, wc)) {
+              ok = false;
+              break;
+            }
+            const uint32_t dst = smem_u32(stages + stage * STAGE_BYTES);
+            mbar_arrive_expect_tx(bar(kFull + stage), STAGE_BYTES);
+            if (de) {  // G block h: rows 0..127, vocabulary 64h .. 64h + 63 (K-major A)
+              bulk_load(dst, tile + h * PART, PART, bar(kFull + stage));
+            } else {   // rows 64h .. 64h + 63 of both 64-column blocks (MN-major A = G^T)
+              bulk_load(dst, tile + h * (PART / 2), PART / 2, bar(kFull + stage));
+              bulk_load(dst + PART / 2, tile + PART + h * (PART / 2), PART / 2, bar(kFull + stage));
+            }
+            const int y = os.x * BM + 64 * h;  // K rows of the operand: C_t rows (dE), E_b rows (dC)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              tma_load_2d(dst + PART + c * X_BOX, de ? &tmC64 : &tmE64, bar(kFull + stage), x0 + 64 * c, y);
+            ++issued[stage];
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+      if (*abort_flag) {
+        for (int u = 0; u < STAGES; ++u)
+          if (issued[u]) mbar_wait_drain(bar(kFull + u), (issued[u] - 1u) & 1u, 200000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc_iter = 0;
+      bool ok = true, issued_any = false;
+      for (uint32_t k = 0; ok; ++k) {
+        const int idx = static_cast<int>(k % RING);
+        if (!mbar_wait(bar(kItemFull + idx), (k / RING) & 1u, wc)) break;
+        WorkItem it;
+        read_item(ring, idx, it);
+        mbar_arrive(bar(kItemEmpty + idx));
+        if (it.kind == kEnd) break;
+        const bool pair = it.kind == kPair;
+        if (pair ? it.s == 0 : it.begin == it.end) continue;  // no MMA for this item
+        const int a = acc_iter & 1;
+        if (!mbar_wait(bar(kAccEmpty + a), ((acc_iter >> 1) & 1u) ^ 1u, wc)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(a * 2 * BN);
+        const int nstage = pair ? num_kb : 2 * (it.end - it.begin);
+        const uint32_t idesc = pair ? IDESC_S : (it.kind == kDE ? IDESC_DE : IDESC_DC);
+        for (int j = 0; j < nstage; ++j) {
+          if (!mbar_wait(bar(kFull + stage), phase, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t s0 = smem_u32(stages + stage * STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // 16 of the stage's 64 K values per MMA
+            uint64_t adesc, bdesc;
+            if (pair) {  // A = E_b K-block, B = C_t0 and C_t1 rows (256 rows of 128 bytes, contiguous)
+              adesc = sdesc_sw128(s0 + 32u * kk, 16, 1024);
+              bdesc = sdesc_sw128(s0 + PART + 32u * kk, 16, 1024);
+            } else {
+              adesc = it.kind == kDE ? sdesc_sw128(s0 + 32u * kk, 16, 1024)
+                                     : sdesc_sw128(s0 + 2048u * kk, PART / 2, 1024);
+              bdesc = sdesc_sw128(s0 + PART + 2048u * kk, X_BOX, 1024);
+            }
+            tc_mma_bf16(d, adesc, bdesc, idesc, (j | kk) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          tc_commit(bar(kEmpty + stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(bar(kAccFull + a));
+        ++acc_iter;
+      }
+      if (*abort_flag && issued_any) {
+        tc_commit(bar(kDrain));
+        mbar_wait_drain(bar(kDrain), 0, 200000000ull);
+      }
+    }
+  } else {
+    // ---------------- write-out ----------------
+    const int q = warp & 3;  // TMEM lane quarter of this warp (warps 2..5 -> 2, 3, 0, 1)
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const bool leader = (warp == 2 && lane == 0);
+    const uint32_t reg0 = smem_u32(region);
+    const uint32_t stg = reg0 + static_cast<uint32_t>(q * STG_WARP);
+    uint32_t acc_iter = 0, rphase = 0, gphase = 0;
+    bool ok = true;
+    // Every lane waits (and acquires) itself; the vote makes the outcome warp-uniform, so the warp
+    // stays converged for the .sync.aligned TMEM loads and takes one branch on failure.
+    auto warp_wait = [&](uint32_t b, uint32_t parity) {
+      const bool r = mbar_wait(b, parity, wc);
+      return __all_sync(0xffffffffu, r ? 1 : 0) != 0;
+    };
+    // Every write-out warp's earlier bulk copies have read the region; then it may be rewritten.
+    auto region_free = [&]() {
+      if (lane == 0) {
+        bulk_wait_group_read0();
+        mbar_arrive(bar(kRegion));
+      }
+      const bool r = warp_wait(bar(kRegion), rphase & 1u);
+      ++rphase;
+      return r;
+    };
+    for (uint32_t k = 0; ok; ++k) {
+      const int idx = static_cast<int>(k % RING);
+      if (!warp_wait(bar(kItemFull + idx), (k / RING) & 1u)) break;
+      WorkItem it;
+      read_item(ring, idx, it);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kItemEmpty + idx));
+      if (it.kind == kEnd) break;
+      const int a = acc_iter & 1;
+
+      if (it.kind == kPair) {
+        const int b = it.key;
+        const int r = b * BM + row;
+        const float lse_l2 = (r < A.N) ? A.lse[r] * kLog2e : 0.f;
+        const float sc = (r < A.N) ? A.scale[r] : 0.f;
+        const int64_t tg = (r < A.N) ? A.targets[r] : A.ignore_index;
+        const bool tvalid = tg != A.ignore_index && tg >= 0 && tg < A.V;
+        const bool mma = it.s != 0;
+        if (mma) {
+          if (!warp_wait(bar(kAccFull + a), (acc_iter >> 1) & 1u)) break;
+          tc_fence_after();
+        }
+        // the chunk's buffer must no longer be read by the dE / dC items of chunk - 2
+        if (leader && it.dep_idx >= 0 && !wait_counter(A.counters + it.dep_idx, it.dep_val, wc)) ok = false;
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        uint8_t* buf = buffer(it.chunk);
+        const int ntiles = it.end >= 0 ? 2 : 1;
+        for (int u = 0; u < ntiles && ok; ++u) {
+          const int t = u == 0 ? it.begin : it.end;
+          const bool kept = (it.s >> u) & 1;
+          const int vb = t * BN;
+          const int64_t rel = tg - vb;
+          const int tcol = (tvalid && rel >= 0 && rel < BN) ? static_cast<int>(rel) : -1;  // -scale_r here
+          if (!region_free()) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            if (kept) {
+              tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * 2 * BN + u * BN + c * 32), v);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = sc * exp2f(fmaf(v[e], kLog2e, -lse_l2));
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = 0.f;
+            }
+            const int col0 = vb + c * 32;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (c * 32 + e == tcol) v[e] -= sc;
+              if (col0 + e >= A.V) v[e] = 0.f;
+            }
+            const uint32_t blk = reg0 + static_cast<uint32_t>((c >> 1) * PART);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const int ch = (c & 1) * 4 + h;
+              st_shared_v4(blk + swz(row, ch), pack_bf16x2(v[8 * h + 0], v[8 * h + 1]),
+                           pack_bf16x2(v[8 * h + 2], v[8 * h + 3]), pack_bf16x2(v[8 * h + 4], v[8 * h + 5]),
+                           pack_bf16x2(v[8 * h + 6], v[8 * h + 7]));
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(bar(kGReady));
+          if (warp == 2) {
+            if (!warp_wait(bar(kGReady), gphase & 1u)) {
+              ok = false;
+            } else if (leader) {
+              bulk_store(buf + static_cast<size_t>(u == 0 ? it.slot0 : it.slot1) * TILE_BYTES, reg0, TILE_BYTES);
+              bulk_commit_group();
+            }
+          }
+          ++gphase;
+        }
+        if (mma) {
+          tc_fence_before();
+          mbar_arrive(bar(kAccEmpty + a));
+          ++acc_iter;
+        }
+        // publish the pair's tiles to the dE / dC items that wait for them
+        if (leader && ok) {
+          bulk_wait_group0();
+          fence_proxy_async_global();
+          red_release_add(A.counters + A.ctr_g_b + it.chunk * A.nb + b, ntiles);
+          red_release_add(A.counters + A.ctr_g_t + it.begin, 1);
+          if (it.end >= 0) red_release_add(A.counters + A.ctr_g_t + it.end, 1);
+        }
+        __syncwarp();
+        if (*abort_flag) ok = false;
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        continue;
+      }
+
+      // dE / dC
+      const bool de = it.kind == kDE;
+      const bool has = it.begin < it.end;
+      if (has) {
+        if (!warp_wait(bar(kAccFull + a), (acc_iter >> 1) & 1u)) break;
+        tc_fence_after();
+      }
+      // every gradient tile of this item has been read into shared memory (the MMAs are done)
+      if (leader) {
+        fence_proxy_async_global();
+        red_release_add(A.counters + A.ctr_b_done + it.chunk, 1);
+      }
+      if (de && !has) continue;  // nothing to add for this row block in this chunk
+      if (!region_free()) break;
+      const int rows_limit = de ? A.N : A.V;
+      const int y = it.key * BM + q * 32;
+      for (int p = 0; p < SLICE / 64; ++p) {
+        const int x = it.s * SLICE + 64 * p;
+        if (x >= A.D) break;
+        float v0[32], v1[32];
+        if (has) {
+          tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * SLICE + 64 * p), v0);
+          tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * SLICE + 64 * p + 32), v1);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v0[e] = v1[e] = 0.f;
+        }
+        // this warp's staging is free once its previous TMA op has read it
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+        if (!de && A.out_bf16) {
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            const float* src = h < 4 ? v0 + 8 * h : v1 + 8 * (h - 4);
+            st_shared_v4(stg + swz(lane, h), pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                         pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            st_shared_v4(stg + swz(lane, h), __float_as_uint(v0[4 * h]), __float_as_uint(v0[4 * h + 1]),
+                         __float_as_uint(v0[4 * h + 2]), __float_as_uint(v0[4 * h + 3]));
+            st_shared_v4(stg + 4096u + swz(lane, h), __float_as_uint(v1[4 * h]), __float_as_uint(v1[4 * h + 1]),
+                         __float_as_uint(v1[4 * h + 2]), __float_as_uint(v1[4 * h + 3]));
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && y < rows_limit) {
+          if (!de && A.out_bf16) {
+            tma_store_2d(&tmdC, stg, x, y);
+          } else if (!de) {
+            tma_store_2d(&tmdC, stg, x, y);
+            if (x + 32 < A.D) tma_store_2d(&tmdC, stg + 4096u, x + 32, y);
+          } else {
+            tma_reduce_add_2d(&tmdE, stg, x, y);
+            if (x + 32 < A.D) tma_reduce_add_2d(&tmdE, stg + 4096u, x + 32, y);
+          }
+          bulk_commit_group();
+        }
+      }
+      if (has) {
+        tc_fence_before();
+        mbar_arrive(bar(kAccEmpty + a));
+        ++acc_iter;
+      }
+    }
+    // every store and reduce-add must be complete before the kernel ends
+    if (lane == 0) bulk_wait_group0();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const BwdLaunch& L, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  bwd_kernel<<<L.num_sms, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE128, L.tmC128, L.tmE64, L.tmC64, L.tmdC, L.tmdE, L.args);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace cce

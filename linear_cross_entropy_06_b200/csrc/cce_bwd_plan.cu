@@ -13,7 +13,7 @@
 //   each (b * 4 + flag, t), row blocks ascending. An entry's position is also its gradient-tile slot.
 // By row block (dE kernel): offsets_b[b] .. offsets_b[b+1] index entries_b, each (t, slot),
 //   vocabulary tiles ascending.
-// Per vocabulary chunk c, flat work lists the backward kernels read with one load per item:
+// Per vocabulary chunk c, flat work lists the backward kernel reads with one load per item:
 //   rb_range[c * nb + b]   the entries [lo, hi) of row block b inside the chunk;
 //   pair_desc/pair_slot    from c * pair_cap: the pairs of consecutive listed tiles of a row block
 //                          inside the chunk, row blocks ascending (pair_off[c] holds their prefix sums).
@@ -215,6 +215,16 @@ __global__ void pair_fill_kernel(const int2* __restrict__ entries_b, const uint8
   }
 }
 
+// Sizes of the backward's queue groups: group 2c holds the pairs of chunk c, group 2c + 1 its dE
+// items (nb * S) and dC items (one per vocabulary tile of the chunk and slice).
+__global__ void group_size_kernel(const int* __restrict__ pair_off, const int* __restrict__ chunk_t, int nb, int S,
+                                  int nchunks, int* __restrict__ grp_size) {
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < nchunks; c += gridDim.x * blockDim.x) {
+    grp_size[2 * c] = pair_off[static_cast<int64_t>(c) * (nb + 1) + nb];
+    grp_size[2 * c + 1] = (nb + chunk_t[c + 1] - chunk_t[c]) * S;
+  }
+}
+
 __global__ void plan_finish_kernel(const int* __restrict__ kept_total, int64_t total, int64_t* __restrict__ filtered) {
   *filtered = total - static_cast<int64_t>(*kept_total);
 }
@@ -256,6 +266,10 @@ cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float
     const int grid_p = static_cast<int>(cbs < (int64_t(1) << 20) ? cbs : (int64_t(1) << 20));
     pair_fill_kernel<<<grid_p, 32, 0, s>>>(P.entries_b, P.flags, nb, nt, P.nchunks, P.chunk_t, P.offsets_t,
                                            P.rb_range, P.pair_off, P.pair_cap, P.pair_desc, P.pair_slot);
+    note_launches(1);
+    group_size_kernel<<<(P.nchunks + 255) / 256, 256, 0, s>>>(P.pair_off, P.chunk_t, nb, P.S, P.nchunks, P.grp_size);
+    note_launches(1);
+    scan_kernel<<<1, 1024, 0, s>>>(P.grp_size, 2 * P.nchunks, P.grp_start);
     note_launches(1);
   }
   plan_finish_kernel<<<1, 1, 0, s>>>(P.kept_total, static_cast<int64_t>(nb) * nt, filtered_tiles);

@@ -98,6 +98,60 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, u
 }
 
 // ------------------------------------------------------------------------------------------------
+// Counters shared by the CTAs of one persistent kernel (release / acquire at GPU scope). Data that
+// one CTA writes with bulk copies (async proxy) and another reads with bulk copies is published as:
+// writer: bulk_wait_group0(); fence_proxy_async_global(); red_release_add(counter, n);
+// reader: wait_counter(counter, target) (acquire + proxy fence), then the bulk loads.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ int ld_relaxed(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Waits until *counter >= target (another CTA of the same grid raises it). Gives up when this
+// CTA was aborted, when any CTA recorded an error, or after the wait limit (then it aborts the
+// CTA and records kErrDeviceTimeout). Never spins without a bound.
+__device__ __forceinline__ bool wait_counter(const int* counter, int target, const WaitCtl& w) {
+  if (ld_acquire(counter) >= target) {
+    fence_proxy_async_global();
+    return true;
+  }
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    __nanosleep(128);
+    if (ld_acquire(counter) >= target) {
+      fence_proxy_async_global();
+      return true;
+    }
+    if (*w.abort) return false;
+    if (ld_relaxed(w.err) != 0) {
+      *w.abort = 1;
+      return false;
+    }
+    if (global_timer_ns() - t0 > w.timeout_ns) {
+      *w.abort = 1;
+      record_error(w.err, kErrDeviceTimeout);
+      return false;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor): tile loads into shared memory and reduce-adds into global memory.
 // Coordinates are in elements, innermost first. No multicast anywhere in this library.
 // ------------------------------------------------------------------------------------------------

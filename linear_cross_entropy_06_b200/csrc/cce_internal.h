@@ -35,14 +35,14 @@ void note_launches(int n);
 // Sets the message cce_last_error_message() returns on the calling thread.
 void set_last_error(const char* msg);
 
-// Split backward (cce_bwd_plan.cu, cce_bwd_g.cu, cce_bwd_gemm.cu).
+// Backward (cce_bwd_plan.cu: tile plan and work lists; cce_bwd.cu: the persistent kernel).
 constexpr int kGradTileBytes = kBwdBM * kBwdBN * 2;      // one bf16 gradient tile, 128B-swizzled
 constexpr int kGemmSlice = 256;                           // columns of D per dC/dE work item
 // A vocabulary chunk spans at most kChunkCBytes of C, so that the C rows of a chunk stay in L2
-// while the gradient-tile and dE kernels re-read them for every row block that lists them.
-constexpr int64_t kChunkCBytes = int64_t(128) << 20;
-// ... and its gradient tiles (at most one per listed row block and vocabulary tile) fit in a
-// fixed scratch of kGradScratchBudget.
+// while they are re-read for every row block that lists them ...
+constexpr int64_t kChunkCBytes = int64_t(64) << 20;
+// ... and the gradient tiles of two chunks (at most one per listed row block and vocabulary tile;
+// one chunk is written while the previous one is read) fit in a fixed kGradScratchBudget.
 constexpr int64_t kGradScratchBudget = int64_t(128) << 20;
 
 struct BwdPlan {
@@ -58,6 +58,7 @@ struct BwdPlan {
   int* kept_total;
   int chunk_vt;     // vocabulary tiles per chunk
   int nchunks;
+  int S;            // 256-column slices of D
   int* chunk_t;     // [nchunks + 1]: first vocabulary tile of each chunk
   int* pair_off;    // [nchunks * (nb + 1)]: per chunk, prefix sums over row blocks of the number of
                     // pairs of consecutive listed tiles of that row block inside the chunk
@@ -65,48 +66,50 @@ struct BwdPlan {
   int64_t pair_cap; // pairs a chunk can hold: nb * ceil(chunk_vt / 2)
   int4* pair_desc;  // [nchunks * pair_cap]: (b, t0, t1 or -1, kept bits)
   int2* pair_slot;  // [nchunks * pair_cap]: gradient-tile slots of t0 and t1, relative to the chunk
+  int* grp_size;    // [2 * nchunks]: work items of each queue group (pairs of chunk c, then its dE/dC)
+  int* grp_start;   // [2 * nchunks + 1]: their prefix sums
 };
 
-struct BwdGradTiles {
-  CUtensorMap tmE, tmC;  // bf16, box 64 x 128
-  int nb;
-  const int* pair_off;    // [nchunks * (nb + 1)]; entry nb of a chunk is its number of pairs
+// Everything the persistent backward kernel reads besides its tensor maps.
+struct BwdArgs {
+  int N, D, V, nb, nt, S, nchunks;
+  int out_bf16;
+  int64_t ignore_index;
   int64_t pair_cap;
-  const int4* pair_desc;  // [nchunks * pair_cap]
-  const int2* pair_slot;  // [nchunks * pair_cap]
-  int N, D, V;
+  size_t buf_bytes;  // one of the two gradient-tile buffers
   const float* lse;
   const float* scale;
   const int64_t* targets;
-  int64_t ignore_index;
+  const int* grp_start;
+  const int* chunk_t;
+  const int4* pair_desc;
+  const int2* pair_slot;
+  const int2* rb_range;
+  const int* offsets_t;
+  const int2* entries_t;
+  const int2* entries_b;
   uint8_t* gscratch;
-  int num_sms;
+  int* qctr;      // queue position, zero at launch
+  int* counters;  // zero at launch: [ctr_g_b] gradient tiles stored per (chunk, row block),
+                  // [ctr_g_t] per vocabulary tile, [ctr_b_done] dE / dC items finished per chunk
+  int ctr_g_b, ctr_g_t, ctr_b_done;
   int* err;
   uint64_t timeout_ns;
 };
 
-struct BwdGemm {
-  CUtensorMap tmE, tmC;  // bf16, box 64 x 64 (operand slices, one K-half of 64 rows per stage)
-  CUtensorMap tmdE;      // fp32 dE accumulator, box 32 x 32 (reduce-add)
-  CUtensorMap tmdC;      // dC output: bf16 box 64 x 32, or fp32 box 32 x 32
-  int N, D, V, nb;
-  const int2* entries_t;
-  const int* offsets_t;
-  const int2* entries_b;
-  const int2* rb_range;  // [nchunks * nb]
-  const uint8_t* gscratch;
-  const int* chunk_t;
-  int dC_bf16;
+struct BwdLaunch {
+  CUtensorMap tmE128, tmC128;  // bf16, box 64 x 128: K-blocks of the recompute
+  CUtensorMap tmE64, tmC64;    // bf16, box 64 x 64: operand slices of the dC / dE MMAs
+  CUtensorMap tmdC;            // dC output: bf16 box 64 x 32, or fp32 box 32 x 32
+  CUtensorMap tmdE;            // fp32 dE accumulator, box 32 x 32 (reduce-add)
+  BwdArgs args;
   int num_sms;
-  int* err;
-  uint64_t timeout_ns;
 };
 
 cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float* lse, const int64_t* targets,
                             int64_t N, int64_t V, int64_t T, int64_t ignore_index, float filter_eps,
                             int64_t* filtered_tiles, cudaStream_t s);
-cudaError_t launch_bwd_g(const BwdGradTiles& L, int chunk, cudaStream_t s);
-cudaError_t launch_bwd_gemm(const BwdGemm& L, int chunk, cudaStream_t s);
+cudaError_t launch_bwd(const BwdLaunch& L, cudaStream_t s);
 
 cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
 
