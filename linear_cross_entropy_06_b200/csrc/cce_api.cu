@@ -101,7 +101,7 @@ struct SplitWs {
   cce::BwdPlan plan;
   int* sync;         // [1 + nchunks * nb + nt + nchunks]: queue position, then the counters
   size_t sync_bytes;
-  uint8_t* gscratch; // 2 * buf_bytes
+  uint8_t* gscratch; // 3 * buf_bytes
   size_t buf_bytes;
   float* dE_acc;
   size_t bytes;
@@ -130,21 +130,22 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.cnt_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nb)));
   w.plan.offsets_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nb + 1)));
   w.plan.entries_b = reinterpret_cast<int2*>(take(sizeof(int2) * static_cast<size_t>(tiles)));
+  w.plan.pos_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(tiles)));
   w.plan.kept_total = reinterpret_cast<int*>(take(sizeof(int)));
   // A chunk spans at most kChunkCBytes of C (its C rows stay in L2 while they are re-read for
-  // every listed row block), and the gradient tiles of two chunks, at most nb per vocabulary tile,
-  // fit in kGradScratchBudget; at least one vocabulary tile per chunk.
+  // every listed row block), and the gradient tiles of three chunks, at most nb per vocabulary
+  // tile, fit in kGradScratchBudget; at least one vocabulary tile per chunk.
   const int64_t vt_bytes = static_cast<int64_t>(cce::kBwdBN) * p->D * 2;
   const int64_t per_vtile = std::max<int64_t>(nb, 1) * cce::kGradTileBytes;
   const int64_t chunk_vt = std::max<int64_t>(
-      1, std::min({nt, cce::kChunkCBytes / vt_bytes, cce::kGradScratchBudget / 2 / per_vtile}));
+      1, std::min({nt, cce::kChunkCBytes / vt_bytes, cce::kGradScratchBudget / 3 / per_vtile}));
   w.plan.chunk_vt = static_cast<int>(chunk_vt);
   w.plan.nchunks = static_cast<int>(ceil_div(nt, chunk_vt));
   w.plan.chunk_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks + 1)));
-  w.plan.pair_off = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks) * (nb + 1)));
   w.plan.rb_range = reinterpret_cast<int2*>(take(sizeof(int2) * static_cast<size_t>(w.plan.nchunks) * nb));
-  w.plan.pair_cap = nb * ((chunk_vt + 1) / 2);
-  const size_t pairs = static_cast<size_t>(w.plan.nchunks) * static_cast<size_t>(w.plan.pair_cap);
+  w.plan.pstart_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt + 1)));
+  // a row block with k listed tiles in a chunk forms ceil(k / 2) pairs there
+  const size_t pairs = static_cast<size_t>((tiles + static_cast<int64_t>(w.plan.nchunks) * nb) / 2 + 1);
   w.plan.pair_desc = reinterpret_cast<int4*>(take(sizeof(int4) * pairs));
   w.plan.pair_slot = reinterpret_cast<int2*>(take(sizeof(int2) * pairs));
   w.plan.S = static_cast<int>(ceil_div(p->D, cce::kGemmSlice));
@@ -153,7 +154,7 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.sync_bytes = sizeof(int) * static_cast<size_t>(1 + w.plan.nchunks * nb + nt + w.plan.nchunks);
   w.sync = reinterpret_cast<int*>(take(w.sync_bytes));
   w.buf_bytes = static_cast<size_t>(nb * chunk_vt) * cce::kGradTileBytes;
-  w.gscratch = reinterpret_cast<uint8_t*>(take(2 * w.buf_bytes));
+  w.gscratch = reinterpret_cast<uint8_t*>(take(3 * w.buf_bytes));
   if (!out_fp32) w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
   w.bytes = off;
   return w;
@@ -272,13 +273,13 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.nchunks = w.plan.nchunks;
   A.out_bf16 = out_fp32 ? 0 : 1;
   A.ignore_index = p->ignore_index;
-  A.pair_cap = w.plan.pair_cap;
   A.buf_bytes = w.buf_bytes;
   A.lse = lse;
   A.scale = w.scale;
   A.targets = targets;
   A.grp_start = w.plan.grp_start;
   A.chunk_t = w.plan.chunk_t;
+  A.pstart_t = w.plan.pstart_t;
   A.pair_desc = w.plan.pair_desc;
   A.pair_slot = w.plan.pair_slot;
   A.rb_range = w.plan.rb_range;

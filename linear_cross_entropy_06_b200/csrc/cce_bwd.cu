@@ -6,7 +6,7 @@
 // functions explainer, "How it works" item 2 (G = p - y, dE = G C, dC = G^T E); Cut Your Losses
 // abstract (logits are recomputed blockwise and never stored).
 //
-// Work items, per vocabulary chunk c (its gradient tiles live in scratch buffer c mod 2):
+// Work items, per vocabulary chunk c (its gradient tiles live in scratch buffer c mod 3):
 //   pair   two consecutive listed 128 x 128 tiles (b, t0), (b, t1) of row block b in the chunk:
 //          S = E_b [C_t0; C_t1]^T (tcgen05 M=128 N=256 K=D; skipped for onehot-only tiles), then
 //          G = scale_r * exp(S - LSE_r) - scale_r * [v = t_r] in fp32, rounded to bf16 into a
@@ -17,12 +17,16 @@
 //          same G tile read MN-major), written once by TMA store: every listed tile of t lies in
 //          t's chunk, so dC needs no reduction.
 //
-// Scheduling: a global queue holds the items in the order pairs(0), dE/dC(0), pairs(1), dE/dC(1),
-// ...; CTAs claim them one at a time with an atomic counter, so a claimed item always belongs to a
-// running CTA. Dependencies point only to earlier items:
+// Scheduling: a global queue holds the items in the order pairs(0), pairs(1), dE/dC(0), pairs(2),
+// dE/dC(1), ..., pairs(n-1), dE/dC(n-2), dE/dC(n-1): the dE/dC items of a chunk come one group of
+// pairs after the chunk's own pairs, so their gradient tiles are normally stored by the time they
+// are claimed. CTAs claim items one at a time with an atomic counter, so a claimed item always
+// belongs to a running CTA. Inside a chunk the pairs are ordered by vocabulary tile and the dE
+// items by slice of D, so that the items running at the same time read the same C tiles and
+// columns from L2. Dependencies point only to earlier items:
 //   a dE item waits until every gradient tile of its row block in the chunk is stored, a dC item
 //   until every gradient tile of its vocabulary tile is, and a pair of chunk c waits, before it
-//   stores, until every dE/dC item of chunk c - 2 (the previous user of the buffer) has read it.
+//   stores, until every dE/dC item of chunk c - 3 (the previous user of the buffer) has read it.
 // Every such wait is bounded. Because items are claimed in order and the smallest unfinished item
 // has no unfinished dependency, the queue always drains; and with no boundary between chunks the
 // machine has a single tail per backward instead of one per chunk and kernel.
@@ -130,14 +134,24 @@ __device__ __forceinline__ void read_item(const WorkItem* ring, int idx, WorkIte
   for (int i = 0; i < 3; ++i) dst[i] = src[i];
 }
 
-// Item w of the queue, in group g (2c: pairs of chunk c; 2c + 1: dE / dC items of chunk c) that
-// starts at item g_begin -> its decoded form (the scheduler's only global reads).
+// Queue group g -> (chunk, whether it holds the chunk's pairs). The groups are pairs(0), then
+// pairs(c), dE/dC(c - 1) for c = 1 .. n-1, then dE/dC(n - 1).
+__device__ __forceinline__ int2 group_of(int g, int nchunks) {
+  if (g == 0) return make_int2(0, 1);
+  if (g == 2 * nchunks - 1) return make_int2(nchunks - 1, 0);
+  const int pos = g - 1, c = pos / 2 + 1;
+  return (pos & 1) == 0 ? make_int2(c, 1) : make_int2(c - 1, 0);
+}
+
+// Item w of the queue, in group g that starts at item g_begin -> its decoded form (the scheduler's
+// only global reads).
 __device__ __forceinline__ void decode_item(int w, int g, int g_begin, const BwdArgs& A, WorkItem& it) {
-  const int c = g >> 1, local = w - g_begin;
+  const int2 gc = group_of(g, A.nchunks);
+  const int c = gc.x, local = w - g_begin;
   const int t_begin = A.chunk_t[c];
   it.chunk = c;
-  if ((g & 1) == 0) {
-    const int64_t pi = static_cast<int64_t>(c) * A.pair_cap + local;
+  if (gc.y) {
+    const int64_t pi = static_cast<int64_t>(A.pstart_t[t_begin]) + local;
     const int4 d = A.pair_desc[pi];
     const int2 sl = A.pair_slot[pi];
     it.kind = kPair;
@@ -147,9 +161,9 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, const Bwd
     it.s = d.w;
     it.slot0 = sl.x;
     it.slot1 = sl.y;
-    if (c >= 2) {  // the buffer's previous chunk must have been read by all of its dE / dC items
-      it.dep_idx = A.ctr_b_done + (c - 2);
-      it.dep_val = A.grp_start[2 * (c - 2) + 2] - A.grp_start[2 * (c - 2) + 1];
+    if (c >= 3) {  // the buffer's previous chunk must have been read by all of its dE / dC items
+      it.dep_idx = A.ctr_b_done + (c - 3);
+      it.dep_val = (A.nb + A.chunk_t[c - 2] - A.chunk_t[c - 3]) * A.S;
     } else {
       it.dep_idx = -1;
       it.dep_val = 0;
@@ -158,10 +172,10 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, const Bwd
     const int S = A.S;
     it.slot0 = A.offsets_t[t_begin];
     it.slot1 = 0;
-    if (local < A.nb * S) {
+    if (local < A.nb * S) {  // slice-major: concurrent dE items read the same columns of C
       it.kind = kDE;
-      it.key = local / S;
-      it.s = local % S;
+      it.key = local % A.nb;
+      it.s = local / A.nb;
       const int2 r = A.rb_range[static_cast<int64_t>(c) * A.nb + it.key];
       it.begin = r.x;
       it.end = r.y;
@@ -227,7 +241,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_holder;
   const WaitCtl wc{abort_flag, A.err, A.timeout_ns};
   const int num_kb = (A.D + BK - 1) / BK;
-  auto buffer = [&](int chunk) { return A.gscratch + static_cast<size_t>(chunk & 1) * A.buf_bytes; };
+  auto buffer = [&](int chunk) { return A.gscratch + static_cast<size_t>(chunk % 3) * A.buf_bytes; };
 
   if (warp == 6) {
     // ---------------- scheduler ----------------

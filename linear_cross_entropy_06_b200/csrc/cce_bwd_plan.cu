@@ -13,10 +13,13 @@
 //   each (b * 4 + flag, t), row blocks ascending. An entry's position is also its gradient-tile slot.
 // By row block (dE kernel): offsets_b[b] .. offsets_b[b+1] index entries_b, each (t, slot),
 //   vocabulary tiles ascending.
-// Per vocabulary chunk c, flat work lists the backward kernel reads with one load per item:
-//   rb_range[c * nb + b]   the entries [lo, hi) of row block b inside the chunk;
-//   pair_desc/pair_slot    from c * pair_cap: the pairs of consecutive listed tiles of a row block
-//                          inside the chunk, row blocks ascending (pair_off[c] holds their prefix sums).
+// Flat work lists the backward kernel reads with one load per item:
+//   rb_range[c * nb + b]   the entries [lo, hi) of row block b inside vocabulary chunk c;
+//   pair_desc/pair_slot    the pairs of consecutive listed tiles of a row block inside a chunk,
+//                          by the vocabulary tile of their first tile (pstart_t[t] is the first
+//                          pair starting in tile t, so a chunk's pairs are contiguous).
+#include <algorithm>
+
 #include "cce_device.cuh"
 #include "cce_internal.h"
 
@@ -116,7 +119,8 @@ __global__ void fill_col_kernel(const uint8_t* __restrict__ flags, const int* __
 // One warp per row block: counts (pass 0) or writes (pass 1) its listed tiles in vocabulary order.
 __global__ void row_list_kernel(const uint8_t* __restrict__ flags, const int* __restrict__ rank,
                                 const int* __restrict__ offsets_t, int nb, int nt, int* __restrict__ cnt_b,
-                                const int* __restrict__ offsets_b, int2* __restrict__ entries_b, int pass) {
+                                const int* __restrict__ offsets_b, int2* __restrict__ entries_b,
+                                int* __restrict__ pos_b, int pass) {
   const int b = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (b >= nb) return;
@@ -128,7 +132,9 @@ __global__ void row_list_kernel(const uint8_t* __restrict__ flags, const int* __
     const unsigned mask = __ballot_sync(0xffffffffu, on);
     if (pass == 1 && on) {
       const int pos = offsets_b[b] + k + __popc(mask & ((1u << lane) - 1u));
-      entries_b[pos] = make_int2(t, offsets_t[t] + rank[static_cast<int64_t>(b) * nt + t]);
+      const int slot = offsets_t[t] + rank[static_cast<int64_t>(b) * nt + t];
+      entries_b[pos] = make_int2(t, slot);
+      pos_b[slot] = pos;
     }
     k += __popc(mask);
   }
@@ -150,78 +156,83 @@ __global__ void chunk_plan_kernel(int nt, int chunk_vt, int nchunks, int* __rest
     chunk_t[c] = min(nt, c * chunk_vt);
 }
 
-// One block per vocabulary chunk: for every row block, the number of pairs of its consecutive
-// listed tiles inside the chunk (the gradient-tile kernel recomputes two vocabulary tiles of one
-// row block at once), and the exclusive prefix sums of those counts.
-__global__ void pair_plan_kernel(const int2* __restrict__ entries_b, const int* __restrict__ offsets_b, int nb,
-                                 const int* __restrict__ chunk_t, int* __restrict__ pair_off,
-                                 int2* __restrict__ rb_range) {
-  __shared__ int buf[1024];
-  __shared__ int carry;
-  const int c = blockIdx.x;
-  const int t0 = chunk_t[c], t1 = chunk_t[c + 1];
-  int* out = pair_off + static_cast<int64_t>(c) * (nb + 1);
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  for (int base = 0; base < nb; base += 1024) {
-    const int b = base + threadIdx.x;
-    int v = 0;
-    if (b < nb) {
-      const int lo = lower_bound_t(entries_b, offsets_b[b], offsets_b[b + 1], t0);
-      const int hi = lower_bound_t(entries_b, lo, offsets_b[b + 1], t1);
-      v = (hi - lo + 1) / 2;
-      rb_range[static_cast<int64_t>(c) * nb + b] = make_int2(lo, hi);
-    }
-    buf[threadIdx.x] = v;
-    __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-      const int add = threadIdx.x >= o ? buf[threadIdx.x - o] : 0;
-      __syncthreads();
-      buf[threadIdx.x] += add;
-      __syncthreads();
-    }
-    if (b < nb) out[b] = carry + buf[threadIdx.x] - v;
-    __syncthreads();
-    if (threadIdx.x == 1023) carry += buf[1023];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) out[nb] = carry;
-}
-
-// One warp per (chunk, row block): writes that row block's pairs into the chunk's pair list.
-// pair_desc = (b, t of the first tile, t of the second tile or -1, kept bits: 1 first, 2 second);
-// pair_slot = the two tiles' gradient-tile slots relative to the chunk's first slot.
-__global__ void pair_fill_kernel(const int2* __restrict__ entries_b, const uint8_t* __restrict__ flags, int nb, int nt,
-                                 int nchunks, const int* __restrict__ chunk_t, const int* __restrict__ offsets_t,
-                                 const int2* __restrict__ rb_range, const int* __restrict__ pair_off,
-                                 int64_t pair_cap, int4* __restrict__ pair_desc, int2* __restrict__ pair_slot) {
+// For every chunk c and row block b, the range [lo, hi) of b's entries_b inside the chunk.
+__global__ void row_range_kernel(const int2* __restrict__ entries_b, const int* __restrict__ offsets_b, int nb,
+                                 int nchunks, const int* __restrict__ chunk_t, int2* __restrict__ rb_range) {
   const int64_t total = static_cast<int64_t>(nb) * nchunks;
-  for (int64_t cb = blockIdx.x; cb < total; cb += gridDim.x) {
+  for (int64_t cb = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; cb < total;
+       cb += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int c = static_cast<int>(cb / nb), b = static_cast<int>(cb % nb);
-    const int2 r = rb_range[cb];
-    const int slot_base = offsets_t[chunk_t[c]];
-    const int64_t out0 = static_cast<int64_t>(c) * pair_cap + pair_off[static_cast<int64_t>(c) * (nb + 1) + b];
-    const int np = (r.y - r.x + 1) / 2;
-    for (int k = threadIdx.x; k < np; k += blockDim.x) {
-      const int i0 = r.x + 2 * k;
-      const bool two = i0 + 1 < r.y;
-      const int2 e0 = entries_b[i0];
-      const int2 e1 = two ? entries_b[i0 + 1] : make_int2(-1, e0.y);
-      const uint8_t* row = flags + static_cast<int64_t>(b) * nt;
-      const int kept = (row[e0.x] == 1 ? 1 : 0) | (two && row[e1.x] == 1 ? 2 : 0);
-      pair_desc[out0 + k] = make_int4(b, e0.x, e1.x, kept);
-      pair_slot[out0 + k] = make_int2(e0.y - slot_base, e1.y - slot_base);
-    }
+    const int lo = lower_bound_t(entries_b, offsets_b[b], offsets_b[b + 1], chunk_t[c]);
+    const int hi = lower_bound_t(entries_b, lo, offsets_b[b + 1], chunk_t[c + 1]);
+    rb_range[cb] = make_int2(lo, hi);
   }
 }
 
-// Sizes of the backward's queue groups: group 2c holds the pairs of chunk c, group 2c + 1 its dE
-// items (nb * S) and dC items (one per vocabulary tile of the chunk and slice).
-__global__ void group_size_kernel(const int* __restrict__ pair_off, const int* __restrict__ chunk_t, int nb, int S,
+// A listed tile (b, t) starts a pair when its position in row block b's list inside t's chunk is
+// even; the pair is (b, t) and b's next listed tile in the chunk, if any. Pairs are listed by the
+// vocabulary tile of their first tile (then row block), so that the recompute of concurrent pairs
+// shares C tiles in L2. One warp per vocabulary tile; pass 0 counts the pairs starting in tile t,
+// pass 1 (after the scan of those counts into pstart_t) writes them.
+__global__ void pair_list_kernel(const int2* __restrict__ entries_t, const int* __restrict__ offsets_t,
+                                 const int2* __restrict__ entries_b, const int* __restrict__ pos_b,
+                                 const int2* __restrict__ rb_range, const uint8_t* __restrict__ flags, int nb, int nt,
+                                 int chunk_vt, const int* __restrict__ chunk_t, int* __restrict__ cnt,
+                                 const int* __restrict__ pstart_t, int4* __restrict__ pair_desc,
+                                 int2* __restrict__ pair_slot, int pass) {
+  const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= nt) return;
+  const int c = t / chunk_vt;
+  const int slot_base = offsets_t[chunk_t[c]];
+  const int i0 = offsets_t[t], i1 = offsets_t[t + 1];
+  int k = 0;
+  for (int base = i0; base < i1; base += 32) {
+    const int i = base + lane;
+    bool start = false;
+    int b = 0, p = 0;
+    int2 rr = make_int2(0, 0);
+    if (i < i1) {
+      b = entries_t[i].x >> 2;
+      p = pos_b[i];
+      rr = rb_range[static_cast<int64_t>(c) * nb + b];
+      start = ((p - rr.x) & 1) == 0;
+    }
+    const unsigned mask = __ballot_sync(0xffffffffu, start);
+    if (pass == 1 && start) {
+      const int out = pstart_t[t] + k + __popc(mask & ((1u << lane) - 1u));
+      const bool two = p + 1 < rr.y;
+      const int t1 = two ? entries_b[p + 1].x : -1;
+      const int slot1 = two ? entries_b[p + 1].y : i;
+      const uint8_t* row = flags + static_cast<int64_t>(b) * nt;
+      const int kept = (row[t] == 1 ? 1 : 0) | (two && row[t1] == 1 ? 2 : 0);
+      pair_desc[out] = make_int4(b, t, t1, kept);
+      pair_slot[out] = make_int2(i - slot_base, slot1 - slot_base);
+    }
+    k += __popc(mask);
+  }
+  if (pass == 0 && lane == 0) cnt[t] = k;
+}
+
+// Sizes of the backward's queue groups, in queue order: pairs(0), then pairs(c) and dE/dC(c - 1)
+// for c = 1 .. n-1, then dE/dC(n - 1). A chunk's pairs are those starting in its vocabulary tiles;
+// its dE/dC group holds nb * S dE items and one dC item per vocabulary tile and slice.
+__global__ void group_size_kernel(const int* __restrict__ pstart_t, const int* __restrict__ chunk_t, int nb, int S,
                                   int nchunks, int* __restrict__ grp_size) {
-  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < nchunks; c += gridDim.x * blockDim.x) {
-    grp_size[2 * c] = pair_off[static_cast<int64_t>(c) * (nb + 1) + nb];
-    grp_size[2 * c + 1] = (nb + chunk_t[c + 1] - chunk_t[c]) * S;
+  for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < 2 * nchunks; g += gridDim.x * blockDim.x) {
+    int c, pairs;
+    if (g == 0) {
+      c = 0;
+      pairs = 1;
+    } else if (g == 2 * nchunks - 1) {
+      c = nchunks - 1;
+      pairs = 0;
+    } else {
+      const int pos = g - 1;
+      c = pos / 2 + 1 - (pos & 1);
+      pairs = (pos & 1) == 0;
+    }
+    grp_size[g] = pairs ? pstart_t[chunk_t[c + 1]] - pstart_t[chunk_t[c]] : (nb + chunk_t[c + 1] - chunk_t[c]) * S;
   }
 }
 
@@ -251,23 +262,32 @@ cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float
     note_launches(1);
     const int grid_b = (nb * 32 + 255) / 256;
     row_list_kernel<<<grid_b, 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt, P.cnt_b, P.offsets_b, P.entries_b,
-                                           0);
+                                           P.pos_b, 0);
     note_launches(1);
     scan_kernel<<<1, 1024, 0, s>>>(P.cnt_b, nb, P.offsets_b);
     note_launches(1);
     row_list_kernel<<<grid_b, 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt, P.cnt_b, P.offsets_b, P.entries_b,
-                                           1);
+                                           P.pos_b, 1);
     note_launches(1);
     chunk_plan_kernel<<<(P.nchunks + 256) / 256, 256, 0, s>>>(nt, P.chunk_vt, P.nchunks, P.chunk_t);
     note_launches(1);
-    pair_plan_kernel<<<P.nchunks, 1024, 0, s>>>(P.entries_b, P.offsets_b, nb, P.chunk_t, P.pair_off, P.rb_range);
-    note_launches(1);
     const int64_t cbs = static_cast<int64_t>(nb) * P.nchunks;
-    const int grid_p = static_cast<int>(cbs < (int64_t(1) << 20) ? cbs : (int64_t(1) << 20));
-    pair_fill_kernel<<<grid_p, 32, 0, s>>>(P.entries_b, P.flags, nb, nt, P.nchunks, P.chunk_t, P.offsets_t,
-                                           P.rb_range, P.pair_off, P.pair_cap, P.pair_desc, P.pair_slot);
+    row_range_kernel<<<static_cast<int>(std::min<int64_t>((cbs + 255) / 256, 4096)), 256, 0, s>>>(
+        P.entries_b, P.offsets_b, nb, P.nchunks, P.chunk_t, P.rb_range);
     note_launches(1);
-    group_size_kernel<<<(P.nchunks + 255) / 256, 256, 0, s>>>(P.pair_off, P.chunk_t, nb, P.S, P.nchunks, P.grp_size);
+    // the pair counts per vocabulary tile reuse cnt_t (its counts are already scanned into offsets_t)
+    const int grid_t = static_cast<int>((static_cast<int64_t>(nt) * 32 + 255) / 256);
+    pair_list_kernel<<<grid_t, 256, 0, s>>>(P.entries_t, P.offsets_t, P.entries_b, P.pos_b, P.rb_range, P.flags, nb,
+                                            nt, P.chunk_vt, P.chunk_t, P.cnt_t, P.pstart_t, P.pair_desc, P.pair_slot,
+                                            0);
+    note_launches(1);
+    scan_kernel<<<1, 1024, 0, s>>>(P.cnt_t, nt, P.pstart_t);
+    note_launches(1);
+    pair_list_kernel<<<grid_t, 256, 0, s>>>(P.entries_t, P.offsets_t, P.entries_b, P.pos_b, P.rb_range, P.flags, nb,
+                                            nt, P.chunk_vt, P.chunk_t, P.cnt_t, P.pstart_t, P.pair_desc, P.pair_slot,
+                                            1);
+    note_launches(1);
+    group_size_kernel<<<(P.nchunks + 255) / 256, 256, 0, s>>>(P.pstart_t, P.chunk_t, nb, P.S, P.nchunks, P.grp_size);
     note_launches(1);
     scan_kernel<<<1, 1024, 0, s>>>(P.grp_size, 2 * P.nchunks, P.grp_start);
     note_launches(1);

@@ -41,8 +41,8 @@ constexpr int kGemmSlice = 256;                           // columns of D per dC
 // A vocabulary chunk spans at most kChunkCBytes of C, so that the C rows of a chunk stay in L2
 // while they are re-read for every row block that lists them ...
 constexpr int64_t kChunkCBytes = int64_t(64) << 20;
-// ... and the gradient tiles of two chunks (at most one per listed row block and vocabulary tile;
-// one chunk is written while the previous one is read) fit in a fixed kGradScratchBudget.
+// ... and the gradient tiles of three chunks (at most one per listed row block and vocabulary
+// tile; a chunk is written while the two before it are read) fit in a fixed kGradScratchBudget.
 constexpr int64_t kGradScratchBudget = int64_t(128) << 20;
 
 struct BwdPlan {
@@ -55,17 +55,16 @@ struct BwdPlan {
   int* cnt_b;       // [nb]
   int* offsets_b;   // [nb + 1]
   int2* entries_b;  // [nb * nt]: (t, slot in entries_t), by row block then vocabulary tile
+  int* pos_b;       // [nb * nt]: for each entries_t position, the tile's position in entries_b
   int* kept_total;
   int chunk_vt;     // vocabulary tiles per chunk
   int nchunks;
   int S;            // 256-column slices of D
   int* chunk_t;     // [nchunks + 1]: first vocabulary tile of each chunk
-  int* pair_off;    // [nchunks * (nb + 1)]: per chunk, prefix sums over row blocks of the number of
-                    // pairs of consecutive listed tiles of that row block inside the chunk
   int2* rb_range;   // [nchunks * nb]: entries [lo, hi) of each row block inside each chunk
-  int64_t pair_cap; // pairs a chunk can hold: nb * ceil(chunk_vt / 2)
-  int4* pair_desc;  // [nchunks * pair_cap]: (b, t0, t1 or -1, kept bits)
-  int2* pair_slot;  // [nchunks * pair_cap]: gradient-tile slots of t0 and t1, relative to the chunk
+  int* pstart_t;    // [nt + 1]: first pair whose first tile is in vocabulary tile t
+  int4* pair_desc;  // [pair capacity]: (b, t0, t1 or -1, kept bits), by t0 then b
+  int2* pair_slot;  // [pair capacity]: gradient-tile slots of t0 and t1, relative to the chunk
   int* grp_size;    // [2 * nchunks]: work items of each queue group (pairs of chunk c, then its dE/dC)
   int* grp_start;   // [2 * nchunks + 1]: their prefix sums
 };
@@ -75,13 +74,13 @@ struct BwdArgs {
   int N, D, V, nb, nt, S, nchunks;
   int out_bf16;
   int64_t ignore_index;
-  int64_t pair_cap;
-  size_t buf_bytes;  // one of the two gradient-tile buffers
+  size_t buf_bytes;  // one of the three gradient-tile buffers
   const float* lse;
   const float* scale;
   const int64_t* targets;
   const int* grp_start;
   const int* chunk_t;
+  const int* pstart_t;
   const int4* pair_desc;
   const int2* pair_slot;
   const int2* rb_range;

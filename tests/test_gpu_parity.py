@@ -266,8 +266,8 @@ def test_no_logit_sized_allocation(device):
 
     Beyond the gradients themselves ((N+V)*D*4 with fp32 outputs) the path holds the forward's
     per-sub-tile maxima and exp sums (8*N*ceil(V/128) bytes), the backward's tile plan
-    (flags, ranks and the two tile lists: 21 bytes per 128x128 tile; the per-chunk pair lists:
-    about 12 more) and the gradient tiles of one vocabulary chunk (at most a fixed 128 MiB).
+    (flags, ranks, the two tile lists and the map between them: 25 bytes per 128x128 tile; the
+    pair lists: about 12 more) and the gradient tiles of one vocabulary chunk (at most a fixed 128 MiB).
     Doubling V must grow that by the tile statistics only.
     """
     N, D = 4096, 1024
