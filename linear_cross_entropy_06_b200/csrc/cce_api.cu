@@ -101,7 +101,7 @@ struct SplitWs {
   cce::BwdPlan plan;
   int* sync;         // [1 + nchunks * nb + nt + nchunks]: queue position, then the counters
   size_t sync_bytes;
-  uint8_t* gscratch; // 3 * buf_bytes
+  uint8_t* gscratch; // kGradBuffers * buf_bytes
   size_t buf_bytes;
   float* dE_acc;
   size_t bytes;
@@ -133,12 +133,12 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.pos_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(tiles)));
   w.plan.kept_total = reinterpret_cast<int*>(take(sizeof(int)));
   // A chunk spans at most kChunkCBytes of C (its C rows stay in L2 while they are re-read for
-  // every listed row block), and the gradient tiles of three chunks, at most nb per vocabulary
-  // tile, fit in kGradScratchBudget; at least one vocabulary tile per chunk.
+  // every listed row block), and the gradient tiles of kGradBuffers chunks, at most nb per
+  // vocabulary tile, fit in kGradScratchBudget; at least one vocabulary tile per chunk.
   const int64_t vt_bytes = static_cast<int64_t>(cce::kBwdBN) * p->D * 2;
   const int64_t per_vtile = std::max<int64_t>(nb, 1) * cce::kGradTileBytes;
   const int64_t chunk_vt = std::max<int64_t>(
-      1, std::min({nt, cce::kChunkCBytes / vt_bytes, cce::kGradScratchBudget / 3 / per_vtile}));
+      1, std::min({nt, cce::kChunkCBytes / vt_bytes, cce::kGradScratchBudget / cce::kGradBuffers / per_vtile}));
   w.plan.chunk_vt = static_cast<int>(chunk_vt);
   w.plan.nchunks = static_cast<int>(ceil_div(nt, chunk_vt));
   w.plan.chunk_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks + 1)));
@@ -154,7 +154,7 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.sync_bytes = sizeof(int) * static_cast<size_t>(1 + w.plan.nchunks * nb + nt + w.plan.nchunks);
   w.sync = reinterpret_cast<int*>(take(w.sync_bytes));
   w.buf_bytes = static_cast<size_t>(nb * chunk_vt) * cce::kGradTileBytes;
-  w.gscratch = reinterpret_cast<uint8_t*>(take(3 * w.buf_bytes));
+  w.gscratch = reinterpret_cast<uint8_t*>(take(cce::kGradBuffers * w.buf_bytes));
   if (!out_fp32) w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
   w.bytes = off;
   return w;

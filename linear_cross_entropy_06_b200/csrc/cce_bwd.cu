@@ -6,7 +6,7 @@
 // functions explainer, "How it works" item 2 (G = p - y, dE = G C, dC = G^T E); Cut Your Losses
 // abstract (logits are recomputed blockwise and never stored).
 //
-// Work items, per vocabulary chunk c (its gradient tiles live in scratch buffer c mod 3):
+// Work items, per vocabulary chunk c (its gradient tiles live in scratch buffer c mod kGradBuffers):
 //   pair   two consecutive listed 128 x 128 tiles (b, t0), (b, t1) of row block b in the chunk:
 //          S = E_b [C_t0; C_t1]^T (tcgen05 M=128 N=256 K=D; skipped for onehot-only tiles), then
 //          G = scale_r * exp(S - LSE_r) - scale_r * [v = t_r] in fp32, rounded to bf16 into a
@@ -26,7 +26,8 @@
 // columns from L2. Dependencies point only to earlier items:
 //   a dE item waits until every gradient tile of its row block in the chunk is stored, a dC item
 //   until every gradient tile of its vocabulary tile is, and a pair of chunk c waits, before it
-//   stores, until every dE/dC item of chunk c - 3 (the previous user of the buffer) has read it.
+//   stores, until every dE/dC item of chunk c - kGradBuffers (the buffer's previous user) has
+//   read it.
 // Every such wait is bounded. Because items are claimed in order and the smallest unfinished item
 // has no unfinished dependency, the queue always drains; and with no boundary between chunks the
 // machine has a single tail per backward instead of one per chunk and kernel.
@@ -161,9 +162,10 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, const Bwd
     it.s = d.w;
     it.slot0 = sl.x;
     it.slot1 = sl.y;
-    if (c >= 3) {  // the buffer's previous chunk must have been read by all of its dE / dC items
-      it.dep_idx = A.ctr_b_done + (c - 3);
-      it.dep_val = (A.nb + A.chunk_t[c - 2] - A.chunk_t[c - 3]) * A.S;
+    if (c >= kGradBuffers) {  // the buffer's previous chunk must have been read by its dE / dC items
+      const int prev = c - kGradBuffers;
+      it.dep_idx = A.ctr_b_done + prev;
+      it.dep_val = (A.nb + A.chunk_t[prev + 1] - A.chunk_t[prev]) * A.S;
     } else {
       it.dep_idx = -1;
       it.dep_val = 0;
@@ -241,7 +243,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_holder;
   const WaitCtl wc{abort_flag, A.err, A.timeout_ns};
   const int num_kb = (A.D + BK - 1) / BK;
-  auto buffer = [&](int chunk) { return A.gscratch + static_cast<size_t>(chunk % 3) * A.buf_bytes; };
+  auto buffer = [&](int chunk) { return A.gscratch + static_cast<size_t>(chunk % kGradBuffers) * A.buf_bytes; };
 
   if (warp == 6) {
     // ---------------- scheduler ----------------

@@ -30,52 +30,56 @@ __device__ __forceinline__ bool valid_target(int64_t t, int64_t V, int64_t ignor
   return t != ignore_index && t >= 0 && t < V;
 }
 
-// One block (128 threads, one per tile row) per vocabulary tile, walking the row blocks in order.
+// One block of 128 threads (one per tile row) per backward tile (b, t) = (i / nt, i % nt): its flag.
 __global__ void tile_flags_kernel(const float* __restrict__ tile_max, const float* __restrict__ lse,
                                   const int64_t* __restrict__ targets, int64_t N, int64_t V, int64_t T,
-                                  int64_t ignore_index, float ln_eps, int filter_on, int nb, uint8_t* __restrict__ flags,
-                                  int* __restrict__ rank, int* __restrict__ cnt_t, int* __restrict__ kept_total) {
+                                  int64_t ignore_index, float ln_eps, int filter_on, int nt,
+                                  uint8_t* __restrict__ flags) {
   __shared__ float wmax[4];
-  const int t = blockIdx.x;
-  const int nt = gridDim.x;
+  const int64_t i = blockIdx.x;
+  const int b = static_cast<int>(i / nt), t = static_cast<int>(i % nt);
   const int64_t v0 = static_cast<int64_t>(t) * kBwdBN;
-  int listed = 0, kept = 0;
-  for (int b = 0; b < nb; ++b) {
-    const int64_t r = static_cast<int64_t>(b) * kBwdBM + threadIdx.x;
-    float m = -INFINITY;
-    bool has_target = false;
-    if (r < N) {
-      const int64_t tr = targets[r];
-      if (valid_target(tr, V, ignore_index)) {
-        has_target = tr >= v0 && tr < v0 + kBwdBN;
-        if (filter_on) {
-          const int64_t j0 = static_cast<int64_t>(t) * (kBwdBN / kSubTile);
-          const int64_t j1 = j0 + kBwdBN / kSubTile < T ? j0 + kBwdBN / kSubTile : T;
-          for (int64_t j = j0; j < j1; ++j) m = fmaxf(m, tile_max[j * N + r]);
-          m -= lse[r];
-        }
+  const int64_t r = static_cast<int64_t>(b) * kBwdBM + threadIdx.x;
+  float m = -INFINITY;
+  bool has_target = false;
+  if (r < N) {
+    const int64_t tr = targets[r];
+    if (valid_target(tr, V, ignore_index)) {
+      has_target = tr >= v0 && tr < v0 + kBwdBN;
+      if (filter_on) {
+        const int64_t j0 = static_cast<int64_t>(t) * (kBwdBN / kSubTile);
+        const int64_t j1 = j0 + kBwdBN / kSubTile < T ? j0 + kBwdBN / kSubTile : T;
+        for (int64_t j = j0; j < j1; ++j) m = fmaxf(m, tile_max[j * N + r]);
+        m -= lse[r];
       }
     }
-    bool keep = true;
-    if (filter_on) {
-      m = warp_max(m);
-      if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
-    }
-    const int any_target = __syncthreads_or(has_target ? 1 : 0);
-    if (filter_on) {
-      const float bm = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
-      keep = bm >= ln_eps;
-    }
-    const uint8_t f = keep ? 1 : (any_target ? 2 : 0);
-    if (threadIdx.x == 0) {
-      flags[static_cast<int64_t>(b) * nt + t] = f;
-      rank[static_cast<int64_t>(b) * nt + t] = listed;
-    }
-    listed += f != 0;
-    kept += f == 1;
-    __syncthreads();  // wmax is rewritten for the next row block
   }
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  const int any_target = __syncthreads_or(has_target ? 1 : 0);
   if (threadIdx.x == 0) {
+    const bool keep = !filter_on || fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3])) >= ln_eps;
+    flags[i] = keep ? 1 : (any_target ? 2 : 0);
+  }
+}
+
+// One warp per vocabulary tile t: the rank of each listed (b, t) among the listed row blocks of t,
+// the number of listed tiles of t, and the kept total.
+__global__ void tile_rank_kernel(const uint8_t* __restrict__ flags, int nb, int nt, int* __restrict__ rank,
+                                 int* __restrict__ cnt_t, int* __restrict__ kept_total) {
+  const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= nt) return;
+  int listed = 0, kept = 0;
+  for (int b0 = 0; b0 < nb; b0 += 32) {
+    const int b = b0 + lane;
+    const uint8_t f = b < nb ? flags[static_cast<int64_t>(b) * nt + t] : 0;
+    const unsigned on = __ballot_sync(0xffffffffu, f != 0);
+    if (f != 0) rank[static_cast<int64_t>(b) * nt + t] = listed + __popc(on & ((1u << lane) - 1u));
+    listed += __popc(on);
+    kept += __popc(__ballot_sync(0xffffffffu, f == 1));
+  }
+  if (lane == 0) {
     cnt_t[t] = listed;
     atomicAdd(kept_total, kept);
   }
@@ -251,12 +255,15 @@ cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float
   cudaError_t e = cudaMemsetAsync(P.kept_total, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
   if (nb > 0) {
-    tile_flags_kernel<<<nt, kBwdBM, 0, s>>>(tile_max, lse, targets, N, V, T, ignore_index, ln_eps, filter_on, nb,
-                                            P.flags, P.rank, P.cnt_t, P.kept_total);
+    const int64_t tiles = static_cast<int64_t>(nb) * nt;
+    tile_flags_kernel<<<static_cast<unsigned>(tiles), kBwdBM, 0, s>>>(tile_max, lse, targets, N, V, T, ignore_index,
+                                                                     ln_eps, filter_on, nt, P.flags);
+    note_launches(1);
+    tile_rank_kernel<<<static_cast<int>((static_cast<int64_t>(nt) * 32 + 255) / 256), 256, 0, s>>>(
+        P.flags, nb, nt, P.rank, P.cnt_t, P.kept_total);
     note_launches(1);
     scan_kernel<<<1, 1024, 0, s>>>(P.cnt_t, nt, P.offsets_t);
     note_launches(1);
-    const int64_t tiles = static_cast<int64_t>(nb) * nt;
     fill_col_kernel<<<static_cast<int>((tiles + 255) / 256), 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt,
                                                                           P.entries_t);
     note_launches(1);

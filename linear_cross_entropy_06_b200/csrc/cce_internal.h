@@ -41,9 +41,13 @@ constexpr int kGemmSlice = 256;                           // columns of D per dC
 // A vocabulary chunk spans at most kChunkCBytes of C, so that the C rows of a chunk stay in L2
 // while they are re-read for every row block that lists them ...
 constexpr int64_t kChunkCBytes = int64_t(64) << 20;
-// ... and the gradient tiles of three chunks (at most one per listed row block and vocabulary
-// tile; a chunk is written while the two before it are read) fit in a fixed kGradScratchBudget.
+// ... and the gradient tiles of kGradBuffers chunks (at most one per listed row block and
+// vocabulary tile; a chunk is written while the one before it is read) fit in a fixed
+// kGradScratchBudget. The backward's queue places the dE/dC items of chunk c - 2 before the pairs
+// of chunk c, so two buffers are the fewest that keep every wait pointing to an earlier item.
 constexpr int64_t kGradScratchBudget = int64_t(128) << 20;
+constexpr int kGradBuffers = 2;
+static_assert(kGradBuffers >= 2, "the pairs of chunk c reuse the buffer of chunk c - kGradBuffers");
 
 struct BwdPlan {
   int nb, nt;
@@ -74,7 +78,7 @@ struct BwdArgs {
   int N, D, V, nb, nt, S, nchunks;
   int out_bf16;
   int64_t ignore_index;
-  size_t buf_bytes;  // one of the three gradient-tile buffers
+  size_t buf_bytes;  // one of the kGradBuffers gradient-tile buffers
   const float* lse;
   const float* scale;
   const int64_t* targets;
