@@ -134,11 +134,12 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.kept_total = reinterpret_cast<int*>(take(sizeof(int)));
   // A chunk spans at most kChunkCBytes of C (its C rows stay in L2 while they are re-read for
   // every listed row block), and the gradient tiles of kGradBuffers chunks, at most nb per
-  // vocabulary tile, fit in kGradScratchBudget; at least one vocabulary tile per chunk.
+  // vocabulary tile, fit in the scratch budget; at least one vocabulary tile per chunk.
   const int64_t vt_bytes = static_cast<int64_t>(cce::kBwdBN) * p->D * 2;
   const int64_t per_vtile = std::max<int64_t>(nb, 1) * cce::kGradTileBytes;
-  const int64_t chunk_vt = std::max<int64_t>(
-      1, std::min({nt, cce::kChunkCBytes / vt_bytes, cce::kGradScratchBudget / cce::kGradBuffers / per_vtile}));
+  const int64_t budget = std::max(cce::kGradScratchMin, nb * cce::kGradScratchPerRowBlock);
+  const int64_t chunk_vt =
+      std::max<int64_t>(1, std::min({nt, cce::kChunkCBytes / vt_bytes, budget / cce::kGradBuffers / per_vtile}));
   w.plan.chunk_vt = static_cast<int>(chunk_vt);
   w.plan.nchunks = static_cast<int>(ceil_div(nt, chunk_vt));
   w.plan.chunk_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks + 1)));

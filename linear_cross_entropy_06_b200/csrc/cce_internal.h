@@ -42,10 +42,13 @@ constexpr int kGemmSlice = 256;                           // columns of D per dC
 // while they are re-read for every row block that lists them ...
 constexpr int64_t kChunkCBytes = int64_t(64) << 20;
 // ... and the gradient tiles of kGradBuffers chunks (at most one per listed row block and
-// vocabulary tile; a chunk is written while the one before it is read) fit in a fixed
-// kGradScratchBudget. The backward's queue places the dE/dC items of chunk c - 2 before the pairs
-// of chunk c, so two buffers are the fewest that keep every wait pointing to an earlier item.
-constexpr int64_t kGradScratchBudget = int64_t(128) << 20;
+// vocabulary tile; a chunk is written while the one before it is read) fit in the scratch: 4 MiB
+// per 128-row block, at least 128 MiB. The scratch grows with N, not with V, so that a chunk keeps
+// the same number of vocabulary tiles as N grows: each chunk adds a full N x D fp32 partial into
+// dE. The backward's queue places the dE/dC items of chunk c - 2 before the pairs of chunk c, so
+// two buffers are the fewest that keep every wait pointing to an earlier item.
+constexpr int64_t kGradScratchPerRowBlock = int64_t(4) << 20;
+constexpr int64_t kGradScratchMin = int64_t(128) << 20;
 constexpr int kGradBuffers = 2;
 static_assert(kGradBuffers >= 2, "the pairs of chunk c reuse the buffer of chunk c - kGradBuffers");
 

@@ -261,36 +261,52 @@ def test_long_batch(device):
     assert rb.filtered <= len(blocks) * nt
 
 
+def _extra_loss_memory(device, N, D, V):
+    """Peak device memory of one forward + backward beyond the inputs and the fp32 gradients."""
+    inp = make_inputs("llama3.1-8b-head", N=N, D=D, V=V, seed=11)
+    E, C, t = inp.E.to(device), inp.C.to(device), inp.targets.to(device)
+    g = torch.ones(1, device=device)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base = torch.cuda.memory_allocated()
+    loss, lse, tmax, count = ops.cce_forward(E, C, t)
+    dE, dC, filt = ops.cce_backward(E, C, t, lse, tmax, count, g, out_fp32=True)
+    torch.cuda.synchronize()
+    extra = torch.cuda.max_memory_allocated() - base
+    del loss, lse, tmax, count, dE, dC, filt
+    return extra - (N + V) * D * 4
+
+
+def _memory_bound(N, V):
+    """Tile statistics (8 N bytes per 128 columns), the tile plan (at most 40 bytes per 128x128
+    tile), the gradient-tile scratch (4 MiB per 128-row block, at least 128 MiB) and 8 MiB of
+    small buffers and allocator rounding."""
+    nb, nt = math.ceil(N / 128), math.ceil(V / 128)
+    return 8 * N * nt + 40 * nb * nt + max(128 << 20, nb * (4 << 20)) + (8 << 20)
+
+
 def test_no_logit_sized_allocation(device):
-    """Extra device memory of forward + backward is O(N*V/128) plus fixed budgets, never O(N*V).
+    """Extra device memory of forward + backward is O(N + N*V/128), never O(N*V).
 
     Beyond the gradients themselves ((N+V)*D*4 with fp32 outputs) the path holds the forward's
     per-sub-tile maxima and exp sums (8*N*ceil(V/128) bytes), the backward's tile plan
     (flags, ranks, the two tile lists and the map between them: 25 bytes per 128x128 tile; the
-    pair lists: about 12 more) and the gradient tiles of one vocabulary chunk (at most a fixed 128 MiB).
-    Doubling V must grow that by the tile statistics only.
+    pair lists: about 12 more) and the gradient tiles of two vocabulary chunks (4 MiB per 128-row
+    block, at least 128 MiB). Doubling V must grow that by the tile statistics only.
     """
     N, D = 4096, 1024
-
-    def loss_memory(V):
-        inp = make_inputs("llama3.1-8b-head", N=N, D=D, V=V, seed=11)
-        E, C, t = inp.E.to(device), inp.C.to(device), inp.targets.to(device)
-        g = torch.ones(1, device=device)
-        torch.cuda.synchronize()
-        torch.cuda.reset_peak_memory_stats()
-        base = torch.cuda.memory_allocated()
-        loss, lse, tmax, count = ops.cce_forward(E, C, t)
-        dE, dC, filt = ops.cce_backward(E, C, t, lse, tmax, count, g, out_fp32=True)
-        torch.cuda.synchronize()
-        extra = torch.cuda.max_memory_allocated() - base
-        del loss, lse, tmax, count, dE, dC, filt
-        return extra - (N + V) * D * 4
-
-    m1, m2 = loss_memory(64128), loss_memory(128256)
+    m1, m2 = _extra_loss_memory(device, N, D, 64128), _extra_loss_memory(device, N, D, 128256)
     for V, m in ((64128, m1), (128256, m2)):
-        tiles = math.ceil(N / 128) * math.ceil(V / 128)
-        bound = 8 * N * math.ceil(V / 128) + 40 * tiles + (128 << 20) + (8 << 20)
-        assert m <= bound, (V, m, bound)
+        assert m <= _memory_bound(N, V), (V, m, _memory_bound(N, V))
     assert m2 < N * 128256 * 2 / 4, m2  # at the Llama-3 vocabulary, far below even bf16 logits
     # growth with V: the tile statistics (8 N bytes per 128 columns), not N*V*2
     assert m2 - m1 <= 8 * N * math.ceil(64128 / 128) * 1.25 + (4 << 20), (m1, m2)
+
+
+def test_no_logit_sized_allocation_long_batch(device):
+    """At the long-batch token count (N = 32768) the scratch grows with N (4 MiB per 128 rows)
+    and the extra memory stays a small fraction of the bf16 logits (N*V*2 = 8.4 GB)."""
+    N, D, V = 32768, 1024, 128256
+    m = _extra_loss_memory(device, N, D, V)
+    assert m <= _memory_bound(N, V), (m, _memory_bound(N, V))
+    assert m < N * V * 2 / 4, m
