@@ -16,8 +16,10 @@ What it computes, and where that is stated:
 * Loss functions (explainer), "How it works" items 1, 2 and 4: the stable
   log-sum-exp ``m + log sum exp(z - m)``; the logit gradient ``p - y``; the mean
   over non-ignored tokens only.
-* mlx-cross-entropy README, "API" table: ``reduction`` in {mean, sum, none} and
-  ``ignore_index`` (default -100) masks a token.
+* mlx-cross-entropy README, "API" table: ``reduction`` in {mean, sum, none},
+  ``ignore_index`` (default -100) masks a token, and an optional classifier bias
+  ``[V]`` is added to every row of logits: ``z = E @ C.T + bias``. Its gradient is
+  the column sum of the logit gradient, ``dbias = sum_r G[r, :]``.
 * mlx-cross-entropy README, "How it works" item 2: the backward skips tiles
   whose softmax is below ``2**-12``. The rule here, per tile of ``tile_m`` rows by
   ``tile_n`` vocabulary columns: the tile is skipped when every non-ignored row
@@ -91,9 +93,21 @@ def validate_targets(targets: np.ndarray, V: int, ignore_index: int) -> None:
         raise ValueError(f"target {int(t[r])} at row {r} is outside [0, {V}) and is not ignore_index")
 
 
-def logits(E: np.ndarray, C: np.ndarray) -> np.ndarray:
-    """z = E @ C.T in float64 (mlx-cross-entropy README, "How it works" item 1: e @ c.T)."""
-    return _f64(E) @ _f64(C).T
+def _bias64(bias, V: int) -> Optional[np.ndarray]:
+    if bias is None:
+        return None
+    b = _f64(bias).reshape(-1)
+    if b.shape[0] != V:
+        raise ValueError(f"bias must have {V} entries, got {b.shape[0]}")
+    return b
+
+
+def logits(E: np.ndarray, C: np.ndarray, bias=None) -> np.ndarray:
+    """z = E @ C.T (+ bias) in float64 (mlx-cross-entropy README, "How it works" item 1: e @ c.T;
+    "API" table: classifier bias [V])."""
+    z = _f64(E) @ _f64(C).T
+    b = _bias64(bias, z.shape[1])
+    return z if b is None else z + b[None, :]
 
 
 def log_sum_exp_rows(z: np.ndarray) -> np.ndarray:
@@ -139,7 +153,7 @@ def reduce_loss(nll: np.ndarray, count: int, reduction: str) -> np.ndarray:
     raise ValueError(f"reduction must be one of {REDUCTIONS}, got {reduction!r}")
 
 
-def forward_rows(E, C, targets, rows: Optional[Sequence[int]] = None, ignore_index: int = -100):
+def forward_rows(E, C, targets, rows: Optional[Sequence[int]] = None, ignore_index: int = -100, bias=None):
     """Per-row LSE, correct-token logit and loss for a subset of rows.
 
     Each row of the loss depends only on its own hidden state, so any subset of
@@ -147,6 +161,7 @@ def forward_rows(E, C, targets, rows: Optional[Sequence[int]] = None, ignore_ind
     """
     E64, C64, t = _f64(E), _f64(C), _i64(targets)
     V = C64.shape[0]
+    b = _bias64(bias, V)
     validate_targets(t, V, ignore_index)
     rows = np.arange(E64.shape[0]) if rows is None else np.asarray(rows, dtype=np.int64)
     lse = np.empty(len(rows))
@@ -154,6 +169,8 @@ def forward_rows(E, C, targets, rows: Optional[Sequence[int]] = None, ignore_ind
     for g in _row_groups(len(rows)):
         rr = rows[g]
         z = E64[rr] @ C64.T
+        if b is not None:
+            z += b[None, :]
         lse[g] = log_sum_exp_rows(z)
         tr = t[rr]
         ok = tr != ignore_index
@@ -164,11 +181,11 @@ def forward_rows(E, C, targets, rows: Optional[Sequence[int]] = None, ignore_ind
     return rows, lse, zt, nll, valid
 
 
-def forward(E, C, targets, ignore_index: int = -100, reduction: str = "mean") -> ForwardResult:
+def forward(E, C, targets, ignore_index: int = -100, reduction: str = "mean", bias=None) -> ForwardResult:
     """Loss and per-row LSE of linear cross-entropy (the forward the CUDA path computes)."""
     if reduction not in REDUCTIONS:
         raise ValueError(f"reduction must be one of {REDUCTIONS}, got {reduction!r}")
-    _, lse, zt, nll, valid = forward_rows(E, C, targets, None, ignore_index)
+    _, lse, zt, nll, valid = forward_rows(E, C, targets, None, ignore_index, bias)
     count = int(valid.sum())
     return ForwardResult(reduce_loss(nll, count, reduction), lse, zt, nll, count)
 
@@ -230,17 +247,18 @@ class BackwardResult:
     filtered: int  # number of skipped tiles
     borderline: int  # tiles whose margin is within `window` of ln(eps)
     n_tiles: int
+    dbias: Optional[np.ndarray] = None  # [V] when a bias is given
 
 
 def backward(E, C, targets, grad_out=1.0, ignore_index: int = -100, reduction: str = "mean",
              filter_eps: float = 2.0 ** -12, tile_m: int = 128, tile_n: int = 256,
-             window: float = 2e-3) -> BackwardResult:
-    """dE and dC of linear cross-entropy, with the tile-skipping rule applied.
+             window: float = 2e-3, bias=None) -> BackwardResult:
+    """dE, dC (and dbias) of linear cross-entropy, with the tile-skipping rule applied.
 
     G = scale_r * (p~ - onehot), p~ = softmax with skipped tiles set to 0;
-    dE = G @ C, dC = G.T @ E (Loss functions explainer, "How it works" item 2:
-    the logit gradient is p - y; mlx-cross-entropy README, "How it works" item 2:
-    skipped tiles contribute nothing).
+    dE = G @ C, dC = G.T @ E, dbias = column sums of G (Loss functions explainer,
+    "How it works" item 2: the logit gradient is p - y; mlx-cross-entropy README,
+    "How it works" item 2: skipped tiles contribute nothing).
     """
     E64, C64, t = _f64(E), _f64(C), _i64(targets)
     N, V = E64.shape[0], C64.shape[0]
@@ -249,7 +267,7 @@ def backward(E, C, targets, grad_out=1.0, ignore_index: int = -100, reduction: s
     count = int(valid.sum())
     scale = row_scale(t, ignore_index, reduction, grad_out, count)
 
-    z = logits(E64, C64)
+    z = logits(E64, C64, bias)
     lse = log_sum_exp_rows(z)
     p = softmax_rows(z, lse)
     margin = tile_log_margin(z - lse[:, None], valid, tile_m, tile_n)
@@ -262,7 +280,8 @@ def backward(E, C, targets, grad_out=1.0, ignore_index: int = -100, reduction: s
     borderline = 0
     if filter_eps > 0:
         borderline = int((np.abs(margin - math.log(filter_eps)) < window).sum())
-    return BackwardResult(G @ C64, G.T @ E64, int(skip.sum()), borderline, skip.size)
+    return BackwardResult(G @ C64, G.T @ E64, int(skip.sum()), borderline, skip.size,
+                          None if bias is None else G.sum(axis=0))
 
 
 @dataclass
@@ -278,22 +297,25 @@ class SampledResult:
     dE_rows: np.ndarray  # [len(rows), D]
     cols: np.ndarray
     dC_cols: np.ndarray  # [len(cols), D]
+    dbias: Optional[np.ndarray] = None  # [V] when a bias is given and compute_cols
 
 
 def sampled(E, C, targets, rows: Sequence[int], cols: Sequence[int], grad_out=1.0,
             ignore_index: int = -100, reduction: str = "mean", filter_eps: float = 2.0 ** -12,
             tile_m: int = 128, tile_n: int = 256, window: float = 2e-3,
-            compute_cols: bool = True) -> SampledResult:
+            compute_cols: bool = True, bias=None) -> SampledResult:
     """The same definitions as ``forward``/``backward``, evaluated for large problems.
 
     The logits are materialised one row group at a time (rows are independent),
     so memory stays at ``ROW_GROUP * V`` doubles. Every row's LSE, every tile's
     skip decision and the loss are exact; dE is returned for the rows ``rows``
     and dC for the vocabulary rows ``cols`` (dC needs every row's softmax at those
-    columns, so ``compute_cols`` makes this a full pass over all rows).
+    columns, so ``compute_cols`` makes this a full pass over all rows; with a bias
+    that pass also gives every entry of dbias).
     """
     E64, C64, t = _f64(E), _f64(C), _i64(targets)
     N, V = E64.shape[0], C64.shape[0]
+    b = _bias64(bias, V)
     validate_targets(t, V, ignore_index)
     valid = t != ignore_index
     count = int(valid.sum())
@@ -309,11 +331,14 @@ def sampled(E, C, targets, rows: Sequence[int], cols: Sequence[int], grad_out=1.
     margin = np.full((nb, nt), -np.inf)
     dE_rows = np.zeros((len(rows), E64.shape[1]))
     dC_cols = np.zeros((len(cols), E64.shape[1]))
+    dbias = np.zeros(V) if (b is not None and compute_cols) else None
     row_pos = {int(r): i for i, r in enumerate(rows)}
     ln_eps = math.log(filter_eps) if filter_eps > 0 else -math.inf
 
     for g in _row_groups(N):
         z = E64[g] @ C64.T
+        if b is not None:
+            z += b[None, :]
         l = log_sum_exp_rows(z)
         lse[g] = l
         tg, vg = t[g], valid[g]
@@ -334,13 +359,15 @@ def sampled(E, C, targets, rows: Sequence[int], cols: Sequence[int], grad_out=1.
             dE_rows[row_pos[i]] = G[i - g.start] @ C64
         if compute_cols:
             dC_cols += G[:, cols].T @ E64[g]
+            if dbias is not None:
+                dbias += G.sum(axis=0)
         del z, p, G
 
     nll = np.where(valid, lse - zt, 0.0)
     skip_all = filtered_tiles(margin, filter_eps)
     borderline = int((np.abs(margin - ln_eps) < window).sum()) if filter_eps > 0 else 0
     return SampledResult(lse, nll, count, reduce_loss(nll, count, reduction), margin,
-                         int(skip_all.sum()), borderline, rows, dE_rows, cols, dC_cols)
+                         int(skip_all.sum()), borderline, rows, dE_rows, cols, dC_cols, dbias)
 
 
 @dataclass
@@ -355,7 +382,7 @@ class RowBlockResult:
 
 def row_blocks(E, C, targets, blocks: Sequence[int], grad_out=1.0, ignore_index: int = -100,
                reduction: str = "mean", filter_eps: float = 2.0 ** -12, tile_m: int = 128,
-               tile_n: int = 256) -> RowBlockResult:
+               tile_n: int = 256, bias=None) -> RowBlockResult:
     """Exact results for whole row blocks of the tile grid.
 
     A tile's skip decision depends only on the rows of its own row block, and a
@@ -365,6 +392,7 @@ def row_blocks(E, C, targets, blocks: Sequence[int], grad_out=1.0, ignore_index:
     """
     E64, C64, t = _f64(E), _f64(C), _i64(targets)
     N, V = E64.shape[0], C64.shape[0]
+    bv = _bias64(bias, V)
     validate_targets(t, V, ignore_index)
     count = int((t != ignore_index).sum())
     scale_all = row_scale(t, ignore_index, reduction, grad_out, count)
@@ -378,6 +406,8 @@ def row_blocks(E, C, targets, blocks: Sequence[int], grad_out=1.0, ignore_index:
     for b in sorted(blocks):
         rr = np.arange(b * tile_m, min((b + 1) * tile_m, N))
         z = E64[rr] @ C64.T
+        if bv is not None:
+            z += bv[None, :]
         l = log_sum_exp_rows(z)
         tb = t[rr]
         vb = tb != ignore_index

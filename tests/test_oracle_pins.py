@@ -323,3 +323,92 @@ def test_row_block_evaluation_agrees_with_full():
     np.testing.assert_allclose(rb.dE, full.dE[rb.rows], rtol=1e-11, atol=1e-14)
     margin = O.tile_log_margin(O.logits(E, C) - f.lse[:, None], t != -100, 8, 64)
     assert rb.filtered == int(O.filtered_tiles(margin[[1, 4]], 2.0 ** -8).sum())
+
+
+# --- classifier bias (mlx-cross-entropy README, "API" table: bias [V]) -------------------------
+
+@pytest.mark.parametrize("reduction", ["mean", "sum", "none"])
+def test_bias_matches_torch_linear_cross_entropy_float64(reduction):
+    """Library special case: F.linear(e, c, bias) + F.cross_entropy with autograd (filter off)."""
+    E, C, t = _rand_problem(N=40, D=24, V=300, seed=21, ignore=(0, 11, 39))
+    bias = np.random.default_rng(22).standard_normal(300) * 2.0
+    Et = torch.tensor(E, requires_grad=True)
+    Ct = torch.tensor(C, requires_grad=True)
+    bt = torch.tensor(bias, requires_grad=True)
+    tt = torch.tensor(t)
+    out = torch.nn.functional.cross_entropy(torch.nn.functional.linear(Et, Ct, bt), tt, ignore_index=-100,
+                                            reduction=reduction)
+    g = np.random.default_rng(23).standard_normal(len(t)) if reduction == "none" else 1.0
+    (out * torch.tensor(g)).sum().backward()
+    f = O.forward(E, C, t, reduction=reduction, bias=bias)
+    b = O.backward(E, C, t, grad_out=g, reduction=reduction, filter_eps=0.0, bias=bias)
+    np.testing.assert_allclose(np.asarray(f.loss), out.detach().numpy(), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(b.dE, Et.grad.numpy(), rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(b.dC, Ct.grad.numpy(), rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(b.dbias, bt.grad.numpy(), rtol=1e-10, atol=1e-14)
+
+
+def test_bias_finite_differences():
+    N, D, V = 8, 16, 64
+    E, C, t = _rand_problem(N, D, V, seed=24, ignore=(2,))
+    bias = np.random.default_rng(25).standard_normal(V)
+    b = O.backward(E, C, t, filter_eps=0.0, bias=bias)
+    h = 1e-5
+    for v in (0, 5, 31, 63, int(t[0])):
+        bp, bm = bias.copy(), bias.copy()
+        bp[v] += h
+        bm[v] -= h
+        fd = (float(O.forward(E, C, t, bias=bp).loss) - float(O.forward(E, C, t, bias=bm).loss)) / (2 * h)
+        assert abs(fd - b.dbias[v]) <= 1e-7 * max(1.0, abs(fd))
+
+
+def test_bias_shift_invariance_and_zero_sum_gradient():
+    """Softmax is shift invariant: a constant added to every bias entry changes neither the loss
+    nor any gradient, and with filtering off dbias sums to zero (each row of p - y sums to 0)."""
+    E, C, t = _rand_problem(N=20, D=8, V=96, seed=26, ignore=(4,))
+    bias = np.random.default_rng(27).standard_normal(96)
+    f0 = O.forward(E, C, t, bias=bias)
+    f1 = O.forward(E, C, t, bias=bias + 3.5)
+    b0 = O.backward(E, C, t, filter_eps=0.0, bias=bias)
+    b1 = O.backward(E, C, t, filter_eps=0.0, bias=bias + 3.5)
+    assert abs(float(f0.loss) - float(f1.loss)) < 1e-12
+    np.testing.assert_allclose(b0.dE, b1.dE, atol=1e-13)
+    np.testing.assert_allclose(b0.dbias, b1.dbias, atol=1e-13)
+    assert abs(b0.dbias.sum()) < 1e-12
+    # and a zero bias is the same as no bias
+    fz = O.forward(E, C, t, bias=np.zeros(96))
+    assert float(fz.loss) == float(O.forward(E, C, t).loss)
+
+
+def test_bias_only_model_has_closed_form():
+    """E = 0: every row's logits are the bias, so each row's loss is log-sum-exp(bias) - bias[t_r]
+    (computed here with math.fsum, not the oracle's routine) and dbias sums softmax(bias) - onehot
+    over the valid rows, divided by their count."""
+    V = 50
+    bias = np.random.default_rng(28).standard_normal(V) * 3.0
+    t = np.array([3, 3, 17, -100, 49])
+    E = np.zeros((5, 4))
+    C = np.random.default_rng(29).standard_normal((V, 4))
+    m = max(bias)
+    lse = m + math.log(math.fsum(math.exp(x - m) for x in bias))
+    want = math.fsum(lse - bias[k] for k in (3, 3, 17, 49)) / 4
+    assert abs(float(O.forward(E, C, t, bias=bias).loss) - want) < 1e-12
+    p = [math.exp(x - lse) for x in bias]
+    want_db = [(4 * p[v] - sum(1 for k in (3, 3, 17, 49) if k == v)) / 4 for v in range(V)]
+    np.testing.assert_allclose(O.backward(E, C, t, filter_eps=0.0, bias=bias).dbias, want_db, atol=1e-13)
+
+
+def test_bias_sampled_and_row_blocks_agree_with_full(monkeypatch):
+    monkeypatch.setattr(O, "ROW_GROUP", 16)
+    E, C, t = _rand_problem(N=48, D=12, V=256, seed=30, ignore=(0, 17))
+    E = E * 2.0
+    bias = np.random.default_rng(31).standard_normal(256)
+    full_f = O.forward(E, C, t, bias=bias)
+    full_b = O.backward(E, C, t, grad_out=0.7, filter_eps=2.0 ** -8, tile_m=8, tile_n=64, bias=bias)
+    s = O.sampled(E, C, t, [1, 40], [0, 200], grad_out=0.7, filter_eps=2.0 ** -8, tile_m=8, tile_n=64, bias=bias)
+    np.testing.assert_allclose(s.lse, full_f.lse, rtol=1e-13)
+    np.testing.assert_allclose(s.dE_rows, full_b.dE[[1, 40]], rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(s.dC_cols, full_b.dC[[0, 200]], rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(s.dbias, full_b.dbias, rtol=1e-11, atol=1e-14)
+    rb = O.row_blocks(E, C, t, [2], grad_out=0.7, filter_eps=2.0 ** -8, tile_m=8, tile_n=64, bias=bias)
+    np.testing.assert_allclose(rb.dE, full_b.dE[16:24], rtol=1e-11, atol=1e-14)
