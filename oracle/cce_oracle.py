@@ -124,7 +124,8 @@ def softmax_rows(z: np.ndarray, lse: np.ndarray) -> np.ndarray:
     return np.exp(z - lse[:, None])
 
 
-def _row_groups(n: int, group: int = ROW_GROUP) -> Iterator[slice]:
+def _row_groups(n: int, group: Optional[int] = None) -> Iterator[slice]:
+    group = ROW_GROUP if group is None else group  # read at call time (tests shrink it)
     for r0 in range(0, n, group):
         yield slice(r0, min(r0 + group, n))
 
@@ -315,7 +316,7 @@ def sampled(E, C, targets, rows: Sequence[int], cols: Sequence[int], grad_out=1.
     """
     E64, C64, t = _f64(E), _f64(C), _i64(targets)
     N, V = E64.shape[0], C64.shape[0]
-    b = _bias64(bias, V)
+    bv = _bias64(bias, V)
     validate_targets(t, V, ignore_index)
     valid = t != ignore_index
     count = int(valid.sum())
@@ -331,14 +332,14 @@ def sampled(E, C, targets, rows: Sequence[int], cols: Sequence[int], grad_out=1.
     margin = np.full((nb, nt), -np.inf)
     dE_rows = np.zeros((len(rows), E64.shape[1]))
     dC_cols = np.zeros((len(cols), E64.shape[1]))
-    dbias = np.zeros(V) if (b is not None and compute_cols) else None
+    dbias = np.zeros(V) if (bv is not None and compute_cols) else None
     row_pos = {int(r): i for i, r in enumerate(rows)}
     ln_eps = math.log(filter_eps) if filter_eps > 0 else -math.inf
 
     for g in _row_groups(N):
         z = E64[g] @ C64.T
-        if b is not None:
-            z += b[None, :]
+        if bv is not None:
+            z += bv[None, :]
         l = log_sum_exp_rows(z)
         lse[g] = l
         tg, vg = t[g], valid[g]

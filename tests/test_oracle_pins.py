@@ -412,3 +412,25 @@ def test_bias_sampled_and_row_blocks_agree_with_full(monkeypatch):
     np.testing.assert_allclose(s.dbias, full_b.dbias, rtol=1e-11, atol=1e-14)
     rb = O.row_blocks(E, C, t, [2], grad_out=0.7, filter_eps=2.0 ** -8, tile_m=8, tile_n=64, bias=bias)
     np.testing.assert_allclose(rb.dE, full_b.dE[16:24], rtol=1e-11, atol=1e-14)
+
+
+def test_sampled_with_skips_in_every_row_group(monkeypatch):
+    """Several row groups, each with skipped tiles, with and without a bias: the group loop's
+    per-tile bookkeeping must not disturb the next group."""
+    monkeypatch.setattr(O, "ROW_GROUP", 16)
+    rng = np.random.default_rng(32)
+    N, D, V = 64, 32, 2048
+    C = rng.standard_normal((V, D)) / np.sqrt(D)
+    t = rng.integers(0, V, N)
+    t[5] = -100
+    E = 24.0 * C[np.where(t >= 0, t, 0)] + rng.standard_normal((N, D))  # peaked: most tiles skipped
+    for bias in (None, np.random.default_rng(33).standard_normal(V) * 0.5):
+        full = O.backward(E, C, t, filter_eps=2.0 ** -12, tile_m=8, tile_n=64, bias=bias)
+        lse = O.forward(E, C, t, bias=bias).lse
+        skip = O.filtered_tiles(O.tile_log_margin(O.logits(E, C, bias) - lse[:, None], t != -100, 8, 64), 2.0 ** -12)
+        assert all(skip[2 * k:2 * k + 2].any() for k in range(4)), "every 16-row group must hold a skipped tile"
+        s = O.sampled(E, C, t, [3, 60], [1, 2000], filter_eps=2.0 ** -12, tile_m=8, tile_n=64, bias=bias)
+        assert s.filtered == full.filtered
+        np.testing.assert_allclose(s.lse, lse, rtol=1e-13)
+        np.testing.assert_allclose(s.dE_rows, full.dE[[3, 60]], rtol=1e-11, atol=1e-14)
+        np.testing.assert_allclose(s.dC_cols, full.dC[[1, 2000]], rtol=1e-11, atol=1e-14)
