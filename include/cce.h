@@ -5,7 +5,8 @@
  * README, "How it works" and "API"): hidden states E [N, D], classifier C [V, D] and targets
  * t [N]. Logits z = E C^T never reach global memory. The forward returns the cross-entropy loss
  * and the per-row log-sum-exp (LSE). The backward recomputes logit tiles, skips tiles whose
- * softmax is below filter_eps (2^-12 by default), and returns dE and dC.
+ * softmax is below filter_eps (2^-12 by default), and returns dE and dC. An optional classifier
+ * bias [V] is added to every row of logits (z = E C^T + bias); its gradient is returned too.
  *
  * Conventions for every call:
  *  - Pointers marked "device" are CUDA device pointers of the current device. The caller owns
@@ -80,18 +81,21 @@ CCE_API void cce_backward_tile_shape(int32_t* tile_rows, int32_t* tile_cols);
 /* Bytes of device workspace cce_forward() needs (0 for a bad problem). */
 CCE_API size_t cce_forward_workspace_size(const cce_problem* p);
 
-/* Bytes of device workspace cce_backward() needs. With out_fp32 = 0 it holds the fp32
- * accumulators of dE and dC, (N + V) * D * 4 bytes; never anything of size N * V. */
+/* Bytes of device workspace cce_backward() needs: the tile plan (about 37 bytes per 128 x 128
+ * tile), the gradient tiles of two vocabulary chunks (4 MiB per 128 rows, at least 128 MiB) and,
+ * with out_fp32 = 0, the fp32 accumulators of dE and dbias, (N * D + V) * 4 bytes. Never anything
+ * of size N * V. */
 CCE_API size_t cce_backward_workspace_size(const cce_problem* p, int32_t out_fp32);
 
 /*
- * Forward: loss and per-row LSE without materialising the logits.
+ * Forward: loss and per-row LSE without materialising the logits z = E C^T + bias.
  * Cut Your Losses abstract (only the correct token's logit is computed; the log-sum-exp over
  * the vocabulary is evaluated on the fly); Cut Cross Entropy from first principles
  * (loss = LSE - z_correct); mlx-cross-entropy README, "How it works" item 1 (tile-wise max and
- * sum-exp) and "API" (reduction, ignore_index).
+ * sum-exp) and "API" (bias, reduction, ignore_index).
  *
  *  E        device bf16 [N, D]          C       device bf16 [V, D]
+ *  bias     device bf16 [V], added to every row of logits; NULL for none
  *  targets  device int64 [N]
  *  loss     device fp32: [1] for mean/sum, [N] for none (0 at ignored tokens)
  *  lse      device fp32 [N]: log-sum-exp of each row's logits (computed for ignored rows too)
@@ -101,12 +105,13 @@ CCE_API size_t cce_backward_workspace_size(const cce_problem* p, int32_t out_fp3
  *           it also holds the device error word read by cce_check_device_error().
  * N = 0 is allowed (loss 0, count 0).
  */
-CCE_API cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
-                       float* loss, float* lse, float* tile_max, int64_t* count, void* workspace,
-                       size_t workspace_bytes, cce_stream_t stream);
+CCE_API cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const void* bias,
+                               const int64_t* targets, float* loss, float* lse, float* tile_max, int64_t* count,
+                               void* workspace, size_t workspace_bytes, cce_stream_t stream);
 
 /*
- * Backward: dE = G C and dC = G^T E with G = scale_r * (p~ - onehot), p = softmax(z),
+ * Backward: dE = G C, dC = G^T E and dbias = sum_r G[r, :] with G = scale_r * (p~ - onehot),
+ * p = softmax(z),
  * recomputed tile by tile from E, C and the saved LSE. p~ is p with every skipped tile set to 0:
  * a tile (tile_rows x tile_cols, see cce_backward_tile_shape) is skipped when, for every
  * non-ignored row r in it, max over its columns of z[r, v] - LSE[r] < ln(filter_eps); a tile
@@ -115,18 +120,20 @@ CCE_API cce_status cce_forward(const cce_problem* p, const void* E, const void* 
  * mlx-cross-entropy README, "How it works" items 2 and 3 (skipping, accumulation).
  * scale_r = g / max(count, 1) (mean), g (sum) or g[r] (none); 0 for ignored rows.
  *
- *  E, C, targets, lse, tile_max, count: as produced/consumed by cce_forward() on the same problem
+ *  E, C, bias, targets, lse, tile_max, count: as given to / produced by cce_forward() on the
+ *           same problem (bias NULL for none)
  *  grad_out device fp32: [1] for mean/sum, [N] for none
- *  dE       device [N, D], dC device [V, D]: bf16 when out_fp32 = 0, fp32 when out_fp32 = 1.
- *           Fully overwritten. Rows of ignored tokens in dE are exactly +0.
+ *  dE       device [N, D], dC device [V, D], dbias device [V] or NULL (not computed): bf16 when
+ *           out_fp32 = 0, fp32 when out_fp32 = 1. Fully overwritten. Rows of ignored tokens in dE
+ *           are exactly +0. dbias is the gradient of the bias (also when bias is NULL, i.e. zero).
  *  filtered_tiles device int64 [1]: number of skipped tiles
  *  workspace: device scratch of at least cce_backward_workspace_size(p, out_fp32) bytes.
  */
-CCE_API cce_status cce_backward(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
-                        const float* lse, const float* tile_max, const int64_t* count,
-                        const float* grad_out, float filter_eps, void* dE, void* dC, int32_t out_fp32,
-                        int64_t* filtered_tiles, void* workspace, size_t workspace_bytes,
-                        cce_stream_t stream);
+CCE_API cce_status cce_backward(const cce_problem* p, const void* E, const void* C, const void* bias,
+                                const int64_t* targets, const float* lse, const float* tile_max,
+                                const int64_t* count, const float* grad_out, float filter_eps, void* dE, void* dC,
+                                void* dbias, int32_t out_fp32, int64_t* filtered_tiles, void* workspace,
+                                size_t workspace_bytes, cce_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device error word kept at the start of
  * `workspace` (a forward or backward workspace passed to an earlier call on that stream).
@@ -158,9 +165,9 @@ CCE_API const char* cce_last_error_message(void);
  *  - Device-side errors (a target outside [0, V)) are not reported by this variant; use
  *    cce_forward() and cce_check_device_error() to diagnose them.
  */
-CCE_API cce_status cce_forward_noalloc(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
-                                       float* loss, float* lse, float* tile_max, int64_t* count,
-                                       cce_stream_t stream);
+CCE_API cce_status cce_forward_noalloc(const cce_problem* p, const void* E, const void* C, const void* bias,
+                                       const int64_t* targets, float* loss, float* lse, float* tile_max,
+                                       int64_t* count, cce_stream_t stream);
 
 /* Optional instrumentation, off by default and per calling thread. When an event pair is set
  * (cudaEvent_t handles created by the caller; NULL clears), cce_forward() records fwd_start and

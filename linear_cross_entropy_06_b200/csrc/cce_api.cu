@@ -17,7 +17,7 @@
 
 namespace {
 
-constexpr int32_t kVersion = 100;  // 0.1.0
+constexpr int32_t kVersion = 200;  // 0.2.0: classifier bias
 constexpr size_t kHeaderBytes = 256;
 constexpr size_t kAlign = 256;
 
@@ -104,6 +104,7 @@ struct SplitWs {
   uint8_t* gscratch; // kGradBuffers * buf_bytes
   size_t buf_bytes;
   float* dE_acc;
+  float* dbias_acc;  // [V] fp32 (absent with out_fp32)
   size_t bytes;
 };
 
@@ -156,7 +157,10 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.sync = reinterpret_cast<int*>(take(w.sync_bytes));
   w.buf_bytes = static_cast<size_t>(nb * chunk_vt) * cce::kGradTileBytes;
   w.gscratch = reinterpret_cast<uint8_t*>(take(cce::kGradBuffers * w.buf_bytes));
-  if (!out_fp32) w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
+  if (!out_fp32) {
+    w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
+    w.dbias_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->V)));
+  }
   w.bytes = off;
   return w;
 }
@@ -231,10 +235,10 @@ uint64_t wait_timeout_ns() {
 
 // The backward: plan the tiles and work lists, then one persistent launch (cce_bwd.cu) forms the
 // gradient tiles chunk by chunk and runs the dC and dE MMAs from them.
-cce_status backward_split(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
+cce_status backward_split(const cce_problem* p, const void* E, const void* C, const void* bias, const int64_t* targets,
                           const float* lse, const float* tile_max, const int64_t* count, const float* grad_out,
-                          float filter_eps, void* dE, void* dC, int32_t out_fp32, int64_t* filtered_tiles,
-                          void* workspace, size_t workspace_bytes, cudaStream_t s) {
+                          float filter_eps, void* dE, void* dC, void* dbias, int32_t out_fp32,
+                          int64_t* filtered_tiles, void* workspace, size_t workspace_bytes, cudaStream_t s) {
   const SplitWs w = carve_split(p, out_fp32, workspace);
   if (workspace_bytes < w.bytes)
     return fail(CCE_ERR_WORKSPACE, "backward workspace is %zu bytes, needs %zu", workspace_bytes, w.bytes);
@@ -243,10 +247,12 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   CCE_CHECK(get_encoder());
   const int64_t N = p->N, D = p->D, V = p->V, T = ceil_div(V, cce::kSubTile);
   float* dE_acc = out_fp32 ? static_cast<float*>(dE) : w.dE_acc;
+  float* dbias_acc = dbias == nullptr ? nullptr : (out_fp32 ? static_cast<float*>(dbias) : w.dbias_acc);
 
   CCE_TRY(cudaMemsetAsync(w.hdr, 0, sizeof(WsHeader), s));
-  if (N == 0) {  // no rows: dC = 0
+  if (N == 0) {  // no rows: dC = 0 (and dbias = 0)
     CCE_TRY(cce::launch_fill_zero(dC, V * D * (out_fp32 ? 4 : 2), s));
+    if (dbias != nullptr) CCE_TRY(cce::launch_fill_zero(dbias, V * (out_fp32 ? 4 : 2), s));
     return cudaMemsetAsync(filtered_tiles, 0, sizeof(int64_t), s) == cudaSuccess ? CCE_OK
                                                                                   : fail(CCE_ERR_CUDA, "memset");
   }
@@ -254,6 +260,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   CCE_TRY(cce::launch_bwd_plan(w.plan, tile_max, lse, targets, N, V, T, p->ignore_index, filter_eps, filtered_tiles,
                                s));
   CCE_TRY(cce::launch_fill_zero(dE_acc, N * D * 4, s));
+  if (dbias_acc != nullptr) CCE_TRY(cce::launch_fill_zero(dbias_acc, V * 4, s));
   CCE_TRY(cudaMemsetAsync(w.sync, 0, w.sync_bytes, s));
 
   cce::BwdLaunch L{};
@@ -278,6 +285,8 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.lse = lse;
   A.scale = w.scale;
   A.targets = targets;
+  A.bias = static_cast<const __nv_bfloat16*>(bias);
+  A.dbias = dbias_acc;
   A.grp_start = w.plan.grp_start;
   A.chunk_t = w.plan.chunk_t;
   A.pstart_t = w.plan.pstart_t;
@@ -301,6 +310,8 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   CCE_TRY(cce::launch_bwd(L, s));
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
   if (!out_fp32) CCE_TRY(cce::launch_to_bf16(dE_acc, static_cast<__nv_bfloat16*>(dE), N * D, s));
+  if (!out_fp32 && dbias != nullptr)
+    CCE_TRY(cce::launch_to_bf16(dbias_acc, static_cast<__nv_bfloat16*>(dbias), V, s));
   return CCE_OK;
 }
 
@@ -360,17 +371,17 @@ size_t cce_backward_workspace_size(const cce_problem* p, int32_t out_fp32) {
   return carve_split(p, out_fp32 ? 1 : 0, nullptr).bytes;
 }
 
-cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const int64_t* targets, float* loss,
-                       float* lse, float* tile_max, int64_t* count, void* workspace, size_t workspace_bytes,
-                       cce_stream_t stream) {
+cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const void* bias, const int64_t* targets,
+                       float* loss, float* lse, float* tile_max, int64_t* count, void* workspace,
+                       size_t workspace_bytes, cce_stream_t stream) {
   g_last_error.clear();
   if (!problem_ok(p, true)) return CCE_ERR_INVALID_ARG;
   const bool has_rows = p->N > 0;
   if (C == nullptr || loss == nullptr || count == nullptr || workspace == nullptr ||
       (has_rows && (E == nullptr || targets == nullptr || lse == nullptr || tile_max == nullptr)))
     return fail(CCE_ERR_INVALID_ARG, "a required pointer is NULL");
-  if (!aligned16(E) || !aligned16(C) || !aligned16(workspace))
-    return fail(CCE_ERR_INVALID_ARG, "E, C and workspace must be 16-byte aligned");
+  if (!aligned16(E) || !aligned16(C) || !aligned16(bias) || !aligned16(workspace))
+    return fail(CCE_ERR_INVALID_ARG, "E, C, bias and workspace must be 16-byte aligned");
   const FwdWs w = carve_fwd(p, workspace);
   if (workspace_bytes < w.bytes)
     return fail(CCE_ERR_WORKSPACE, "forward workspace is %zu bytes, needs %zu", workspace_bytes, w.bytes);
@@ -381,10 +392,12 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
   const int64_t N = p->N, D = p->D, V = p->V, T = ceil_div(V, cce::kSubTile);
   const auto* Eb = static_cast<const __nv_bfloat16*>(E);
   const auto* Cb = static_cast<const __nv_bfloat16*>(C);
+  const auto* Bb = static_cast<const __nv_bfloat16*>(bias);
 
   CCE_TRY(cudaMemsetAsync(w.hdr, 0, sizeof(WsHeader), s));
   if (has_rows) {
     cce::FwdLaunch L{};
+    L.bias = Bb;
     CCE_CHECK(make_map(&L.tmE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kFwdBM));
     CCE_CHECK(make_map(&L.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, cce::kFwdBN));
     L.N = static_cast<int>(N);
@@ -400,7 +413,7 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
     // (reported as CCE_ERR_DEVICE_TIMEOUT by cce_check_device_error; the outputs are undefined).
     const char* stall = std::getenv("CCE_TEST_INJECT_STALL");
     L.inject_stall = (stall != nullptr && stall[0] == '1') ? 1 : 0;
-    CCE_TRY(cce::launch_target_logit(Eb, Cb, targets, N, D, V, p->ignore_index, w.z_target, &w.hdr->err, s));
+    CCE_TRY(cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, p->ignore_index, w.z_target, &w.hdr->err, s));
     if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[0], s));
     CCE_TRY(cce::launch_fwd_lse(L, s));
     if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[1], s));
@@ -412,10 +425,10 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
   return CCE_OK;
 }
 
-cce_status cce_backward(const cce_problem* p, const void* E, const void* C, const int64_t* targets, const float* lse,
-                        const float* tile_max, const int64_t* count, const float* grad_out, float filter_eps,
-                        void* dE, void* dC, int32_t out_fp32, int64_t* filtered_tiles, void* workspace,
-                        size_t workspace_bytes, cce_stream_t stream) {
+cce_status cce_backward(const cce_problem* p, const void* E, const void* C, const void* bias, const int64_t* targets,
+                        const float* lse, const float* tile_max, const int64_t* count, const float* grad_out,
+                        float filter_eps, void* dE, void* dC, void* dbias, int32_t out_fp32,
+                        int64_t* filtered_tiles, void* workspace, size_t workspace_bytes, cce_stream_t stream) {
   g_last_error.clear();
   if (!problem_ok(p, true)) return CCE_ERR_INVALID_ARG;
   const bool has_rows = p->N > 0;
@@ -423,11 +436,12 @@ cce_status cce_backward(const cce_problem* p, const void* E, const void* C, cons
       (has_rows && (E == nullptr || targets == nullptr || lse == nullptr || tile_max == nullptr || dE == nullptr ||
                     grad_out == nullptr)))
     return fail(CCE_ERR_INVALID_ARG, "a required pointer is NULL");
-  if (!aligned16(E) || !aligned16(C) || !aligned16(dE) || !aligned16(dC) || !aligned16(workspace))
-    return fail(CCE_ERR_INVALID_ARG, "E, C, dE, dC and workspace must be 16-byte aligned");
+  if (!aligned16(E) || !aligned16(C) || !aligned16(bias) || !aligned16(dE) || !aligned16(dC) ||
+      !aligned16(dbias) || !aligned16(workspace))
+    return fail(CCE_ERR_INVALID_ARG, "E, C, bias, dE, dC, dbias and workspace must be 16-byte aligned");
   if (std::isnan(filter_eps)) return fail(CCE_ERR_INVALID_ARG, "filter_eps is NaN");
   out_fp32 = out_fp32 ? 1 : 0;
-  return backward_split(p, E, C, targets, lse, tile_max, count, grad_out, filter_eps, dE, dC, out_fp32,
+  return backward_split(p, E, C, bias, targets, lse, tile_max, count, grad_out, filter_eps, dE, dC, dbias, out_fp32,
                         filtered_tiles, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -36,8 +36,9 @@ __device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
 
 // One warp per row; lanes read 16-byte pieces, so a warp reads 512 contiguous bytes per step.
 __global__ void target_logit_kernel(const __nv_bfloat16* __restrict__ E, const __nv_bfloat16* __restrict__ C,
-                                    const int64_t* __restrict__ targets, int64_t N, int64_t D, int64_t V,
-                                    int64_t ignore_index, float* __restrict__ z_target, int* err) {
+                                    const __nv_bfloat16* __restrict__ bias, const int64_t* __restrict__ targets,
+                                    int64_t N, int64_t D, int64_t V, int64_t ignore_index,
+                                    float* __restrict__ z_target, int* err) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= N) return;
@@ -59,7 +60,7 @@ __global__ void target_logit_kernel(const __nv_bfloat16* __restrict__ E, const _
   }
   if (d < D) acc0 = dot8_bf16(ld_global_nc_v4(e + d), ld_global_nc_v4(c + d), acc0);
   const float s = warp_sum(acc0 + acc1);
-  if (lane == 0) z_target[row] = s;
+  if (lane == 0) z_target[row] = bias != nullptr ? s + __bfloat162float(bias[t]) : s;
 }
 
 __device__ __forceinline__ void lse_merge(float& M, float& S, float m, float s) {
@@ -160,9 +161,12 @@ __global__ void row_scale_kernel(const int64_t* __restrict__ targets, const int6
   scale[r] = (targets[r] != ignore_index) ? s : 0.f;
 }
 
-__global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t n8) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+// Eight elements per thread and step (16-byte stores), then the last n % 8 one by one.
+__global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t n) {
+  const int64_t n8 = n / 8;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (tid < n - 8 * n8) dst[8 * n8 + tid] = __float2bfloat16_rn(src[8 * n8 + tid]);
+  for (int64_t i = tid; i < n8; i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const float4 a = reinterpret_cast<const float4*>(src)[2 * i];
     const float4 b = reinterpret_cast<const float4*>(src)[2 * i + 1];
     uint4 o;
@@ -174,10 +178,12 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __r
   }
 }
 
-__global__ void fill_zero_kernel(uint4* __restrict__ dst, int64_t n16) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    dst[i] = make_uint4(0, 0, 0, 0);
+// 16 bytes per thread and step, then the last bytes % 16 one by one.
+__global__ void fill_zero_kernel(uint4* __restrict__ dst, int64_t bytes) {
+  const int64_t n16 = bytes / 16;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (tid < bytes - 16 * n16) reinterpret_cast<uint8_t*>(dst)[16 * n16 + tid] = 0;
+  for (int64_t i = tid; i < n16; i += static_cast<int64_t>(gridDim.x) * blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
 }
 
 int grid_for(int64_t items, int per_block, int cap) {
@@ -187,12 +193,12 @@ int grid_for(int64_t items, int per_block, int cap) {
 
 }  // namespace
 
-cudaError_t launch_target_logit(const __nv_bfloat16* E, const __nv_bfloat16* C, const int64_t* targets, int64_t N,
-                                int64_t D, int64_t V, int64_t ignore_index, float* z_target, int* err,
-                                cudaStream_t s) {
+cudaError_t launch_target_logit(const __nv_bfloat16* E, const __nv_bfloat16* C, const __nv_bfloat16* bias,
+                                const int64_t* targets, int64_t N, int64_t D, int64_t V, int64_t ignore_index,
+                                float* z_target, int* err, cudaStream_t s) {
   if (N == 0) return cudaSuccess;
   const int grid = static_cast<int>((N + 7) / 8);
-  target_logit_kernel<<<grid, 256, 0, s>>>(E, C, targets, N, D, V, ignore_index, z_target, err);
+  target_logit_kernel<<<grid, 256, 0, s>>>(E, C, bias, targets, N, D, V, ignore_index, z_target, err);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -226,16 +232,16 @@ cudaError_t launch_row_scale(const int64_t* targets, const int64_t* count, const
 
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, int64_t n, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
-  const int64_t n8 = n / 8;  // n is a multiple of 8 (D is)
-  to_bf16_kernel<<<grid_for(n8, 256, 148 * 16), 256, 0, s>>>(src, dst, n8);
+  // src and dst 16-byte aligned; the tail of fewer than 8 elements is taken by the first threads
+  to_bf16_kernel<<<grid_for(n / 8, 256, 148 * 16), 256, 0, s>>>(src, dst, n);
   note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fill_zero(void* dst, int64_t bytes, cudaStream_t s) {
   if (bytes == 0) return cudaSuccess;
-  const int64_t n16 = bytes / 16;  // callers pass multiples of 16 bytes
-  fill_zero_kernel<<<grid_for(n16, 256, 148 * 16), 256, 0, s>>>(static_cast<uint4*>(dst), n16);
+  // dst 16-byte aligned; the tail of fewer than 16 bytes is taken by the first threads
+  fill_zero_kernel<<<grid_for(bytes / 16, 256, 148 * 16), 256, 0, s>>>(static_cast<uint4*>(dst), bytes);
   note_launches(1);
   return cudaGetLastError();
 }

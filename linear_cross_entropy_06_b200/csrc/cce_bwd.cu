@@ -485,15 +485,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < BN / 32; ++c) {
             float v[32];
+            const int col0 = vb + c * 32;
             if (kept) {
               tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * 2 * BN + u * BN + c * 32), v);
+              if (A.bias != nullptr) add_bias32(v, A.bias, col0, A.V);
 #pragma unroll
               for (int e = 0; e < 32; ++e) v[e] = sc * exp2f(fmaf(v[e], kLog2e, -lse_l2));
             } else {
 #pragma unroll
               for (int e = 0; e < 32; ++e) v[e] = 0.f;
             }
-            const int col0 = vb + c * 32;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               if (c * 32 + e == tcol) v[e] -= sc;
@@ -506,6 +507,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               st_shared_v4(blk + swz(row, ch), pack_bf16x2(v[8 * h + 0], v[8 * h + 1]),
                            pack_bf16x2(v[8 * h + 2], v[8 * h + 3]), pack_bf16x2(v[8 * h + 4], v[8 * h + 5]),
                            pack_bf16x2(v[8 * h + 6], v[8 * h + 7]));
+            }
+            if (A.dbias != nullptr) {  // dbias += column sums of G (this warp's 32 rows), fp32
+              const float cs = warp_column_sums32(v, lane);
+              if (col0 + lane < A.V && cs != 0.f) atomicAdd(A.dbias + col0 + lane, cs);
             }
           }
           fence_proxy_async_smem();

@@ -279,10 +279,50 @@ __device__ __forceinline__ uint4 ld_global_nc_v4(const void* p) {
   return v;
 }
 
+// v[i] += bias[col0 + i] for the 32 columns from col0 that lie below V (bias: bf16 [V], 16-byte
+// aligned; col0 a multiple of 32, so the full-width case is four 16-byte loads).
+__device__ __forceinline__ void add_bias32(float (&v)[32], const __nv_bfloat16* bias, int col0, int V) {
+  if (col0 + 32 <= V) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 u = ld_global_nc_v4(bias + col0 + 8 * q);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __nv_bfloat162 h;
+        *reinterpret_cast<uint32_t*>(&h) = w[k];
+        v[8 * q + 2 * k] += __low2float(h);
+        v[8 * q + 2 * k + 1] += __high2float(h);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (col0 + i < V) v[i] += __bfloat162float(bias[col0 + i]);
+  }
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
+}
+
+// Column sums of a warp's 32 x 32 block (lane = row, v[i] = column i): afterwards lane l returns
+// the sum over the 32 lanes of v[l]. Recursive halving: at each step a lane keeps half of its
+// partial sums and adds the partner's matching half, 31 shuffles in all. Clobbers v.
+__device__ __forceinline__ float warp_column_sums32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? v[i] : v[i + off];
+      const float keep = upper ? v[i + off] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
 }
 
 __device__ __forceinline__ float warp_max(float v) {

@@ -53,8 +53,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_lse_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC, int N, int D,
-                   int V, int T, float* __restrict__ tile_max, float* __restrict__ tile_sum, int* err,
-                   uint64_t timeout_ns, int inject_stall) {
+                   int V, int T, const __nv_bfloat16* __restrict__ bias, float* __restrict__ tile_max,
+                   float* __restrict__ tile_sum, int* err, uint64_t timeout_ns, int inject_stall) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm = carve(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -195,6 +195,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           float v[32];
           tmem_ld32(tbase + static_cast<uint32_t>(sub * kSubTile + c * 32), v);
           const int col0 = t * BN + sub * kSubTile + c * 32;
+          if (bias != nullptr) add_bias32(v, bias, col0, V);
           if (col0 + 32 > V) {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
@@ -244,8 +245,8 @@ cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(fwd_lse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(total < L.num_sms ? total : L.num_sms);
-  fwd_lse_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmC, L.N, L.D, L.V, L.T, L.tile_max, L.tile_sum,
-                                                       L.err, L.timeout_ns, L.inject_stall);
+  fwd_lse_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmC, L.N, L.D, L.V, L.T, L.bias, L.tile_max,
+                                                       L.tile_sum, L.err, L.timeout_ns, L.inject_stall);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -21,6 +21,7 @@ struct FwdLaunch {
   CUtensorMap tmE;  // bf16 [N, D], box 64 x 128, 128B swizzle
   CUtensorMap tmC;  // bf16 [V, D], box 64 x 256, 128B swizzle
   int N, D, V, T;   // T = ceil(V / 128)
+  const __nv_bfloat16* bias;  // [V] added to every row of logits, or null
   float* tile_max;  // [T, N]
   float* tile_sum;  // [T, N]: sum over the sub-tile of exp(z - tile_max)
   int* err;
@@ -85,6 +86,8 @@ struct BwdArgs {
   const float* lse;
   const float* scale;
   const int64_t* targets;
+  const __nv_bfloat16* bias;  // [V] or null
+  float* dbias;               // [V] fp32 accumulator of the column sums of G, or null
   const int* grp_start;
   const int* chunk_t;
   const int* pstart_t;
@@ -120,9 +123,9 @@ cudaError_t launch_bwd(const BwdLaunch& L, cudaStream_t s);
 cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
 
 // Small kernels (cce_aux.cu).
-cudaError_t launch_target_logit(const __nv_bfloat16* E, const __nv_bfloat16* C, const int64_t* targets, int64_t N,
-                                int64_t D, int64_t V, int64_t ignore_index, float* z_target, int* err,
-                                cudaStream_t s);
+cudaError_t launch_target_logit(const __nv_bfloat16* E, const __nv_bfloat16* C, const __nv_bfloat16* bias,
+                                const int64_t* targets, int64_t N, int64_t D, int64_t V, int64_t ignore_index,
+                                float* z_target, int* err, cudaStream_t s);
 cudaError_t launch_lse_loss(const float* tile_max, const float* tile_sum, const float* z_target,
                             const int64_t* targets, int64_t N, int64_t T, int64_t ignore_index, int64_t V,
                             float* lse, float* loss_rows, cudaStream_t s);

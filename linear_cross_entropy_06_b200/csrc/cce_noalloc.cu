@@ -86,9 +86,9 @@ cce_status encode(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols,
 
 }  // namespace
 
-extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, const void* C, const int64_t* targets,
-                                          float* loss, float* lse, float* tile_max, int64_t* count,
-                                          cce_stream_t stream) {
+extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, const void* C, const void* bias,
+                                          const int64_t* targets, float* loss, float* lse, float* tile_max,
+                                          int64_t* count, cce_stream_t stream) {
   cce::set_last_error("");
   if (p == nullptr || p->N < 0 || p->D < 8 || p->D % 8 != 0 || p->V < 1 || p->reduction < 0 || p->reduction > 2 ||
       p->reserved != 0 || p->N >= (int64_t(1) << 31) - 256 || p->V >= (int64_t(1) << 31) - 256 ||
@@ -99,8 +99,8 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   if (C == nullptr || loss == nullptr || count == nullptr ||
       (N > 0 && (E == nullptr || targets == nullptr || lse == nullptr || tile_max == nullptr)))
     return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: a required pointer is NULL");
-  if ((reinterpret_cast<uintptr_t>(E) | reinterpret_cast<uintptr_t>(C)) & 15u)
-    return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: E and C must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(E) | reinterpret_cast<uintptr_t>(C) | reinterpret_cast<uintptr_t>(bias)) & 15u)
+    return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: E, C and bias must be 16-byte aligned");
   // Same layout as the forward workspace: header | tile_sum [T, N] | z_target [N] | loss_rows [N].
   const size_t off_sum = kHeader;
   const size_t off_zt = up(off_sum + sizeof(float) * static_cast<size_t>(T * N));
@@ -126,6 +126,7 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const auto* Eb = static_cast<const __nv_bfloat16*>(E);
   const auto* Cb = static_cast<const __nv_bfloat16*>(C);
+  const auto* Bb = static_cast<const __nv_bfloat16*>(bias);
 
   // The array keeps the previous call's contents: the error word must start at zero; every other
   // scratch value is written before it is read.
@@ -144,7 +145,8 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
     L.timeout_ns = 4000000000ull;
     L.num_sms = num_sms;
     L.inject_stall = 0;
-    if (cce::launch_target_logit(Eb, Cb, targets, N, D, V, p->ignore_index, z_target, err, s) != cudaSuccess ||
+    L.bias = Bb;
+    if (cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, p->ignore_index, z_target, err, s) != cudaSuccess ||
         cce::launch_fwd_lse(L, s) != cudaSuccess ||
         cce::launch_lse_loss(tile_max, tile_sum, z_target, targets, N, T, p->ignore_index, V, lse,
                              p->reduction == CCE_REDUCTION_NONE ? loss : loss_rows, s) != cudaSuccess)

@@ -6,7 +6,7 @@ The library is loaded on first use; a missing library or a machine without a
 CUDA device raises ``CCEError`` (there is no fallback of any kind).
 
 API shape follows the mlx-cross-entropy README ("API" table and "Usage"):
-``linear_cross_entropy(e, c, targets, reduction="mean", ignore_index=-100)`` with
+``linear_cross_entropy(e, c, targets, bias=None, reduction="mean", ignore_index=-100)`` with
 ``[..., D]`` hidden states flattened to ``[N, D]`` and, for ``reduction="none"``,
 the per-token loss returned in the targets' shape.
 """
@@ -59,15 +59,16 @@ SIGNATURES = {
     "cce_backward_tile_shape": (None, [ctypes.POINTER(_I32), ctypes.POINTER(_I32)]),
     "cce_forward_workspace_size": (_SZ, [_PP]),
     "cce_backward_workspace_size": (_SZ, [_PP, _I32]),
-    "cce_forward": (_I32, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
-    "cce_backward": (_I32, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _F32, _VP, _VP, _I32, _VP, _VP, _SZ, _VP]),
+    "cce_forward": (_I32, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "cce_backward": (_I32, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _F32, _VP, _VP, _VP, _I32, _VP, _VP, _SZ,
+                            _VP]),
     "cce_check_device_error": (_I32, [_VP, _VP]),
     "cce_status_string": (ctypes.c_char_p, [_I32]),
     "cce_last_error_message": (ctypes.c_char_p, []),
     "cce_version": (_I32, []),
     "cce_set_kernel_events": (None, [_VP, _VP, _VP, _VP]),
     "cce_kernel_launch_count": (_I64, []),
-    "cce_forward_noalloc": (_I32, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "cce_forward_noalloc": (_I32, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -126,14 +127,25 @@ def backward_tile_shape() -> Tuple[int, int]:
     return r.value, c.value
 
 
+def _bias_arg(bias: Optional[torch.Tensor], V: int, dev: torch.device) -> Optional[torch.Tensor]:
+    if bias is None:
+        return None
+    if bias.device != dev:
+        raise CCEError(1, "bias must be on the same device as E and C")
+    if bias.numel() != V:
+        raise CCEError(1, f"bias must have V={V} entries, got {bias.numel()}")
+    return bias.reshape(-1).to(torch.bfloat16).contiguous()
+
+
 def cce_forward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, ignore_index: int = -100,
-                reduction: str = "mean", check: bool = False):
-    """Run the forward. Returns (loss, lse, tile_max, count) as device tensors."""
+                reduction: str = "mean", check: bool = False, bias: Optional[torch.Tensor] = None):
+    """Run the forward (logits E C^T + bias). Returns (loss, lse, tile_max, count) as device tensors."""
     lib = load_library()
     dev = _require_cuda(E, C, targets)
     E, C, targets = E.contiguous(), C.contiguous(), targets.contiguous()
     N, D = E.shape
     V = C.shape[0]
+    bias = _bias_arg(bias, V, dev)
     p = _problem(N, D, V, ignore_index, reduction)
     loss = torch.empty(N if reduction == "none" else 1, device=dev, dtype=torch.float32)
     lse = torch.empty(N, device=dev, dtype=torch.float32)
@@ -145,7 +157,7 @@ def cce_forward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, ignore_
     ws_bytes = lib.cce_forward_workspace_size(ctypes.byref(p))
     ws = torch.empty(max(ws_bytes, 1), device=dev, dtype=torch.uint8)
     with torch.cuda.device(dev):
-        _check(lib.cce_forward(ctypes.byref(p), _ptr(E), _ptr(C), _ptr(targets), _ptr(loss), _ptr(lse),
+        _check(lib.cce_forward(ctypes.byref(p), _ptr(E), _ptr(C), _ptr(bias), _ptr(targets), _ptr(loss), _ptr(lse),
                                _ptr(tile_max), _ptr(count), _ptr(ws), ws_bytes, _stream(dev)))
         if check:
             _check(lib.cce_check_device_error(_ptr(ws), _stream(dev)))
@@ -155,58 +167,67 @@ def cce_forward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, ignore_
 def cce_backward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, lse: torch.Tensor,
                  tile_max: torch.Tensor, count: torch.Tensor, grad_out: torch.Tensor,
                  filter_eps: float = DEFAULT_FILTER_EPS, ignore_index: int = -100,
-                 reduction: str = "mean", out_fp32: bool = False, check: bool = False):
-    """Run the backward. Returns (dE, dC, filtered_tiles) as device tensors."""
+                 reduction: str = "mean", out_fp32: bool = False, check: bool = False,
+                 bias: Optional[torch.Tensor] = None, dbias: Optional[bool] = None):
+    """Run the backward. Returns (dE, dC, filtered_tiles) as device tensors, and dbias as a fourth
+    when it is computed (``dbias``; by default whenever ``bias`` is given)."""
     lib = load_library()
     dev = _require_cuda(E, C, targets, lse, tile_max, count)
     E, C, targets = E.contiguous(), C.contiguous(), targets.contiguous()
     N, D = E.shape
     V = C.shape[0]
+    bias = _bias_arg(bias, V, dev)
+    want_dbias = (bias is not None) if dbias is None else bool(dbias)
     p = _problem(N, D, V, ignore_index, reduction)
     g = grad_out.to(device=dev, dtype=torch.float32).reshape(-1).contiguous()
     out_dtype = torch.float32 if out_fp32 else torch.bfloat16
     dE = torch.empty(N, D, device=dev, dtype=out_dtype)
     dC = torch.empty(V, D, device=dev, dtype=out_dtype)
+    db = torch.empty(V, device=dev, dtype=out_dtype) if want_dbias else None
     filtered = torch.empty(1, device=dev, dtype=torch.int64)
     ws_bytes = lib.cce_backward_workspace_size(ctypes.byref(p), int(out_fp32))
     ws = torch.empty(max(ws_bytes, 1), device=dev, dtype=torch.uint8)
     with torch.cuda.device(dev):
-        _check(lib.cce_backward(ctypes.byref(p), _ptr(E), _ptr(C), _ptr(targets), _ptr(lse), _ptr(tile_max),
-                                _ptr(count), _ptr(g), float(filter_eps), _ptr(dE), _ptr(dC), int(out_fp32),
-                                _ptr(filtered), _ptr(ws), ws_bytes, _stream(dev)))
+        _check(lib.cce_backward(ctypes.byref(p), _ptr(E), _ptr(C), _ptr(bias), _ptr(targets), _ptr(lse),
+                                _ptr(tile_max), _ptr(count), _ptr(g), float(filter_eps), _ptr(dE), _ptr(dC), _ptr(db),
+                                int(out_fp32), _ptr(filtered), _ptr(ws), ws_bytes, _stream(dev)))
         if check:
             _check(lib.cce_check_device_error(_ptr(ws), _stream(dev)))
-    return dE, dC, filtered
+    return (dE, dC, filtered, db) if want_dbias else (dE, dC, filtered)
 
 
 class _LinearCrossEntropy(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, E, C, targets, ignore_index, reduction, filter_eps):
-        loss, lse, tile_max, count = cce_forward(E, C, targets, ignore_index, reduction)
-        ctx.save_for_backward(E, C, targets, lse, tile_max, count)
+    def forward(ctx, E, C, bias, targets, ignore_index, reduction, filter_eps):
+        loss, lse, tile_max, count = cce_forward(E, C, targets, ignore_index, reduction, bias=bias)
+        ctx.save_for_backward(E, C, bias, targets, lse, tile_max, count)
         ctx.cfg = (ignore_index, reduction, filter_eps)
         return loss if reduction == "none" else loss.reshape(())
 
     @staticmethod
     def backward(ctx, grad_loss):
-        E, C, targets, lse, tile_max, count = ctx.saved_tensors
+        E, C, bias, targets, lse, tile_max, count = ctx.saved_tensors
         ignore_index, reduction, filter_eps = ctx.cfg
-        dE, dC, _ = cce_backward(E, C, targets, lse, tile_max, count, grad_loss, filter_eps,
-                                 ignore_index, reduction, out_fp32=False)
-        return dE.to(E.dtype), dC.to(C.dtype), None, None, None, None
+        want_db = bias is not None and ctx.needs_input_grad[2]
+        out = cce_backward(E, C, targets, lse, tile_max, count, grad_loss, filter_eps, ignore_index, reduction,
+                           out_fp32=False, bias=bias, dbias=want_db)
+        dbias = out[3].to(bias.dtype) if want_db else None
+        return out[0].to(E.dtype), out[1].to(C.dtype), dbias, None, None, None, None
 
 
-def linear_cross_entropy(e: torch.Tensor, c: torch.Tensor, targets: torch.Tensor, reduction: str = "mean",
-                         ignore_index: int = -100, filter_eps: float = DEFAULT_FILTER_EPS) -> torch.Tensor:
-    """Cross-entropy of softmax(e @ c.T) at ``targets`` without materialising the logits.
+def linear_cross_entropy(e: torch.Tensor, c: torch.Tensor, targets: torch.Tensor,
+                         bias: Optional[torch.Tensor] = None, reduction: str = "mean", ignore_index: int = -100,
+                         filter_eps: float = DEFAULT_FILTER_EPS) -> torch.Tensor:
+    """Cross-entropy of softmax(e @ c.T + bias) at ``targets`` without materialising the logits.
 
-    e: [..., D] bf16 hidden states; c: [V, D] bf16 classifier; targets: [...] int64.
-    Returns a scalar (mean/sum) or the per-token loss in the shape of ``targets`` (none).
+    e: [..., D] bf16 hidden states; c: [V, D] bf16 classifier; targets: [...] int64; bias: optional
+    [V] classifier bias (mlx-cross-entropy README, "API" table). Returns a scalar (mean/sum) or the
+    per-token loss in the shape of ``targets`` (none).
     """
     if e.shape[:-1] != targets.shape:
         raise ValueError(f"targets shape {tuple(targets.shape)} must equal e.shape[:-1] {tuple(e.shape[:-1])}")
     lead = targets.shape
     E = e.reshape(-1, e.shape[-1])
     t = targets.reshape(-1).to(torch.int64)
-    out = _LinearCrossEntropy.apply(E, c, t, ignore_index, reduction, filter_eps)
+    out = _LinearCrossEntropy.apply(E, c, bias, t, ignore_index, reduction, filter_eps)
     return out.reshape(lead) if reduction == "none" else out

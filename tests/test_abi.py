@@ -70,27 +70,32 @@ def test_bad_problems_are_rejected_before_any_cuda_call(lib, bad):
     p = _p(**bad)
     assert lib.cce_tile_max_len(ctypes.byref(p)) == -1
     assert lib.cce_forward_workspace_size(ctypes.byref(p)) == 0
-    st = lib.cce_forward(ctypes.byref(p), 16, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None)
+    st = lib.cce_forward(ctypes.byref(p), 16, 16, None, 16, 16, 16, 16, 16, 16, 1 << 20, None)
     assert st == 1  # CCE_ERR_INVALID_ARG
     assert lib.cce_last_error_message()
 
 
 def test_null_and_misaligned_pointers_are_rejected(lib):
     p = _p()
-    assert lib.cce_forward(ctypes.byref(p), None, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None) == 1
-    assert lib.cce_forward(ctypes.byref(p), 18, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None) == 1
+    assert lib.cce_forward(ctypes.byref(p), None, 16, None, 16, 16, 16, 16, 16, 16, 1 << 20, None) == 1
+    assert lib.cce_forward(ctypes.byref(p), 18, 16, None, 16, 16, 16, 16, 16, 16, 1 << 20, None) == 1
     assert b"aligned" in lib.cce_last_error_message()
-    assert lib.cce_backward(ctypes.byref(p), 16, 16, 16, 16, 16, 16, 16, float("nan"), 16, 16, 0, 16, 16,
-                            1 << 40, None) == 1
+    # a bias that is not 16-byte aligned
+    assert lib.cce_forward(ctypes.byref(p), 16, 16, 24, 16, 16, 16, 16, 16, 16, 1 << 20, None) == 1
+    assert b"aligned" in lib.cce_last_error_message()
+    assert lib.cce_backward(ctypes.byref(p), 16, 16, None, 16, 16, 16, 16, 16, float("nan"), 16, 16, None, 0, 16,
+                            16, 1 << 40, None) == 1
+    assert lib.cce_backward(ctypes.byref(p), 16, 16, None, 16, 16, 16, 16, 16, 0.5, 16, 16, 40, 0, 16, 16,
+                            1 << 40, None) == 1  # misaligned dbias
 
 
 def test_small_workspace_is_rejected(lib):
     p = _p()
     need = lib.cce_forward_workspace_size(ctypes.byref(p))
-    assert lib.cce_forward(ctypes.byref(p), 16, 16, 16, 16, 16, 16, 16, 16, need - 1, None) == 3
+    assert lib.cce_forward(ctypes.byref(p), 16, 16, None, 16, 16, 16, 16, 16, 16, need - 1, None) == 3
 
 
 def test_status_strings(lib):
     for code in range(7):
         assert lib.cce_status_string(code)
-    assert lib.cce_version() >= 100
+    assert lib.cce_version() >= 200

@@ -30,7 +30,7 @@ def _noalloc(E, C, t, reduction, ignore_index=-100):
     lse = torch.full((N,), float("nan"), device=E.device)
     tmax = torch.full((max(lib.cce_tile_max_len(ctypes.byref(p)), 1),), float("nan"), device=E.device)
     count = torch.full((1,), -1, dtype=torch.int64, device=E.device)
-    st = lib.cce_forward_noalloc(ctypes.byref(p), E.data_ptr(), C.data_ptr(), t.data_ptr(), loss.data_ptr(),
+    st = lib.cce_forward_noalloc(ctypes.byref(p), E.data_ptr(), C.data_ptr(), None, t.data_ptr(), loss.data_ptr(),
                                  lse.data_ptr(), tmax.data_ptr(), count.data_ptr(),
                                  torch.cuda.current_stream(E.device).cuda_stream)
     return st, loss, lse, tmax, count
@@ -58,7 +58,7 @@ def test_noalloc_rejects_problems_beyond_its_scratch(device):
     lib = ops.load_library()
     N, D, V = 65536, 128, 128256  # tile sums alone need ceil(V/128) * N * 4 = 263 MB
     p = ops.Problem(N, D, V, -100, 1, 0)
-    st = lib.cce_forward_noalloc(ctypes.byref(p), 256, 256, 256, 256, 256, 256, 256, None)
+    st = lib.cce_forward_noalloc(ctypes.byref(p), 256, 256, None, 256, 256, 256, 256, 256, None)
     assert st == 2  # CCE_ERR_UNSUPPORTED, before anything is enqueued
     assert b"scratch" in lib.cce_last_error_message()
     torch.cuda.synchronize()
