@@ -27,6 +27,14 @@ What it computes, and where that is stated:
   A tile with no non-ignored row is skipped. ``eps <= 0`` turns skipping off.
   The onehot term of the gradient is never skipped.
 
+* Loss functions (explainer), "How it works" item 3 and its listing: label
+  smoothing replaces the one-hot target with ``(1 - ls) * onehot + ls / V``; the
+  loss is ``-sum_v target_v * log p_v`` and the gradient stays ``p - target``.
+  Per row that is ``LSE - (1 - ls) * z_t - (ls / V) * sum_v z_v``.
+* Loss functions (explainer), "Implementation notes": the z-loss adds
+  ``zl * LSE**2`` per token (PaLM uses zl = 1e-4); its logit gradient is
+  ``2 * zl * LSE * p``.
+
 Readings where the pages leave a step open:
 
 * ``mean`` with every token ignored gives loss 0 and a zero gradient: the sum
@@ -36,6 +44,9 @@ Readings where the pages leave a step open:
 * The gradient's upstream factor ``grad_out`` is a scalar for mean/sum and a
   per-token vector for none. The scale of row ``r`` is ``g / max(count, 1)``
   (mean), ``g`` (sum) or ``g[r]`` (none), and 0 for ignored rows.
+* Tile skipping drops only the softmax part of the gradient,
+  ``(1 + 2 zl LSE) * p``; the target part ``(1 - ls) * onehot + ls / V`` is
+  never skipped (it does not depend on the logits).
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
 values the pages print, finite differences, brute force and an independent
@@ -154,7 +165,34 @@ def reduce_loss(nll: np.ndarray, count: int, reduction: str) -> np.ndarray:
     raise ValueError(f"reduction must be one of {REDUCTIONS}, got {reduction!r}")
 
 
-def forward_rows(E, C, targets, rows: Optional[Sequence[int]] = None, ignore_index: int = -100, bias=None):
+def row_loss(lse, z_target, z_sum, V: int, valid, label_smoothing: float = 0.0, z_loss: float = 0.0):
+    """Per-token loss: LSE - (1 - ls) z_t - (ls / V) sum_v z_v + zl LSE^2; 0 for ignored tokens.
+
+    Cut Cross Entropy from first principles (loss = -correct_token + LSE); Loss
+    functions explainer, "How it works" item 3 (smoothed target) and "Implementation
+    notes" (z-loss).
+    """
+    nll = lse - (1.0 - label_smoothing) * z_target - (label_smoothing / V) * z_sum + z_loss * lse * lse
+    return np.where(valid, nll, 0.0)
+
+
+def logit_grad(p, lse, targets, valid, scale, label_smoothing: float = 0.0, z_loss: float = 0.0):
+    """G = scale_r * ((1 + 2 zl LSE_r) * p - (1 - ls) * onehot - ls / V) for the rows given.
+
+    ``p`` may have skipped tiles already set to 0 (only the softmax part is skipped).
+    Loss functions explainer, "How it works" items 2 and 3: the gradient is p - target.
+    """
+    V = p.shape[1]
+    G = (scale * (1.0 + 2.0 * z_loss * lse))[:, None] * p
+    rv = np.flatnonzero(valid)
+    G[rv, targets[rv]] -= scale[rv] * (1.0 - label_smoothing)
+    if label_smoothing:
+        G[rv] -= (scale[rv] * (label_smoothing / V))[:, None]
+    return G
+
+
+def forward_rows(E, C, targets, rows: Optional[Sequence[int]] = None, ignore_index: int = -100, bias=None,
+                 label_smoothing: float = 0.0, z_loss: float = 0.0):
     """Per-row LSE, correct-token logit and loss for a subset of rows.
 
     Each row of the loss depends only on its own hidden state, so any subset of
@@ -167,26 +205,28 @@ def forward_rows(E, C, targets, rows: Optional[Sequence[int]] = None, ignore_ind
     rows = np.arange(E64.shape[0]) if rows is None else np.asarray(rows, dtype=np.int64)
     lse = np.empty(len(rows))
     zt = np.zeros(len(rows))
+    zs = np.zeros(len(rows))
     for g in _row_groups(len(rows)):
         rr = rows[g]
         z = E64[rr] @ C64.T
         if b is not None:
             z += b[None, :]
         lse[g] = log_sum_exp_rows(z)
+        zs[g] = z.sum(axis=1)
         tr = t[rr]
         ok = tr != ignore_index
         zt[g] = np.where(ok, z[np.arange(len(rr)), np.where(ok, tr, 0)], 0.0)
     valid = t[rows] != ignore_index
-    # Cut Cross Entropy from first principles: loss = -correct_token + LSE.
-    nll = np.where(valid, lse - zt, 0.0)
+    nll = row_loss(lse, zt, zs, V, valid, label_smoothing, z_loss)
     return rows, lse, zt, nll, valid
 
 
-def forward(E, C, targets, ignore_index: int = -100, reduction: str = "mean", bias=None) -> ForwardResult:
+def forward(E, C, targets, ignore_index: int = -100, reduction: str = "mean", bias=None,
+            label_smoothing: float = 0.0, z_loss: float = 0.0) -> ForwardResult:
     """Loss and per-row LSE of linear cross-entropy (the forward the CUDA path computes)."""
     if reduction not in REDUCTIONS:
         raise ValueError(f"reduction must be one of {REDUCTIONS}, got {reduction!r}")
-    _, lse, zt, nll, valid = forward_rows(E, C, targets, None, ignore_index, bias)
+    _, lse, zt, nll, valid = forward_rows(E, C, targets, None, ignore_index, bias, label_smoothing, z_loss)
     count = int(valid.sum())
     return ForwardResult(reduce_loss(nll, count, reduction), lse, zt, nll, count)
 
@@ -253,7 +293,7 @@ class BackwardResult:
 
 def backward(E, C, targets, grad_out=1.0, ignore_index: int = -100, reduction: str = "mean",
              filter_eps: float = 2.0 ** -12, tile_m: int = 128, tile_n: int = 256,
-             window: float = 2e-3, bias=None) -> BackwardResult:
+             window: float = 2e-3, bias=None, label_smoothing: float = 0.0, z_loss: float = 0.0) -> BackwardResult:
     """dE, dC (and dbias) of linear cross-entropy, with the tile-skipping rule applied.
 
     G = scale_r * (p~ - onehot), p~ = softmax with skipped tiles set to 0;
@@ -275,9 +315,7 @@ def backward(E, C, targets, grad_out=1.0, ignore_index: int = -100, reduction: s
     skip = filtered_tiles(margin, filter_eps)
     for b, tt in zip(*np.nonzero(skip)):
         p[b * tile_m:(b + 1) * tile_m, tt * tile_n:(tt + 1) * tile_n] = 0.0
-    onehot = np.zeros((N, V))
-    onehot[np.flatnonzero(valid), t[valid]] = 1.0
-    G = scale[:, None] * (p - onehot)
+    G = logit_grad(p, lse, t, valid, scale, label_smoothing, z_loss)
     borderline = 0
     if filter_eps > 0:
         borderline = int((np.abs(margin - math.log(filter_eps)) < window).sum())
@@ -304,7 +342,8 @@ class SampledResult:
 def sampled(E, C, targets, rows: Sequence[int], cols: Sequence[int], grad_out=1.0,
             ignore_index: int = -100, reduction: str = "mean", filter_eps: float = 2.0 ** -12,
             tile_m: int = 128, tile_n: int = 256, window: float = 2e-3,
-            compute_cols: bool = True, bias=None) -> SampledResult:
+            compute_cols: bool = True, bias=None, label_smoothing: float = 0.0,
+            z_loss: float = 0.0) -> SampledResult:
     """The same definitions as ``forward``/``backward``, evaluated for large problems.
 
     The logits are materialised one row group at a time (rows are independent),
@@ -328,6 +367,7 @@ def sampled(E, C, targets, rows: Sequence[int], cols: Sequence[int], grad_out=1.
 
     lse = np.empty(N)
     zt = np.zeros(N)
+    zs = np.zeros(N)
     nb, nt = -(-N // tile_m), -(-V // tile_n)
     margin = np.full((nb, nt), -np.inf)
     dE_rows = np.zeros((len(rows), E64.shape[1]))
@@ -342,6 +382,7 @@ def sampled(E, C, targets, rows: Sequence[int], cols: Sequence[int], grad_out=1.
             z += bv[None, :]
         l = log_sum_exp_rows(z)
         lse[g] = l
+        zs[g] = z.sum(axis=1)
         tg, vg = t[g], valid[g]
         zt[g] = np.where(vg, z[np.arange(z.shape[0]), np.where(vg, tg, 0)], 0.0)
         m = tile_log_margin(z - l[:, None], vg, tile_m, tile_n)
@@ -354,8 +395,7 @@ def sampled(E, C, targets, rows: Sequence[int], cols: Sequence[int], grad_out=1.
         skip = filtered_tiles(m, filter_eps)
         for b, tt in zip(*np.nonzero(skip)):
             p[b * tile_m:(b + 1) * tile_m, tt * tile_n:(tt + 1) * tile_n] = 0.0
-        G = scale[g][:, None] * p
-        G[np.flatnonzero(vg), tg[vg]] -= scale[g][vg]
+        G = logit_grad(p, l, tg, vg, scale[g], label_smoothing, z_loss)
         for i in need_rows:
             dE_rows[row_pos[i]] = G[i - g.start] @ C64
         if compute_cols:
@@ -364,7 +404,7 @@ def sampled(E, C, targets, rows: Sequence[int], cols: Sequence[int], grad_out=1.
                 dbias += G.sum(axis=0)
         del z, p, G
 
-    nll = np.where(valid, lse - zt, 0.0)
+    nll = row_loss(lse, zt, zs, V, valid, label_smoothing, z_loss)
     skip_all = filtered_tiles(margin, filter_eps)
     borderline = int((np.abs(margin - ln_eps) < window).sum()) if filter_eps > 0 else 0
     return SampledResult(lse, nll, count, reduce_loss(nll, count, reduction), margin,
@@ -383,7 +423,7 @@ class RowBlockResult:
 
 def row_blocks(E, C, targets, blocks: Sequence[int], grad_out=1.0, ignore_index: int = -100,
                reduction: str = "mean", filter_eps: float = 2.0 ** -12, tile_m: int = 128,
-               tile_n: int = 256, bias=None) -> RowBlockResult:
+               tile_n: int = 256, bias=None, label_smoothing: float = 0.0, z_loss: float = 0.0) -> RowBlockResult:
     """Exact results for whole row blocks of the tile grid.
 
     A tile's skip decision depends only on the rows of its own row block, and a
@@ -418,11 +458,10 @@ def row_blocks(E, C, targets, blocks: Sequence[int], grad_out=1.0, ignore_index:
         p = softmax_rows(z, l)
         for tt in np.flatnonzero(skip[0]):
             p[:, tt * tile_n:(tt + 1) * tile_n] = 0.0
-        G = scale_all[rr][:, None] * p
-        G[np.flatnonzero(vb), tb[vb]] -= scale_all[rr][vb]
+        G = logit_grad(p, l, tb, vb, scale_all[rr], label_smoothing, z_loss)
         zt = np.where(vb, z[np.arange(len(rr)), np.where(vb, tb, 0)], 0.0)
         lse[pos:pos + len(rr)] = l
-        nll[pos:pos + len(rr)] = np.where(vb, l - zt, 0.0)
+        nll[pos:pos + len(rr)] = row_loss(l, zt, z.sum(axis=1), V, vb, label_smoothing, z_loss)
         dE[pos:pos + len(rr)] = G @ C64
         margins.append(m[0])
         pos += len(rr)

@@ -64,20 +64,22 @@ def test_large_logit_stays_finite():
     np.testing.assert_allclose(b.dE[0], [1.0, -1.0], atol=1e-300)
 
 
-def test_explainer_worked_example_finite_differences():
+@pytest.mark.parametrize("smoothing", ["page", 0.0])
+def test_explainer_worked_example_finite_differences(smoothing):
     g = _golden("explainer_worked_logits.json")
+    ls = g["label_smoothing"] if smoothing == "page" else smoothing
     n, k = g["n"], g["k"]
     z = np.array([((i * 37 % 13) - 6) * 0.8 for i in range(n * k)], dtype=np.float64).reshape(n, k)
     t = np.array(g["targets"])
     C = np.eye(k)  # E @ C.T = E, so E plays the logits
-    b = O.backward(z, C, t, ignore_index=g["ignore_index"], filter_eps=0.0)
+    b = O.backward(z, C, t, ignore_index=g["ignore_index"], filter_eps=0.0, label_smoothing=ls)
     h, tol = g["fd_step"], g["fd_tolerance"]
     for i in g["fd_entries"]:
         zp, zm = z.copy(), z.copy()
         zp.flat[i] += h
         zm.flat[i] -= h
-        lp = float(O.forward(zp, C, t, g["ignore_index"]).loss)
-        lm = float(O.forward(zm, C, t, g["ignore_index"]).loss)
+        lp = float(O.forward(zp, C, t, g["ignore_index"], label_smoothing=ls).loss)
+        lm = float(O.forward(zm, C, t, g["ignore_index"], label_smoothing=ls).loss)
         assert abs((lp - lm) / (2 * h) - b.dE.flat[i]) < tol
     # the ignored row has zero gradient and the mean divides by 3 non-ignored rows
     assert (b.dE[2] == 0).all()
@@ -434,3 +436,93 @@ def test_sampled_with_skips_in_every_row_group(monkeypatch):
         np.testing.assert_allclose(s.lse, lse, rtol=1e-13)
         np.testing.assert_allclose(s.dE_rows, full.dE[[3, 60]], rtol=1e-11, atol=1e-14)
         np.testing.assert_allclose(s.dC_cols, full.dC[[1, 2000]], rtol=1e-11, atol=1e-14)
+
+
+
+# --- label smoothing and z-loss (Loss functions explainer: How it works item 3; Implementation
+# notes: z-loss) ---------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("reduction", ["mean", "sum", "none"])
+def test_smoothing_and_z_loss_match_torch_float64(reduction):
+    """Library special case: F.cross_entropy(label_smoothing=ls) (torch spreads ls over all V
+    classes, the page's definition) plus zl * logsumexp^2 per non-ignored token, with autograd."""
+    E, C, t = _rand_problem(N=40, D=24, V=300, seed=41, ignore=(0, 11, 39))
+    bias = np.random.default_rng(42).standard_normal(300)
+    ls, zl = 0.1, 1e-2
+    Et = torch.tensor(E, requires_grad=True)
+    Ct = torch.tensor(C, requires_grad=True)
+    bt = torch.tensor(bias, requires_grad=True)
+    tt = torch.tensor(t)
+    z = torch.nn.functional.linear(Et, Ct, bt)
+    ce = torch.nn.functional.cross_entropy(z, tt, ignore_index=-100, reduction="none", label_smoothing=ls)
+    valid = (tt != -100).double()
+    per_tok = (ce + zl * torch.logsumexp(z, dim=1) ** 2) * valid
+    out = {"mean": per_tok.sum() / valid.sum(), "sum": per_tok.sum(), "none": per_tok}[reduction]
+    g = np.random.default_rng(43).standard_normal(len(t)) if reduction == "none" else 1.0
+    (out * torch.tensor(g)).sum().backward()
+    f = O.forward(E, C, t, reduction=reduction, bias=bias, label_smoothing=ls, z_loss=zl)
+    b = O.backward(E, C, t, grad_out=g, reduction=reduction, filter_eps=0.0, bias=bias, label_smoothing=ls,
+                   z_loss=zl)
+    np.testing.assert_allclose(np.asarray(f.loss), out.detach().numpy(), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(b.dE, Et.grad.numpy(), rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(b.dC, Ct.grad.numpy(), rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(b.dbias, bt.grad.numpy(), rtol=1e-10, atol=1e-14)
+
+
+@pytest.mark.parametrize("reduction", ["mean", "none"])
+def test_smoothing_and_z_loss_finite_differences(reduction):
+    N, D, V = 8, 16, 64
+    E, C, t = _rand_problem(N, D, V, seed=44, ignore=(5,))
+    ls, zl = 0.2, 0.05
+    g = np.random.default_rng(45).standard_normal(N) if reduction == "none" else 1.0
+
+    def L(E_, C_):
+        f = O.forward(E_, C_, t, reduction=reduction, label_smoothing=ls, z_loss=zl)
+        return float(np.sum(np.asarray(f.loss) * g)) if reduction == "none" else float(f.loss)
+
+    b = O.backward(E, C, t, grad_out=g, reduction=reduction, filter_eps=0.0, label_smoothing=ls, z_loss=zl)
+    h = 1e-5
+    rng = np.random.default_rng(46)
+    for _ in range(10):
+        i, j = rng.integers(0, N), rng.integers(0, D)
+        Ep, Em = E.copy(), E.copy()
+        Ep[i, j] += h
+        Em[i, j] -= h
+        assert abs((L(Ep, C) - L(Em, C)) / (2 * h) - b.dE[i, j]) <= 1e-6 * max(1.0, abs(b.dE[i, j]))
+        v, j = rng.integers(0, V), rng.integers(0, D)
+        Cp, Cm = C.copy(), C.copy()
+        Cp[v, j] += h
+        Cm[v, j] -= h
+        assert abs((L(E, Cp) - L(E, Cm)) / (2 * h) - b.dC[v, j]) <= 1e-6 * max(1.0, abs(b.dC[v, j]))
+
+
+def test_full_smoothing_and_pure_z_loss_closed_forms():
+    """ls = 1: the target is uniform, so each token's loss is LSE - mean_v z_v; zl alone adds
+    zl * LSE^2. Both written out with math.fsum over the logits."""
+    E, C, t = _rand_problem(N=6, D=5, V=40, seed=47, ignore=(2,))
+    z = E @ C.T
+    want_u, want_z = [], []
+    for r in range(6):
+        if t[r] == -100:
+            continue
+        m = max(z[r])
+        lse = m + math.log(math.fsum(math.exp(x - m) for x in z[r]))
+        want_u.append(lse - math.fsum(z[r]) / 40)
+        want_z.append(lse - z[r][t[r]] + 0.3 * lse * lse)
+    assert abs(float(O.forward(E, C, t, label_smoothing=1.0).loss) - math.fsum(want_u) / 5) < 1e-12
+    assert abs(float(O.forward(E, C, t, z_loss=0.3).loss) - math.fsum(want_z) / 5) < 1e-12
+
+
+def test_skipping_keeps_the_smoothing_term():
+    """Tile skipping removes only (1 + 2 zl LSE) p; the ls / V part of the target, which does not
+    depend on the logits, survives in every tile: a fully skipped problem still carries it."""
+    E, C, t = _rand_problem(N=16, D=8, V=128, seed=48, ignore=())
+    ls, zl = 0.1, 1e-3
+    b_all = O.backward(E, C, t, filter_eps=2.0, tile_m=8, tile_n=64, label_smoothing=ls, z_loss=zl)  # eps > 1
+    assert b_all.filtered == b_all.n_tiles
+    scale = 1.0 / 16
+    # G = -scale ((1 - ls) onehot + ls / V) exactly, so dC_v = -scale sum_r ((1-ls)[t_r = v] + ls/V) E_r
+    G = np.full((16, 128), -scale * ls / 128)
+    G[np.arange(16), t] -= scale * (1 - ls)
+    np.testing.assert_allclose(b_all.dC, G.T @ E, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(b_all.dE, G @ C, rtol=1e-12, atol=1e-15)
