@@ -65,6 +65,13 @@ typedef struct {
   int64_t ignore_index; /* a target equal to this masks the token (no loss, zero gradient) */
   int32_t reduction;    /* cce_reduction */
   int32_t reserved;     /* must be 0 */
+  /* Loss variants (Loss functions explainer, "How it works" item 3 and "Implementation notes");
+   * 0 and 0 give the plain cross-entropy. Per non-ignored token the loss is
+   *   LSE - (1 - label_smoothing) z_t - (label_smoothing / V) sum_v z_v + z_loss LSE^2
+   * and its logit gradient (1 + 2 z_loss LSE) p - (1 - label_smoothing) onehot - label_smoothing / V.
+   * Tile skipping drops only the softmax part; the rest is exact. */
+  float label_smoothing; /* in [0, 1] */
+  float z_loss;          /* >= 0 (PaLM uses 1e-4) */
 } cce_problem;
 
 /* Width of the vocabulary sub-tile whose per-row maximum logit the forward saves. */
@@ -156,7 +163,7 @@ CCE_API const char* cce_last_error_message(void);
  * counterpart; it is an addition for such callers. Arguments and results are those of
  * cce_forward() without the workspace.
  *  - Scratch lives in one device array of CCE_NOALLOC_SCRATCH_BYTES that every GPU loading the
- *    library holds until exit. Problems needing more (about ceil(V/128) * N * 4 + 8 N bytes; at
+ *    library holds until exit. Problems needing more (about ceil(V/128) * N * 4 + 12 N + 4 D bytes; at
  *    V = 128256 up to N of about 8000) are rejected with CCE_ERR_UNSUPPORTED before anything runs.
  *  - The first call on each device looks up the array's device address; make that first call
  *    before any stream capture.

@@ -60,6 +60,8 @@ bool problem_ok(const cce_problem* p, bool set_error) {
   if (p->V < 1) return bad("V must be >= 1");
   if (p->reduction < 0 || p->reduction > 2) return bad("reduction must be 0 (none), 1 (mean) or 2 (sum)");
   if (p->reserved != 0) return bad("reserved must be 0");
+  if (!(p->label_smoothing >= 0.f && p->label_smoothing <= 1.f)) return bad("label_smoothing must be in [0, 1]");
+  if (!(p->z_loss >= 0.f && p->z_loss < INFINITY)) return bad("z_loss must be finite and >= 0");
   // Kernel indices are 32-bit for rows and tiles; keep every count well inside that.
   if (p->N >= (int64_t(1) << 31) - 256 || p->V >= (int64_t(1) << 31) - 256 || p->D >= (int64_t(1) << 24))
     return bad("N, V or D too large");
@@ -73,6 +75,8 @@ struct FwdWs {
   float* tile_sum;
   float* z_target;
   float* loss_rows;
+  float* csum;   // [D + 1]: column sums of C and the bias sum (label smoothing only)
+  float* z_sum;  // [N]: sum over the vocabulary of each row's logits (label smoothing only)
   size_t bytes;
 };
 
@@ -87,6 +91,10 @@ FwdWs carve_fwd(const cce_problem* p, void* base) {
   w.z_target = reinterpret_cast<float*>(b + off);
   off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
   w.loss_rows = reinterpret_cast<float*>(b + off);
+  off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
+  w.csum = reinterpret_cast<float*>(b + off);
+  off = align_up(off + sizeof(float) * static_cast<size_t>(p->D + 1));
+  w.z_sum = reinterpret_cast<float*>(b + off);
   off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
   w.bytes = off;
   return w;
@@ -105,6 +113,8 @@ struct SplitWs {
   size_t buf_bytes;
   float* dE_acc;
   float* dbias_acc;  // [V] fp32 (absent with out_fp32)
+  float* csum;       // [D + 1]: column sums of C (label smoothing only)
+  float* wsum;       // [D + 1]: sum_r scale_r E_r and sum_r scale_r (label smoothing only)
   size_t bytes;
 };
 
@@ -161,6 +171,8 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
     w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
     w.dbias_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->V)));
   }
+  w.csum = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->D + 1)));
+  w.wsum = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->D + 1)));
   w.bytes = off;
   return w;
 }
@@ -262,6 +274,15 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   CCE_TRY(cce::launch_fill_zero(dE_acc, N * D * 4, s));
   if (dbias_acc != nullptr) CCE_TRY(cce::launch_fill_zero(dbias_acc, V * 4, s));
   CCE_TRY(cudaMemsetAsync(w.sync, 0, w.sync_bytes, s));
+  // Label smoothing: the ls / V part of every row's target is a rank-one term, added exactly:
+  // dE_r -= scale_r (ls / V) sum_v C_v, dC_v -= (ls / V) sum_r scale_r E_r, dbias_v -= (ls / V) sum_r scale_r.
+  const bool smooth = p->label_smoothing > 0.f;
+  const float ls_v = p->label_smoothing / static_cast<float>(V);
+  const auto* Eb = static_cast<const __nv_bfloat16*>(E);
+  if (smooth) {
+    CCE_TRY(cce::launch_weighted_colsum(static_cast<const __nv_bfloat16*>(C), V, D, nullptr, nullptr, w.csum, s));
+    CCE_TRY(cce::launch_weighted_colsum(Eb, N, D, w.scale, nullptr, w.wsum, s));
+  }
 
   cce::BwdLaunch L{};
   CCE_CHECK(make_map(&L.tmE128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kBwdBM));
@@ -287,6 +308,10 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.targets = targets;
   A.bias = static_cast<const __nv_bfloat16*>(bias);
   A.dbias = dbias_acc;
+  A.z_loss = p->z_loss;
+  A.onehot_coef = 1.f - p->label_smoothing;
+  A.dc_add = smooth ? w.wsum : nullptr;
+  A.dc_coef = -ls_v;
   A.grp_start = w.plan.grp_start;
   A.chunk_t = w.plan.chunk_t;
   A.pstart_t = w.plan.pstart_t;
@@ -309,6 +334,10 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
   CCE_TRY(cce::launch_bwd(L, s));
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
+  if (smooth) {
+    CCE_TRY(cce::launch_add_rank1(dE_acc, N, D, w.scale, -ls_v, w.csum, s));
+    if (dbias_acc != nullptr) CCE_TRY(cce::launch_add_scalar(dbias_acc, V, -ls_v, w.wsum + D, s));
+  }
   if (!out_fp32) CCE_TRY(cce::launch_to_bf16(dE_acc, static_cast<__nv_bfloat16*>(dE), N * D, s));
   if (!out_fp32 && dbias != nullptr)
     CCE_TRY(cce::launch_to_bf16(dbias_acc, static_cast<__nv_bfloat16*>(dbias), V, s));
@@ -413,13 +442,16 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
     // (reported as CCE_ERR_DEVICE_TIMEOUT by cce_check_device_error; the outputs are undefined).
     const char* stall = std::getenv("CCE_TEST_INJECT_STALL");
     L.inject_stall = (stall != nullptr && stall[0] == '1') ? 1 : 0;
-    CCE_TRY(cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, p->ignore_index, w.z_target, &w.hdr->err, s));
+    const bool smooth = p->label_smoothing > 0.f;
+    if (smooth) CCE_TRY(cce::launch_weighted_colsum(Cb, V, D, nullptr, Bb, w.csum, s));
+    CCE_TRY(cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, p->ignore_index, w.z_target,
+                                     smooth ? w.csum : nullptr, smooth ? w.z_sum : nullptr, &w.hdr->err, s));
     if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[0], s));
     CCE_TRY(cce::launch_fwd_lse(L, s));
     if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[1], s));
     float* rows_out = p->reduction == CCE_REDUCTION_NONE ? loss : w.loss_rows;
-    CCE_TRY(cce::launch_lse_loss(tile_max, w.tile_sum, w.z_target, targets, N, T, p->ignore_index, V, lse, rows_out,
-                                 s));
+    CCE_TRY(cce::launch_lse_loss(tile_max, w.tile_sum, w.z_target, smooth ? w.z_sum : nullptr, targets, N, T,
+                                 p->ignore_index, V, p->label_smoothing, p->z_loss, lse, rows_out, s));
   }
   CCE_TRY(cce::launch_loss_reduce(w.loss_rows, targets, N, p->ignore_index, p->reduction, loss, count, s));
   return CCE_OK;

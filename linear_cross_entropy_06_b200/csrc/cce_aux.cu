@@ -35,14 +35,38 @@ __device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
 }
 
 // One warp per row; lanes read 16-byte pieces, so a warp reads 512 contiguous bytes per step.
+__device__ __forceinline__ float dot8_f32(uint4 a, const float* __restrict__ b, float acc) {
+  const float4 b0 = *reinterpret_cast<const float4*>(b), b1 = *reinterpret_cast<const float4*>(b + 4);
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+  const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    __nv_bfloat162 h;
+    *reinterpret_cast<uint32_t*>(&h) = w[k];
+    acc = fmaf(__low2float(h), bb[2 * k], acc);
+    acc = fmaf(__high2float(h), bb[2 * k + 1], acc);
+  }
+  return acc;
+}
+
+// One warp per row: z_target[r] = E_r . C_{t_r} (+ bias[t_r]); with csum (the column sums of C
+// and, at index D, the sum of the bias) also z_sum[r] = sum_v z[r, v] = E_r . csum + csum[D].
 __global__ void target_logit_kernel(const __nv_bfloat16* __restrict__ E, const __nv_bfloat16* __restrict__ C,
                                     const __nv_bfloat16* __restrict__ bias, const int64_t* __restrict__ targets,
                                     int64_t N, int64_t D, int64_t V, int64_t ignore_index,
-                                    float* __restrict__ z_target, int* err) {
+                                    float* __restrict__ z_target, const float* __restrict__ csum,
+                                    float* __restrict__ z_sum, int* err) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= N) return;
   const int64_t t = targets[row];
+  const __nv_bfloat16* e = E + row * D;
+  if (csum != nullptr) {  // every row, ignored ones included (their loss is 0 anyway)
+    float zs = 0.f;
+    for (int64_t d = static_cast<int64_t>(lane) * 8; d < D; d += 256) zs = dot8_f32(ld_global_nc_v4(e + d), csum + d, zs);
+    zs = warp_sum(zs);
+    if (lane == 0) z_sum[row] = zs + csum[D];
+  }
   if (!valid_target(t, V, ignore_index)) {
     if (lane == 0) {
       z_target[row] = 0.f;
@@ -50,7 +74,6 @@ __global__ void target_logit_kernel(const __nv_bfloat16* __restrict__ E, const _
     }
     return;
   }
-  const __nv_bfloat16* e = E + row * D;
   const __nv_bfloat16* c = C + t * D;
   float acc0 = 0.f, acc1 = 0.f;
   int64_t d = static_cast<int64_t>(lane) * 8;
@@ -80,8 +103,9 @@ constexpr int kLseWarps = 32;
 // the 32 partial results merge in shared memory.
 __global__ void __launch_bounds__(kLseWarps * 32)
     lse_loss_kernel(const float* __restrict__ tile_max, const float* __restrict__ tile_sum,
-                    const float* __restrict__ z_target, const int64_t* __restrict__ targets, int64_t N, int64_t T,
-                    int64_t ignore_index, int64_t V, float* __restrict__ lse, float* __restrict__ loss_rows) {
+                    const float* __restrict__ z_target, const float* __restrict__ z_sum,
+                    const int64_t* __restrict__ targets, int64_t N, int64_t T, int64_t ignore_index, int64_t V,
+                    float label_smoothing, float z_loss, float* __restrict__ lse, float* __restrict__ loss_rows) {
   __shared__ float sm_m[kLseWarps][32], sm_s[kLseWarps][32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * 32 + lane;
@@ -108,7 +132,10 @@ __global__ void __launch_bounds__(kLseWarps * 32)
     const float L = Mt + logf(St);
     lse[r] = L;
     const int64_t t = targets[r];
-    loss_rows[r] = valid_target(t, V, ignore_index) ? L - z_target[r] : 0.f;
+    // LSE - (1 - ls) z_t - (ls / V) sum_v z_v + zl LSE^2 (ls and zl are 0 unless requested)
+    float l = L - (1.f - label_smoothing) * z_target[r] + z_loss * L * L;
+    if (z_sum != nullptr) l -= label_smoothing / static_cast<float>(V) * z_sum[r];
+    loss_rows[r] = valid_target(t, V, ignore_index) ? l : 0.f;
   }
 }
 
@@ -178,6 +205,58 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __r
   }
 }
 
+// out[d] += sum_r w_r X[r, d] for d < D (w_r = 1 without weights), and out[D] += sum_r w_r (with
+// weights) or sum_r extra[r] (with an extra bf16 vector). One block per kRowsPerBlock rows; each
+// thread owns 8 columns at a time and adds its partial sums atomically (fp32).
+constexpr int kColsumRows = 512;
+
+__global__ void weighted_colsum_kernel(const __nv_bfloat16* __restrict__ X, int64_t rows, int64_t D,
+                                       const float* __restrict__ w, const __nv_bfloat16* __restrict__ extra,
+                                       float* __restrict__ out) {
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kColsumRows;
+  const int64_t r1 = r0 + kColsumRows < rows ? r0 + kColsumRows : rows;
+  for (int64_t c = static_cast<int64_t>(threadIdx.x) * 8; c < D; c += static_cast<int64_t>(blockDim.x) * 8) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int64_t r = r0; r < r1; ++r) {
+      const float wr = w != nullptr ? w[r] : 1.f;
+      const uint4 u = ld_global_nc_v4(X + r * D + c);
+      const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __nv_bfloat162 h;
+        *reinterpret_cast<uint32_t*>(&h) = q[k];
+        acc[2 * k] = fmaf(wr, __low2float(h), acc[2 * k]);
+        acc[2 * k + 1] = fmaf(wr, __high2float(h), acc[2 * k + 1]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) atomicAdd(out + c + k, acc[k]);
+  }
+  if (threadIdx.x < 32 && (w != nullptr || extra != nullptr)) {
+    float a = 0.f;
+    for (int64_t r = r0 + threadIdx.x; r < r1; r += 32) a += w != nullptr ? w[r] : __bfloat162float(extra[r]);
+    a = warp_sum(a);
+    if (threadIdx.x == 0) atomicAdd(out + D, a);
+  }
+}
+
+// X[r, d] += coef * scale[r] * u[d] (fp32, in place).
+__global__ void add_rank1_kernel(float* __restrict__ X, int64_t rows, int64_t D, const float* __restrict__ scale,
+                                 float coef, const float* __restrict__ u) {
+  const int64_t n = rows * D;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    X[i] = fmaf(coef * scale[i / D], u[i % D], X[i]);
+}
+
+// X[i] += coef * (*c) (fp32, in place).
+__global__ void add_scalar_kernel(float* __restrict__ X, int64_t n, float coef, const float* __restrict__ c) {
+  const float v = coef * *c;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    X[i] += v;
+}
+
 // 16 bytes per thread and step, then the last bytes % 16 one by one.
 __global__ void fill_zero_kernel(uint4* __restrict__ dst, int64_t bytes) {
   const int64_t n16 = bytes / 16;
@@ -195,21 +274,21 @@ int grid_for(int64_t items, int per_block, int cap) {
 
 cudaError_t launch_target_logit(const __nv_bfloat16* E, const __nv_bfloat16* C, const __nv_bfloat16* bias,
                                 const int64_t* targets, int64_t N, int64_t D, int64_t V, int64_t ignore_index,
-                                float* z_target, int* err, cudaStream_t s) {
+                                float* z_target, const float* csum, float* z_sum, int* err, cudaStream_t s) {
   if (N == 0) return cudaSuccess;
-  const int grid = static_cast<int>((N + 7) / 8);
-  target_logit_kernel<<<grid, 256, 0, s>>>(E, C, bias, targets, N, D, V, ignore_index, z_target, err);
+  const int grid = static_cast<int>((N + 7) / 8);  // 8 warps (rows) per block
+  target_logit_kernel<<<grid, 256, 0, s>>>(E, C, bias, targets, N, D, V, ignore_index, z_target, csum, z_sum, err);
   note_launches(1);
   return cudaGetLastError();
 }
 
-cudaError_t launch_lse_loss(const float* tile_max, const float* tile_sum, const float* z_target,
+cudaError_t launch_lse_loss(const float* tile_max, const float* tile_sum, const float* z_target, const float* z_sum,
                             const int64_t* targets, int64_t N, int64_t T, int64_t ignore_index, int64_t V,
-                            float* lse, float* loss_rows, cudaStream_t s) {
+                            float label_smoothing, float z_loss, float* lse, float* loss_rows, cudaStream_t s) {
   if (N == 0) return cudaSuccess;
   const int grid = static_cast<int>((N + 31) / 32);
-  lse_loss_kernel<<<grid, kLseWarps * 32, 0, s>>>(tile_max, tile_sum, z_target, targets, N, T, ignore_index, V, lse,
-                                                  loss_rows);
+  lse_loss_kernel<<<grid, kLseWarps * 32, 0, s>>>(tile_max, tile_sum, z_target, z_sum, targets, N, T, ignore_index,
+                                                  V, label_smoothing, z_loss, lse, loss_rows);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -242,6 +321,31 @@ cudaError_t launch_fill_zero(void* dst, int64_t bytes, cudaStream_t s) {
   if (bytes == 0) return cudaSuccess;
   // dst 16-byte aligned; the tail of fewer than 16 bytes is taken by the first threads
   fill_zero_kernel<<<grid_for(bytes / 16, 256, 148 * 16), 256, 0, s>>>(static_cast<uint4*>(dst), bytes);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_weighted_colsum(const __nv_bfloat16* X, int64_t rows, int64_t D, const float* w,
+                                   const __nv_bfloat16* extra, float* out, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * static_cast<size_t>(D + 1), s);
+  if (e != cudaSuccess || rows == 0) return e;
+  weighted_colsum_kernel<<<static_cast<int>((rows + kColsumRows - 1) / kColsumRows), 256, 0, s>>>(X, rows, D, w,
+                                                                                                 extra, out);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_add_rank1(float* X, int64_t rows, int64_t D, const float* scale, float coef, const float* u,
+                             cudaStream_t s) {
+  if (rows * D == 0) return cudaSuccess;
+  add_rank1_kernel<<<grid_for(rows * D, 256, 148 * 16), 256, 0, s>>>(X, rows, D, scale, coef, u);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_add_scalar(float* X, int64_t n, float coef, const float* c, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  add_scalar_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, s>>>(X, n, coef, c);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -458,8 +458,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (it.kind == kPair) {
         const int b = it.key;
         const int r = b * BM + row;
-        const float lse_l2 = (r < A.N) ? A.lse[r] * kLog2e : 0.f;
+        const float lse_r = (r < A.N) ? A.lse[r] : 0.f;
+        const float lse_l2 = lse_r * kLog2e;
         const float sc = (r < A.N) ? A.scale[r] : 0.f;
+        const float sc_p = sc * fmaf(2.f * A.z_loss, lse_r, 1.f);  // softmax part: (1 + 2 zl LSE) p
+        const float sc_y = sc * A.onehot_coef;                     // onehot part: (1 - ls) y
         const int64_t tg = (r < A.N) ? A.targets[r] : A.ignore_index;
         const bool tvalid = tg != A.ignore_index && tg >= 0 && tg < A.V;
         const bool mma = it.s != 0;
@@ -490,14 +493,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * 2 * BN + u * BN + c * 32), v);
               if (A.bias != nullptr) add_bias32(v, A.bias, col0, A.V);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] = sc * exp2f(fmaf(v[e], kLog2e, -lse_l2));
+              for (int e = 0; e < 32; ++e) v[e] = sc_p * exp2f(fmaf(v[e], kLog2e, -lse_l2));
             } else {
 #pragma unroll
               for (int e = 0; e < 32; ++e) v[e] = 0.f;
             }
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              if (c * 32 + e == tcol) v[e] -= sc;
+              if (c * 32 + e == tcol) v[e] -= sc_y;
               if (col0 + e >= A.V) v[e] = 0.f;
             }
             const uint32_t blk = reg0 + static_cast<uint32_t>((c >> 1) * PART);
@@ -570,6 +573,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) v0[e] = v1[e] = 0.f;
+        }
+        if (!de && A.dc_add != nullptr) {  // the smoothing term, the same for every row of dC
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (x + e < A.D) v0[e] = fmaf(A.dc_coef, A.dc_add[x + e], v0[e]);
+            if (x + 32 + e < A.D) v1[e] = fmaf(A.dc_coef, A.dc_add[x + 32 + e], v1[e]);
+          }
         }
         // this warp's staging is free once its previous TMA op has read it
         if (lane == 0) bulk_wait_group_read0();

@@ -88,6 +88,10 @@ struct BwdArgs {
   const int64_t* targets;
   const __nv_bfloat16* bias;  // [V] or null
   float* dbias;               // [V] fp32 accumulator of the column sums of G, or null
+  float z_loss;               // softmax part of G scaled by 1 + 2 z_loss LSE_r
+  float onehot_coef;          // 1 - label_smoothing: weight of the onehot part of G
+  const float* dc_add;        // [D] or null: added, times dc_coef, to every row of dC
+  float dc_coef;
   const int* grp_start;
   const int* chunk_t;
   const int* pstart_t;
@@ -125,10 +129,18 @@ cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
 // Small kernels (cce_aux.cu).
 cudaError_t launch_target_logit(const __nv_bfloat16* E, const __nv_bfloat16* C, const __nv_bfloat16* bias,
                                 const int64_t* targets, int64_t N, int64_t D, int64_t V, int64_t ignore_index,
-                                float* z_target, int* err, cudaStream_t s);
-cudaError_t launch_lse_loss(const float* tile_max, const float* tile_sum, const float* z_target,
+                                float* z_target, const float* csum, float* z_sum, int* err, cudaStream_t s);
+cudaError_t launch_lse_loss(const float* tile_max, const float* tile_sum, const float* z_target, const float* z_sum,
                             const int64_t* targets, int64_t N, int64_t T, int64_t ignore_index, int64_t V,
-                            float* lse, float* loss_rows, cudaStream_t s);
+                            float label_smoothing, float z_loss, float* lse, float* loss_rows, cudaStream_t s);
+// out[0:D] = sum_r w_r X[r, :] (w_r = 1 when w is null); out[D] = sum_r w_r, or the sum of extra[0:rows].
+cudaError_t launch_weighted_colsum(const __nv_bfloat16* X, int64_t rows, int64_t D, const float* w,
+                                   const __nv_bfloat16* extra, float* out, cudaStream_t s);
+// X[r, :] += coef * scale[r] * u (fp32 [rows, D], in place).
+cudaError_t launch_add_rank1(float* X, int64_t rows, int64_t D, const float* scale, float coef, const float* u,
+                             cudaStream_t s);
+// X[0:n] += coef * (*c).
+cudaError_t launch_add_scalar(float* X, int64_t n, float coef, const float* c, cudaStream_t s);
 cudaError_t launch_loss_reduce(const float* loss_rows, const int64_t* targets, int64_t N, int64_t ignore_index,
                                int reduction, float* loss, int64_t* count, cudaStream_t s);
 cudaError_t launch_row_scale(const int64_t* targets, const int64_t* count, const float* grad_out, int64_t N,

@@ -92,7 +92,8 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   cce::set_last_error("");
   if (p == nullptr || p->N < 0 || p->D < 8 || p->D % 8 != 0 || p->V < 1 || p->reduction < 0 || p->reduction > 2 ||
       p->reserved != 0 || p->N >= (int64_t(1) << 31) - 256 || p->V >= (int64_t(1) << 31) - 256 ||
-      p->D >= (int64_t(1) << 24))
+      p->D >= (int64_t(1) << 24) || !(p->label_smoothing >= 0.f && p->label_smoothing <= 1.f) ||
+      !(p->z_loss >= 0.f && p->z_loss < INFINITY))
     return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: invalid problem");
   const int64_t N = p->N, D = p->D, V = p->V;
   const int64_t T = (V + cce::kSubTile - 1) / cce::kSubTile;
@@ -101,11 +102,14 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
     return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: a required pointer is NULL");
   if ((reinterpret_cast<uintptr_t>(E) | reinterpret_cast<uintptr_t>(C) | reinterpret_cast<uintptr_t>(bias)) & 15u)
     return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: E, C and bias must be 16-byte aligned");
-  // Same layout as the forward workspace: header | tile_sum [T, N] | z_target [N] | loss_rows [N].
+  // Same layout as the forward workspace: header | tile_sum [T, N] | z_target [N] | loss_rows [N] |
+  // csum [D + 1] | z_sum [N] (the last two for label smoothing).
   const size_t off_sum = kHeader;
   const size_t off_zt = up(off_sum + sizeof(float) * static_cast<size_t>(T * N));
   const size_t off_rows = up(off_zt + sizeof(float) * static_cast<size_t>(N));
-  const size_t need = up(off_rows + sizeof(float) * static_cast<size_t>(N));
+  const size_t off_csum = up(off_rows + sizeof(float) * static_cast<size_t>(N));
+  const size_t off_zsum = up(off_csum + sizeof(float) * static_cast<size_t>(D + 1));
+  const size_t need = up(off_zsum + sizeof(float) * static_cast<size_t>(N));
   if (need > kNoAllocScratchBytes) {
     char msg[256];
     snprintf(msg, sizeof(msg),
@@ -123,6 +127,9 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   float* tile_sum = reinterpret_cast<float*>(b + off_sum);
   float* z_target = reinterpret_cast<float*>(b + off_zt);
   float* loss_rows = reinterpret_cast<float*>(b + off_rows);
+  float* csum = reinterpret_cast<float*>(b + off_csum);
+  float* z_sum = reinterpret_cast<float*>(b + off_zsum);
+  const bool smooth = p->label_smoothing > 0.f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const auto* Eb = static_cast<const __nv_bfloat16*>(E);
   const auto* Cb = static_cast<const __nv_bfloat16*>(C);
@@ -146,9 +153,12 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
     L.num_sms = num_sms;
     L.inject_stall = 0;
     L.bias = Bb;
-    if (cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, p->ignore_index, z_target, err, s) != cudaSuccess ||
+    if ((smooth && cce::launch_weighted_colsum(Cb, V, D, nullptr, Bb, csum, s) != cudaSuccess) ||
+        cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, p->ignore_index, z_target, smooth ? csum : nullptr,
+                                 smooth ? z_sum : nullptr, err, s) != cudaSuccess ||
         cce::launch_fwd_lse(L, s) != cudaSuccess ||
-        cce::launch_lse_loss(tile_max, tile_sum, z_target, targets, N, T, p->ignore_index, V, lse,
+        cce::launch_lse_loss(tile_max, tile_sum, z_target, smooth ? z_sum : nullptr, targets, N, T, p->ignore_index,
+                             V, p->label_smoothing, p->z_loss, lse,
                              p->reduction == CCE_REDUCTION_NONE ? loss : loss_rows, s) != cudaSuccess)
       return fail(CCE_ERR_CUDA, "cce_forward_noalloc: kernel launch failed");
   }

@@ -48,6 +48,8 @@ class Problem(ctypes.Structure):
         ("ignore_index", ctypes.c_int64),
         ("reduction", ctypes.c_int32),
         ("reserved", ctypes.c_int32),
+        ("label_smoothing", ctypes.c_float),
+        ("z_loss", ctypes.c_float),
     ]
 
 
@@ -104,10 +106,11 @@ def _stream(device: torch.device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
-def _problem(N: int, D: int, V: int, ignore_index: int, reduction: str) -> Problem:
+def _problem(N: int, D: int, V: int, ignore_index: int, reduction: str, label_smoothing: float = 0.0,
+             z_loss: float = 0.0) -> Problem:
     if reduction not in REDUCTION_CODES:
         raise ValueError(f"reduction must be one of {tuple(REDUCTION_CODES)}, got {reduction!r}")
-    return Problem(N, D, V, ignore_index, REDUCTION_CODES[reduction], 0)
+    return Problem(N, D, V, ignore_index, REDUCTION_CODES[reduction], 0, float(label_smoothing), float(z_loss))
 
 
 def _require_cuda(*tensors: torch.Tensor) -> torch.device:
@@ -138,7 +141,8 @@ def _bias_arg(bias: Optional[torch.Tensor], V: int, dev: torch.device) -> Option
 
 
 def cce_forward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, ignore_index: int = -100,
-                reduction: str = "mean", check: bool = False, bias: Optional[torch.Tensor] = None):
+                reduction: str = "mean", check: bool = False, bias: Optional[torch.Tensor] = None,
+                label_smoothing: float = 0.0, z_loss: float = 0.0):
     """Run the forward (logits E C^T + bias). Returns (loss, lse, tile_max, count) as device tensors."""
     lib = load_library()
     dev = _require_cuda(E, C, targets)
@@ -146,7 +150,7 @@ def cce_forward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, ignore_
     N, D = E.shape
     V = C.shape[0]
     bias = _bias_arg(bias, V, dev)
-    p = _problem(N, D, V, ignore_index, reduction)
+    p = _problem(N, D, V, ignore_index, reduction, label_smoothing, z_loss)
     loss = torch.empty(N if reduction == "none" else 1, device=dev, dtype=torch.float32)
     lse = torch.empty(N, device=dev, dtype=torch.float32)
     tm_len = lib.cce_tile_max_len(ctypes.byref(p))
@@ -168,7 +172,8 @@ def cce_backward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, lse: t
                  tile_max: torch.Tensor, count: torch.Tensor, grad_out: torch.Tensor,
                  filter_eps: float = DEFAULT_FILTER_EPS, ignore_index: int = -100,
                  reduction: str = "mean", out_fp32: bool = False, check: bool = False,
-                 bias: Optional[torch.Tensor] = None, dbias: Optional[bool] = None):
+                 bias: Optional[torch.Tensor] = None, dbias: Optional[bool] = None,
+                 label_smoothing: float = 0.0, z_loss: float = 0.0):
     """Run the backward. Returns (dE, dC, filtered_tiles) as device tensors, and dbias as a fourth
     when it is computed (``dbias``; by default whenever ``bias`` is given)."""
     lib = load_library()
@@ -178,7 +183,7 @@ def cce_backward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, lse: t
     V = C.shape[0]
     bias = _bias_arg(bias, V, dev)
     want_dbias = (bias is not None) if dbias is None else bool(dbias)
-    p = _problem(N, D, V, ignore_index, reduction)
+    p = _problem(N, D, V, ignore_index, reduction, label_smoothing, z_loss)
     g = grad_out.to(device=dev, dtype=torch.float32).reshape(-1).contiguous()
     out_dtype = torch.float32 if out_fp32 else torch.bfloat16
     dE = torch.empty(N, D, device=dev, dtype=out_dtype)
@@ -198,36 +203,57 @@ def cce_backward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, lse: t
 
 class _LinearCrossEntropy(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, E, C, bias, targets, ignore_index, reduction, filter_eps):
-        loss, lse, tile_max, count = cce_forward(E, C, targets, ignore_index, reduction, bias=bias)
+    def forward(ctx, E, C, bias, targets, ignore_index, reduction, filter_eps, label_smoothing, z_loss):
+        loss, lse, tile_max, count = cce_forward(E, C, targets, ignore_index, reduction, bias=bias,
+                                                 label_smoothing=label_smoothing, z_loss=z_loss)
         ctx.save_for_backward(E, C, bias, targets, lse, tile_max, count)
-        ctx.cfg = (ignore_index, reduction, filter_eps)
+        ctx.cfg = (ignore_index, reduction, filter_eps, label_smoothing, z_loss)
         return loss if reduction == "none" else loss.reshape(())
 
     @staticmethod
     def backward(ctx, grad_loss):
         E, C, bias, targets, lse, tile_max, count = ctx.saved_tensors
-        ignore_index, reduction, filter_eps = ctx.cfg
+        ignore_index, reduction, filter_eps, label_smoothing, z_loss = ctx.cfg
         want_db = bias is not None and ctx.needs_input_grad[2]
         out = cce_backward(E, C, targets, lse, tile_max, count, grad_loss, filter_eps, ignore_index, reduction,
-                           out_fp32=False, bias=bias, dbias=want_db)
+                           out_fp32=False, bias=bias, dbias=want_db, label_smoothing=label_smoothing, z_loss=z_loss)
         dbias = out[3].to(bias.dtype) if want_db else None
-        return out[0].to(E.dtype), out[1].to(C.dtype), dbias, None, None, None, None
+        return out[0].to(E.dtype), out[1].to(C.dtype), dbias, None, None, None, None, None, None
+
+
+def shift_targets(targets: torch.Tensor, ignore_index: int = -100) -> torch.Tensor:
+    """Causal-LM targets for hidden states of shape [..., T, D]: position i predicts token i + 1,
+    and the last position of each sequence has no target (``ignore_index``)."""
+    out = torch.full_like(targets, ignore_index)
+    out[..., :-1] = targets[..., 1:]
+    return out
 
 
 def linear_cross_entropy(e: torch.Tensor, c: torch.Tensor, targets: torch.Tensor,
                          bias: Optional[torch.Tensor] = None, reduction: str = "mean", ignore_index: int = -100,
-                         filter_eps: float = DEFAULT_FILTER_EPS) -> torch.Tensor:
+                         filter_eps: float = DEFAULT_FILTER_EPS, label_smoothing: float = 0.0, z_loss: float = 0.0,
+                         shift: bool = False) -> torch.Tensor:
     """Cross-entropy of softmax(e @ c.T + bias) at ``targets`` without materialising the logits.
 
     e: [..., D] bf16 hidden states; c: [V, D] bf16 classifier; targets: [...] int64; bias: optional
-    [V] classifier bias (mlx-cross-entropy README, "API" table). Returns a scalar (mean/sum) or the
-    per-token loss in the shape of ``targets`` (none).
+    [V] classifier bias (mlx-cross-entropy README, "API" table). ``label_smoothing`` and ``z_loss``
+    select the smoothed target and the z-loss of the Loss functions explainer (0 and 0: plain
+    cross-entropy). ``shift`` makes e[..., i, :] predict targets[..., i + 1] (causal language
+    modelling over a trailing sequence axis); the last position of each sequence is then ignored.
+    Returns a scalar (mean/sum) or the per-token loss in the shape of ``targets`` (none; with
+    ``shift``, one position shorter along the sequence axis).
     """
     if e.shape[:-1] != targets.shape:
         raise ValueError(f"targets shape {tuple(targets.shape)} must equal e.shape[:-1] {tuple(e.shape[:-1])}")
+    if shift:
+        if targets.dim() < 1 or targets.shape[-1] < 1:
+            raise ValueError("shift needs a sequence axis of length >= 1")
+        targets = shift_targets(targets, ignore_index)
     lead = targets.shape
     E = e.reshape(-1, e.shape[-1])
     t = targets.reshape(-1).to(torch.int64)
-    out = _LinearCrossEntropy.apply(E, c, bias, t, ignore_index, reduction, filter_eps)
-    return out.reshape(lead) if reduction == "none" else out
+    out = _LinearCrossEntropy.apply(E, c, bias, t, ignore_index, reduction, filter_eps, label_smoothing, z_loss)
+    if reduction != "none":
+        return out
+    out = out.reshape(lead)
+    return out[..., :-1] if shift else out

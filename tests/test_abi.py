@@ -53,7 +53,9 @@ def test_sizes(lib):
     T = -(-1000 // 128)
     assert lib.cce_tile_max_len(ctypes.byref(p)) == T * 300
     fw = lib.cce_forward_workspace_size(ctypes.byref(p))
-    assert 0 < fw < 256 + 4 * (T * 300 + 600) + 4 * 256
+    # header, tile sums [T, N], target logits, row losses, and for label smoothing the column
+    # sums of C [D + 1] and the row sums of the logits [N]; 256-byte alignment of each
+    assert 0 < fw < 256 + 4 * (T * 300 + 900 + 137) + 6 * 256
     bw32 = lib.cce_backward_workspace_size(ctypes.byref(p), 1)
     bw16 = lib.cce_backward_workspace_size(ctypes.byref(p), 0)
     assert bw16 - bw32 >= 4 * 300 * 136  # the fp32 dE accumulator (dC is summed on chip)
@@ -87,6 +89,16 @@ def test_null_and_misaligned_pointers_are_rejected(lib):
                             16, 1 << 40, None) == 1
     assert lib.cce_backward(ctypes.byref(p), 16, 16, None, 16, 16, 16, 16, 16, 0.5, 16, 16, 40, 0, 16, 16,
                             1 << 40, None) == 1  # misaligned dbias
+
+
+@pytest.mark.parametrize("field,value", [("label_smoothing", -0.1), ("label_smoothing", 1.5),
+                                         ("label_smoothing", float("nan")), ("z_loss", -1.0), ("z_loss", float("inf"))])
+def test_bad_loss_variants_are_rejected(lib, field, value):
+    p = _p()
+    setattr(p, field, value)
+    assert lib.cce_tile_max_len(ctypes.byref(p)) == -1
+    assert lib.cce_forward(ctypes.byref(p), 16, 16, None, 16, 16, 16, 16, 16, 16, 1 << 20, None) == 1
+    assert field.encode() in lib.cce_last_error_message()
 
 
 def test_small_workspace_is_rejected(lib):

@@ -26,34 +26,36 @@ def make_bias(V, seed, scale=2.0):
     return torch.from_numpy(b).to(torch.bfloat16)
 
 
-def run_with_bias(inp, bias, device, filter_eps, reduction, out_fp32=False, grad_out=None, dbias=True):
+def run_with_bias(inp, bias, device, filter_eps, reduction, out_fp32=False, grad_out=None, dbias=True, ls=0.0,
+                  zl=0.0):
     E, C, t = inp.E.to(device), inp.C.to(device), inp.targets.to(device)
     b = None if bias is None else bias.to(device)
     g = (inp.grad_out if grad_out is None else grad_out).to(device)
     if reduction != "none":
         g = g[:1]
-    loss, lse, tmax, count = ops.cce_forward(E, C, t, -100, reduction, check=True, bias=b)
+    loss, lse, tmax, count = ops.cce_forward(E, C, t, -100, reduction, check=True, bias=b, label_smoothing=ls,
+                                             z_loss=zl)
     dE, dC, filt, db = ops.cce_backward(E, C, t, lse, tmax, count, g, filter_eps, -100, reduction, out_fp32,
-                                        check=True, bias=b, dbias=dbias)
+                                        check=True, bias=b, dbias=dbias, label_smoothing=ls, z_loss=zl)
     torch.cuda.synchronize()
     return dict(loss=loss.double().cpu().numpy(), lse=lse.double().cpu().numpy(), count=int(count.item()),
                 dE=dE.double().cpu().numpy(), dC=dC.double().cpu().numpy(), dbias=db.double().cpu().numpy(),
                 filtered=int(filt.item()), dE_raw=dE.cpu())
 
 
-def check_bias(inp, bias, device, reduction, grad_out=None, out_fp32=False):
+def check_bias(inp, bias, device, reduction, grad_out=None, out_fp32=False, ls=0.0, zl=0.0):
     tm, tn = ops.backward_tile_shape()
     g = inp.grad_out if grad_out is None else grad_out
     g_or = g.numpy() if reduction == "none" else float(g.reshape(-1)[0])
     ob = None if bias is None else bias
-    f = O.forward(inp.E, inp.C, inp.targets, -100, reduction, bias=ob)
-    sc = O.row_scale(inp.targets, -100, reduction, g_or, f.count)
+    f = O.forward(inp.E, inp.C, inp.targets, -100, reduction, bias=ob, label_smoothing=ls, z_loss=zl)
+    sc = O.row_scale(inp.targets, -100, reduction, g_or, f.count) * (1.0 + 2.0 * zl * np.abs(f.lse).max())
     floors = {"dE": fp32_floor(f.lse, sc, inp.C), "dC": fp32_floor(f.lse, sc, inp.E),
               "dbias": fp32_floor(f.lse, sc, 1.0)}
     for eps in (0.0, EPS):
         b = O.backward(inp.E, inp.C, inp.targets, g_or, -100, reduction, eps, tm, tn,
-                       bias=np.zeros(inp.C.shape[0]) if bias is None else ob)
-        r = run_with_bias(inp, bias, device, eps, reduction, out_fp32, grad_out)
+                       bias=np.zeros(inp.C.shape[0]) if bias is None else ob, label_smoothing=ls, z_loss=zl)
+        r = run_with_bias(inp, bias, device, eps, reduction, out_fp32, grad_out, ls=ls, zl=zl)
         if reduction == "sum":
             assert abs(r["loss"][0] - float(f.loss)) <= LOSS_TOL * max(f.count, 1)
         else:
