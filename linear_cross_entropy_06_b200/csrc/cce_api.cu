@@ -17,7 +17,7 @@
 
 namespace {
 
-constexpr int32_t kVersion = 200;  // 0.2.0: classifier bias
+constexpr int32_t kVersion = 300;  // 0.3.0: loss variants (label smoothing, z-loss)
 constexpr size_t kHeaderBytes = 256;
 constexpr size_t kAlign = 256;
 

@@ -110,4 +110,4 @@ def test_small_workspace_is_rejected(lib):
 def test_status_strings(lib):
     for code in range(7):
         assert lib.cce_status_string(code)
-    assert lib.cce_version() >= 200
+    assert lib.cce_version() >= 300
