@@ -177,7 +177,8 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, const Bwd
     if (local < A.nb * S) {  // slice-major: concurrent dE items read the same columns of C
       it.kind = kDE;
       it.key = local % A.nb;
-      it.s = local / A.nb;
+      // serpentine over chunks: a chunk starts on the slices of dE the previous one touched last
+      it.s = (c & 1) ? S - 1 - local / A.nb : local / A.nb;
       const int2 r = A.rb_range[static_cast<int64_t>(c) * A.nb + it.key];
       it.begin = r.x;
       it.end = r.y;

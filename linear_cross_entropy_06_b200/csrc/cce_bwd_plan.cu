@@ -66,7 +66,7 @@ __global__ void tile_flags_kernel(const float* __restrict__ tile_max, const floa
 // One warp per vocabulary tile t: the rank of each listed (b, t) among the listed row blocks of t,
 // the number of listed tiles of t, and the kept total.
 __global__ void tile_rank_kernel(const uint8_t* __restrict__ flags, int nb, int nt, int* __restrict__ rank,
-                                 int* __restrict__ cnt_t, int* __restrict__ kept_total) {
+                                 int* __restrict__ cnt_t, int* __restrict__ cnt_b, int* __restrict__ kept_total) {
   const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= nt) return;
@@ -75,7 +75,10 @@ __global__ void tile_rank_kernel(const uint8_t* __restrict__ flags, int nb, int 
     const int b = b0 + lane;
     const uint8_t f = b < nb ? flags[static_cast<int64_t>(b) * nt + t] : 0;
     const unsigned on = __ballot_sync(0xffffffffu, f != 0);
-    if (f != 0) rank[static_cast<int64_t>(b) * nt + t] = listed + __popc(on & ((1u << lane) - 1u));
+    if (f != 0) {
+      rank[static_cast<int64_t>(b) * nt + t] = listed + __popc(on & ((1u << lane) - 1u));
+      atomicAdd(cnt_b + b, 1);
+    }
     listed += __popc(on);
     kept += __popc(__ballot_sync(0xffffffffu, f == 1));
   }
@@ -120,29 +123,39 @@ __global__ void fill_col_kernel(const uint8_t* __restrict__ flags, const int* __
   entries_t[offsets_t[t] + rank[i]] = make_int2(b * 4 + f, t);
 }
 
-// One warp per row block: counts (pass 0) or writes (pass 1) its listed tiles in vocabulary order.
+// One block of 1024 threads per row block: writes its listed tiles in vocabulary order (a block-wide
+// scan of the listed flags, 1024 vocabulary tiles per step), and the inverse map pos_b.
 __global__ void row_list_kernel(const uint8_t* __restrict__ flags, const int* __restrict__ rank,
-                                const int* __restrict__ offsets_t, int nb, int nt, int* __restrict__ cnt_b,
-                                const int* __restrict__ offsets_b, int2* __restrict__ entries_b,
-                                int* __restrict__ pos_b, int pass) {
-  const int b = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
-  const int lane = threadIdx.x & 31;
-  if (b >= nb) return;
+                                const int* __restrict__ offsets_t, int nt, const int* __restrict__ offsets_b,
+                                int2* __restrict__ entries_b, int* __restrict__ pos_b) {
+  __shared__ int wsum[32];
+  __shared__ int carry;
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const uint8_t* row = flags + static_cast<int64_t>(b) * nt;
-  int k = 0;
-  for (int t0 = 0; t0 < nt; t0 += 32) {
-    const int t = t0 + lane;
+  if (threadIdx.x == 0) carry = offsets_b[b];
+  __syncthreads();
+  for (int t0 = 0; t0 < nt; t0 += 1024) {
+    const int t = t0 + threadIdx.x;
     const bool on = t < nt && row[t] != 0;
-    const unsigned mask = __ballot_sync(0xffffffffu, on);
-    if (pass == 1 && on) {
-      const int pos = offsets_b[b] + k + __popc(mask & ((1u << lane) - 1u));
+    const unsigned m = __ballot_sync(0xffffffffu, on);
+    if (lane == 0) wsum[w] = __popc(m);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int k = 0; k < 32; ++k) {
+      before += k < w ? wsum[k] : 0;
+      total += wsum[k];
+    }
+    if (on) {
+      const int pos = carry + before + __popc(m & ((1u << lane) - 1u));
       const int slot = offsets_t[t] + rank[static_cast<int64_t>(b) * nt + t];
       entries_b[pos] = make_int2(t, slot);
       pos_b[slot] = pos;
     }
-    k += __popc(mask);
+    __syncthreads();  // everyone has read carry and wsum
+    if (threadIdx.x == 0) carry += total;
+    __syncthreads();
   }
-  if (pass == 0 && lane == 0) cnt_b[b] = k;
 }
 
 __device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int t) {
@@ -259,22 +272,19 @@ cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float
     tile_flags_kernel<<<static_cast<unsigned>(tiles), kBwdBM, 0, s>>>(tile_max, lse, targets, N, V, T, ignore_index,
                                                                      ln_eps, filter_on, nt, P.flags);
     note_launches(1);
+    e = cudaMemsetAsync(P.cnt_b, 0, sizeof(int) * static_cast<size_t>(nb), s);
+    if (e != cudaSuccess) return e;
     tile_rank_kernel<<<static_cast<int>((static_cast<int64_t>(nt) * 32 + 255) / 256), 256, 0, s>>>(
-        P.flags, nb, nt, P.rank, P.cnt_t, P.kept_total);
+        P.flags, nb, nt, P.rank, P.cnt_t, P.cnt_b, P.kept_total);
     note_launches(1);
     scan_kernel<<<1, 1024, 0, s>>>(P.cnt_t, nt, P.offsets_t);
     note_launches(1);
     fill_col_kernel<<<static_cast<int>((tiles + 255) / 256), 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt,
                                                                           P.entries_t);
     note_launches(1);
-    const int grid_b = (nb * 32 + 255) / 256;
-    row_list_kernel<<<grid_b, 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt, P.cnt_b, P.offsets_b, P.entries_b,
-                                           P.pos_b, 0);
-    note_launches(1);
     scan_kernel<<<1, 1024, 0, s>>>(P.cnt_b, nb, P.offsets_b);
     note_launches(1);
-    row_list_kernel<<<grid_b, 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt, P.cnt_b, P.offsets_b, P.entries_b,
-                                           P.pos_b, 1);
+    row_list_kernel<<<nb, 1024, 0, s>>>(P.flags, P.rank, P.offsets_t, nt, P.offsets_b, P.entries_b, P.pos_b);
     note_launches(1);
     chunk_plan_kernel<<<(P.nchunks + 256) / 256, 256, 0, s>>>(nt, P.chunk_vt, P.nchunks, P.chunk_t);
     note_launches(1);
