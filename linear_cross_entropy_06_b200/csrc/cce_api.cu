@@ -329,6 +329,10 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.ctr_b_done = A.ctr_g_t + w.plan.nt;
   A.err = &w.hdr->err;
   A.timeout_ns = wait_timeout_ns();
+  // Failure-detection test hook: CCE_TEST_INJECT_STALL=2 makes the backward's dE items of the first
+  // chunk wait for a gradient tile that is never stored (reported as CCE_ERR_DEVICE_TIMEOUT).
+  const char* stall = std::getenv("CCE_TEST_INJECT_STALL");
+  A.inject_stall = (stall != nullptr && stall[0] == '2') ? 1 : 0;
   L.num_sms = num_sms;
 
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));

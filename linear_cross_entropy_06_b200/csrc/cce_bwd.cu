@@ -193,6 +193,9 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, const Bwd
       it.dep_idx = A.ctr_g_t + it.key;
     }
     it.dep_val = it.end - it.begin;
+    // test hook: the dE items of the first chunk wait for one gradient tile more than the pairs
+    // store, so their bounded wait runs out
+    if (A.inject_stall && c == 0 && it.kind == kDE) ++it.dep_val;
   }
 }
 

@@ -108,6 +108,7 @@ struct BwdArgs {
   int ctr_g_b, ctr_g_t, ctr_b_done;
   int* err;
   uint64_t timeout_ns;
+  int inject_stall;  // test hook: the first dE item waits for a count no item produces
 };
 
 struct BwdLaunch {
