@@ -163,6 +163,9 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.S = static_cast<int>(ceil_div(p->D, cce::kGemmSlice));
   w.plan.grp_size = reinterpret_cast<int*>(take(sizeof(int) * 2 * static_cast<size_t>(w.plan.nchunks)));
   w.plan.grp_start = reinterpret_cast<int*>(take(sizeof(int) * (2 * static_cast<size_t>(w.plan.nchunks) + 1)));
+  w.plan.oh_cnt = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt)));
+  w.plan.oh_off = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt + 1)));
+  w.plan.oh_rows = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(std::max<int64_t>(p->N, 1))));
   w.sync_bytes = sizeof(int) * static_cast<size_t>(1 + w.plan.nchunks * nb + nt + w.plan.nchunks);
   w.sync = reinterpret_cast<int*>(take(w.sync_bytes));
   w.buf_bytes = static_cast<size_t>(nb * chunk_vt) * cce::kGradTileBytes;
@@ -312,6 +315,9 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.onehot_coef = 1.f - p->label_smoothing;
   A.dc_add = smooth ? w.wsum : nullptr;
   A.dc_coef = -ls_v;
+  A.E = Eb;
+  A.oh_off = w.plan.oh_off;
+  A.oh_rows = w.plan.oh_rows;
   A.grp_start = w.plan.grp_start;
   A.chunk_t = w.plan.chunk_t;
   A.pstart_t = w.plan.pstart_t;
@@ -338,6 +344,8 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
   CCE_TRY(cce::launch_bwd(L, s));
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
+  CCE_TRY(cce::launch_onehot_rows(w.plan.oh_off, w.plan.nt, w.plan.oh_rows, targets, w.scale, 1.f - p->label_smoothing,
+                                  static_cast<const __nv_bfloat16*>(C), D, dE_acc, dbias_acc, N, s));
   if (smooth) {
     CCE_TRY(cce::launch_add_rank1(dE_acc, N, D, w.scale, -ls_v, w.csum, s));
     if (dbias_acc != nullptr) CCE_TRY(cce::launch_add_scalar(dbias_acc, V, -ls_v, w.wsum + D, s));

@@ -257,6 +257,46 @@ __global__ void add_scalar_kernel(float* __restrict__ X, int64_t n, float coef, 
     X[i] += v;
 }
 
+// One warp per listed row r (rows[i], i < off[nt]): dE_acc[r, :] -= coef * scale[r] * C[t_r, :]
+// and dbias_acc[t_r] -= coef * scale[r]. Each row is listed once, so the dE rows need no atomics.
+__global__ void onehot_rows_apply_kernel(const int* __restrict__ off, int nt, const int* __restrict__ rows,
+                                         const int64_t* __restrict__ targets, const float* __restrict__ scale,
+                                         float coef, const __nv_bfloat16* __restrict__ C, int64_t D,
+                                         float* __restrict__ dE_acc, float* __restrict__ dbias_acc) {
+  const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (i >= off[nt]) return;
+  const int64_t r = rows[i];
+  const int64_t t = targets[r];
+  const float a = -coef * scale[r];
+  if (dbias_acc != nullptr && lane == 0) atomicAdd(dbias_acc + t, a);
+  const __nv_bfloat16* c = C + t * D;
+  float* out = dE_acc + r * D;
+  for (int64_t d = static_cast<int64_t>(lane) * 8; d < D; d += 256) {
+    const uint4 u = ld_global_nc_v4(c + d);
+    const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+    float4 o0 = *reinterpret_cast<float4*>(out + d), o1 = *reinterpret_cast<float4*>(out + d + 4);
+    float cv[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      __nv_bfloat162 h;
+      *reinterpret_cast<uint32_t*>(&h) = q[k];
+      cv[2 * k] = __low2float(h);
+      cv[2 * k + 1] = __high2float(h);
+    }
+    o0.x = fmaf(a, cv[0], o0.x);
+    o0.y = fmaf(a, cv[1], o0.y);
+    o0.z = fmaf(a, cv[2], o0.z);
+    o0.w = fmaf(a, cv[3], o0.w);
+    o1.x = fmaf(a, cv[4], o1.x);
+    o1.y = fmaf(a, cv[5], o1.y);
+    o1.z = fmaf(a, cv[6], o1.z);
+    o1.w = fmaf(a, cv[7], o1.w);
+    *reinterpret_cast<float4*>(out + d) = o0;
+    *reinterpret_cast<float4*>(out + d + 4) = o1;
+  }
+}
+
 // 16 bytes per thread and step, then the last bytes % 16 one by one.
 __global__ void fill_zero_kernel(uint4* __restrict__ dst, int64_t bytes) {
   const int64_t n16 = bytes / 16;
@@ -346,6 +386,16 @@ cudaError_t launch_add_rank1(float* X, int64_t rows, int64_t D, const float* sca
 cudaError_t launch_add_scalar(float* X, int64_t n, float coef, const float* c, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   add_scalar_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, s>>>(X, n, coef, c);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_onehot_rows(const int* off, int nt, const int* rows, const int64_t* targets,
+                               const float* scale, float coef, const __nv_bfloat16* C, int64_t D, float* dE_acc,
+                               float* dbias_acc, int64_t max_rows, cudaStream_t s) {
+  if (max_rows == 0) return cudaSuccess;
+  const int grid = static_cast<int>((max_rows + 7) / 8);  // 8 warps per block, one listed row each
+  onehot_rows_apply_kernel<<<grid, 256, 0, s>>>(off, nt, rows, targets, scale, coef, C, D, dE_acc, dbias_acc);
   note_launches(1);
   return cudaGetLastError();
 }

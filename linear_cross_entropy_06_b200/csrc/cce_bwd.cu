@@ -8,7 +8,7 @@
 //
 // Work items, per vocabulary chunk c (its gradient tiles live in scratch buffer c mod kGradBuffers):
 //   pair   two consecutive listed 128 x 128 tiles (b, t0), (b, t1) of row block b in the chunk:
-//          S = E_b [C_t0; C_t1]^T (tcgen05 M=128 N=256 K=D; skipped for onehot-only tiles), then
+//          S = E_b [C_t0; C_t1]^T (tcgen05 M=128 N=256 K=D), then
 //          G = scale_r * exp(S - LSE_r) - scale_r * [v = t_r] in fp32, rounded to bf16 into a
 //          128B-swizzled shared tile, one 32 KB bulk store per tile into the scratch buffer.
 //   dE     (row block b, 256-column slice s of D): sum over the chunk's listed t of G_bt C_t[:, s]
@@ -75,7 +75,9 @@ struct alignas(16) WorkItem {
   int slot1;       // pair: slot of t1
   int dep_idx;     // counter this item waits on (-1: none): before its loads (dE, dC) or stores (pair)
   int dep_val;     // value the counter must reach
-  int pad[6];
+  int oh_begin;    // dC: rows whose target tile in this vocabulary tile was skipped, oh_rows[oh_begin:oh_end]
+  int oh_end;
+  int pad[4];
 };
 static_assert(sizeof(WorkItem) == 64, "ring entries are 64 bytes");
 
@@ -151,6 +153,7 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, const Bwd
   const int c = gc.x, local = w - g_begin;
   const int t_begin = A.chunk_t[c];
   it.chunk = c;
+  it.oh_begin = it.oh_end = 0;
   if (gc.y) {
     const int64_t pi = static_cast<int64_t>(A.pstart_t[t_begin]) + local;
     const int4 d = A.pair_desc[pi];
@@ -191,6 +194,8 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, const Bwd
       it.begin = A.offsets_t[it.key];
       it.end = A.offsets_t[it.key + 1];
       it.dep_idx = A.ctr_g_t + it.key;
+      it.oh_begin = A.oh_off[it.key];
+      it.oh_end = A.oh_off[it.key + 1];
     }
     it.dep_val = it.end - it.begin;
     // test hook: the dE items of the first chunk wait for one gradient tile more than the pairs
@@ -564,9 +569,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         red_release_add(A.counters + A.ctr_b_done + it.chunk, 1);
       }
       if (de && !has) continue;  // nothing to add for this row block in this chunk
+      // dC: onehot terms of rows whose target tile was skipped and whose target is this thread's
+      // row of the tile (at most two remembered; more are rare and handled by a second scan)
+      int oh_r[2] = {-1, -1};
+      float oh_c[2] = {0.f, 0.f};
+      bool oh_more = false;
+      if (!de && it.oh_begin < it.oh_end) {
+        const int64_t my_v = static_cast<int64_t>(it.key) * BN + q * 32 + lane;
+        int n = 0;
+        for (int i = it.oh_begin; i < it.oh_end; ++i) {
+          const int r = A.oh_rows[i];
+          if (A.targets[r] != my_v) continue;
+          if (n < 2) {
+            oh_r[n] = r;
+            oh_c[n] = -A.scale[r] * A.onehot_coef;
+          } else {
+            oh_more = true;
+          }
+          ++n;
+        }
+      }
       if (!region_free()) break;
       const int rows_limit = de ? A.N : A.V;
       const int y = it.key * BM + q * 32;
+      // the first matched row's 64 columns for the next step are loaded one step ahead
+      uint4 oh_next[8];
+      auto load_row = [&](int x) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          oh_next[k] = x + 8 * k < A.D ? ld_global_nc_v4(A.E + static_cast<int64_t>(oh_r[0]) * A.D + x + 8 * k)
+                                       : make_uint4(0, 0, 0, 0);
+      };
+      if (oh_r[0] >= 0) load_row(it.s * SLICE);
       for (int p = 0; p < SLICE / 64; ++p) {
         const int x = it.s * SLICE + 64 * p;
         if (x >= A.D) break;
@@ -577,6 +611,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) v0[e] = v1[e] = 0.f;
+        }
+        if (oh_r[0] >= 0) {  // -scale_r (1 - ls) E_r for those rows
+          auto add_vals = [&](const uint4 (&u8)[8], float coef) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint32_t w4[4] = {u8[k].x, u8[k].y, u8[k].z, u8[k].w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                __nv_bfloat162 h;
+                *reinterpret_cast<uint32_t*>(&h) = w4[j];
+                float* dst = k < 4 ? v0 + 8 * k + 2 * j : v1 + 8 * (k - 4) + 2 * j;
+                dst[0] = fmaf(coef, __low2float(h), dst[0]);
+                dst[1] = fmaf(coef, __high2float(h), dst[1]);
+              }
+            }
+          };
+          auto add_row = [&](int r, float coef) {
+            uint4 u8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              u8[k] = x + 8 * k < A.D ? ld_global_nc_v4(A.E + static_cast<int64_t>(r) * A.D + x + 8 * k)
+                                      : make_uint4(0, 0, 0, 0);
+            add_vals(u8, coef);
+          };
+          uint4 cur[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) cur[k] = oh_next[k];
+          if (p + 1 < SLICE / 64 && x + 64 < A.D) load_row(x + 64);
+          add_vals(cur, oh_c[0]);
+          if (oh_r[1] >= 0) add_row(oh_r[1], oh_c[1]);
+          if (oh_more) {
+            const int64_t my_v = static_cast<int64_t>(it.key) * BN + q * 32 + lane;
+            int n = 0;
+            for (int i = it.oh_begin; i < it.oh_end; ++i) {
+              const int r = A.oh_rows[i];
+              if (A.targets[r] != my_v) continue;
+              if (n++ >= 2) add_row(r, -A.scale[r] * A.onehot_coef);
+            }
+          }
         }
         if (!de && A.dc_add != nullptr) {  // the smoothing term, the same for every row of dC
 #pragma unroll

@@ -5,10 +5,12 @@
 // max over the tile of z[r, v] - LSE_r >= ln(eps) (mlx-cross-entropy README, "How it works" item 2:
 // skip tiles whose softmax is below 2^-12), judged from the forward's saved per-sub-tile maxima.
 // A skipped tile that holds the target of one of its rows still carries the onehot term of
-// p - y (Loss functions explainer, "How it works" item 2), which is never skipped; it is listed as
-// "onehot only" (its gradient tile is -scale_r at (r, t_r) and zero elsewhere, no recompute).
+// p - y (Loss functions explainer, "How it works" item 2), which is never skipped. Such a tile
+// ("onehot only") is not listed: its rows' onehot terms are applied one row at a time, listed by
+// vocabulary tile in oh_off / oh_rows (dC adds -scale_r (1 - ls) E_r to row t_r, dE adds
+// -scale_r (1 - ls) C_{t_r} to row r).
 //
-// flags[b * nt + t]: 0 = no gradient, 1 = kept, 2 = onehot only.
+// flags[b * nt + t]: 0 = no gradient, 1 = kept (listed), 2 = onehot only.
 // By vocabulary tile (recompute and dC kernels): offsets_t[t] .. offsets_t[t+1] index entries_t,
 //   each (b * 4 + flag, t), row blocks ascending. An entry's position is also its gradient-tile slot.
 // By row block (dE kernel): offsets_b[b] .. offsets_b[b+1] index entries_b, each (t, slot),
@@ -74,8 +76,8 @@ __global__ void tile_rank_kernel(const uint8_t* __restrict__ flags, int nb, int 
   for (int b0 = 0; b0 < nb; b0 += 32) {
     const int b = b0 + lane;
     const uint8_t f = b < nb ? flags[static_cast<int64_t>(b) * nt + t] : 0;
-    const unsigned on = __ballot_sync(0xffffffffu, f != 0);
-    if (f != 0) {
+    const unsigned on = __ballot_sync(0xffffffffu, f == 1);
+    if (f == 1) {
       rank[static_cast<int64_t>(b) * nt + t] = listed + __popc(on & ((1u << lane) - 1u));
       atomicAdd(cnt_b + b, 1);
     }
@@ -118,7 +120,7 @@ __global__ void fill_col_kernel(const uint8_t* __restrict__ flags, const int* __
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= static_cast<int64_t>(nb) * nt) return;
   const uint8_t f = flags[i];
-  if (f == 0) return;
+  if (f != 1) return;
   const int b = static_cast<int>(i / nt), t = static_cast<int>(i % nt);
   entries_t[offsets_t[t] + rank[i]] = make_int2(b * 4 + f, t);
 }
@@ -137,7 +139,7 @@ __global__ void row_list_kernel(const uint8_t* __restrict__ flags, const int* __
   __syncthreads();
   for (int t0 = 0; t0 < nt; t0 += 1024) {
     const int t = t0 + threadIdx.x;
-    const bool on = t < nt && row[t] != 0;
+    const bool on = t < nt && row[t] == 1;
     const unsigned m = __ballot_sync(0xffffffffu, on);
     if (lane == 0) wsum[w] = __popc(m);
     __syncthreads();
@@ -253,6 +255,22 @@ __global__ void group_size_kernel(const int* __restrict__ pstart_t, const int* _
   }
 }
 
+// Rows whose target tile is onehot only: counted (pass 0) or written (pass 1, positions from the
+// scanned counts and a per-tile cursor) per vocabulary tile of the target.
+__global__ void onehot_rows_kernel(const uint8_t* __restrict__ flags, const int64_t* __restrict__ targets,
+                                   int64_t N, int64_t V, int64_t ignore_index, int nt, int* __restrict__ cnt,
+                                   const int* __restrict__ off, int* __restrict__ rows, int pass) {
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < N;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t tr = targets[r];
+    if (!valid_target(tr, V, ignore_index)) continue;
+    const int t = static_cast<int>(tr / kBwdBN);
+    if (flags[(r / kBwdBM) * nt + t] != 2) continue;
+    const int k = atomicAdd(cnt + t, 1);
+    if (pass == 1) rows[off[t] + k] = static_cast<int>(r);
+  }
+}
+
 __global__ void plan_finish_kernel(const int* __restrict__ kept_total, int64_t total, int64_t* __restrict__ filtered) {
   *filtered = total - static_cast<int64_t>(*kept_total);
 }
@@ -307,6 +325,21 @@ cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float
     group_size_kernel<<<(P.nchunks + 255) / 256, 256, 0, s>>>(P.pstart_t, P.chunk_t, nb, P.S, P.nchunks, P.grp_size);
     note_launches(1);
     scan_kernel<<<1, 1024, 0, s>>>(P.grp_size, 2 * P.nchunks, P.grp_start);
+    note_launches(1);
+  }
+  if (nb > 0) {
+    e = cudaMemsetAsync(P.oh_cnt, 0, sizeof(int) * static_cast<size_t>(nt), s);
+    if (e != cudaSuccess) return e;
+    const int grid_r = static_cast<int>(std::min<int64_t>((N + 255) / 256, 4096));
+    onehot_rows_kernel<<<grid_r, 256, 0, s>>>(P.flags, targets, N, V, ignore_index, nt, P.oh_cnt, P.oh_off,
+                                              P.oh_rows, 0);
+    note_launches(1);
+    scan_kernel<<<1, 1024, 0, s>>>(P.oh_cnt, nt, P.oh_off);
+    note_launches(1);
+    e = cudaMemsetAsync(P.oh_cnt, 0, sizeof(int) * static_cast<size_t>(nt), s);
+    if (e != cudaSuccess) return e;
+    onehot_rows_kernel<<<grid_r, 256, 0, s>>>(P.flags, targets, N, V, ignore_index, nt, P.oh_cnt, P.oh_off,
+                                              P.oh_rows, 1);
     note_launches(1);
   }
   plan_finish_kernel<<<1, 1, 0, s>>>(P.kept_total, static_cast<int64_t>(nb) * nt, filtered_tiles);

@@ -75,6 +75,9 @@ struct BwdPlan {
   int2* pair_slot;  // [pair capacity]: gradient-tile slots of t0 and t1, relative to the chunk
   int* grp_size;    // [2 * nchunks]: work items of each queue group (pairs of chunk c, then its dE/dC)
   int* grp_start;   // [2 * nchunks + 1]: their prefix sums
+  int* oh_cnt;      // [nt]: rows whose target tile is onehot only, per vocabulary tile (scratch)
+  int* oh_off;      // [nt + 1]: their prefix sums
+  int* oh_rows;     // [N]: those rows, grouped by the vocabulary tile of their target
 };
 
 // Everything the persistent backward kernel reads besides its tensor maps.
@@ -92,6 +95,9 @@ struct BwdArgs {
   float onehot_coef;          // 1 - label_smoothing: weight of the onehot part of G
   const float* dc_add;        // [D] or null: added, times dc_coef, to every row of dC
   float dc_coef;
+  const __nv_bfloat16* E;     // rows of the onehot-only targets, added into their dC rows
+  const int* oh_off;          // [nt + 1]
+  const int* oh_rows;         // rows whose target tile is onehot only, by vocabulary tile
   const int* grp_start;
   const int* chunk_t;
   const int* pstart_t;
@@ -142,6 +148,11 @@ cudaError_t launch_add_rank1(float* X, int64_t rows, int64_t D, const float* sca
                              cudaStream_t s);
 // X[0:n] += coef * (*c).
 cudaError_t launch_add_scalar(float* X, int64_t n, float coef, const float* c, cudaStream_t s);
+// The onehot term of rows whose target tile was skipped: dE_acc[r] -= coef scale_r C[t_r] and
+// dbias_acc[t_r] -= coef scale_r (dbias_acc may be null), for the rows listed in rows[0:off[nt]].
+cudaError_t launch_onehot_rows(const int* off, int nt, const int* rows, const int64_t* targets,
+                               const float* scale, float coef, const __nv_bfloat16* C, int64_t D, float* dE_acc,
+                               float* dbias_acc, int64_t max_rows, cudaStream_t s);
 cudaError_t launch_loss_reduce(const float* loss_rows, const int64_t* targets, int64_t N, int64_t ignore_index,
                                int reduction, float* loss, int64_t* count, cudaStream_t s);
 cudaError_t launch_row_scale(const int64_t* targets, const int64_t* count, const float* grad_out, int64_t N,
