@@ -38,7 +38,7 @@ L2_FLUSH_BYTES = 512 << 20
 # 1117061120 algorithmic bytes (E and C read once, the per-sub-tile max and sum written once).
 FWD_TRAFFIC_BYTES = {(4096, 4096, 128256): 1084700416 + 32192256}
 # The same for one bwd_kernel launch (a one-pass capture of the current kernel at that shape).
-BWD_TRAFFIC_BYTES = {(4096, 4096, 128256): 5885730560 + 2328704256}
+BWD_TRAFFIC_BYTES = {(4096, 4096, 128256): 5922187776 + 2340610304}
 
 
 def load_peaks():

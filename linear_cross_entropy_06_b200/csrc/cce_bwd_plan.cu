@@ -32,36 +32,47 @@ __device__ __forceinline__ bool valid_target(int64_t t, int64_t V, int64_t ignor
   return t != ignore_index && t >= 0 && t < V;
 }
 
-// One block of 128 threads (one per tile row) per backward tile (b, t) = (i / nt, i % nt): its flag.
+// One block of 128 threads (one per tile row) per row block b and run of kFlagTiles vocabulary
+// tiles: the flags of those tiles. The rows' targets and LSE are read once for the whole run.
+constexpr int kFlagTiles = 8;
+
 __global__ void tile_flags_kernel(const float* __restrict__ tile_max, const float* __restrict__ lse,
                                   const int64_t* __restrict__ targets, int64_t N, int64_t V, int64_t T,
-                                  int64_t ignore_index, float ln_eps, int filter_on, int nt,
+                                  int64_t ignore_index, float ln_eps, int filter_on, int nt, int runs,
                                   uint8_t* __restrict__ flags) {
-  __shared__ float wmax[4];
-  const int64_t i = blockIdx.x;
-  const int b = static_cast<int>(i / nt), t = static_cast<int>(i % nt);
-  const int64_t v0 = static_cast<int64_t>(t) * kBwdBN;
+  __shared__ float wmax[kFlagTiles][4];
+  __shared__ int any_target[kFlagTiles];
+  const int b = static_cast<int>(blockIdx.x / runs), t0 = static_cast<int>(blockIdx.x % runs) * kFlagTiles;
   const int64_t r = static_cast<int64_t>(b) * kBwdBM + threadIdx.x;
-  float m = -INFINITY;
-  bool has_target = false;
+  if (threadIdx.x < kFlagTiles) any_target[threadIdx.x] = 0;
+  __syncthreads();
+  bool valid = false;
+  float l = 0.f;
+  int64_t tr = -1;
   if (r < N) {
-    const int64_t tr = targets[r];
-    if (valid_target(tr, V, ignore_index)) {
-      has_target = tr >= v0 && tr < v0 + kBwdBN;
-      if (filter_on) {
-        const int64_t j0 = static_cast<int64_t>(t) * (kBwdBN / kSubTile);
-        const int64_t j1 = j0 + kBwdBN / kSubTile < T ? j0 + kBwdBN / kSubTile : T;
-        for (int64_t j = j0; j < j1; ++j) m = fmaxf(m, tile_max[j * N + r]);
-        m -= lse[r];
-      }
-    }
+    tr = targets[r];
+    valid = valid_target(tr, V, ignore_index);
+    if (valid && filter_on) l = lse[r];
   }
-  m = warp_max(m);
-  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
-  const int any_target = __syncthreads_or(has_target ? 1 : 0);
-  if (threadIdx.x == 0) {
-    const bool keep = !filter_on || fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3])) >= ln_eps;
-    flags[i] = keep ? 1 : (any_target ? 2 : 0);
+  if (valid && tr / kBwdBN >= t0 && tr / kBwdBN < t0 + kFlagTiles) any_target[tr / kBwdBN - t0] = 1;
+#pragma unroll
+  for (int k = 0; k < kFlagTiles; ++k) {
+    const int t = t0 + k;
+    float m = -INFINITY;
+    if (valid && filter_on && t < nt) {
+      const int64_t j0 = static_cast<int64_t>(t) * (kBwdBN / kSubTile);
+      const int64_t j1 = j0 + kBwdBN / kSubTile < T ? j0 + kBwdBN / kSubTile : T;
+      for (int64_t j = j0; j < j1; ++j) m = fmaxf(m, tile_max[j * N + r]);
+      m -= l;
+    }
+    m = warp_max(m);
+    if ((threadIdx.x & 31) == 0) wmax[k][threadIdx.x >> 5] = m;
+  }
+  __syncthreads();
+  if (threadIdx.x < kFlagTiles && t0 + threadIdx.x < nt) {
+    const int k = threadIdx.x;
+    const bool keep = !filter_on || fmaxf(fmaxf(wmax[k][0], wmax[k][1]), fmaxf(wmax[k][2], wmax[k][3])) >= ln_eps;
+    flags[static_cast<int64_t>(b) * nt + t0 + k] = keep ? 1 : (any_target[k] ? 2 : 0);
   }
 }
 
@@ -287,8 +298,9 @@ cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float
   if (e != cudaSuccess) return e;
   if (nb > 0) {
     const int64_t tiles = static_cast<int64_t>(nb) * nt;
-    tile_flags_kernel<<<static_cast<unsigned>(tiles), kBwdBM, 0, s>>>(tile_max, lse, targets, N, V, T, ignore_index,
-                                                                     ln_eps, filter_on, nt, P.flags);
+    const int runs = (nt + kFlagTiles - 1) / kFlagTiles;
+    tile_flags_kernel<<<static_cast<unsigned>(static_cast<int64_t>(nb) * runs), kBwdBM, 0, s>>>(
+        tile_max, lse, targets, N, V, T, ignore_index, ln_eps, filter_on, nt, runs, P.flags);
     note_launches(1);
     e = cudaMemsetAsync(P.cnt_b, 0, sizeof(int) * static_cast<size_t>(nb), s);
     if (e != cudaSuccess) return e;
