@@ -7,15 +7,17 @@
 // abstract (logits are recomputed blockwise and never stored).
 //
 // Work items, per vocabulary chunk c (its gradient tiles live in scratch buffer c mod kGradBuffers):
-//   pair   two consecutive listed 128 x 128 tiles (b, t0), (b, t1) of row block b in the chunk:
-//          S = E_b [C_t0; C_t1]^T (tcgen05 M=128 N=256 K=D), then
-//          G = scale_r * exp(S - LSE_r) - scale_r * [v = t_r] in fp32, rounded to bf16 into a
-//          128B-swizzled shared tile, one 32 KB bulk store per tile into the scratch buffer.
+//   pair   two consecutive listed (kept) 128 x 128 tiles (b, t0), (b, t1) of row block b in the
+//          chunk: S = E_b [C_t0; C_t1]^T (+ bias) (tcgen05 M=128 N=256 K=D), then
+//          G = scale_r (1 + 2 zl LSE_r) exp(S - LSE_r) - scale_r (1 - ls) [v = t_r] in fp32, rounded
+//          to bf16 into a 128B-swizzled shared tile, one 32 KB bulk store per tile into the scratch
+//          buffer; with a dbias output, the column sums of the fp32 G are added into it.
 //   dE     (row block b, 256-column slice s of D): sum over the chunk's listed t of G_bt C_t[:, s]
 //          in TMEM, then one fp32 TMA reduce-add into dE_acc (split-reduce over chunks).
 //   dC     (vocabulary tile t, slice s): sum over the listed b of G_bt^T E_b[:, s] in TMEM (A = the
-//          same G tile read MN-major), written once by TMA store: every listed tile of t lies in
-//          t's chunk, so dC needs no reduction.
+//          same G tile read MN-major), plus the onehot terms of rows whose target tile in t was
+//          skipped and the label-smoothing term, written once by TMA store: every listed tile of t
+//          lies in t's chunk, so dC needs no reduction.
 //
 // Scheduling: a global queue holds the items in the order pairs(0), pairs(1), dE/dC(0), pairs(2),
 // dE/dC(1), ..., pairs(n-1), dE/dC(n-2), dE/dC(n-1): the dE/dC items of a chunk come one group of
@@ -39,7 +41,8 @@
 //   warp 1      TMEM owner (two 256-column fp32 buffers); one lane issues tcgen05.mma M=128 N=256.
 //   warps 2..5  write-out: G formation and bulk stores (pair), or TMEM -> swizzled staging -> TMA
 //               store / reduce-add (dC / dE), while the MMA fills the other TMEM buffer.
-//   warp 6      scheduler: claims and decodes items into an 8-deep shared ring.
+//   warp 6      scheduler: claims and decodes items into an 8-deep shared ring, at most LOOKAHEAD
+//               items ahead of the producer.
 #include "cce_device.cuh"
 #include "cce_internal.h"
 
