@@ -62,3 +62,44 @@ def test_noalloc_rejects_problems_beyond_its_scratch(device):
     assert st == 2  # CCE_ERR_UNSUPPORTED, before anything is enqueued
     assert b"scratch" in lib.cce_last_error_message()
     torch.cuda.synchronize()
+
+
+def test_noalloc_forward_replays_in_a_cuda_graph(device):
+    """The caller this entry point serves: the forward captured in a CUDA graph (no allocation
+    during capture), replayed on new inputs copied into the captured buffers."""
+    N, D, V = 512, 256, 8192
+    first = make_inputs("tiny", N=N, D=D, V=V, seed=61)
+    second = make_inputs("llama3.1-8b-head", N=N, D=D, V=V, seed=62)
+    E = first.E.to(device).clone()
+    C = first.C.to(device).clone()
+    t = first.targets.to(device).clone()
+    # warm-up call outside capture: resolves the scratch address and the driver entry point
+    st, *_ = _noalloc(E, C, t, "mean")
+    assert st == 0
+    torch.cuda.synchronize()
+    lib = ops.load_library()
+    p = ops.Problem(N, D, V, -100, ops.REDUCTION_CODES["mean"], 0)
+    loss = torch.empty(1, device=device)
+    lse = torch.empty(N, device=device)
+    tmax = torch.empty(lib.cce_tile_max_len(ctypes.byref(p)), device=device)
+    count = torch.empty(1, dtype=torch.int64, device=device)
+    graph = torch.cuda.CUDAGraph()
+    stream = torch.cuda.Stream(device)
+    stream.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(graph, stream=stream):
+            st = lib.cce_forward_noalloc(ctypes.byref(p), E.data_ptr(), C.data_ptr(), None, t.data_ptr(),
+                                         loss.data_ptr(), lse.data_ptr(), tmax.data_ptr(), count.data_ptr(),
+                                         stream.cuda_stream)
+    assert st == 0
+    for inp in (second, first):
+        E.copy_(inp.E.to(device))
+        C.copy_(inp.C.to(device))
+        t.copy_(inp.targets.to(device))
+        graph.replay()
+        torch.cuda.synchronize()
+        ref_loss, ref_lse, _, ref_count = ops.cce_forward(inp.E.to(device), inp.C.to(device),
+                                                          inp.targets.to(device), check=True)
+        assert abs(float(loss) - float(ref_loss)) <= 1e-5
+        assert (lse - ref_lse).abs().max().item() <= 1e-5
+        assert int(count) == int(ref_count)
