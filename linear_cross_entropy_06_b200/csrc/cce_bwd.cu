@@ -23,9 +23,9 @@
 // dE/dC(1), ..., pairs(n-1), dE/dC(n-2), dE/dC(n-1): the dE/dC items of a chunk come one group of
 // pairs after the chunk's own pairs, so their gradient tiles are normally stored by the time they
 // are claimed. CTAs claim items one at a time with an atomic counter, so a claimed item always
-// belongs to a running CTA. Inside a chunk the pairs are ordered by vocabulary tile and the dE
-// items by slice of D, so that the items running at the same time read the same C tiles and
-// columns from L2. Dependencies point only to earlier items:
+// belongs to a running CTA. Inside a chunk the pairs are ordered by vocabulary tile and the dE and
+// dC items by slice of D, so that the items running at the same time read the same C tiles and
+// the same columns of C and E from L2. Dependencies point only to earlier items:
 //   a dE item waits until every gradient tile of its row block in the chunk is stored, a dC item
 //   until every gradient tile of its vocabulary tile is, and a pair of chunk c waits, before it
 //   stores, until every dE/dC item of chunk c - kGradBuffers (the buffer's previous user) has
@@ -189,11 +189,12 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, const Bwd
       it.begin = r.x;
       it.end = r.y;
       it.dep_idx = A.ctr_g_b + c * A.nb + it.key;
-    } else {
+    } else {  // slice-major too: concurrent dC items read the same columns of E
       const int v = local - A.nb * S;
+      const int nvt = A.chunk_t[c + 1] - t_begin;
       it.kind = kDC;
-      it.key = t_begin + v / S;
-      it.s = v % S;
+      it.key = t_begin + v % nvt;
+      it.s = v / nvt;
       it.begin = A.offsets_t[it.key];
       it.end = A.offsets_t[it.key + 1];
       it.dep_idx = A.ctr_g_t + it.key;

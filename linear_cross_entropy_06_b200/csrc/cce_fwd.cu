@@ -13,8 +13,8 @@
 //               into one of two 256-column fp32 accumulators.
 //   warps 2..5  epilogue: TMEM -> registers, per-row max / sum-exp over each 128-column sub-tile
 //               while the MMA fills the other accumulator.
-// Tiles are visited row-block fastest, so the CTAs working at one time share a few C tiles
-// (read once from HBM, then from L2) and E stays in L2.
+// Tiles are visited row-block fastest within groups of 32 row blocks (see tile_coords), so the
+// CTAs working at one time share a few C tiles and E stays in L2.
 #include "cce_device.cuh"
 #include "cce_internal.h"
 
@@ -49,6 +49,21 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.tmem_holder = reinterpret_cast<uint32_t*>(s.bars + NUM_BARRIERS);
   s.abort = reinterpret_cast<int*>(s.tmem_holder + 1);
   return s;
+}
+
+// Tile w -> (row block, vocabulary tile). Row blocks are taken in groups of kRowGroup (32 x 128
+// rows: 8 MB of E per 1024 of D): row block fastest inside a group, then the next vocabulary tile,
+// and the next group after the last vocabulary tile. The CTAs running at one time then share a
+// few C tiles (read once from HBM per group) and at most one group of E rows, which stays in L2
+// however large N is.
+constexpr int kRowGroup = 32;
+
+__device__ __forceinline__ void tile_coords(int w, int nb, int nt, int& b, int& t) {
+  const int per_group = kRowGroup * nt;
+  const int g = w / per_group, in = w - g * per_group;
+  const int rows = min(kRowGroup, nb - g * kRowGroup);  // the last group may be short
+  t = in / rows;
+  b = g * kRowGroup + in % rows;
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -105,7 +120,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t issued[STAGES] = {0, 0, 0, 0};
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const int b = tile % nb, t = tile / nb;
+        int b, t;
+        tile_coords(tile, nb, nt, b, t);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, wc)) {
             ok = false;
@@ -182,7 +198,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const int b = tile % nb, t = tile / nb;
+      int b, t;
+      tile_coords(tile, nb, nt, b, t);
       if (!mbar_wait(tfull_bar(acc), acc_phase, wc)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
