@@ -14,7 +14,6 @@ constexpr int kErrTargetRange = 4;
 constexpr int kErrDeviceTimeout = 5;
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
