@@ -68,3 +68,30 @@ def test_token_shift_through_autograd(device):
     assert nll.shape == (B, T - 1)
     fn = O.forward(Es, inp.C, ts, reduction="none")
     assert np.abs(nll.double().cpu().numpy().reshape(-1) - fn.loss).max() <= LOSS_TOL
+
+
+@pytest.mark.parametrize("ignore_index", [3, 1000])
+def test_custom_ignore_index(device, ignore_index):
+    """ignore_index inside [0, V) masks exactly the tokens whose target equals it (class 3 is then
+    never a target), and one equal to V masks tokens whose target is V; with smoothing and z-loss,
+    reduction sum."""
+    N, D, V = 300, 136, 1000
+    inp = make_inputs("tiny", N=N, D=D, V=V, seed=71, ignore_frac=0.0)
+    t = inp.targets.clone()
+    t[::7] = ignore_index
+    t[1::11] = 3 if ignore_index != 3 else 4
+    E, C, tt = inp.E.to(device), inp.C.to(device), t.to(device)
+    g = torch.tensor([0.5], device=device)
+    loss, lse, tmax, count = ops.cce_forward(E, C, tt, ignore_index, "sum", check=True, label_smoothing=0.1,
+                                             z_loss=1e-3)
+    dE, dC, filt = ops.cce_backward(E, C, tt, lse, tmax, count, g, EPS, ignore_index, "sum", check=True,
+                                    label_smoothing=0.1, z_loss=1e-3)
+    f = O.forward(inp.E, inp.C, t, ignore_index, "sum", label_smoothing=0.1, z_loss=1e-3)
+    b = O.backward(inp.E, inp.C, t, 0.5, ignore_index, "sum", EPS, *ops.backward_tile_shape(), label_smoothing=0.1,
+                   z_loss=1e-3)
+    assert int(count.item()) == f.count == int((t != ignore_index).sum())
+    assert abs(float(loss.item()) - float(f.loss)) <= LOSS_TOL * f.count
+    assert rel_frob(dE.double().cpu().numpy(), b.dE) <= 1e-2
+    assert rel_frob(dC.double().cpu().numpy(), b.dC) <= 1e-2
+    raw = dE.cpu()[t == ignore_index]
+    assert (raw.view(torch.int16) == 0).all(), "dE rows of ignored tokens must be exactly +0"
