@@ -111,3 +111,29 @@ def test_status_strings(lib):
     for code in range(7):
         assert lib.cce_status_string(code)
     assert lib.cce_version() >= 300
+
+
+def test_plain_c_caller_compiles_links_and_runs():
+    """include/cce.h is valid C99 and libcce.so serves a C caller that has no Python or torch."""
+    import shutil
+    import subprocess
+    import tempfile
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(LIB)
+    with tempfile.TemporaryDirectory() as tmp:
+        exe = os.path.join(tmp, "abi_example")
+        subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                        os.path.join(root, "tests", "c", "abi_example.c"), "-o", exe, "-L", libdir, "-lcce",
+                        "-Wl,-rpath," + libdir], check=True, capture_output=True, text=True)
+        out = subprocess.run([exe], check=True, capture_output=True, text=True, timeout=60).stdout
+    vals = dict(line.split(" ", 1) for line in out.strip().splitlines())
+    assert int(vals["version"]) >= 300
+    assert vals["tile"] == "128 128"
+    assert int(vals["tile_max_len"]) == 4096 * ((128256 + 127) // 128)
+    assert int(vals["fwd_ws"]) > 0 and int(vals["bwd_ws"]) > 0
+    assert vals["bad_status"].startswith("1 ")  # CCE_ERR_INVALID_ARG
+    assert "multiple of 8" in vals["message"]
