@@ -327,3 +327,11 @@ def test_no_logit_sized_allocation_long_batch(device):
     m = _extra_loss_memory(device, N, D, V)
     assert m <= _memory_bound(N, V), (m, _memory_bound(N, V))
     assert m < N * V * 2 / 4, m
+
+
+@pytest.mark.parametrize("D", [8192, 12296])
+def test_large_hidden_sizes(device, D):
+    """Hidden sizes beyond the pages' heads: many 256-column slices per dE/dC item, and (12296 =
+    48 * 256 + 8) a last slice of 8 columns."""
+    inp = make_inputs("tiny", N=200, D=D, V=1500, seed=D, ignore_frac=0.1)
+    check_full(inp, device, "mean")
