@@ -140,14 +140,12 @@ def barrier(world: int):
 
 
 def algorithmic_flops(N: int, D: int, V: int, kept_tiles: int, tile: tuple) -> tuple:
-    """2NVD forward; 6 * rows * cols * D per kept backward tile (all tiles full at the bench shape)."""
+    """2NVD forward; 6 * rows * cols * D per kept backward tile (recompute, dE, dC).
+
+    Kept tiles are counted at their full size: at every bench workload N and V are multiples of
+    the tile, so none is partial (for ragged shapes this slightly overcounts the backward)."""
     tm, tn = tile
-    fwd = 2.0 * N * V * D
-    if N % tm == 0 and V % tn == 0:
-        bwd = 6.0 * tm * tn * D * kept_tiles
-    else:  # bound: kept tiles counted at full size
-        bwd = 6.0 * tm * tn * D * kept_tiles
-    return fwd, bwd
+    return 2.0 * N * V * D, 6.0 * tm * tn * D * kept_tiles
 
 
 def oracle_sample_seconds(inp, rows: int):

@@ -63,3 +63,17 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
 
     bench.run_reference(Args, world=2, rank=1)  # a non-zero rank does no work and prints nothing
     assert capsys.readouterr().out == ""
+
+
+def test_algorithmic_flops_definition():
+    """The metric's flop count: 2 N V D forward, 6 * 128 * 128 * D per kept 128 x 128 tile."""
+    import bench
+
+    fwd, bwd = bench.algorithmic_flops(4096, 4096, 128256, 7407, (128, 128))
+    assert fwd == 2 * 4096 * 128256 * 4096
+    assert bwd == 6 * 128 * 128 * 4096 * 7407
+    # every workload of the bench has N and V multiples of 128 (no partial tile is counted)
+    from linear_cross_entropy_06_b200.inputs import WORKLOADS
+    for w in WORKLOADS.values():
+        if w.name != "tiny":
+            assert w.N % 128 == 0 and w.V % 128 == 0, w.name
