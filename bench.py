@@ -31,6 +31,9 @@ import torch  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 EPS = 2.0 ** -12
+# The headline metric: tokens/s of one forward + backward at the Llama-3.1-8B head shape, with the
+# fraction of the B200 bf16 tensor peak reported beside it (tensor_peak_frac).
+METRIC = "fwd+bwd tokens/s at Llama-3-8B head shape; % of B200 BF16 tensor peak"
 L2_FLUSH_BYTES = 512 << 20
 # DRAM bytes (read + write) of one fwd_lse_kernel launch from a one-pass ncu capture of that launch
 # (dram__bytes_read.sum + dram__bytes_write.sum) at the given (N, D, V), reported as the roofline's
@@ -185,7 +188,7 @@ def run_reference(args, world, rank):
     value = rows * args.steps / total
     cores = torch.get_num_threads()
     line = {
-        "impl": "reference", "metric": "fwd+bwd tokens/s", "value": value, "unit": "tokens/s",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, args.gpus),
@@ -367,7 +370,7 @@ def run_ours(args, world, rank, local):
     if rank != 0:
         return
     line = {
-        "metric": "fwd+bwd tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w, world, (N, D, V)),
         "tensor_peak_frac": {"achieved_tflops": path_tflops, "peak": peak_tf, "frac": path_tflops / peak_tf,
