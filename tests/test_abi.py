@@ -137,3 +137,20 @@ def test_plain_c_caller_compiles_links_and_runs():
     assert int(vals["fwd_ws"]) > 0 and int(vals["bwd_ws"]) > 0
     assert vals["bad_status"].startswith("1 ")  # CCE_ERR_INVALID_ARG
     assert "multiple of 8" in vals["message"]
+
+
+def test_backward_scratch_grows_with_tokens_not_vocabulary(lib):
+    """The gradient-tile scratch is max(128 MiB, 4 MiB per 128 rows): doubling V adds only the
+    tile plan (tens of bytes per 128 x 128 tile), while going from 4096 to 32768 tokens adds the
+    scratch of 224 more row blocks besides the fp32 dE accumulator."""
+    def bw(N, V, D=4096, out_fp32=1):
+        p = _p(N=N, D=D, V=V, red=0)
+        return lib.cce_backward_workspace_size(ctypes.byref(p), out_fp32)
+
+    small, wide = bw(4096, 64128), bw(4096, 128256)
+    tiles_added = (4096 // 128) * (128256 // 128 - 64128 // 128)
+    assert 0 < wide - small <= 48 * tiles_added + (1 << 20)
+    big = bw(32768, 128256)
+    assert big - wide >= 224 * (4 << 20)
+    # nothing of size N*V: at the long-batch shape far below the bf16 logits (8.4 GB)
+    assert big < 32768 * 128256 * 2 // 4
