@@ -123,6 +123,25 @@ def _require_cuda(*tensors: torch.Tensor) -> torch.device:
     return dev
 
 
+def _require(cond: bool, message: str) -> None:
+    if not cond:
+        raise CCEError(1, message)
+
+
+def _check_operands(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor) -> Tuple[int, int, int]:
+    """Dtype and shape checks of E [N, D] bf16, C [V, D] bf16 and targets [N] int64 before any pointer
+    reaches the library: the kernels read exactly N*D, V*D and N elements of those types."""
+    _require(E.dim() == 2 and C.dim() == 2, f"E and C must be 2-D, got {tuple(E.shape)} and {tuple(C.shape)}")
+    _require(E.dtype == torch.bfloat16 and C.dtype == torch.bfloat16,
+             f"E and C must be bfloat16, got {E.dtype} and {C.dtype}")
+    N, D = E.shape
+    V = C.shape[0]
+    _require(C.shape[1] == D, f"C must be [V, {D}], got {tuple(C.shape)}")
+    _require(targets.dtype == torch.int64, f"targets must be int64, got {targets.dtype}")
+    _require(targets.numel() == N, f"targets must have N={N} entries, got {targets.numel()}")
+    return N, D, V
+
+
 def backward_tile_shape() -> Tuple[int, int]:
     lib = load_library()
     r, c = _I32(), _I32()
@@ -145,10 +164,9 @@ def cce_forward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, ignore_
                 label_smoothing: float = 0.0, z_loss: float = 0.0):
     """Run the forward (logits E C^T + bias). Returns (loss, lse, tile_max, count) as device tensors."""
     lib = load_library()
+    N, D, V = _check_operands(E, C, targets)
     dev = _require_cuda(E, C, targets)
     E, C, targets = E.contiguous(), C.contiguous(), targets.contiguous()
-    N, D = E.shape
-    V = C.shape[0]
     bias = _bias_arg(bias, V, dev)
     p = _problem(N, D, V, ignore_index, reduction, label_smoothing, z_loss)
     loss = torch.empty(N if reduction == "none" else 1, device=dev, dtype=torch.float32)
@@ -177,13 +195,22 @@ def cce_backward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, lse: t
     """Run the backward. Returns (dE, dC, filtered_tiles) as device tensors, and dbias as a fourth
     when it is computed (``dbias``; by default whenever ``bias`` is given)."""
     lib = load_library()
+    N, D, V = _check_operands(E, C, targets)
+    p = _problem(N, D, V, ignore_index, reduction, label_smoothing, z_loss)
+    tm_len = lib.cce_tile_max_len(ctypes.byref(p))
+    _require(tm_len >= 0, f"bad problem N={N} D={D} V={V}: {lib.cce_last_error_message().decode()}")
+    # the saved forward state, read in full by the backward's kernels
+    _require(lse.dtype == torch.float32 and lse.numel() == N, f"lse must be float32 with N={N} entries")
+    _require(tile_max.dtype == torch.float32 and tile_max.numel() >= tm_len,
+             f"tile_max must be float32 with at least {tm_len} entries")
+    _require(count.dtype == torch.int64 and count.numel() >= 1, "count must be an int64 tensor of one entry")
+    _require(grad_out.numel() == (N if reduction == "none" else 1),
+             f"grad_out must have {N if reduction == 'none' else 1} entries for reduction={reduction!r}")
     dev = _require_cuda(E, C, targets, lse, tile_max, count)
     E, C, targets = E.contiguous(), C.contiguous(), targets.contiguous()
-    N, D = E.shape
-    V = C.shape[0]
+    lse, tile_max, count = lse.contiguous(), tile_max.contiguous(), count.contiguous()
     bias = _bias_arg(bias, V, dev)
     want_dbias = (bias is not None) if dbias is None else bool(dbias)
-    p = _problem(N, D, V, ignore_index, reduction, label_smoothing, z_loss)
     g = grad_out.to(device=dev, dtype=torch.float32).reshape(-1).contiguous()
     out_dtype = torch.float32 if out_fp32 else torch.bfloat16
     dE = torch.empty(N, D, device=dev, dtype=out_dtype)

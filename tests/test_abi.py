@@ -154,3 +154,62 @@ def test_backward_scratch_grows_with_tokens_not_vocabulary(lib):
     assert big - wide >= 224 * (4 << 20)
     # nothing of size N*V: at the long-batch shape far below the bf16 logits (8.4 GB)
     assert big < 32768 * 128256 * 2 // 4
+
+
+def _operands(N=256, D=128, V=1000, e_dtype=None, t_dtype=None):
+    import torch
+    E = torch.zeros(N, D, dtype=e_dtype or torch.bfloat16)
+    C = torch.zeros(V, D, dtype=torch.bfloat16)
+    t = torch.zeros(N, dtype=t_dtype or torch.int64)
+    return E, C, t
+
+
+@pytest.mark.parametrize("case,needle", [
+    (dict(e_dtype="float32"), "bfloat16"),
+    (dict(e_dtype="float16"), "bfloat16"),
+    (dict(t_dtype="int32"), "int64"),
+])
+def test_binding_rejects_wrong_dtypes_before_the_library(lib, case, needle):
+    """The kernels read bf16 operands and int64 targets through raw pointers: any other dtype would
+    be read as the wrong type (int32 targets: past the end of their buffer), so the binding refuses."""
+    import torch
+    kw = {k: getattr(torch, v) for k, v in case.items()}
+    E, C, t = _operands(**kw)
+    with pytest.raises(ops.CCEError, match=needle) as ei:
+        ops.cce_forward(E, C, t)
+    assert ei.value.status == 1
+
+
+def test_binding_rejects_mismatched_shapes(lib):
+    import torch
+    E, C, t = _operands()
+    with pytest.raises(ops.CCEError, match="must be \\[V, 128\\]"):
+        ops.cce_forward(E, C[:, :64].contiguous(), t)
+    with pytest.raises(ops.CCEError, match="N=256 entries"):
+        ops.cce_forward(E, C, t[:255])
+    with pytest.raises(ops.CCEError, match="2-D"):
+        ops.cce_forward(E.reshape(2, 128, 128), C, t)
+
+
+def test_binding_checks_the_saved_forward_state_in_the_backward(lib):
+    """lse, tile_max and count are read in full by the backward's kernels: a short or mistyped buffer
+    is refused on the host (here on CPU tensors, which would be refused next anyway)."""
+    import torch
+    E, C, t = _operands()
+    p = _p(N=256, D=128, V=1000)
+    tm_len = lib.cce_tile_max_len(ctypes.byref(p))
+    lse = torch.zeros(256)
+    tmax = torch.zeros(tm_len)
+    count = torch.zeros(1, dtype=torch.int64)
+    g = torch.ones(())
+    with pytest.raises(ops.CCEError, match="tile_max"):
+        ops.cce_backward(E, C, t, lse, tmax[:-1], count, g)
+    with pytest.raises(ops.CCEError, match="lse"):
+        ops.cce_backward(E, C, t, lse.double(), tmax, count, g)
+    with pytest.raises(ops.CCEError, match="count"):
+        ops.cce_backward(E, C, t, lse, tmax, count.int(), g)
+    with pytest.raises(ops.CCEError, match="grad_out must have 256"):
+        ops.cce_backward(E, C, t, lse, tmax, count, g, reduction="none")
+    # well-formed CPU tensors reach the device check: there is no CPU path
+    with pytest.raises(ops.CCEError, match="no CPU path"):
+        ops.cce_backward(E, C, t, lse, tmax, count, g)
