@@ -125,7 +125,9 @@ CCE_API cce_status cce_forward(const cce_problem* p, const void* E, const void* 
  * without a non-ignored row is skipped too. filter_eps <= 0 keeps every tile. The onehot term
  * is never skipped. Loss functions explainer, "How it works" item 2 (gradient p - y);
  * mlx-cross-entropy README, "How it works" items 2 and 3 (skipping, accumulation).
- * scale_r = g / max(count, 1) (mean), g (sum) or g[r] (none); 0 for ignored rows.
+ * scale_r = g / max(count, 1) (mean), g (sum) or g[r] (none); 0 for ignored rows. With the loss
+ * variants of cce_problem, G is scale_r times the logit gradient given there; only its softmax
+ * part (1 + 2 z_loss LSE) p~ is skipped.
  *
  *  E, C, bias, targets, lse, tile_max, count: as given to / produced by cce_forward() on the
  *           same problem (bias NULL for none)
