@@ -37,11 +37,11 @@ METRIC = "fwd+bwd tokens/s at Llama-3-8B head shape; % of B200 BF16 tensor peak"
 L2_FLUSH_BYTES = 512 << 20
 # DRAM bytes (read + write) of one fwd_lse_kernel launch from a one-pass ncu capture of that launch
 # (dram__bytes_read.sum + dram__bytes_write.sum) at the given (N, D, V), reported as the roofline's
-# "traffic". At the Llama-3.1-8B head shape: 1084700416 read + 32192256 written, against
+# "traffic". At the Llama-3.1-8B head shape: 1085342464 read + 35840256 written, against
 # 1117061120 algorithmic bytes (E and C read once, the per-sub-tile max and sum written once).
-FWD_TRAFFIC_BYTES = {(4096, 4096, 128256): 1084700416 + 32192256}
-# The same for one bwd_kernel launch (a one-pass capture of the current kernel at that shape).
-BWD_TRAFFIC_BYTES = {(4096, 4096, 128256): 5922187776 + 2340610304}
+FWD_TRAFFIC_BYTES = {(4096, 4096, 128256): 1085342464 + 35840256}
+# The same for one bwd_kernel launch (the same capture, of the current kernel at that shape).
+BWD_TRAFFIC_BYTES = {(4096, 4096, 128256): 5987639040 + 2336519168}
 
 
 def load_peaks():
