@@ -35,6 +35,9 @@ EPS = 2.0 ** -12
 # fraction of the B200 bf16 tensor peak reported beside it (tensor_peak_frac).
 METRIC = "fwd+bwd tokens/s at Llama-3-8B head shape; % of B200 BF16 tensor peak"
 L2_FLUSH_BYTES = 512 << 20
+# The skip rule's tile (rows x vocabulary columns) given to the oracle when it is timed: the
+# backward's tile shape, stated here so that timing the oracle never loads the CUDA library.
+ORACLE_SKIP_TILE = (128, 128)
 # DRAM bytes (read + write) of one fwd_lse_kernel launch from a one-pass ncu capture of that launch
 # (dram__bytes_read.sum + dram__bytes_write.sum) at the given (N, D, V), reported as the roofline's
 # "traffic". At the Llama-3.1-8B head shape: 1085342464 read + 35840256 written, against
@@ -155,13 +158,7 @@ def oracle_sample_seconds(inp, rows: int):
     """fp64 oracle forward + backward on the first `rows` tokens of the workload (full vocabulary)."""
     from oracle import cce_oracle as O
 
-    from linear_cross_entropy_06_b200.ops import backward_tile_shape
-
-    tm, tn = 128, 128
-    try:
-        tm, tn = backward_tile_shape()
-    except Exception:
-        pass
+    tm, tn = ORACLE_SKIP_TILE
     w = inp.workload
     E, t = inp.E[:rows], inp.targets[:rows]
     g = inp.grad_out[:rows] if w.reduction == "none" else inp.grad_out

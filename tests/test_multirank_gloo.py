@@ -77,3 +77,36 @@ def test_algorithmic_flops_definition():
     for w in WORKLOADS.values():
         if w.name != "tiny":
             assert w.N % 128 == 0 and w.V % 128 == 0, w.name
+
+
+def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
+    """--impl reference on rank 0: one JSON line timing the fp64 oracle on the host, with its own
+    cpu_baseline and an e2e that moves no bytes; the CUDA library is never loaded for it."""
+    import json
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from linear_cross_entropy_06_b200 import ops
+
+    def refuse(*a, **k):
+        raise AssertionError("the reference arm loaded the CUDA library")
+
+    monkeypatch.setattr(ops, "load_library", refuse)
+
+    class Args:
+        workload, steps, warmup, ref_rows, gpus = "tiny", 2, 1, 16, 1
+
+    bench.run_reference(Args, world=1, rank=0)
+    out = capsys.readouterr().out.strip().splitlines()
+    assert len(out) == 1
+    line = json.loads(out[0])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True and line["value"] > 0
+    assert line["steps"] == 2 and line["warmup"] == 1 and line["n_gpus"] == 1
+    assert line["config"]["workload"] == "tiny"
+    cpu = line["cpu_baseline"]
+    assert cpu["kind"] == "oracle" and cpu["value"] == line["value"] and cpu["cores"] >= 1 and cpu["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert bench.ORACLE_SKIP_TILE == (128, 128)
