@@ -42,7 +42,7 @@ def _worker(rank, world, port, out):
 def test_two_gloo_ranks_agree_on_the_slowest_time():
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:  # no fork of this multi-threaded process
         out = m.dict()
         mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
         res = dict(out)
