@@ -10,8 +10,9 @@
  *
  * Conventions for every call:
  *  - Pointers marked "device" are CUDA device pointers of the current device. The caller owns
- *    every buffer, workspaces included; the library allocates nothing and keeps no state
- *    between calls.
+ *    every buffer, workspaces included. The library allocates nothing and keeps no state between
+ *    calls, with two exceptions: the fixed scratch array of cce_forward_noalloc() and the
+ *    optional per-thread instrumentation set by cce_set_kernel_events().
  *  - E and C are bf16, row-major with contiguous rows (row stride = D elements). D must be a
  *    multiple of 8 and every pointer 16-byte aligned. targets is int64 [N].
  *  - All work is enqueued on `stream` and is asynchronous. Argument errors are returned
