@@ -68,24 +68,28 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.path = None
+        self.out = None
 
     def start(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+        self.out = os.fdopen(fd, "w")
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
         time.sleep(0.3)
 
     def stop(self):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+        self.out.close()
         if self.proc is None:
+            os.unlink(self.path)
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.2)
-        self.proc.terminate()
-        self.proc.wait(timeout=10)
         rows = []
         with open(self.path) as f:
             for line in f:
@@ -100,9 +104,9 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
         busy = [s for s in sm if s > 0.5 * (max(sm) if sm else 0)]
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
         return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None}
 
 
 def dist_setup():
@@ -169,6 +173,16 @@ def oracle_sample_seconds(inp, rows: int):
     return time.perf_counter() - t0
 
 
+def oracle_threads() -> int:
+    """Threads the oracle's arithmetic runs on: its one library step is numpy's matmul, so the size
+    of the BLAS thread pool numpy loaded (threadpoolctl), not torch's intra-op pool."""
+    import numpy  # noqa: F401  (loads the BLAS whose pool is inspected)
+    from threadpoolctl import threadpool_info
+
+    blas = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+    return max(blas) if blas else 1
+
+
 def run_reference(args, world, rank):
     """--impl reference: the fp64 CPU oracle, as it stands, on a bounded row sample per step."""
     if rank != 0:
@@ -183,7 +197,7 @@ def run_reference(args, world, rank):
     secs = [oracle_sample_seconds(inp, rows) for _ in range(args.steps)]
     total = sum(secs)
     value = rows * args.steps / total
-    cores = torch.get_num_threads()
+    cores = oracle_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
@@ -371,7 +385,7 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu:
         rows = args.cpu_rows
         secs = oracle_sample_seconds(inp, rows)
-        cpu = {"value": rows / secs, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
+        cpu = {"value": rows / secs, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
                "sample": f"first {rows} of {N} tokens, full V={V} and D={D}, fp64 forward + backward, {secs:.1f} s"}
 
     if rank != 0:

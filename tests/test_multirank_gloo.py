@@ -110,3 +110,45 @@ def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert bench.ORACLE_SKIP_TILE == (128, 128)
+    # cores = the BLAS pool that runs the oracle's matmul, at least one thread and at most the host's CPUs
+    assert cpu["cores"] == bench.oracle_threads() and 1 <= cpu["cores"] <= (os.cpu_count() or 1)
+
+
+def test_clock_sampler_parses_samples_and_reasons(monkeypatch):
+    """The clocks object of the bench line, from nvidia-smi's CSV: median SM clock under load (idle
+    samples below half the top clock are left out), max clock, and every throttle reason seen."""
+    import subprocess
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    samples = [
+        "0, 345, 1965, 120.5, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, 1965, 1965, 650.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1950, 1965, 700.2, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1905, 1965, 710.9, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+
+    class FakeSmi:
+        def __init__(self, cmd, stdout=None, stderr=None):
+            assert cmd[0] == "nvidia-smi" and "-lms" in cmd
+            stdout.write("\n".join(samples) + "\n")
+            stdout.flush()
+
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    monkeypatch.setattr(subprocess, "Popen", FakeSmi)
+    monkeypatch.setattr(bench.time, "sleep", lambda s: None)
+    c = bench.ClockSampler(0)
+    c.start()
+    out = c.stop()
+    assert out["sm_mhz"] == 1950.0  # median of 1965, 1950, 1905; the idle 345 is left out
+    assert out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"]
+    assert out["samples"] == 4 and out["power_w_max"] == 710.9
+    assert not os.path.exists(c.path)
