@@ -12,15 +12,6 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built libcce.so")
 
 
-def cuda_ready() -> bool:
-    try:
-        import torch
-
-        return torch.cuda.is_available()
-    except Exception:  # pragma: no cover
-        return False
-
-
 @pytest.fixture(scope="session")
 def device():
     import torch
