@@ -289,6 +289,7 @@ class BackwardResult:
     borderline: int  # tiles whose margin is within `window` of ln(eps)
     n_tiles: int
     dbias: Optional[np.ndarray] = None  # [V] when a bias is given
+    margin: Optional[np.ndarray] = None  # [ceil(N/tile_m), ceil(V/tile_n)] max over valid rows of z - LSE
 
 
 def backward(E, C, targets, grad_out=1.0, ignore_index: int = -100, reduction: str = "mean",
@@ -320,7 +321,7 @@ def backward(E, C, targets, grad_out=1.0, ignore_index: int = -100, reduction: s
     if filter_eps > 0:
         borderline = int((np.abs(margin - math.log(filter_eps)) < window).sum())
     return BackwardResult(G @ C64, G.T @ E64, int(skip.sum()), borderline, skip.size,
-                          None if bias is None else G.sum(axis=0))
+                          None if bias is None else G.sum(axis=0), margin)
 
 
 @dataclass
@@ -466,3 +467,80 @@ def row_blocks(E, C, targets, blocks: Sequence[int], grad_out=1.0, ignore_index:
         margins.append(m[0])
         pos += len(rr)
     return RowBlockResult(rows, lse, nll, np.array(margins), filtered, dE)
+
+
+@dataclass
+class VocabTileResult:
+    tiles: np.ndarray  # the vocabulary tiles evaluated, ascending
+    cols: np.ndarray  # their columns, tile after tile
+    margin: np.ndarray  # [ceil(N/tile_m), len(tiles)]
+    filtered: int  # skipped (row block, tile) pairs among the chosen tiles
+    dC: np.ndarray  # [len(cols), D]
+    dbias: Optional[np.ndarray] = None  # [len(cols)] when a bias is given
+
+
+def vocab_tiles(E, C, targets, lse, tiles: Sequence[int], grad_out=1.0, ignore_index: int = -100,
+                reduction: str = "mean", filter_eps: float = 2.0 ** -12, tile_m: int = 128, tile_n: int = 256,
+                bias=None, label_smoothing: float = 0.0, z_loss: float = 0.0) -> VocabTileResult:
+    """Exact dC (and dbias) rows of whole vocabulary tiles, given every row's LSE.
+
+    Column v of the logit gradient G needs only z[:, v], each row's LSE and the skip
+    decisions of the tiles that hold v; a tile's decision reads only its own rows and
+    columns (mlx-cross-entropy README, "How it works" item 2). So dC = G^T E and
+    dbias = sum_r G[r, :] restricted to whole tiles follow from E, the rows of C in
+    those tiles and the LSE vector of the same problem (from ``forward`` or
+    ``sampled``), with the per-row G of ``logit_grad`` (Loss functions explainer,
+    "How it works" items 2 and 3):
+    G[r, v] = scale_r ((1 + 2 zl LSE_r) p~[r, v] - (1 - ls) [v = t_r] - ls / V).
+    """
+    E64, C64, t = _f64(E), _f64(C), _i64(targets)
+    N, V = E64.shape[0], C64.shape[0]
+    bv = _bias64(bias, V)
+    validate_targets(t, V, ignore_index)
+    lse = _f64(lse).reshape(-1)
+    if lse.shape[0] != N:
+        raise ValueError(f"lse must have {N} entries, got {lse.shape[0]}")
+    tiles = np.asarray(sorted(set(int(x) for x in tiles)), dtype=np.int64)
+    nt = -(-V // tile_n)
+    if tiles.size and (tiles[0] < 0 or tiles[-1] >= nt):
+        raise ValueError(f"vocabulary tiles must lie in [0, {nt})")
+    if ROW_GROUP % tile_m:
+        raise ValueError("ROW_GROUP must be a multiple of tile_m")
+    cols = np.concatenate([np.arange(k * tile_n, min((k + 1) * tile_n, V)) for k in tiles]) if tiles.size \
+        else np.zeros(0, dtype=np.int64)
+    valid = t != ignore_index
+    count = int(valid.sum())
+    scale = row_scale(t, ignore_index, reduction, grad_out, count)
+    Cc = C64[cols]
+    nb = -(-N // tile_m)
+    margin = np.full((nb, len(tiles)), -np.inf)
+    dC = np.zeros((len(cols), E64.shape[1]))
+    dbias = np.zeros(len(cols)) if bv is not None else None
+    col_of = {int(v): j for j, v in enumerate(cols)}
+    for g in _row_groups(N):
+        z = E64[g] @ Cc.T
+        if bv is not None:
+            z += bv[cols][None, :]
+        l = lse[g]
+        vg, tg = valid[g], t[g]
+        m = tile_log_margin(z - l[:, None], vg, tile_m, tile_n)
+        b0 = g.start // tile_m
+        margin[b0:b0 + m.shape[0]] = m
+        p = softmax_rows(z, l)
+        skip = filtered_tiles(m, filter_eps)
+        for b, k in zip(*np.nonzero(skip)):
+            p[b * tile_m:(b + 1) * tile_m, k * tile_n:(k + 1) * tile_n] = 0.0
+        sc = scale[g]
+        G = (sc * (1.0 + 2.0 * z_loss * l))[:, None] * p
+        for i in np.flatnonzero(vg):
+            j = col_of.get(int(tg[i]))
+            if j is not None:
+                G[i, j] -= sc[i] * (1.0 - label_smoothing)
+        if label_smoothing:
+            G[vg] -= (sc[vg] * (label_smoothing / V))[:, None]
+        dC += G.T @ E64[g]
+        if dbias is not None:
+            dbias += G.sum(axis=0)
+        del z, p, G
+    skip_all = filtered_tiles(margin, filter_eps)
+    return VocabTileResult(tiles, cols, margin, int(skip_all.sum()), dC, dbias)

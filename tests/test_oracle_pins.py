@@ -526,3 +526,36 @@ def test_skipping_keeps_the_smoothing_term():
     G[np.arange(16), t] -= scale * (1 - ls)
     np.testing.assert_allclose(b_all.dC, G.T @ E, rtol=1e-12, atol=1e-15)
     np.testing.assert_allclose(b_all.dE, G @ C, rtol=1e-12, atol=1e-15)
+
+
+def test_vocab_tile_evaluation_agrees_with_full(monkeypatch):
+    """dC and dbias rows of whole vocabulary tiles from the LSE vector equal the full evaluation's,
+    with skipped tiles among the chosen ones, a ragged last tile, a bias, smoothing and z-loss."""
+    monkeypatch.setattr(O, "ROW_GROUP", 16)
+    rng = np.random.default_rng(34)
+    N, D, V, tn = 56, 128, 1000, 64  # 16 vocabulary tiles, the last one 40 columns wide
+    C = rng.standard_normal((V, D)) / np.sqrt(D)
+    t = rng.integers(0, V, N)
+    t[[4, 33]] = -100
+    t[:8] = rng.integers(0, 64, 8)  # some targets inside tile 0
+    E = 18.0 * C[np.where(t >= 0, t, 0)] + rng.standard_normal((N, D))
+    bias = rng.standard_normal(V) * 0.3
+    kw = dict(filter_eps=2.0 ** -12, tile_m=8, tile_n=tn, bias=bias, label_smoothing=0.1, z_loss=1e-3)
+    tiles = [15, 0, 7, 3]
+    for red in ("mean", "none"):
+        g = rng.standard_normal(N) if red == "none" else 0.7
+        f = O.forward(E, C, t, reduction=red, bias=bias, label_smoothing=0.1, z_loss=1e-3)
+        full = O.backward(E, C, t, grad_out=g, reduction=red, **kw)
+        r = O.vocab_tiles(E, C, t, f.lse, tiles, grad_out=g, reduction=red, **kw)
+        assert list(r.tiles) == sorted(tiles) and r.cols[-1] == V - 1 and len(r.cols) == 3 * tn + 40
+        np.testing.assert_allclose(r.dC, full.dC[r.cols], rtol=1e-11, atol=1e-14)
+        np.testing.assert_allclose(r.dbias, full.dbias[r.cols], rtol=1e-11, atol=1e-14)
+        margin = O.tile_log_margin(O.logits(E, C, bias) - f.lse[:, None], t != -100, 8, tn)[:, sorted(tiles)]
+        np.testing.assert_allclose(r.margin, margin, rtol=1e-13)
+        skipped = int(O.filtered_tiles(margin, 2.0 ** -12).sum())
+        assert r.filtered == skipped and 0 < skipped < margin.size
+    # a wrong LSE (one row shifted) must change the result: the function really reads it
+    lse_bad = f.lse.copy()
+    lse_bad[10] += 0.5
+    r_bad = O.vocab_tiles(E, C, t, lse_bad, tiles, grad_out=g, reduction="none", **kw)
+    assert np.abs(r_bad.dC - r.dC).max() > 1e-6
