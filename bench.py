@@ -38,13 +38,40 @@ L2_FLUSH_BYTES = 512 << 20
 # The skip rule's tile (rows x vocabulary columns) given to the oracle when it is timed: the
 # backward's tile shape, stated here so that timing the oracle never loads the CUDA library.
 ORACLE_SKIP_TILE = (128, 128)
-# DRAM bytes (read + write) of one fwd_lse_kernel launch from a one-pass ncu capture of that launch
-# (dram__bytes_read.sum + dram__bytes_write.sum) at the given (N, D, V), reported as the roofline's
-# "traffic". At the Llama-3.1-8B head shape: 1085342464 read + 35840256 written, against
-# 1117061120 algorithmic bytes (E and C read once, the per-sub-tile max and sum written once).
-FWD_TRAFFIC_BYTES = {(4096, 4096, 128256): 1085342464 + 35840256}
-# The same for one bwd_kernel launch (the same capture, of the current kernel at that shape).
-BWD_TRAFFIC_BYTES = {(4096, 4096, 128256): 5987639040 + 2336519168}
+# DRAM bytes (read + write) of one launch of each tensor-core kernel, from a one-kernel, one-launch,
+# one-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), reported as the roofline's
+# "traffic". Each entry is keyed by the workload's (N, D, V) and holds the SHA-256 of the kernel's
+# sources at the time of the capture: when those sources change, the figure no longer describes the
+# kernel and the bench reports null instead. See profiles/dram_traffic_*.md for the captures.
+KERNEL_SOURCES = {
+    "fwd_lse_kernel": ("cce_fwd.cu", "cce_device.cuh", "cce_internal.h"),
+    "bwd_kernel": ("cce_bwd.cu", "cce_device.cuh", "cce_internal.h"),
+}
+TRAFFIC_BYTES = {
+    "fwd_lse_kernel": {},
+    "bwd_kernel": {},
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """SHA-256 over the kernel's source files, in a fixed order."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "linear_cross_entropy_06_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel: str, shape: tuple):
+    """DRAM bytes per launch from the capture of this kernel at this shape, or None when there is
+    none or the kernel's sources changed since it was taken."""
+    entry = TRAFFIC_BYTES.get(kernel, {}).get(tuple(shape))
+    if entry is None:
+        return None
+    sha, nbytes = entry
+    return nbytes if sha == kernel_source_hash(kernel) else None
 
 
 def load_peaks():
@@ -298,21 +325,25 @@ def run_ours(args, world, rank, local):
     fwd_flop, bwd_flop = algorithmic_flops(N, D, V, kept, tile)
     peaks, peak_kind = load_peaks()
     peak_tf = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
-    fwd_avg, bwd_avg = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    peak_sus = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+
+    def kernel_line(flop, ms_list, what):
+        avg = statistics.mean(ms_list)
+        return {"ms": avg, "ms_median": statistics.median(ms_list), "ms_min": min(ms_list), "launches_per_step": 1,
+                "tflops": flop / avg / 1e9, "frac": flop / avg / 1e9 / peak_tf,
+                "frac_sustained": flop / avg / 1e9 / peak_sus, "what": what}
+
     kernels = {
-        "fwd_lse_kernel": {"ms": fwd_avg, "launches_per_step": 1, "tflops": fwd_flop / fwd_avg / 1e9,
-                           "frac": fwd_flop / fwd_avg / 1e9 / peak_tf},
-        "bwd_kernel": {
-            "ms": bwd_avg, "tflops": bwd_flop / bwd_avg / 1e9, "frac": bwd_flop / bwd_avg / 1e9 / peak_tf,
-            "launches_per_step": 1,
-            "what": "one persistent launch per step: recompute, gradient tiles, dC and dE MMAs"},
+        "fwd_lse_kernel": kernel_line(fwd_flop, fwd_ms, "persistent logit tiles with per-row max and sum-exp"),
+        "bwd_kernel": kernel_line(bwd_flop, bwd_ms,
+                                  "one persistent launch per step: recompute, gradient tiles, dC and dE MMAs"),
     }
     # The dominant kernel: the forward and the backward are one launch each per step; the roofline
-    # line reports the longer one.
-    if bwd_avg > fwd_avg:
-        dom, dom_flop, dom_ms, dom_traffic = "bwd_kernel", bwd_flop, bwd_avg, BWD_TRAFFIC_BYTES.get((N, D, V))
-    else:
-        dom, dom_flop, dom_ms, dom_traffic = "fwd_lse_kernel", fwd_flop, fwd_avg, FWD_TRAFFIC_BYTES.get((N, D, V))
+    # line reports the longer one (by average launch duration over the timed steps).
+    dom = "bwd_kernel" if kernels["bwd_kernel"]["ms"] > kernels["fwd_lse_kernel"]["ms"] else "fwd_lse_kernel"
+    dom_flop = bwd_flop if dom == "bwd_kernel" else fwd_flop
+    dom_ms = kernels[dom]["ms"]
+    dom_traffic = measured_traffic(dom, (N, D, V))
     ms_step = 1e3 * total_s / args.steps
     path_tflops = (fwd_flop + bwd_flop) / (ms_step / 1e3) / 1e12
 
@@ -394,12 +425,17 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w, world, (N, D, V)),
+        "ms_per_step_median": statistics.median(step_ms), "ms_per_step_min": min(step_ms),
         "tensor_peak_frac": {"achieved_tflops": path_tflops, "peak": peak_tf, "frac": path_tflops / peak_tf,
+                             "frac_sustained": path_tflops / peak_sus, "peak_sustained": peak_sus,
                              "peak_kind": f"bf16_tflops ({peak_kind})",
                              "flops_per_step": fwd_flop + bwd_flop, "kept_tiles": kept, "filtered_tiles": filtered},
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_flop / dom_ms / 1e9, "peak": peak_tf,
                      "unit": "TFLOP/s", "frac": dom_flop / dom_ms / 1e9 / peak_tf,
+                     "frac_sustained": dom_flop / dom_ms / 1e9 / peak_sus,
                      "traffic": dom_traffic,
+                     "traffic_source": None if dom_traffic is None else f"ncu capture of {dom} at this shape, "
+                                                                       f"sources sha256 {kernel_source_hash(dom)[:12]}",
                      "peak_kind": f"bf16_tflops ({peak_kind}, burst; the kernel is timed alone)",
                      "algorithmic_flops_per_launch": dom_flop},
         "kernels": kernels,

@@ -152,3 +152,21 @@ def test_clock_sampler_parses_samples_and_reasons(monkeypatch):
     assert out["reasons"] == ["sw_power_cap"]
     assert out["samples"] == 4 and out["power_w_max"] == 710.9
     assert not os.path.exists(c.path)
+
+
+def test_roofline_traffic_is_dropped_when_the_kernel_changes(monkeypatch):
+    """The roofline's DRAM traffic is a past ncu capture; it is reported only while the kernel's
+    sources hash to the value recorded with it, and is null for any other shape."""
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    sha = bench.kernel_source_hash("bwd_kernel")
+    assert len(sha) == 64 and sha == bench.kernel_source_hash("bwd_kernel")
+    assert sha != bench.kernel_source_hash("fwd_lse_kernel")
+    monkeypatch.setitem(bench.TRAFFIC_BYTES, "bwd_kernel", {(4096, 4096, 128256): (sha, 123456789)})
+    assert bench.measured_traffic("bwd_kernel", (4096, 4096, 128256)) == 123456789
+    assert bench.measured_traffic("bwd_kernel", (2048, 2048, 128256)) is None
+    monkeypatch.setitem(bench.TRAFFIC_BYTES, "bwd_kernel", {(4096, 4096, 128256): ("0" * 64, 123456789)})
+    assert bench.measured_traffic("bwd_kernel", (4096, 4096, 128256)) is None
