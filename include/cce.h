@@ -73,7 +73,23 @@ typedef struct {
    * Tile skipping drops only the softmax part; the rest is exact. */
   float label_smoothing; /* in [0, 1] */
   float z_loss;          /* >= 0 (PaLM uses 1e-4) */
+  /* Vocabulary sharding (the classifier split by rows over several GPUs, each holding a contiguous
+   * range of the vocabulary). vocab_total = 0: not sharded, C is the whole classifier (vocab_start
+   * must then be 0). vocab_total > 0: C holds rows [vocab_start, vocab_start + V) of a classifier of
+   * vocab_total rows, targets are ids in [0, vocab_total), and a target outside this shard's range
+   * marks a token that is scored here (its logits enter the softmax) but whose onehot term and
+   * correct-token logit belong to another shard. Forward: cce_forward_partial on every shard, an
+   * exchange of the partial results, then cce_forward_merge. Backward: cce_backward on every shard
+   * with the merged LSE and count; dC (and dbias) are this shard's rows, dE is this shard's part of
+   * dE, summed over the shards by the caller. */
+  int64_t vocab_start;
+  int64_t vocab_total;
 } cce_problem;
+
+/* Output dtypes of cce_backward (its out_fp32 argument). */
+#define CCE_OUT_BF16 0     /* dE, dC, dbias bf16 */
+#define CCE_OUT_FP32 1     /* dE, dC, dbias fp32 */
+#define CCE_OUT_DE_FP32 2  /* dE fp32 (a shard's part, to be summed over shards), dC and dbias bf16 */
 
 /* Width of the vocabulary sub-tile whose per-row maximum logit the forward saves. */
 #define CCE_VOCAB_SUBTILE 128
@@ -111,7 +127,7 @@ CCE_API size_t cce_backward_workspace_size(const cce_problem* p, int32_t out_fp3
  *  count    device int64 [1]: number of non-ignored tokens
  *  workspace/workspace_bytes: device scratch of at least cce_forward_workspace_size(p) bytes;
  *           it also holds the device error word read by cce_check_device_error().
- * N = 0 is allowed (loss 0, count 0).
+ * N = 0 is allowed (loss 0, count 0). After a device error the loss is NaN (every entry for none).
  */
 CCE_API cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const void* bias,
                                const int64_t* targets, float* loss, float* lse, float* tile_max, int64_t* count,
@@ -133,9 +149,12 @@ CCE_API cce_status cce_forward(const cce_problem* p, const void* E, const void* 
  *  E, C, bias, targets, lse, tile_max, count: as given to / produced by cce_forward() on the
  *           same problem (bias NULL for none)
  *  grad_out device fp32: [1] for mean/sum, [N] for none
- *  dE       device [N, D], dC device [V, D], dbias device [V] or NULL (not computed): bf16 when
- *           out_fp32 = 0, fp32 when out_fp32 = 1. Fully overwritten. Rows of ignored tokens in dE
- *           are exactly +0. dbias is the gradient of the bias (also when bias is NULL, i.e. zero).
+ *  dE       device [N, D], dC device [V, D], dbias device [V] or NULL (not computed): all bf16 when
+ *           out_fp32 = CCE_OUT_BF16, all fp32 when CCE_OUT_FP32, dE fp32 and the others bf16 when
+ *           CCE_OUT_DE_FP32. Fully overwritten. Rows of ignored tokens in dE are exactly +0. dbias is
+ *           the gradient of the bias (also when bias is NULL, i.e. zero).
+ *  For a vocabulary shard (p->vocab_total > 0): lse and count are the merged values of
+ *  cce_forward_merge, tile_max is this shard's from cce_forward_partial; dE is this shard's part.
  *  filtered_tiles device int64 [1]: number of skipped tiles
  *  workspace: device scratch of at least cce_backward_workspace_size(p, out_fp32) bytes.
  */
@@ -144,6 +163,47 @@ CCE_API cce_status cce_backward(const cce_problem* p, const void* E, const void*
                                 const int64_t* count, const float* grad_out, float filter_eps, void* dE, void* dC,
                                 void* dbias, int32_t out_fp32, int64_t* filtered_tiles, void* workspace,
                                 size_t workspace_bytes, cce_stream_t stream);
+
+/* The skip decision of every backward tile taken by the last cce_backward() that ran on `workspace`
+ * for the same problem: skipped[b * nt + t] = 1 when tile (row block b, vocabulary tile t) was
+ * skipped and 0 when it was kept, with nb = ceil(N / tile_rows) row blocks, nt = ceil(V / tile_cols)
+ * vocabulary tiles (cce_backward_tile_shape) and b < nb, t < nt. A diagnostic of the skip rule of
+ * mlx-cross-entropy README, "How it works" item 2: the count of ones equals filtered_tiles.
+ *  workspace: the backward workspace of that call (workspace_bytes as given to it); it is read,
+ *             not changed, so call this after the backward on the same stream.
+ *  skipped:   device uint8 [nb * nt].
+ * Enqueued on `stream`; argument errors return synchronously. N = 0 writes nothing. */
+CCE_API cce_status cce_backward_skip_map(const cce_problem* p, const void* workspace, size_t workspace_bytes,
+                                         uint8_t* skipped, cce_stream_t stream);
+
+/*
+ * Forward of one vocabulary shard (p->vocab_total > 0; also valid for an unsharded problem). Per row
+ * it returns the partial results that cce_forward_merge combines over all shards:
+ *  partial  device fp32 [3, N]: row 0 the log-sum-exp of the row's logits over this shard's
+ *           columns, row 1 the correct-token logit when the target lies in this shard (else 0),
+ *           row 2 the sum of the row's logits over this shard (label smoothing only; else 0).
+ *  tile_max device fp32 [cce_tile_max_len(p)]: this shard's saved maxima, for cce_backward.
+ *  E, C (this shard's rows), bias (this shard's entries, or NULL), targets (global ids) and the
+ *  workspace (cce_forward_workspace_size(p) bytes; it holds the device error word: a target outside
+ *  [0, vocab_total) that is not ignore_index) as for cce_forward.
+ * The log-sum-exp over the whole vocabulary is the log-sum-exp of the shards' row-0 values (Loss
+ * functions explainer, "How it works" item 1: stable log-sum-exp; mlx-cross-entropy README, "How it
+ * works" item 1: partial maxima and sums combine).
+ */
+CCE_API cce_status cce_forward_partial(const cce_problem* p, const void* E, const void* C, const void* bias,
+                                       const int64_t* targets, float* partial, float* tile_max, void* workspace,
+                                       size_t workspace_bytes, cce_stream_t stream);
+
+/*
+ * Combines the partial results of `shards` vocabulary shards (each [3, N] from cce_forward_partial,
+ * stacked as device fp32 [shards, 3, N] in any shard order) into the loss, the LSE over the whole
+ * vocabulary and the count, as cce_forward returns them. p describes the whole problem: V is the
+ * full vocabulary size (vocab_total of the shards), vocab_start = 0 and vocab_total = 0 or V.
+ * Needs no workspace; the reduction over rows runs in a fixed order (deterministic).
+ */
+CCE_API cce_status cce_forward_merge(const cce_problem* p, const float* partials, int32_t shards,
+                                     const int64_t* targets, float* loss, float* lse, int64_t* count,
+                                     cce_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device error word kept at the start of
  * `workspace` (a forward or backward workspace passed to an earlier call on that stream).
@@ -161,19 +221,24 @@ CCE_API const char* cce_last_error_message(void);
 
 /*
  * Forward that allocates nothing and takes no workspace, for callers that cannot allocate device
- * memory where they compute the loss (for example code running during CUDA graph capture, or an
- * embedding that only hands the library fixed buffers for inputs and outputs). The pages have no
+ * memory where they compute the loss: an embedding host that hands the library only fixed,
+ * pre-registered buffers for inputs and outputs and owns all other device memory, or a runtime
+ * whose allocator must not be re-entered from inside a loss callback. The pages have no
  * counterpart; it is an addition for such callers. Arguments and results are those of
  * cce_forward() without the workspace.
  *  - Scratch lives in one device array of CCE_NOALLOC_SCRATCH_BYTES that every GPU loading the
  *    library holds until exit. Problems needing more (about ceil(V/128) * N * 4 + 12 N + 4 D bytes; at
  *    V = 128256 up to N of about 8000) are rejected with CCE_ERR_UNSUPPORTED before anything runs.
- *  - The first call on each device looks up the array's device address; make that first call
- *    before any stream capture.
- *  - Every call shares the array, so calls whose work overlaps on the GPU (other streams, other
+ *  - The first call on each device looks up the array's device address (with that device
+ *    current); make that first call before any stream capture.
+ *  - Every call shares the array and the array keeps the last call's contents (the call clears
+ *    what must start at zero), so calls whose work overlaps on the GPU (other streams, other
  *    threads) race and give undefined results; serialise them.
- *  - Device-side errors (a target outside [0, V)) are not reported by this variant; use
- *    cce_forward() and cce_check_device_error() to diagnose them.
+ *  - Device-side errors (a target outside [0, V) that is not ignore_index; a bounded wait inside a
+ *    kernel that ran out, after CCE_WAIT_TIMEOUT_MS milliseconds as for cce_forward) cannot be
+ *    returned, since the call does not wait for the GPU: the loss (every entry for reduction none)
+ *    is then written as NaN, and lse / tile_max are undefined. cce_forward() with
+ *    cce_check_device_error() names the error.
  */
 CCE_API cce_status cce_forward_noalloc(const cce_problem* p, const void* E, const void* C, const void* bias,
                                        const int64_t* targets, float* loss, float* lse, float* tile_max,

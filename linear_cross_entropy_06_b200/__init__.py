@@ -11,6 +11,7 @@ from .ops import (  # noqa: F401
     cce_backward,
     linear_cross_entropy,
     load_library,
+    perplexity,
 )
 
-__all__ = ["CCEError", "cce_forward", "cce_backward", "linear_cross_entropy", "load_library"]
+__all__ = ["CCEError", "cce_forward", "cce_backward", "linear_cross_entropy", "load_library", "perplexity"]

@@ -17,7 +17,7 @@
 
 namespace {
 
-constexpr int32_t kVersion = 300;  // 0.3.0: loss variants (label smoothing, z-loss)
+constexpr int32_t kVersion = 400;  // 0.4.0: vocabulary shards, skip map, output dtype modes
 constexpr size_t kHeaderBytes = 256;
 constexpr size_t kAlign = 256;
 
@@ -49,6 +49,15 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Size of the whole vocabulary: the classifier's rows, or vocab_total for a shard of it.
+int64_t vocab_total(const cce_problem* p) { return p->vocab_total > 0 ? p->vocab_total : p->V; }
+
+bool sharded(const cce_problem* p) { return p->vocab_total > 0 && p->vocab_total != p->V; }
+
+// Output dtypes of cce_backward's out_fp32 argument (CCE_OUT_*).
+bool de_fp32(int32_t out) { return out == CCE_OUT_FP32 || out == CCE_OUT_DE_FP32; }
+bool dc_fp32(int32_t out) { return out == CCE_OUT_FP32; }
+
 bool problem_ok(const cce_problem* p, bool set_error) {
   auto bad = [&](const char* msg) {
     if (set_error) fail(CCE_ERR_INVALID_ARG, "%s", msg);
@@ -62,6 +71,11 @@ bool problem_ok(const cce_problem* p, bool set_error) {
   if (p->reserved != 0) return bad("reserved must be 0");
   if (!(p->label_smoothing >= 0.f && p->label_smoothing <= 1.f)) return bad("label_smoothing must be in [0, 1]");
   if (!(p->z_loss >= 0.f && p->z_loss < INFINITY)) return bad("z_loss must be finite and >= 0");
+  if (p->vocab_total < 0) return bad("vocab_total must be >= 0");
+  if (p->vocab_total == 0 && p->vocab_start != 0) return bad("vocab_start must be 0 when vocab_total is 0");
+  if (p->vocab_total > 0 && (p->vocab_start < 0 || p->vocab_start > p->vocab_total - p->V))
+    return bad("a vocabulary shard needs 0 <= vocab_start and vocab_start + V <= vocab_total");
+  if (p->vocab_total >= (int64_t(1) << 31) - 256) return bad("vocab_total too large");
   // Kernel indices are 32-bit for rows and tiles; keep every count well inside that.
   if (p->N >= (int64_t(1) << 31) - 256 || p->V >= (int64_t(1) << 31) - 256 || p->D >= (int64_t(1) << 24))
     return bad("N, V or D too large");
@@ -112,7 +126,7 @@ struct SplitWs {
   uint8_t* gscratch; // kGradBuffers * buf_bytes
   size_t buf_bytes;
   float* dE_acc;
-  float* dbias_acc;  // [V] fp32 (absent with out_fp32)
+  float* dbias_acc;  // [V] fp32 (absent when dbias is written in fp32)
   float* csum;       // [D + 1]: column sums of C (label smoothing only)
   float* wsum;       // [D + 1]: sum_r scale_r E_r and sum_r scale_r (label smoothing only)
   size_t bytes;
@@ -142,7 +156,8 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.offsets_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nb + 1)));
   w.plan.entries_b = reinterpret_cast<int2*>(take(sizeof(int2) * static_cast<size_t>(tiles)));
   w.plan.pos_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(tiles)));
-  w.plan.kept_total = reinterpret_cast<int*>(take(sizeof(int)));
+  w.plan.kept_total = reinterpret_cast<int*>(take(2 * sizeof(int)));
+  w.plan.n_empty = w.plan.kept_total + 1;
   // A chunk spans at most kChunkCBytes of C (its C rows stay in L2 while they are re-read for
   // every listed row block), and the gradient tiles of kGradBuffers chunks, at most nb per
   // vocabulary tile, fit in the scratch budget; at least one vocabulary tile per chunk.
@@ -163,6 +178,11 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.S = static_cast<int>(ceil_div(p->D, cce::kGemmSlice));
   w.plan.grp_size = reinterpret_cast<int*>(take(sizeof(int) * 2 * static_cast<size_t>(w.plan.nchunks)));
   w.plan.grp_start = reinterpret_cast<int*>(take(sizeof(int) * (2 * static_cast<size_t>(w.plan.nchunks) + 1)));
+  w.plan.vt_order = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt)));
+  w.plan.ndc = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks)));
+  w.plan.de_list = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks) * nb));
+  w.plan.nde = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks)));
+  w.plan.empty_list = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt)));
   w.plan.oh_cnt = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt)));
   w.plan.oh_off = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt + 1)));
   w.plan.oh_rows = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(std::max<int64_t>(p->N, 1))));
@@ -170,10 +190,8 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.sync = reinterpret_cast<int*>(take(w.sync_bytes));
   w.buf_bytes = static_cast<size_t>(nb * chunk_vt) * cce::kGradTileBytes;
   w.gscratch = reinterpret_cast<uint8_t*>(take(cce::kGradBuffers * w.buf_bytes));
-  if (!out_fp32) {
-    w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
-    w.dbias_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->V)));
-  }
+  if (!de_fp32(out_fp32)) w.dE_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->N * p->D)));
+  if (!dc_fp32(out_fp32)) w.dbias_acc = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->V)));
   w.csum = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->D + 1)));
   w.wsum = reinterpret_cast<float*>(take(sizeof(float) * static_cast<size_t>(p->D + 1)));
   w.bytes = off;
@@ -229,13 +247,6 @@ cce_status make_map(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem, co
   return CCE_OK;
 }
 
-uint64_t wait_timeout_ns() {
-  const char* s = std::getenv("CCE_WAIT_TIMEOUT_MS");
-  double ms = s ? std::atof(s) : 4000.0;
-  if (!(ms > 0)) ms = 4000.0;
-  return static_cast<uint64_t>(ms * 1e6);
-}
-
 #define CCE_TRY(expr)                                \
   do {                                               \
     cudaError_t e_ = (expr);                         \
@@ -261,26 +272,28 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   CCE_CHECK(check_device(&num_sms));
   CCE_CHECK(get_encoder());
   const int64_t N = p->N, D = p->D, V = p->V, T = ceil_div(V, cce::kSubTile);
-  float* dE_acc = out_fp32 ? static_cast<float*>(dE) : w.dE_acc;
-  float* dbias_acc = dbias == nullptr ? nullptr : (out_fp32 ? static_cast<float*>(dbias) : w.dbias_acc);
+  const bool e32 = de_fp32(out_fp32), c32 = dc_fp32(out_fp32);
+  const int64_t vs = p->vocab_start, vtot = vocab_total(p);
+  float* dE_acc = e32 ? static_cast<float*>(dE) : w.dE_acc;
+  float* dbias_acc = dbias == nullptr ? nullptr : (c32 ? static_cast<float*>(dbias) : w.dbias_acc);
 
   CCE_TRY(cudaMemsetAsync(w.hdr, 0, sizeof(WsHeader), s));
   if (N == 0) {  // no rows: dC = 0 (and dbias = 0)
-    CCE_TRY(cce::launch_fill_zero(dC, V * D * (out_fp32 ? 4 : 2), s));
-    if (dbias != nullptr) CCE_TRY(cce::launch_fill_zero(dbias, V * (out_fp32 ? 4 : 2), s));
+    CCE_TRY(cce::launch_fill_zero(dC, V * D * (c32 ? 4 : 2), s));
+    if (dbias != nullptr) CCE_TRY(cce::launch_fill_zero(dbias, V * (c32 ? 4 : 2), s));
     return cudaMemsetAsync(filtered_tiles, 0, sizeof(int64_t), s) == cudaSuccess ? CCE_OK
                                                                                   : fail(CCE_ERR_CUDA, "memset");
   }
   CCE_TRY(cce::launch_row_scale(targets, count, grad_out, N, p->ignore_index, p->reduction, w.scale, s));
-  CCE_TRY(cce::launch_bwd_plan(w.plan, tile_max, lse, targets, N, V, T, p->ignore_index, filter_eps, filtered_tiles,
-                               s));
+  CCE_TRY(cce::launch_bwd_plan(w.plan, tile_max, lse, targets, N, V, vs, vtot, T, p->ignore_index, filter_eps,
+                               filtered_tiles, s));
   CCE_TRY(cce::launch_fill_zero(dE_acc, N * D * 4, s));
   if (dbias_acc != nullptr) CCE_TRY(cce::launch_fill_zero(dbias_acc, V * 4, s));
   CCE_TRY(cudaMemsetAsync(w.sync, 0, w.sync_bytes, s));
   // Label smoothing: the ls / V part of every row's target is a rank-one term, added exactly:
   // dE_r -= scale_r (ls / V) sum_v C_v, dC_v -= (ls / V) sum_r scale_r E_r, dbias_v -= (ls / V) sum_r scale_r.
   const bool smooth = p->label_smoothing > 0.f;
-  const float ls_v = p->label_smoothing / static_cast<float>(V);
+  const float ls_v = p->label_smoothing / static_cast<float>(vtot);
   const auto* Eb = static_cast<const __nv_bfloat16*>(E);
   if (smooth) {
     CCE_TRY(cce::launch_weighted_colsum(static_cast<const __nv_bfloat16*>(C), V, D, nullptr, nullptr, w.csum, s));
@@ -293,7 +306,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   CCE_CHECK(make_map(&L.tmE64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, 64));
   CCE_CHECK(make_map(&L.tmC64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, 64));
   CCE_CHECK(make_map(&L.tmdE, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dE_acc, N, D, 32, 32));
-  if (out_fp32) CCE_CHECK(make_map(&L.tmdC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dC, V, D, 32, 32));
+  if (c32) CCE_CHECK(make_map(&L.tmdC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dC, V, D, 32, 32));
   else CCE_CHECK(make_map(&L.tmdC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dC, V, D, 64, 32));
   cce::BwdArgs& A = L.args;
   A.N = static_cast<int>(N);
@@ -303,8 +316,9 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.nt = w.plan.nt;
   A.S = w.plan.S;
   A.nchunks = w.plan.nchunks;
-  A.out_bf16 = out_fp32 ? 0 : 1;
+  A.out_bf16 = c32 ? 0 : 1;
   A.ignore_index = p->ignore_index;
+  A.vocab_start = vs;
   A.buf_bytes = w.buf_bytes;
   A.lse = lse;
   A.scale = w.scale;
@@ -319,6 +333,10 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.oh_off = w.plan.oh_off;
   A.oh_rows = w.plan.oh_rows;
   A.grp_start = w.plan.grp_start;
+  A.vt_order = w.plan.vt_order;
+  A.ndc = w.plan.ndc;
+  A.de_list = w.plan.de_list;
+  A.nde = w.plan.nde;
   A.chunk_t = w.plan.chunk_t;
   A.pstart_t = w.plan.pstart_t;
   A.pair_desc = w.plan.pair_desc;
@@ -334,7 +352,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.ctr_g_t = w.plan.nchunks * w.plan.nb;
   A.ctr_b_done = A.ctr_g_t + w.plan.nt;
   A.err = &w.hdr->err;
-  A.timeout_ns = wait_timeout_ns();
+  A.timeout_ns = cce::wait_timeout_ns();
   // Failure-detection test hook: CCE_TEST_INJECT_STALL=2 makes the backward's dE items of the first
   // chunk wait for a gradient tile that is never stored (reported as CCE_ERR_DEVICE_TIMEOUT).
   const char* stall = std::getenv("CCE_TEST_INJECT_STALL");
@@ -344,14 +362,18 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
   CCE_TRY(cce::launch_bwd(L, s));
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
-  CCE_TRY(cce::launch_onehot_rows(w.plan.oh_off, w.plan.nt, w.plan.oh_rows, targets, w.scale, 1.f - p->label_smoothing,
+  // dC rows of vocabulary tiles no row block lists: written without the tensor cores
+  CCE_TRY(cce::launch_dc_fill_empty(w.plan, targets, vs, w.scale, 1.f - p->label_smoothing, Eb, D, V,
+                                    smooth ? w.wsum : nullptr, -ls_v, dC, c32 ? 0 : 1, num_sms, s));
+  CCE_TRY(cce::launch_onehot_rows(w.plan.oh_off, w.plan.nt, w.plan.oh_rows, targets, vs, w.scale,
+                                  1.f - p->label_smoothing,
                                   static_cast<const __nv_bfloat16*>(C), D, dE_acc, dbias_acc, N, s));
   if (smooth) {
     CCE_TRY(cce::launch_add_rank1(dE_acc, N, D, w.scale, -ls_v, w.csum, s));
     if (dbias_acc != nullptr) CCE_TRY(cce::launch_add_scalar(dbias_acc, V, -ls_v, w.wsum + D, s));
   }
-  if (!out_fp32) CCE_TRY(cce::launch_to_bf16(dE_acc, static_cast<__nv_bfloat16*>(dE), N * D, s));
-  if (!out_fp32 && dbias != nullptr)
+  if (!e32) CCE_TRY(cce::launch_to_bf16(dE_acc, static_cast<__nv_bfloat16*>(dE), N * D, s));
+  if (!c32 && dbias != nullptr)
     CCE_TRY(cce::launch_to_bf16(dbias_acc, static_cast<__nv_bfloat16*>(dbias), V, s));
   return CCE_OK;
 }
@@ -360,6 +382,12 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
 
 namespace cce {
 void note_launches(int n) { g_launches += n; }
+uint64_t wait_timeout_ns() {
+  const char* s = std::getenv("CCE_WAIT_TIMEOUT_MS");
+  double ms = s ? std::atof(s) : 4000.0;
+  if (!(ms > 0)) ms = 4000.0;
+  return static_cast<uint64_t>(ms * 1e6);
+}
 void set_last_error(const char* msg) { g_last_error = msg; }
 }  // namespace cce
 
@@ -408,8 +436,8 @@ size_t cce_forward_workspace_size(const cce_problem* p) {
 }
 
 size_t cce_backward_workspace_size(const cce_problem* p, int32_t out_fp32) {
-  if (!problem_ok(p, false)) return 0;
-  return carve_split(p, out_fp32 ? 1 : 0, nullptr).bytes;
+  if (!problem_ok(p, false) || out_fp32 < CCE_OUT_BF16 || out_fp32 > CCE_OUT_DE_FP32) return 0;
+  return carve_split(p, out_fp32, nullptr).bytes;
 }
 
 cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const void* bias, const int64_t* targets,
@@ -417,6 +445,9 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
                        size_t workspace_bytes, cce_stream_t stream) {
   g_last_error.clear();
   if (!problem_ok(p, true)) return CCE_ERR_INVALID_ARG;
+  if (sharded(p))
+    return fail(CCE_ERR_INVALID_ARG, "a vocabulary shard's loss needs every shard: use cce_forward_partial and "
+                                     "cce_forward_merge");
   const bool has_rows = p->N > 0;
   if (C == nullptr || loss == nullptr || count == nullptr || workspace == nullptr ||
       (has_rows && (E == nullptr || targets == nullptr || lse == nullptr || tile_max == nullptr)))
@@ -448,7 +479,7 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
     L.tile_max = tile_max;
     L.tile_sum = w.tile_sum;
     L.err = &w.hdr->err;
-    L.timeout_ns = wait_timeout_ns();
+    L.timeout_ns = cce::wait_timeout_ns();
     L.num_sms = num_sms;
     // Failure-detection test hook: CCE_TEST_INJECT_STALL=1 makes the forward's bounded wait run out
     // (reported as CCE_ERR_DEVICE_TIMEOUT by cce_check_device_error; the outputs are undefined).
@@ -456,7 +487,7 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
     L.inject_stall = (stall != nullptr && stall[0] == '1') ? 1 : 0;
     const bool smooth = p->label_smoothing > 0.f;
     if (smooth) CCE_TRY(cce::launch_weighted_colsum(Cb, V, D, nullptr, Bb, w.csum, s));
-    CCE_TRY(cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, p->ignore_index, w.z_target,
+    CCE_TRY(cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, 0, V, p->ignore_index, w.z_target,
                                      smooth ? w.csum : nullptr, smooth ? w.z_sum : nullptr, &w.hdr->err, s));
     if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[0], s));
     CCE_TRY(cce::launch_fwd_lse(L, s));
@@ -465,7 +496,8 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
     CCE_TRY(cce::launch_lse_loss(tile_max, w.tile_sum, w.z_target, smooth ? w.z_sum : nullptr, targets, N, T,
                                  p->ignore_index, V, p->label_smoothing, p->z_loss, lse, rows_out, s));
   }
-  CCE_TRY(cce::launch_loss_reduce(w.loss_rows, targets, N, p->ignore_index, p->reduction, loss, count, s));
+  CCE_TRY(cce::launch_loss_reduce(w.loss_rows, targets, N, p->ignore_index, p->reduction, loss, count,
+                                   &w.hdr->err, s));
   return CCE_OK;
 }
 
@@ -484,9 +516,94 @@ cce_status cce_backward(const cce_problem* p, const void* E, const void* C, cons
       !aligned16(dbias) || !aligned16(workspace))
     return fail(CCE_ERR_INVALID_ARG, "E, C, bias, dE, dC, dbias and workspace must be 16-byte aligned");
   if (std::isnan(filter_eps)) return fail(CCE_ERR_INVALID_ARG, "filter_eps is NaN");
-  out_fp32 = out_fp32 ? 1 : 0;
+  if (out_fp32 < CCE_OUT_BF16 || out_fp32 > CCE_OUT_DE_FP32)
+    return fail(CCE_ERR_INVALID_ARG, "out_fp32 must be CCE_OUT_BF16, CCE_OUT_FP32 or CCE_OUT_DE_FP32");
   return backward_split(p, E, C, bias, targets, lse, tile_max, count, grad_out, filter_eps, dE, dC, dbias, out_fp32,
                         filtered_tiles, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+cce_status cce_forward_partial(const cce_problem* p, const void* E, const void* C, const void* bias,
+                               const int64_t* targets, float* partial, float* tile_max, void* workspace,
+                               size_t workspace_bytes, cce_stream_t stream) {
+  g_last_error.clear();
+  if (!problem_ok(p, true)) return CCE_ERR_INVALID_ARG;
+  const int64_t N = p->N, D = p->D, V = p->V, T = ceil_div(V, cce::kSubTile);
+  if (C == nullptr || workspace == nullptr ||
+      (N > 0 && (E == nullptr || targets == nullptr || partial == nullptr || tile_max == nullptr)))
+    return fail(CCE_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(E) || !aligned16(C) || !aligned16(bias) || !aligned16(workspace))
+    return fail(CCE_ERR_INVALID_ARG, "E, C, bias and workspace must be 16-byte aligned");
+  const FwdWs w = carve_fwd(p, workspace);
+  if (workspace_bytes < w.bytes)
+    return fail(CCE_ERR_WORKSPACE, "forward workspace is %zu bytes, needs %zu", workspace_bytes, w.bytes);
+  int num_sms = 0;
+  CCE_CHECK(check_device(&num_sms));
+  CCE_CHECK(get_encoder());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CCE_TRY(cudaMemsetAsync(w.hdr, 0, sizeof(WsHeader), s));
+  if (N == 0) return CCE_OK;
+  const auto* Eb = static_cast<const __nv_bfloat16*>(E);
+  const auto* Cb = static_cast<const __nv_bfloat16*>(C);
+  const auto* Bb = static_cast<const __nv_bfloat16*>(bias);
+  float* lse_part = partial;
+  float* zt_part = partial + N;
+  float* zs_part = partial + 2 * N;
+  const bool smooth = p->label_smoothing > 0.f;
+  cce::FwdLaunch L{};
+  L.bias = Bb;
+  CCE_CHECK(make_map(&L.tmE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kFwdBM));
+  CCE_CHECK(make_map(&L.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, cce::kFwdBN));
+  L.N = static_cast<int>(N);
+  L.D = static_cast<int>(D);
+  L.V = static_cast<int>(V);
+  L.T = static_cast<int>(T);
+  L.tile_max = tile_max;
+  L.tile_sum = w.tile_sum;
+  L.err = &w.hdr->err;
+  L.timeout_ns = cce::wait_timeout_ns();
+  L.num_sms = num_sms;
+  L.inject_stall = 0;
+  if (smooth) CCE_TRY(cce::launch_weighted_colsum(Cb, V, D, nullptr, Bb, w.csum, s));
+  else CCE_TRY(cudaMemsetAsync(zs_part, 0, sizeof(float) * static_cast<size_t>(N), s));
+  CCE_TRY(cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, p->vocab_start, vocab_total(p), p->ignore_index,
+                                   zt_part, smooth ? w.csum : nullptr, smooth ? zs_part : nullptr, &w.hdr->err, s));
+  if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[0], s));
+  CCE_TRY(cce::launch_fwd_lse(L, s));
+  if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[1], s));
+  CCE_TRY(cce::launch_lse_loss(tile_max, w.tile_sum, nullptr, nullptr, targets, N, T, p->ignore_index, V, 0.f, 0.f,
+                               lse_part, nullptr, s));
+  return CCE_OK;
+}
+
+cce_status cce_forward_merge(const cce_problem* p, const float* partials, int32_t shards, const int64_t* targets,
+                             float* loss, float* lse, int64_t* count, cce_stream_t stream) {
+  g_last_error.clear();
+  if (!problem_ok(p, true)) return CCE_ERR_INVALID_ARG;
+  if (sharded(p)) return fail(CCE_ERR_INVALID_ARG, "cce_forward_merge takes the whole problem, not a shard");
+  if (shards < 1) return fail(CCE_ERR_INVALID_ARG, "shards must be >= 1");
+  if (loss == nullptr || count == nullptr || (p->N > 0 && (partials == nullptr || targets == nullptr || lse == nullptr)))
+    return fail(CCE_ERR_INVALID_ARG, "a required pointer is NULL");
+  int num_sms = 0;
+  CCE_CHECK(check_device(&num_sms));
+  CCE_TRY(cce::launch_shard_merge(partials, shards, targets, p->N, p->V, p->ignore_index, p->label_smoothing,
+                                  p->z_loss, p->reduction, loss, lse, count, reinterpret_cast<cudaStream_t>(stream)));
+  return CCE_OK;
+}
+
+cce_status cce_backward_skip_map(const cce_problem* p, const void* workspace, size_t workspace_bytes,
+                                 uint8_t* skipped, cce_stream_t stream) {
+  g_last_error.clear();
+  if (!problem_ok(p, true)) return CCE_ERR_INVALID_ARG;
+  if (workspace == nullptr || (p->N > 0 && skipped == nullptr))
+    return fail(CCE_ERR_INVALID_ARG, "a required pointer is NULL");
+  // The tile flags sit at the same place in both workspace layouts; the smaller one bounds them.
+  const SplitWs w = carve_split(p, 1, const_cast<void*>(workspace));
+  if (workspace_bytes < w.bytes)
+    return fail(CCE_ERR_WORKSPACE, "backward workspace is %zu bytes, needs %zu", workspace_bytes, w.bytes);
+  if (p->N == 0) return CCE_OK;
+  const int64_t tiles = static_cast<int64_t>(w.plan.nb) * w.plan.nt;
+  CCE_TRY(cce::launch_skip_map(w.plan.flags, tiles, skipped, reinterpret_cast<cudaStream_t>(stream)));
+  return CCE_OK;
 }
 
 cce_status cce_check_device_error(void* workspace, cce_stream_t stream) {

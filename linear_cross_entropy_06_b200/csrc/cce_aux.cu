@@ -51,9 +51,12 @@ __device__ __forceinline__ float dot8_f32(uint4 a, const float* __restrict__ b, 
 
 // One warp per row: z_target[r] = E_r . C_{t_r} (+ bias[t_r]); with csum (the column sums of C
 // and, at index D, the sum of the bias) also z_sum[r] = sum_v z[r, v] = E_r . csum + csum[D].
+// C holds vocabulary rows [vs, vs + V) of vtot (a shard, or the whole vocabulary with vs = 0 and
+// vtot = V): a target outside the shard but inside [0, vtot) gets z_target 0 here (another shard
+// holds its logit); a target outside [0, vtot) that is not ignore_index is a device error.
 __global__ void target_logit_kernel(const __nv_bfloat16* __restrict__ E, const __nv_bfloat16* __restrict__ C,
                                     const __nv_bfloat16* __restrict__ bias, const int64_t* __restrict__ targets,
-                                    int64_t N, int64_t D, int64_t V, int64_t ignore_index,
+                                    int64_t N, int64_t D, int64_t V, int64_t vs, int64_t vtot, int64_t ignore_index,
                                     float* __restrict__ z_target, const float* __restrict__ csum,
                                     float* __restrict__ z_sum, int* err) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -67,14 +70,15 @@ __global__ void target_logit_kernel(const __nv_bfloat16* __restrict__ E, const _
     zs = warp_sum(zs);
     if (lane == 0) z_sum[row] = zs + csum[D];
   }
-  if (!valid_target(t, V, ignore_index)) {
+  if (!valid_target(t - vs, V, ignore_index - vs)) {  // not ignored and inside this shard
     if (lane == 0) {
       z_target[row] = 0.f;
-      if (t != ignore_index) record_error(err, kErrTargetRange);
+      if (!valid_target(t, vtot, ignore_index) && t != ignore_index) record_error(err, kErrTargetRange);
     }
     return;
   }
-  const __nv_bfloat16* c = C + t * D;
+  const int64_t tl = t - vs;
+  const __nv_bfloat16* c = C + tl * D;
   float acc0 = 0.f, acc1 = 0.f;
   int64_t d = static_cast<int64_t>(lane) * 8;
   for (; d + 256 < D; d += 512) {
@@ -83,7 +87,7 @@ __global__ void target_logit_kernel(const __nv_bfloat16* __restrict__ E, const _
   }
   if (d < D) acc0 = dot8_bf16(ld_global_nc_v4(e + d), ld_global_nc_v4(c + d), acc0);
   const float s = warp_sum(acc0 + acc1);
-  if (lane == 0) z_target[row] = bias != nullptr ? s + __bfloat162float(bias[t]) : s;
+  if (lane == 0) z_target[row] = bias != nullptr ? s + __bfloat162float(bias[tl]) : s;
 }
 
 __device__ __forceinline__ void lse_merge(float& M, float& S, float m, float s) {
@@ -131,6 +135,7 @@ __global__ void __launch_bounds__(kLseWarps * 32)
     for (int k = 0; k < kLseWarps; ++k) lse_merge(Mt, St, sm_m[k][lane], sm_s[k][lane]);
     const float L = Mt + logf(St);
     lse[r] = L;
+    if (loss_rows == nullptr) return;  // a vocabulary shard: the loss needs every shard's LSE
     const int64_t t = targets[r];
     // LSE - (1 - ls) z_t - (ls / V) sum_v z_v + zl LSE^2 (ls and zl are 0 unless requested)
     float l = L - (1.f - label_smoothing) * z_target[r] + z_loss * L * L;
@@ -141,10 +146,13 @@ __global__ void __launch_bounds__(kLseWarps * 32)
 
 constexpr int kReduceThreads = 1024;
 
-// Single block: deterministic order (strided fp64 partial sums, then a fixed tree).
+// Single block: deterministic order (strided fp64 partial sums, then a fixed tree). When an earlier
+// kernel of the call recorded a device error (err != 0), the loss is written as NaN instead (every
+// entry for reduction none, whose per-row losses live in `loss`), so that a caller who never reads
+// the error word still sees that the result is not valid.
 __global__ void loss_reduce_kernel(const float* __restrict__ loss_rows, const int64_t* __restrict__ targets,
                                    int64_t N, int64_t ignore_index, int reduction, float* __restrict__ loss,
-                                   int64_t* __restrict__ count) {
+                                   int64_t* __restrict__ count, const int* err) {
   __shared__ double ssum[kReduceThreads];
   __shared__ long long scnt[kReduceThreads];
   double acc = 0.0;
@@ -152,6 +160,61 @@ __global__ void loss_reduce_kernel(const float* __restrict__ loss_rows, const in
   for (int64_t r = threadIdx.x; r < N; r += kReduceThreads) {
     if (targets[r] != ignore_index) ++cnt;
     if (reduction != 0) acc += static_cast<double>(loss_rows[r]);
+  }
+  ssum[threadIdx.x] = acc;
+  scnt[threadIdx.x] = cnt;
+  __syncthreads();
+  for (int o = kReduceThreads / 2; o > 0; o >>= 1) {
+    if (static_cast<int>(threadIdx.x) < o) {
+      ssum[threadIdx.x] += ssum[threadIdx.x + o];
+      scnt[threadIdx.x] += scnt[threadIdx.x + o];
+    }
+    __syncthreads();
+  }
+  const bool failed = *reinterpret_cast<const volatile int*>(err) != 0;
+  if (threadIdx.x == 0) {
+    const long long c = scnt[0];
+    *count = c;
+    if (reduction == 1) *loss = failed ? NAN : static_cast<float>(ssum[0] / static_cast<double>(c > 0 ? c : 1));
+    if (reduction == 2) *loss = failed ? NAN : static_cast<float>(ssum[0]);
+  }
+  if (failed && reduction == 0)
+    for (int64_t r = threadIdx.x; r < N; r += kReduceThreads) loss[r] = NAN;
+}
+
+// The vocabulary shards' partial results [shards, 3, N] (per row: the shard's log-sum-exp, the
+// correct-token logit if the target lies in the shard, the sum of the shard's logits) combined into
+// the row's LSE over the whole vocabulary, LSE = M + ln sum_s exp(lse_s - M) with M = max_s lse_s
+// (Loss functions explainer, "How it works" item 1), its loss
+// LSE - (1 - ls) z_t - (ls / V) sum_v z_v + zl LSE^2 (0 for ignored rows), and the count and
+// reduction of loss_reduce_kernel, in one block with the same fixed summation order.
+__global__ void shard_merge_kernel(const float* __restrict__ partials, int shards, const int64_t* __restrict__ targets,
+                                   int64_t N, int64_t V, int64_t ignore_index, float label_smoothing, float z_loss,
+                                   int reduction, float* __restrict__ loss, float* __restrict__ lse,
+                                   int64_t* __restrict__ count) {
+  __shared__ double ssum[kReduceThreads];
+  __shared__ long long scnt[kReduceThreads];
+  double acc = 0.0;
+  long long cnt = 0;
+  for (int64_t r = threadIdx.x; r < N; r += kReduceThreads) {
+    float M = -INFINITY;
+    for (int k = 0; k < shards; ++k) M = fmaxf(M, partials[(static_cast<int64_t>(k) * 3) * N + r]);
+    float S = 0.f, zt = 0.f, zs = 0.f;
+    for (int k = 0; k < shards; ++k) {
+      const float* q = partials + static_cast<int64_t>(k) * 3 * N;
+      if (q[r] != -INFINITY) S += exp2f((q[r] - M) * kLog2e);
+      zt += q[N + r];
+      zs += q[2 * N + r];
+    }
+    const float L = M + logf(S);
+    lse[r] = L;
+    const bool valid = valid_target(targets[r], V, ignore_index);
+    const float l = valid ? L - (1.f - label_smoothing) * zt - label_smoothing / static_cast<float>(V) * zs +
+                                z_loss * L * L
+                          : 0.f;
+    if (reduction == 0) loss[r] = l;
+    if (targets[r] != ignore_index) ++cnt;
+    acc += static_cast<double>(l);
   }
   ssum[threadIdx.x] = acc;
   scnt[threadIdx.x] = cnt;
@@ -260,14 +323,15 @@ __global__ void add_scalar_kernel(float* __restrict__ X, int64_t n, float coef, 
 // One warp per listed row r (rows[i], i < off[nt]): dE_acc[r, :] -= coef * scale[r] * C[t_r, :]
 // and dbias_acc[t_r] -= coef * scale[r]. Each row is listed once, so the dE rows need no atomics.
 __global__ void onehot_rows_apply_kernel(const int* __restrict__ off, int nt, const int* __restrict__ rows,
-                                         const int64_t* __restrict__ targets, const float* __restrict__ scale,
-                                         float coef, const __nv_bfloat16* __restrict__ C, int64_t D,
-                                         float* __restrict__ dE_acc, float* __restrict__ dbias_acc) {
+                                         const int64_t* __restrict__ targets, int64_t vs,
+                                         const float* __restrict__ scale, float coef,
+                                         const __nv_bfloat16* __restrict__ C, int64_t D, float* __restrict__ dE_acc,
+                                         float* __restrict__ dbias_acc) {
   const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (i >= off[nt]) return;
   const int64_t r = rows[i];
-  const int64_t t = targets[r];
+  const int64_t t = targets[r] - vs;  // listed rows have their target in this shard
   const float a = -coef * scale[r];
   if (dbias_acc != nullptr && lane == 0) atomicAdd(dbias_acc + t, a);
   const __nv_bfloat16* c = C + t * D;
@@ -313,11 +377,13 @@ int grid_for(int64_t items, int per_block, int cap) {
 }  // namespace
 
 cudaError_t launch_target_logit(const __nv_bfloat16* E, const __nv_bfloat16* C, const __nv_bfloat16* bias,
-                                const int64_t* targets, int64_t N, int64_t D, int64_t V, int64_t ignore_index,
-                                float* z_target, const float* csum, float* z_sum, int* err, cudaStream_t s) {
+                                const int64_t* targets, int64_t N, int64_t D, int64_t V, int64_t vs, int64_t vtot,
+                                int64_t ignore_index, float* z_target, const float* csum, float* z_sum, int* err,
+                                cudaStream_t s) {
   if (N == 0) return cudaSuccess;
   const int grid = static_cast<int>((N + 7) / 8);  // 8 warps (rows) per block
-  target_logit_kernel<<<grid, 256, 0, s>>>(E, C, bias, targets, N, D, V, ignore_index, z_target, csum, z_sum, err);
+  target_logit_kernel<<<grid, 256, 0, s>>>(E, C, bias, targets, N, D, V, vs, vtot, ignore_index, z_target, csum,
+                                           z_sum, err);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -334,8 +400,17 @@ cudaError_t launch_lse_loss(const float* tile_max, const float* tile_sum, const 
 }
 
 cudaError_t launch_loss_reduce(const float* loss_rows, const int64_t* targets, int64_t N, int64_t ignore_index,
-                               int reduction, float* loss, int64_t* count, cudaStream_t s) {
-  loss_reduce_kernel<<<1, kReduceThreads, 0, s>>>(loss_rows, targets, N, ignore_index, reduction, loss, count);
+                               int reduction, float* loss, int64_t* count, const int* err, cudaStream_t s) {
+  loss_reduce_kernel<<<1, kReduceThreads, 0, s>>>(loss_rows, targets, N, ignore_index, reduction, loss, count, err);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shard_merge(const float* partials, int shards, const int64_t* targets, int64_t N, int64_t V,
+                               int64_t ignore_index, float label_smoothing, float z_loss, int reduction, float* loss,
+                               float* lse, int64_t* count, cudaStream_t s) {
+  shard_merge_kernel<<<1, kReduceThreads, 0, s>>>(partials, shards, targets, N, V, ignore_index, label_smoothing,
+                                                  z_loss, reduction, loss, lse, count);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -390,12 +465,12 @@ cudaError_t launch_add_scalar(float* X, int64_t n, float coef, const float* c, c
   return cudaGetLastError();
 }
 
-cudaError_t launch_onehot_rows(const int* off, int nt, const int* rows, const int64_t* targets,
+cudaError_t launch_onehot_rows(const int* off, int nt, const int* rows, const int64_t* targets, int64_t vs,
                                const float* scale, float coef, const __nv_bfloat16* C, int64_t D, float* dE_acc,
                                float* dbias_acc, int64_t max_rows, cudaStream_t s) {
   if (max_rows == 0) return cudaSuccess;
   const int grid = static_cast<int>((max_rows + 7) / 8);  // 8 warps per block, one listed row each
-  onehot_rows_apply_kernel<<<grid, 256, 0, s>>>(off, nt, rows, targets, scale, coef, C, D, dE_acc, dbias_acc);
+  onehot_rows_apply_kernel<<<grid, 256, 0, s>>>(off, nt, rows, targets, vs, scale, coef, C, D, dE_acc, dbias_acc);
   note_launches(1);
   return cudaGetLastError();
 }

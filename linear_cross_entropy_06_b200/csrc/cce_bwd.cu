@@ -171,30 +171,33 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, const Bwd
     if (c >= kGradBuffers) {  // the buffer's previous chunk must have been read by its dE / dC items
       const int prev = c - kGradBuffers;
       it.dep_idx = A.ctr_b_done + prev;
-      it.dep_val = (A.nb + A.chunk_t[prev + 1] - A.chunk_t[prev]) * A.S;
+      it.dep_val = (A.nde[prev] + A.ndc[prev]) * A.S;
     } else {
       it.dep_idx = -1;
       it.dep_val = 0;
     }
   } else {
+    // Only row blocks and vocabulary tiles with a listed tile in the chunk have items; the dC rows of
+    // vocabulary tiles no row block lists are written by the streaming fill outside this kernel.
     const int S = A.S;
+    const int nde = A.nde[c];
     it.slot0 = A.offsets_t[t_begin];
     it.slot1 = 0;
-    if (local < A.nb * S) {  // slice-major: concurrent dE items read the same columns of C
+    if (local < nde * S) {  // slice-major: concurrent dE items read the same columns of C
       it.kind = kDE;
-      it.key = local % A.nb;
+      it.key = A.de_list[static_cast<int64_t>(c) * A.nb + local % nde];
       // serpentine over chunks: a chunk starts on the slices of dE the previous one touched last
-      it.s = (c & 1) ? S - 1 - local / A.nb : local / A.nb;
+      it.s = (c & 1) ? S - 1 - local / nde : local / nde;
       const int2 r = A.rb_range[static_cast<int64_t>(c) * A.nb + it.key];
       it.begin = r.x;
       it.end = r.y;
       it.dep_idx = A.ctr_g_b + c * A.nb + it.key;
     } else {  // slice-major too: concurrent dC items read the same columns of E
-      const int v = local - A.nb * S;
-      const int nvt = A.chunk_t[c + 1] - t_begin;
+      const int v = local - nde * S;
+      const int ndc = A.ndc[c];
       it.kind = kDC;
-      it.key = t_begin + v % nvt;
-      it.s = v / nvt;
+      it.key = A.vt_order[t_begin + v % ndc];
+      it.s = v / ndc;
       it.begin = A.offsets_t[it.key];
       it.end = A.offsets_t[it.key + 1];
       it.dep_idx = A.ctr_g_t + it.key;
@@ -476,8 +479,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float sc = (r < A.N) ? A.scale[r] : 0.f;
         const float sc_p = sc * fmaf(2.f * A.z_loss, lse_r, 1.f);  // softmax part: (1 + 2 zl LSE) p
         const float sc_y = sc * A.onehot_coef;                     // onehot part: (1 - ls) y
-        const int64_t tg = (r < A.N) ? A.targets[r] : A.ignore_index;
-        const bool tvalid = tg != A.ignore_index && tg >= 0 && tg < A.V;
+        // target in this problem's vocabulary coordinates (the shard's rows, for a vocabulary shard)
+        const int64_t tg = (r < A.N) ? A.targets[r] - A.vocab_start : A.ignore_index - A.vocab_start;
+        const bool tvalid = tg != A.ignore_index - A.vocab_start && tg >= 0 && tg < A.V;
         const bool mma = it.s != 0;
         if (mma) {
           if (!warp_wait(bar(kAccFull + a), (acc_iter >> 1) & 1u)) break;
@@ -583,7 +587,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int n = 0;
         for (int i = it.oh_begin; i < it.oh_end; ++i) {
           const int r = A.oh_rows[i];
-          if (A.targets[r] != my_v) continue;
+          if (A.targets[r] - A.vocab_start != my_v) continue;
           if (n < 2) {
             oh_r[n] = r;
             oh_c[n] = -A.scale[r] * A.onehot_coef;
@@ -650,7 +654,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int n = 0;
             for (int i = it.oh_begin; i < it.oh_end; ++i) {
               const int r = A.oh_rows[i];
-              if (A.targets[r] != my_v) continue;
+              if (A.targets[r] - A.vocab_start != my_v) continue;
               if (n++ >= 2) add_row(r, -A.scale[r] * A.onehot_coef);
             }
           }

@@ -37,24 +37,26 @@ __device__ __forceinline__ bool valid_target(int64_t t, int64_t V, int64_t ignor
 constexpr int kFlagTiles = 8;
 
 __global__ void tile_flags_kernel(const float* __restrict__ tile_max, const float* __restrict__ lse,
-                                  const int64_t* __restrict__ targets, int64_t N, int64_t V, int64_t T,
-                                  int64_t ignore_index, float ln_eps, int filter_on, int nt, int runs,
-                                  uint8_t* __restrict__ flags) {
+                                  const int64_t* __restrict__ targets, int64_t N, int64_t V, int64_t vs,
+                                  int64_t vtot, int64_t T, int64_t ignore_index, float ln_eps, int filter_on, int nt,
+                                  int runs, uint8_t* __restrict__ flags) {
   __shared__ float wmax[kFlagTiles][4];
   __shared__ int any_target[kFlagTiles];
   const int b = static_cast<int>(blockIdx.x / runs), t0 = static_cast<int>(blockIdx.x % runs) * kFlagTiles;
   const int64_t r = static_cast<int64_t>(b) * kBwdBM + threadIdx.x;
   if (threadIdx.x < kFlagTiles) any_target[threadIdx.x] = 0;
   __syncthreads();
-  bool valid = false;
+  bool valid = false, local = false;
   float l = 0.f;
   int64_t tr = -1;
   if (r < N) {
     tr = targets[r];
-    valid = valid_target(tr, V, ignore_index);
+    valid = valid_target(tr, vtot, ignore_index);      // the row is scored (by every shard)
+    local = valid && valid_target(tr - vs, V, ignore_index - vs);  // its target lies in this shard
     if (valid && filter_on) l = lse[r];
+    tr -= vs;
   }
-  if (valid && tr / kBwdBN >= t0 && tr / kBwdBN < t0 + kFlagTiles) any_target[tr / kBwdBN - t0] = 1;
+  if (local && tr / kBwdBN >= t0 && tr / kBwdBN < t0 + kFlagTiles) any_target[tr / kBwdBN - t0] = 1;
 #pragma unroll
   for (int k = 0; k < kFlagTiles; ++k) {
     const int t = t0 + k;
@@ -180,21 +182,16 @@ __device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int 
   return lo;
 }
 
-// Chunk boundaries: chunk c covers vocabulary tiles [c * chunk_vt, min(nt, (c + 1) * chunk_vt)).
-__global__ void chunk_plan_kernel(int nt, int chunk_vt, int nchunks, int* __restrict__ chunk_t) {
-  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c <= nchunks; c += gridDim.x * blockDim.x)
-    chunk_t[c] = min(nt, c * chunk_vt);
-}
-
 // For every chunk c and row block b, the range [lo, hi) of b's entries_b inside the chunk.
+// Chunk c covers vocabulary tiles [c * chunk_vt, min(nt, (c + 1) * chunk_vt)).
 __global__ void row_range_kernel(const int2* __restrict__ entries_b, const int* __restrict__ offsets_b, int nb,
-                                 int nchunks, const int* __restrict__ chunk_t, int2* __restrict__ rb_range) {
+                                 int nchunks, int nt, int chunk_vt, int2* __restrict__ rb_range) {
   const int64_t total = static_cast<int64_t>(nb) * nchunks;
   for (int64_t cb = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; cb < total;
        cb += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int c = static_cast<int>(cb / nb), b = static_cast<int>(cb % nb);
-    const int lo = lower_bound_t(entries_b, offsets_b[b], offsets_b[b + 1], chunk_t[c]);
-    const int hi = lower_bound_t(entries_b, lo, offsets_b[b + 1], chunk_t[c + 1]);
+    const int lo = lower_bound_t(entries_b, offsets_b[b], offsets_b[b + 1], min(nt, c * chunk_vt));
+    const int hi = lower_bound_t(entries_b, lo, offsets_b[b + 1], min(nt, (c + 1) * chunk_vt));
     rb_range[cb] = make_int2(lo, hi);
   }
 }
@@ -207,14 +204,14 @@ __global__ void row_range_kernel(const int2* __restrict__ entries_b, const int* 
 __global__ void pair_list_kernel(const int2* __restrict__ entries_t, const int* __restrict__ offsets_t,
                                  const int2* __restrict__ entries_b, const int* __restrict__ pos_b,
                                  const int2* __restrict__ rb_range, const uint8_t* __restrict__ flags, int nb, int nt,
-                                 int chunk_vt, const int* __restrict__ chunk_t, int* __restrict__ cnt,
+                                 int chunk_vt, int* __restrict__ cnt,
                                  const int* __restrict__ pstart_t, int4* __restrict__ pair_desc,
                                  int2* __restrict__ pair_slot, int pass) {
   const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= nt) return;
   const int c = t / chunk_vt;
-  const int slot_base = offsets_t[chunk_t[c]];
+  const int slot_base = offsets_t[c * chunk_vt];
   const int i0 = offsets_t[t], i1 = offsets_t[t + 1];
   int k = 0;
   for (int base = i0; base < i1; base += 32) {
@@ -244,42 +241,176 @@ __global__ void pair_list_kernel(const int2* __restrict__ entries_t, const int* 
   if (pass == 0 && lane == 0) cnt[t] = k;
 }
 
-// Sizes of the backward's queue groups, in queue order: pairs(0), then pairs(c) and dE/dC(c - 1)
-// for c = 1 .. n-1, then dE/dC(n - 1). A chunk's pairs are those starting in its vocabulary tiles;
-// its dE/dC group holds nb * S dE items and one dC item per vocabulary tile and slice.
-__global__ void group_size_kernel(const int* __restrict__ pstart_t, const int* __restrict__ chunk_t, int nb, int S,
-                                  int nchunks, int* __restrict__ grp_size) {
-  for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < 2 * nchunks; g += gridDim.x * blockDim.x) {
-    int c, pairs;
-    if (g == 0) {
-      c = 0;
-      pairs = 1;
-    } else if (g == 2 * nchunks - 1) {
-      c = nchunks - 1;
-      pairs = 0;
-    } else {
-      const int pos = g - 1;
-      c = pos / 2 + 1 - (pos & 1);
-      pairs = (pos & 1) == 0;
+// Block-wide ordered compaction helper: every thread holds one flag; returns the number of set flags
+// before this thread in the block (ascending thread order) and sets *total to the block's count.
+// blockDim.x is a multiple of 32, at most 1024; `warps` is shared scratch of 32 ints.
+__device__ __forceinline__ int block_rank(bool flag, int* warps, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const unsigned m = __ballot_sync(0xffffffffu, flag);
+  if (lane == 0) warps[w] = __popc(m);
+  __syncthreads();
+  int before = 0, all = 0;
+  for (int k = 0; k < nw; ++k) {
+    before += k < w ? warps[k] : 0;
+    all += warps[k];
+  }
+  __syncthreads();  // warps[] may be rewritten by the next call
+  *total = all;
+  return before + __popc(m & ((1u << lane) - 1u));
+}
+
+// One block per vocabulary chunk c: its work lists and the sizes of its two queue groups.
+//  - vt_order: the chunk's vocabulary tiles with a listed tile first (they get dC items), then the
+//    empty ones (no row block lists them: their dC rows hold only onehot and smoothing terms and are
+//    written by dc_fill_empty_kernel); both ascending.
+//  - de_list: the row blocks with a listed tile in the chunk (they get dE items), ascending.
+//  - empty_list: the chunk's empty tiles, appended to one list for the whole vocabulary.
+//  - grp_size: pairs(c) and dE/dC(c), at their places in the queue order pairs(0), then pairs(c) and
+//    dE/dC(c - 1) for c = 1 .. n-1, then dE/dC(n - 1): pairs(c) is group 2c - 1 (0 for c = 0) and
+//    dE/dC(c) group min(2c + 2, 2n - 1).
+__global__ void chunk_items_kernel(const int* __restrict__ offsets_t, const int2* __restrict__ rb_range,
+                                   const int* __restrict__ pstart_t, int nt, int chunk_vt, int nb, int S,
+                                   int nchunks, int* __restrict__ chunk_t, int* __restrict__ vt_order,
+                                   int* __restrict__ ndc, int* __restrict__ de_list, int* __restrict__ nde,
+                                   int* __restrict__ empty_list, int* __restrict__ n_empty,
+                                   int* __restrict__ grp_size) {
+  __shared__ int warps[32];
+  __shared__ int em_base;
+  const int c = blockIdx.x;
+  const int t0 = min(nt, c * chunk_vt), t1 = min(nt, (c + 1) * chunk_vt);
+  if (threadIdx.x == 0) {
+    chunk_t[c] = t0;
+    if (c == nchunks - 1) chunk_t[nchunks] = t1;
+  }
+  // vocabulary tiles: count the listed ones first, so that the empty ones can follow them
+  int n_listed = 0;
+  for (int base = t0; base < t1; base += blockDim.x) {
+    const int t = base + threadIdx.x;
+    const bool on = t < t1 && offsets_t[t + 1] > offsets_t[t];
+    int total;
+    const int pos = block_rank(on, warps, &total);
+    if (on) vt_order[t0 + n_listed + pos] = t;
+    n_listed += total;
+  }
+  const int n_em = (t1 - t0) - n_listed;
+  if (threadIdx.x == 0) em_base = n_em > 0 ? atomicAdd(n_empty, n_em) : 0;
+  __syncthreads();
+  int n_seen = 0;
+  for (int base = t0; base < t1; base += blockDim.x) {
+    const int t = base + threadIdx.x;
+    const bool em = t < t1 && offsets_t[t + 1] == offsets_t[t];
+    int total;
+    const int pos = block_rank(em, warps, &total);
+    if (em) {
+      vt_order[t0 + n_listed + n_seen + pos] = t;
+      empty_list[em_base + n_seen + pos] = t;
     }
-    grp_size[g] = pairs ? pstart_t[chunk_t[c + 1]] - pstart_t[chunk_t[c]] : (nb + chunk_t[c + 1] - chunk_t[c]) * S;
+    n_seen += total;
+  }
+  // row blocks with a listed tile in the chunk
+  int n_rb = 0;
+  for (int base = 0; base < nb; base += blockDim.x) {
+    const int b = base + threadIdx.x;
+    bool on = false;
+    if (b < nb) {
+      const int2 r = rb_range[static_cast<int64_t>(c) * nb + b];
+      on = r.x < r.y;
+    }
+    int total;
+    const int pos = block_rank(on, warps, &total);
+    if (on) de_list[static_cast<int64_t>(c) * nb + n_rb + pos] = b;
+    n_rb += total;
+  }
+  if (threadIdx.x == 0) {
+    ndc[c] = n_listed;
+    nde[c] = n_rb;
+    grp_size[c == 0 ? 0 : 2 * c - 1] = pstart_t[t1] - pstart_t[t0];
+    grp_size[min(2 * c + 2, 2 * nchunks - 1)] = (n_rb + n_listed) * S;
+  }
+}
+
+// dC rows of the vocabulary tiles that no row block lists. Every logit of such a tile is skipped,
+// so only the target part of the logit gradient reaches them (Loss functions explainer, "How it
+// works" items 2 and 3): -scale_r (1 - ls) E_r for each row r whose target v lies there, and the
+// smoothing term dc_coef * dc_add shared by every row of dC. No tensor core is involved: a work unit
+// is 4 vocabulary rows x 512 columns, one thread per 8 columns, 16-byte loads and stores along a
+// row. The target rows of tile t are oh_rows[oh_off[t] .. oh_off[t + 1]) (for an empty tile every
+// non-ignored row targeting it is listed there), scanned in order, so the result is deterministic.
+constexpr int kFillCols = 512;
+
+__global__ void __launch_bounds__(256, 4) dc_fill_empty_kernel(
+    const int* __restrict__ empty_list, const int* __restrict__ n_empty, const int* __restrict__ oh_off,
+    const int* __restrict__ oh_rows, const int64_t* __restrict__ targets, int64_t vs, const float* __restrict__ scale,
+    float onehot_coef, const __nv_bfloat16* __restrict__ E, int64_t D, int64_t V, const float* __restrict__ dc_add,
+    float dc_coef, void* __restrict__ dC, int out_bf16) {
+  const int col_chunks = static_cast<int>((D + kFillCols - 1) / kFillCols);
+  const int units_per_tile = (kBwdBN / 4) * col_chunks;
+  const int64_t units = static_cast<int64_t>(*n_empty) * units_per_tile;
+  const int row_in_unit = threadIdx.x >> 6;  // 4 rows of 64 threads
+  const int col_thread = (threadIdx.x & 63) * 8;
+  for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+    const int e = static_cast<int>(u / units_per_tile);
+    const int rem = static_cast<int>(u % units_per_tile);
+    const int t = empty_list[e];
+    const int row = (rem / col_chunks) * 4 + row_in_unit;
+    const int64_t v = static_cast<int64_t>(t) * kBwdBN + row;
+    const int64_t d = static_cast<int64_t>(rem % col_chunks) * kFillCols + col_thread;
+    if (v >= V || d >= D) continue;
+    float acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = dc_add != nullptr ? dc_coef * dc_add[d + k] : 0.f;
+    const int i1 = oh_off[t + 1];
+    for (int i = oh_off[t]; i < i1; ++i) {
+      const int r = oh_rows[i];
+      if (targets[r] - vs != v) continue;
+      const float a = -scale[r] * onehot_coef;
+      const uint4 q = ld_global_nc_v4(E + static_cast<int64_t>(r) * D + d);
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __nv_bfloat162 h;
+        *reinterpret_cast<uint32_t*>(&h) = w[k];
+        acc[2 * k] = fmaf(a, __low2float(h), acc[2 * k]);
+        acc[2 * k + 1] = fmaf(a, __high2float(h), acc[2 * k + 1]);
+      }
+    }
+    if (out_bf16) {
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dC) + v * D + d) = o;
+    } else {
+      float4* out = reinterpret_cast<float4*>(static_cast<float*>(dC) + v * D + d);
+      out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
   }
 }
 
 // Rows whose target tile is onehot only: counted (pass 0) or written (pass 1, positions from the
 // scanned counts and a per-tile cursor) per vocabulary tile of the target.
 __global__ void onehot_rows_kernel(const uint8_t* __restrict__ flags, const int64_t* __restrict__ targets,
-                                   int64_t N, int64_t V, int64_t ignore_index, int nt, int* __restrict__ cnt,
-                                   const int* __restrict__ off, int* __restrict__ rows, int pass) {
+                                   int64_t N, int64_t V, int64_t vs, int64_t ignore_index, int nt,
+                                   int* __restrict__ cnt, const int* __restrict__ off, int* __restrict__ rows,
+                                   int pass) {
   for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < N;
        r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t tr = targets[r];
-    if (!valid_target(tr, V, ignore_index)) continue;
+    const int64_t tr = targets[r] - vs;  // only targets inside this shard have an onehot term here
+    if (!valid_target(tr, V, ignore_index - vs)) continue;
     const int t = static_cast<int>(tr / kBwdBN);
     if (flags[(r / kBwdBM) * nt + t] != 2) continue;
     const int k = atomicAdd(cnt + t, 1);
     if (pass == 1) rows[off[t] + k] = static_cast<int>(r);
   }
+}
+
+// out[i] = 1 when backward tile i (row block i / nt, vocabulary tile i % nt) was skipped, 0 when kept.
+__global__ void skip_map_kernel(const uint8_t* __restrict__ flags, int64_t n, uint8_t* __restrict__ out) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = flags[i] == 1 ? 0 : 1;
 }
 
 __global__ void plan_finish_kernel(const int* __restrict__ kept_total, int64_t total, int64_t* __restrict__ filtered) {
@@ -288,19 +419,37 @@ __global__ void plan_finish_kernel(const int* __restrict__ kept_total, int64_t t
 
 }  // namespace
 
+cudaError_t launch_dc_fill_empty(const BwdPlan& P, const int64_t* targets, int64_t vs, const float* scale,
+                                 float onehot_coef, const __nv_bfloat16* E, int64_t D, int64_t V, const float* dc_add,
+                                 float dc_coef, void* dC, int out_bf16, int num_sms, cudaStream_t s) {
+  if (P.nb == 0) return cudaSuccess;
+  // persistent: the number of empty tiles is known on the device only
+  dc_fill_empty_kernel<<<num_sms * 8, 256, 0, s>>>(P.empty_list, P.n_empty, P.oh_off, P.oh_rows, targets, vs,
+                                                   scale, onehot_coef, E, D, V, dc_add, dc_coef, dC, out_bf16);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_skip_map(const uint8_t* flags, int64_t tiles, uint8_t* out, cudaStream_t s) {
+  if (tiles == 0) return cudaSuccess;
+  skip_map_kernel<<<static_cast<int>(std::min<int64_t>((tiles + 255) / 256, 4096)), 256, 0, s>>>(flags, tiles, out);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float* lse, const int64_t* targets,
-                            int64_t N, int64_t V, int64_t T, int64_t ignore_index, float filter_eps,
-                            int64_t* filtered_tiles, cudaStream_t s) {
+                            int64_t N, int64_t V, int64_t vs, int64_t vtot, int64_t T, int64_t ignore_index,
+                            float filter_eps, int64_t* filtered_tiles, cudaStream_t s) {
   const int nb = P.nb, nt = P.nt;
   const int filter_on = filter_eps > 0.f ? 1 : 0;
   const float ln_eps = filter_on ? logf(filter_eps) : -INFINITY;
-  cudaError_t e = cudaMemsetAsync(P.kept_total, 0, sizeof(int), s);
+  cudaError_t e = cudaMemsetAsync(P.kept_total, 0, 2 * sizeof(int), s);  // kept_total and n_empty
   if (e != cudaSuccess) return e;
   if (nb > 0) {
     const int64_t tiles = static_cast<int64_t>(nb) * nt;
     const int runs = (nt + kFlagTiles - 1) / kFlagTiles;
     tile_flags_kernel<<<static_cast<unsigned>(static_cast<int64_t>(nb) * runs), kBwdBM, 0, s>>>(
-        tile_max, lse, targets, N, V, T, ignore_index, ln_eps, filter_on, nt, runs, P.flags);
+        tile_max, lse, targets, N, V, vs, vtot, T, ignore_index, ln_eps, filter_on, nt, runs, P.flags);
     note_launches(1);
     e = cudaMemsetAsync(P.cnt_b, 0, sizeof(int) * static_cast<size_t>(nb), s);
     if (e != cudaSuccess) return e;
@@ -316,25 +465,27 @@ cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float
     note_launches(1);
     row_list_kernel<<<nb, 1024, 0, s>>>(P.flags, P.rank, P.offsets_t, nt, P.offsets_b, P.entries_b, P.pos_b);
     note_launches(1);
-    chunk_plan_kernel<<<(P.nchunks + 256) / 256, 256, 0, s>>>(nt, P.chunk_vt, P.nchunks, P.chunk_t);
-    note_launches(1);
     const int64_t cbs = static_cast<int64_t>(nb) * P.nchunks;
     row_range_kernel<<<static_cast<int>(std::min<int64_t>((cbs + 255) / 256, 4096)), 256, 0, s>>>(
-        P.entries_b, P.offsets_b, nb, P.nchunks, P.chunk_t, P.rb_range);
+        P.entries_b, P.offsets_b, nb, P.nchunks, nt, P.chunk_vt, P.rb_range);
     note_launches(1);
     // the pair counts per vocabulary tile reuse cnt_t (its counts are already scanned into offsets_t)
     const int grid_t = static_cast<int>((static_cast<int64_t>(nt) * 32 + 255) / 256);
     pair_list_kernel<<<grid_t, 256, 0, s>>>(P.entries_t, P.offsets_t, P.entries_b, P.pos_b, P.rb_range, P.flags, nb,
-                                            nt, P.chunk_vt, P.chunk_t, P.cnt_t, P.pstart_t, P.pair_desc, P.pair_slot,
+                                            nt, P.chunk_vt, P.cnt_t, P.pstart_t, P.pair_desc, P.pair_slot,
                                             0);
     note_launches(1);
     scan_kernel<<<1, 1024, 0, s>>>(P.cnt_t, nt, P.pstart_t);
     note_launches(1);
     pair_list_kernel<<<grid_t, 256, 0, s>>>(P.entries_t, P.offsets_t, P.entries_b, P.pos_b, P.rb_range, P.flags, nb,
-                                            nt, P.chunk_vt, P.chunk_t, P.cnt_t, P.pstart_t, P.pair_desc, P.pair_slot,
+                                            nt, P.chunk_vt, P.cnt_t, P.pstart_t, P.pair_desc, P.pair_slot,
                                             1);
     note_launches(1);
-    group_size_kernel<<<(P.nchunks + 255) / 256, 256, 0, s>>>(P.pstart_t, P.chunk_t, nb, P.S, P.nchunks, P.grp_size);
+    // (pair_list pass 0 left each vocabulary tile's pair count in cnt_t; chunk_items reads the
+    // listed-tile counts as differences of offsets_t)
+    chunk_items_kernel<<<P.nchunks, 256, 0, s>>>(P.offsets_t, P.rb_range, P.pstart_t, nt, P.chunk_vt, nb, P.S,
+                                                 P.nchunks, P.chunk_t, P.vt_order, P.ndc, P.de_list, P.nde,
+                                                 P.empty_list, P.n_empty, P.grp_size);
     note_launches(1);
     scan_kernel<<<1, 1024, 0, s>>>(P.grp_size, 2 * P.nchunks, P.grp_start);
     note_launches(1);
@@ -343,14 +494,14 @@ cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float
     e = cudaMemsetAsync(P.oh_cnt, 0, sizeof(int) * static_cast<size_t>(nt), s);
     if (e != cudaSuccess) return e;
     const int grid_r = static_cast<int>(std::min<int64_t>((N + 255) / 256, 4096));
-    onehot_rows_kernel<<<grid_r, 256, 0, s>>>(P.flags, targets, N, V, ignore_index, nt, P.oh_cnt, P.oh_off,
+    onehot_rows_kernel<<<grid_r, 256, 0, s>>>(P.flags, targets, N, V, vs, ignore_index, nt, P.oh_cnt, P.oh_off,
                                               P.oh_rows, 0);
     note_launches(1);
     scan_kernel<<<1, 1024, 0, s>>>(P.oh_cnt, nt, P.oh_off);
     note_launches(1);
     e = cudaMemsetAsync(P.oh_cnt, 0, sizeof(int) * static_cast<size_t>(nt), s);
     if (e != cudaSuccess) return e;
-    onehot_rows_kernel<<<grid_r, 256, 0, s>>>(P.flags, targets, N, V, ignore_index, nt, P.oh_cnt, P.oh_off,
+    onehot_rows_kernel<<<grid_r, 256, 0, s>>>(P.flags, targets, N, V, vs, ignore_index, nt, P.oh_cnt, P.oh_off,
                                               P.oh_rows, 1);
     note_launches(1);
   }

@@ -33,6 +33,9 @@ struct FwdLaunch {
 // Counts every kernel launch of the calling thread (instrumentation for benchmarks).
 void note_launches(int n);
 
+// Limit of one bounded wait inside a kernel: CCE_WAIT_TIMEOUT_MS milliseconds (default 4000).
+uint64_t wait_timeout_ns();
+
 // Sets the message cce_last_error_message() returns on the calling thread.
 void set_last_error(const char* msg);
 
@@ -75,6 +78,13 @@ struct BwdPlan {
   int2* pair_slot;  // [pair capacity]: gradient-tile slots of t0 and t1, relative to the chunk
   int* grp_size;    // [2 * nchunks]: work items of each queue group (pairs of chunk c, then its dE/dC)
   int* grp_start;   // [2 * nchunks + 1]: their prefix sums
+  int* vt_order;    // [nt]: chunk c's vocabulary tiles at [chunk_t[c], chunk_t[c + 1]): first the ndc[c]
+                    // with a listed tile (dC items), ascending, then the empty ones, ascending
+  int* ndc;         // [nchunks]
+  int* de_list;     // [nchunks * nb]: row blocks with a listed tile in chunk c, ascending, at c * nb
+  int* nde;         // [nchunks]
+  int* empty_list;  // [nt]: the vocabulary tiles no row block lists (their dC rows are filled directly)
+  int* n_empty;     // [1], zero before planning
   int* oh_cnt;      // [nt]: rows whose target tile is onehot only, per vocabulary tile (scratch)
   int* oh_off;      // [nt + 1]: their prefix sums
   int* oh_rows;     // [N]: those rows, grouped by the vocabulary tile of their target
@@ -85,6 +95,7 @@ struct BwdArgs {
   int N, D, V, nb, nt, S, nchunks;
   int out_bf16;
   int64_t ignore_index;
+  int64_t vocab_start;  // C holds vocabulary rows [vocab_start, vocab_start + V); targets are global ids
   size_t buf_bytes;  // one of the kGradBuffers gradient-tile buffers
   const float* lse;
   const float* scale;
@@ -99,6 +110,10 @@ struct BwdArgs {
   const int* oh_off;          // [nt + 1]
   const int* oh_rows;         // rows whose target tile is onehot only, by vocabulary tile
   const int* grp_start;
+  const int* vt_order;
+  const int* ndc;
+  const int* de_list;
+  const int* nde;
   const int* chunk_t;
   const int* pstart_t;
   const int4* pair_desc;
@@ -126,17 +141,29 @@ struct BwdLaunch {
   int num_sms;
 };
 
+// Targets are ids in [0, vtot); this problem's C holds rows [vs, vs + V).
 cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float* lse, const int64_t* targets,
-                            int64_t N, int64_t V, int64_t T, int64_t ignore_index, float filter_eps,
-                            int64_t* filtered_tiles, cudaStream_t s);
+                            int64_t N, int64_t V, int64_t vs, int64_t vtot, int64_t T, int64_t ignore_index,
+                            float filter_eps, int64_t* filtered_tiles, cudaStream_t s);
 cudaError_t launch_bwd(const BwdLaunch& L, cudaStream_t s);
+// dC rows of the vocabulary tiles no row block lists (plan.empty_list): dc_coef * dc_add (or 0)
+// plus, for each row r whose target lies there, -scale_r * onehot_coef * E_r. bf16 or fp32 output.
+cudaError_t launch_dc_fill_empty(const BwdPlan& P, const int64_t* targets, int64_t vs, const float* scale,
+                                 float onehot_coef,
+                                 const __nv_bfloat16* E, int64_t D, int64_t V, const float* dc_add, float dc_coef,
+                                 void* dC, int out_bf16, int num_sms, cudaStream_t s);
+// out[i] = 1 if tile i of the plan's flags was skipped, 0 if it was kept (i < tiles).
+cudaError_t launch_skip_map(const uint8_t* flags, int64_t tiles, uint8_t* out, cudaStream_t s);
 
 cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
 
 // Small kernels (cce_aux.cu).
+// C holds vocabulary rows [vs, vs + V) of vtot (vs = 0, vtot = V for the whole vocabulary).
 cudaError_t launch_target_logit(const __nv_bfloat16* E, const __nv_bfloat16* C, const __nv_bfloat16* bias,
-                                const int64_t* targets, int64_t N, int64_t D, int64_t V, int64_t ignore_index,
-                                float* z_target, const float* csum, float* z_sum, int* err, cudaStream_t s);
+                                const int64_t* targets, int64_t N, int64_t D, int64_t V, int64_t vs, int64_t vtot,
+                                int64_t ignore_index, float* z_target, const float* csum, float* z_sum, int* err,
+                                cudaStream_t s);
+// loss_rows may be null (a vocabulary shard): then only lse is written.
 cudaError_t launch_lse_loss(const float* tile_max, const float* tile_sum, const float* z_target, const float* z_sum,
                             const int64_t* targets, int64_t N, int64_t T, int64_t ignore_index, int64_t V,
                             float label_smoothing, float z_loss, float* lse, float* loss_rows, cudaStream_t s);
@@ -150,11 +177,16 @@ cudaError_t launch_add_rank1(float* X, int64_t rows, int64_t D, const float* sca
 cudaError_t launch_add_scalar(float* X, int64_t n, float coef, const float* c, cudaStream_t s);
 // The onehot term of rows whose target tile was skipped: dE_acc[r] -= coef scale_r C[t_r] and
 // dbias_acc[t_r] -= coef scale_r (dbias_acc may be null), for the rows listed in rows[0:off[nt]].
-cudaError_t launch_onehot_rows(const int* off, int nt, const int* rows, const int64_t* targets,
+cudaError_t launch_onehot_rows(const int* off, int nt, const int* rows, const int64_t* targets, int64_t vs,
                                const float* scale, float coef, const __nv_bfloat16* C, int64_t D, float* dE_acc,
                                float* dbias_acc, int64_t max_rows, cudaStream_t s);
+// LSE over the whole vocabulary, loss, count and reduction from the shards' partial results [shards, 3, N].
+cudaError_t launch_shard_merge(const float* partials, int shards, const int64_t* targets, int64_t N, int64_t V,
+                               int64_t ignore_index, float label_smoothing, float z_loss, int reduction, float* loss,
+                               float* lse, int64_t* count, cudaStream_t s);
+// Count, reduction and, when *err != 0 (a device error earlier in the call), a NaN loss.
 cudaError_t launch_loss_reduce(const float* loss_rows, const int64_t* targets, int64_t N, int64_t ignore_index,
-                               int reduction, float* loss, int64_t* count, cudaStream_t s);
+                               int reduction, float* loss, int64_t* count, const int* err, cudaStream_t s);
 cudaError_t launch_row_scale(const int64_t* targets, const int64_t* count, const float* grad_out, int64_t N,
                              int64_t ignore_index, int reduction, float* scale, cudaStream_t s);
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, int64_t n, cudaStream_t s);

@@ -1,14 +1,17 @@
 // cce_forward_noalloc: the forward for callers that cannot allocate device memory.
 //
 // Some callers cannot call cudaMalloc or an allocator of their own at the point where they
-// compute the loss: code running while a CUDA graph is being captured, an embedding that
-// hands this library only fixed, pre-registered buffers for inputs and outputs, or a runtime
-// whose allocator must not be re-entered from inside a loss callback. For them this entry point
-// keeps its scratch (per-sub-tile exp sums, target logits, per-row losses and the device error
-// word) in one file-scope device array of kNoAllocScratchBytes, which every GPU that loads the
-// library holds until the process exits. The caller passes inputs and outputs only.
+// compute the loss: an embedding host that hands this library only fixed, pre-registered buffers
+// for inputs and outputs and owns all other device memory itself, or a runtime whose allocator
+// must not be re-entered from inside a loss callback (it may hold its own lock there, or account
+// every byte against a fixed budget). For them this entry point keeps its scratch (per-sub-tile
+// exp sums, target logits, per-row losses and the device error word) in one file-scope device
+// array of kNoAllocScratchBytes, which every GPU that loads the library holds until the process
+// exits. The caller passes inputs and outputs only.
 //
-// It launches the same kernels as cce_forward(); only where the scratch lives differs.
+// It launches the same kernels as cce_forward(); only where the scratch lives differs. A device
+// error (a target outside [0, V), a bounded wait that ran out) cannot be returned by this call,
+// which does not wait for the GPU; the final kernel then writes the loss as NaN instead.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -93,8 +96,8 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   if (p == nullptr || p->N < 0 || p->D < 8 || p->D % 8 != 0 || p->V < 1 || p->reduction < 0 || p->reduction > 2 ||
       p->reserved != 0 || p->N >= (int64_t(1) << 31) - 256 || p->V >= (int64_t(1) << 31) - 256 ||
       p->D >= (int64_t(1) << 24) || !(p->label_smoothing >= 0.f && p->label_smoothing <= 1.f) ||
-      !(p->z_loss >= 0.f && p->z_loss < INFINITY))
-    return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: invalid problem");
+      !(p->z_loss >= 0.f && p->z_loss < INFINITY) || p->vocab_start != 0 || (p->vocab_total != 0 && p->vocab_total != p->V))
+    return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: invalid problem (or a vocabulary shard)");
   const int64_t N = p->N, D = p->D, V = p->V;
   const int64_t T = (V + cce::kSubTile - 1) / cce::kSubTile;
   if (C == nullptr || loss == nullptr || count == nullptr ||
@@ -149,12 +152,13 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
     L.tile_max = tile_max;
     L.tile_sum = tile_sum;
     L.err = err;
-    L.timeout_ns = 4000000000ull;
+    L.timeout_ns = cce::wait_timeout_ns();
     L.num_sms = num_sms;
     L.inject_stall = 0;
     L.bias = Bb;
     if ((smooth && cce::launch_weighted_colsum(Cb, V, D, nullptr, Bb, csum, s) != cudaSuccess) ||
-        cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, p->ignore_index, z_target, smooth ? csum : nullptr,
+        cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, 0, V, p->ignore_index, z_target,
+                                 smooth ? csum : nullptr,
                                  smooth ? z_sum : nullptr, err, s) != cudaSuccess ||
         cce::launch_fwd_lse(L, s) != cudaSuccess ||
         cce::launch_lse_loss(tile_max, tile_sum, z_target, smooth ? z_sum : nullptr, targets, N, T, p->ignore_index,
@@ -162,7 +166,8 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
                              p->reduction == CCE_REDUCTION_NONE ? loss : loss_rows, s) != cudaSuccess)
       return fail(CCE_ERR_CUDA, "cce_forward_noalloc: kernel launch failed");
   }
-  if (cce::launch_loss_reduce(loss_rows, targets, N, p->ignore_index, p->reduction, loss, count, s) != cudaSuccess)
+  if (cce::launch_loss_reduce(loss_rows, targets, N, p->ignore_index, p->reduction, loss, count, err, s) !=
+      cudaSuccess)
     return fail(CCE_ERR_CUDA, "cce_forward_noalloc: kernel launch failed");
   return CCE_OK;
 }

@@ -50,6 +50,8 @@ class Problem(ctypes.Structure):
         ("reserved", ctypes.c_int32),
         ("label_smoothing", ctypes.c_float),
         ("z_loss", ctypes.c_float),
+        ("vocab_start", ctypes.c_int64),
+        ("vocab_total", ctypes.c_int64),
     ]
 
 
@@ -71,7 +73,12 @@ SIGNATURES = {
     "cce_set_kernel_events": (None, [_VP, _VP, _VP, _VP]),
     "cce_kernel_launch_count": (_I64, []),
     "cce_forward_noalloc": (_I32, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "cce_backward_skip_map": (_I32, [_PP, _VP, _SZ, _VP, _VP]),
+    "cce_forward_partial": (_I32, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "cce_forward_merge": (_I32, [_PP, _VP, _I32, _VP, _VP, _VP, _VP, _VP]),
 }
+
+OUT_BF16, OUT_FP32, OUT_DE_FP32 = 0, 1, 2  # cce_backward's output dtype modes
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -107,10 +114,11 @@ def _stream(device: torch.device) -> int:
 
 
 def _problem(N: int, D: int, V: int, ignore_index: int, reduction: str, label_smoothing: float = 0.0,
-             z_loss: float = 0.0) -> Problem:
+             z_loss: float = 0.0, vocab_start: int = 0, vocab_total: int = 0) -> Problem:
     if reduction not in REDUCTION_CODES:
         raise ValueError(f"reduction must be one of {tuple(REDUCTION_CODES)}, got {reduction!r}")
-    return Problem(N, D, V, ignore_index, REDUCTION_CODES[reduction], 0, float(label_smoothing), float(z_loss))
+    return Problem(N, D, V, ignore_index, REDUCTION_CODES[reduction], 0, float(label_smoothing), float(z_loss),
+                   int(vocab_start), int(vocab_total))
 
 
 def _require_cuda(*tensors: torch.Tensor) -> torch.device:
@@ -189,14 +197,19 @@ def cce_forward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, ignore_
 def cce_backward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, lse: torch.Tensor,
                  tile_max: torch.Tensor, count: torch.Tensor, grad_out: torch.Tensor,
                  filter_eps: float = DEFAULT_FILTER_EPS, ignore_index: int = -100,
-                 reduction: str = "mean", out_fp32: bool = False, check: bool = False,
+                 reduction: str = "mean", out_fp32=False, check: bool = False,
                  bias: Optional[torch.Tensor] = None, dbias: Optional[bool] = None,
-                 label_smoothing: float = 0.0, z_loss: float = 0.0):
-    """Run the backward. Returns (dE, dC, filtered_tiles) as device tensors, and dbias as a fourth
-    when it is computed (``dbias``; by default whenever ``bias`` is given)."""
+                 label_smoothing: float = 0.0, z_loss: float = 0.0, skip_map: bool = False,
+                 vocab_start: int = 0, vocab_total: int = 0):
+    """Run the backward. Returns (dE, dC, filtered_tiles) as device tensors, then dbias when it is
+    computed (``dbias``; by default whenever ``bias`` is given), then, with ``skip_map``, the uint8
+    [ceil(N / tile_rows), ceil(V / tile_cols)] map of skipped tiles (1 skipped, 0 kept).
+    ``out_fp32``: False / OUT_BF16, True / OUT_FP32, or OUT_DE_FP32 (dE fp32, dC and dbias bf16).
+    ``vocab_start`` / ``vocab_total``: C is rows [vocab_start, vocab_start + V) of a classifier of
+    vocab_total rows (0: not sharded); lse and count are then the merged ones."""
     lib = load_library()
     N, D, V = _check_operands(E, C, targets)
-    p = _problem(N, D, V, ignore_index, reduction, label_smoothing, z_loss)
+    p = _problem(N, D, V, ignore_index, reduction, label_smoothing, z_loss, vocab_start, vocab_total)
     tm_len = lib.cce_tile_max_len(ctypes.byref(p))
     _require(tm_len >= 0, f"bad problem N={N} D={D} V={V}: {lib.cce_last_error_message().decode()}")
     # the saved forward state, read in full by the backward's kernels
@@ -212,20 +225,78 @@ def cce_backward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, lse: t
     bias = _bias_arg(bias, V, dev)
     want_dbias = (bias is not None) if dbias is None else bool(dbias)
     g = grad_out.to(device=dev, dtype=torch.float32).reshape(-1).contiguous()
-    out_dtype = torch.float32 if out_fp32 else torch.bfloat16
-    dE = torch.empty(N, D, device=dev, dtype=out_dtype)
-    dC = torch.empty(V, D, device=dev, dtype=out_dtype)
-    db = torch.empty(V, device=dev, dtype=out_dtype) if want_dbias else None
+    mode = int(out_fp32)
+    _require(mode in (OUT_BF16, OUT_FP32, OUT_DE_FP32), f"out_fp32 must be 0, 1 or 2, got {out_fp32!r}")
+    de_dtype = torch.float32 if mode in (OUT_FP32, OUT_DE_FP32) else torch.bfloat16
+    dc_dtype = torch.float32 if mode == OUT_FP32 else torch.bfloat16
+    dE = torch.empty(N, D, device=dev, dtype=de_dtype)
+    dC = torch.empty(V, D, device=dev, dtype=dc_dtype)
+    db = torch.empty(V, device=dev, dtype=dc_dtype) if want_dbias else None
     filtered = torch.empty(1, device=dev, dtype=torch.int64)
-    ws_bytes = lib.cce_backward_workspace_size(ctypes.byref(p), int(out_fp32))
+    ws_bytes = lib.cce_backward_workspace_size(ctypes.byref(p), mode)
+    _require(ws_bytes > 0, f"bad problem: {lib.cce_last_error_message().decode()}")
     ws = torch.empty(max(ws_bytes, 1), device=dev, dtype=torch.uint8)
     with torch.cuda.device(dev):
         _check(lib.cce_backward(ctypes.byref(p), _ptr(E), _ptr(C), _ptr(bias), _ptr(targets), _ptr(lse),
                                 _ptr(tile_max), _ptr(count), _ptr(g), float(filter_eps), _ptr(dE), _ptr(dC), _ptr(db),
-                                int(out_fp32), _ptr(filtered), _ptr(ws), ws_bytes, _stream(dev)))
+                                mode, _ptr(filtered), _ptr(ws), ws_bytes, _stream(dev)))
+        smap = None
+        if skip_map:
+            tr, tc = backward_tile_shape()
+            smap = torch.empty(-(-N // tr), -(-V // tc), device=dev, dtype=torch.uint8)
+            _check(lib.cce_backward_skip_map(ctypes.byref(p), _ptr(ws), ws_bytes, _ptr(smap), _stream(dev)))
         if check:
             _check(lib.cce_check_device_error(_ptr(ws), _stream(dev)))
-    return (dE, dC, filtered, db) if want_dbias else (dE, dC, filtered)
+    out = (dE, dC, filtered) + ((db,) if want_dbias else ())
+    return out + (smap,) if skip_map else out
+
+
+def cce_forward_partial(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, vocab_start: int, vocab_total: int,
+                        ignore_index: int = -100, bias: Optional[torch.Tensor] = None, label_smoothing: float = 0.0,
+                        check: bool = False):
+    """Forward of one vocabulary shard: C is rows [vocab_start, vocab_start + V) of a classifier of
+    vocab_total rows. Returns (partial [3, N] fp32, tile_max) as device tensors: per row the shard's
+    log-sum-exp, the correct-token logit when the target lies in the shard (else 0), and the sum of
+    the shard's logits (label smoothing only; else 0)."""
+    lib = load_library()
+    N, D, V = _check_operands(E, C, targets)
+    dev = _require_cuda(E, C, targets)
+    E, C, targets = E.contiguous(), C.contiguous(), targets.contiguous()
+    bias = _bias_arg(bias, V, dev)
+    p = _problem(N, D, V, ignore_index, "none", label_smoothing, 0.0, vocab_start, vocab_total)
+    tm_len = lib.cce_tile_max_len(ctypes.byref(p))
+    _require(tm_len >= 0, f"bad problem: {lib.cce_last_error_message().decode()}")
+    partial = torch.empty(3, N, device=dev, dtype=torch.float32)
+    tile_max = torch.empty(max(tm_len, 1), device=dev, dtype=torch.float32)
+    ws_bytes = lib.cce_forward_workspace_size(ctypes.byref(p))
+    ws = torch.empty(max(ws_bytes, 1), device=dev, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        _check(lib.cce_forward_partial(ctypes.byref(p), _ptr(E), _ptr(C), _ptr(bias), _ptr(targets), _ptr(partial),
+                                       _ptr(tile_max), _ptr(ws), ws_bytes, _stream(dev)))
+        if check:
+            _check(lib.cce_check_device_error(_ptr(ws), _stream(dev)))
+    return partial, tile_max
+
+
+def cce_forward_merge(partials: torch.Tensor, targets: torch.Tensor, V: int, D: int, ignore_index: int = -100,
+                      reduction: str = "mean", label_smoothing: float = 0.0, z_loss: float = 0.0):
+    """Loss, LSE over the whole vocabulary of V entries, and count, from every shard's partial
+    results stacked as [shards, 3, N]. Returns (loss, lse, count) as device tensors."""
+    lib = load_library()
+    _require(partials.dim() == 3 and partials.shape[1] == 3 and partials.dtype == torch.float32,
+             f"partials must be float32 [shards, 3, N], got {partials.dtype} {tuple(partials.shape)}")
+    shards, _, N = partials.shape
+    _require(targets.dtype == torch.int64 and targets.numel() == N, f"targets must be int64 with N={N} entries")
+    dev = _require_cuda(partials, targets)
+    partials, targets = partials.contiguous(), targets.contiguous()
+    p = _problem(N, D, V, ignore_index, reduction, label_smoothing, z_loss)
+    loss = torch.empty(N if reduction == "none" else 1, device=dev, dtype=torch.float32)
+    lse = torch.empty(N, device=dev, dtype=torch.float32)
+    count = torch.empty(1, device=dev, dtype=torch.int64)
+    with torch.cuda.device(dev):
+        _check(lib.cce_forward_merge(ctypes.byref(p), _ptr(partials), shards, _ptr(targets), _ptr(loss), _ptr(lse),
+                                     _ptr(count), _stream(dev)))
+    return loss, lse, count
 
 
 class _LinearCrossEntropy(torch.autograd.Function):
@@ -284,3 +355,16 @@ def linear_cross_entropy(e: torch.Tensor, c: torch.Tensor, targets: torch.Tensor
         return out
     out = out.reshape(lead)
     return out[..., :-1] if shift else out
+
+
+def perplexity(e: torch.Tensor, c: torch.Tensor, targets: torch.Tensor, bias: Optional[torch.Tensor] = None,
+               ignore_index: int = -100, shift: bool = False) -> torch.Tensor:
+    """Perplexity exp(mean NLL) of the classifier on ``targets``, the mean taken over non-ignored
+    tokens (mlx-cross-entropy README, "Computing related quantities": the exponential of the mean
+    per-token negative log-likelihood). The mean NLL is the library's forward with reduction
+    "mean" (computed in its kernels, no logits stored); only the exponential of that one number is
+    taken here. With every token ignored the mean is 0 and the perplexity 1. No gradient flows."""
+    with torch.no_grad():
+        nll = linear_cross_entropy(e, c, targets, bias=bias, reduction="mean", ignore_index=ignore_index,
+                                   shift=shift)
+    return torch.exp(nll)

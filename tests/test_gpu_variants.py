@@ -95,3 +95,19 @@ def test_custom_ignore_index(device, ignore_index):
     assert rel_frob(dC.double().cpu().numpy(), b.dC) <= 1e-2
     raw = dE.cpu()[t == ignore_index]
     assert (raw.view(torch.int16) == 0).all(), "dE rows of ignored tokens must be exactly +0"
+
+
+@pytest.mark.parametrize("shift", [False, True])
+def test_perplexity_helper(device, shift):
+    """perplexity = exp(mean NLL over non-ignored tokens) (mlx-cross-entropy README, "Computing
+    related quantities"), against the oracle's per-token losses; every token ignored gives 1."""
+    inp = make_inputs("tiny", N=192, D=128, V=3000, seed=61, ignore_frac=0.1)
+    e = inp.E.reshape(4, 48, 128)
+    t = inp.targets.reshape(4, 48)
+    ppl = ops.perplexity(e.to(device), inp.C.to(device), t.to(device), shift=shift)
+    tt = ops.shift_targets(t) if shift else t
+    f = O.forward(inp.E, inp.C, tt.reshape(-1), -100, "none")
+    want = np.exp(f.nll.sum() / f.count)
+    assert abs(float(ppl) - want) <= want * LOSS_TOL
+    none = torch.full_like(t, -100)
+    assert float(ops.perplexity(e.to(device), inp.C.to(device), none.to(device))) == 1.0
