@@ -40,9 +40,11 @@ cce_status cuda_fail(cudaError_t e, const char* what) {
   return fail(CCE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-// Layout of the error word area at the start of every workspace.
+// Layout of the area at the start of every workspace (zeroed by every call).
 struct WsHeader {
-  int err;
+  int err;   // device error word
+  int done;  // blocks of the forward's finish kernel that are done
+  int bar;   // grid barrier counter of the backward's planning launch
 };
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -86,32 +88,58 @@ bool problem_ok(const cce_problem* p, bool set_error) {
 
 struct FwdWs {
   WsHeader* hdr;
-  float* tile_sum;
-  float* z_target;
-  float* loss_rows;
-  float* csum;   // [D + 1]: column sums of C and the bias sum (label smoothing only)
-  float* z_sum;  // [N]: sum over the vocabulary of each row's logits (label smoothing only)
+  float* tile_sum;           // [T, N]
+  float* csum;               // [D + 1]: column sums of C and the bias sum (label smoothing only)
+  double* block_sums;        // [ceil(N / 32)]: per-block loss sums of the finish kernel
+  long long* block_counts;   // [ceil(N / 32)]
   size_t bytes;
 };
 
 FwdWs carve_fwd(const cce_problem* p, void* base) {
   const int64_t T = ceil_div(p->V, cce::kSubTile);
+  const size_t nblk = static_cast<size_t>(std::max<int64_t>(ceil_div(p->N, cce::kFinishRows), 1));
   FwdWs w{};
   size_t off = kHeaderBytes;
   char* b = static_cast<char*>(base);
   w.hdr = reinterpret_cast<WsHeader*>(b);
   w.tile_sum = reinterpret_cast<float*>(b + off);
   off = align_up(off + sizeof(float) * static_cast<size_t>(T * p->N));
-  w.z_target = reinterpret_cast<float*>(b + off);
-  off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
-  w.loss_rows = reinterpret_cast<float*>(b + off);
-  off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
   w.csum = reinterpret_cast<float*>(b + off);
   off = align_up(off + sizeof(float) * static_cast<size_t>(p->D + 1));
-  w.z_sum = reinterpret_cast<float*>(b + off);
-  off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
+  w.block_sums = reinterpret_cast<double*>(b + off);
+  off = align_up(off + sizeof(double) * nblk);
+  w.block_counts = reinterpret_cast<long long*>(b + off);
+  off = align_up(off + sizeof(long long) * nblk);
   w.bytes = off;
   return w;
+}
+
+// The finish kernel's arguments common to the whole-vocabulary and the shard forward.
+cce::FwdFinish finish_args(const cce_problem* p, const FwdWs& w, const void* E, const void* C, const void* bias,
+                           const int64_t* targets, const float* tile_max, bool smooth) {
+  cce::FwdFinish F{};
+  F.tile_max = tile_max;
+  F.tile_sum = w.tile_sum;
+  F.N = p->N;
+  F.T = ceil_div(p->V, cce::kSubTile);
+  F.D = p->D;
+  F.V = p->V;
+  F.vs = p->vocab_start;
+  F.vtot = vocab_total(p);
+  F.ignore_index = p->ignore_index;
+  F.E = static_cast<const __nv_bfloat16*>(E);
+  F.C = static_cast<const __nv_bfloat16*>(C);
+  F.bias = static_cast<const __nv_bfloat16*>(bias);
+  F.targets = targets;
+  F.csum = smooth ? w.csum : nullptr;
+  F.label_smoothing = p->label_smoothing;
+  F.z_loss = p->z_loss;
+  F.reduction = p->reduction;
+  F.block_sums = w.block_sums;
+  F.block_counts = w.block_counts;
+  F.done = &w.hdr->done;
+  F.err = &w.hdr->err;
+  return F;
 }
 
 // Workspace of the backward: the tile plan and work lists, the queue counters, two gradient-tile
@@ -184,6 +212,7 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.nde = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks)));
   w.plan.empty_list = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt)));
   w.plan.oh_cnt = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt)));
+  w.plan.oh_cur = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt)));
   w.plan.oh_off = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt + 1)));
   w.plan.oh_rows = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(std::max<int64_t>(p->N, 1))));
   w.sync_bytes = sizeof(int) * static_cast<size_t>(1 + w.plan.nchunks * nb + nt + w.plan.nchunks);
@@ -284,12 +313,35 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
     return cudaMemsetAsync(filtered_tiles, 0, sizeof(int64_t), s) == cudaSuccess ? CCE_OK
                                                                                   : fail(CCE_ERR_CUDA, "memset");
   }
-  CCE_TRY(cce::launch_row_scale(targets, count, grad_out, N, p->ignore_index, p->reduction, w.scale, s));
-  CCE_TRY(cce::launch_bwd_plan(w.plan, tile_max, lse, targets, N, V, vs, vtot, T, p->ignore_index, filter_eps,
-                               filtered_tiles, s));
-  CCE_TRY(cce::launch_fill_zero(dE_acc, N * D * 4, s));
-  if (dbias_acc != nullptr) CCE_TRY(cce::launch_fill_zero(dbias_acc, V * 4, s));
   CCE_TRY(cudaMemsetAsync(w.sync, 0, w.sync_bytes, s));
+  {
+    cce::PlanArgs PA{};
+    PA.P = w.plan;
+    PA.tile_max = tile_max;
+    PA.lse = lse;
+    PA.targets = targets;
+    PA.count = count;
+    PA.grad_out = grad_out;
+    PA.N = N;
+    PA.D = D;
+    PA.V = V;
+    PA.T = T;
+    PA.vs = vs;
+    PA.vtot = vtot;
+    PA.ignore_index = p->ignore_index;
+    PA.reduction = p->reduction;
+    PA.filter_on = filter_eps > 0.f ? 1 : 0;
+    PA.ln_eps = PA.filter_on ? logf(filter_eps) : -INFINITY;
+    PA.scale = w.scale;
+    PA.onehot_coef = 1.f - p->label_smoothing;
+    PA.dE_acc = dE_acc;
+    PA.dbias_acc = dbias_acc;
+    PA.filtered_tiles = filtered_tiles;
+    PA.bar = &w.hdr->bar;
+    PA.err = &w.hdr->err;
+    PA.timeout_ns = cce::wait_timeout_ns();
+    CCE_TRY(cce::launch_bwd_plan(PA, num_sms, s));
+  }
   // Label smoothing: the ls / V part of every row's target is a rank-one term, added exactly:
   // dE_r -= scale_r (ls / V) sum_v C_v, dC_v -= (ls / V) sum_r scale_r E_r, dbias_v -= (ls / V) sum_r scale_r.
   const bool smooth = p->label_smoothing > 0.f;
@@ -362,19 +414,34 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
   CCE_TRY(cce::launch_bwd(L, s));
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
-  // dC rows of vocabulary tiles no row block lists: written without the tensor cores
-  CCE_TRY(cce::launch_dc_fill_empty(w.plan, targets, vs, w.scale, 1.f - p->label_smoothing, Eb, D, V,
-                                    smooth ? w.wsum : nullptr, -ls_v, dC, c32 ? 0 : 1, num_sms, s));
-  CCE_TRY(cce::launch_onehot_rows(w.plan.oh_off, w.plan.nt, w.plan.oh_rows, targets, vs, w.scale,
-                                  1.f - p->label_smoothing,
-                                  static_cast<const __nv_bfloat16*>(C), D, dE_acc, dbias_acc, N, s));
-  if (smooth) {
-    CCE_TRY(cce::launch_add_rank1(dE_acc, N, D, w.scale, -ls_v, w.csum, s));
-    if (dbias_acc != nullptr) CCE_TRY(cce::launch_add_scalar(dbias_acc, V, -ls_v, w.wsum + D, s));
-  }
-  if (!e32) CCE_TRY(cce::launch_to_bf16(dE_acc, static_cast<__nv_bfloat16*>(dE), N * D, s));
-  if (!c32 && dbias != nullptr)
-    CCE_TRY(cce::launch_to_bf16(dbias_acc, static_cast<__nv_bfloat16*>(dbias), V, s));
+  // the rest: dE's last terms and conversion, dC rows of vocabulary tiles no row block lists, dbias
+  cce::BwdFinalize F{};
+  F.N = N;
+  F.D = D;
+  F.V = V;
+  F.vs = vs;
+  F.ignore_index = p->ignore_index;
+  F.nt = w.plan.nt;
+  F.flags = w.plan.flags;
+  F.empty_list = w.plan.empty_list;
+  F.n_empty = w.plan.n_empty;
+  F.oh_off = w.plan.oh_off;
+  F.oh_rows = w.plan.oh_rows;
+  F.targets = targets;
+  F.scale = w.scale;
+  F.onehot_coef = 1.f - p->label_smoothing;
+  F.ls_v = ls_v;
+  F.E = Eb;
+  F.C = static_cast<const __nv_bfloat16*>(C);
+  F.csum = smooth ? w.csum : nullptr;
+  F.wsum = smooth ? w.wsum : nullptr;
+  F.dE_acc = dE_acc;
+  F.dE_out = e32 ? nullptr : dE;
+  F.dC = dC;
+  F.dc_bf16 = c32 ? 0 : 1;
+  F.dbias_acc = dbias_acc;
+  F.dbias_out = (dbias != nullptr && !c32) ? dbias : nullptr;
+  CCE_TRY(cce::launch_bwd_finalize(F, num_sms, s));
   return CCE_OK;
 }
 
@@ -462,11 +529,11 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
   CCE_CHECK(get_encoder());
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t N = p->N, D = p->D, V = p->V, T = ceil_div(V, cce::kSubTile);
-  const auto* Eb = static_cast<const __nv_bfloat16*>(E);
   const auto* Cb = static_cast<const __nv_bfloat16*>(C);
   const auto* Bb = static_cast<const __nv_bfloat16*>(bias);
 
   CCE_TRY(cudaMemsetAsync(w.hdr, 0, sizeof(WsHeader), s));
+  const bool smooth = p->label_smoothing > 0.f;
   if (has_rows) {
     cce::FwdLaunch L{};
     L.bias = Bb;
@@ -485,19 +552,16 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
     // (reported as CCE_ERR_DEVICE_TIMEOUT by cce_check_device_error; the outputs are undefined).
     const char* stall = std::getenv("CCE_TEST_INJECT_STALL");
     L.inject_stall = (stall != nullptr && stall[0] == '1') ? 1 : 0;
-    const bool smooth = p->label_smoothing > 0.f;
     if (smooth) CCE_TRY(cce::launch_weighted_colsum(Cb, V, D, nullptr, Bb, w.csum, s));
-    CCE_TRY(cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, 0, V, p->ignore_index, w.z_target,
-                                     smooth ? w.csum : nullptr, smooth ? w.z_sum : nullptr, &w.hdr->err, s));
     if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[0], s));
     CCE_TRY(cce::launch_fwd_lse(L, s));
     if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[1], s));
-    float* rows_out = p->reduction == CCE_REDUCTION_NONE ? loss : w.loss_rows;
-    CCE_TRY(cce::launch_lse_loss(tile_max, w.tile_sum, w.z_target, smooth ? w.z_sum : nullptr, targets, N, T,
-                                 p->ignore_index, V, p->label_smoothing, p->z_loss, lse, rows_out, s));
   }
-  CCE_TRY(cce::launch_loss_reduce(w.loss_rows, targets, N, p->ignore_index, p->reduction, loss, count,
-                                   &w.hdr->err, s));
+  cce::FwdFinish F = finish_args(p, w, E, C, bias, targets, tile_max, smooth);
+  F.lse = lse;
+  F.loss = loss;
+  F.count = count;
+  CCE_TRY(cce::launch_fwd_finish(F, s));
   return CCE_OK;
 }
 
@@ -542,12 +606,8 @@ cce_status cce_forward_partial(const cce_problem* p, const void* E, const void* 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   CCE_TRY(cudaMemsetAsync(w.hdr, 0, sizeof(WsHeader), s));
   if (N == 0) return CCE_OK;
-  const auto* Eb = static_cast<const __nv_bfloat16*>(E);
   const auto* Cb = static_cast<const __nv_bfloat16*>(C);
   const auto* Bb = static_cast<const __nv_bfloat16*>(bias);
-  float* lse_part = partial;
-  float* zt_part = partial + N;
-  float* zs_part = partial + 2 * N;
   const bool smooth = p->label_smoothing > 0.f;
   cce::FwdLaunch L{};
   L.bias = Bb;
@@ -564,14 +624,15 @@ cce_status cce_forward_partial(const cce_problem* p, const void* E, const void* 
   L.num_sms = num_sms;
   L.inject_stall = 0;
   if (smooth) CCE_TRY(cce::launch_weighted_colsum(Cb, V, D, nullptr, Bb, w.csum, s));
-  else CCE_TRY(cudaMemsetAsync(zs_part, 0, sizeof(float) * static_cast<size_t>(N), s));
-  CCE_TRY(cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, p->vocab_start, vocab_total(p), p->ignore_index,
-                                   zt_part, smooth ? w.csum : nullptr, smooth ? zs_part : nullptr, &w.hdr->err, s));
   if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[0], s));
   CCE_TRY(cce::launch_fwd_lse(L, s));
   if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[1], s));
-  CCE_TRY(cce::launch_lse_loss(tile_max, w.tile_sum, nullptr, nullptr, targets, N, T, p->ignore_index, V, 0.f, 0.f,
-                               lse_part, nullptr, s));
+  // partial rows: the shard's log-sum-exp, correct-token logit and logit sum (0 without smoothing)
+  cce::FwdFinish F = finish_args(p, w, E, C, bias, targets, tile_max, smooth);
+  F.lse = partial;
+  F.zt_out = partial + N;
+  F.zs_out = partial + 2 * N;
+  CCE_TRY(cce::launch_fwd_finish(F, s));
   return CCE_OK;
 }
 

@@ -444,6 +444,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t reg0 = smem_u32(region);
     const uint32_t stg = reg0 + static_cast<uint32_t>(q * STG_WARP);
     uint32_t acc_iter = 0, rphase = 0, gphase = 0;
+    uint32_t img = 0;  // which of the two 4 KB staging images of this warp comes next
     bool ok = true;
     // Every lane waits (and acquires) itself; the vote makes the outcome warp-uniform, so the warp
     // stays converged for the .sync.aligned TMEM loads and takes one branch on failure.
@@ -666,38 +667,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (x + 32 + e < A.D) v1[e] = fmaf(A.dc_coef, A.dc_add[x + 32 + e], v1[e]);
           }
         }
-        // this warp's staging is free once its previous TMA op has read it
-        if (lane == 0) bulk_wait_group_read0();
-        __syncwarp();
-        if (!de && A.out_bf16) {
+        if (y >= rows_limit) continue;  // this warp's 32 rows lie past the end of dE / dC
+        // The warp's 8 KB of staging holds two 4 KB images used in turn; an image is rewritten once
+        // the TMA operation issued from it two images earlier has read it, so one operation is
+        // always in flight while the next image is written.
+        auto next_image = [&]() {
+          if (lane == 0) bulk_wait_group_read1();
+          __syncwarp();
+          return stg + 4096u * (img++ & 1u);
+        };
+        auto put_f32 = [&](const float (&v)[32], int xc) {  // 32 rows x 32 fp32 columns
+          const uint32_t im = next_image();
+#pragma unroll
+          for (int h = 0; h < 8; ++h)
+            st_shared_v4(im + swz(lane, h), __float_as_uint(v[4 * h]), __float_as_uint(v[4 * h + 1]),
+                         __float_as_uint(v[4 * h + 2]), __float_as_uint(v[4 * h + 3]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (de) tma_reduce_add_2d(&tmdE, im, xc, y);
+            else tma_store_2d(&tmdC, im, xc, y);
+            bulk_commit_group();
+          }
+        };
+        if (!de && A.out_bf16) {  // 32 rows x 64 bf16 columns in one image
+          const uint32_t im = next_image();
 #pragma unroll
           for (int h = 0; h < 8; ++h) {
             const float* src = h < 4 ? v0 + 8 * h : v1 + 8 * (h - 4);
-            st_shared_v4(stg + swz(lane, h), pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+            st_shared_v4(im + swz(lane, h), pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
                          pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmdC, im, x, y);
+            bulk_commit_group();
+          }
         } else {
-#pragma unroll
-          for (int h = 0; h < 8; ++h) {
-            st_shared_v4(stg + swz(lane, h), __float_as_uint(v0[4 * h]), __float_as_uint(v0[4 * h + 1]),
-                         __float_as_uint(v0[4 * h + 2]), __float_as_uint(v0[4 * h + 3]));
-            st_shared_v4(stg + 4096u + swz(lane, h), __float_as_uint(v1[4 * h]), __float_as_uint(v1[4 * h + 1]),
-                         __float_as_uint(v1[4 * h + 2]), __float_as_uint(v1[4 * h + 3]));
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && y < rows_limit) {
-          if (!de && A.out_bf16) {
-            tma_store_2d(&tmdC, stg, x, y);
-          } else if (!de) {
-            tma_store_2d(&tmdC, stg, x, y);
-            if (x + 32 < A.D) tma_store_2d(&tmdC, stg + 4096u, x + 32, y);
-          } else {
-            tma_reduce_add_2d(&tmdE, stg, x, y);
-            if (x + 32 < A.D) tma_reduce_add_2d(&tmdE, stg + 4096u, x + 32, y);
-          }
-          bulk_commit_group();
+          put_f32(v0, x);
+          if (x + 32 < A.D) put_f32(v1, x + 32);
         }
       }
       if (has) {

@@ -32,89 +32,59 @@ __device__ __forceinline__ bool valid_target(int64_t t, int64_t V, int64_t ignor
   return t != ignore_index && t >= 0 && t < V;
 }
 
-// One block of 128 threads (one per tile row) per row block b and run of kFlagTiles vocabulary
-// tiles: the flags of those tiles. The rows' targets and LSE are read once for the whole run.
-constexpr int kFlagTiles = 8;
+// The planning runs as one cooperative launch of one 1024-thread block per SM: a sequence of
+// phases separated by grid-wide barriers (bounded waits; a block that gives up records
+// CCE_ERR_DEVICE_TIMEOUT and every block then leaves). Each phase spreads its work over the grid.
+constexpr int kPlanThreads = 1024;
+constexpr int kFlagTiles = 8;    // vocabulary tiles per flag unit
+constexpr int kFlagGroups = kPlanThreads / kBwdBM;  // flag units per block at a time (128 threads each)
 
-__global__ void tile_flags_kernel(const float* __restrict__ tile_max, const float* __restrict__ lse,
-                                  const int64_t* __restrict__ targets, int64_t N, int64_t V, int64_t vs,
-                                  int64_t vtot, int64_t T, int64_t ignore_index, float ln_eps, int filter_on, int nt,
-                                  int runs, uint8_t* __restrict__ flags) {
-  __shared__ float wmax[kFlagTiles][4];
-  __shared__ int any_target[kFlagTiles];
-  const int b = static_cast<int>(blockIdx.x / runs), t0 = static_cast<int>(blockIdx.x % runs) * kFlagTiles;
-  const int64_t r = static_cast<int64_t>(b) * kBwdBM + threadIdx.x;
-  if (threadIdx.x < kFlagTiles) any_target[threadIdx.x] = 0;
+struct PlanCtl {
+  int* bar;        // barrier counter, zero at launch
+  int* err;
+  uint64_t timeout_ns;
+};
+
+// Grid-wide barrier number `round` (1, 2, ...): every block's writes before it are visible to every
+// block after it. Returns false when the wait ran out or another block recorded an error.
+__device__ bool grid_barrier(const PlanCtl& ctl, int round) {
+  __shared__ int ok;
   __syncthreads();
-  bool valid = false, local = false;
-  float l = 0.f;
-  int64_t tr = -1;
-  if (r < N) {
-    tr = targets[r];
-    valid = valid_target(tr, vtot, ignore_index);      // the row is scored (by every shard)
-    local = valid && valid_target(tr - vs, V, ignore_index - vs);  // its target lies in this shard
-    if (valid && filter_on) l = lse[r];
-    tr -= vs;
-  }
-  if (local && tr / kBwdBN >= t0 && tr / kBwdBN < t0 + kFlagTiles) any_target[tr / kBwdBN - t0] = 1;
-#pragma unroll
-  for (int k = 0; k < kFlagTiles; ++k) {
-    const int t = t0 + k;
-    float m = -INFINITY;
-    if (valid && filter_on && t < nt) {
-      const int64_t j0 = static_cast<int64_t>(t) * (kBwdBN / kSubTile);
-      const int64_t j1 = j0 + kBwdBN / kSubTile < T ? j0 + kBwdBN / kSubTile : T;
-      for (int64_t j = j0; j < j1; ++j) m = fmaxf(m, tile_max[j * N + r]);
-      m -= l;
+  if (threadIdx.x == 0) {
+    ok = 1;
+    __threadfence();
+    red_release_add(ctl.bar, 1);
+    const int target = round * static_cast<int>(gridDim.x);
+    const uint64_t t0 = global_timer_ns();
+    while (ld_acquire(ctl.bar) < target) {
+      if (ld_relaxed(ctl.err) != 0) {
+        ok = 0;
+        break;
+      }
+      if (global_timer_ns() - t0 > ctl.timeout_ns) {
+        record_error(ctl.err, kErrDeviceTimeout);
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
     }
-    m = warp_max(m);
-    if ((threadIdx.x & 31) == 0) wmax[k][threadIdx.x >> 5] = m;
   }
   __syncthreads();
-  if (threadIdx.x < kFlagTiles && t0 + threadIdx.x < nt) {
-    const int k = threadIdx.x;
-    const bool keep = !filter_on || fmaxf(fmaxf(wmax[k][0], wmax[k][1]), fmaxf(wmax[k][2], wmax[k][3])) >= ln_eps;
-    flags[static_cast<int64_t>(b) * nt + t0 + k] = keep ? 1 : (any_target[k] ? 2 : 0);
-  }
+  return ok != 0;
 }
 
-// One warp per vocabulary tile t: the rank of each listed (b, t) among the listed row blocks of t,
-// the number of listed tiles of t, and the kept total.
-__global__ void tile_rank_kernel(const uint8_t* __restrict__ flags, int nb, int nt, int* __restrict__ rank,
-                                 int* __restrict__ cnt_t, int* __restrict__ cnt_b, int* __restrict__ kept_total) {
-  const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= nt) return;
-  int listed = 0, kept = 0;
-  for (int b0 = 0; b0 < nb; b0 += 32) {
-    const int b = b0 + lane;
-    const uint8_t f = b < nb ? flags[static_cast<int64_t>(b) * nt + t] : 0;
-    const unsigned on = __ballot_sync(0xffffffffu, f == 1);
-    if (f == 1) {
-      rank[static_cast<int64_t>(b) * nt + t] = listed + __popc(on & ((1u << lane) - 1u));
-      atomicAdd(cnt_b + b, 1);
-    }
-    listed += __popc(on);
-    kept += __popc(__ballot_sync(0xffffffffu, f == 1));
-  }
-  if (lane == 0) {
-    cnt_t[t] = listed;
-    atomicAdd(kept_total, kept);
-  }
-}
-
-// Exclusive scan of cnt[0..n) into off[0..n]; one block of 1024 threads, in chunks.
-__global__ void scan_kernel(const int* __restrict__ cnt, int n, int* __restrict__ off) {
-  __shared__ int buf[1024];
+// Exclusive scan of cnt[0..n) into off[0..n] by the calling block (1024 threads), in chunks.
+__device__ void block_scan(const int* __restrict__ cnt, int n, int* __restrict__ off) {
+  __shared__ int buf[kPlanThreads];
   __shared__ int carry;
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
-  for (int base = 0; base < n; base += 1024) {
+  for (int base = 0; base < n; base += kPlanThreads) {
     const int i = base + threadIdx.x;
     const int v = i < n ? cnt[i] : 0;
     buf[threadIdx.x] = v;
     __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
+    for (int o = 1; o < kPlanThreads; o <<= 1) {
       const int add = threadIdx.x >= o ? buf[threadIdx.x - o] : 0;
       __syncthreads();
       buf[threadIdx.x] += add;
@@ -122,35 +92,90 @@ __global__ void scan_kernel(const int* __restrict__ cnt, int n, int* __restrict_
     }
     if (i < n) off[i] = carry + buf[threadIdx.x] - v;
     __syncthreads();
-    if (threadIdx.x == 1023) carry += buf[1023];
+    if (threadIdx.x == kPlanThreads - 1) carry += buf[kPlanThreads - 1];
     __syncthreads();
   }
   if (threadIdx.x == 0) off[n] = carry;
+  __syncthreads();
 }
 
-__global__ void fill_col_kernel(const uint8_t* __restrict__ flags, const int* __restrict__ rank,
-                                const int* __restrict__ offsets_t, int nb, int nt, int2* __restrict__ entries_t) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= static_cast<int64_t>(nb) * nt) return;
-  const uint8_t f = flags[i];
-  if (f != 1) return;
-  const int b = static_cast<int>(i / nt), t = static_cast<int>(i % nt);
-  entries_t[offsets_t[t] + rank[i]] = make_int2(b * 4 + f, t);
+// Block-wide ordered compaction: every thread holds one flag; returns the number of set flags
+// before this thread (ascending thread order) and sets *total to the block's count.
+__device__ __forceinline__ int block_rank(bool flag, int* total) {
+  __shared__ int warps[32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const unsigned m = __ballot_sync(0xffffffffu, flag);
+  if (lane == 0) warps[w] = __popc(m);
+  __syncthreads();
+  int before = 0, all = 0;
+  for (int k = 0; k < nw; ++k) {
+    before += k < w ? warps[k] : 0;
+    all += warps[k];
+  }
+  __syncthreads();  // warps[] may be rewritten by the next call
+  *total = all;
+  return before + __popc(m & ((1u << lane) - 1u));
 }
 
-// One block of 1024 threads per row block: writes its listed tiles in vocabulary order (a block-wide
-// scan of the listed flags, 1024 vocabulary tiles per step), and the inverse map pos_b.
-__global__ void row_list_kernel(const uint8_t* __restrict__ flags, const int* __restrict__ rank,
-                                const int* __restrict__ offsets_t, int nt, const int* __restrict__ offsets_b,
-                                int2* __restrict__ entries_b, int* __restrict__ pos_b) {
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Flags of one row block b and run of kFlagTiles vocabulary tiles from t0, by 128 threads (one per
+// tile row; named barrier `group + 1`). The rows' targets and LSE are read once for the run.
+__device__ void tile_flags_unit(const PlanArgs& A, int group, int b, int t0) {
+  __shared__ float wmax[kFlagGroups][kFlagTiles][4];
+  __shared__ int any_target[kFlagGroups][kFlagTiles];
+  const int tid = threadIdx.x & (kBwdBM - 1);
+  const int nt = A.P.nt;
+  const int64_t r = static_cast<int64_t>(b) * kBwdBM + tid;
+  if (tid < kFlagTiles) any_target[group][tid] = 0;
+  named_barrier(group + 1, kBwdBM);
+  bool valid = false, local = false;
+  float l = 0.f;
+  int64_t tr = -1;
+  if (r < A.N) {
+    tr = A.targets[r];
+    valid = valid_target(tr, A.vtot, A.ignore_index);                 // the row is scored (by every shard)
+    local = valid && valid_target(tr - A.vs, A.V, A.ignore_index - A.vs);  // its target lies in this shard
+    if (valid && A.filter_on) l = A.lse[r];
+    tr -= A.vs;
+  }
+  if (local && tr / kBwdBN >= t0 && tr / kBwdBN < t0 + kFlagTiles) any_target[group][tr / kBwdBN - t0] = 1;
+#pragma unroll
+  for (int k = 0; k < kFlagTiles; ++k) {
+    const int t = t0 + k;
+    float m = -INFINITY;
+    if (valid && A.filter_on && t < nt) {
+      const int64_t j0 = static_cast<int64_t>(t) * (kBwdBN / kSubTile);
+      const int64_t j1 = j0 + kBwdBN / kSubTile < A.T ? j0 + kBwdBN / kSubTile : A.T;
+      for (int64_t j = j0; j < j1; ++j) m = fmaxf(m, A.tile_max[j * A.N + r]);
+      m -= l;
+    }
+    m = warp_max(m);
+    if ((tid & 31) == 0) wmax[group][k][tid >> 5] = m;
+  }
+  named_barrier(group + 1, kBwdBM);
+  if (tid < kFlagTiles && t0 + tid < nt) {
+    const float* wm = wmax[group][tid];
+    const bool keep = !A.filter_on || fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3])) >= A.ln_eps;
+    A.P.flags[static_cast<int64_t>(b) * nt + t0 + tid] = keep ? 1 : (any_target[group][tid] ? 2 : 0);
+  }
+  named_barrier(group + 1, kBwdBM);  // the shared arrays are reused by the group's next unit
+}
+
+// The listed tiles of row block b in vocabulary order (a block-wide scan of its flags, 1024 vocabulary
+// tiles per step) and the inverse map pos_b; the whole block.
+__device__ void row_list_block(const PlanArgs& A, int b) {
   __shared__ int wsum[32];
   __shared__ int carry;
-  const int b = blockIdx.x;
+  const BwdPlan& P = A.P;
+  const int nt = P.nt;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const uint8_t* row = flags + static_cast<int64_t>(b) * nt;
-  if (threadIdx.x == 0) carry = offsets_b[b];
+  const uint8_t* row = P.flags + static_cast<int64_t>(b) * nt;
+  if (threadIdx.x == 0) carry = P.offsets_b[b];
   __syncthreads();
-  for (int t0 = 0; t0 < nt; t0 += 1024) {
+  for (int t0 = 0; t0 < nt; t0 += kPlanThreads) {
     const int t = t0 + threadIdx.x;
     const bool on = t < nt && row[t] == 1;
     const unsigned m = __ballot_sync(0xffffffffu, on);
@@ -163,9 +188,9 @@ __global__ void row_list_kernel(const uint8_t* __restrict__ flags, const int* __
     }
     if (on) {
       const int pos = carry + before + __popc(m & ((1u << lane) - 1u));
-      const int slot = offsets_t[t] + rank[static_cast<int64_t>(b) * nt + t];
-      entries_b[pos] = make_int2(t, slot);
-      pos_b[slot] = pos;
+      const int slot = P.offsets_t[t] + P.rank[static_cast<int64_t>(b) * nt + t];
+      P.entries_b[pos] = make_int2(t, slot);
+      P.pos_b[slot] = pos;
     }
     __syncthreads();  // everyone has read carry and wsum
     if (threadIdx.x == 0) carry += total;
@@ -182,37 +207,18 @@ __device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int 
   return lo;
 }
 
-// For every chunk c and row block b, the range [lo, hi) of b's entries_b inside the chunk.
-// Chunk c covers vocabulary tiles [c * chunk_vt, min(nt, (c + 1) * chunk_vt)).
-__global__ void row_range_kernel(const int2* __restrict__ entries_b, const int* __restrict__ offsets_b, int nb,
-                                 int nchunks, int nt, int chunk_vt, int2* __restrict__ rb_range) {
-  const int64_t total = static_cast<int64_t>(nb) * nchunks;
-  for (int64_t cb = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; cb < total;
-       cb += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(cb / nb), b = static_cast<int>(cb % nb);
-    const int lo = lower_bound_t(entries_b, offsets_b[b], offsets_b[b + 1], min(nt, c * chunk_vt));
-    const int hi = lower_bound_t(entries_b, lo, offsets_b[b + 1], min(nt, (c + 1) * chunk_vt));
-    rb_range[cb] = make_int2(lo, hi);
-  }
-}
-
 // A listed tile (b, t) starts a pair when its position in row block b's list inside t's chunk is
 // even; the pair is (b, t) and b's next listed tile in the chunk, if any. Pairs are listed by the
 // vocabulary tile of their first tile (then row block), so that the recompute of concurrent pairs
-// shares C tiles in L2. One warp per vocabulary tile; pass 0 counts the pairs starting in tile t,
-// pass 1 (after the scan of those counts into pstart_t) writes them.
-__global__ void pair_list_kernel(const int2* __restrict__ entries_t, const int* __restrict__ offsets_t,
-                                 const int2* __restrict__ entries_b, const int* __restrict__ pos_b,
-                                 const int2* __restrict__ rb_range, const uint8_t* __restrict__ flags, int nb, int nt,
-                                 int chunk_vt, int* __restrict__ cnt,
-                                 const int* __restrict__ pstart_t, int4* __restrict__ pair_desc,
-                                 int2* __restrict__ pair_slot, int pass) {
-  const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= nt) return;
-  const int c = t / chunk_vt;
-  const int slot_base = offsets_t[c * chunk_vt];
-  const int i0 = offsets_t[t], i1 = offsets_t[t + 1];
+// shares C tiles in L2. One warp per vocabulary tile; pass 0 counts the pairs starting in tile t
+// (into cnt_t, whose tile counts are already scanned into offsets_t), pass 1 (after the scan of
+// those counts into pstart_t) writes them.
+__device__ void pair_list_warp(const PlanArgs& A, int t, int lane, int pass) {
+  const BwdPlan& P = A.P;
+  const int nb = P.nb, nt = P.nt;
+  const int c = t / P.chunk_vt;
+  const int slot_base = P.offsets_t[c * P.chunk_vt];
+  const int i0 = P.offsets_t[t], i1 = P.offsets_t[t + 1];
   int k = 0;
   for (int base = i0; base < i1; base += 32) {
     const int i = base + lane;
@@ -220,189 +226,366 @@ __global__ void pair_list_kernel(const int2* __restrict__ entries_t, const int* 
     int b = 0, p = 0;
     int2 rr = make_int2(0, 0);
     if (i < i1) {
-      b = entries_t[i].x >> 2;
-      p = pos_b[i];
-      rr = rb_range[static_cast<int64_t>(c) * nb + b];
+      b = P.entries_t[i].x >> 2;
+      p = P.pos_b[i];
+      rr = P.rb_range[static_cast<int64_t>(c) * nb + b];
       start = ((p - rr.x) & 1) == 0;
     }
     const unsigned mask = __ballot_sync(0xffffffffu, start);
     if (pass == 1 && start) {
-      const int out = pstart_t[t] + k + __popc(mask & ((1u << lane) - 1u));
+      const int out = P.pstart_t[t] + k + __popc(mask & ((1u << lane) - 1u));
       const bool two = p + 1 < rr.y;
-      const int t1 = two ? entries_b[p + 1].x : -1;
-      const int slot1 = two ? entries_b[p + 1].y : i;
-      const uint8_t* row = flags + static_cast<int64_t>(b) * nt;
+      const int t1 = two ? P.entries_b[p + 1].x : -1;
+      const int slot1 = two ? P.entries_b[p + 1].y : i;
+      const uint8_t* row = P.flags + static_cast<int64_t>(b) * nt;
       const int kept = (row[t] == 1 ? 1 : 0) | (two && row[t1] == 1 ? 2 : 0);
-      pair_desc[out] = make_int4(b, t, t1, kept);
-      pair_slot[out] = make_int2(i - slot_base, slot1 - slot_base);
+      P.pair_desc[out] = make_int4(b, t, t1, kept);
+      P.pair_slot[out] = make_int2(i - slot_base, slot1 - slot_base);
     }
     k += __popc(mask);
   }
-  if (pass == 0 && lane == 0) cnt[t] = k;
+  if (pass == 0 && lane == 0) P.cnt_t[t] = k;
 }
 
-// Block-wide ordered compaction helper: every thread holds one flag; returns the number of set flags
-// before this thread in the block (ascending thread order) and sets *total to the block's count.
-// blockDim.x is a multiple of 32, at most 1024; `warps` is shared scratch of 32 ints.
-__device__ __forceinline__ int block_rank(bool flag, int* warps, int* total) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const unsigned m = __ballot_sync(0xffffffffu, flag);
-  if (lane == 0) warps[w] = __popc(m);
-  __syncthreads();
-  int before = 0, all = 0;
-  for (int k = 0; k < nw; ++k) {
-    before += k < w ? warps[k] : 0;
-    all += warps[k];
-  }
-  __syncthreads();  // warps[] may be rewritten by the next call
-  *total = all;
-  return before + __popc(m & ((1u << lane) - 1u));
-}
-
-// One block per vocabulary chunk c: its work lists and the sizes of its two queue groups.
+// Work lists of vocabulary chunk c and the sizes of its two queue groups; the whole block.
 //  - vt_order: the chunk's vocabulary tiles with a listed tile first (they get dC items), then the
 //    empty ones (no row block lists them: their dC rows hold only onehot and smoothing terms and are
-//    written by dc_fill_empty_kernel); both ascending.
+//    written by bwd_finalize_kernel); both ascending.
 //  - de_list: the row blocks with a listed tile in the chunk (they get dE items), ascending.
 //  - empty_list: the chunk's empty tiles, appended to one list for the whole vocabulary.
 //  - grp_size: pairs(c) and dE/dC(c), at their places in the queue order pairs(0), then pairs(c) and
 //    dE/dC(c - 1) for c = 1 .. n-1, then dE/dC(n - 1): pairs(c) is group 2c - 1 (0 for c = 0) and
 //    dE/dC(c) group min(2c + 2, 2n - 1).
-__global__ void chunk_items_kernel(const int* __restrict__ offsets_t, const int2* __restrict__ rb_range,
-                                   const int* __restrict__ pstart_t, int nt, int chunk_vt, int nb, int S,
-                                   int nchunks, int* __restrict__ chunk_t, int* __restrict__ vt_order,
-                                   int* __restrict__ ndc, int* __restrict__ de_list, int* __restrict__ nde,
-                                   int* __restrict__ empty_list, int* __restrict__ n_empty,
-                                   int* __restrict__ grp_size) {
-  __shared__ int warps[32];
+__device__ void chunk_items_block(const PlanArgs& A, int c) {
   __shared__ int em_base;
-  const int c = blockIdx.x;
-  const int t0 = min(nt, c * chunk_vt), t1 = min(nt, (c + 1) * chunk_vt);
+  const BwdPlan& P = A.P;
+  const int nt = P.nt, nb = P.nb, nchunks = P.nchunks;
+  const int t0 = min(nt, c * P.chunk_vt), t1 = min(nt, (c + 1) * P.chunk_vt);
   if (threadIdx.x == 0) {
-    chunk_t[c] = t0;
-    if (c == nchunks - 1) chunk_t[nchunks] = t1;
+    P.chunk_t[c] = t0;
+    if (c == nchunks - 1) P.chunk_t[nchunks] = t1;
   }
-  // vocabulary tiles: count the listed ones first, so that the empty ones can follow them
   int n_listed = 0;
   for (int base = t0; base < t1; base += blockDim.x) {
     const int t = base + threadIdx.x;
-    const bool on = t < t1 && offsets_t[t + 1] > offsets_t[t];
+    const bool on = t < t1 && P.offsets_t[t + 1] > P.offsets_t[t];
     int total;
-    const int pos = block_rank(on, warps, &total);
-    if (on) vt_order[t0 + n_listed + pos] = t;
+    const int pos = block_rank(on, &total);
+    if (on) P.vt_order[t0 + n_listed + pos] = t;
     n_listed += total;
   }
   const int n_em = (t1 - t0) - n_listed;
-  if (threadIdx.x == 0) em_base = n_em > 0 ? atomicAdd(n_empty, n_em) : 0;
+  if (threadIdx.x == 0) em_base = n_em > 0 ? atomicAdd(P.n_empty, n_em) : 0;
   __syncthreads();
   int n_seen = 0;
   for (int base = t0; base < t1; base += blockDim.x) {
     const int t = base + threadIdx.x;
-    const bool em = t < t1 && offsets_t[t + 1] == offsets_t[t];
+    const bool em = t < t1 && P.offsets_t[t + 1] == P.offsets_t[t];
     int total;
-    const int pos = block_rank(em, warps, &total);
+    const int pos = block_rank(em, &total);
     if (em) {
-      vt_order[t0 + n_listed + n_seen + pos] = t;
-      empty_list[em_base + n_seen + pos] = t;
+      P.vt_order[t0 + n_listed + n_seen + pos] = t;
+      P.empty_list[em_base + n_seen + pos] = t;
     }
     n_seen += total;
   }
-  // row blocks with a listed tile in the chunk
   int n_rb = 0;
   for (int base = 0; base < nb; base += blockDim.x) {
     const int b = base + threadIdx.x;
     bool on = false;
     if (b < nb) {
-      const int2 r = rb_range[static_cast<int64_t>(c) * nb + b];
+      const int2 r = P.rb_range[static_cast<int64_t>(c) * nb + b];
       on = r.x < r.y;
     }
     int total;
-    const int pos = block_rank(on, warps, &total);
-    if (on) de_list[static_cast<int64_t>(c) * nb + n_rb + pos] = b;
+    const int pos = block_rank(on, &total);
+    if (on) P.de_list[static_cast<int64_t>(c) * nb + n_rb + pos] = b;
     n_rb += total;
   }
   if (threadIdx.x == 0) {
-    ndc[c] = n_listed;
-    nde[c] = n_rb;
-    grp_size[c == 0 ? 0 : 2 * c - 1] = pstart_t[t1] - pstart_t[t0];
-    grp_size[min(2 * c + 2, 2 * nchunks - 1)] = (n_rb + n_listed) * S;
+    P.ndc[c] = n_listed;
+    P.nde[c] = n_rb;
+    P.grp_size[c == 0 ? 0 : 2 * c - 1] = P.pstart_t[t1] - P.pstart_t[t0];
+    P.grp_size[min(2 * c + 2, 2 * nchunks - 1)] = (n_rb + n_listed) * P.S;
+  }
+  __syncthreads();  // em_base is reused by the block's next chunk
+}
+
+// The whole plan. Phases (each spread over the grid; a barrier after each):
+//  0  zero the counters and the fp32 accumulators of dE and dbias; the row scales
+//  1  tile flags
+//  2  per vocabulary tile: ranks of its listed tiles and their count; per row block: its count; the
+//     kept total; per vocabulary tile: rows whose target tile is onehot only, and their dbias terms
+//  3  scans: offsets_t, offsets_b, oh_off (three blocks)
+//  4  entries_t; row lists (entries_b, pos_b); the onehot-only rows, grouped by vocabulary tile
+//  5  row ranges per chunk
+//  6  pair counts per vocabulary tile
+//  7  scan of the pair counts (pstart_t)
+//  8  pairs; chunk work lists and queue group sizes
+//  9  scan of the group sizes (grp_start); the skipped count
+__global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_constant__ PlanArgs A) {
+  const BwdPlan& P = A.P;
+  const int nb = P.nb, nt = P.nt;
+  const int64_t tiles = static_cast<int64_t>(nb) * nt;
+  const int64_t gthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int gwarps = static_cast<int>(gthreads >> 5), gwarp = static_cast<int>(gtid >> 5), lane = threadIdx.x & 31;
+  const PlanCtl ctl{A.bar, A.err, A.timeout_ns};
+  int round = 0;
+
+  // 0
+  if (gtid < 2) P.kept_total[gtid] = 0;  // kept_total and n_empty
+  for (int64_t i = gtid; i < nb; i += gthreads) P.cnt_b[i] = 0;
+  for (int64_t i = gtid; i < nt; i += gthreads) {
+    P.oh_cnt[i] = 0;
+    P.oh_cur[i] = 0;
+  }
+  {
+    float4* z = reinterpret_cast<float4*>(A.dE_acc);
+    const int64_t n4 = A.N * A.D / 4;  // D is a multiple of 8
+    for (int64_t i = gtid; i < n4; i += gthreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (A.dbias_acc != nullptr)
+      for (int64_t i = gtid; i < A.V; i += gthreads) A.dbias_acc[i] = 0.f;
+  }
+  for (int64_t r = gtid; r < A.N; r += gthreads) {
+    float s;
+    if (A.reduction == 1) {
+      const long long c = *A.count;
+      s = A.grad_out[0] / static_cast<float>(c > 0 ? c : 1);
+    } else if (A.reduction == 2) {
+      s = A.grad_out[0];
+    } else {
+      s = A.grad_out[r];
+    }
+    A.scale[r] = A.targets[r] != A.ignore_index ? s : 0.f;
+  }
+  if (!grid_barrier(ctl, ++round)) return;
+
+  // 1
+  {
+    const int runs = (nt + kFlagTiles - 1) / kFlagTiles;
+    const int64_t units = static_cast<int64_t>(nb) * runs;
+    const int group = threadIdx.x / kBwdBM;
+    for (int64_t u0 = static_cast<int64_t>(blockIdx.x) * kFlagGroups; u0 < units;
+         u0 += static_cast<int64_t>(gridDim.x) * kFlagGroups) {
+      const int64_t u = u0 + group;
+      if (u < units) tile_flags_unit(A, group, static_cast<int>(u / runs), static_cast<int>(u % runs) * kFlagTiles);
+    }
+  }
+  if (!grid_barrier(ctl, ++round)) return;
+
+  // 2
+  for (int t = gwarp; t < nt; t += gwarps) {
+    int listed = 0;
+    for (int b0 = 0; b0 < nb; b0 += 32) {
+      const int b = b0 + lane;
+      const uint8_t f = b < nb ? P.flags[static_cast<int64_t>(b) * nt + t] : 0;
+      const unsigned on = __ballot_sync(0xffffffffu, f == 1);
+      if (f == 1) {
+        P.rank[static_cast<int64_t>(b) * nt + t] = listed + __popc(on & ((1u << lane) - 1u));
+        atomicAdd(P.cnt_b + b, 1);
+      }
+      listed += __popc(on);
+    }
+    if (lane == 0) {
+      P.cnt_t[t] = listed;
+      atomicAdd(P.kept_total, listed);
+    }
+  }
+  for (int64_t r = gtid; r < A.N; r += gthreads) {
+    const int64_t tr = A.targets[r] - A.vs;  // only targets inside this shard have an onehot term here
+    if (!valid_target(tr, A.V, A.ignore_index - A.vs)) continue;
+    const int t = static_cast<int>(tr / kBwdBN);
+    if (P.flags[(r / kBwdBM) * nt + t] != 2) continue;
+    atomicAdd(P.oh_cnt + t, 1);
+    if (A.dbias_acc != nullptr) atomicAdd(A.dbias_acc + tr, -A.onehot_coef * A.scale[r]);
+  }
+  if (!grid_barrier(ctl, ++round)) return;
+
+  // 3
+  if (blockIdx.x == 0) block_scan(P.cnt_t, nt, P.offsets_t);
+  if (blockIdx.x == 1 % gridDim.x) block_scan(P.cnt_b, nb, P.offsets_b);
+  if (blockIdx.x == 2 % gridDim.x) block_scan(P.oh_cnt, nt, P.oh_off);
+  if (!grid_barrier(ctl, ++round)) return;
+
+  // 4
+  for (int64_t i = gtid; i < tiles; i += gthreads) {
+    if (P.flags[i] != 1) continue;
+    const int b = static_cast<int>(i / nt), t = static_cast<int>(i % nt);
+    P.entries_t[P.offsets_t[t] + P.rank[i]] = make_int2(b * 4 + 1, t);
+  }
+  for (int b = blockIdx.x; b < nb; b += gridDim.x) row_list_block(A, b);
+  for (int64_t r = gtid; r < A.N; r += gthreads) {
+    const int64_t tr = A.targets[r] - A.vs;
+    if (!valid_target(tr, A.V, A.ignore_index - A.vs)) continue;
+    const int t = static_cast<int>(tr / kBwdBN);
+    if (P.flags[(r / kBwdBM) * nt + t] != 2) continue;
+    P.oh_rows[P.oh_off[t] + atomicAdd(P.oh_cur + t, 1)] = static_cast<int>(r);
+  }
+  if (!grid_barrier(ctl, ++round)) return;
+
+  // 5
+  for (int64_t cb = gtid; cb < static_cast<int64_t>(nb) * P.nchunks; cb += gthreads) {
+    const int c = static_cast<int>(cb / nb), b = static_cast<int>(cb % nb);
+    const int lo = lower_bound_t(P.entries_b, P.offsets_b[b], P.offsets_b[b + 1], min(nt, c * P.chunk_vt));
+    const int hi = lower_bound_t(P.entries_b, lo, P.offsets_b[b + 1], min(nt, (c + 1) * P.chunk_vt));
+    P.rb_range[cb] = make_int2(lo, hi);
+  }
+  if (!grid_barrier(ctl, ++round)) return;
+
+  // 6
+  for (int t = gwarp; t < nt; t += gwarps) pair_list_warp(A, t, lane, 0);
+  if (!grid_barrier(ctl, ++round)) return;
+
+  // 7
+  if (blockIdx.x == 0) block_scan(P.cnt_t, nt, P.pstart_t);
+  if (!grid_barrier(ctl, ++round)) return;
+
+  // 8
+  for (int t = gwarp; t < nt; t += gwarps) pair_list_warp(A, t, lane, 1);
+  for (int c = blockIdx.x; c < P.nchunks; c += gridDim.x) chunk_items_block(A, c);
+  if (!grid_barrier(ctl, ++round)) return;
+
+  // 9
+  if (blockIdx.x == 0) {
+    block_scan(P.grp_size, 2 * P.nchunks, P.grp_start);
+    if (threadIdx.x == 0) *A.filtered_tiles = tiles - static_cast<int64_t>(*P.kept_total);
   }
 }
 
-// dC rows of the vocabulary tiles that no row block lists. Every logit of such a tile is skipped,
-// so only the target part of the logit gradient reaches them (Loss functions explainer, "How it
-// works" items 2 and 3): -scale_r (1 - ls) E_r for each row r whose target v lies there, and the
-// smoothing term dc_coef * dc_add shared by every row of dC. No tensor core is involved: a work unit
-// is 4 vocabulary rows x 512 columns, one thread per 8 columns, 16-byte loads and stores along a
-// row. The target rows of tile t are oh_rows[oh_off[t] .. oh_off[t + 1]) (for an empty tile every
-// non-ignored row targeting it is listed there), scanned in order, so the result is deterministic.
-constexpr int kFillCols = 512;
+// The backward's last launch, after the tensor-core kernel: every element-wise step left, in one
+// persistent kernel whose blocks take work units in turn (256 threads; 64 threads x 8 columns cover
+// 512 columns of a row, 16-byte loads and stores, four rows at a time):
+//  A. dE, 32 rows x 512 columns per unit: dE_acc plus, for a row whose target tile was skipped
+//     ("onehot only"), its onehot term -scale_r (1 - ls) C_{t_r}, and with label smoothing the rank-one
+//     term -scale_r (ls / V) sum_v C_v; written as bf16 (or in place in fp32).
+//  B. dC rows of the vocabulary tiles no row block lists, 128 rows x 512 columns per unit. Every
+//     logit of such a tile is skipped, so only the target part of the logit gradient reaches them
+//     (Loss functions explainer, "How it works" items 2 and 3): -scale_r (1 - ls) E_r for each row r
+//     whose target v lies there, and the smoothing term dc_coef * wsum shared by every row of dC. The
+//     target rows (oh_rows[oh_off[t] .. oh_off[t + 1]): for an empty tile every non-ignored row
+//     targeting it is listed there) are staged in shared memory and scanned in list order, so the
+//     result is deterministic.
+//  C. dbias, 2048 entries per unit: dbias_acc (the G column sums and the onehot terms) plus the
+//     smoothing constant, written as bf16 (or in place in fp32).
+constexpr int kFinCols = 512;
+constexpr int kFinList = 256;  // target rows staged per B unit; longer lists are read from global memory
+constexpr int kFinRowsA = 32;
+constexpr int kFinBias = 2048;
 
-__global__ void __launch_bounds__(256, 4) dc_fill_empty_kernel(
-    const int* __restrict__ empty_list, const int* __restrict__ n_empty, const int* __restrict__ oh_off,
-    const int* __restrict__ oh_rows, const int64_t* __restrict__ targets, int64_t vs, const float* __restrict__ scale,
-    float onehot_coef, const __nv_bfloat16* __restrict__ E, int64_t D, int64_t V, const float* __restrict__ dc_add,
-    float dc_coef, void* __restrict__ dC, int out_bf16) {
-  const int col_chunks = static_cast<int>((D + kFillCols - 1) / kFillCols);
-  const int units_per_tile = (kBwdBN / 4) * col_chunks;
-  const int64_t units = static_cast<int64_t>(*n_empty) * units_per_tile;
-  const int row_in_unit = threadIdx.x >> 6;  // 4 rows of 64 threads
+__global__ void __launch_bounds__(256, 2) bwd_finalize_kernel(const __grid_constant__ BwdFinalize F) {
+  __shared__ int s_row[kFinList];
+  __shared__ int s_r[kFinList];
+  __shared__ float s_a[kFinList];
+  const int64_t D = F.D;
+  const int col_chunks = static_cast<int>((D + kFinCols - 1) / kFinCols);
+  const int64_t units_a = (F.N + kFinRowsA - 1) / kFinRowsA * col_chunks;
+  const int64_t units_b = static_cast<int64_t>(*F.n_empty) * col_chunks;
+  const int64_t units_c = F.dbias_acc != nullptr ? (F.V + kFinBias - 1) / kFinBias : 0;
+  const int row0 = threadIdx.x >> 6;
   const int col_thread = (threadIdx.x & 63) * 8;
-  for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
-    const int e = static_cast<int>(u / units_per_tile);
-    const int rem = static_cast<int>(u % units_per_tile);
-    const int t = empty_list[e];
-    const int row = (rem / col_chunks) * 4 + row_in_unit;
-    const int64_t v = static_cast<int64_t>(t) * kBwdBN + row;
-    const int64_t d = static_cast<int64_t>(rem % col_chunks) * kFillCols + col_thread;
-    if (v >= V || d >= D) continue;
-    float acc[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) acc[k] = dc_add != nullptr ? dc_coef * dc_add[d + k] : 0.f;
-    const int i1 = oh_off[t + 1];
-    for (int i = oh_off[t]; i < i1; ++i) {
-      const int r = oh_rows[i];
-      if (targets[r] - vs != v) continue;
-      const float a = -scale[r] * onehot_coef;
-      const uint4 q = ld_global_nc_v4(E + static_cast<int64_t>(r) * D + d);
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        __nv_bfloat162 h;
-        *reinterpret_cast<uint32_t*>(&h) = w[k];
-        acc[2 * k] = fmaf(a, __low2float(h), acc[2 * k]);
-        acc[2 * k + 1] = fmaf(a, __high2float(h), acc[2 * k + 1]);
-      }
-    }
-    if (out_bf16) {
+  auto store8 = [&](void* base, int bf16, int64_t idx, const float (&acc)[8]) {
+    if (bf16) {
       uint4 o;
       o.x = pack_bf16x2(acc[0], acc[1]);
       o.y = pack_bf16x2(acc[2], acc[3]);
       o.z = pack_bf16x2(acc[4], acc[5]);
       o.w = pack_bf16x2(acc[6], acc[7]);
-      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dC) + v * D + d) = o;
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + idx) = o;
     } else {
-      float4* out = reinterpret_cast<float4*>(static_cast<float*>(dC) + v * D + d);
+      float4* out = reinterpret_cast<float4*>(static_cast<float*>(base) + idx);
       out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
       out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
-  }
-}
-
-// Rows whose target tile is onehot only: counted (pass 0) or written (pass 1, positions from the
-// scanned counts and a per-tile cursor) per vocabulary tile of the target.
-__global__ void onehot_rows_kernel(const uint8_t* __restrict__ flags, const int64_t* __restrict__ targets,
-                                   int64_t N, int64_t V, int64_t vs, int64_t ignore_index, int nt,
-                                   int* __restrict__ cnt, const int* __restrict__ off, int* __restrict__ rows,
-                                   int pass) {
-  for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < N;
-       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t tr = targets[r] - vs;  // only targets inside this shard have an onehot term here
-    if (!valid_target(tr, V, ignore_index - vs)) continue;
-    const int t = static_cast<int>(tr / kBwdBN);
-    if (flags[(r / kBwdBM) * nt + t] != 2) continue;
-    const int k = atomicAdd(cnt + t, 1);
-    if (pass == 1) rows[off[t] + k] = static_cast<int>(r);
+  };
+  auto add_bf16x8 = [&](float (&acc)[8], const __nv_bfloat16* src, float a) {
+    const uint4 q = ld_global_nc_v4(src);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      __nv_bfloat162 h;
+      *reinterpret_cast<uint32_t*>(&h) = w[k];
+      acc[2 * k] = fmaf(a, __low2float(h), acc[2 * k]);
+      acc[2 * k + 1] = fmaf(a, __high2float(h), acc[2 * k + 1]);
+    }
+  };
+  for (int64_t u = blockIdx.x; u < units_a + units_b + units_c; u += gridDim.x) {
+    if (u < units_a) {  // A: dE rows
+      const int64_t d = (u % col_chunks) * kFinCols + col_thread;
+      if (d >= D) continue;
+      float cs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (F.csum != nullptr) {
+        const float4 c0 = *reinterpret_cast<const float4*>(F.csum + d);
+        const float4 c1 = *reinterpret_cast<const float4*>(F.csum + d + 4);
+        cs[0] = c0.x; cs[1] = c0.y; cs[2] = c0.z; cs[3] = c0.w;
+        cs[4] = c1.x; cs[5] = c1.y; cs[6] = c1.z; cs[7] = c1.w;
+      }
+      const int64_t rbase = (u / col_chunks) * kFinRowsA;
+      for (int i = row0; i < kFinRowsA; i += 4) {
+        const int64_t r = rbase + i;
+        if (r >= F.N) break;
+        const float* src = F.dE_acc + r * D + d;
+        const float4 a0 = *reinterpret_cast<const float4*>(src);
+        const float4 a1 = *reinterpret_cast<const float4*>(src + 4);
+        float acc[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float sc = F.scale[r];
+        if (F.csum != nullptr) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] = fmaf(-F.ls_v * sc, cs[k], acc[k]);
+        }
+        const int64_t tl = F.targets[r] - F.vs;
+        if (tl >= 0 && tl < F.V && F.targets[r] != F.ignore_index &&
+            F.flags[(r / kBwdBM) * F.nt + tl / kBwdBN] == 2)
+          add_bf16x8(acc, F.C + tl * D + d, -F.onehot_coef * sc);
+        store8(F.dE_out != nullptr ? F.dE_out : static_cast<void*>(F.dE_acc), F.dE_out != nullptr, r * D + d, acc);
+      }
+    } else if (u < units_a + units_b) {  // B: dC rows of an empty vocabulary tile
+      const int64_t ub = u - units_a;
+      const int t = F.empty_list[ub / col_chunks];
+      const int64_t d = (ub % col_chunks) * kFinCols + col_thread;
+      const int i0 = F.oh_off[t], i1 = F.oh_off[t + 1];
+      const bool staged = i1 - i0 <= kFinList;
+      __syncthreads();  // the previous B unit is done with the staged rows
+      if (staged) {
+        for (int i = threadIdx.x; i < i1 - i0; i += blockDim.x) {
+          const int r = F.oh_rows[i0 + i];
+          s_r[i] = r;
+          s_row[i] = static_cast<int>(F.targets[r] - F.vs - static_cast<int64_t>(t) * kBwdBN);
+          s_a[i] = -F.scale[r] * F.onehot_coef;
+        }
+      }
+      __syncthreads();
+      if (d >= D) continue;
+      float base[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) base[k] = F.wsum != nullptr ? -F.ls_v * F.wsum[d + k] : 0.f;
+      for (int row = row0; row < kBwdBN; row += 4) {
+        const int64_t v = static_cast<int64_t>(t) * kBwdBN + row;
+        if (v >= F.V) break;
+        float acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = base[k];
+        if (staged) {
+          for (int i = 0; i < i1 - i0; ++i)
+            if (s_row[i] == row) add_bf16x8(acc, F.E + static_cast<int64_t>(s_r[i]) * D + d, s_a[i]);
+        } else {
+          for (int i = i0; i < i1; ++i) {
+            const int r = F.oh_rows[i];
+            if (F.targets[r] - F.vs == v) add_bf16x8(acc, F.E + static_cast<int64_t>(r) * D + d,
+                                                     -F.scale[r] * F.onehot_coef);
+          }
+        }
+        store8(F.dC, F.dc_bf16, v * D + d, acc);
+      }
+    } else {  // C: dbias
+      const int64_t v0 = (u - units_a - units_b) * kFinBias;
+      const float add = F.wsum != nullptr ? -F.ls_v * F.wsum[D] : 0.f;
+      for (int64_t v = v0 + threadIdx.x; v < v0 + kFinBias && v < F.V; v += blockDim.x) {
+        const float x = F.dbias_acc[v] + add;
+        if (F.dbias_out != nullptr) static_cast<__nv_bfloat16*>(F.dbias_out)[v] = __float2bfloat16_rn(x);
+        else F.dbias_acc[v] = x;
+      }
+    }
   }
 }
 
@@ -413,19 +596,11 @@ __global__ void skip_map_kernel(const uint8_t* __restrict__ flags, int64_t n, ui
     out[i] = flags[i] == 1 ? 0 : 1;
 }
 
-__global__ void plan_finish_kernel(const int* __restrict__ kept_total, int64_t total, int64_t* __restrict__ filtered) {
-  *filtered = total - static_cast<int64_t>(*kept_total);
-}
-
 }  // namespace
 
-cudaError_t launch_dc_fill_empty(const BwdPlan& P, const int64_t* targets, int64_t vs, const float* scale,
-                                 float onehot_coef, const __nv_bfloat16* E, int64_t D, int64_t V, const float* dc_add,
-                                 float dc_coef, void* dC, int out_bf16, int num_sms, cudaStream_t s) {
-  if (P.nb == 0) return cudaSuccess;
-  // persistent: the number of empty tiles is known on the device only
-  dc_fill_empty_kernel<<<num_sms * 8, 256, 0, s>>>(P.empty_list, P.n_empty, P.oh_off, P.oh_rows, targets, vs,
-                                                   scale, onehot_coef, E, D, V, dc_add, dc_coef, dC, out_bf16);
+cudaError_t launch_bwd_finalize(const BwdFinalize& F, int num_sms, cudaStream_t s) {
+  if (F.N == 0) return cudaSuccess;
+  bwd_finalize_kernel<<<num_sms * 4, 256, 0, s>>>(F);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -437,77 +612,17 @@ cudaError_t launch_skip_map(const uint8_t* flags, int64_t tiles, uint8_t* out, c
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float* lse, const int64_t* targets,
-                            int64_t N, int64_t V, int64_t vs, int64_t vtot, int64_t T, int64_t ignore_index,
-                            float filter_eps, int64_t* filtered_tiles, cudaStream_t s) {
-  const int nb = P.nb, nt = P.nt;
-  const int filter_on = filter_eps > 0.f ? 1 : 0;
-  const float ln_eps = filter_on ? logf(filter_eps) : -INFINITY;
-  cudaError_t e = cudaMemsetAsync(P.kept_total, 0, 2 * sizeof(int), s);  // kept_total and n_empty
+cudaError_t launch_bwd_plan(const PlanArgs& A, int num_sms, cudaStream_t s) {
+  if (A.P.nb == 0) return cudaSuccess;
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_kernel, kPlanThreads, 0);
   if (e != cudaSuccess) return e;
-  if (nb > 0) {
-    const int64_t tiles = static_cast<int64_t>(nb) * nt;
-    const int runs = (nt + kFlagTiles - 1) / kFlagTiles;
-    tile_flags_kernel<<<static_cast<unsigned>(static_cast<int64_t>(nb) * runs), kBwdBM, 0, s>>>(
-        tile_max, lse, targets, N, V, vs, vtot, T, ignore_index, ln_eps, filter_on, nt, runs, P.flags);
-    note_launches(1);
-    e = cudaMemsetAsync(P.cnt_b, 0, sizeof(int) * static_cast<size_t>(nb), s);
-    if (e != cudaSuccess) return e;
-    tile_rank_kernel<<<static_cast<int>((static_cast<int64_t>(nt) * 32 + 255) / 256), 256, 0, s>>>(
-        P.flags, nb, nt, P.rank, P.cnt_t, P.cnt_b, P.kept_total);
-    note_launches(1);
-    scan_kernel<<<1, 1024, 0, s>>>(P.cnt_t, nt, P.offsets_t);
-    note_launches(1);
-    fill_col_kernel<<<static_cast<int>((tiles + 255) / 256), 256, 0, s>>>(P.flags, P.rank, P.offsets_t, nb, nt,
-                                                                          P.entries_t);
-    note_launches(1);
-    scan_kernel<<<1, 1024, 0, s>>>(P.cnt_b, nb, P.offsets_b);
-    note_launches(1);
-    row_list_kernel<<<nb, 1024, 0, s>>>(P.flags, P.rank, P.offsets_t, nt, P.offsets_b, P.entries_b, P.pos_b);
-    note_launches(1);
-    const int64_t cbs = static_cast<int64_t>(nb) * P.nchunks;
-    row_range_kernel<<<static_cast<int>(std::min<int64_t>((cbs + 255) / 256, 4096)), 256, 0, s>>>(
-        P.entries_b, P.offsets_b, nb, P.nchunks, nt, P.chunk_vt, P.rb_range);
-    note_launches(1);
-    // the pair counts per vocabulary tile reuse cnt_t (its counts are already scanned into offsets_t)
-    const int grid_t = static_cast<int>((static_cast<int64_t>(nt) * 32 + 255) / 256);
-    pair_list_kernel<<<grid_t, 256, 0, s>>>(P.entries_t, P.offsets_t, P.entries_b, P.pos_b, P.rb_range, P.flags, nb,
-                                            nt, P.chunk_vt, P.cnt_t, P.pstart_t, P.pair_desc, P.pair_slot,
-                                            0);
-    note_launches(1);
-    scan_kernel<<<1, 1024, 0, s>>>(P.cnt_t, nt, P.pstart_t);
-    note_launches(1);
-    pair_list_kernel<<<grid_t, 256, 0, s>>>(P.entries_t, P.offsets_t, P.entries_b, P.pos_b, P.rb_range, P.flags, nb,
-                                            nt, P.chunk_vt, P.cnt_t, P.pstart_t, P.pair_desc, P.pair_slot,
-                                            1);
-    note_launches(1);
-    // (pair_list pass 0 left each vocabulary tile's pair count in cnt_t; chunk_items reads the
-    // listed-tile counts as differences of offsets_t)
-    chunk_items_kernel<<<P.nchunks, 256, 0, s>>>(P.offsets_t, P.rb_range, P.pstart_t, nt, P.chunk_vt, nb, P.S,
-                                                 P.nchunks, P.chunk_t, P.vt_order, P.ndc, P.de_list, P.nde,
-                                                 P.empty_list, P.n_empty, P.grp_size);
-    note_launches(1);
-    scan_kernel<<<1, 1024, 0, s>>>(P.grp_size, 2 * P.nchunks, P.grp_start);
-    note_launches(1);
-  }
-  if (nb > 0) {
-    e = cudaMemsetAsync(P.oh_cnt, 0, sizeof(int) * static_cast<size_t>(nt), s);
-    if (e != cudaSuccess) return e;
-    const int grid_r = static_cast<int>(std::min<int64_t>((N + 255) / 256, 4096));
-    onehot_rows_kernel<<<grid_r, 256, 0, s>>>(P.flags, targets, N, V, vs, ignore_index, nt, P.oh_cnt, P.oh_off,
-                                              P.oh_rows, 0);
-    note_launches(1);
-    scan_kernel<<<1, 1024, 0, s>>>(P.oh_cnt, nt, P.oh_off);
-    note_launches(1);
-    e = cudaMemsetAsync(P.oh_cnt, 0, sizeof(int) * static_cast<size_t>(nt), s);
-    if (e != cudaSuccess) return e;
-    onehot_rows_kernel<<<grid_r, 256, 0, s>>>(P.flags, targets, N, V, vs, ignore_index, nt, P.oh_cnt, P.oh_off,
-                                              P.oh_rows, 1);
-    note_launches(1);
-  }
-  plan_finish_kernel<<<1, 1, 0, s>>>(P.kept_total, static_cast<int64_t>(nb) * nt, filtered_tiles);
+  if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+  void* args[] = {const_cast<PlanArgs*>(&A)};
+  e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(plan_kernel), dim3(num_sms), dim3(kPlanThreads), args,
+                                  0, s);
   note_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace cce

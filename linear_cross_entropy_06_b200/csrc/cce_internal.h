@@ -86,6 +86,7 @@ struct BwdPlan {
   int* empty_list;  // [nt]: the vocabulary tiles no row block lists (their dC rows are filled directly)
   int* n_empty;     // [1], zero before planning
   int* oh_cnt;      // [nt]: rows whose target tile is onehot only, per vocabulary tile (scratch)
+  int* oh_cur;      // [nt]: cursors while those rows are written (scratch)
   int* oh_off;      // [nt + 1]: their prefix sums
   int* oh_rows;     // [N]: those rows, grouped by the vocabulary tile of their target
 };
@@ -141,55 +142,97 @@ struct BwdLaunch {
   int num_sms;
 };
 
-// Targets are ids in [0, vtot); this problem's C holds rows [vs, vs + V).
-cudaError_t launch_bwd_plan(const BwdPlan& P, const float* tile_max, const float* lse, const int64_t* targets,
-                            int64_t N, int64_t V, int64_t vs, int64_t vtot, int64_t T, int64_t ignore_index,
-                            float filter_eps, int64_t* filtered_tiles, cudaStream_t s);
+// Everything the backward's planning launch reads and writes besides the plan itself (cce_bwd_plan.cu).
+struct PlanArgs {
+  BwdPlan P;
+  const float* tile_max;   // [T, N] from the forward
+  const float* lse;        // [N]
+  const int64_t* targets;  // [N] ids in [0, vtot); this problem's C holds rows [vs, vs + V)
+  const int64_t* count;    // [1] non-ignored rows (from the forward)
+  const float* grad_out;   // [1] or [N]
+  int64_t N, D, V, T, vs, vtot, ignore_index;
+  int reduction;
+  int filter_on;
+  float ln_eps;
+  float* scale;            // [N] out: the row scales of the gradient
+  float onehot_coef;       // 1 - label_smoothing
+  float* dE_acc;           // [N, D] fp32, zeroed here
+  float* dbias_acc;        // [V] fp32 or null, zeroed here; receives the onehot-only rows' terms
+  int64_t* filtered_tiles;
+  int* bar;                // grid barrier counter, zero at launch
+  int* err;
+  uint64_t timeout_ns;
+};
+// One cooperative launch: the row scales, the tile flags, both tile lists, the pair list, the
+// chunks' work lists and queue groups, the onehot-only rows, and the skipped count.
+cudaError_t launch_bwd_plan(const PlanArgs& A, int num_sms, cudaStream_t s);
 cudaError_t launch_bwd(const BwdLaunch& L, cudaStream_t s);
-// dC rows of the vocabulary tiles no row block lists (plan.empty_list): dc_coef * dc_add (or 0)
-// plus, for each row r whose target lies there, -scale_r * onehot_coef * E_r. bf16 or fp32 output.
-cudaError_t launch_dc_fill_empty(const BwdPlan& P, const int64_t* targets, int64_t vs, const float* scale,
-                                 float onehot_coef,
-                                 const __nv_bfloat16* E, int64_t D, int64_t V, const float* dc_add, float dc_coef,
-                                 void* dC, int out_bf16, int num_sms, cudaStream_t s);
+// Everything the backward computes after its tensor-core kernel (cce_bwd_plan.cu, one launch): the
+// last terms of dE and its conversion, the dC rows of the vocabulary tiles no row block lists, and
+// dbias. See bwd_finalize_kernel.
+struct BwdFinalize {
+  int64_t N, D, V, vs, ignore_index;
+  int nt;
+  const uint8_t* flags;       // the plan's tile flags [nb * nt]
+  const int* empty_list;
+  const int* n_empty;
+  const int* oh_off;
+  const int* oh_rows;
+  const int64_t* targets;
+  const float* scale;
+  float onehot_coef;          // 1 - label_smoothing
+  float ls_v;                 // label_smoothing / vocab_total
+  const __nv_bfloat16* E;
+  const __nv_bfloat16* C;
+  const float* csum;          // [D] column sums of C (label smoothing) or null
+  const float* wsum;          // [D + 1] sum_r scale_r E_r and sum_r scale_r (label smoothing) or null
+  float* dE_acc;              // [N, D] fp32
+  void* dE_out;               // bf16 [N, D], or null: dE_acc is the output (fp32)
+  void* dC;                   // [V, D]
+  int dc_bf16;
+  float* dbias_acc;           // [V] fp32, or null (no dbias)
+  void* dbias_out;            // bf16 [V], or null: dbias_acc is the output (fp32)
+};
+cudaError_t launch_bwd_finalize(const BwdFinalize& F, int num_sms, cudaStream_t s);
 // out[i] = 1 if tile i of the plan's flags was skipped, 0 if it was kept (i < tiles).
 cudaError_t launch_skip_map(const uint8_t* flags, int64_t tiles, uint8_t* out, cudaStream_t s);
 
 cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
 
 // Small kernels (cce_aux.cu).
-// C holds vocabulary rows [vs, vs + V) of vtot (vs = 0, vtot = V for the whole vocabulary).
-cudaError_t launch_target_logit(const __nv_bfloat16* E, const __nv_bfloat16* C, const __nv_bfloat16* bias,
-                                const int64_t* targets, int64_t N, int64_t D, int64_t V, int64_t vs, int64_t vtot,
-                                int64_t ignore_index, float* z_target, const float* csum, float* z_sum, int* err,
-                                cudaStream_t s);
-// loss_rows may be null (a vocabulary shard): then only lse is written.
-cudaError_t launch_lse_loss(const float* tile_max, const float* tile_sum, const float* z_target, const float* z_sum,
-                            const int64_t* targets, int64_t N, int64_t T, int64_t ignore_index, int64_t V,
-                            float label_smoothing, float z_loss, float* lse, float* loss_rows, cudaStream_t s);
+// Everything the forward computes after its tensor-core kernel (one launch).
+struct FwdFinish {
+  const float* tile_max;  // [T, N]
+  const float* tile_sum;  // [T, N]
+  int64_t N, T, D, V;
+  int64_t vs, vtot;       // C holds vocabulary rows [vs, vs + V) of vtot (0 and V: the whole vocabulary)
+  int64_t ignore_index;
+  const __nv_bfloat16* E;
+  const __nv_bfloat16* C;
+  const __nv_bfloat16* bias;  // [V] or null
+  const int64_t* targets;
+  const float* csum;          // [D + 1] column sums of C and the bias sum (label smoothing), or null
+  float label_smoothing, z_loss;
+  float* lse;                 // [N]
+  float* zt_out;              // vocabulary shard: [N] correct-token logits and [N] logit sums; else null
+  float* zs_out;
+  float* loss;                // [1] or [N] (reduction none); null for a vocabulary shard
+  int reduction;
+  int64_t* count;
+  double* block_sums;         // [ceil(N / kFinishRows)] scratch
+  long long* block_counts;    // [ceil(N / kFinishRows)] scratch
+  int* done;                  // zero at launch
+  int* err;
+};
+constexpr int kFinishRows = 32;  // rows per block of the finish kernel
+cudaError_t launch_fwd_finish(const FwdFinish& F, cudaStream_t s);
 // out[0:D] = sum_r w_r X[r, :] (w_r = 1 when w is null); out[D] = sum_r w_r, or the sum of extra[0:rows].
 cudaError_t launch_weighted_colsum(const __nv_bfloat16* X, int64_t rows, int64_t D, const float* w,
                                    const __nv_bfloat16* extra, float* out, cudaStream_t s);
-// X[r, :] += coef * scale[r] * u (fp32 [rows, D], in place).
-cudaError_t launch_add_rank1(float* X, int64_t rows, int64_t D, const float* scale, float coef, const float* u,
-                             cudaStream_t s);
-// X[0:n] += coef * (*c).
-cudaError_t launch_add_scalar(float* X, int64_t n, float coef, const float* c, cudaStream_t s);
-// The onehot term of rows whose target tile was skipped: dE_acc[r] -= coef scale_r C[t_r] and
-// dbias_acc[t_r] -= coef scale_r (dbias_acc may be null), for the rows listed in rows[0:off[nt]].
-cudaError_t launch_onehot_rows(const int* off, int nt, const int* rows, const int64_t* targets, int64_t vs,
-                               const float* scale, float coef, const __nv_bfloat16* C, int64_t D, float* dE_acc,
-                               float* dbias_acc, int64_t max_rows, cudaStream_t s);
 // LSE over the whole vocabulary, loss, count and reduction from the shards' partial results [shards, 3, N].
 cudaError_t launch_shard_merge(const float* partials, int shards, const int64_t* targets, int64_t N, int64_t V,
                                int64_t ignore_index, float label_smoothing, float z_loss, int reduction, float* loss,
                                float* lse, int64_t* count, cudaStream_t s);
-// Count, reduction and, when *err != 0 (a device error earlier in the call), a NaN loss.
-cudaError_t launch_loss_reduce(const float* loss_rows, const int64_t* targets, int64_t N, int64_t ignore_index,
-                               int reduction, float* loss, int64_t* count, const int* err, cudaStream_t s);
-cudaError_t launch_row_scale(const int64_t* targets, const int64_t* count, const float* grad_out, int64_t N,
-                             int64_t ignore_index, int reduction, float* scale, cudaStream_t s);
-cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, int64_t n, cudaStream_t s);
 cudaError_t launch_fill_zero(void* dst, int64_t bytes, cudaStream_t s);
 
 }  // namespace cce

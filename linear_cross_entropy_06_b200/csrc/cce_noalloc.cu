@@ -105,14 +105,14 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
     return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: a required pointer is NULL");
   if ((reinterpret_cast<uintptr_t>(E) | reinterpret_cast<uintptr_t>(C) | reinterpret_cast<uintptr_t>(bias)) & 15u)
     return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: E, C and bias must be 16-byte aligned");
-  // Same layout as the forward workspace: header | tile_sum [T, N] | z_target [N] | loss_rows [N] |
-  // csum [D + 1] | z_sum [N] (the last two for label smoothing).
+  // Same layout as the forward workspace: header (error word, finish counter) | tile_sum [T, N] |
+  // csum [D + 1] (label smoothing) | per-block loss sums and counts of the finish kernel.
+  const size_t nblk = static_cast<size_t>(N > 0 ? (N + cce::kFinishRows - 1) / cce::kFinishRows : 1);
   const size_t off_sum = kHeader;
-  const size_t off_zt = up(off_sum + sizeof(float) * static_cast<size_t>(T * N));
-  const size_t off_rows = up(off_zt + sizeof(float) * static_cast<size_t>(N));
-  const size_t off_csum = up(off_rows + sizeof(float) * static_cast<size_t>(N));
-  const size_t off_zsum = up(off_csum + sizeof(float) * static_cast<size_t>(D + 1));
-  const size_t need = up(off_zsum + sizeof(float) * static_cast<size_t>(N));
+  const size_t off_csum = up(off_sum + sizeof(float) * static_cast<size_t>(T * N));
+  const size_t off_bsum = up(off_csum + sizeof(float) * static_cast<size_t>(D + 1));
+  const size_t off_bcnt = up(off_bsum + sizeof(double) * nblk);
+  const size_t need = up(off_bcnt + sizeof(long long) * nblk);
   if (need > kNoAllocScratchBytes) {
     char msg[256];
     snprintf(msg, sizeof(msg),
@@ -127,19 +127,16 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   if (st != CCE_OK) return st;
   char* b = static_cast<char*>(base);
   int* err = reinterpret_cast<int*>(b);
+  int* done = err + 1;
   float* tile_sum = reinterpret_cast<float*>(b + off_sum);
-  float* z_target = reinterpret_cast<float*>(b + off_zt);
-  float* loss_rows = reinterpret_cast<float*>(b + off_rows);
   float* csum = reinterpret_cast<float*>(b + off_csum);
-  float* z_sum = reinterpret_cast<float*>(b + off_zsum);
   const bool smooth = p->label_smoothing > 0.f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const auto* Eb = static_cast<const __nv_bfloat16*>(E);
   const auto* Cb = static_cast<const __nv_bfloat16*>(C);
   const auto* Bb = static_cast<const __nv_bfloat16*>(bias);
 
-  // The array keeps the previous call's contents: the error word must start at zero; every other
-  // scratch value is written before it is read.
+  // The array keeps the previous call's contents: the error word and the finish kernel's counter must
+  // start at zero; every other scratch value is written before it is read.
   if (cudaMemsetAsync(err, 0, kHeader, s) != cudaSuccess) return fail(CCE_ERR_CUDA, "cce_forward_noalloc: memset");
   if (N > 0) {
     cce::FwdLaunch L{};
@@ -157,17 +154,34 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
     L.inject_stall = 0;
     L.bias = Bb;
     if ((smooth && cce::launch_weighted_colsum(Cb, V, D, nullptr, Bb, csum, s) != cudaSuccess) ||
-        cce::launch_target_logit(Eb, Cb, Bb, targets, N, D, V, 0, V, p->ignore_index, z_target,
-                                 smooth ? csum : nullptr,
-                                 smooth ? z_sum : nullptr, err, s) != cudaSuccess ||
-        cce::launch_fwd_lse(L, s) != cudaSuccess ||
-        cce::launch_lse_loss(tile_max, tile_sum, z_target, smooth ? z_sum : nullptr, targets, N, T, p->ignore_index,
-                             V, p->label_smoothing, p->z_loss, lse,
-                             p->reduction == CCE_REDUCTION_NONE ? loss : loss_rows, s) != cudaSuccess)
+        cce::launch_fwd_lse(L, s) != cudaSuccess)
       return fail(CCE_ERR_CUDA, "cce_forward_noalloc: kernel launch failed");
   }
-  if (cce::launch_loss_reduce(loss_rows, targets, N, p->ignore_index, p->reduction, loss, count, err, s) !=
-      cudaSuccess)
-    return fail(CCE_ERR_CUDA, "cce_forward_noalloc: kernel launch failed");
+  cce::FwdFinish F{};
+  F.tile_max = tile_max;
+  F.tile_sum = tile_sum;
+  F.N = N;
+  F.T = T;
+  F.D = D;
+  F.V = V;
+  F.vs = 0;
+  F.vtot = V;
+  F.ignore_index = p->ignore_index;
+  F.E = static_cast<const __nv_bfloat16*>(E);
+  F.C = Cb;
+  F.bias = Bb;
+  F.targets = targets;
+  F.csum = smooth ? csum : nullptr;
+  F.label_smoothing = p->label_smoothing;
+  F.z_loss = p->z_loss;
+  F.lse = lse;
+  F.loss = loss;
+  F.reduction = p->reduction;
+  F.count = count;
+  F.block_sums = reinterpret_cast<double*>(b + off_bsum);
+  F.block_counts = reinterpret_cast<long long*>(b + off_bcnt);
+  F.done = done;
+  F.err = err;
+  if (cce::launch_fwd_finish(F, s) != cudaSuccess) return fail(CCE_ERR_CUDA, "cce_forward_noalloc: kernel launch failed");
   return CCE_OK;
 }
