@@ -642,7 +642,8 @@ cce_status cce_forward_merge(const cce_problem* p, const float* partials, int32_
   if (!problem_ok(p, true)) return CCE_ERR_INVALID_ARG;
   if (sharded(p)) return fail(CCE_ERR_INVALID_ARG, "cce_forward_merge takes the whole problem, not a shard");
   if (shards < 1) return fail(CCE_ERR_INVALID_ARG, "shards must be >= 1");
-  if (loss == nullptr || count == nullptr || (p->N > 0 && (partials == nullptr || targets == nullptr || lse == nullptr)))
+  if (loss == nullptr || count == nullptr ||
+      (p->N > 0 && (partials == nullptr || targets == nullptr || lse == nullptr)))
     return fail(CCE_ERR_INVALID_ARG, "a required pointer is NULL");
   int num_sms = 0;
   CCE_CHECK(check_device(&num_sms));

@@ -60,7 +60,8 @@ cce_status scratch_for_current_device(void** out, int* num_sms) {
   if (g_scratch_addr[dev] == nullptr) {
     void* ptr = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess || ptr == nullptr) return fail(CCE_ERR_CUDA, "cce_forward_noalloc: cudaGetSymbolAddress failed");
+    if (e != cudaSuccess || ptr == nullptr)
+      return fail(CCE_ERR_CUDA, "cce_forward_noalloc: cudaGetSymbolAddress failed");
     g_scratch_addr[dev] = ptr;
   }
   if (g_encode_fn == nullptr) {
@@ -96,7 +97,8 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   if (p == nullptr || p->N < 0 || p->D < 8 || p->D % 8 != 0 || p->V < 1 || p->reduction < 0 || p->reduction > 2 ||
       p->reserved != 0 || p->N >= (int64_t(1) << 31) - 256 || p->V >= (int64_t(1) << 31) - 256 ||
       p->D >= (int64_t(1) << 24) || !(p->label_smoothing >= 0.f && p->label_smoothing <= 1.f) ||
-      !(p->z_loss >= 0.f && p->z_loss < INFINITY) || p->vocab_start != 0 || (p->vocab_total != 0 && p->vocab_total != p->V))
+      !(p->z_loss >= 0.f && p->z_loss < INFINITY) || p->vocab_start != 0 ||
+      (p->vocab_total != 0 && p->vocab_total != p->V))
     return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: invalid problem (or a vocabulary shard)");
   const int64_t N = p->N, D = p->D, V = p->V;
   const int64_t T = (V + cce::kSubTile - 1) / cce::kSubTile;
@@ -182,6 +184,7 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   F.block_counts = reinterpret_cast<long long*>(b + off_bcnt);
   F.done = done;
   F.err = err;
-  if (cce::launch_fwd_finish(F, s) != cudaSuccess) return fail(CCE_ERR_CUDA, "cce_forward_noalloc: kernel launch failed");
+  if (cce::launch_fwd_finish(F, s) != cudaSuccess)
+    return fail(CCE_ERR_CUDA, "cce_forward_noalloc: kernel launch failed");
   return CCE_OK;
 }

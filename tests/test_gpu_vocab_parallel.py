@@ -93,7 +93,8 @@ def test_vocabulary_shards_match_the_whole_problem(device, shards, variant, redu
 
 def test_shards_agree_with_the_unsharded_path(device):
     """Two shards against cce_forward / cce_backward on the whole classifier: the same loss and LSE up
-    to the merge's rounding, and the same gradients up to the fp32 summation order of dE."""
+    to the merge's rounding, and the same gradients up to the fp32 summation order of dE (the
+    shards' parts are added last)."""
     inp = make_inputs("llama3.1-8b-head", N=512, D=512, V=8192, alpha=12.0, seed=74)
     E, C, t = inp.E.to(device), inp.C.to(device), inp.targets.to(device)
     loss, lse, tmax, count = ops.cce_forward(E, C, t, check=True)
@@ -102,7 +103,7 @@ def test_shards_agree_with_the_unsharded_path(device):
     assert abs(float(r["loss"][0]) - float(loss)) <= 1e-5
     assert np.abs(r["lse"] - lse.double().cpu().numpy()).max() <= 1e-5
     assert r["filtered"] == int(filt.item())
-    assert rel_frob(r["dE"], dE.double().cpu().numpy()) <= 1e-5
+    assert rel_frob(r["dE"], dE.double().cpu().numpy()) <= 1e-4  # fp32 sums of the shards' parts
     assert rel_frob(r["dC"], dC.double().cpu().numpy()) <= 5e-3  # bf16 rounding of the shards' dC
 
 
