@@ -196,6 +196,10 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
       std::max<int64_t>(1, std::min({nt, cce::kChunkCBytes / vt_bytes, budget / cce::kGradBuffers / per_vtile}));
   w.plan.chunk_vt = static_cast<int>(chunk_vt);
   w.plan.nchunks = static_cast<int>(ceil_div(nt, chunk_vt));
+  w.plan.chunk_c_tiles = std::max<int64_t>(1, cce::kChunkCBytes / vt_bytes);
+  w.plan.chunk_g_tiles = static_cast<int64_t>(nb) * chunk_vt;
+  w.plan.nchunks_dev = reinterpret_cast<int*>(take(sizeof(int)));
+  w.plan.chunk_of = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt)));
   w.plan.chunk_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks + 1)));
   w.plan.rb_range = reinterpret_cast<int2*>(take(sizeof(int2) * static_cast<size_t>(w.plan.nchunks) * nb));
   w.plan.pstart_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt + 1)));
@@ -367,7 +371,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.nb = w.plan.nb;
   A.nt = w.plan.nt;
   A.S = w.plan.S;
-  A.nchunks = w.plan.nchunks;
+  A.nchunks = w.plan.nchunks_dev;
   A.out_bf16 = c32 ? 0 : 1;
   A.ignore_index = p->ignore_index;
   A.vocab_start = vs;

@@ -151,8 +151,9 @@ __device__ __forceinline__ int2 group_of(int g, int nchunks) {
 
 // Item w of the queue, in group g that starts at item g_begin -> its decoded form (the scheduler's
 // only global reads).
-__device__ __forceinline__ void decode_item(int w, int g, int g_begin, const BwdArgs& A, WorkItem& it) {
-  const int2 gc = group_of(g, A.nchunks);
+__device__ __forceinline__ void decode_item(int w, int g, int g_begin, int nchunks, const BwdArgs& A,
+                                            WorkItem& it) {
+  const int2 gc = group_of(g, nchunks);
   const int c = gc.x, local = w - g_begin;
   const int t_begin = A.chunk_t[c];
   it.chunk = c;
@@ -264,7 +265,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 6) {
     // ---------------- scheduler ----------------
     if (lane == 0) {
-      const int total = A.grp_start[2 * A.nchunks];
+      const int nchunks = *A.nchunks;
+      const int total = A.grp_start[2 * nchunks];
       int g = 0, g_begin = 0, g_end = A.grp_start[1];  // this CTA's claims only increase
       for (uint32_t k = 0;; ++k) {
         const int idx = static_cast<int>(k % RING);
@@ -283,7 +285,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             g_begin = g_end;
             g_end = A.grp_start[g + 1];
           }
-          decode_item(w, g, g_begin, A, it);
+          decode_item(w, g, g_begin, nchunks, A, it);
         }
         int4* dst = reinterpret_cast<int4*>(ring + idx);
         const int4* src = reinterpret_cast<const int4*>(&it);
@@ -445,6 +447,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t stg = reg0 + static_cast<uint32_t>(q * STG_WARP);
     uint32_t acc_iter = 0, rphase = 0, gphase = 0;
     uint32_t img = 0;  // which of the two 4 KB staging images of this warp comes next
+    bool region_shared = true;  // the last item used the whole region (a pair's G tile)
     bool ok = true;
     // Every lane waits (and acquires) itself; the vote makes the outcome warp-uniform, so the warp
     // stays converged for the .sync.aligned TMEM loads and takes one branch on failure.
@@ -562,6 +565,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         if (*abort_flag) ok = false;
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        region_shared = true;
         continue;
       }
 
@@ -598,7 +602,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ++n;
         }
       }
-      if (!region_free()) break;
+      // After a pair every warp's earlier bulk stores must have read the whole region; between dE / dC
+      // items each warp only reuses its own staging images, which next_image() guards.
+      if (region_shared && !region_free()) break;
+      region_shared = false;
       const int rows_limit = de ? A.N : A.V;
       const int y = it.key * BM + q * 32;
       // the first matched row's 64 columns for the next step are loaded one step ahead
@@ -615,8 +622,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (x >= A.D) break;
         float v0[32], v1[32];
         if (has) {
-          tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * SLICE + 64 * p), v0);
-          tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * SLICE + 64 * p + 32), v1);
+          tmem_ld64(tmem_base + lane_off + static_cast<uint32_t>(a * SLICE + 64 * p), v0, v1);
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) v0[e] = v1[e] = 0.f;

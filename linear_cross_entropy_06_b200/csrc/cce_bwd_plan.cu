@@ -216,8 +216,8 @@ __device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int 
 __device__ void pair_list_warp(const PlanArgs& A, int t, int lane, int pass) {
   const BwdPlan& P = A.P;
   const int nb = P.nb, nt = P.nt;
-  const int c = t / P.chunk_vt;
-  const int slot_base = P.offsets_t[c * P.chunk_vt];
+  const int c = P.chunk_of[t];
+  const int slot_base = P.offsets_t[P.chunk_t[c]];
   const int i0 = P.offsets_t[t], i1 = P.offsets_t[t + 1];
   int k = 0;
   for (int base = i0; base < i1; base += 32) {
@@ -256,15 +256,11 @@ __device__ void pair_list_warp(const PlanArgs& A, int t, int lane, int pass) {
 //  - grp_size: pairs(c) and dE/dC(c), at their places in the queue order pairs(0), then pairs(c) and
 //    dE/dC(c - 1) for c = 1 .. n-1, then dE/dC(n - 1): pairs(c) is group 2c - 1 (0 for c = 0) and
 //    dE/dC(c) group min(2c + 2, 2n - 1).
-__device__ void chunk_items_block(const PlanArgs& A, int c) {
+__device__ void chunk_items_block(const PlanArgs& A, int c, int nchunks) {
   __shared__ int em_base;
   const BwdPlan& P = A.P;
-  const int nt = P.nt, nb = P.nb, nchunks = P.nchunks;
-  const int t0 = min(nt, c * P.chunk_vt), t1 = min(nt, (c + 1) * P.chunk_vt);
-  if (threadIdx.x == 0) {
-    P.chunk_t[c] = t0;
-    if (c == nchunks - 1) P.chunk_t[nchunks] = t1;
-  }
+  const int nb = P.nb;
+  const int t0 = P.chunk_t[c], t1 = P.chunk_t[c + 1];
   int n_listed = 0;
   for (int base = t0; base < t1; base += blockDim.x) {
     const int t = base + threadIdx.x;
@@ -311,14 +307,80 @@ __device__ void chunk_items_block(const PlanArgs& A, int c) {
   __syncthreads();  // em_base is reused by the block's next chunk
 }
 
+// Vocabulary chunks, by the calling block: consecutive vocabulary tiles, each chunk as long as its
+// gradient tiles fit one buffer (at most chunk_g_tiles listed tiles) and the C rows its tiles read
+// stay within kChunkCBytes (at most chunk_c_tiles vocabulary tiles with a listed tile), so that a
+// sparse stretch of the vocabulary forms one long chunk: fewer chunks mean fewer partial sums of dE
+// and longer groups of pairs ahead of each chunk's dE / dC items. A chunk of the fixed length
+// chunk_vt always satisfies both limits, so there are never more than P.nchunks chunks. Greedy
+// over the prefix sums offsets_t, staged in shared memory; thread 0 decides.
+__device__ void chunk_partition(const PlanArgs& A) {
+  __shared__ int off[kPlanThreads + 1];
+  __shared__ int st[4];  // chunk count, first tile, listed tiles before it, non-empty tiles so far
+  const BwdPlan& P = A.P;
+  const int nt = P.nt;
+  if (threadIdx.x == 0) {
+    st[0] = 0;
+    st[1] = 0;
+    st[2] = 0;
+    st[3] = 0;
+    P.chunk_t[0] = 0;
+  }
+  for (int base = 0; base < nt; base += kPlanThreads) {
+    __syncthreads();
+    for (int i = threadIdx.x; i <= kPlanThreads; i += blockDim.x) off[i] = P.offsets_t[min(base + i, nt)];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int n = st[0], first_listed = st[2], nonempty = st[3];
+      for (int i = 0; i < kPlanThreads && base + i < nt; ++i) {
+        const int t = base + i;
+        const int listed = off[i + 1] - off[i];
+        const bool fits = off[i + 1] - first_listed <= P.chunk_g_tiles &&
+                          nonempty + (listed > 0 ? 1 : 0) <= P.chunk_c_tiles;
+        if (!fits && t > st[1]) {  // close the chunk before tile t
+          if (++n < P.nchunks) P.chunk_t[n] = t;  // (more than P.nchunks cannot happen; see below)
+          st[1] = t;
+          first_listed = off[i];
+          nonempty = 0;
+        }
+        nonempty += listed > 0 ? 1 : 0;
+      }
+      st[0] = n;
+      st[2] = first_listed;
+      st[3] = nonempty;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (st[0] + 1 <= P.nchunks) {
+      P.chunk_t[st[0] + 1] = nt;
+      *P.nchunks_dev = st[0] + 1;
+    } else {  // defensive: the fixed partition, which always fits the arrays and the buffers
+      for (int c = 0; c <= P.nchunks; ++c) P.chunk_t[c] = min(nt, c * P.chunk_vt);
+      *P.nchunks_dev = P.nchunks;
+    }
+  }
+}
+
+__device__ __forceinline__ int chunk_containing(const int* chunk_t, int n, int t) {
+  int lo = 0, hi = n;  // chunk_t[lo] <= t < chunk_t[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (chunk_t[mid] <= t) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
 // The whole plan. Phases (each spread over the grid; a barrier after each):
 //  0  zero the counters and the fp32 accumulators of dE and dbias; the row scales
 //  1  tile flags
 //  2  per vocabulary tile: ranks of its listed tiles and their count; per row block: its count; the
 //     kept total; per vocabulary tile: rows whose target tile is onehot only, and their dbias terms
 //  3  scans: offsets_t, offsets_b, oh_off (three blocks)
-//  4  entries_t; row lists (entries_b, pos_b); the onehot-only rows, grouped by vocabulary tile
-//  5  row ranges per chunk
+//  4  entries_t; row lists (entries_b, pos_b); the onehot-only rows, grouped by vocabulary tile;
+//     the vocabulary chunks (one block)
+//  5  row ranges per chunk; the chunk of every vocabulary tile
 //  6  pair counts per vocabulary tile
 //  7  scan of the pair counts (pstart_t)
 //  8  pairs; chunk work lists and queue group sizes
@@ -422,15 +484,19 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     if (P.flags[(r / kBwdBM) * nt + t] != 2) continue;
     P.oh_rows[P.oh_off[t] + atomicAdd(P.oh_cur + t, 1)] = static_cast<int>(r);
   }
+  if (blockIdx.x == gridDim.x - 1) chunk_partition(A);
   if (!grid_barrier(ctl, ++round)) return;
+  const int nchunks = *reinterpret_cast<volatile int*>(P.nchunks_dev);
 
   // 5
-  for (int64_t cb = gtid; cb < static_cast<int64_t>(nb) * P.nchunks; cb += gthreads) {
+  for (int64_t cb = gtid; cb < static_cast<int64_t>(nb) * nchunks; cb += gthreads) {
     const int c = static_cast<int>(cb / nb), b = static_cast<int>(cb % nb);
-    const int lo = lower_bound_t(P.entries_b, P.offsets_b[b], P.offsets_b[b + 1], min(nt, c * P.chunk_vt));
-    const int hi = lower_bound_t(P.entries_b, lo, P.offsets_b[b + 1], min(nt, (c + 1) * P.chunk_vt));
+    const int lo = lower_bound_t(P.entries_b, P.offsets_b[b], P.offsets_b[b + 1], P.chunk_t[c]);
+    const int hi = lower_bound_t(P.entries_b, lo, P.offsets_b[b + 1], P.chunk_t[c + 1]);
     P.rb_range[cb] = make_int2(lo, hi);
   }
+  for (int64_t t = gtid; t < nt; t += gthreads)
+    P.chunk_of[t] = chunk_containing(P.chunk_t, nchunks, static_cast<int>(t));
   if (!grid_barrier(ctl, ++round)) return;
 
   // 6
@@ -443,12 +509,12 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
 
   // 8
   for (int t = gwarp; t < nt; t += gwarps) pair_list_warp(A, t, lane, 1);
-  for (int c = blockIdx.x; c < P.nchunks; c += gridDim.x) chunk_items_block(A, c);
+  for (int c = blockIdx.x; c < nchunks; c += gridDim.x) chunk_items_block(A, c, nchunks);
   if (!grid_barrier(ctl, ++round)) return;
 
   // 9
   if (blockIdx.x == 0) {
-    block_scan(P.grp_size, 2 * P.nchunks, P.grp_start);
+    block_scan(P.grp_size, 2 * nchunks, P.grp_start);
     if (threadIdx.x == 0) *A.filtered_tiles = tiles - static_cast<int64_t>(*P.kept_total);
   }
 }

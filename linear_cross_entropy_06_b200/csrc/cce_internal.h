@@ -68,10 +68,14 @@ struct BwdPlan {
   int2* entries_b;  // [nb * nt]: (t, slot in entries_t), by row block then vocabulary tile
   int* pos_b;       // [nb * nt]: for each entries_t position, the tile's position in entries_b
   int* kept_total;
-  int chunk_vt;     // vocabulary tiles per chunk
-  int nchunks;
+  int chunk_vt;     // vocabulary tiles per chunk at most once every tile is listed (sizes the arrays)
+  int nchunks;      // chunks at most (arrays are sized for it); the plan's own count is *nchunks_dev
+  int* nchunks_dev; // [1]: chunks of this plan
+  int* chunk_of;    // [nt]: chunk of each vocabulary tile
   int S;            // 256-column slices of D
   int* chunk_t;     // [nchunks + 1]: first vocabulary tile of each chunk
+  int64_t chunk_c_tiles;  // vocabulary tiles with a listed tile a chunk may hold (kChunkCBytes of C)
+  int64_t chunk_g_tiles;  // listed tiles a chunk may hold (one gradient-tile buffer)
   int2* rb_range;   // [nchunks * nb]: entries [lo, hi) of each row block inside each chunk
   int* pstart_t;    // [nt + 1]: first pair whose first tile is in vocabulary tile t
   int4* pair_desc;  // [pair capacity]: (b, t0, t1 or -1, kept bits), by t0 then b
@@ -93,7 +97,8 @@ struct BwdPlan {
 
 // Everything the persistent backward kernel reads besides its tensor maps.
 struct BwdArgs {
-  int N, D, V, nb, nt, S, nchunks;
+  int N, D, V, nb, nt, S;
+  const int* nchunks;  // [1] the plan's chunk count
   int out_bf16;
   int64_t ignore_index;
   int64_t vocab_start;  // C holds vocabulary rows [vocab_start, vocab_start + V); targets are global ids
