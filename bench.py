@@ -48,8 +48,14 @@ KERNEL_SOURCES = {
     "bwd_kernel": ("cce_bwd.cu", "cce_device.cuh", "cce_internal.h"),
 }
 TRAFFIC_BYTES = {
-    "fwd_lse_kernel": {},
-    "bwd_kernel": {},
+    "fwd_lse_kernel": {
+        (4096, 4096, 128256): ("d741d132ee5687379de08c2b1994100355a6551833650c05e62176ed204badb1",
+                               1084471296 + 37252864),
+    },
+    "bwd_kernel": {
+        (4096, 4096, 128256): ("3c7e6d9e2249ad598ff936c22ac20055784646526dd6c42c6be3a22ecf1a5fcd",
+                               5942506496 + 2340444672),
+    },
 }
 
 
