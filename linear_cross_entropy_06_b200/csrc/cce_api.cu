@@ -317,9 +317,10 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
     return cudaMemsetAsync(filtered_tiles, 0, sizeof(int64_t), s) == cudaSuccess ? CCE_OK
                                                                                   : fail(CCE_ERR_CUDA, "memset");
   }
-  CCE_TRY(cudaMemsetAsync(w.sync, 0, w.sync_bytes, s));
   {
     cce::PlanArgs PA{};
+    PA.sync = w.sync;
+    PA.sync_ints = static_cast<int64_t>(w.sync_bytes / sizeof(int));
     PA.P = w.plan;
     PA.tile_max = tile_max;
     PA.lse = lse;
@@ -359,8 +360,28 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   cce::BwdLaunch L{};
   CCE_CHECK(make_map(&L.tmE128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kBwdBM));
   CCE_CHECK(make_map(&L.tmC128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, cce::kBwdBN));
-  CCE_CHECK(make_map(&L.tmE64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, 64));
-  CCE_CHECK(make_map(&L.tmC64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, 64));
+  // The dE / dC items load a 64-row x 256-column operand slice per stage. With D a multiple of 256
+  // it is one 3-D TMA load (64 columns x 64 rows x 4 column blocks: the same shared-memory image as
+  // four 64 x 64 boxes); otherwise four 2-D boxes (the last slice of D may be partial).
+  const bool slab3d = D % 256 == 0;
+  if (slab3d) {
+    auto map3 = [&](CUtensorMap* m, const void* ptr, int64_t rows) {
+      cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(D / 64)};
+      cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, 128};
+      cuuint32_t box[3] = {64, 64, 4};
+      cuuint32_t estr[3] = {1, 1, 1};
+      CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      return r == CUDA_SUCCESS ? CCE_OK
+                               : fail(CCE_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d)", static_cast<int>(r));
+    };
+    CCE_CHECK(map3(&L.tmE64, E, N));
+    CCE_CHECK(map3(&L.tmC64, C, V));
+  } else {
+    CCE_CHECK(make_map(&L.tmE64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, 64));
+    CCE_CHECK(make_map(&L.tmC64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, 64));
+  }
   CCE_CHECK(make_map(&L.tmdE, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dE_acc, N, D, 32, 32));
   if (c32) CCE_CHECK(make_map(&L.tmdC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dC, V, D, 32, 32));
   else CCE_CHECK(make_map(&L.tmdC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dC, V, D, 64, 32));
@@ -373,6 +394,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.S = w.plan.S;
   A.nchunks = w.plan.nchunks_dev;
   A.out_bf16 = c32 ? 0 : 1;
+  A.slab3d = slab3d ? 1 : 0;
   A.ignore_index = p->ignore_index;
   A.vocab_start = vs;
   A.buf_bytes = w.buf_bytes;

@@ -363,9 +363,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               bulk_load(dst + PART / 2, tile + PART + h * (PART / 2), PART / 2, bar(kFull + stage));
             }
             const int y = os.x * BM + 64 * h;  // K rows of the operand: C_t rows (dE), E_b rows (dC)
+            if (A.slab3d) {
+              tma_load_3d(dst + PART, de ? &tmC64 : &tmE64, bar(kFull + stage), 0, y, x0 / 64);
+            } else {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-              tma_load_2d(dst + PART + c * X_BOX, de ? &tmC64 : &tmE64, bar(kFull + stage), x0 + 64 * c, y);
+              for (int c = 0; c < 4; ++c)
+                tma_load_2d(dst + PART + c * X_BOX, de ? &tmC64 : &tmE64, bar(kFull + stage), x0 + 64 * c, y);
+            }
             ++issued[stage];
             if (++stage == STAGES) {
               stage = 0;

@@ -36,7 +36,7 @@ __device__ __forceinline__ bool valid_target(int64_t t, int64_t V, int64_t ignor
 // phases separated by grid-wide barriers (bounded waits; a block that gives up records
 // CCE_ERR_DEVICE_TIMEOUT and every block then leaves). Each phase spreads its work over the grid.
 constexpr int kPlanThreads = 1024;
-constexpr int kFlagTiles = 8;    // vocabulary tiles per flag unit
+constexpr int kFlagTiles = 32;   // vocabulary tiles per flag unit
 constexpr int kFlagGroups = kPlanThreads / kBwdBM;  // flag units per block at a time (128 threads each)
 
 struct PlanCtl {
@@ -121,44 +121,51 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Column maxima of a warp's 32 x 32 block (lane = row, v[i] = column i): afterwards lane l returns the
+// maximum over the 32 lanes of v[l]. Recursive halving, 31 shuffles. Clobbers v.
+__device__ __forceinline__ float warp_column_max32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = upper ? v[i] : v[i + o];
+      const float keep = upper ? v[i + o] : v[i];
+      v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+    }
+  }
+  return v[0];
+}
+
 // Flags of one row block b and run of kFlagTiles vocabulary tiles from t0, by 128 threads (one per
-// tile row; named barrier `group + 1`). The rows' targets and LSE are read once for the run.
+// tile row; named barrier `group + 1`). Every load of the unit (the rows' targets and LSE, the run's
+// saved maxima) is issued before any of them is used, so they are in flight together.
 __device__ void tile_flags_unit(const PlanArgs& A, int group, int b, int t0) {
-  __shared__ float wmax[kFlagGroups][kFlagTiles][4];
+  __shared__ float wmax[kFlagGroups][4][kFlagTiles];
   __shared__ int any_target[kFlagGroups][kFlagTiles];
-  const int tid = threadIdx.x & (kBwdBM - 1);
+  const int tid = threadIdx.x & (kBwdBM - 1), lane = tid & 31;
   const int nt = A.P.nt;
   const int64_t r = static_cast<int64_t>(b) * kBwdBM + tid;
+  const bool row_in = r < A.N;
   if (tid < kFlagTiles) any_target[group][tid] = 0;
+  float mt[kFlagTiles];
+#pragma unroll
+  for (int k = 0; k < kFlagTiles; ++k)
+    mt[k] = (row_in && A.filter_on && t0 + k < nt) ? A.tile_max[static_cast<int64_t>(t0 + k) * A.N + r] : -INFINITY;
+  int64_t tr = row_in ? A.targets[r] : A.ignore_index;
+  const float l = (row_in && A.filter_on) ? A.lse[r] : 0.f;
   named_barrier(group + 1, kBwdBM);
-  bool valid = false, local = false;
-  float l = 0.f;
-  int64_t tr = -1;
-  if (r < A.N) {
-    tr = A.targets[r];
-    valid = valid_target(tr, A.vtot, A.ignore_index);                 // the row is scored (by every shard)
-    local = valid && valid_target(tr - A.vs, A.V, A.ignore_index - A.vs);  // its target lies in this shard
-    if (valid && A.filter_on) l = A.lse[r];
-    tr -= A.vs;
-  }
+  const bool valid = row_in && valid_target(tr, A.vtot, A.ignore_index);  // the row is scored (by every shard)
+  const bool local = valid && valid_target(tr - A.vs, A.V, A.ignore_index - A.vs);  // its target is in this shard
+  tr -= A.vs;
   if (local && tr / kBwdBN >= t0 && tr / kBwdBN < t0 + kFlagTiles) any_target[group][tr / kBwdBN - t0] = 1;
 #pragma unroll
-  for (int k = 0; k < kFlagTiles; ++k) {
-    const int t = t0 + k;
-    float m = -INFINITY;
-    if (valid && A.filter_on && t < nt) {
-      const int64_t j0 = static_cast<int64_t>(t) * (kBwdBN / kSubTile);
-      const int64_t j1 = j0 + kBwdBN / kSubTile < A.T ? j0 + kBwdBN / kSubTile : A.T;
-      for (int64_t j = j0; j < j1; ++j) m = fmaxf(m, A.tile_max[j * A.N + r]);
-      m -= l;
-    }
-    m = warp_max(m);
-    if ((tid & 31) == 0) wmax[group][k][tid >> 5] = m;
-  }
+  for (int k = 0; k < kFlagTiles; ++k) mt[k] = valid ? mt[k] - l : -INFINITY;
+  wmax[group][tid >> 5][lane] = warp_column_max32(mt, lane);  // lane k: the warp's max of tile t0 + k
   named_barrier(group + 1, kBwdBM);
   if (tid < kFlagTiles && t0 + tid < nt) {
-    const float* wm = wmax[group][tid];
-    const bool keep = !A.filter_on || fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3])) >= A.ln_eps;
+    const float m = fmaxf(fmaxf(wmax[group][0][tid], wmax[group][1][tid]), fmaxf(wmax[group][2][tid], wmax[group][3][tid]));
+    const bool keep = !A.filter_on || m >= A.ln_eps;
     A.P.flags[static_cast<int64_t>(b) * nt + t0 + tid] = keep ? 1 : (any_target[group][tid] ? 2 : 0);
   }
   named_barrier(group + 1, kBwdBM);  // the shared arrays are reused by the group's next unit
@@ -312,49 +319,58 @@ __device__ void chunk_items_block(const PlanArgs& A, int c, int nchunks) {
 // stay within kChunkCBytes (at most chunk_c_tiles vocabulary tiles with a listed tile), so that a
 // sparse stretch of the vocabulary forms one long chunk: fewer chunks mean fewer partial sums of dE
 // and longer groups of pairs ahead of each chunk's dE / dC items. A chunk of the fixed length
-// chunk_vt always satisfies both limits, so there are never more than P.nchunks chunks. Greedy
-// over the prefix sums offsets_t, staged in shared memory; thread 0 decides.
+// chunk_vt always satisfies both limits, so there are never more than P.nchunks chunks.
+// Greedy, decided by warp 0 over 32 vocabulary tiles at a time (the prefix sums offsets_t staged in
+// shared memory by the block): each lane tests whether its tile still fits the open chunk, and the
+// first lane that does not starts the next one.
 __device__ void chunk_partition(const PlanArgs& A) {
   __shared__ int off[kPlanThreads + 1];
-  __shared__ int st[4];  // chunk count, first tile, listed tiles before it, non-empty tiles so far
   const BwdPlan& P = A.P;
   const int nt = P.nt;
-  if (threadIdx.x == 0) {
-    st[0] = 0;
-    st[1] = 0;
-    st[2] = 0;
-    st[3] = 0;
-    P.chunk_t[0] = 0;
-  }
+  const int lane = threadIdx.x & 31;
+  const bool decider = threadIdx.x < 32;
+  int n = 0, start = 0, start_listed = 0, ne = 0;  // closed chunks; the open chunk's first tile,
+                                                   // listed tiles before it, its non-empty tiles
+  if (threadIdx.x == 0) P.chunk_t[0] = 0;
   for (int base = 0; base < nt; base += kPlanThreads) {
     __syncthreads();
     for (int i = threadIdx.x; i <= kPlanThreads; i += blockDim.x) off[i] = P.offsets_t[min(base + i, nt)];
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int n = st[0], first_listed = st[2], nonempty = st[3];
-      for (int i = 0; i < kPlanThreads && base + i < nt; ++i) {
-        const int t = base + i;
-        const int listed = off[i + 1] - off[i];
-        const bool fits = off[i + 1] - first_listed <= P.chunk_g_tiles &&
-                          nonempty + (listed > 0 ? 1 : 0) <= P.chunk_c_tiles;
-        if (!fits && t > st[1]) {  // close the chunk before tile t
-          if (++n < P.nchunks) P.chunk_t[n] = t;  // (more than P.nchunks cannot happen; see below)
-          st[1] = t;
-          first_listed = off[i];
-          nonempty = 0;
+    if (!decider) continue;
+    for (int sub = 0; sub < kPlanThreads && base + sub < nt; sub += 32) {
+      const int i = sub + lane;
+      const bool in = base + i < nt;
+      const int end_listed = in ? off[i + 1] : 0;  // listed tiles before the end of tile base + i
+      const bool nonempty = in && off[i + 1] > off[i];
+      const unsigned ne_mask = __ballot_sync(0xffffffffu, nonempty);
+      const unsigned le = lane == 31 ? 0xffffffffu : ((2u << lane) - 1u);  // lanes <= this one
+      int from = 0;
+      for (int guard = 0; guard <= 32; ++guard) {
+        const unsigned live = from >= 32 ? 0u : (0xffffffffu << from);
+        const int cum_ne = __popc(ne_mask & live & le);
+        const bool bad = in && lane >= from &&
+                         (end_listed - start_listed > P.chunk_g_tiles || ne + cum_ne > P.chunk_c_tiles);
+        const unsigned bad_mask = __ballot_sync(0xffffffffu, bad);
+        const int j = bad_mask ? __ffs(bad_mask) - 1 : 32;
+        if (j == 32 || base + sub + j <= start) {  // the rest of this group fits the open chunk
+          ne += __popc(ne_mask & live);
+          break;
         }
-        nonempty += listed > 0 ? 1 : 0;
+        // close the open chunk before tile base + sub + j, which starts the next one
+        ++n;
+        if (lane == 0 && n < P.nchunks) P.chunk_t[n] = base + sub + j;
+        start = base + sub + j;
+        start_listed = off[sub + j];
+        ne = 0;
+        from = j;
       }
-      st[0] = n;
-      st[2] = first_listed;
-      st[3] = nonempty;
     }
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    if (st[0] + 1 <= P.nchunks) {
-      P.chunk_t[st[0] + 1] = nt;
-      *P.nchunks_dev = st[0] + 1;
+    if (n + 1 <= P.nchunks) {
+      P.chunk_t[n + 1] = nt;
+      *P.nchunks_dev = n + 1;
     } else {  // defensive: the fixed partition, which always fits the arrays and the buffers
       for (int c = 0; c <= P.nchunks; ++c) P.chunk_t[c] = min(nt, c * P.chunk_vt);
       *P.nchunks_dev = P.nchunks;
@@ -373,7 +389,8 @@ __device__ __forceinline__ int chunk_containing(const int* chunk_t, int n, int t
 }
 
 // The whole plan. Phases (each spread over the grid; a barrier after each):
-//  0  zero the counters and the fp32 accumulators of dE and dbias; the row scales
+//  0  zero the counters (the backward kernel's too) and the fp32 accumulator of dbias; the row
+//     scales (the fp32 accumulator of dE is zeroed a tenth per phase)
 //  1  tile flags
 //  2  per vocabulary tile: ranks of its listed tiles and their count; per row block: its count; the
 //     kept total; per vocabulary tile: rows whose target tile is onehot only, and their dbias terms
@@ -397,18 +414,23 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
 
   // 0
   if (gtid < 2) P.kept_total[gtid] = 0;  // kept_total and n_empty
+  for (int64_t i = gtid; i < A.sync_ints; i += gthreads) A.sync[i] = 0;
   for (int64_t i = gtid; i < nb; i += gthreads) P.cnt_b[i] = 0;
   for (int64_t i = gtid; i < nt; i += gthreads) {
     P.oh_cnt[i] = 0;
     P.oh_cur[i] = 0;
   }
-  {
+  // dE_acc is first read by the tensor-core kernel, so its zeroing (bandwidth-bound) is spread over
+  // the phases, beside their latency-bound work: one tenth at the start of each phase.
+  const int64_t n4 = A.N * A.D / 4;  // D is a multiple of 8
+  auto zero_part = [&](int k) {
     float4* z = reinterpret_cast<float4*>(A.dE_acc);
-    const int64_t n4 = A.N * A.D / 4;  // D is a multiple of 8
-    for (int64_t i = gtid; i < n4; i += gthreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (A.dbias_acc != nullptr)
-      for (int64_t i = gtid; i < A.V; i += gthreads) A.dbias_acc[i] = 0.f;
-  }
+    const int64_t lo = n4 * k / 10, hi = n4 * (k + 1) / 10;
+    for (int64_t i = lo + gtid; i < hi; i += gthreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  zero_part(0);
+  if (A.dbias_acc != nullptr)  // receives atomics in phase 2
+    for (int64_t i = gtid; i < A.V; i += gthreads) A.dbias_acc[i] = 0.f;
   for (int64_t r = gtid; r < A.N; r += gthreads) {
     float s;
     if (A.reduction == 1) {
@@ -422,6 +444,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     A.scale[r] = A.targets[r] != A.ignore_index ? s : 0.f;
   }
   if (!grid_barrier(ctl, ++round)) return;
+  zero_part(round);
 
   // 1
   {
@@ -435,6 +458,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     }
   }
   if (!grid_barrier(ctl, ++round)) return;
+  zero_part(round);
 
   // 2
   for (int t = gwarp; t < nt; t += gwarps) {
@@ -463,12 +487,14 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     if (A.dbias_acc != nullptr) atomicAdd(A.dbias_acc + tr, -A.onehot_coef * A.scale[r]);
   }
   if (!grid_barrier(ctl, ++round)) return;
+  zero_part(round);
 
   // 3
   if (blockIdx.x == 0) block_scan(P.cnt_t, nt, P.offsets_t);
   if (blockIdx.x == 1 % gridDim.x) block_scan(P.cnt_b, nb, P.offsets_b);
   if (blockIdx.x == 2 % gridDim.x) block_scan(P.oh_cnt, nt, P.oh_off);
   if (!grid_barrier(ctl, ++round)) return;
+  zero_part(round);
 
   // 4
   for (int64_t i = gtid; i < tiles; i += gthreads) {
@@ -486,6 +512,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
   }
   if (blockIdx.x == gridDim.x - 1) chunk_partition(A);
   if (!grid_barrier(ctl, ++round)) return;
+  zero_part(round);
   const int nchunks = *reinterpret_cast<volatile int*>(P.nchunks_dev);
 
   // 5
@@ -498,19 +525,23 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
   for (int64_t t = gtid; t < nt; t += gthreads)
     P.chunk_of[t] = chunk_containing(P.chunk_t, nchunks, static_cast<int>(t));
   if (!grid_barrier(ctl, ++round)) return;
+  zero_part(round);
 
   // 6
   for (int t = gwarp; t < nt; t += gwarps) pair_list_warp(A, t, lane, 0);
   if (!grid_barrier(ctl, ++round)) return;
+  zero_part(round);
 
   // 7
   if (blockIdx.x == 0) block_scan(P.cnt_t, nt, P.pstart_t);
   if (!grid_barrier(ctl, ++round)) return;
+  zero_part(round);
 
   // 8
   for (int t = gwarp; t < nt; t += gwarps) pair_list_warp(A, t, lane, 1);
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x) chunk_items_block(A, c, nchunks);
   if (!grid_barrier(ctl, ++round)) return;
+  zero_part(round);
 
   // 9
   if (blockIdx.x == 0) {

@@ -100,6 +100,7 @@ struct BwdArgs {
   int N, D, V, nb, nt, S;
   const int* nchunks;  // [1] the plan's chunk count
   int out_bf16;
+  int slab3d;  // operand slices by one 3-D TMA load (D a multiple of 64)
   int64_t ignore_index;
   int64_t vocab_start;  // C holds vocabulary rows [vocab_start, vocab_start + V); targets are global ids
   size_t buf_bytes;  // one of the kGradBuffers gradient-tile buffers
@@ -140,7 +141,8 @@ struct BwdArgs {
 
 struct BwdLaunch {
   CUtensorMap tmE128, tmC128;  // bf16, box 64 x 128: K-blocks of the recompute
-  CUtensorMap tmE64, tmC64;    // bf16, box 64 x 64: operand slices of the dC / dE MMAs
+  CUtensorMap tmE64, tmC64;    // bf16 operand slices of the dC / dE MMAs: 3-D box 64 x 64 x 4 (D % 256 == 0)
+                               // or 2-D box 64 x 64
   CUtensorMap tmdC;            // dC output: bf16 box 64 x 32, or fp32 box 32 x 32
   CUtensorMap tmdE;            // fp32 dE accumulator, box 32 x 32 (reduce-add)
   BwdArgs args;
@@ -164,6 +166,8 @@ struct PlanArgs {
   float* dE_acc;           // [N, D] fp32, zeroed here
   float* dbias_acc;        // [V] fp32 or null, zeroed here; receives the onehot-only rows' terms
   int64_t* filtered_tiles;
+  int* sync;               // [sync_ints] the backward kernel's queue position and counters, zeroed here
+  int64_t sync_ints;
   int* bar;                // grid barrier counter, zero at launch
   int* err;
   uint64_t timeout_ns;
