@@ -227,7 +227,7 @@ CCE_API const char* cce_last_error_message(void);
  * counterpart; it is an addition for such callers. Arguments and results are those of
  * cce_forward() without the workspace.
  *  - Scratch lives in one device array of CCE_NOALLOC_SCRATCH_BYTES that every GPU loading the
- *    library holds until exit. Problems needing more (about ceil(V/128) * N * 4 + 12 N + 4 D bytes; at
+ *    library holds until exit. Problems needing more (about ceil(V/128) * N * 4 + 5 N + 4 D bytes; at
  *    V = 128256 up to N of about 8000) are rejected with CCE_ERR_UNSUPPORTED before anything runs.
  *  - The first call on each device looks up the array's device address (with that device
  *    current); make that first call before any stream capture.

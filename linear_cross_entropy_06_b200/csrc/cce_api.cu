@@ -89,6 +89,7 @@ bool problem_ok(const cce_problem* p, bool set_error) {
 struct FwdWs {
   WsHeader* hdr;
   float* tile_sum;           // [T, N]
+  float* zt;                 // [N]: correct-token logits picked by the forward kernel
   float* csum;               // [D + 1]: column sums of C and the bias sum (label smoothing only)
   double* block_sums;        // [ceil(N / 32)]: per-block loss sums of the finish kernel
   long long* block_counts;   // [ceil(N / 32)]
@@ -104,6 +105,8 @@ FwdWs carve_fwd(const cce_problem* p, void* base) {
   w.hdr = reinterpret_cast<WsHeader*>(b);
   w.tile_sum = reinterpret_cast<float*>(b + off);
   off = align_up(off + sizeof(float) * static_cast<size_t>(T * p->N));
+  w.zt = reinterpret_cast<float*>(b + off);
+  off = align_up(off + sizeof(float) * static_cast<size_t>(p->N));
   w.csum = reinterpret_cast<float*>(b + off);
   off = align_up(off + sizeof(float) * static_cast<size_t>(p->D + 1));
   w.block_sums = reinterpret_cast<double*>(b + off);
@@ -115,8 +118,8 @@ FwdWs carve_fwd(const cce_problem* p, void* base) {
 }
 
 // The finish kernel's arguments common to the whole-vocabulary and the shard forward.
-cce::FwdFinish finish_args(const cce_problem* p, const FwdWs& w, const void* E, const void* C, const void* bias,
-                           const int64_t* targets, const float* tile_max, bool smooth) {
+cce::FwdFinish finish_args(const cce_problem* p, const FwdWs& w, const void* E, const int64_t* targets,
+                           const float* tile_max, bool smooth) {
   cce::FwdFinish F{};
   F.tile_max = tile_max;
   F.tile_sum = w.tile_sum;
@@ -128,9 +131,8 @@ cce::FwdFinish finish_args(const cce_problem* p, const FwdWs& w, const void* E, 
   F.vtot = vocab_total(p);
   F.ignore_index = p->ignore_index;
   F.E = static_cast<const __nv_bfloat16*>(E);
-  F.C = static_cast<const __nv_bfloat16*>(C);
-  F.bias = static_cast<const __nv_bfloat16*>(bias);
   F.targets = targets;
+  F.zt = w.zt;
   F.csum = smooth ? w.csum : nullptr;
   F.label_smoothing = p->label_smoothing;
   F.z_loss = p->z_loss;
@@ -292,6 +294,7 @@ cce_status make_map(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem, co
     if (s_ != CCE_OK) return s_;   \
   } while (0)
 
+
 // The backward: plan the tiles and work lists, then one persistent launch (cce_bwd.cu) forms the
 // gradient tiles chunk by chunk and runs the dC and dE MMAs from them.
 cce_status backward_split(const cce_problem* p, const void* E, const void* C, const void* bias, const int64_t* targets,
@@ -440,7 +443,8 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
   CCE_TRY(cce::launch_bwd(L, s));
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
-  // the rest: dE's last terms and conversion, dC rows of vocabulary tiles no row block lists, dbias
+  // the rest: dC rows of vocabulary tiles no row block lists, then dE's last terms and conversion,
+  // and dbias
   cce::BwdFinalize F{};
   F.N = N;
   F.D = D;
@@ -467,6 +471,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   F.dc_bf16 = c32 ? 0 : 1;
   F.dbias_acc = dbias_acc;
   F.dbias_out = (dbias != nullptr && !c32) ? dbias : nullptr;
+  CCE_TRY(cce::launch_empty_tiles(F, num_sms, s));
   CCE_TRY(cce::launch_bwd_finalize(F, num_sms, s));
   return CCE_OK;
 }
@@ -571,6 +576,10 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
     L.T = static_cast<int>(T);
     L.tile_max = tile_max;
     L.tile_sum = w.tile_sum;
+    L.targets = targets;
+    L.vs = 0;
+    L.ignore_index = p->ignore_index;
+    L.zt = w.zt;
     L.err = &w.hdr->err;
     L.timeout_ns = cce::wait_timeout_ns();
     L.num_sms = num_sms;
@@ -583,7 +592,7 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
     CCE_TRY(cce::launch_fwd_lse(L, s));
     if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[1], s));
   }
-  cce::FwdFinish F = finish_args(p, w, E, C, bias, targets, tile_max, smooth);
+  cce::FwdFinish F = finish_args(p, w, E, targets, tile_max, smooth);
   F.lse = lse;
   F.loss = loss;
   F.count = count;
@@ -645,6 +654,10 @@ cce_status cce_forward_partial(const cce_problem* p, const void* E, const void* 
   L.T = static_cast<int>(T);
   L.tile_max = tile_max;
   L.tile_sum = w.tile_sum;
+  L.targets = targets;
+  L.vs = p->vocab_start;
+  L.ignore_index = p->ignore_index;
+  L.zt = w.zt;
   L.err = &w.hdr->err;
   L.timeout_ns = cce::wait_timeout_ns();
   L.num_sms = num_sms;
@@ -654,7 +667,7 @@ cce_status cce_forward_partial(const cce_problem* p, const void* E, const void* 
   CCE_TRY(cce::launch_fwd_lse(L, s));
   if (g_fwd_ev[0] && g_fwd_ev[1]) CCE_TRY(cudaEventRecord(g_fwd_ev[1], s));
   // partial rows: the shard's log-sum-exp, correct-token logit and logit sum (0 without smoothing)
-  cce::FwdFinish F = finish_args(p, w, E, C, bias, targets, tile_max, smooth);
+  cce::FwdFinish F = finish_args(p, w, E, targets, tile_max, smooth);
   F.lse = partial;
   F.zt_out = partial + N;
   F.zs_out = partial + 2 * N;

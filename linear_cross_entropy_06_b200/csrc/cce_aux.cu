@@ -1,10 +1,10 @@
 // The bandwidth-bound and bookkeeping kernels around the tensor-core kernels:
 //  fwd_finish     per row LSE = M + ln sum_j s_j exp(m_j - M) over the saved sub-tile (max, sum-exp)
-//                 pairs, the correct-token logit z_t = E[r] . C[t_r] (fp32 accumulation of bf16
-//                 products) with target validation, loss_r = LSE_r - z_t (0 for ignored rows), and
-//                 the count and mean/sum in a fixed order (fp64). Loss functions explainer, "How it
-//                 works" items 1 and 4; Cut Your Losses abstract (only the correct token's logit);
-//                 Cut Cross Entropy from first principles; mlx-cross-entropy README, "API".
+//                 pairs, target validation, loss_r = LSE_r - z_t with the correct-token logit z_t
+//                 the forward kernel picked from its logit tile (0 for ignored rows), and the count
+//                 and mean/sum in a fixed order (fp64). Loss functions explainer, "How it works"
+//                 items 1 and 4; Cut Cross Entropy from first principles; mlx-cross-entropy README,
+//                 "API".
 //  shard_merge    the same loss from the partial results of several vocabulary shards.
 //  weighted_colsum  column sums of C or of scale_r E_r (label smoothing's rank-one terms).
 //  fill_zero      zeroes a buffer (the fp32 accumulators of dE and dbias).
@@ -18,19 +18,6 @@ namespace {
 
 __device__ __forceinline__ bool valid_target(int64_t t, int64_t V, int64_t ignore_index) {
   return t != ignore_index && t >= 0 && t < V;
-}
-
-__device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
-  const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
-  const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 fx = __bfloat1622float2(x[i]);
-    const float2 fy = __bfloat1622float2(y[i]);
-    acc = fmaf(fx.x, fy.x, acc);
-    acc = fmaf(fx.y, fy.y, acc);
-  }
-  return acc;
 }
 
 // One warp per row; lanes read 16-byte pieces, so a warp reads 512 contiguous bytes per step.
@@ -58,18 +45,20 @@ __device__ __forceinline__ void lse_merge(float& M, float& S, float m, float s) 
   }
 }
 
-constexpr int kFinishWarps = kFinishRows;  // rows per block; one warp per row for the dot products
+constexpr int kFinishWarps = kFinishRows;  // rows per block; one warp per row for the dot product
+constexpr int kFinishBatch = 8;            // sub-tiles a warp loads before merging them
 constexpr int kReduceThreads = 1024;
 
 // The rest of the forward after the tensor-core kernel, one block of 32 warps per 32 rows:
 //  1. LSE_r = M + ln sum_j s_j exp(m_j - M) over the saved per-sub-tile (max, sum-exp) pairs
 //     (Loss functions explainer, "How it works" item 1). Warp w merges sub-tiles j = w, w + 32, ...
-//     of the block's rows (lane = row: 128-byte loads), four sub-tiles per step.
-//  2. warp w: the correct-token logit z_t = E_r . C_{t_r} (+ bias) of row r0 + w, fp32 accumulation
-//     of bf16 products, 16-byte loads (Cut Your Losses abstract: only the correct token's logit);
-//     with label smoothing also z_sum = sum_v z[r, v] = E_r . colsum(C) (+ sum of the bias). C holds
-//     vocabulary rows [vs, vs + V) of vtot: a target elsewhere gets z_t = 0 (another shard's), and a
-//     target outside [0, vtot) that is not ignore_index is a device error.
+//     of the block's rows (lane = row: 128-byte loads), kFinishBatch sub-tiles per step.
+//  2. warp w, row r0 + w: the correct-token logit z_t, which the forward kernel took from its fp32
+//     logit tile (Cut Your Losses abstract: only the correct token's logit is computed); with label
+//     smoothing also z_sum = sum_v z[r, v] = E_r . colsum(C) (+ sum of the bias), fp32 accumulation
+//     of bf16 products, 16-byte loads. C holds vocabulary rows [vs, vs + V) of vtot: a target
+//     elsewhere gets z_t = 0 (another shard's), and a target outside [0, vtot) that is not
+//     ignore_index is a device error.
 //  3. the loss of each row, LSE - (1 - ls) z_t - (ls / V) z_sum + zl LSE^2 (0 for ignored rows; Cut
 //     Cross Entropy from first principles; explainer items 3 and 4, z-loss), and the block's fp64
 //     sum and count; the last block to finish adds the blocks' sums in block order (a fixed order:
@@ -89,16 +78,16 @@ __global__ void __launch_bounds__(kFinishWarps * 32) fwd_finish_kernel(const __g
     const int64_t r = r0 + lane;
     float M = -INFINITY, S = 0.f;
     if (r < N) {
-      for (int64_t j = w; j < T; j += 4 * kFinishWarps) {
-        float m[4], sv[4];
+      for (int64_t j = w; j < T; j += kFinishBatch * kFinishWarps) {
+        float m[kFinishBatch], sv[kFinishBatch];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kFinishBatch; ++u) {
           const int64_t jj = j + u * kFinishWarps;
           m[u] = jj < T ? F.tile_max[jj * N + r] : -INFINITY;
           sv[u] = jj < T ? F.tile_sum[jj * N + r] : 0.f;
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) lse_merge(M, S, m[u], sv[u]);
+        for (int u = 0; u < kFinishBatch; ++u) lse_merge(M, S, m[u], sv[u]);
       }
     }
     sm_m[w][lane] = M;
@@ -116,17 +105,7 @@ __global__ void __launch_bounds__(kFinishWarps * 32) fwd_finish_kernel(const __g
         zs = warp_sum(zs) + F.csum[D];
       }
       if (valid_target(t - F.vs, F.V, F.ignore_index - F.vs)) {  // not ignored, inside this shard
-        const int64_t tl = t - F.vs;
-        const __nv_bfloat16* c = F.C + tl * D;
-        float acc0 = 0.f, acc1 = 0.f;
-        int64_t d = static_cast<int64_t>(lane) * 8;
-        for (; d + 256 < D; d += 512) {
-          acc0 = dot8_bf16(ld_global_nc_v4(e + d), ld_global_nc_v4(c + d), acc0);
-          acc1 = dot8_bf16(ld_global_nc_v4(e + d + 256), ld_global_nc_v4(c + d + 256), acc1);
-        }
-        if (d < D) acc0 = dot8_bf16(ld_global_nc_v4(e + d), ld_global_nc_v4(c + d), acc0);
-        zt = warp_sum(acc0 + acc1);
-        if (F.bias != nullptr) zt += __bfloat162float(F.bias[tl]);
+        zt = F.zt[r];
       } else if (lane == 0 && t != F.ignore_index && !valid_target(t, F.vtot, F.ignore_index)) {
         record_error(F.err, kErrTargetRange);
       }

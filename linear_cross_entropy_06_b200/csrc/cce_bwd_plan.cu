@@ -550,63 +550,154 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
   }
 }
 
-// The backward's last launch, after the tensor-core kernel: every element-wise step left, in one
-// persistent kernel whose blocks take work units in turn (256 threads; 64 threads x 8 columns cover
-// 512 columns of a row, 16-byte loads and stores, four rows at a time):
-//  A. dE, 32 rows x 512 columns per unit: dE_acc plus, for a row whose target tile was skipped
-//     ("onehot only"), its onehot term -scale_r (1 - ls) C_{t_r}, and with label smoothing the rank-one
-//     term -scale_r (ls / V) sum_v C_v; written as bf16 (or in place in fp32).
-//  B. dC rows of the vocabulary tiles no row block lists, 128 rows x 512 columns per unit. Every
-//     logit of such a tile is skipped, so only the target part of the logit gradient reaches them
-//     (Loss functions explainer, "How it works" items 2 and 3): -scale_r (1 - ls) E_r for each row r
-//     whose target v lies there, and the smoothing term dc_coef * wsum shared by every row of dC. The
-//     target rows (oh_rows[oh_off[t] .. oh_off[t + 1]): for an empty tile every non-ignored row
-//     targeting it is listed there) are staged in shared memory and scanned in list order, so the
-//     result is deterministic.
-//  C. dbias, 2048 entries per unit: dbias_acc (the G column sums and the onehot terms) plus the
-//     smoothing constant, written as bf16 (or in place in fp32).
+// The element-wise steps of the backward after the tensor-core kernel, in two launches:
+//  empty_tiles_kernel: dC rows of the vocabulary tiles no row block lists. Every logit of such a
+//   tile is skipped, so only the target part of the logit gradient reaches them (Loss functions
+//   explainer, "How it works" items 2 and 3): -scale_r (1 - ls) E_r for each row r whose target v
+//   lies there, and the smoothing term -(ls / V) wsum shared by every row of dC. The target rows
+//   (oh_rows[oh_off[t] .. oh_off[t + 1]]: for an empty tile every non-ignored row targeting it is
+//   listed there) are added in list order, so the result is deterministic. The constant rows go out
+//   as bulk copies from shared memory.
+//  bwd_finalize_kernel (256 threads; 64 threads x 8 columns cover 512 columns of a row, 16-byte
+//  loads and stores, four rows at a time):
+//   A. dE, 32 rows x 512 columns per unit: dE_acc plus, for a row whose target tile was skipped
+//      ("onehot only"), its onehot term -scale_r (1 - ls) C_{t_r}, and with label smoothing the
+//      rank-one term -scale_r (ls / V) sum_v C_v; written as bf16 (or in place in fp32).
+//   C. dbias, 2048 entries per unit: dbias_acc (the G column sums and the onehot terms) plus the
+//      smoothing constant, written as bf16 (or in place in fp32).
 constexpr int kFinCols = 512;
-constexpr int kFinList = 256;  // target rows staged per B unit; longer lists are read from global memory
+constexpr int kFillThreads = 128;
+constexpr int64_t kFillImageBytes = 64 << 10;  // shared-memory image of the constant rows
 constexpr int kFinRowsA = 32;
 constexpr int kFinBias = 2048;
 
+__device__ __forceinline__ void store8(void* base, int bf16, int64_t idx, const float (&acc)[8]) {
+  if (bf16) {
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + idx) = o;
+  } else {
+    float4* out = reinterpret_cast<float4*>(static_cast<float*>(base) + idx);
+    out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const __nv_bfloat16* src, float a) {
+  const uint4 q = ld_global_nc_v4(src);
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    __nv_bfloat162 h;
+    *reinterpret_cast<uint32_t*>(&h) = w[k];
+    acc[2 * k] = fmaf(a, __low2float(h), acc[2 * k]);
+    acc[2 * k + 1] = fmaf(a, __high2float(h), acc[2 * k + 1]);
+  }
+}
+
+// One warp per empty vocabulary tile t. Its rows of dC are the constant row c = -(ls / V) wsum
+// (zeros without label smoothing) except the rows of tokens some row r targets. The block keeps
+// image_rows copies of c (columns [d0, d0 + win) of it when a row is wider than the image) in
+// shared memory, and lane 0 writes every run of constant rows of t with bulk copies from that
+// image, so the copy engine streams the bytes out while the warp computes the target rows:
+// c + sum of a_r E_r over the list entries of that token, in list order, 16-byte loads and stores.
+__global__ void __launch_bounds__(kFillThreads) empty_tiles_kernel(const __grid_constant__ BwdFinalize F,
+                                                                   int64_t win, int image_rows) {
+  extern __shared__ __align__(128) uint8_t img[];
+  const int64_t D = F.D;
+  const int es = F.dc_bf16 ? 2 : 4;
+  const int64_t rowbytes = D * es;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kWarps = kFillThreads / 32;
+  const int n_empty = *F.n_empty;
+  const uint32_t img_u32 = smem_u32(img);
+  char* dC = static_cast<char*>(F.dC);
+  for (int64_t d0 = 0; d0 < D; d0 += win) {
+    const int64_t w = D - d0 < win ? D - d0 : win;
+    __syncthreads();  // every bulk copy of the previous window has read the image
+    for (int64_t i = threadIdx.x; i < image_rows * w; i += kFillThreads) {
+      const float c = F.wsum != nullptr ? -F.ls_v * F.wsum[d0 + i % w] : 0.f;
+      if (F.dc_bf16) reinterpret_cast<__nv_bfloat16*>(img)[i] = __float2bfloat16_rn(c);
+      else reinterpret_cast<float*>(img)[i] = c;
+    }
+    fence_proxy_async_smem();  // the image, written by threads, is read by the copy engine
+    __syncthreads();
+    for (int u = warp * gridDim.x + blockIdx.x; u < n_empty; u += gridDim.x * kWarps) {  // blocks first
+      const int t = F.empty_list[u];
+      const int64_t v0 = static_cast<int64_t>(t) * kBwdBN;
+      const int rows = F.V - v0 < kBwdBN ? static_cast<int>(F.V - v0) : kBwdBN;
+      const int i0 = F.oh_off[t], i1 = F.oh_off[t + 1];
+      // rows of t that some row targets: bit k % 32 of mk, k / 32 = 0..3
+      uint32_t m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u;
+      for (int c0 = i0; c0 < i1; c0 += 32) {
+        const int col = c0 + lane < i1 ? static_cast<int>(F.targets[F.oh_rows[c0 + lane]] - F.vs - v0) : -1;
+        const uint32_t bit = col >= 0 ? 1u << (col & 31) : 0u;
+        m0 |= __reduce_or_sync(0xffffffffu, (col >> 5) == 0 ? bit : 0u);
+        m1 |= __reduce_or_sync(0xffffffffu, (col >> 5) == 1 ? bit : 0u);
+        m2 |= __reduce_or_sync(0xffffffffu, (col >> 5) == 2 ? bit : 0u);
+        m3 |= __reduce_or_sync(0xffffffffu, (col >> 5) == 3 ? bit : 0u);
+      }
+      const uint64_t lo = (static_cast<uint64_t>(m1) << 32) | m0, hi = (static_cast<uint64_t>(m3) << 32) | m2;
+      auto target_row = [lo, hi](int row) { return (((row < 64 ? lo : hi) >> (row & 63)) & 1u) != 0; };
+      if (lane == 0) {
+        for (int row = 0; row < rows;) {
+          if (target_row(row)) {
+            ++row;
+            continue;
+          }
+          int end = row + 1;
+          while (end < rows && end - row < image_rows && !target_row(end)) ++end;
+          char* dst = dC + ((v0 + row) * D + d0) * es;
+          bulk_store(dst, img_u32, static_cast<uint32_t>(w == D ? (end - row) * rowbytes : w * es));
+          row = end;
+        }
+        bulk_commit_group();
+      }
+      if (d0 != 0) continue;  // target rows are written whole, with the first window
+      for (int k = 0; k < 2; ++k) {
+        for (uint64_t bits = k == 0 ? lo : hi; bits != 0; bits &= bits - 1) {
+          const int row = k * 64 + __ffsll(static_cast<long long>(bits)) - 1;
+          for (int64_t db = 0; db < D; db += 256) {
+            const int64_t d = db + lane * 8;
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = F.wsum != nullptr && d < D ? -F.ls_v * F.wsum[d + j] : 0.f;
+            for (int c0 = i0; c0 < i1; c0 += 32) {
+              int r = 0, col = -1;
+              float a = 0.f;
+              if (c0 + lane < i1) {
+                r = F.oh_rows[c0 + lane];
+                col = static_cast<int>(F.targets[r] - F.vs - v0);
+                a = -F.scale[r] * F.onehot_coef;
+              }
+              for (unsigned m = __ballot_sync(0xffffffffu, col == row); m != 0; m &= m - 1) {  // list order
+                const int q = __ffs(m) - 1;
+                const int rq = __shfl_sync(0xffffffffu, r, q);
+                const float aq = __shfl_sync(0xffffffffu, a, q);
+                if (d < D) add_bf16x8(acc, F.E + static_cast<int64_t>(rq) * D + d, aq);
+              }
+            }
+            if (d < D) store8(F.dC, F.dc_bf16, (v0 + row) * D + d, acc);
+          }
+        }
+      }
+    }
+    if (lane == 0) bulk_wait_group_read0();  // before the image is rewritten
+  }
+  if (lane == 0) bulk_wait_group0();  // the bulk copies are complete before the block exits
+}
+
 __global__ void __launch_bounds__(256, 2) bwd_finalize_kernel(const __grid_constant__ BwdFinalize F) {
-  __shared__ int s_row[kFinList];
-  __shared__ int s_r[kFinList];
-  __shared__ float s_a[kFinList];
   const int64_t D = F.D;
   const int col_chunks = static_cast<int>((D + kFinCols - 1) / kFinCols);
   const int64_t units_a = (F.N + kFinRowsA - 1) / kFinRowsA * col_chunks;
-  const int64_t units_b = static_cast<int64_t>(*F.n_empty) * col_chunks;
   const int64_t units_c = F.dbias_acc != nullptr ? (F.V + kFinBias - 1) / kFinBias : 0;
   const int row0 = threadIdx.x >> 6;
   const int col_thread = (threadIdx.x & 63) * 8;
-  auto store8 = [&](void* base, int bf16, int64_t idx, const float (&acc)[8]) {
-    if (bf16) {
-      uint4 o;
-      o.x = pack_bf16x2(acc[0], acc[1]);
-      o.y = pack_bf16x2(acc[2], acc[3]);
-      o.z = pack_bf16x2(acc[4], acc[5]);
-      o.w = pack_bf16x2(acc[6], acc[7]);
-      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + idx) = o;
-    } else {
-      float4* out = reinterpret_cast<float4*>(static_cast<float*>(base) + idx);
-      out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-    }
-  };
-  auto add_bf16x8 = [&](float (&acc)[8], const __nv_bfloat16* src, float a) {
-    const uint4 q = ld_global_nc_v4(src);
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      __nv_bfloat162 h;
-      *reinterpret_cast<uint32_t*>(&h) = w[k];
-      acc[2 * k] = fmaf(a, __low2float(h), acc[2 * k]);
-      acc[2 * k + 1] = fmaf(a, __high2float(h), acc[2 * k + 1]);
-    }
-  };
-  for (int64_t u = blockIdx.x; u < units_a + units_b + units_c; u += gridDim.x) {
+  for (int64_t u = blockIdx.x; u < units_a + units_c; u += gridDim.x) {
     if (u < units_a) {  // A: dE rows
       const int64_t d = (u % col_chunks) * kFinCols + col_thread;
       if (d >= D) continue;
@@ -636,46 +727,8 @@ __global__ void __launch_bounds__(256, 2) bwd_finalize_kernel(const __grid_const
           add_bf16x8(acc, F.C + tl * D + d, -F.onehot_coef * sc);
         store8(F.dE_out != nullptr ? F.dE_out : static_cast<void*>(F.dE_acc), F.dE_out != nullptr, r * D + d, acc);
       }
-    } else if (u < units_a + units_b) {  // B: dC rows of an empty vocabulary tile
-      const int64_t ub = u - units_a;
-      const int t = F.empty_list[ub / col_chunks];
-      const int64_t d = (ub % col_chunks) * kFinCols + col_thread;
-      const int i0 = F.oh_off[t], i1 = F.oh_off[t + 1];
-      const bool staged = i1 - i0 <= kFinList;
-      __syncthreads();  // the previous B unit is done with the staged rows
-      if (staged) {
-        for (int i = threadIdx.x; i < i1 - i0; i += blockDim.x) {
-          const int r = F.oh_rows[i0 + i];
-          s_r[i] = r;
-          s_row[i] = static_cast<int>(F.targets[r] - F.vs - static_cast<int64_t>(t) * kBwdBN);
-          s_a[i] = -F.scale[r] * F.onehot_coef;
-        }
-      }
-      __syncthreads();
-      if (d >= D) continue;
-      float base[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) base[k] = F.wsum != nullptr ? -F.ls_v * F.wsum[d + k] : 0.f;
-      for (int row = row0; row < kBwdBN; row += 4) {
-        const int64_t v = static_cast<int64_t>(t) * kBwdBN + row;
-        if (v >= F.V) break;
-        float acc[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = base[k];
-        if (staged) {
-          for (int i = 0; i < i1 - i0; ++i)
-            if (s_row[i] == row) add_bf16x8(acc, F.E + static_cast<int64_t>(s_r[i]) * D + d, s_a[i]);
-        } else {
-          for (int i = i0; i < i1; ++i) {
-            const int r = F.oh_rows[i];
-            if (F.targets[r] - F.vs == v) add_bf16x8(acc, F.E + static_cast<int64_t>(r) * D + d,
-                                                     -F.scale[r] * F.onehot_coef);
-          }
-        }
-        store8(F.dC, F.dc_bf16, v * D + d, acc);
-      }
     } else {  // C: dbias
-      const int64_t v0 = (u - units_a - units_b) * kFinBias;
+      const int64_t v0 = (u - units_a) * kFinBias;
       const float add = F.wsum != nullptr ? -F.ls_v * F.wsum[D] : 0.f;
       for (int64_t v = v0 + threadIdx.x; v < v0 + kFinBias && v < F.V; v += blockDim.x) {
         const float x = F.dbias_acc[v] + add;
@@ -694,6 +747,21 @@ __global__ void skip_map_kernel(const uint8_t* __restrict__ flags, int64_t n, ui
 }
 
 }  // namespace
+
+cudaError_t launch_empty_tiles(const BwdFinalize& F, int num_sms, cudaStream_t s) {
+  if (F.N == 0) return cudaSuccess;
+  const int64_t es = F.dc_bf16 ? 2 : 4, rowbytes = F.D * es;
+  // whole rows when one fits the image (up to 128 of them); otherwise windows of whole 16-byte pieces
+  const int64_t win = rowbytes <= kFillImageBytes ? F.D : kFillImageBytes / es / 8 * 8;
+  const int image_rows = static_cast<int>(rowbytes <= kFillImageBytes ? std::min<int64_t>(kBwdBN, kFillImageBytes / rowbytes) : 1);
+  const size_t smem = static_cast<size_t>(image_rows * win * es);
+  cudaError_t e = cudaFuncSetAttribute(empty_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kFillImageBytes));
+  if (e != cudaSuccess) return e;
+  empty_tiles_kernel<<<num_sms * 2, kFillThreads, smem, s>>>(F, win, image_rows);
+  note_launches(1);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_finalize(const BwdFinalize& F, int num_sms, cudaStream_t s) {
   if (F.N == 0) return cudaSuccess;

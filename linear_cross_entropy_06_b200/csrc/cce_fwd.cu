@@ -11,8 +11,9 @@
 //   warp 0      TMA producer: E and C tiles (bf16, 128B swizzle) into a 4-stage ring.
 //   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma (M=128, N=256, K=16)
 //               into one of two 256-column fp32 accumulators.
-//   warps 2..5  epilogue: TMEM -> registers, per-row max / sum-exp over each 128-column sub-tile
-//               while the MMA fills the other accumulator.
+//   warps 2..5  epilogue: TMEM -> registers, per-row max / sum-exp over each 128-column sub-tile,
+//               and the correct-token logit of rows whose target falls in the tile, while the MMA
+//               fills the other accumulator.
 // Tiles are visited row-block fastest within groups of 32 row blocks (see tile_coords), so the
 // CTAs working at one time share a few C tiles and E stays in L2.
 #include "cce_device.cuh"
@@ -69,7 +70,8 @@ __device__ __forceinline__ void tile_coords(int w, int nb, int nt, int& b, int& 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_lse_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmC, int N, int D,
                    int V, int T, const __nv_bfloat16* __restrict__ bias, float* __restrict__ tile_max,
-                   float* __restrict__ tile_sum, int* err, uint64_t timeout_ns, int inject_stall) {
+                   float* __restrict__ tile_sum, const int64_t* __restrict__ targets, int64_t vs,
+                   int64_t ignore_index, float* __restrict__ zt, int* err, uint64_t timeout_ns, int inject_stall) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm = carve(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -204,6 +206,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const int r = b * BM + row_in_tile;
+      // The row's correct-token column inside this tile (-1: elsewhere, ignored, or no row)
+      int tcol = -1;
+      if (r < N) {
+        const int64_t tl = targets[r] - vs;
+        if (targets[r] != ignore_index && tl >= static_cast<int64_t>(t) * BN && tl < min(t * BN + BN, V))
+          tcol = static_cast<int>(tl) - t * BN;
+      }
 #pragma unroll
       for (int sub = 0; sub < BN / kSubTile; ++sub) {
         float m = -INFINITY, s = 0.f;
@@ -213,6 +222,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_ld32(tbase + static_cast<uint32_t>(sub * kSubTile + c * 32), v);
           const int col0 = t * BN + sub * kSubTile + c * 32;
           if (bias != nullptr) add_bias32(v, bias, col0, V);
+          // Cut Your Losses (abstract): of the logits only the correct token's is kept, picked here
+          // from the same fp32 tile the log-sum-exp reads. Each row has one such column, so the branch
+          // is rare.
+          const int k = tcol - (sub * kSubTile + c * 32);
+          const bool hit = k >= 0 && k < 32;
+          if (__any_sync(0xffffffffu, hit)) {
+            float z = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) z = i == k ? v[i] : z;
+            if (hit) zt[r] = z;
+          }
           if (col0 + 32 > V) {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
@@ -263,7 +283,8 @@ cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(total < L.num_sms ? total : L.num_sms);
   fwd_lse_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE, L.tmC, L.N, L.D, L.V, L.T, L.bias, L.tile_max,
-                                                       L.tile_sum, L.err, L.timeout_ns, L.inject_stall);
+                                                       L.tile_sum, L.targets, L.vs, L.ignore_index, L.zt, L.err,
+                                                       L.timeout_ns, L.inject_stall);
   note_launches(1);
   return cudaGetLastError();
 }

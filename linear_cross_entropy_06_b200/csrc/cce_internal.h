@@ -24,6 +24,9 @@ struct FwdLaunch {
   const __nv_bfloat16* bias;  // [V] added to every row of logits, or null
   float* tile_max;  // [T, N]
   float* tile_sum;  // [T, N]: sum over the sub-tile of exp(z - tile_max)
+  const int64_t* targets;  // [N]: rows whose target v lies in C (vs <= v < vs + V, v != ignore_index) ...
+  int64_t vs, ignore_index;
+  float* zt;              // ... get zt[r] = z[r, v] (bias included), taken from the logit tile; others untouched
   int* err;
   uint64_t timeout_ns;
   int num_sms;
@@ -100,7 +103,7 @@ struct BwdArgs {
   int N, D, V, nb, nt, S;
   const int* nchunks;  // [1] the plan's chunk count
   int out_bf16;
-  int slab3d;  // operand slices by one 3-D TMA load (D a multiple of 64)
+  int slab3d;  // operand slices by one 3-D TMA load (D a multiple of 256)
   int64_t ignore_index;
   int64_t vocab_start;  // C holds vocabulary rows [vocab_start, vocab_start + V); targets are global ids
   size_t buf_bytes;  // one of the kGradBuffers gradient-tile buffers
@@ -202,6 +205,9 @@ struct BwdFinalize {
   float* dbias_acc;           // [V] fp32, or null (no dbias)
   void* dbias_out;            // bf16 [V], or null: dbias_acc is the output (fp32)
 };
+// dC rows of the vocabulary tiles no row block lists.
+cudaError_t launch_empty_tiles(const BwdFinalize& F, int num_sms, cudaStream_t s);
+// dE's last terms and conversion, dbias (after the tensor-core kernel and launch_empty_tiles).
 cudaError_t launch_bwd_finalize(const BwdFinalize& F, int num_sms, cudaStream_t s);
 // out[i] = 1 if tile i of the plan's flags was skipped, 0 if it was kept (i < tiles).
 cudaError_t launch_skip_map(const uint8_t* flags, int64_t tiles, uint8_t* out, cudaStream_t s);
@@ -217,9 +223,8 @@ struct FwdFinish {
   int64_t vs, vtot;       // C holds vocabulary rows [vs, vs + V) of vtot (0 and V: the whole vocabulary)
   int64_t ignore_index;
   const __nv_bfloat16* E;
-  const __nv_bfloat16* C;
-  const __nv_bfloat16* bias;  // [V] or null
   const int64_t* targets;
+  const float* zt;            // [N] correct-token logits written by the forward kernel (rows with a local target)
   const float* csum;          // [D + 1] column sums of C and the bias sum (label smoothing), or null
   float label_smoothing, z_loss;
   float* lse;                 // [N]

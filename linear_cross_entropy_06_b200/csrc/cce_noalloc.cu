@@ -108,10 +108,12 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   if ((reinterpret_cast<uintptr_t>(E) | reinterpret_cast<uintptr_t>(C) | reinterpret_cast<uintptr_t>(bias)) & 15u)
     return fail(CCE_ERR_INVALID_ARG, "cce_forward_noalloc: E, C and bias must be 16-byte aligned");
   // Same layout as the forward workspace: header (error word, finish counter) | tile_sum [T, N] |
-  // csum [D + 1] (label smoothing) | per-block loss sums and counts of the finish kernel.
+  // zt [N] (correct-token logits) | csum [D + 1] (label smoothing) | per-block loss sums and counts
+  // of the finish kernel.
   const size_t nblk = static_cast<size_t>(N > 0 ? (N + cce::kFinishRows - 1) / cce::kFinishRows : 1);
   const size_t off_sum = kHeader;
-  const size_t off_csum = up(off_sum + sizeof(float) * static_cast<size_t>(T * N));
+  const size_t off_zt = up(off_sum + sizeof(float) * static_cast<size_t>(T * N));
+  const size_t off_csum = up(off_zt + sizeof(float) * static_cast<size_t>(N));
   const size_t off_bsum = up(off_csum + sizeof(float) * static_cast<size_t>(D + 1));
   const size_t off_bcnt = up(off_bsum + sizeof(double) * nblk);
   const size_t need = up(off_bcnt + sizeof(long long) * nblk);
@@ -131,6 +133,7 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   int* err = reinterpret_cast<int*>(b);
   int* done = err + 1;
   float* tile_sum = reinterpret_cast<float*>(b + off_sum);
+  float* zt = reinterpret_cast<float*>(b + off_zt);
   float* csum = reinterpret_cast<float*>(b + off_csum);
   const bool smooth = p->label_smoothing > 0.f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -150,6 +153,10 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
     L.T = static_cast<int>(T);
     L.tile_max = tile_max;
     L.tile_sum = tile_sum;
+    L.targets = targets;
+    L.vs = 0;
+    L.ignore_index = p->ignore_index;
+    L.zt = zt;
     L.err = err;
     L.timeout_ns = cce::wait_timeout_ns();
     L.num_sms = num_sms;
@@ -170,9 +177,8 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   F.vtot = V;
   F.ignore_index = p->ignore_index;
   F.E = static_cast<const __nv_bfloat16*>(E);
-  F.C = Cb;
-  F.bias = Bb;
   F.targets = targets;
+  F.zt = zt;
   F.csum = smooth ? csum : nullptr;
   F.label_smoothing = p->label_smoothing;
   F.z_loss = p->z_loss;
