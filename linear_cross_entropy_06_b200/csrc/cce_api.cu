@@ -188,9 +188,9 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.pos_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(tiles)));
   w.plan.kept_total = reinterpret_cast<int*>(take(2 * sizeof(int)));
   w.plan.n_empty = w.plan.kept_total + 1;
-  // A chunk spans at most kChunkCBytes of C (its C rows stay in L2 while they are re-read for
-  // every listed row block), and the gradient tiles of kGradBuffers chunks, at most nb per
-  // vocabulary tile, fit in the scratch budget; at least one vocabulary tile per chunk.
+  // A chunk spans at most kChunkCBytes of C (the trade-off between dE's split-reduce passes and
+  // re-reads of C), and the gradient tiles of kGradBuffers chunks, at most nb per vocabulary tile,
+  // fit in the scratch budget; at least one vocabulary tile per chunk.
   const int64_t vt_bytes = static_cast<int64_t>(cce::kBwdBN) * p->D * 2;
   const int64_t per_vtile = std::max<int64_t>(nb, 1) * cce::kGradTileBytes;
   const int64_t budget = std::max(cce::kGradScratchMin, nb * cce::kGradScratchPerRowBlock);
