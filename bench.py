@@ -42,19 +42,19 @@ ORACLE_SKIP_TILE = (128, 128)
 # one-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), reported as the roofline's
 # "traffic". Each entry is keyed by the workload's (N, D, V) and holds the SHA-256 of the kernel's
 # sources at the time of the capture: when those sources change, the figure no longer describes the
-# kernel and the bench reports null instead. See profiles/dram_traffic_*.md for the captures.
-KERNEL_SOURCES = {
-    "fwd_lse_kernel": ("cce_fwd.cu", "cce_device.cuh", "cce_internal.h"),
-    "bwd_kernel": ("cce_bwd.cu", "cce_device.cuh", "cce_internal.h"),
+# kernel and the bench reports null instead. The ncu summaries under profiles/ give the commands.
+KERNEL_SOURCES = {  # the kernel and what sets up its work (maps, plan, chunking)
+    "fwd_lse_kernel": ("cce_fwd.cu", "cce_device.cuh", "cce_internal.h", "cce_api.cu"),
+    "bwd_kernel": ("cce_bwd.cu", "cce_device.cuh", "cce_internal.h", "cce_api.cu", "cce_bwd_plan.cu"),
 }
 TRAFFIC_BYTES = {
     "fwd_lse_kernel": {
-        (4096, 4096, 128256): ("d741d132ee5687379de08c2b1994100355a6551833650c05e62176ed204badb1",
-                               1084471296 + 37252864),
+        (4096, 4096, 128256): ("87fc4bcab2fc023023e794ccdd3b2cd157dd7b0a663d2db72e048f6164e6646d",
+                               1084925952 + 36845568),
     },
     "bwd_kernel": {
-        (4096, 4096, 128256): ("3c7e6d9e2249ad598ff936c22ac20055784646526dd6c42c6be3a22ecf1a5fcd",
-                               5942506496 + 2340444672),
+        (4096, 4096, 128256): ("b33d7d69c315ecd43495815e4382193d08254d2c86c9e9ac569b19411547b930",
+                               5460505088 + 1801052672),
     },
 }
 
