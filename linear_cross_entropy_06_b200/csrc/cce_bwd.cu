@@ -571,6 +571,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // dE / dC
       const bool de = it.kind == kDE;
       const bool has = it.begin < it.end;
+      // dC: the onehot terms -scale_r (1 - ls) E_r of the rows r whose target tile here was skipped
+      // and whose target falls in this warp's 32 rows of the tile, in list order. The first two such
+      // entries have this item's 256 columns of E_r loaded by the whole warp at once (16 bytes per
+      // lane), before the accumulator is waited for; at each step the entry's owner lane takes its 64
+      // columns by shuffles. Later entries (several rows targeting this warp's rows) are loaded by
+      // their owner lane at each step.
+      const int x_item = it.s * SLICE;
+      int h_owner0 = -1, h_owner1 = -1;  // warp-uniform: the lane whose row gets held entry 0 / 1
+      float h_coef0 = 0.f, h_coef1 = 0.f;
+      uint4 h_cols0 = make_uint4(0, 0, 0, 0), h_cols1 = make_uint4(0, 0, 0, 0);  // columns x_item + 8 lane
+      int oh_rest = -1;  // warp-uniform: first list entry handled step by step, or -1
+      if (!de && it.oh_begin < it.oh_end) {
+        const int64_t base_v = static_cast<int64_t>(it.key) * BN + q * 32 + A.vocab_start;
+        const int64_t col = x_item + 8 * lane;
+        int held = 0;
+        for (int i0 = it.oh_begin; i0 < it.oh_end && oh_rest < 0; i0 += 32) {
+          int r = 0, owner = -1;
+          if (i0 + lane < it.oh_end) {
+            r = A.oh_rows[i0 + lane];
+            const int64_t o = A.targets[r] - base_v;
+            owner = o >= 0 && o < 32 ? static_cast<int>(o) : -1;
+          }
+          for (unsigned m = __ballot_sync(0xffffffffu, owner >= 0); m != 0; m &= m - 1) {
+            const int k = __ffs(m) - 1;
+            if (held == 2) {
+              oh_rest = i0 + k;
+              break;
+            }
+            const int rk = __shfl_sync(0xffffffffu, r, k), ok = __shfl_sync(0xffffffffu, owner, k);
+            const float ck = -A.scale[rk] * A.onehot_coef;
+            const uint4 cols = col < A.D ? ld_global_nc_v4(A.E + static_cast<int64_t>(rk) * A.D + col)
+                                         : make_uint4(0, 0, 0, 0);
+            if (held == 0) {
+              h_owner0 = ok;
+              h_coef0 = ck;
+              h_cols0 = cols;
+            } else {
+              h_owner1 = ok;
+              h_coef1 = ck;
+              h_cols1 = cols;
+            }
+            ++held;
+          }
+        }
+      }
       if (has) {
         if (!warp_wait(bar(kAccFull + a), (acc_iter >> 1) & 1u)) break;
         tc_fence_after();
@@ -581,43 +626,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         red_release_add(A.counters + A.ctr_b_done + it.chunk, 1);
       }
       if (de && !has) continue;  // nothing to add for this row block in this chunk
-      // dC: onehot terms of rows whose target tile was skipped and whose target is this thread's
-      // row of the tile (at most two remembered; more are rare and handled by a second scan)
-      int oh_r[2] = {-1, -1};
-      float oh_c[2] = {0.f, 0.f};
-      bool oh_more = false;
-      if (!de && it.oh_begin < it.oh_end) {
-        const int64_t my_v = static_cast<int64_t>(it.key) * BN + q * 32 + lane;
-        int n = 0;
-        for (int i = it.oh_begin; i < it.oh_end; ++i) {
-          const int r = A.oh_rows[i];
-          if (A.targets[r] - A.vocab_start != my_v) continue;
-          if (n < 2) {
-            oh_r[n] = r;
-            oh_c[n] = -A.scale[r] * A.onehot_coef;
-          } else {
-            oh_more = true;
-          }
-          ++n;
-        }
-      }
       // After a pair every warp's earlier bulk stores must have read the whole region; between dE / dC
       // items each warp only reuses its own staging images, which next_image() guards.
       if (region_shared && !region_free()) break;
       region_shared = false;
       const int rows_limit = de ? A.N : A.V;
       const int y = it.key * BM + q * 32;
-      // the first matched row's 64 columns for the next step are loaded one step ahead
-      uint4 oh_next[8];
-      auto load_row = [&](int x) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          oh_next[k] = x + 8 * k < A.D ? ld_global_nc_v4(A.E + static_cast<int64_t>(oh_r[0]) * A.D + x + 8 * k)
-                                       : make_uint4(0, 0, 0, 0);
-      };
-      if (oh_r[0] >= 0) load_row(it.s * SLICE);
       for (int p = 0; p < SLICE / 64; ++p) {
-        const int x = it.s * SLICE + 64 * p;
+        const int x = x_item + 64 * p;
         if (x >= A.D) break;
         float v0[32], v1[32];
         if (has) {
@@ -626,43 +642,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) v0[e] = v1[e] = 0.f;
         }
-        if (oh_r[0] >= 0) {  // -scale_r (1 - ls) E_r for those rows
-          auto add_vals = [&](const uint4 (&u8)[8], float coef) {
+        auto add_vals = [&](const uint4 (&u8)[8], float coef) {  // u8: this step's 64 columns
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint32_t w4[4] = {u8[k].x, u8[k].y, u8[k].z, u8[k].w};
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t w4[4] = {u8[k].x, u8[k].y, u8[k].z, u8[k].w};
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                __nv_bfloat162 h;
-                *reinterpret_cast<uint32_t*>(&h) = w4[j];
-                float* dst = k < 4 ? v0 + 8 * k + 2 * j : v1 + 8 * (k - 4) + 2 * j;
-                dst[0] = fmaf(coef, __low2float(h), dst[0]);
-                dst[1] = fmaf(coef, __high2float(h), dst[1]);
-              }
+            for (int j = 0; j < 4; ++j) {
+              __nv_bfloat162 h;
+              *reinterpret_cast<uint32_t*>(&h) = w4[j];
+              float* dst = k < 4 ? v0 + 8 * k + 2 * j : v1 + 8 * (k - 4) + 2 * j;
+              dst[0] = fmaf(coef, __low2float(h), dst[0]);
+              dst[1] = fmaf(coef, __high2float(h), dst[1]);
             }
-          };
-          auto add_row = [&](int r, float coef) {
+          }
+        };
+        auto add_held = [&](const uint4& cols, int owner, float coef) {  // lanes 8p .. 8p + 7 hold the step
+          uint4 u8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            u8[k].x = __shfl_sync(0xffffffffu, cols.x, 8 * p + k);
+            u8[k].y = __shfl_sync(0xffffffffu, cols.y, 8 * p + k);
+            u8[k].z = __shfl_sync(0xffffffffu, cols.z, 8 * p + k);
+            u8[k].w = __shfl_sync(0xffffffffu, cols.w, 8 * p + k);
+          }
+          if (lane == owner) add_vals(u8, coef);
+        };
+        if (h_owner0 >= 0) add_held(h_cols0, h_owner0, h_coef0);
+        if (h_owner1 >= 0) add_held(h_cols1, h_owner1, h_coef1);
+        if (oh_rest >= 0) {  // the rest of the list, each entry by its owner lane
+          const int64_t my_v = static_cast<int64_t>(it.key) * BN + q * 32 + lane;
+          for (int i = oh_rest; i < it.oh_end; ++i) {
+            const int r = A.oh_rows[i];
+            if (A.targets[r] - A.vocab_start != my_v) continue;
             uint4 u8[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               u8[k] = x + 8 * k < A.D ? ld_global_nc_v4(A.E + static_cast<int64_t>(r) * A.D + x + 8 * k)
                                       : make_uint4(0, 0, 0, 0);
-            add_vals(u8, coef);
-          };
-          uint4 cur[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) cur[k] = oh_next[k];
-          if (p + 1 < SLICE / 64 && x + 64 < A.D) load_row(x + 64);
-          add_vals(cur, oh_c[0]);
-          if (oh_r[1] >= 0) add_row(oh_r[1], oh_c[1]);
-          if (oh_more) {
-            const int64_t my_v = static_cast<int64_t>(it.key) * BN + q * 32 + lane;
-            int n = 0;
-            for (int i = it.oh_begin; i < it.oh_end; ++i) {
-              const int r = A.oh_rows[i];
-              if (A.targets[r] - A.vocab_start != my_v) continue;
-              if (n++ >= 2) add_row(r, -A.scale[r] * A.onehot_coef);
-            }
+            add_vals(u8, -A.scale[r] * A.onehot_coef);
           }
         }
         if (!de && A.dc_add != nullptr) {  // the smoothing term, the same for every row of dC
