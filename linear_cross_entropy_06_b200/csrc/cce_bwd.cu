@@ -260,8 +260,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 6) {
     // ---------------- scheduler ----------------
     if (lane == 0) {
-      const int nchunks = *A.nchunks;
-      const int total = A.grp_start[2 * nchunks];
+      // A planning launch that gave up (its bounded barrier wait ran out; the error word is set)
+      // leaves the work lists unfinished: then no item is handed out at all.
+      const bool planned = ld_relaxed(A.err) == 0;
+      const int nchunks = planned ? *A.nchunks : 0;
+      const int total = planned ? A.grp_start[2 * nchunks] : 0;
       int g = 0, g_begin = 0, g_end = A.grp_start[1];  // this CTA's claims only increase
       for (uint32_t k = 0;; ++k) {
         const int idx = static_cast<int>(k % RING);

@@ -36,6 +36,7 @@ __device__ __forceinline__ bool valid_target(int64_t t, int64_t V, int64_t ignor
 // phases separated by grid-wide barriers (bounded waits; a block that gives up records
 // CCE_ERR_DEVICE_TIMEOUT and every block then leaves). Each phase spreads its work over the grid.
 constexpr int kPlanThreads = 1024;
+static_assert(kPlanThreads == 32 * 32, "block_scan keeps one total per warp in 32 lanes");
 constexpr int kFlagTiles = 32;   // vocabulary tiles per flag unit
 constexpr int kFlagGroups = kPlanThreads / kBwdBM;  // flag units per block at a time (128 threads each)
 
@@ -73,26 +74,38 @@ __device__ bool grid_barrier(const PlanCtl& ctl, int round) {
   return ok != 0;
 }
 
-// Exclusive scan of cnt[0..n) into off[0..n] by the calling block (1024 threads), in chunks.
+// Exclusive scan of cnt[0..n) into off[0..n] by the calling block (1024 threads = 32 warps), in
+// chunks of 1024: a shuffle scan inside each warp, then one over the 32 warp totals.
 __device__ void block_scan(const int* __restrict__ cnt, int n, int* __restrict__ off) {
-  __shared__ int buf[kPlanThreads];
+  __shared__ int wsum[32];
   __shared__ int carry;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
   for (int base = 0; base < n; base += kPlanThreads) {
     const int i = base + threadIdx.x;
     const int v = i < n ? cnt[i] : 0;
-    buf[threadIdx.x] = v;
-    __syncthreads();
-    for (int o = 1; o < kPlanThreads; o <<= 1) {
-      const int add = threadIdx.x >= o ? buf[threadIdx.x - o] : 0;
-      __syncthreads();
-      buf[threadIdx.x] += add;
-      __syncthreads();
+    int x = v;  // inclusive scan within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    if (i < n) off[i] = carry + buf[threadIdx.x] - v;
+    if (lane == 31) wsum[w] = x;
     __syncthreads();
-    if (threadIdx.x == kPlanThreads - 1) carry += buf[kPlanThreads - 1];
+    if (w == 0) {  // inclusive scan of the warp totals
+      int t = wsum[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      wsum[lane] = t;
+    }
+    __syncthreads();
+    if (i < n) off[i] = carry + (w > 0 ? wsum[w - 1] : 0) + x - v;
+    __syncthreads();  // every thread has read carry and wsum
+    if (threadIdx.x == 0) carry += wsum[31];
     __syncthreads();
   }
   if (threadIdx.x == 0) off[n] = carry;
@@ -388,10 +401,10 @@ __device__ __forceinline__ int chunk_containing(const int* chunk_t, int n, int t
   return lo;
 }
 
-// The whole plan. Phases (each spread over the grid; a barrier after each):
+// The whole plan. Phases (each spread over the grid; a grid barrier after each from phase 1 on):
 //  0  zero the counters (the backward kernel's too) and the fp32 accumulator of dbias; the row
 //     scales (the fp32 accumulator of dE is zeroed a tenth per phase)
-//  1  tile flags
+//  1  tile flags (run with phase 0, whose results they do not read)
 //  2  per vocabulary tile: ranks of its listed tiles and their count; per row block: its count; the
 //     kept total; per vocabulary tile: rows whose target tile is onehot only, and their dbias terms
 //  3  scans: offsets_t, offsets_b, oh_off (three blocks)
@@ -401,7 +414,7 @@ __device__ __forceinline__ int chunk_containing(const int* chunk_t, int n, int t
 //  6  pair counts per vocabulary tile
 //  7  scan of the pair counts (pstart_t)
 //  8  pairs; chunk work lists and queue group sizes
-//  9  scan of the group sizes (grp_start); the skipped count
+//  9  scan of the group sizes (grp_start); the skipped count: by the last block to finish phase 8
 __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_constant__ PlanArgs A) {
   const BwdPlan& P = A.P;
   const int nb = P.nb, nt = P.nt;
@@ -423,7 +436,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
   // dE_acc is first read by the tensor-core kernel, so its zeroing (bandwidth-bound) is spread over
   // the phases, beside their latency-bound work: one tenth at the start of each phase.
   const int64_t n4 = A.N * A.D / 4;  // D is a multiple of 8
-  auto zero_part = [&](int k) {
+  auto zero_part = [&](int k) {  // k = 0 .. 9
     float4* z = reinterpret_cast<float4*>(A.dE_acc);
     const int64_t lo = n4 * k / 10, hi = n4 * (k + 1) / 10;
     for (int64_t i = lo + gtid; i < hi; i += gthreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -443,10 +456,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     }
     A.scale[r] = A.targets[r] != A.ignore_index ? s : 0.f;
   }
-  if (!grid_barrier(ctl, ++round)) return;
-  zero_part(round);
-
-  // 1
+  // 1 (no barrier before it: the flags read none of the above)
+  zero_part(1);
   {
     const int runs = (nt + kFlagTiles - 1) / kFlagTiles;
     const int64_t units = static_cast<int64_t>(nb) * runs;
@@ -458,7 +469,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     }
   }
   if (!grid_barrier(ctl, ++round)) return;
-  zero_part(round);
+  zero_part(round + 1);
 
   // 2
   for (int t = gwarp; t < nt; t += gwarps) {
@@ -487,14 +498,14 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     if (A.dbias_acc != nullptr) atomicAdd(A.dbias_acc + tr, -A.onehot_coef * A.scale[r]);
   }
   if (!grid_barrier(ctl, ++round)) return;
-  zero_part(round);
+  zero_part(round + 1);
 
   // 3
   if (blockIdx.x == 0) block_scan(P.cnt_t, nt, P.offsets_t);
   if (blockIdx.x == 1 % gridDim.x) block_scan(P.cnt_b, nb, P.offsets_b);
   if (blockIdx.x == 2 % gridDim.x) block_scan(P.oh_cnt, nt, P.oh_off);
   if (!grid_barrier(ctl, ++round)) return;
-  zero_part(round);
+  zero_part(round + 1);
 
   // 4
   for (int64_t i = gtid; i < tiles; i += gthreads) {
@@ -512,7 +523,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
   }
   if (blockIdx.x == gridDim.x - 1) chunk_partition(A);
   if (!grid_barrier(ctl, ++round)) return;
-  zero_part(round);
+  zero_part(round + 1);
   const int nchunks = *reinterpret_cast<volatile int*>(P.nchunks_dev);
 
   // 5
@@ -525,29 +536,35 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
   for (int64_t t = gtid; t < nt; t += gthreads)
     P.chunk_of[t] = chunk_containing(P.chunk_t, nchunks, static_cast<int>(t));
   if (!grid_barrier(ctl, ++round)) return;
-  zero_part(round);
+  zero_part(round + 1);
 
   // 6
   for (int t = gwarp; t < nt; t += gwarps) pair_list_warp(A, t, lane, 0);
   if (!grid_barrier(ctl, ++round)) return;
-  zero_part(round);
+  zero_part(round + 1);
 
   // 7
   if (blockIdx.x == 0) block_scan(P.cnt_t, nt, P.pstart_t);
   if (!grid_barrier(ctl, ++round)) return;
-  zero_part(round);
+  zero_part(round + 1);
 
   // 8
   for (int t = gwarp; t < nt; t += gwarps) pair_list_warp(A, t, lane, 1);
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x) chunk_items_block(A, c, nchunks);
-  if (!grid_barrier(ctl, ++round)) return;
-  zero_part(round);
+  zero_part(9);
 
-  // 9
-  if (blockIdx.x == 0) {
-    block_scan(P.grp_size, 2 * nchunks, P.grp_start);
-    if (threadIdx.x == 0) *A.filtered_tiles = tiles - static_cast<int64_t>(*P.kept_total);
+  // 9, by the last block to finish phase 8 (counted on the barrier counter; no grid barrier)
+  __shared__ int last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last = atomicAdd(ctl.bar, 1) == (round + 1) * static_cast<int>(gridDim.x) - 1;
   }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();  // the other blocks' grp_size entries are visible
+  block_scan(P.grp_size, 2 * nchunks, P.grp_start);
+  if (threadIdx.x == 0) *A.filtered_tiles = tiles - static_cast<int64_t>(*P.kept_total);
 }
 
 // The element-wise steps of the backward after the tensor-core kernel, in two launches:
