@@ -53,8 +53,8 @@ TRAFFIC_BYTES = {
                                1084925952 + 36845568),
     },
     "bwd_kernel": {
-        (4096, 4096, 128256): ("b33d7d69c315ecd43495815e4382193d08254d2c86c9e9ac569b19411547b930",
-                               5460505088 + 1801052672),
+        (4096, 4096, 128256): ("89cc70c3ff0b1bb5423cbfd1ea8fab1f51e2643199001b85d706b0b9a5029aad",
+                               5470501632 + 1791983872),
     },
 }
 
@@ -418,6 +418,44 @@ def run_ours(args, world, rank, local):
         e2e = measure_e2e(copy_c=True)
         e2e_resident = measure_e2e(copy_c=False)
 
+    # Context, not the product (the pages' own comparison): the logits materialised in bf16 by a
+    # cuBLAS matmul and torch's cross_entropy, forward and backward through autograd, on the same
+    # inputs, timed like the steps above (L2 flushed between steps).
+    def measure_torch_ce(steps=5, warmup=2):
+        e_, c_ = E.detach().requires_grad_(True), C.detach().requires_grad_(True)
+
+        def run():
+            logits = e_ @ c_.t()
+            loss = torch.nn.functional.cross_entropy(logits, t, ignore_index=-100, reduction=w.reduction)
+            loss.backward(g if w.reduction == "none" else None)
+            e_.grad = c_.grad = None
+
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        try:
+            for _ in range(warmup):
+                run()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for k in range(steps):
+                flush.fill_(k & 0xFF)
+                evs[k][0].record()
+                run()
+                evs[k][1].record()
+            torch.cuda.synchronize()
+        except torch.cuda.OutOfMemoryError:
+            return {"skipped": "out of memory"}
+        ms = [a.elapsed_time(b) for a, b in evs]
+        return {"value": N * steps / (sum(ms) / 1e3), "unit": "tokens/s", "ms_per_step": statistics.mean(ms),
+                "ms_per_step_median": statistics.median(ms), "steps": steps,
+                "peak_extra_bytes": torch.cuda.max_memory_allocated(dev) - base,
+                "what": "bf16 logits E @ C.T (cuBLAS) + torch.nn.functional.cross_entropy, forward + backward "
+                        "through autograd; context, not a target"}
+
+    comparators = None
+    if world == 1 and not args.no_compare:
+        comparators = {"torch_standard_ce": measure_torch_ce()}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         rows = args.cpu_rows
@@ -451,6 +489,7 @@ def run_ours(args, world, rank, local):
         "e2e": e2e,
         "e2e_classifier_resident": e2e_resident,
         "cpu_baseline": cpu,
+        "comparators": comparators,
     }
     print(json.dumps(line), flush=True)
 
@@ -468,6 +507,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1536)
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-compare", action="store_true", help="skip the torch standard cross-entropy comparator")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
