@@ -470,6 +470,7 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w, world, (N, D, V)),
         "ms_per_step_median": statistics.median(step_ms), "ms_per_step_min": min(step_ms),
+        "ms_per_step_each": [round(x, 4) for x in step_ms],
         "tensor_peak_frac": {"achieved_tflops": path_tflops, "peak": peak_tf, "frac": path_tflops / peak_tf,
                              "frac_sustained": path_tflops / peak_sus, "peak_sustained": peak_sus,
                              "peak_kind": f"bf16_tflops ({peak_kind})",
