@@ -95,7 +95,7 @@ class ClockSampler:
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,power.limit")
 
     def __init__(self, index: int):
         self.index = index
@@ -138,8 +138,10 @@ class ClockSampler:
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
         busy = [s for s in sm if s > 0.5 * (max(sm) if sm else 0)]
         power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        limit = [float(r[9]) for r in rows if len(r) > 9 and r[9].replace(".", "").isdigit()]
         return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None}
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None,
+                "power_limit_w": max(limit) if limit else None}
 
 
 def dist_setup():

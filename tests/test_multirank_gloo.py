@@ -124,10 +124,10 @@ def test_clock_sampler_parses_samples_and_reasons(monkeypatch):
     import bench
 
     samples = [
-        "0, 345, 1965, 120.5, 0x0, Not Active, Not Active, Not Active, Not Active",
-        "0, 1965, 1965, 650.0, 0x4, Not Active, Not Active, Not Active, Active",
-        "0, 1950, 1965, 700.2, 0x4, Not Active, Not Active, Not Active, Active",
-        "0, 1905, 1965, 710.9, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, 345, 1965, 120.5, 0x0, Not Active, Not Active, Not Active, Not Active, 1000.00",
+        "0, 1965, 1965, 650.0, 0x4, Not Active, Not Active, Not Active, Active, 1000.00",
+        "0, 1950, 1965, 700.2, 0x4, Not Active, Not Active, Not Active, Active, 1000.00",
+        "0, 1905, 1965, 710.9, 0x0, Not Active, Not Active, Not Active, Not Active, 1000.00",
     ]
 
     class FakeSmi:
@@ -150,7 +150,7 @@ def test_clock_sampler_parses_samples_and_reasons(monkeypatch):
     assert out["sm_mhz"] == 1950.0  # median of 1965, 1950, 1905; the idle 345 is left out
     assert out["sm_max_mhz"] == 1965.0
     assert out["reasons"] == ["sw_power_cap"]
-    assert out["samples"] == 4 and out["power_w_max"] == 710.9
+    assert out["samples"] == 4 and out["power_w_max"] == 710.9 and out["power_limit_w"] == 1000.0
     assert not os.path.exists(c.path)
 
 
