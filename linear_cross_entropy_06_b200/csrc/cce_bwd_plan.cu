@@ -177,7 +177,8 @@ __device__ void tile_flags_unit(const PlanArgs& A, int group, int b, int t0) {
   wmax[group][tid >> 5][lane] = warp_column_max32(mt, lane);  // lane k: the warp's max of tile t0 + k
   named_barrier(group + 1, kBwdBM);
   if (tid < kFlagTiles && t0 + tid < nt) {
-    const float m = fmaxf(fmaxf(wmax[group][0][tid], wmax[group][1][tid]), fmaxf(wmax[group][2][tid], wmax[group][3][tid]));
+    const float m =
+        fmaxf(fmaxf(wmax[group][0][tid], wmax[group][1][tid]), fmaxf(wmax[group][2][tid], wmax[group][3][tid]));
     const bool keep = !A.filter_on || m >= A.ln_eps;
     A.P.flags[static_cast<int64_t>(b) * nt + t0 + tid] = keep ? 1 : (any_target[group][tid] ? 2 : 0);
   }
@@ -770,7 +771,8 @@ cudaError_t launch_empty_tiles(const BwdFinalize& F, int num_sms, cudaStream_t s
   const int64_t es = F.dc_bf16 ? 2 : 4, rowbytes = F.D * es;
   // whole rows when one fits the image (up to 128 of them); otherwise windows of whole 16-byte pieces
   const int64_t win = rowbytes <= kFillImageBytes ? F.D : kFillImageBytes / es / 8 * 8;
-  const int image_rows = static_cast<int>(rowbytes <= kFillImageBytes ? std::min<int64_t>(kBwdBN, kFillImageBytes / rowbytes) : 1);
+  const int image_rows =
+      static_cast<int>(rowbytes <= kFillImageBytes ? std::min<int64_t>(kBwdBN, kFillImageBytes / rowbytes) : 1);
   const size_t smem = static_cast<size_t>(image_rows * win * es);
   cudaError_t e = cudaFuncSetAttribute(empty_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kFillImageBytes));
