@@ -348,6 +348,10 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
     PA.bar = &w.hdr->bar;
     PA.err = &w.hdr->err;
     PA.timeout_ns = cce::wait_timeout_ns();
+    // Failure-detection test hook: CCE_TEST_INJECT_STALL=3 makes the planning launch's first grid
+    // barrier wait run out (reported as CCE_ERR_DEVICE_TIMEOUT; the backward then hands out no work).
+    const char* stall = std::getenv("CCE_TEST_INJECT_STALL");
+    PA.inject_stall = (stall != nullptr && stall[0] == '3') ? 1 : 0;
     CCE_TRY(cce::launch_bwd_plan(PA, num_sms, s));
   }
   // Label smoothing: the ls / V part of every row's target is a rank-one term, added exactly:

@@ -469,6 +469,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
       if (u < units) tile_flags_unit(A, group, static_cast<int>(u / runs), static_cast<int>(u % runs) * kFlagTiles);
     }
   }
+  if (A.inject_stall && blockIdx.x == 0) return;  // test hook: the other blocks' barrier wait runs out
   if (!grid_barrier(ctl, ++round)) return;
   zero_part(round + 1);
 

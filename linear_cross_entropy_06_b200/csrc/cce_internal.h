@@ -177,14 +177,15 @@ struct PlanArgs {
   int* bar;                // grid barrier counter, zero at launch
   int* err;
   uint64_t timeout_ns;
+  int inject_stall;        // test hook: block 0 leaves before the first grid barrier, whose wait then runs out
 };
 // One cooperative launch: the row scales, the tile flags, both tile lists, the pair list, the
 // chunks' work lists and queue groups, the onehot-only rows, and the skipped count.
 cudaError_t launch_bwd_plan(const PlanArgs& A, int num_sms, cudaStream_t s);
 cudaError_t launch_bwd(const BwdLaunch& L, cudaStream_t s);
-// Everything the backward computes after its tensor-core kernel (cce_bwd_plan.cu, one launch): the
-// last terms of dE and its conversion, the dC rows of the vocabulary tiles no row block lists, and
-// dbias. See bwd_finalize_kernel.
+// Everything the backward computes after its tensor-core kernel (cce_bwd_plan.cu, two launches): the
+// dC rows of the vocabulary tiles no row block lists (empty_tiles_kernel), the last terms of dE and
+// its conversion, and dbias (bwd_finalize_kernel).
 struct BwdFinalize {
   int64_t N, D, V, vs, ignore_index;
   int nt;

@@ -4,8 +4,9 @@ Forward: the kernel's producer is told (through a test-only environment switch, 
 time) to issue no loads, so the MMA warp's wait on the first stage gives up after
 CCE_WAIT_TIMEOUT_MS. Backward: the dE items of the first vocabulary chunk are told to wait for
 one gradient tile more than the recompute stores, so their wait on a counter raised by other
-CTAs gives up; the other CTAs see the recorded error and stop too. In both cases the kernel
-records CCE_ERR_DEVICE_TIMEOUT and exits cleanly; the test checks the status and that the same
+CTAs gives up; the other CTAs see the recorded error and stop too. Planning: one block of the
+cooperative planning launch leaves before the first grid barrier, so the other blocks' wait there
+gives up. In every case the kernel records CCE_ERR_DEVICE_TIMEOUT and exits cleanly; the test checks the status and that the same
 process then computes correct results again. Run in a child process so that the environment
 switches cannot leak into other tests.
 """
@@ -78,6 +79,22 @@ print("RECOVERED", rel <= 1e-2)
 def test_backward_dependency_wait_timeout_is_reported_and_context_survives():
     env = dict(os.environ, CCE_ROOT=ROOT, CCE_WAIT_TIMEOUT_MS="200")
     out = subprocess.run([sys.executable, "-c", CHILD_BWD], env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert "STATUS 5" in out.stdout, out.stdout  # CCE_ERR_DEVICE_TIMEOUT
+    assert "RECOVERED True" in out.stdout, out.stdout
+
+
+CHILD_PLAN = CHILD_BWD.replace('os.environ["CCE_TEST_INJECT_STALL"] = "2"', 'os.environ["CCE_TEST_INJECT_STALL"] = "3"')
+
+
+def test_planning_barrier_timeout_is_reported_and_context_survives():
+    """The planning launch's first grid barrier: one block leaves before it (test hook), so the
+    others' bounded wait runs out and records CCE_ERR_DEVICE_TIMEOUT; the tensor-core kernel then
+    hands out no work from the unfinished plan, and the next backward on the same context is
+    correct."""
+    assert CHILD_PLAN != CHILD_BWD
+    env = dict(os.environ, CCE_ROOT=ROOT, CCE_WAIT_TIMEOUT_MS="200")
+    out = subprocess.run([sys.executable, "-c", CHILD_PLAN], env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
     assert "STATUS 5" in out.stdout, out.stdout  # CCE_ERR_DEVICE_TIMEOUT
     assert "RECOVERED True" in out.stdout, out.stdout
