@@ -7,9 +7,11 @@ Elementwise: |gpu - oracle| <= 3e-2 * rms(that row of the oracle) + 3e-2 * |orac
 floor = 8 * 2^-23 * max|LSE| * max(scale_r) * max|operand| is the absolute error fp32 leaves in one
 term of G = scale_r * (exp(z - LSE) - y) when p is close to 1 (p - 1 is then far below the fp32
 resolution of z and LSE), carried through one product with E (dC) or C (dE). It matters only for
-rows of dC or dE made of such terms alone. Rows of ignored tokens in dE are exactly +0 and
-skipped-tile counts equal the oracle's (unless the oracle reports a tile whose margin lies within
-2e-3 of ln eps, in which case the difference is bounded by that number).
+rows of dC or dE made of such terms alone; when every row is (one very peaked row, say), the
+relative Frobenius bound gives way to the same floor on the whole matrix, floor * sqrt(elements).
+Rows of ignored tokens in dE are exactly +0 and skipped-tile counts equal the oracle's (unless the
+oracle reports a tile whose margin lies within 2e-3 of ln eps, in which case the difference is
+bounded by that number).
 """
 import math
 import os
@@ -87,6 +89,12 @@ def fp32_floor(lse, scale, operand):
     return 8 * 2.0 ** -23 * max(_absmax(lse), 1.0) * _absmax(scale) * _absmax(operand)
 
 
+def frob_ok(got, want, tol, floor=0.0):
+    """Relative Frobenius error within tol, or an absolute error within the fp32 floor per element
+    (for gradients made only of terms p - 1 with p rounded to 1 in fp32)."""
+    return rel_frob(got, want) <= tol or np.linalg.norm(got - want) <= floor * np.sqrt(got.size)
+
+
 def assert_close_elementwise(a, b, what, floor=0.0):
     # Row-wise scale: a row of dE or dC is one column of G times E or C, so its rounding error
     # grows with that row's own magnitude (rows of popular targets are far larger than the rest).
@@ -96,8 +104,8 @@ def assert_close_elementwise(a, b, what, floor=0.0):
 
 
 def assert_grads(g_dE, g_dC, o_dE, o_dC, tol, what="", floor_dE=0.0, floor_dC=0.0):
-    assert rel_frob(g_dE, o_dE) <= tol, f"{what} dE rel-Frobenius {rel_frob(g_dE, o_dE):.3e}"
-    assert rel_frob(g_dC, o_dC) <= tol, f"{what} dC rel-Frobenius {rel_frob(g_dC, o_dC):.3e}"
+    assert frob_ok(g_dE, o_dE, tol, floor_dE), f"{what} dE rel-Frobenius {rel_frob(g_dE, o_dE):.3e}"
+    assert frob_ok(g_dC, o_dC, tol, floor_dC), f"{what} dC rel-Frobenius {rel_frob(g_dC, o_dC):.3e}"
     assert_close_elementwise(g_dE, o_dE, what + " dE", floor_dE)
     assert_close_elementwise(g_dC, o_dC, what + " dC", floor_dC)
 

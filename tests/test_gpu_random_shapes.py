@@ -1,0 +1,45 @@
+"""GPU parity on 50 randomly drawn small problems (hypothesis, derandomized: the same draws every run).
+
+Every draw runs the CUDA path through the C ABI and the fp64 oracle on the same seeded inputs, with
+tile skipping off and at eps = 2^-12, and compares the loss, the LSE, dE, dC and dbias with the
+tolerances of the other parity tests (`test_gpu_bias.check_bias`). The draws cover shapes the fixed
+tests do not: N down to 1, every D that is a multiple of 8 up to 520 (one 256-column slice of dE/dC
+and a partial one), V from 1 to 3000 (a ragged last vocabulary tile), every reduction, ignored rows,
+a classifier bias, label smoothing and the z-loss, and peaked inputs that make tiles skip.
+
+One pair is left out: V = 1 with label smoothing. With one class LSE = z_t, the loss is the same for
+every input and every gradient is zero; the library computes that zero as the sum of the gradient
+tile scale_r ((1 + 2 zl LSE) p - (1 - ls)) = scale_r ls, rounded to bf16, and the fp32 rank-one
+smoothing term -scale_r ls / V, so what remains is the bf16 rounding of scale_r ls (about 2^-9 of
+it) times C, which no bound relative to a zero result accepts.
+"""
+import numpy as np
+import pytest
+import torch
+from hypothesis import HealthCheck, assume, given, settings
+from hypothesis import strategies as st
+
+from linear_cross_entropy_06_b200.inputs import make_inputs
+
+from test_gpu_bias import check_bias, make_bias
+
+pytestmark = pytest.mark.gpu
+
+
+@settings(max_examples=50, derandomize=True, deadline=None,
+          suppress_health_check=[HealthCheck.function_scoped_fixture, HealthCheck.too_slow])
+@given(N=st.integers(1, 700), D8=st.integers(1, 65), V=st.integers(1, 4000),
+       reduction=st.sampled_from(["mean", "sum", "none"]), with_bias=st.booleans(),
+       ls=st.sampled_from([0.0, 0.1]), zl=st.sampled_from([0.0, 1e-4]), ignore=st.sampled_from([0.0, 0.1]),
+       peaked=st.booleans(), seed=st.integers(0, 10_000))
+def test_random_problem_matches_the_oracle(device, N, D8, V, reduction, with_bias, ls, zl, ignore, peaked, seed):
+    assume(not (V == 1 and ls > 0))
+    D = 8 * D8
+    if peaked:  # E rows pulled toward their target's classifier row: large margins, skipped tiles
+        inp = make_inputs("llama3.2-1b-head", N=N, D=D, V=V, seed=seed, alpha=16.0, ignore_frac=ignore)
+    else:
+        inp = make_inputs("tiny", N=N, D=D, V=V, seed=seed, ignore_frac=ignore)
+    g = torch.from_numpy(np.random.default_rng(seed + 1).standard_normal(N).astype(np.float32)) \
+        if reduction == "none" else torch.tensor([0.75])
+    bias = make_bias(V, seed + 2, scale=0.5) if with_bias else None
+    check_bias(inp, bias, device, reduction, grad_out=g, ls=ls, zl=zl)
