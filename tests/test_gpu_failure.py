@@ -7,8 +7,8 @@ one gradient tile more than the recompute stores, so their wait on a counter rai
 CTAs gives up; the other CTAs see the recorded error and stop too. Planning: one block of the
 cooperative planning launch leaves before the first grid barrier, so the other blocks' wait there
 gives up. In every case the kernel records CCE_ERR_DEVICE_TIMEOUT and exits cleanly; the test
-checks the status and that the same process then computes correct results again. Run in a child process so that the environment
-switches cannot leak into other tests.
+checks the status and that the same process then computes correct results again. Run in a child
+process so that the environment switches cannot leak into other tests.
 """
 import os
 import subprocess
