@@ -5,7 +5,8 @@ tile skipping off and at eps = 2^-12, and compares the loss, the LSE, dE, dC and
 tolerances of the other parity tests (`test_gpu_bias.check_bias`). The draws cover shapes the fixed
 tests do not: N down to 1, every D that is a multiple of 8 up to 520 (one 256-column slice of dE/dC
 and a partial one), V from 1 to 3000 (a ragged last vocabulary tile), every reduction, ignored rows,
-a classifier bias, label smoothing and the z-loss, and peaked inputs that make tiles skip.
+a classifier bias, label smoothing and the z-loss, peaked inputs that make tiles skip, and bf16 or
+fp32 outputs.
 
 One pair is left out: V = 1 with label smoothing. With one class LSE = z_t, the loss is the same for
 every input and every gradient is zero; the library computes that zero as the sum of the gradient
@@ -31,8 +32,9 @@ pytestmark = pytest.mark.gpu
 @given(N=st.integers(1, 700), D8=st.integers(1, 65), V=st.integers(1, 4000),
        reduction=st.sampled_from(["mean", "sum", "none"]), with_bias=st.booleans(),
        ls=st.sampled_from([0.0, 0.1]), zl=st.sampled_from([0.0, 1e-4]), ignore=st.sampled_from([0.0, 0.1]),
-       peaked=st.booleans(), seed=st.integers(0, 10_000))
-def test_random_problem_matches_the_oracle(device, N, D8, V, reduction, with_bias, ls, zl, ignore, peaked, seed):
+       peaked=st.booleans(), out_fp32=st.booleans(), seed=st.integers(0, 10_000))
+def test_random_problem_matches_the_oracle(device, N, D8, V, reduction, with_bias, ls, zl, ignore, peaked, out_fp32,
+                                           seed):
     assume(not (V == 1 and ls > 0))
     D = 8 * D8
     if peaked:  # E rows pulled toward their target's classifier row: large margins, skipped tiles
@@ -42,4 +44,4 @@ def test_random_problem_matches_the_oracle(device, N, D8, V, reduction, with_bia
     g = torch.from_numpy(np.random.default_rng(seed + 1).standard_normal(N).astype(np.float32)) \
         if reduction == "none" else torch.tensor([0.75])
     bias = make_bias(V, seed + 2, scale=0.5) if with_bias else None
-    check_bias(inp, bias, device, reduction, grad_out=g, ls=ls, zl=zl)
+    check_bias(inp, bias, device, reduction, grad_out=g, out_fp32=out_fp32, ls=ls, zl=zl)

@@ -12,6 +12,8 @@ side, must be the oracle's tile by tile.
 import numpy as np
 import pytest
 import torch
+from hypothesis import HealthCheck, assume, given, settings
+from hypothesis import strategies as st
 
 from linear_cross_entropy_06_b200 import ops
 from linear_cross_entropy_06_b200.inputs import make_inputs
@@ -19,7 +21,7 @@ from linear_cross_entropy_06_b200.vocab_parallel import shard_range
 from oracle import cce_oracle as O
 
 from test_gpu_bias import make_bias
-from test_gpu_parity import (EPS, LOSS_TOL, assert_close_elementwise, assert_skip_decisions, fp32_floor,
+from test_gpu_parity import (EPS, LOSS_TOL, assert_close_elementwise, assert_skip_decisions, fp32_floor, frob_ok,
                              oracle_decisions, rel_frob)
 
 pytestmark = pytest.mark.gpu
@@ -61,6 +63,32 @@ def run_shards(inp, bias, device, shards, reduction, eps, g, ls, zl):
                 filtered=filtered)
 
 
+def check_shards(inp, bias, device, shards, reduction, g, ls, zl):
+    """The shards' merged loss, LSE and count, their gradients put together, and their skip
+    decisions side by side, against the oracle of the whole problem (skipping off and on)."""
+    N, V = inp.E.shape[0], inp.C.shape[0]
+    g_or = g.numpy() if reduction == "none" else float(g.reshape(-1)[0])
+    tm, tn = ops.backward_tile_shape()
+    f = O.forward(inp.E, inp.C, inp.targets, -100, reduction, bias=bias, label_smoothing=ls, z_loss=zl)
+    sc = O.row_scale(inp.targets, -100, reduction, g_or, f.count) * (1.0 + 2.0 * zl * np.abs(f.lse).max())
+    for eps in (0.0, EPS):
+        o = O.backward(inp.E, inp.C, inp.targets, g_or, -100, reduction, eps, tm, tn,
+                       bias=np.zeros(V) if bias is None else bias, label_smoothing=ls, z_loss=zl)
+        r = run_shards(inp, bias, device, shards, reduction, eps, g, ls, zl)
+        assert np.abs(r["loss"].reshape(np.shape(f.loss)) - f.loss).max() <= LOSS_TOL * (
+            max(f.count, 1) if reduction == "sum" else 1)
+        assert np.abs(r["lse"] - f.lse).max() <= LOSS_TOL
+        assert r["count"] == f.count
+        for name, got, want, operand in (("dE", r["dE"], o.dE, inp.C), ("dC", r["dC"], o.dC, inp.E),
+                                         ("dbias", r["dbias"][:, None], o.dbias[:, None], 1.0)):
+            floor = fp32_floor(f.lse, sc, operand)
+            assert frob_ok(got, want, 1e-2, floor), (name, eps, rel_frob(got, want))
+            assert_close_elementwise(got, want, f"{name} eps={eps}", floor)
+        assert_skip_decisions(r["skipped"], r["filtered"], *oracle_decisions(o.margin, eps), f"{shards} shards")
+        ign = (inp.targets == -100).numpy()
+        assert not r["dE"][ign].any()
+
+
 @pytest.mark.parametrize("shards", [2, 3])
 @pytest.mark.parametrize("variant", ["plain", "bias+smoothing+z-loss"])
 @pytest.mark.parametrize("reduction", ["mean", "none"])
@@ -71,24 +99,28 @@ def test_vocabulary_shards_match_the_whole_problem(device, shards, variant, redu
     bias, ls, zl = (make_bias(V, 72, scale=0.5), 0.1, 1e-4) if variant != "plain" else (None, 0.0, 0.0)
     g = torch.from_numpy(np.random.default_rng(73).standard_normal(N).astype(np.float32)) if reduction == "none" \
         else torch.tensor([1.0])
-    g_or = g.numpy() if reduction == "none" else 1.0
-    tm, tn = ops.backward_tile_shape()
-    f = O.forward(inp.E, inp.C, inp.targets, -100, reduction, bias=bias, label_smoothing=ls, z_loss=zl)
-    sc = O.row_scale(inp.targets, -100, reduction, g_or, f.count) * (1.0 + 2.0 * zl * np.abs(f.lse).max())
-    for eps in (0.0, EPS):
-        o = O.backward(inp.E, inp.C, inp.targets, g_or, -100, reduction, eps, tm, tn,
-                       bias=np.zeros(V) if bias is None else bias, label_smoothing=ls, z_loss=zl)
-        r = run_shards(inp, bias, device, shards, reduction, eps, g, ls, zl)
-        assert np.abs(r["loss"].reshape(np.shape(f.loss)) - f.loss).max() <= LOSS_TOL
-        assert np.abs(r["lse"] - f.lse).max() <= LOSS_TOL
-        assert r["count"] == f.count
-        for name, got, want, operand in (("dE", r["dE"], o.dE, inp.C), ("dC", r["dC"], o.dC, inp.E),
-                                         ("dbias", r["dbias"][:, None], o.dbias[:, None], 1.0)):
-            assert rel_frob(got, want) <= 1e-2, (name, eps, rel_frob(got, want))
-            assert_close_elementwise(got, want, f"{name} eps={eps}", fp32_floor(f.lse, sc, operand))
-        assert_skip_decisions(r["skipped"], r["filtered"], *oracle_decisions(o.margin, eps), f"{shards} shards")
-        ign = (inp.targets == -100).numpy()
-        assert not r["dE"][ign].any()
+    check_shards(inp, bias, device, shards, reduction, g, ls, zl)
+
+
+@settings(max_examples=20, derandomize=True, deadline=None,
+          suppress_health_check=[HealthCheck.function_scoped_fixture, HealthCheck.too_slow])
+@given(shards=st.integers(2, 5), N=st.integers(1, 400), D8=st.integers(1, 40), V=st.integers(129, 3000),
+       reduction=st.sampled_from(["mean", "sum", "none"]), with_bias=st.booleans(),
+       ls=st.sampled_from([0.0, 0.1]), zl=st.sampled_from([0.0, 1e-4]), peaked=st.booleans(),
+       seed=st.integers(0, 10_000))
+def test_random_shards_match_the_whole_problem(device, shards, N, D8, V, reduction, with_bias, ls, zl, peaked,
+                                               seed):
+    """Random problems and shard counts (every shard at least one 128-row tile of the classifier)."""
+    assume(V > 128 * (shards - 1))
+    D = 8 * D8
+    if peaked:
+        inp = make_inputs("llama3.2-1b-head", N=N, D=D, V=V, seed=seed, alpha=16.0, ignore_frac=0.1)
+    else:
+        inp = make_inputs("tiny", N=N, D=D, V=V, seed=seed, ignore_frac=0.1)
+    g = torch.from_numpy(np.random.default_rng(seed + 1).standard_normal(N).astype(np.float32)) \
+        if reduction == "none" else torch.tensor([0.75])
+    bias = make_bias(V, seed + 2, scale=0.5) if with_bias else None
+    check_shards(inp, bias, device, shards, reduction, g, ls, zl)
 
 
 def test_shards_agree_with_the_unsharded_path(device):
