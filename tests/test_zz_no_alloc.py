@@ -13,6 +13,8 @@ import ctypes
 import numpy as np
 import pytest
 import torch
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
 
 from linear_cross_entropy_06_b200 import ops
 from linear_cross_entropy_06_b200.inputs import make_inputs
@@ -107,3 +109,28 @@ def test_noalloc_device_error_gives_nan_loss_then_recovers(device, reduction):
     f = O.forward(inp.E, inp.C, inp.targets, -100, reduction)
     assert np.abs(loss.double().cpu().numpy().reshape(np.shape(f.loss)) - f.loss).max() <= LOSS_TOL
     assert int(count.item()) == f.count
+
+
+@settings(max_examples=25, derandomize=True, deadline=None,
+          suppress_health_check=[HealthCheck.function_scoped_fixture, HealthCheck.too_slow])
+@given(N=st.integers(1, 700), D8=st.integers(1, 65), V=st.integers(1, 4000),
+       reduction=st.sampled_from(["mean", "sum", "none"]), with_bias=st.booleans(),
+       ls=st.sampled_from([0.0, 0.1]), zl=st.sampled_from([0.0, 1e-4]), seed=st.integers(0, 10_000))
+def test_noalloc_random_problems_match_the_oracle(device, N, D8, V, reduction, with_bias, ls, zl, seed):
+    """Random shapes and options, one call after another on the shared array: the loss, LSE and
+    count of each against the fp64 oracle."""
+    D = 8 * D8
+    inp = make_inputs("tiny", N=N, D=D, V=V, seed=seed, ignore_frac=0.1)
+    bias = None
+    if with_bias:
+        bias = torch.from_numpy(np.random.default_rng(seed + 2).standard_normal(V).astype(np.float32) * 0.5)
+        bias = bias.to(torch.bfloat16)
+    E, C, t = inp.E.to(device), inp.C.to(device), inp.targets.to(device)
+    st_, loss, lse, _, count = _noalloc(E, C, t, reduction, None if bias is None else bias.to(device), ls, zl)
+    assert st_ == 0, ops.load_library().cce_last_error_message()
+    torch.cuda.synchronize()
+    f = O.forward(inp.E, inp.C, inp.targets, -100, reduction, bias=bias, label_smoothing=ls, z_loss=zl)
+    assert int(count.item()) == f.count
+    tol = LOSS_TOL * (max(f.count, 1) if reduction == "sum" else 1)
+    assert np.abs(loss.double().cpu().numpy().reshape(np.shape(f.loss)) - f.loss).max() <= tol
+    assert np.abs(lse.double().cpu().numpy() - f.lse).max() <= LOSS_TOL
