@@ -49,12 +49,12 @@ KERNEL_SOURCES = {  # the kernel and what sets up its work (maps, plan, chunking
 }
 TRAFFIC_BYTES = {
     "fwd_lse_kernel": {
-        (4096, 4096, 128256): ("87fc4bcab2fc023023e794ccdd3b2cd157dd7b0a663d2db72e048f6164e6646d",
-                               1084925952 + 36845568),
+        (4096, 4096, 128256): ("78bc8104dbff3216f1b60add73745a7a674307a6706e88a5069dc98355b54357",
+                               1084998144 + 34948096),
     },
     "bwd_kernel": {
-        (4096, 4096, 128256): ("89cc70c3ff0b1bb5423cbfd1ea8fab1f51e2643199001b85d706b0b9a5029aad",
-                               5470501632 + 1791983872),
+        (4096, 4096, 128256): ("2e8ba86bffc35cbda45431d27e2ceb35b98437723bf78a252734429621dc50f7",
+                               5480887296 + 1792022784),
     },
 }
 
