@@ -445,7 +445,9 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   L.num_sms = num_sms;
 
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[0], s));
-  CCE_TRY(cce::launch_bwd(L, s));
+  // launches that overlap the previous kernel's tail, unless a timing event sits between them
+  const bool timed = g_bwd_ev[0] && g_bwd_ev[1];
+  CCE_TRY(cce::launch_bwd(L, !timed, s));
   if (g_bwd_ev[0] && g_bwd_ev[1]) CCE_TRY(cudaEventRecord(g_bwd_ev[1], s));
   // the rest: dC rows of vocabulary tiles no row block lists, then dE's last terms and conversion,
   // and dbias
@@ -475,7 +477,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   F.dc_bf16 = c32 ? 0 : 1;
   F.dbias_acc = dbias_acc;
   F.dbias_out = (dbias != nullptr && !c32) ? dbias : nullptr;
-  CCE_TRY(cce::launch_empty_tiles(F, num_sms, s));
+  CCE_TRY(cce::launch_empty_tiles(F, num_sms, !timed, s));
   CCE_TRY(cce::launch_bwd_finalize(F, num_sms, s));
   return CCE_OK;
 }
@@ -600,7 +602,8 @@ cce_status cce_forward(const cce_problem* p, const void* E, const void* C, const
   F.lse = lse;
   F.loss = loss;
   F.count = count;
-  CCE_TRY(cce::launch_fwd_finish(F, s));
+  // overlap the finish's launch with the tensor-core kernel's tail, unless a timing event sits between
+  CCE_TRY(cce::launch_fwd_finish(F, has_rows && !(g_fwd_ev[0] && g_fwd_ev[1]), s));
   return CCE_OK;
 }
 
@@ -675,7 +678,7 @@ cce_status cce_forward_partial(const cce_problem* p, const void* E, const void* 
   F.lse = partial;
   F.zt_out = partial + N;
   F.zs_out = partial + 2 * N;
-  CCE_TRY(cce::launch_fwd_finish(F, s));
+  CCE_TRY(cce::launch_fwd_finish(F, !(g_fwd_ev[0] && g_fwd_ev[1]), s));  // N > 0: the tensor-core kernel ran
   return CCE_OK;
 }
 

@@ -71,6 +71,7 @@ __global__ void __launch_bounds__(kFinishWarps * 32) fwd_finish_kernel(const __g
   __shared__ double s_sum[kReduceThreads];
   __shared__ long long s_cnt[kReduceThreads];
   __shared__ int s_last;
+  wait_for_previous_grid();  // the tensor-core kernel's sub-tile statistics and picked logits
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kFinishWarps;
   const int64_t N = F.N, T = F.T, D = F.D;
@@ -286,9 +287,15 @@ int grid_for(int64_t items, int per_block, int cap) {
 
 }  // namespace
 
-cudaError_t launch_fwd_finish(const FwdFinish& F, cudaStream_t s) {
+cudaError_t launch_fwd_finish(const FwdFinish& F, bool after_kernel, cudaStream_t s) {
   const int64_t blocks = (F.N + kFinishWarps - 1) / kFinishWarps;
-  fwd_finish_kernel<<<static_cast<unsigned>(blocks > 0 ? blocks : 1), kFinishWarps * 32, 0, s>>>(F);
+  const dim3 grid(static_cast<unsigned>(blocks > 0 ? blocks : 1)), block(kFinishWarps * 32);
+  if (after_kernel) {
+    const cudaError_t e = launch_after_previous(fwd_finish_kernel, grid, block, 0, s, F);
+    if (e != cudaSuccess) return e;
+  } else {
+    fwd_finish_kernel<<<grid, block, 0, s>>>(F);
+  }
   note_launches(1);
   return cudaGetLastError();
 }

@@ -253,6 +253,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  wait_for_previous_grid();  // the plan (and the zeroed counters) of the planning launch
   const WaitCtl wc{abort_flag, A.err, A.timeout_ns};
   const int num_kb = (A.D + BK - 1) / BK;
   auto buffer = [&](int chunk) { return A.gscratch + static_cast<size_t>(chunk % kGradBuffers) * A.buf_bytes; };
@@ -756,10 +757,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 }  // namespace
 
-cudaError_t launch_bwd(const BwdLaunch& L, cudaStream_t s) {
+cudaError_t launch_bwd(const BwdLaunch& L, bool after_kernel, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  bwd_kernel<<<L.num_sms, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE128, L.tmC128, L.tmE64, L.tmC64, L.tmdC, L.tmdE, L.args);
+  if (after_kernel) {
+    e = launch_after_previous(bwd_kernel, dim3(L.num_sms), dim3(NUM_THREADS), SMEM_BYTES, s, L.tmE128, L.tmC128,
+                              L.tmE64, L.tmC64, L.tmdC, L.tmdE, L.args);
+    if (e != cudaSuccess) return e;
+  } else {
+    bwd_kernel<<<L.num_sms, NUM_THREADS, SMEM_BYTES, s>>>(L.tmE128, L.tmC128, L.tmE64, L.tmC64, L.tmdC, L.tmdE,
+                                                           L.args);
+  }
   note_launches(1);
   return cudaGetLastError();
 }

@@ -626,6 +626,7 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const __nv_bfloat16*
 __global__ void __launch_bounds__(kFillThreads) empty_tiles_kernel(const __grid_constant__ BwdFinalize F,
                                                                    int64_t win, int image_rows) {
   extern __shared__ __align__(128) uint8_t img[];
+  wait_for_previous_grid();  // the plan's empty tiles; dC rows the tensor-core kernel does not write
   const int64_t D = F.D;
   const int es = F.dc_bf16 ? 2 : 4;
   const int64_t rowbytes = D * es;
@@ -710,6 +711,7 @@ __global__ void __launch_bounds__(kFillThreads) empty_tiles_kernel(const __grid_
 }
 
 __global__ void __launch_bounds__(256, 2) bwd_finalize_kernel(const __grid_constant__ BwdFinalize F) {
+  wait_for_previous_grid();  // dE_acc and dbias_acc of the tensor-core kernel, complete
   const int64_t D = F.D;
   const int col_chunks = static_cast<int>((D + kFinCols - 1) / kFinCols);
   const int64_t units_a = (F.N + kFinRowsA - 1) / kFinRowsA * col_chunks;
@@ -767,7 +769,7 @@ __global__ void skip_map_kernel(const uint8_t* __restrict__ flags, int64_t n, ui
 
 }  // namespace
 
-cudaError_t launch_empty_tiles(const BwdFinalize& F, int num_sms, cudaStream_t s) {
+cudaError_t launch_empty_tiles(const BwdFinalize& F, int num_sms, bool after_kernel, cudaStream_t s) {
   if (F.N == 0) return cudaSuccess;
   const int64_t es = F.dc_bf16 ? 2 : 4, rowbytes = F.D * es;
   // whole rows when one fits the image (up to 128 of them); otherwise windows of whole 16-byte pieces
@@ -778,14 +780,20 @@ cudaError_t launch_empty_tiles(const BwdFinalize& F, int num_sms, cudaStream_t s
   cudaError_t e = cudaFuncSetAttribute(empty_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kFillImageBytes));
   if (e != cudaSuccess) return e;
-  empty_tiles_kernel<<<num_sms * 2, kFillThreads, smem, s>>>(F, win, image_rows);
+  if (after_kernel) {
+    e = launch_after_previous(empty_tiles_kernel, dim3(num_sms * 2), dim3(kFillThreads), smem, s, F, win, image_rows);
+    if (e != cudaSuccess) return e;
+  } else {
+    empty_tiles_kernel<<<num_sms * 2, kFillThreads, smem, s>>>(F, win, image_rows);
+  }
   note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_finalize(const BwdFinalize& F, int num_sms, cudaStream_t s) {
   if (F.N == 0) return cudaSuccess;
-  bwd_finalize_kernel<<<num_sms * 4, 256, 0, s>>>(F);
+  const cudaError_t e = launch_after_previous(bwd_finalize_kernel, dim3(num_sms * 4), dim3(256), 0, s, F);
+  if (e != cudaSuccess) return e;
   note_launches(1);
   return cudaGetLastError();
 }

@@ -177,6 +177,12 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32
                : "memory");
 }
 
+// Programmatic dependent launch: waits until the previous kernel of the stream has completed and its
+// memory operations are visible. A kernel launched with launch_after_previous() may start while that
+// kernel's last blocks still run; it calls this before it reads anything the previous kernel wrote.
+// Without that launch attribute it returns at once.
+__device__ __forceinline__ void wait_for_previous_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Bulk copy of `bytes` (a multiple of 16) from shared memory to global memory, both 16-byte aligned.
 __device__ __forceinline__ void bulk_store(void* gdst, uint32_t src, uint32_t bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(src), "r"(bytes)

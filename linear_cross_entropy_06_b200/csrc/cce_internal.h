@@ -4,7 +4,10 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
 #include <stdint.h>
+
+#include <utility>
 
 namespace cce {
 
@@ -35,6 +38,25 @@ struct FwdLaunch {
 
 // Counts every kernel launch of the calling thread (instrumentation for benchmarks).
 void note_launches(int n);
+
+// Launches `kernel` on `s` with programmatic stream serialisation: it may be scheduled while the
+// previous kernel of the stream finishes, and must call wait_for_previous_grid() before it reads
+// that kernel's results. Used only where the previous operation on the stream is a kernel.
+template <typename... Params, typename... Args>
+cudaError_t launch_after_previous(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                  Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Limit of one bounded wait inside a kernel: CCE_WAIT_TIMEOUT_MS milliseconds (default 4000).
 uint64_t wait_timeout_ns();
@@ -182,7 +204,8 @@ struct PlanArgs {
 // One cooperative launch: the row scales, the tile flags, both tile lists, the pair list, the
 // chunks' work lists and queue groups, the onehot-only rows, and the skipped count.
 cudaError_t launch_bwd_plan(const PlanArgs& A, int num_sms, cudaStream_t s);
-cudaError_t launch_bwd(const BwdLaunch& L, cudaStream_t s);
+// after_kernel: the previous operation on s is a kernel (the planning launch or a column sum).
+cudaError_t launch_bwd(const BwdLaunch& L, bool after_kernel, cudaStream_t s);
 // Everything the backward computes after its tensor-core kernel (cce_bwd_plan.cu, two launches): the
 // dC rows of the vocabulary tiles no row block lists (empty_tiles_kernel), the last terms of dE and
 // its conversion, and dbias (bwd_finalize_kernel).
@@ -210,7 +233,7 @@ struct BwdFinalize {
   void* dbias_out;            // bf16 [V], or null: dbias_acc is the output (fp32)
 };
 // dC rows of the vocabulary tiles no row block lists.
-cudaError_t launch_empty_tiles(const BwdFinalize& F, int num_sms, cudaStream_t s);
+cudaError_t launch_empty_tiles(const BwdFinalize& F, int num_sms, bool after_kernel, cudaStream_t s);
 // dE's last terms and conversion, dbias (after the tensor-core kernel and launch_empty_tiles).
 cudaError_t launch_bwd_finalize(const BwdFinalize& F, int num_sms, cudaStream_t s);
 // out[i] = 1 if tile i of the plan's flags was skipped, 0 if it was kept (i < tiles).
@@ -243,7 +266,9 @@ struct FwdFinish {
   int* err;
 };
 constexpr int kFinishRows = 32;  // rows per block of the finish kernel
-cudaError_t launch_fwd_finish(const FwdFinish& F, cudaStream_t s);
+// after_kernel: the previous operation on s is the forward's tensor-core kernel (launched to overlap
+// its tail).
+cudaError_t launch_fwd_finish(const FwdFinish& F, bool after_kernel, cudaStream_t s);
 // out[0:D] = sum_r w_r X[r, :] (w_r = 1 when w is null); out[D] = sum_r w_r, or the sum of extra[0:rows].
 cudaError_t launch_weighted_colsum(const __nv_bfloat16* X, int64_t rows, int64_t D, const float* w,
                                    const __nv_bfloat16* extra, float* out, cudaStream_t s);

@@ -190,7 +190,7 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
   F.block_counts = reinterpret_cast<long long*>(b + off_bcnt);
   F.done = done;
   F.err = err;
-  if (cce::launch_fwd_finish(F, s) != cudaSuccess)
+  if (cce::launch_fwd_finish(F, N > 0, s) != cudaSuccess)
     return fail(CCE_ERR_CUDA, "cce_forward_noalloc: kernel launch failed");
   return CCE_OK;
 }
