@@ -49,12 +49,12 @@ KERNEL_SOURCES = {  # the kernel and what sets up its work (maps, plan, chunking
 }
 TRAFFIC_BYTES = {
     "fwd_lse_kernel": {
-        (4096, 4096, 128256): ("78bc8104dbff3216f1b60add73745a7a674307a6706e88a5069dc98355b54357",
-                               1084998144 + 34948096),
+        (4096, 4096, 128256): ("0bc9bf643c878f3d96ad63d257c0eabff47f44f9268a46d5a7e5e7dac74f6965",
+                               1086168832 + 35518464),
     },
     "bwd_kernel": {
-        (4096, 4096, 128256): ("2e8ba86bffc35cbda45431d27e2ceb35b98437723bf78a252734429621dc50f7",
-                               5480887296 + 1792022784),
+        (4096, 4096, 128256): ("93bdf2989a0bcddd804e9f94519c79a12156e4dc6fd5cd9a1c74e60733aeb9a9",
+                               5536615936 + 1791868672),
     },
 }
 
