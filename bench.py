@@ -49,12 +49,12 @@ KERNEL_SOURCES = {  # the kernel and what sets up its work (maps, plan, chunking
 }
 TRAFFIC_BYTES = {
     "fwd_lse_kernel": {
-        (4096, 4096, 128256): ("0bc9bf643c878f3d96ad63d257c0eabff47f44f9268a46d5a7e5e7dac74f6965",
-                               1086168832 + 35518464),
+        (4096, 4096, 128256): ("274bc2c2fdd722d6dcf0ad78e8fc152431dbf70a49bafff5edc45fa2ed59d1bd",
+                               1085109504 + 35097856),
     },
     "bwd_kernel": {
-        (4096, 4096, 128256): ("93bdf2989a0bcddd804e9f94519c79a12156e4dc6fd5cd9a1c74e60733aeb9a9",
-                               5536615936 + 1791868672),
+        (4096, 4096, 128256): ("8aa37d8deeff27865444105210447e1c4d2b9b897fd67b7048465d22fc480c08",
+                               5528850176 + 1791886848),
     },
 }
 

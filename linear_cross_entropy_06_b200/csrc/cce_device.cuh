@@ -374,10 +374,4 @@ __device__ __forceinline__ float warp_column_sums32(float (&v)[32], int lane) {
   return v[0];
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
 }  // namespace cce
