@@ -37,7 +37,7 @@ METRIC = "fwd+bwd tokens/s at Llama-3-8B head shape; % of B200 BF16 tensor peak"
 L2_FLUSH_BYTES = 512 << 20
 # The skip rule's tile (rows x vocabulary columns) given to the oracle when it is timed: the
 # backward's tile shape, stated here so that timing the oracle never loads the CUDA library.
-ORACLE_SKIP_TILE = (128, 128)
+ORACLE_SKIP_TILE = (128, 64)
 # DRAM bytes (read + write) of one launch of each tensor-core kernel, from a one-kernel, one-launch,
 # one-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), reported as the roofline's
 # "traffic". Each entry is keyed by the workload's (N, D, V) and holds the SHA-256 of the kernel's
@@ -185,12 +185,27 @@ def barrier(world: int):
 
 
 def algorithmic_flops(N: int, D: int, V: int, kept_tiles: int, tile: tuple) -> tuple:
-    """2NVD forward; 6 * rows * cols * D per kept backward tile (recompute, dE, dC).
+    """2NVD forward; 6 * rows * cols * D per kept unit of the skip rule (recompute, dE, dC).
 
-    Kept tiles are counted at their full size: at every bench workload N and V are multiples of
-    the tile, so none is partial (for ragged shapes this slightly overcounts the backward)."""
+    Kept units are counted at their full size: at every bench workload N and V are multiples of
+    the unit, so none is partial (for ragged shapes this slightly overcounts the backward)."""
     tm, tn = tile
     return 2.0 * N * V * D, 6.0 * tm * tn * D * kept_tiles
+
+
+def listed_tile_count(skip_map) -> int:
+    """128 x 128 tiles with a kept 128 x 64 unit: the tiles whose dC MMAs run (over both halves)."""
+    kept = (skip_map == 0)
+    if kept.shape[1] % 2:
+        kept = torch.nn.functional.pad(kept, (0, 1))
+    return int((kept[:, 0::2] | kept[:, 1::2]).sum().item())
+
+
+def issued_mma_flops(D: int, kept_units: int, listed_tiles: int, tile: tuple) -> float:
+    """The backward's tensor-core work as issued: the recompute and the dE MMAs run over the kept
+    units only, the dC MMAs over every listed tile's two units (a skipped unit reads as zeros)."""
+    tm, tn = tile
+    return 4.0 * tm * tn * D * kept_units + 2.0 * tm * (2 * tn) * D * listed_tiles
 
 
 def oracle_sample_seconds(inp, rows: int):
@@ -276,10 +291,13 @@ def run_ours(args, world, rank, local):
         dE, dC, filt = ops.cce_backward(E, C, t, lse, tmax, count, g, EPS, -100, w.reduction, out_fp32=False)
         return loss, filt
 
-    # check once that nothing was reported on the device
+    # check once that nothing was reported on the device; the skip map of that call gives the
+    # tensor-core work the backward issues (below)
     loss0, lse0, tmax0, count0 = ops.cce_forward(E, C, t, -100, w.reduction, check=True)
-    ops.cce_backward(E, C, t, lse0, tmax0, count0, g, EPS, -100, w.reduction, check=True)
-    del loss0, lse0, tmax0, count0
+    skip_map = ops.cce_backward(E, C, t, lse0, tmax0, count0, g, EPS, -100, w.reduction, check=True,
+                                skip_map=True)[-1]
+    listed_tiles = listed_tile_count(skip_map)
+    del loss0, lse0, tmax0, count0, skip_map
 
     # peak device memory of one forward + backward beyond the resident inputs (untimed): the bf16
     # gradients themselves, plus everything the loss needs, which must stay far below N*V*2
@@ -346,6 +364,10 @@ def run_ours(args, world, rank, local):
         "bwd_kernel": kernel_line(bwd_flop, bwd_ms,
                                   "one persistent launch per step: recompute, gradient tiles, dC and dE MMAs"),
     }
+    issued = issued_mma_flops(D, kept, listed_tiles, tile)
+    kernels["bwd_kernel"].update(listed_tiles=listed_tiles, issued_mma_flops=issued,
+                                 issued_mma_tflops=issued / kernels["bwd_kernel"]["ms"] / 1e9,
+                                 issued_mma_frac=issued / kernels["bwd_kernel"]["ms"] / 1e9 / peak_tf)
     # The dominant kernel: the forward and the backward are one launch each per step; the roofline
     # line reports the longer one (by average launch duration over the timed steps).
     dom = "bwd_kernel" if kernels["bwd_kernel"]["ms"] > kernels["fwd_lse_kernel"]["ms"] else "fwd_lse_kernel"

@@ -92,20 +92,21 @@ typedef struct {
 #define CCE_OUT_DE_FP32 2  /* dE fp32 (a shard's part, to be summed over shards), dC and dbias bf16 */
 
 /* Width of the vocabulary sub-tile whose per-row maximum logit the forward saves. */
-#define CCE_VOCAB_SUBTILE 128
+#define CCE_VOCAB_SUBTILE 64
 
-/* Number of floats in the saved tile-max buffer: ceil(V / 128) * N. Layout [ceil(V/128), N]:
- * entry (j, r) is max_{v in [128 j, 128 j + 128) and v < V} z[r, v]. -1 for a bad problem. */
+/* Number of floats in the saved tile-max buffer: ceil(V / 64) * N. Layout [ceil(V/64), N]:
+ * entry (j, r) is max_{v in [64 j, 64 j + 64) and v < V} z[r, v]. -1 for a bad problem. */
 CCE_API int64_t cce_tile_max_len(const cce_problem* p);
 
-/* Rows and vocabulary columns of one backward tile. The skip rule of the backward decides per
- * tile of this size (mlx-cross-entropy README, "How it works" item 2). */
+/* Rows and vocabulary columns of one unit of the backward's skip rule (128 x 64): the rule decides
+ * per unit of this size (mlx-cross-entropy README, "How it works" item 2); the kernels work on
+ * 128 x 128 tiles made of two such units and skip the work of a skipped one. */
 CCE_API void cce_backward_tile_shape(int32_t* tile_rows, int32_t* tile_cols);
 
 /* Bytes of device workspace cce_forward() needs (0 for a bad problem). */
 CCE_API size_t cce_forward_workspace_size(const cce_problem* p);
 
-/* Bytes of device workspace cce_backward() needs: the tile plan (about 37 bytes per 128 x 128
+/* Bytes of device workspace cce_backward() needs: the tile plan (about 41 bytes per 128 x 128
  * tile), the gradient tiles of two vocabulary chunks (4 MiB per 128 rows, at least 128 MiB) and,
  * with out_fp32 = 0, the fp32 accumulators of dE and dbias, (N * D + V) * 4 bytes. Never anything
  * of size N * V. */
@@ -136,10 +137,10 @@ CCE_API cce_status cce_forward(const cce_problem* p, const void* E, const void* 
 /*
  * Backward: dE = G C, dC = G^T E and dbias = sum_r G[r, :] with G = scale_r * (p~ - onehot),
  * p = softmax(z),
- * recomputed tile by tile from E, C and the saved LSE. p~ is p with every skipped tile set to 0:
- * a tile (tile_rows x tile_cols, see cce_backward_tile_shape) is skipped when, for every
- * non-ignored row r in it, max over its columns of z[r, v] - LSE[r] < ln(filter_eps); a tile
- * without a non-ignored row is skipped too. filter_eps <= 0 keeps every tile. The onehot term
+ * recomputed tile by tile from E, C and the saved LSE. p~ is p with every skipped unit set to 0:
+ * a unit (tile_rows x tile_cols, see cce_backward_tile_shape) is skipped when, for every
+ * non-ignored row r in it, max over its columns of z[r, v] - LSE[r] < ln(filter_eps); a unit
+ * without a non-ignored row is skipped too. filter_eps <= 0 keeps every unit. The onehot term
  * is never skipped. Loss functions explainer, "How it works" item 2 (gradient p - y);
  * mlx-cross-entropy README, "How it works" items 2 and 3 (skipping, accumulation).
  * scale_r = g / max(count, 1) (mean), g (sum) or g[r] (none); 0 for ignored rows. With the loss
@@ -155,7 +156,7 @@ CCE_API cce_status cce_forward(const cce_problem* p, const void* E, const void* 
  *           the gradient of the bias (also when bias is NULL, i.e. zero).
  *  For a vocabulary shard (p->vocab_total > 0): lse and count are the merged values of
  *  cce_forward_merge, tile_max is this shard's from cce_forward_partial; dE is this shard's part.
- *  filtered_tiles device int64 [1]: number of skipped tiles
+ *  filtered_tiles device int64 [1]: number of skipped units (tile_rows x tile_cols)
  *  workspace: device scratch of at least cce_backward_workspace_size(p, out_fp32) bytes.
  */
 CCE_API cce_status cce_backward(const cce_problem* p, const void* E, const void* C, const void* bias,
@@ -164,11 +165,12 @@ CCE_API cce_status cce_backward(const cce_problem* p, const void* E, const void*
                                 void* dbias, int32_t out_fp32, int64_t* filtered_tiles, void* workspace,
                                 size_t workspace_bytes, cce_stream_t stream);
 
-/* The skip decision of every backward tile taken by the last cce_backward() that ran on `workspace`
- * for the same problem: skipped[b * nt + t] = 1 when tile (row block b, vocabulary tile t) was
- * skipped and 0 when it was kept, with nb = ceil(N / tile_rows) row blocks, nt = ceil(V / tile_cols)
- * vocabulary tiles (cce_backward_tile_shape) and b < nb, t < nt. A diagnostic of the skip rule of
- * mlx-cross-entropy README, "How it works" item 2: the count of ones equals filtered_tiles.
+/* The skip decision of every unit of the skip rule taken by the last cce_backward() that ran on
+ * `workspace` for the same problem: skipped[b * nt + t] = 1 when unit (row block b, vocabulary
+ * block t) was skipped and 0 when it was kept, with nb = ceil(N / tile_rows) row blocks,
+ * nt = ceil(V / tile_cols) vocabulary blocks (cce_backward_tile_shape) and b < nb, t < nt. A
+ * diagnostic of the skip rule of mlx-cross-entropy README, "How it works" item 2: the count of ones
+ * equals filtered_tiles.
  *  workspace: the backward workspace of that call (workspace_bytes as given to it); it is read,
  *             not changed, so call this after the backward on the same stream.
  *  skipped:   device uint8 [nb * nt].
@@ -227,8 +229,8 @@ CCE_API const char* cce_last_error_message(void);
  * counterpart; it is an addition for such callers. Arguments and results are those of
  * cce_forward() without the workspace.
  *  - Scratch lives in one device array of CCE_NOALLOC_SCRATCH_BYTES that every GPU loading the
- *    library holds until exit. Problems needing more (about ceil(V/128) * N * 4 + 5 N + 4 D bytes; at
- *    V = 128256 up to N of about 8000) are rejected with CCE_ERR_UNSUPPORTED before anything runs.
+ *    library holds until exit. Problems needing more (about ceil(V/64) * N * 4 + 5 N + 4 D bytes; at
+ *    V = 128256 up to N of about 4100) are rejected with CCE_ERR_UNSUPPORTED before anything runs.
  *  - The first call on each device looks up the array's device address (with that device
  *    current); make that first call before any stream capture.
  *  - Every call shares the array and the array keeps the last call's contents (the call clears

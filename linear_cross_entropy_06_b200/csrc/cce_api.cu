@@ -17,7 +17,7 @@
 
 namespace {
 
-constexpr int32_t kVersion = 400;  // 0.4.0: vocabulary shards, skip map, output dtype modes
+constexpr int32_t kVersion = 500;  // 0.5.0: the skip rule on 128 x 64 units (saved maxima per 64 columns)
 constexpr size_t kHeaderBytes = 256;
 constexpr size_t kAlign = 256;
 
@@ -81,7 +81,8 @@ bool problem_ok(const cce_problem* p, bool set_error) {
   // Kernel indices are 32-bit for rows and tiles; keep every count well inside that.
   if (p->N >= (int64_t(1) << 31) - 256 || p->V >= (int64_t(1) << 31) - 256 || p->D >= (int64_t(1) << 24))
     return bad("N, V or D too large");
-  if (ceil_div(p->N, cce::kBwdBM) * ceil_div(p->V, cce::kBwdBN) >= (int64_t(1) << 31))
+  // (a tile's gradient slot shares a 32-bit word with its kept halves)
+  if (ceil_div(p->N, cce::kBwdBM) * ceil_div(p->V, cce::kBwdBN) >= (int64_t(1) << cce::kSlotBits))
     return bad("too many backward tiles");
   return true;
 }
@@ -159,6 +160,7 @@ struct SplitWs {
   float* dbias_acc;  // [V] fp32 (absent when dbias is written in fp32)
   float* csum;       // [D + 1]: column sums of C (label smoothing only)
   float* wsum;       // [D + 1]: sum_r scale_r E_r and sum_r scale_r (label smoothing only)
+  void* zero_half;   // [kZeroHalfBytes]: zeros read in place of a skipped half
   size_t bytes;
 };
 
@@ -186,6 +188,10 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.offsets_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nb + 1)));
   w.plan.entries_b = reinterpret_cast<int2*>(take(sizeof(int2) * static_cast<size_t>(tiles)));
   w.plan.pos_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(tiles)));
+  w.plan.cnt_hb = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nb)));
+  w.plan.off_hb = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nb + 1)));
+  w.plan.hp_b = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(tiles + 1)));
+  w.zero_half = take(cce::kZeroHalfBytes);
   w.plan.kept_total = reinterpret_cast<int*>(take(2 * sizeof(int)));
   w.plan.n_empty = w.plan.kept_total + 1;
   // A chunk spans at most kChunkCBytes of C (the trade-off between dE's split-reduce passes and
@@ -344,6 +350,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
     PA.onehot_coef = 1.f - p->label_smoothing;
     PA.dE_acc = dE_acc;
     PA.dbias_acc = dbias_acc;
+    PA.zero_half = w.zero_half;
     PA.filtered_tiles = filtered_tiles;
     PA.bar = &w.hdr->bar;
     PA.err = &w.hdr->err;
@@ -366,7 +373,7 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
 
   cce::BwdLaunch L{};
   CCE_CHECK(make_map(&L.tmE128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, D, 64, cce::kBwdBM));
-  CCE_CHECK(make_map(&L.tmC128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, cce::kBwdBN));
+  CCE_CHECK(make_map(&L.tmC128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, V, D, 64, cce::kSubTile));
   // The dE / dC items load a 64-row x 256-column operand slice per stage. With D a multiple of 256
   // it is one 3-D TMA load (64 columns x 64 rows x 4 column blocks: the same shared-memory image as
   // four 64 x 64 boxes); otherwise four 2-D boxes (the last slice of D may be partial).
@@ -430,6 +437,8 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.offsets_t = w.plan.offsets_t;
   A.entries_t = w.plan.entries_t;
   A.entries_b = w.plan.entries_b;
+  A.hp_b = w.plan.hp_b;
+  A.zero_half = w.zero_half;
   A.gscratch = w.gscratch;
   A.qctr = w.sync;
   A.counters = w.sync + 1;
@@ -531,7 +540,7 @@ int64_t cce_tile_max_len(const cce_problem* p) {
 
 void cce_backward_tile_shape(int32_t* tile_rows, int32_t* tile_cols) {
   if (tile_rows) *tile_rows = cce::kBwdBM;
-  if (tile_cols) *tile_cols = cce::kBwdBN;
+  if (tile_cols) *tile_cols = cce::kSubTile;
 }
 
 size_t cce_forward_workspace_size(const cce_problem* p) {
@@ -709,8 +718,8 @@ cce_status cce_backward_skip_map(const cce_problem* p, const void* workspace, si
   if (workspace_bytes < w.bytes)
     return fail(CCE_ERR_WORKSPACE, "backward workspace is %zu bytes, needs %zu", workspace_bytes, w.bytes);
   if (p->N == 0) return CCE_OK;
-  const int64_t tiles = static_cast<int64_t>(w.plan.nb) * w.plan.nt;
-  CCE_TRY(cce::launch_skip_map(w.plan.flags, tiles, skipped, reinterpret_cast<cudaStream_t>(stream)));
+  CCE_TRY(cce::launch_skip_map(w.plan.flags, w.plan.nb, w.plan.nt, ceil_div(p->V, cce::kSubTile), skipped,
+                               reinterpret_cast<cudaStream_t>(stream)));
   return CCE_OK;
 }
 

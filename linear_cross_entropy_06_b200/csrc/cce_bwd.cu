@@ -7,17 +7,20 @@
 // abstract (logits are recomputed blockwise and never stored).
 //
 // Work items, per vocabulary chunk c (its gradient tiles live in scratch buffer c mod kGradBuffers):
-//   pair   two consecutive listed (kept) 128 x 128 tiles (b, t0), (b, t1) of row block b in the
-//          chunk: S = E_b [C_t0; C_t1]^T (+ bias) (tcgen05 M=128 N=256 K=D), then
+//   pair   two consecutive listed 128 x 128 tiles (b, t0), (b, t1) of row block b in the chunk, of
+//          which only the kept 64-column halves (one to four) are computed: S = E_b [C_h ...]^T
+//          (+ bias) over those halves (tcgen05 M=128 N=64 x halves K=D), then
 //          G = scale_r (1 + 2 zl LSE_r) exp(S - LSE_r) - scale_r (1 - ls) [v = t_r] in fp32, rounded
-//          to bf16 into a 128B-swizzled shared tile, one 32 KB bulk store per tile into the scratch
-//          buffer; with a dbias output, the column sums of the fp32 G are added into it.
-//   dE     (row block b, 256-column slice s of D): sum over the chunk's listed t of G_bt C_t[:, s]
-//          in TMEM, then one fp32 TMA reduce-add into dE_acc (split-reduce over chunks).
+//          to bf16 into a 128B-swizzled shared tile, one 16 KB bulk store per kept half into the
+//          tile's slot of the scratch buffer; with a dbias output, the column sums of the fp32 G are
+//          added into it.
+//   dE     (row block b, 256-column slice s of D): sum over the kept halves h of the chunk's listed
+//          tiles t of G_bth C_th[:, s] in TMEM, then one fp32 TMA reduce-add into dE_acc
+//          (split-reduce over chunks).
 //   dC     (vocabulary tile t, slice s): sum over the listed b of G_bt^T E_b[:, s] in TMEM (A = the
-//          same G tile read MN-major), plus the onehot terms of rows whose target tile in t was
-//          skipped and the label-smoothing term, written once by TMA store: every listed tile of t
-//          lies in t's chunk, so dC needs no reduction.
+//          same G tile read MN-major, a skipped half read as zeros), plus the onehot terms of rows
+//          whose target half in t was skipped and the label-smoothing term, written once by TMA
+//          store: every listed tile of t lies in t's chunk, so dC needs no reduction.
 //
 // Scheduling: a global queue holds the items in the order pairs(0), pairs(1), dE/dC(0), pairs(2),
 // dE/dC(1), ..., pairs(n-1), dE/dC(n-2), dE/dC(n-1): the dE/dC items of a chunk come one group of
@@ -35,9 +38,9 @@
 // machine has a single tail per backward instead of one per chunk and kernel.
 //
 // Design (B200): one CTA per SM, 7 warps, 224 KB of shared memory.
-//   warp 0      producer: per stage (48 KB, 4 deep) either E_b, C_t0, C_t1 K-blocks of 64 (pair), or
-//               one K-half of a gradient tile (16 KB bulk copy) and the 64 x 256 operand slice
-//               (four TMA boxes of 64 x 64) (dE, dC).
+//   warp 0      producer: per stage (at most 48 KB, 4 deep) either the E_b K-block of 64 and one
+//               64 x 64 C box per kept half (pair), or one K-half of a gradient tile (16 KB bulk
+//               copy, or zeros for a skipped half) and the 64 x 256 operand slice (dE, dC).
 //   warp 1      TMEM owner (two 256-column fp32 buffers); one lane issues tcgen05.mma M=128 N=256.
 //   warps 2..5  write-out: G formation and bulk stores (pair), or TMEM -> swizzled staging -> TMA
 //               store / reduce-add (dC / dE), while the MMA fills the other TMEM buffer.
@@ -72,10 +75,10 @@ struct alignas(16) WorkItem {
   int kind;
   int chunk;
   int key;         // pair, dE: row block b; dC: vocabulary tile t
-  int s;           // dE, dC: slice of D; pair: kept bits (1 first tile, 2 second tile)
+  int s;           // dE, dC: slice of D; pair: kept halves (bits 0-1 of t0, bits 2-3 of t1)
   int begin, end;  // dE, dC: list entries; pair: vocabulary tiles t0 and t1 (-1 when absent)
   int slot0;       // pair: slot of t0 in the chunk's buffer; dE, dC: the chunk's first slot
-  int slot1;       // pair: slot of t1
+  int slot1;       // pair: slot of t1; dE: stages (kept halves of the entries)
   int dep_idx;     // counter this item waits on (-1: none): before its loads (dE, dC) or stores (pair)
   int dep_val;     // value the counter must reach
   int oh_begin;    // dC: rows whose target tile in this vocabulary tile was skipped, oh_rows[oh_begin:oh_end]
@@ -105,7 +108,12 @@ constexpr uint32_t LOOKAHEAD = 2;
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + REGION_BYTES + kNumBars * 8 + RING * 64 + 16;
 static_assert(SMEM_BYTES <= 232448, "fits the 227 KB opt-in shared memory of an SM");
 
-constexpr uint32_t IDESC_S = idesc_bf16(BM, 2 * BN, false, false);  // S = E_b [C_t0; C_t1]^T
+// S = E_b [C_h ...]^T over nh kept halves: N = 64 nh
+__device__ __forceinline__ uint32_t idesc_pair(int nh) {
+  constexpr uint32_t d1 = idesc_bf16(BM, 1 * kSubTile, false, false), d2 = idesc_bf16(BM, 2 * kSubTile, false, false),
+                     d3 = idesc_bf16(BM, 3 * kSubTile, false, false), d4 = idesc_bf16(BM, 4 * kSubTile, false, false);
+  return nh <= 1 ? d1 : nh == 2 ? d2 : nh == 3 ? d3 : d4;
+}
 constexpr uint32_t IDESC_DC = idesc_bf16(BN, SLICE, true, true);    // M = vocabulary (G^T, MN-major)
 constexpr uint32_t IDESC_DE = idesc_bf16(BM, SLICE, false, true);   // M = rows (G, K-major)
 
@@ -187,6 +195,7 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, int nchun
       const int2 r = A.rb_range[static_cast<int64_t>(c) * A.nb + it.key];
       it.begin = r.x;
       it.end = r.y;
+      it.slot1 = A.hp_b[r.y] - A.hp_b[r.x];
       it.dep_idx = A.ctr_g_b + c * A.nb + it.key;
     } else {  // slice-major too: concurrent dC items read the same columns of E
       const int v = local - nde * S;
@@ -310,19 +319,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive(bar(kItemTaken + idx));
         if (it.kind == kEnd) break;
         if (it.kind == kPair) {
-          if (it.s == 0) continue;  // onehot-only tiles need no recompute
+          if (it.s == 0) continue;  // no kept half: nothing to recompute
           const int rb = it.key * BM;
-          const int vb0 = it.begin * BN, vb1 = (it.end >= 0 ? it.end : it.begin) * BN;
+          const uint32_t stage_bytes = PART + static_cast<uint32_t>(__popc(it.s)) * X_BOX;
           for (int kb = 0; kb < num_kb; ++kb) {
             if (!mbar_wait(bar(kEmpty + stage), phase ^ 1u, wc)) {
               ok = false;
               break;
             }
             const uint32_t dst = smem_u32(stages + stage * STAGE_BYTES);
-            mbar_arrive_expect_tx(bar(kFull + stage), STAGE_BYTES);
+            mbar_arrive_expect_tx(bar(kFull + stage), stage_bytes);
             tma_load_2d(dst, &tmE128, bar(kFull + stage), kb * BK, rb);
-            tma_load_2d(dst + PART, &tmC128, bar(kFull + stage), kb * BK, vb0);
-            tma_load_2d(dst + 2 * PART, &tmC128, bar(kFull + stage), kb * BK, vb1);
+            uint32_t off = PART;  // the kept halves' C rows, in the order of their bits
+#pragma unroll
+            for (int bit = 0; bit < 4; ++bit) {
+              if ((it.s >> bit) & 1) {
+                const int vrow = (bit < 2 ? it.begin : it.end) * BN + (bit & 1) * kSubTile;
+                tma_load_2d(dst + off, &tmC128, bar(kFull + stage), kb * BK, vrow);
+                off += X_BOX;
+              }
+            }
             ++issued[stage];
             if (++stage == STAGES) {
               stage = 0;
@@ -336,19 +352,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool de = it.kind == kDE;
         const uint8_t* buf = buffer(it.chunk);
         const int x0 = it.s * SLICE;
-        auto entry = [&](int i) {  // (tile index of the other operand, slot in the chunk's buffer)
+        // (tile index of the other operand, slot in the chunk's buffer, kept halves of the tile)
+        auto entry = [&](int i) {
           if (de) {
             const int2 en = A.entries_b[i];
-            return make_int2(en.x, en.y - it.slot0);
+            return make_int3(en.x, (en.y & kSlotMask) - it.slot0, en.y >> kSlotBits);
           }
-          return make_int2(A.entries_t[i].x >> 2, i - it.slot0);
+          const int x = A.entries_t[i].x;
+          return make_int3(x >> 4, i - it.slot0, flag_halves(x & 15));
         };
-        int2 os_next = it.begin < it.end ? entry(it.begin) : make_int2(0, 0);
+        const uint8_t* zero = static_cast<const uint8_t*>(A.zero_half);
+        int3 os_next = it.begin < it.end ? entry(it.begin) : make_int3(0, 0, 0);
         for (int i = it.begin; i < it.end && ok; ++i) {
-          const int2 os = os_next;
+          const int3 os = os_next;
           if (i + 1 < it.end) os_next = entry(i + 1);
           const uint8_t* tile = buf + static_cast<size_t>(os.y) * TILE_BYTES;
           for (int h = 0; h < 2; ++h) {  // K-halves: 64 vocabulary columns (dE) or 64 rows (dC)
+            if (de && !((os.z >> h) & 1)) continue;  // a skipped half adds nothing to dE
             if (!mbar_wait(bar(kEmpty + stage), phase ^ 1u, wc)) {
               ok = false;
               break;
@@ -357,9 +377,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_arrive_expect_tx(bar(kFull + stage), STAGE_BYTES);
             if (de) {  // G block h: rows 0..127, vocabulary 64h .. 64h + 63 (K-major A)
               bulk_load(dst, tile + h * PART, PART, bar(kFull + stage));
-            } else {   // rows 64h .. 64h + 63 of both 64-column blocks (MN-major A = G^T)
-              bulk_load(dst, tile + h * (PART / 2), PART / 2, bar(kFull + stage));
-              bulk_load(dst + PART / 2, tile + PART + h * (PART / 2), PART / 2, bar(kFull + stage));
+            } else {   // rows 64h .. 64h + 63 of both 64-column blocks (MN-major A = G^T); zeros for a
+                       // skipped half
+              bulk_load(dst, (os.z & 1) ? tile + h * (PART / 2) : zero, PART / 2, bar(kFull + stage));
+              bulk_load(dst + PART / 2, (os.z & 2) ? tile + PART + h * (PART / 2) : zero, PART / 2,
+                        bar(kFull + stage));
             }
             const int y = os.x * BM + 64 * h;  // K rows of the operand: C_t rows (dE), E_b rows (dC)
             if (A.slab3d) {
@@ -402,8 +424,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(bar(kAccEmpty + a), ((acc_iter >> 1) & 1u) ^ 1u, wc)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(a * 2 * BN);
-        const int nstage = pair ? num_kb : 2 * (it.end - it.begin);
-        const uint32_t idesc = pair ? IDESC_S : (it.kind == kDE ? IDESC_DE : IDESC_DC);
+        const int nstage = pair ? num_kb : (it.kind == kDE ? it.slot1 : 2 * (it.end - it.begin));
+        const uint32_t idesc = pair ? idesc_pair(__popc(it.s)) : (it.kind == kDE ? IDESC_DE : IDESC_DC);
         for (int j = 0; j < nstage; ++j) {
           if (!mbar_wait(bar(kFull + stage), phase, wc)) {
             ok = false;
@@ -414,7 +436,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // 16 of the stage's 64 K values per MMA
             uint64_t adesc, bdesc;
-            if (pair) {  // A = E_b K-block, B = C_t0 and C_t1 rows (256 rows of 128 bytes, contiguous)
+            if (pair) {  // A = E_b K-block, B = the kept halves' C rows (64 nh rows of 128 bytes, contiguous)
               adesc = sdesc_sw128(s0 + 32u * kk, 16, 1024);
               bdesc = sdesc_sw128(s0 + PART + 32u * kk, 16, 1024);
             } else {
@@ -501,7 +523,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int ntiles = it.end >= 0 ? 2 : 1;
         for (int u = 0; u < ntiles && ok; ++u) {
           const int t = u == 0 ? it.begin : it.end;
-          const bool kept = (it.s >> u) & 1;
+          const int hm = (it.s >> (2 * u)) & 3;  // this tile's kept halves
           const int vb = t * BN;
           const int64_t rel = tg - vb;
           const int tcol = (tvalid && rel >= 0 && rel < BN) ? static_cast<int>(rel) : -1;  // -scale_r here
@@ -511,17 +533,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
 #pragma unroll
           for (int c = 0; c < BN / 32; ++c) {
+            const int hf = c / (kSubTile / 32);  // the half this 32-column piece lies in
+            if (!((hm >> hf) & 1)) continue;      // a skipped half has no gradient tile part
             float v[32];
             const int col0 = vb + c * 32;
-            if (kept) {
-              tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * 2 * BN + u * BN + c * 32), v);
-              if (A.bias != nullptr) add_bias32(v, A.bias, col0, A.V);
+            // accumulator columns: 64 per kept half of the pair, in the order of their bits
+            const int acol = __popc(it.s & ((1 << (2 * u + hf)) - 1)) * kSubTile + (c % (kSubTile / 32)) * 32;
+            tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * 2 * BN + acol), v);
+            if (A.bias != nullptr) add_bias32(v, A.bias, col0, A.V);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] = sc_p * exp2f(fmaf(v[e], kLog2e, -lse_l2));
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] = 0.f;
-            }
+            for (int e = 0; e < 32; ++e) v[e] = sc_p * exp2f(fmaf(v[e], kLog2e, -lse_l2));
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               if (c * 32 + e == tcol) v[e] -= sc_y;
@@ -546,7 +567,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!warp_wait(bar(kGReady), gphase & 1u)) {
               ok = false;
             } else if (leader) {
-              bulk_store(buf + static_cast<size_t>(u == 0 ? it.slot0 : it.slot1) * TILE_BYTES, reg0, TILE_BYTES);
+              uint8_t* slot = buf + static_cast<size_t>(u == 0 ? it.slot0 : it.slot1) * TILE_BYTES;
+              for (int hf = 0; hf < 2; ++hf)
+                if ((hm >> hf) & 1) bulk_store(slot + hf * PART, reg0 + static_cast<uint32_t>(hf * PART), PART);
               bulk_commit_group();
             }
           }

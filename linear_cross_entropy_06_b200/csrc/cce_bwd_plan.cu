@@ -1,20 +1,21 @@
 // Planning of the backward: which (row block b, vocabulary tile t) tiles carry gradient, and two
 // compact lists of them.
 //
-// A tile of 128 rows x 128 vocabulary columns is kept when some non-ignored row r of block b has
-// max over the tile of z[r, v] - LSE_r >= ln(eps) (mlx-cross-entropy README, "How it works" item 2:
-// skip tiles whose softmax is below 2^-12), judged from the forward's saved per-sub-tile maxima.
-// A skipped tile that holds the target of one of its rows still carries the onehot term of
-// p - y (Loss functions explainer, "How it works" item 2), which is never skipped. Such a tile
-// ("onehot only") is not listed: its rows' onehot terms are applied one row at a time, listed by
-// vocabulary tile in oh_off / oh_rows (dC adds -scale_r (1 - ls) E_r to row t_r, dE adds
-// -scale_r (1 - ls) C_{t_r} to row r).
+// The skip rule works on halves of a tile: 128 rows x 64 vocabulary columns. A half is kept when some
+// non-ignored row r of block b has max over the half of z[r, v] - LSE_r >= ln(eps) (mlx-cross-entropy
+// README, "How it works" item 2: skip tiles whose softmax is below 2^-12), judged from the forward's
+// saved per-64-column maxima. A tile (128 x 128) with a kept half is listed; only its kept halves are
+// recomputed and multiplied into dE, and its skipped half reads as zeros in the dC MMAs.
+// The onehot term of p - y (Loss functions explainer, "How it works" item 2) is never skipped. A row
+// whose target lies in a skipped half (of a listed tile, or of a tile with no kept half, "onehot
+// only") gets its onehot term one row at a time, listed by vocabulary tile in oh_off / oh_rows (dC
+// adds -scale_r (1 - ls) E_r to row t_r, dE adds -scale_r (1 - ls) C_{t_r} to row r).
 //
-// flags[b * nt + t]: 0 = no gradient, 1 = kept (listed), 2 = onehot only.
+// flags[b * nt + t]: the state (nothing, listed, onehot only) and the kept halves (cce_internal.h).
 // By vocabulary tile (recompute and dC kernels): offsets_t[t] .. offsets_t[t+1] index entries_t,
-//   each (b * 4 + flag, t), row blocks ascending. An entry's position is also its gradient-tile slot.
-// By row block (dE kernel): offsets_b[b] .. offsets_b[b+1] index entries_b, each (t, slot),
-//   vocabulary tiles ascending.
+//   each (b * 16 + flag, t), row blocks ascending. An entry's position is also its gradient-tile slot.
+// By row block (dE kernel): offsets_b[b] .. offsets_b[b+1] index entries_b, each (t, slot | kept
+//   halves << kSlotBits), vocabulary tiles ascending; hp_b counts the kept halves before each entry.
 // Flat work lists the backward kernel reads with one load per item:
 //   rb_range[c * nb + b]   the entries [lo, hi) of row block b inside vocabulary chunk c;
 //   pair_desc/pair_slot    the pairs of consecutive listed tiles of a row block inside a chunk,
@@ -32,12 +33,20 @@ __device__ __forceinline__ bool valid_target(int64_t t, int64_t V, int64_t ignor
   return t != ignore_index && t >= 0 && t < V;
 }
 
+// Whether the onehot term of a row whose target is column tr (of this problem's vocabulary) is
+// applied on its own: the half of the target's tile that holds tr is not kept. f is the flag of the
+// row's block and the target's tile.
+__device__ __forceinline__ bool target_half_skipped(int f, int64_t tr) {
+  const int h = static_cast<int>((tr % kBwdBN) / kSubTile);
+  return flag_state(f) == kFlagOnehotOnly || (flag_state(f) == kFlagListed && !((flag_halves(f) >> h) & 1));
+}
+
 // The planning runs as one cooperative launch of one 1024-thread block per SM: a sequence of
 // phases separated by grid-wide barriers (bounded waits; a block that gives up records
 // CCE_ERR_DEVICE_TIMEOUT and every block then leaves). Each phase spreads its work over the grid.
 constexpr int kPlanThreads = 1024;
 static_assert(kPlanThreads == 32 * 32, "block_scan keeps one total per warp in 32 lanes");
-constexpr int kFlagTiles = 32;   // vocabulary tiles per flag unit
+constexpr int kFlagTiles = 16;   // vocabulary tiles per flag unit (32 halves: one per lane of a column max)
 constexpr int kFlagGroups = kPlanThreads / kBwdBM;  // flag units per block at a time (128 threads each)
 
 struct PlanCtl {
@@ -154,17 +163,18 @@ __device__ __forceinline__ float warp_column_max32(float (&v)[32], int lane) {
 // tile row; named barrier `group + 1`). Every load of the unit (the rows' targets and LSE, the run's
 // saved maxima) is issued before any of them is used, so they are in flight together.
 __device__ void tile_flags_unit(const PlanArgs& A, int group, int b, int t0) {
-  __shared__ float wmax[kFlagGroups][4][kFlagTiles];
+  __shared__ float wmax[kFlagGroups][4][2 * kFlagTiles];
   __shared__ int any_target[kFlagGroups][kFlagTiles];
   const int tid = threadIdx.x & (kBwdBM - 1), lane = tid & 31;
   const int nt = A.P.nt;
   const int64_t r = static_cast<int64_t>(b) * kBwdBM + tid;
   const bool row_in = r < A.N;
   if (tid < kFlagTiles) any_target[group][tid] = 0;
-  float mt[kFlagTiles];
+  const int64_t j0 = 2 * static_cast<int64_t>(t0);  // the run's first half (saved sub-tile)
+  float mt[2 * kFlagTiles];
 #pragma unroll
-  for (int k = 0; k < kFlagTiles; ++k)
-    mt[k] = (row_in && A.filter_on && t0 + k < nt) ? A.tile_max[static_cast<int64_t>(t0 + k) * A.N + r] : -INFINITY;
+  for (int k = 0; k < 2 * kFlagTiles; ++k)
+    mt[k] = (row_in && A.filter_on && j0 + k < A.T) ? A.tile_max[(j0 + k) * A.N + r] : -INFINITY;
   int64_t tr = row_in ? A.targets[r] : A.ignore_index;
   const float l = (row_in && A.filter_on) ? A.lse[r] : 0.f;
   named_barrier(group + 1, kBwdBM);
@@ -173,48 +183,74 @@ __device__ void tile_flags_unit(const PlanArgs& A, int group, int b, int t0) {
   tr -= A.vs;
   if (local && tr / kBwdBN >= t0 && tr / kBwdBN < t0 + kFlagTiles) any_target[group][tr / kBwdBN - t0] = 1;
 #pragma unroll
-  for (int k = 0; k < kFlagTiles; ++k) mt[k] = valid ? mt[k] - l : -INFINITY;
-  wmax[group][tid >> 5][lane] = warp_column_max32(mt, lane);  // lane k: the warp's max of tile t0 + k
+  for (int k = 0; k < 2 * kFlagTiles; ++k) mt[k] = valid ? mt[k] - l : -INFINITY;
+  wmax[group][tid >> 5][lane] = warp_column_max32(mt, lane);  // lane k: the warp's max of half j0 + k
   named_barrier(group + 1, kBwdBM);
   if (tid < kFlagTiles && t0 + tid < nt) {
-    const float m =
-        fmaxf(fmaxf(wmax[group][0][tid], wmax[group][1][tid]), fmaxf(wmax[group][2][tid], wmax[group][3][tid]));
-    const bool keep = !A.filter_on || m >= A.ln_eps;
-    A.P.flags[static_cast<int64_t>(b) * nt + t0 + tid] = keep ? 1 : (any_target[group][tid] ? 2 : 0);
+    int halves = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int k = 2 * tid + h;
+      const float m = fmaxf(fmaxf(wmax[group][0][k], wmax[group][1][k]), fmaxf(wmax[group][2][k], wmax[group][3][k]));
+      if (j0 + k < A.T && (!A.filter_on || m >= A.ln_eps)) halves |= 1 << h;
+    }
+    A.P.flags[static_cast<int64_t>(b) * nt + t0 + tid] = static_cast<uint8_t>(
+        halves != 0 ? (kFlagListed | (halves << 2)) : (any_target[group][tid] ? kFlagOnehotOnly : 0));
   }
   named_barrier(group + 1, kBwdBM);  // the shared arrays are reused by the group's next unit
 }
 
 // The listed tiles of row block b in vocabulary order (a block-wide scan of its flags, 1024 vocabulary
-// tiles per step) and the inverse map pos_b; the whole block.
+// tiles per step), the kept halves before each of them (hp_b, counted from the row block's offset
+// off_hb[b]) and the inverse map pos_b; the whole block.
 __device__ void row_list_block(const PlanArgs& A, int b) {
-  __shared__ int wsum[32];
-  __shared__ int carry;
+  __shared__ int wsum[32], hsum[32];
+  __shared__ int carry, hcarry;
   const BwdPlan& P = A.P;
   const int nt = P.nt;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const uint8_t* row = P.flags + static_cast<int64_t>(b) * nt;
-  if (threadIdx.x == 0) carry = P.offsets_b[b];
+  if (threadIdx.x == 0) {
+    carry = P.offsets_b[b];
+    hcarry = P.off_hb[b];
+  }
   __syncthreads();
   for (int t0 = 0; t0 < nt; t0 += kPlanThreads) {
     const int t = t0 + threadIdx.x;
-    const bool on = t < nt && row[t] == 1;
+    const int f = t < nt ? row[t] : 0;
+    const bool on = flag_state(f) == kFlagListed;
+    const int nh = on ? __popc(flag_halves(f)) : 0;
     const unsigned m = __ballot_sync(0xffffffffu, on);
-    if (lane == 0) wsum[w] = __popc(m);
+    int hx = nh;  // inclusive scan of the kept halves within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, hx, o);
+      if (lane >= o) hx += y;
+    }
+    if (lane == 31) {
+      wsum[w] = __popc(m);
+      hsum[w] = hx;
+    }
     __syncthreads();
-    int before = 0, total = 0;
+    int before = 0, total = 0, hbefore = 0, htotal = 0;
     for (int k = 0; k < 32; ++k) {
       before += k < w ? wsum[k] : 0;
       total += wsum[k];
+      hbefore += k < w ? hsum[k] : 0;
+      htotal += hsum[k];
     }
     if (on) {
       const int pos = carry + before + __popc(m & ((1u << lane) - 1u));
       const int slot = P.offsets_t[t] + P.rank[static_cast<int64_t>(b) * nt + t];
-      P.entries_b[pos] = make_int2(t, slot);
+      P.entries_b[pos] = make_int2(t, slot | (flag_halves(f) << kSlotBits));
+      P.hp_b[pos] = hcarry + hbefore + hx - nh;
       P.pos_b[slot] = pos;
     }
-    __syncthreads();  // everyone has read carry and wsum
-    if (threadIdx.x == 0) carry += total;
+    __syncthreads();  // everyone has read carry and the warp sums
+    if (threadIdx.x == 0) {
+      carry += total;
+      hcarry += htotal;
+    }
     __syncthreads();
   }
 }
@@ -247,7 +283,7 @@ __device__ void pair_list_warp(const PlanArgs& A, int t, int lane, int pass) {
     int b = 0, p = 0;
     int2 rr = make_int2(0, 0);
     if (i < i1) {
-      b = P.entries_t[i].x >> 2;
+      b = P.entries_t[i].x >> 4;
       p = P.pos_b[i];
       rr = P.rb_range[static_cast<int64_t>(c) * nb + b];
       start = ((p - rr.x) & 1) == 0;
@@ -257,9 +293,9 @@ __device__ void pair_list_warp(const PlanArgs& A, int t, int lane, int pass) {
       const int out = P.pstart_t[t] + k + __popc(mask & ((1u << lane) - 1u));
       const bool two = p + 1 < rr.y;
       const int t1 = two ? P.entries_b[p + 1].x : -1;
-      const int slot1 = two ? P.entries_b[p + 1].y : i;
+      const int slot1 = two ? (P.entries_b[p + 1].y & kSlotMask) : i;
       const uint8_t* row = P.flags + static_cast<int64_t>(b) * nt;
-      const int kept = (row[t] == 1 ? 1 : 0) | (two && row[t1] == 1 ? 2 : 0);
+      const int kept = flag_halves(row[t]) | (two ? flag_halves(row[t1]) << 2 : 0);
       P.pair_desc[out] = make_int4(b, t, t1, kept);
       P.pair_slot[out] = make_int2(i - slot_base, slot1 - slot_base);
     }
@@ -406,11 +442,12 @@ __device__ __forceinline__ int chunk_containing(const int* chunk_t, int n, int t
 //  0  zero the counters (the backward kernel's too) and the fp32 accumulator of dbias; the row
 //     scales (the fp32 accumulator of dE is zeroed a tenth per phase)
 //  1  tile flags (run with phase 0, whose results they do not read)
-//  2  per vocabulary tile: ranks of its listed tiles and their count; per row block: its count; the
-//     kept total; per vocabulary tile: rows whose target tile is onehot only, and their dbias terms
-//  3  scans: offsets_t, offsets_b, oh_off (three blocks)
-//  4  entries_t; row lists (entries_b, pos_b); the onehot-only rows, grouped by vocabulary tile;
-//     the vocabulary chunks (one block)
+//  2  per vocabulary tile: ranks of its listed tiles and their count; per row block: its listed tiles
+//     and kept halves; the kept halves in all; per vocabulary tile: rows whose target half is skipped,
+//     and their dbias terms
+//  3  scans: offsets_t, offsets_b, off_hb, oh_off (four blocks)
+//  4  entries_t; row lists (entries_b, hp_b, pos_b); the rows whose target half is skipped, grouped
+//     by vocabulary tile; the vocabulary chunks (one block)
 //  5  row ranges per chunk; the chunk of every vocabulary tile
 //  6  pair counts per vocabulary tile
 //  7  scan of the pair counts (pstart_t)
@@ -429,7 +466,12 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
   // 0
   if (gtid < 2) P.kept_total[gtid] = 0;  // kept_total and n_empty
   for (int64_t i = gtid; i < A.sync_ints; i += gthreads) A.sync[i] = 0;
-  for (int64_t i = gtid; i < nb; i += gthreads) P.cnt_b[i] = 0;
+  for (int64_t i = gtid; i < nb; i += gthreads) {
+    P.cnt_b[i] = 0;
+    P.cnt_hb[i] = 0;
+  }
+  for (int64_t i = gtid; i < kZeroHalfBytes / 16; i += gthreads)
+    reinterpret_cast<float4*>(A.zero_half)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int64_t i = gtid; i < nt; i += gthreads) {
     P.oh_cnt[i] = 0;
     P.oh_cur[i] = 0;
@@ -475,27 +517,32 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
 
   // 2
   for (int t = gwarp; t < nt; t += gwarps) {
-    int listed = 0;
+    int listed = 0, halves = 0;
     for (int b0 = 0; b0 < nb; b0 += 32) {
       const int b = b0 + lane;
-      const uint8_t f = b < nb ? P.flags[static_cast<int64_t>(b) * nt + t] : 0;
-      const unsigned on = __ballot_sync(0xffffffffu, f == 1);
-      if (f == 1) {
-        P.rank[static_cast<int64_t>(b) * nt + t] = listed + __popc(on & ((1u << lane) - 1u));
+      const int f = b < nb ? P.flags[static_cast<int64_t>(b) * nt + t] : 0;
+      const bool on = flag_state(f) == kFlagListed;
+      const unsigned m = __ballot_sync(0xffffffffu, on);
+      if (on) {
+        const int nh = __popc(flag_halves(f));
+        P.rank[static_cast<int64_t>(b) * nt + t] = listed + __popc(m & ((1u << lane) - 1u));
         atomicAdd(P.cnt_b + b, 1);
+        atomicAdd(P.cnt_hb + b, nh);
+        halves += nh;
       }
-      listed += __popc(on);
+      listed += __popc(m);
     }
+    halves = __reduce_add_sync(0xffffffffu, halves);
     if (lane == 0) {
       P.cnt_t[t] = listed;
-      atomicAdd(P.kept_total, listed);
+      atomicAdd(P.kept_total, halves);
     }
   }
   for (int64_t r = gtid; r < A.N; r += gthreads) {
     const int64_t tr = A.targets[r] - A.vs;  // only targets inside this shard have an onehot term here
     if (!valid_target(tr, A.V, A.ignore_index - A.vs)) continue;
     const int t = static_cast<int>(tr / kBwdBN);
-    if (P.flags[(r / kBwdBM) * nt + t] != 2) continue;
+    if (!target_half_skipped(P.flags[(r / kBwdBM) * nt + t], tr)) continue;
     atomicAdd(P.oh_cnt + t, 1);
     if (A.dbias_acc != nullptr) atomicAdd(A.dbias_acc + tr, -A.onehot_coef * A.scale[r]);
   }
@@ -506,21 +553,24 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
   if (blockIdx.x == 0) block_scan(P.cnt_t, nt, P.offsets_t);
   if (blockIdx.x == 1 % gridDim.x) block_scan(P.cnt_b, nb, P.offsets_b);
   if (blockIdx.x == 2 % gridDim.x) block_scan(P.oh_cnt, nt, P.oh_off);
+  if (blockIdx.x == 3 % gridDim.x) block_scan(P.cnt_hb, nb, P.off_hb);
   if (!grid_barrier(ctl, ++round)) return;
   zero_part(round + 1);
 
   // 4
   for (int64_t i = gtid; i < tiles; i += gthreads) {
-    if (P.flags[i] != 1) continue;
+    const int f = P.flags[i];
+    if (flag_state(f) != kFlagListed) continue;
     const int b = static_cast<int>(i / nt), t = static_cast<int>(i % nt);
-    P.entries_t[P.offsets_t[t] + P.rank[i]] = make_int2(b * 4 + 1, t);
+    P.entries_t[P.offsets_t[t] + P.rank[i]] = make_int2(b * 16 + f, t);
   }
+  if (gtid == 0) P.hp_b[P.offsets_b[nb]] = P.off_hb[nb];  // one past the last entry
   for (int b = blockIdx.x; b < nb; b += gridDim.x) row_list_block(A, b);
   for (int64_t r = gtid; r < A.N; r += gthreads) {
     const int64_t tr = A.targets[r] - A.vs;
     if (!valid_target(tr, A.V, A.ignore_index - A.vs)) continue;
     const int t = static_cast<int>(tr / kBwdBN);
-    if (P.flags[(r / kBwdBM) * nt + t] != 2) continue;
+    if (!target_half_skipped(P.flags[(r / kBwdBM) * nt + t], tr)) continue;
     P.oh_rows[P.oh_off[t] + atomicAdd(P.oh_cur + t, 1)] = static_cast<int>(r);
   }
   if (blockIdx.x == gridDim.x - 1) chunk_partition(A);
@@ -566,7 +616,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
   if (!last) return;
   __threadfence();  // the other blocks' grp_size entries are visible
   block_scan(P.grp_size, 2 * nchunks, P.grp_start);
-  if (threadIdx.x == 0) *A.filtered_tiles = tiles - static_cast<int64_t>(*P.kept_total);
+  if (threadIdx.x == 0) *A.filtered_tiles = static_cast<int64_t>(nb) * A.T - static_cast<int64_t>(*P.kept_total);
 }
 
 // The element-wise steps of the backward after the tensor-core kernel, in two launches:
@@ -744,7 +794,7 @@ __global__ void __launch_bounds__(256, 2) bwd_finalize_kernel(const __grid_const
         }
         const int64_t tl = F.targets[r] - F.vs;
         if (tl >= 0 && tl < F.V && F.targets[r] != F.ignore_index &&
-            F.flags[(r / kBwdBM) * F.nt + tl / kBwdBN] == 2)
+            target_half_skipped(F.flags[(r / kBwdBM) * F.nt + tl / kBwdBN], tl))
           add_bf16x8(acc, F.C + tl * D + d, -F.onehot_coef * sc);
         store8(F.dE_out != nullptr ? F.dE_out : static_cast<void*>(F.dE_acc), F.dE_out != nullptr, r * D + d, acc);
       }
@@ -761,10 +811,14 @@ __global__ void __launch_bounds__(256, 2) bwd_finalize_kernel(const __grid_const
 }
 
 // out[i] = 1 when backward tile i (row block i / nt, vocabulary tile i % nt) was skipped, 0 when kept.
-__global__ void skip_map_kernel(const uint8_t* __restrict__ flags, int64_t n, uint8_t* __restrict__ out) {
+__global__ void skip_map_kernel(const uint8_t* __restrict__ flags, int nt, int64_t T, int64_t n,
+                                uint8_t* __restrict__ out) {
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    out[i] = flags[i] == 1 ? 0 : 1;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = i / T, j = i % T;
+    const int f = flags[b * nt + j / 2];
+    out[i] = flag_state(f) == kFlagListed && ((flag_halves(f) >> (j & 1)) & 1) ? 0 : 1;
+  }
 }
 
 }  // namespace
@@ -798,9 +852,10 @@ cudaError_t launch_bwd_finalize(const BwdFinalize& F, int num_sms, cudaStream_t 
   return cudaGetLastError();
 }
 
-cudaError_t launch_skip_map(const uint8_t* flags, int64_t tiles, uint8_t* out, cudaStream_t s) {
-  if (tiles == 0) return cudaSuccess;
-  skip_map_kernel<<<static_cast<int>(std::min<int64_t>((tiles + 255) / 256, 4096)), 256, 0, s>>>(flags, tiles, out);
+cudaError_t launch_skip_map(const uint8_t* flags, int nb, int nt, int64_t T, uint8_t* out, cudaStream_t s) {
+  const int64_t n = static_cast<int64_t>(nb) * T;
+  if (n == 0) return cudaSuccess;
+  skip_map_kernel<<<static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096)), 256, 0, s>>>(flags, nt, T, n, out);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -14,16 +14,33 @@ namespace cce {
 // Forward tile: 128 rows x 256 vocabulary columns, K in blocks of 64 (one 128-byte swizzle row).
 constexpr int kFwdBM = 128;
 constexpr int kFwdBN = 256;
-constexpr int kSubTile = 128;  // vocabulary width of one saved tile max
+constexpr int kSubTile = 64;  // vocabulary width of one saved tile max (and of a skip-rule unit)
 
-// Backward tile: 128 rows x 128 vocabulary columns (the unit of the skip rule and of a gradient tile).
+// Backward tile: 128 rows x 128 vocabulary columns (a gradient tile and the unit of the work lists),
+// made of two 64-column halves. The skip rule decides each half (128 rows x kSubTile columns) on its
+// own; a tile is listed when either half is kept, and only its kept halves are recomputed, stored and
+// multiplied into dE.
 constexpr int kBwdBM = 128;
 constexpr int kBwdBN = 128;
+static_assert(kBwdBN == 2 * kSubTile, "a backward tile is two skip-rule halves");
+
+// Tile flags of the plan, one byte per (row block, vocabulary tile): bits 0-1 the state (0 nothing,
+// 1 listed, 2 onehot only: no half kept but a row of the block has its target in the tile), bits 2-3
+// the kept halves of a listed tile.
+constexpr int kFlagListed = 1;
+constexpr int kFlagOnehotOnly = 2;
+__host__ __device__ constexpr int flag_state(int f) { return f & 3; }
+__host__ __device__ constexpr int flag_halves(int f) { return (f >> 2) & 3; }
+// Slots in entries_b carry the tile's kept halves in bits 29-30.
+constexpr int kSlotBits = 29;
+constexpr int kSlotMask = (1 << kSlotBits) - 1;
+// Zeros standing for one 64-row K-block of a skipped half in the dC MMAs (64 x 64 bf16).
+constexpr int kZeroHalfBytes = 64 * kSubTile * 2;
 
 struct FwdLaunch {
   CUtensorMap tmE;  // bf16 [N, D], box 64 x 128, 128B swizzle
   CUtensorMap tmC;  // bf16 [V, D], box 64 x 256, 128B swizzle
-  int N, D, V, T;   // T = ceil(V / 128)
+  int N, D, V, T;   // T = ceil(V / kSubTile)
   const __nv_bfloat16* bias;  // [V] added to every row of logits, or null
   float* tile_max;  // [T, N]
   float* tile_sum;  // [T, N]: sum over the sub-tile of exp(z - tile_max)
@@ -86,16 +103,20 @@ static_assert(kGradBuffers >= 2, "the pairs of chunk c reuse the buffer of chunk
 
 struct BwdPlan {
   int nb, nt;
-  uint8_t* flags;   // [nb * nt]: 0 none, 1 kept, 2 onehot only
+  uint8_t* flags;   // [nb * nt]: state and kept halves (kFlagListed, kFlagOnehotOnly, flag_halves)
   int* rank;        // [nb * nt]: position of (b, t) among the listed row blocks of t
   int* cnt_t;       // [nt]
   int* offsets_t;   // [nt + 1]
-  int2* entries_t;  // [nb * nt]: (b * 4 + flag, t), by vocabulary tile then row block
+  int2* entries_t;  // [nb * nt]: (b * 16 + flag, t), by vocabulary tile then row block
   int* cnt_b;       // [nb]
   int* offsets_b;   // [nb + 1]
-  int2* entries_b;  // [nb * nt]: (t, slot in entries_t), by row block then vocabulary tile
+  int* cnt_hb;      // [nb]: kept halves per row block
+  int* off_hb;      // [nb + 1]: their prefix sums
+  int2* entries_b;  // [nb * nt]: (t, slot in entries_t | kept halves << kSlotBits), by row block then
+                    // vocabulary tile
+  int* hp_b;        // [nb * nt + 1]: kept halves before each entries_b position (over all row blocks)
   int* pos_b;       // [nb * nt]: for each entries_t position, the tile's position in entries_b
-  int* kept_total;
+  int* kept_total;  // kept halves
   int chunk_vt;     // vocabulary tiles per chunk at most once every tile is listed (sizes the arrays)
   int nchunks;      // chunks at most (arrays are sized for it); the plan's own count is *nchunks_dev
   int* nchunks_dev; // [1]: chunks of this plan
@@ -106,7 +127,8 @@ struct BwdPlan {
   int64_t chunk_g_tiles;  // listed tiles a chunk may hold (one gradient-tile buffer)
   int2* rb_range;   // [nchunks * nb]: entries [lo, hi) of each row block inside each chunk
   int* pstart_t;    // [nt + 1]: first pair whose first tile is in vocabulary tile t
-  int4* pair_desc;  // [pair capacity]: (b, t0, t1 or -1, kept bits), by t0 then b
+  int4* pair_desc;  // [pair capacity]: (b, t0, t1 or -1, kept halves: t0's in bits 0-1, t1's in 2-3),
+                    // by t0 then b
   int2* pair_slot;  // [pair capacity]: gradient-tile slots of t0 and t1, relative to the chunk
   int* grp_size;    // [2 * nchunks]: work items of each queue group (pairs of chunk c, then its dE/dC)
   int* grp_start;   // [2 * nchunks + 1]: their prefix sums
@@ -157,6 +179,8 @@ struct BwdArgs {
   const int* offsets_t;
   const int2* entries_t;
   const int2* entries_b;
+  const int* hp_b;
+  const void* zero_half;  // 8 KB of zeros: the gradient of a skipped half, as the dC MMAs read it
   uint8_t* gscratch;
   int* qctr;      // queue position, zero at launch
   int* counters;  // zero at launch: [ctr_g_b] gradient tiles stored per (chunk, row block),
@@ -168,7 +192,8 @@ struct BwdArgs {
 };
 
 struct BwdLaunch {
-  CUtensorMap tmE128, tmC128;  // bf16, box 64 x 128: K-blocks of the recompute
+  CUtensorMap tmE128;          // bf16, box 64 x 128: E K-blocks of the recompute
+  CUtensorMap tmC128;          // bf16, box 64 x 64: C K-blocks of one kept half of the recompute
   CUtensorMap tmE64, tmC64;    // bf16 operand slices of the dC / dE MMAs: 3-D box 64 x 64 x 4 (D % 256 == 0)
                                // or 2-D box 64 x 64
   CUtensorMap tmdC;            // dC output: bf16 box 64 x 32, or fp32 box 32 x 32
@@ -193,6 +218,7 @@ struct PlanArgs {
   float onehot_coef;       // 1 - label_smoothing
   float* dE_acc;           // [N, D] fp32, zeroed here
   float* dbias_acc;        // [V] fp32 or null, zeroed here; receives the onehot-only rows' terms
+  void* zero_half;         // [kZeroHalfBytes] zeroed here, read by the backward kernel
   int64_t* filtered_tiles;
   int* sync;               // [sync_ints] the backward kernel's queue position and counters, zeroed here
   int64_t sync_ints;
@@ -212,7 +238,7 @@ cudaError_t launch_bwd(const BwdLaunch& L, bool after_kernel, cudaStream_t s);
 struct BwdFinalize {
   int64_t N, D, V, vs, ignore_index;
   int nt;
-  const uint8_t* flags;       // the plan's tile flags [nb * nt]
+  const uint8_t* flags;       // the plan's tile flags [nb * nt] (state and kept halves)
   const int* empty_list;
   const int* n_empty;
   const int* oh_off;
@@ -236,8 +262,8 @@ struct BwdFinalize {
 cudaError_t launch_empty_tiles(const BwdFinalize& F, int num_sms, bool after_kernel, cudaStream_t s);
 // dE's last terms and conversion, dbias (after the tensor-core kernel and launch_empty_tiles).
 cudaError_t launch_bwd_finalize(const BwdFinalize& F, int num_sms, cudaStream_t s);
-// out[i] = 1 if tile i of the plan's flags was skipped, 0 if it was kept (i < tiles).
-cudaError_t launch_skip_map(const uint8_t* flags, int64_t tiles, uint8_t* out, cudaStream_t s);
+// out[b * T + j] = 1 if half j of row block b was skipped, 0 if it was kept (b < nb, j < T).
+cudaError_t launch_skip_map(const uint8_t* flags, int nb, int nt, int64_t T, uint8_t* out, cudaStream_t s);
 
 cudaError_t launch_fwd_lse(const FwdLaunch& L, cudaStream_t s);
 

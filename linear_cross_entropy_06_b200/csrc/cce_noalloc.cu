@@ -121,7 +121,7 @@ extern "C" cce_status cce_forward_noalloc(const cce_problem* p, const void* E, c
     char msg[256];
     snprintf(msg, sizeof(msg),
              "cce_forward_noalloc: this problem needs %zu bytes of scratch, more than the %zu bytes the library "
-             "holds for allocation-free calls (about ceil(V/128) * N * 4 bytes); use cce_forward with a workspace",
+             "holds for allocation-free calls (about ceil(V/64) * N * 4 bytes); use cce_forward with a workspace",
              need, kNoAllocScratchBytes);
     return fail(CCE_ERR_UNSUPPORTED, msg);
   }

@@ -203,7 +203,7 @@ def cce_backward(E: torch.Tensor, C: torch.Tensor, targets: torch.Tensor, lse: t
                  vocab_start: int = 0, vocab_total: int = 0):
     """Run the backward. Returns (dE, dC, filtered_tiles) as device tensors, then dbias when it is
     computed (``dbias``; by default whenever ``bias`` is given), then, with ``skip_map``, the uint8
-    [ceil(N / tile_rows), ceil(V / tile_cols)] map of skipped tiles (1 skipped, 0 kept).
+    [ceil(N / tile_rows), ceil(V / tile_cols)] map of the skip rule's units (1 skipped, 0 kept).
     ``out_fp32``: False / OUT_BF16, True / OUT_FP32, or OUT_DE_FP32 (dE fp32, dC and dbias bf16).
     ``vocab_start`` / ``vocab_total``: C is rows [vocab_start, vocab_start + V) of a classifier of
     vocab_total rows (0: not sharded); lse and count are then the merged ones."""

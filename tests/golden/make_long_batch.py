@@ -1,7 +1,8 @@
 """Writes long_batch_oracle.npz: the fp64 oracle's per-row LSE and per-token loss, its skip
 decision for every tile (and which tiles lie within the oracle's borderline window of ln eps) for
 the long-batch workload (N = 32768 tokens, D = 4096, V = 128256, Zipf
-targets, 5 % ignored, reduction 'none', skipping at 2^-12 on 128 x 128 tiles).
+targets, 5 % ignored, reduction 'none', skipping at 2^-12 on units of 128 rows x 64 vocabulary
+columns).
 
 A full fp64 pass over that problem takes minutes of CPU time, so the GPU parity test reads these
 values instead of recomputing them; it evaluates the cheaper parts (dE of whole row blocks, dC of
@@ -25,7 +26,7 @@ from linear_cross_entropy_06_b200.inputs import make_inputs  # noqa: E402
 from oracle import cce_oracle as O  # noqa: E402
 
 EPS = 2.0 ** -12
-TILE = (128, 128)  # rows x vocabulary columns of the skip rule's tile
+TILE = (128, 64)  # rows x vocabulary columns of the skip rule's unit
 WINDOW = 2e-3  # the oracle's borderline window (its default)
 OUT = os.path.join(HERE, "long_batch_oracle.npz")
 

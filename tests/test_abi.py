@@ -60,7 +60,7 @@ def _p(N=256, D=128, V=4096, red=1, ignore=-100, reserved=0):
 
 def test_sizes(lib):
     p = _p(N=300, D=136, V=1000)
-    T = -(-1000 // 128)
+    T = -(-1000 // 64)  # saved maxima per 64 vocabulary columns
     assert lib.cce_tile_max_len(ctypes.byref(p)) == T * 300
     fw = lib.cce_forward_workspace_size(ctypes.byref(p))
     # header, tile sums [T, N], target logits, row losses, and for label smoothing the column
@@ -74,7 +74,7 @@ def test_sizes(lib):
     assert lib.cce_forward_workspace_size(ctypes.byref(big)) < 32768 * 128256 * 2 // 8
     assert lib.cce_tile_max_len(ctypes.byref(big)) * 4 < 32768 * 128256 * 2 // 8
     r, c = ops.backward_tile_shape()
-    assert (r, c) == (128, 128)
+    assert (r, c) == (128, 64)
 
 
 @pytest.mark.parametrize("bad", [dict(D=7), dict(D=0), dict(V=0), dict(N=-1), dict(red=3), dict(reserved=1)])
@@ -142,8 +142,8 @@ def test_plain_c_caller_compiles_links_and_runs():
         out = subprocess.run([exe], check=True, capture_output=True, text=True, timeout=60).stdout
     vals = dict(line.split(" ", 1) for line in out.strip().splitlines())
     assert int(vals["version"]) >= 300
-    assert vals["tile"] == "128 128"
-    assert int(vals["tile_max_len"]) == 4096 * ((128256 + 127) // 128)
+    assert vals["tile"] == "128 64"
+    assert int(vals["tile_max_len"]) == 4096 * ((128256 + 63) // 64)
     assert int(vals["fwd_ws"]) > 0 and int(vals["bwd_ws"]) > 0
     assert vals["bad_status"].startswith("1 ")  # CCE_ERR_INVALID_ARG
     assert "multiple of 8" in vals["message"]

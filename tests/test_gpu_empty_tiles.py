@@ -23,7 +23,8 @@ from test_gpu_bias import check_bias, make_bias
 
 pytestmark = pytest.mark.gpu
 
-TILE = 128
+TILE = 128  # vocabulary tile of the work lists
+HALF = 64   # vocabulary columns of a skip-rule unit (half a tile)
 
 
 def crowded_inputs(seed):
@@ -49,14 +50,14 @@ def test_empty_tiles_with_long_target_lists(device, variant, reduction):
         r = check_bias(inp, None, device, reduction, grad_out=g)
     else:
         r = check_bias(inp, make_bias(V, 83, scale=0.05), device, reduction, grad_out=g, ls=0.1, zl=1e-4)
-    assert r["filtered"] == (N // TILE) * (V // TILE)  # every tile skipped at eps = 2^-12
+    assert r["filtered"] == (N // TILE) * (V // HALF)  # every half skipped at eps = 2^-12
 
 
 def test_empty_tiles_fp32_outputs(device):
     inp = crowded_inputs(84)
     r = check_bias(inp, make_bias(inp.C.shape[0], 85, scale=0.05), device, "sum", grad_out=torch.tensor([0.5]),
                    out_fp32=True, ls=0.2)
-    assert r["filtered"] == (512 // TILE) * (16384 // TILE)
+    assert r["filtered"] == (512 // TILE) * (16384 // HALF)
 
 
 @pytest.mark.parametrize("D,out_fp32", [(33000, False), (16400, True)])
@@ -64,10 +65,11 @@ def test_empty_tiles_wider_than_the_image(device, D, out_fp32):
     """A dC row wider than the kernel's 64 KB shared-memory image (bf16 D > 32768, fp32 D > 16384):
     the constant row goes out in column windows. A bias of 20 on token 5 puts every row's LSE near
     20, so every vocabulary tile but the first is skipped in every row block (the targets elsewhere
-    keep their onehot rows), with label smoothing for a non-zero constant row."""
+    keep their onehot rows), and the first tile keeps only the half that holds token 5 (its other
+    half reads as zeros in the dC MMAs), with label smoothing for a non-zero constant row."""
     N, V = 128, 1024
     inp = make_inputs("tiny", N=N, D=D, V=V, seed=86 + D, ignore_frac=0.05)
     bias = torch.zeros(V, dtype=torch.bfloat16)
     bias[5] = 20.0
     r = check_bias(inp, bias, device, "mean", out_fp32=out_fp32, ls=0.1)
-    assert r["filtered"] == (N // TILE) * (V // TILE) - 1
+    assert r["filtered"] == (N // TILE) * (V // HALF) - 1  # only the half holding token 5 is kept

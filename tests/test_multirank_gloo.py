@@ -65,14 +65,32 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     assert capsys.readouterr().out == ""
 
 
-def test_algorithmic_flops_definition():
-    """The metric's flop count: 2 N V D forward, 6 * 128 * 128 * D per kept 128 x 128 tile."""
+def test_issued_backward_work():
+    """The backward's issued tensor-core work: recompute and dE over kept 128 x 64 units, dC over
+    both units of every 128 x 128 tile with a kept unit."""
+    import torch
     import bench
 
-    fwd, bwd = bench.algorithmic_flops(4096, 4096, 128256, 7407, (128, 128))
+    # 2 row blocks x 5 units (the last tile has one unit): 0 = kept, 1 = skipped
+    skip_map = torch.tensor([[0, 1, 1, 1, 1],
+                             [1, 0, 0, 0, 0]], dtype=torch.uint8)
+    assert bench.listed_tile_count(skip_map) == 1 + 3
+    kept_units = int((skip_map == 0).sum())
+    assert kept_units == 5
+    D = 256
+    assert bench.issued_mma_flops(D, kept_units, 4, (128, 64)) == \
+        4 * 128 * 64 * D * 5 + 2 * 128 * 128 * D * 4
+
+
+def test_algorithmic_flops_definition():
+    """The metric's flop count: 2 N V D forward, 6 * 128 * 64 * D per kept 128 x 64 unit of the skip
+    rule (recompute, dE and dC of its logits)."""
+    import bench
+
+    fwd, bwd = bench.algorithmic_flops(4096, 4096, 128256, 8062, (128, 64))
     assert fwd == 2 * 4096 * 128256 * 4096
-    assert bwd == 6 * 128 * 128 * 4096 * 7407
-    # every workload of the bench has N and V multiples of 128 (no partial tile is counted)
+    assert bwd == 6 * 128 * 64 * 4096 * 8062
+    # every workload of the bench has N and V multiples of 128 (no partial unit is counted)
     from linear_cross_entropy_06_b200.inputs import WORKLOADS
     for w in WORKLOADS.values():
         if w.name != "tiny":
@@ -109,7 +127,7 @@ def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
     assert cpu["kind"] == "oracle" and cpu["value"] == line["value"] and cpu["cores"] >= 1 and cpu["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
-    assert bench.ORACLE_SKIP_TILE == (128, 128)
+    assert bench.ORACLE_SKIP_TILE == (128, 64)
     # cores = the BLAS pool that runs the oracle's matmul, at least one thread and at most the host's CPUs
     assert cpu["cores"] == bench.oracle_threads() and 1 <= cpu["cores"] <= (os.cpu_count() or 1)
 
