@@ -49,12 +49,12 @@ KERNEL_SOURCES = {  # the kernel and what sets up its work (maps, plan, chunking
 }
 TRAFFIC_BYTES = {
     "fwd_lse_kernel": {
-        (4096, 4096, 128256): ("274bc2c2fdd722d6dcf0ad78e8fc152431dbf70a49bafff5edc45fa2ed59d1bd",
-                               1085109504 + 35097856),
+        (4096, 4096, 128256): ("88deeb025a0b2e01974e376c5d1e0a0f628c3c281c1b57310147076a4a529f48",
+                               1085084928 + 67180288),
     },
     "bwd_kernel": {
-        (4096, 4096, 128256): ("8aa37d8deeff27865444105210447e1c4d2b9b897fd67b7048465d22fc480c08",
-                               5528850176 + 1791886848),
+        (4096, 4096, 128256): ("6526e827035f2ab17d905cc8499f4fa38b38ab4ae3e922ffbe2df9989fd1a433",
+                               4313867520 + 1672815360),
     },
 }
 
