@@ -211,10 +211,12 @@ SplitWs carve_split(const cce_problem* p, int32_t out_fp32, void* base) {
   w.plan.chunk_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(w.plan.nchunks + 1)));
   w.plan.rb_range = reinterpret_cast<int2*>(take(sizeof(int2) * static_cast<size_t>(w.plan.nchunks) * nb));
   w.plan.pstart_t = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt + 1)));
-  // a row block with k listed tiles in a chunk forms ceil(k / 2) pairs there
-  const size_t pairs = static_cast<size_t>((tiles + static_cast<int64_t>(w.plan.nchunks) * nb) / 2 + 1);
-  w.plan.pair_desc = reinterpret_cast<int4*>(take(sizeof(int4) * pairs));
-  w.plan.pair_slot = reinterpret_cast<int2*>(take(sizeof(int2) * pairs));
+  // a row block with k kept halves (at most 2 per listed tile) in a chunk forms ceil(k / 4) quads there
+  const size_t quads = static_cast<size_t>(tiles / 2 + static_cast<int64_t>(w.plan.nchunks) * nb + 1);
+  w.plan.quad_b = reinterpret_cast<int*>(take(sizeof(int) * quads));
+  w.plan.quad_h = reinterpret_cast<int4*>(take(sizeof(int4) * quads));
+  w.plan.quad_s = reinterpret_cast<int4*>(take(sizeof(int4) * quads));
+  w.plan.cnt_ht = reinterpret_cast<int*>(take(sizeof(int) * static_cast<size_t>(nt)));
   w.plan.S = static_cast<int>(ceil_div(p->D, cce::kGemmSlice));
   w.plan.grp_size = reinterpret_cast<int*>(take(sizeof(int) * 2 * static_cast<size_t>(w.plan.nchunks)));
   w.plan.grp_start = reinterpret_cast<int*>(take(sizeof(int) * (2 * static_cast<size_t>(w.plan.nchunks) + 1)));
@@ -431,8 +433,10 @@ cce_status backward_split(const cce_problem* p, const void* E, const void* C, co
   A.nde = w.plan.nde;
   A.chunk_t = w.plan.chunk_t;
   A.pstart_t = w.plan.pstart_t;
-  A.pair_desc = w.plan.pair_desc;
-  A.pair_slot = w.plan.pair_slot;
+  A.quad_b = w.plan.quad_b;
+  A.quad_h = w.plan.quad_h;
+  A.quad_s = w.plan.quad_s;
+  A.cnt_ht = w.plan.cnt_ht;
   A.rb_range = w.plan.rb_range;
   A.offsets_t = w.plan.offsets_t;
   A.entries_t = w.plan.entries_t;

@@ -7,13 +7,13 @@
 // abstract (logits are recomputed blockwise and never stored).
 //
 // Work items, per vocabulary chunk c (its gradient tiles live in scratch buffer c mod kGradBuffers):
-//   pair   two consecutive listed 128 x 128 tiles (b, t0), (b, t1) of row block b in the chunk, of
-//          which only the kept 64-column halves (one to four) are computed: S = E_b [C_h ...]^T
-//          (+ bias) over those halves (tcgen05 M=128 N=64 x halves K=D), then
+//   quad   up to four consecutive kept 64-column halves of row block b in the chunk (from one or
+//          several of its listed tiles): S = E_b [C_h ...]^T (+ bias) over those halves (tcgen05
+//          M=128 N=64 x halves K=D), then
 //          G = scale_r (1 + 2 zl LSE_r) exp(S - LSE_r) - scale_r (1 - ls) [v = t_r] in fp32, rounded
-//          to bf16 into a 128B-swizzled shared tile, one 16 KB bulk store per kept half into the
-//          tile's slot of the scratch buffer; with a dbias output, the column sums of the fp32 G are
-//          added into it.
+//          to bf16 into a 128B-swizzled shared region (two halves at a time), one 16 KB bulk store
+//          per half into its tile's slot of the scratch buffer; with a dbias output, the column sums
+//          of the fp32 G are added into it.
 //   dE     (row block b, 256-column slice s of D): sum over the kept halves h of the chunk's listed
 //          tiles t of G_bth C_th[:, s] in TMEM, then one fp32 TMA reduce-add into dE_acc
 //          (split-reduce over chunks).
@@ -22,15 +22,15 @@
 //          whose target half in t was skipped and the label-smoothing term, written once by TMA
 //          store: every listed tile of t lies in t's chunk, so dC needs no reduction.
 //
-// Scheduling: a global queue holds the items in the order pairs(0), pairs(1), dE/dC(0), pairs(2),
-// dE/dC(1), ..., pairs(n-1), dE/dC(n-2), dE/dC(n-1): the dE/dC items of a chunk come one group of
-// pairs after the chunk's own pairs, so their gradient tiles are normally stored by the time they
+// Scheduling: a global queue holds the items in the order quads(0), quads(1), dE/dC(0), quads(2),
+// dE/dC(1), ..., quads(n-1), dE/dC(n-2), dE/dC(n-1): the dE/dC items of a chunk come one group of
+// quads after the chunk's own quads, so their gradient halves are normally stored by the time they
 // are claimed. CTAs claim items one at a time with an atomic counter, so a claimed item always
-// belongs to a running CTA. Inside a chunk the pairs are ordered by vocabulary tile and the dE and
+// belongs to a running CTA. Inside a chunk the quads are ordered by vocabulary tile and the dE and
 // dC items by slice of D, so that the items running at the same time read the same C tiles and
 // the same columns of C and E from L2. Dependencies point only to earlier items:
-//   a dE item waits until every gradient tile of its row block in the chunk is stored, a dC item
-//   until every gradient tile of its vocabulary tile is, and a pair of chunk c waits, before it
+//   a dE item waits until every kept half of its row block in the chunk is stored, a dC item
+//   until every kept half of its vocabulary tile is, and a quad of chunk c waits, before it
 //   stores, until every dE/dC item of chunk c - kGradBuffers (the buffer's previous user) has
 //   read it.
 // Every such wait is bounded. Because items are claimed in order and the smallest unfinished item
@@ -39,10 +39,10 @@
 //
 // Design (B200): one CTA per SM, 7 warps, 224 KB of shared memory.
 //   warp 0      producer: per stage (at most 48 KB, 4 deep) either the E_b K-block of 64 and one
-//               64 x 64 C box per kept half (pair), or one K-half of a gradient tile (16 KB bulk
+//               64 x 64 C box per half of the quad, or one K-half of a gradient tile (16 KB bulk
 //               copy, or zeros for a skipped half) and the 64 x 256 operand slice (dE, dC).
 //   warp 1      TMEM owner (two 256-column fp32 buffers); one lane issues tcgen05.mma M=128 N=256.
-//   warps 2..5  write-out: G formation and bulk stores (pair), or TMEM -> swizzled staging -> TMA
+//   warps 2..5  write-out: G formation and bulk stores (quad), or TMEM -> swizzled staging -> TMA
 //               store / reduce-add (dC / dE), while the MMA fills the other TMEM buffer.
 //   warp 6      scheduler: claims and decodes items into an 8-deep shared ring, at most LOOKAHEAD
 //               items ahead of the producer.
@@ -61,29 +61,29 @@ constexpr int PART = 16384;              // 128 x 64 bf16: one K-block of 128 ro
 constexpr int X_BOX = 8192;              // 64 x 64 bf16
 constexpr int STAGE_BYTES = 3 * PART;    // 48 KB
 constexpr int TILE_BYTES = kGradTileBytes;
-constexpr int REGION_BYTES = TILE_BYTES;  // one G tile (pair) or 4 x 8 KB staging (dE / dC)
+constexpr int REGION_BYTES = TILE_BYTES;  // two G halves (quad) or 4 x 8 KB staging (dE / dC)
 constexpr int STG_WARP = 8192;
 constexpr int RING = 8;
 constexpr int NUM_THREADS = 224;
 constexpr int TMEM_COLS = 512;
 
-enum Kind : int { kPair = 0, kDE = 1, kDC = 2, kEnd = 3 };
+enum Kind : int { kQuad = 0, kDE = 1, kDC = 2, kEnd = 3 };
 
 // A decoded work item, written by the scheduler into the shared ring (16-byte aligned: it is
 // copied as int4).
 struct alignas(16) WorkItem {
   int kind;
   int chunk;
-  int key;         // pair, dE: row block b; dC: vocabulary tile t
-  int s;           // dE, dC: slice of D; pair: kept halves (bits 0-1 of t0, bits 2-3 of t1)
-  int begin, end;  // dE, dC: list entries; pair: vocabulary tiles t0 and t1 (-1 when absent)
-  int slot0;       // pair: slot of t0 in the chunk's buffer; dE, dC: the chunk's first slot
-  int slot1;       // pair: slot of t1; dE: stages (kept halves of the entries)
-  int dep_idx;     // counter this item waits on (-1: none): before its loads (dE, dC) or stores (pair)
+  int key;         // quad, dE: row block b; dC: vocabulary tile t
+  int s;           // dE, dC: slice of D; quad: its halves (1 to 4)
+  int begin, end;  // dE, dC: list entries; quad: halves 0 and 1, each 2 t + h (-1 when absent)
+  int slot0;       // quad: slot of half 0's tile in the chunk's buffer; dE, dC: the chunk's first slot
+  int slot1;       // quad: slot of half 1's tile; dE: stages (kept halves of the entries)
+  int dep_idx;     // counter this item waits on (-1: none): before its loads (dE, dC) or stores (quad)
   int dep_val;     // value the counter must reach
-  int oh_begin;    // dC: rows whose target tile in this vocabulary tile was skipped, oh_rows[oh_begin:oh_end]
-  int oh_end;
-  int pad[4];
+  int oh_begin;    // dC: rows whose target half in this vocabulary tile was skipped,
+  int oh_end;      //     oh_rows[oh_begin:oh_end]; quad: halves 2 and 3
+  int pad[4];      // quad: slots of halves 2 and 3
 };
 static_assert(sizeof(WorkItem) == 64, "ring entries are 64 bytes");
 
@@ -108,8 +108,8 @@ constexpr uint32_t LOOKAHEAD = 2;
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + REGION_BYTES + kNumBars * 8 + RING * 64 + 16;
 static_assert(SMEM_BYTES <= 232448, "fits the 227 KB opt-in shared memory of an SM");
 
-// S = E_b [C_h ...]^T over nh kept halves: N = 64 nh
-__device__ __forceinline__ uint32_t idesc_pair(int nh) {
+// S = E_b [C_h ...]^T over the quad's nh halves: N = 64 nh
+__device__ __forceinline__ uint32_t idesc_quad(int nh) {
   constexpr uint32_t d1 = idesc_bf16(BM, 1 * kSubTile, false, false), d2 = idesc_bf16(BM, 2 * kSubTile, false, false),
                      d3 = idesc_bf16(BM, 3 * kSubTile, false, false), d4 = idesc_bf16(BM, 4 * kSubTile, false, false);
   return nh <= 1 ? d1 : nh == 2 ? d2 : nh == 3 ? d3 : d4;
@@ -140,11 +140,19 @@ __device__ __forceinline__ void read_item(const WorkItem* ring, int idx, WorkIte
   const int4* src = reinterpret_cast<const int4*>(ring + idx);
   int4* dst = reinterpret_cast<int4*>(&it);
 #pragma unroll
-  for (int i = 0; i < 3; ++i) dst[i] = src[i];
+  for (int i = 0; i < 4; ++i) dst[i] = src[i];
 }
 
-// Queue group g -> (chunk, whether it holds the chunk's pairs). The groups are pairs(0), then
-// pairs(c), dE/dC(c - 1) for c = 1 .. n-1, then dE/dC(n - 1).
+// Half j (0..3) of a quad item: 2 t + h, and its tile's slot in the chunk's buffer.
+__device__ __forceinline__ int quad_half(const WorkItem& it, int j) {
+  return j == 0 ? it.begin : j == 1 ? it.end : j == 2 ? it.oh_begin : it.oh_end;
+}
+__device__ __forceinline__ int quad_slot(const WorkItem& it, int j) {
+  return j == 0 ? it.slot0 : j == 1 ? it.slot1 : j == 2 ? it.pad[0] : it.pad[1];
+}
+
+// Queue group g -> (chunk, whether it holds the chunk's quads). The groups are quads(0), then
+// quads(c), dE/dC(c - 1) for c = 1 .. n-1, then dE/dC(n - 1).
 __device__ __forceinline__ int2 group_of(int g, int nchunks) {
   if (g == 0) return make_int2(0, 1);
   if (g == 2 * nchunks - 1) return make_int2(nchunks - 1, 0);
@@ -163,15 +171,19 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, int nchun
   it.oh_begin = it.oh_end = 0;
   if (gc.y) {
     const int64_t pi = static_cast<int64_t>(A.pstart_t[t_begin]) + local;
-    const int4 d = A.pair_desc[pi];
-    const int2 sl = A.pair_slot[pi];
-    it.kind = kPair;
-    it.key = d.x;
-    it.begin = d.y;
-    it.end = d.z;
-    it.s = d.w;
-    it.slot0 = sl.x;
+    const int4 h = A.quad_h[pi];
+    const int4 sl = A.quad_s[pi];
+    it.kind = kQuad;
+    it.key = A.quad_b[pi];
+    it.begin = h.x;  // the halves, 2 t + h
+    it.end = h.y;
+    it.oh_begin = h.z;
+    it.oh_end = h.w;
+    it.s = (h.x >= 0 ? 1 : 0) + (h.y >= 0 ? 1 : 0) + (h.z >= 0 ? 1 : 0) + (h.w >= 0 ? 1 : 0);
+    it.slot0 = sl.x;  // their tiles' slots
     it.slot1 = sl.y;
+    it.pad[0] = sl.z;
+    it.pad[1] = sl.w;
     if (c >= kGradBuffers) {  // the buffer's previous chunk must have been read by its dE / dC items
       const int prev = c - kGradBuffers;
       it.dep_idx = A.ctr_b_done + prev;
@@ -197,6 +209,7 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, int nchun
       it.end = r.y;
       it.slot1 = A.hp_b[r.y] - A.hp_b[r.x];
       it.dep_idx = A.ctr_g_b + c * A.nb + it.key;
+      it.dep_val = it.slot1;  // every kept half of the row block in the chunk is stored
     } else {  // slice-major too: concurrent dC items read the same columns of E
       const int v = local - nde * S;
       const int ndc = A.ndc[c];
@@ -206,11 +219,11 @@ __device__ __forceinline__ void decode_item(int w, int g, int g_begin, int nchun
       it.begin = A.offsets_t[it.key];
       it.end = A.offsets_t[it.key + 1];
       it.dep_idx = A.ctr_g_t + it.key;
+      it.dep_val = A.cnt_ht[it.key];  // every kept half of the vocabulary tile is stored
       it.oh_begin = A.oh_off[it.key];
       it.oh_end = A.oh_off[it.key + 1];
     }
-    it.dep_val = it.end - it.begin;
-    // test hook: the dE items of the first chunk wait for one gradient tile more than the pairs
+    // test hook: the dE items of the first chunk wait for one gradient half more than the quads
     // store, so their bounded wait runs out
     if (A.inject_stall && c == 0 && it.kind == kDE) ++it.dep_val;
   }
@@ -298,7 +311,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int4* dst = reinterpret_cast<int4*>(ring + idx);
         const int4* src = reinterpret_cast<const int4*>(&it);
 #pragma unroll
-        for (int i = 0; i < 3; ++i) dst[i] = src[i];
+        for (int i = 0; i < 4; ++i) dst[i] = src[i];
         mbar_arrive(bar(kItemFull + idx));  // release: the entry is visible to the waiters
         if (it.kind == kEnd) break;
       }
@@ -318,10 +331,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive(bar(kItemEmpty + idx));
         mbar_arrive(bar(kItemTaken + idx));
         if (it.kind == kEnd) break;
-        if (it.kind == kPair) {
-          if (it.s == 0) continue;  // no kept half: nothing to recompute
+        if (it.kind == kQuad) {
+          if (it.s == 0) continue;  // no half: nothing to recompute
           const int rb = it.key * BM;
-          const uint32_t stage_bytes = PART + static_cast<uint32_t>(__popc(it.s)) * X_BOX;
+          const uint32_t stage_bytes = PART + static_cast<uint32_t>(it.s) * X_BOX;
           for (int kb = 0; kb < num_kb; ++kb) {
             if (!mbar_wait(bar(kEmpty + stage), phase ^ 1u, wc)) {
               ok = false;
@@ -330,13 +343,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t dst = smem_u32(stages + stage * STAGE_BYTES);
             mbar_arrive_expect_tx(bar(kFull + stage), stage_bytes);
             tma_load_2d(dst, &tmE128, bar(kFull + stage), kb * BK, rb);
-            uint32_t off = PART;  // the kept halves' C rows, in the order of their bits
 #pragma unroll
-            for (int bit = 0; bit < 4; ++bit) {
-              if ((it.s >> bit) & 1) {
-                const int vrow = (bit < 2 ? it.begin : it.end) * BN + (bit & 1) * kSubTile;
-                tma_load_2d(dst + off, &tmC128, bar(kFull + stage), kb * BK, vrow);
-                off += X_BOX;
+            for (int j = 0; j < 4; ++j) {  // the quad's halves' C rows, in order
+              if (j < it.s) {
+                const int th = quad_half(it, j);
+                const int vrow = (th >> 1) * BN + (th & 1) * kSubTile;
+                tma_load_2d(dst + PART + j * X_BOX, &tmC128, bar(kFull + stage), kb * BK, vrow);
               }
             }
             ++issued[stage];
@@ -418,14 +430,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         read_item(ring, idx, it);
         mbar_arrive(bar(kItemEmpty + idx));
         if (it.kind == kEnd) break;
-        const bool pair = it.kind == kPair;
-        if (pair ? it.s == 0 : it.begin == it.end) continue;  // no MMA for this item
+        const bool quad = it.kind == kQuad;
+        if (quad ? it.s == 0 : it.begin == it.end) continue;  // no MMA for this item
         const int a = acc_iter & 1;
         if (!mbar_wait(bar(kAccEmpty + a), ((acc_iter >> 1) & 1u) ^ 1u, wc)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(a * 2 * BN);
-        const int nstage = pair ? num_kb : (it.kind == kDE ? it.slot1 : 2 * (it.end - it.begin));
-        const uint32_t idesc = pair ? idesc_pair(__popc(it.s)) : (it.kind == kDE ? IDESC_DE : IDESC_DC);
+        const int nstage = quad ? num_kb : (it.kind == kDE ? it.slot1 : 2 * (it.end - it.begin));
+        const uint32_t idesc = quad ? idesc_quad(it.s) : (it.kind == kDE ? IDESC_DE : IDESC_DC);
         for (int j = 0; j < nstage; ++j) {
           if (!mbar_wait(bar(kFull + stage), phase, wc)) {
             ok = false;
@@ -436,7 +448,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // 16 of the stage's 64 K values per MMA
             uint64_t adesc, bdesc;
-            if (pair) {  // A = E_b K-block, B = the kept halves' C rows (64 nh rows of 128 bytes, contiguous)
+            if (quad) {  // A = E_b K-block, B = the quad's halves' C rows (64 per half, rows of 128 bytes)
               adesc = sdesc_sw128(s0 + 32u * kk, 16, 1024);
               bdesc = sdesc_sw128(s0 + PART + 32u * kk, 16, 1024);
             } else {
@@ -472,7 +484,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t stg = reg0 + static_cast<uint32_t>(q * STG_WARP);
     uint32_t acc_iter = 0, rphase = 0, gphase = 0;
     uint32_t img = 0;  // which of the two 4 KB staging images of this warp comes next
-    bool region_shared = true;  // the last item used the whole region (a pair's G tile)
+    bool region_shared = true;  // the last item used the whole region (a quad's G halves)
     bool ok = true;
     // Every lane waits (and acquires) itself; the vote makes the outcome warp-uniform, so the warp
     // stays converged for the .sync.aligned TMEM loads and takes one branch on failure.
@@ -500,7 +512,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (it.kind == kEnd) break;
       const int a = acc_iter & 1;
 
-      if (it.kind == kPair) {
+      if (it.kind == kQuad) {
         const int b = it.key;
         const int r = b * BM + row;
         const float lse_r = (r < A.N) ? A.lse[r] : 0.f;
@@ -520,45 +532,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (leader && it.dep_idx >= 0 && !wait_counter(A.counters + it.dep_idx, it.dep_val, wc)) ok = false;
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         uint8_t* buf = buffer(it.chunk);
-        const int ntiles = it.end >= 0 ? 2 : 1;
-        for (int u = 0; u < ntiles && ok; ++u) {
-          const int t = u == 0 ? it.begin : it.end;
-          const int hm = (it.s >> (2 * u)) & 3;  // this tile's kept halves
-          const int vb = t * BN;
-          const int64_t rel = tg - vb;
-          const int tcol = (tvalid && rel >= 0 && rel < BN) ? static_cast<int>(rel) : -1;  // -scale_r here
+        // rounds of up to two halves: the region holds two 64-column parts
+        for (int j0 = 0; j0 < it.s && ok; j0 += 2) {
           if (!region_free()) {
             ok = false;
             break;
           }
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            const int hf = c / (kSubTile / 32);  // the half this 32-column piece lies in
-            if (!((hm >> hf) & 1)) continue;      // a skipped half has no gradient tile part
-            float v[32];
-            const int col0 = vb + c * 32;
-            // accumulator columns: 64 per kept half of the pair, in the order of their bits
-            const int acol = __popc(it.s & ((1 << (2 * u + hf)) - 1)) * kSubTile + (c % (kSubTile / 32)) * 32;
-            tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * 2 * BN + acol), v);
-            if (A.bias != nullptr) add_bias32(v, A.bias, col0, A.V);
+          for (int jj = 0; jj < 2; ++jj) {
+            const int j = j0 + jj;
+            if (j >= it.s) break;
+            const int th = quad_half(it, j);
+            const int vb = (th >> 1) * BN + (th & 1) * kSubTile;  // the half's first vocabulary column
+            const int64_t rel = tg - vb;
+            const int tcol = (tvalid && rel >= 0 && rel < kSubTile) ? static_cast<int>(rel) : -1;  // -scale_r
+            const uint32_t blk = reg0 + static_cast<uint32_t>(jj * PART);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = sc_p * exp2f(fmaf(v[e], kLog2e, -lse_l2));
+            for (int c = 0; c < kSubTile / 32; ++c) {
+              float v[32];
+              const int col0 = vb + c * 32;
+              tmem_ld32(tmem_base + lane_off + static_cast<uint32_t>(a * 2 * BN + j * kSubTile + c * 32), v);
+              if (A.bias != nullptr) add_bias32(v, A.bias, col0, A.V);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if (c * 32 + e == tcol) v[e] -= sc_y;
-              if (col0 + e >= A.V) v[e] = 0.f;
-            }
-            const uint32_t blk = reg0 + static_cast<uint32_t>((c >> 1) * PART);
+              for (int e = 0; e < 32; ++e) v[e] = sc_p * exp2f(fmaf(v[e], kLog2e, -lse_l2));
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const int ch = (c & 1) * 4 + h;
-              st_shared_v4(blk + swz(row, ch), pack_bf16x2(v[8 * h + 0], v[8 * h + 1]),
-                           pack_bf16x2(v[8 * h + 2], v[8 * h + 3]), pack_bf16x2(v[8 * h + 4], v[8 * h + 5]),
-                           pack_bf16x2(v[8 * h + 6], v[8 * h + 7]));
-            }
-            if (A.dbias != nullptr) {  // dbias += column sums of G (this warp's 32 rows), fp32
-              const float cs = warp_column_sums32(v, lane);
-              if (col0 + lane < A.V && cs != 0.f) atomicAdd(A.dbias + col0 + lane, cs);
+              for (int e = 0; e < 32; ++e) {
+                if (c * 32 + e == tcol) v[e] -= sc_y;
+                if (col0 + e >= A.V) v[e] = 0.f;
+              }
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const int ch = c * 4 + h;
+                st_shared_v4(blk + swz(row, ch), pack_bf16x2(v[8 * h + 0], v[8 * h + 1]),
+                             pack_bf16x2(v[8 * h + 2], v[8 * h + 3]), pack_bf16x2(v[8 * h + 4], v[8 * h + 5]),
+                             pack_bf16x2(v[8 * h + 6], v[8 * h + 7]));
+              }
+              if (A.dbias != nullptr) {  // dbias += column sums of G (this warp's 32 rows), fp32
+                const float cs = warp_column_sums32(v, lane);
+                if (col0 + lane < A.V && cs != 0.f) atomicAdd(A.dbias + col0 + lane, cs);
+              }
             }
           }
           fence_proxy_async_smem();
@@ -567,9 +579,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!warp_wait(bar(kGReady), gphase & 1u)) {
               ok = false;
             } else if (leader) {
-              uint8_t* slot = buf + static_cast<size_t>(u == 0 ? it.slot0 : it.slot1) * TILE_BYTES;
-              for (int hf = 0; hf < 2; ++hf)
-                if ((hm >> hf) & 1) bulk_store(slot + hf * PART, reg0 + static_cast<uint32_t>(hf * PART), PART);
+              for (int jj = 0; jj < 2 && j0 + jj < it.s; ++jj) {  // each half into its tile's slot
+                const int th = quad_half(it, j0 + jj);
+                uint8_t* dst = buf + static_cast<size_t>(quad_slot(it, j0 + jj)) * TILE_BYTES + (th & 1) * PART;
+                bulk_store(dst, reg0 + static_cast<uint32_t>(jj * PART), PART);
+              }
               bulk_commit_group();
             }
           }
@@ -580,13 +594,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mbar_arrive(bar(kAccEmpty + a));
           ++acc_iter;
         }
-        // publish the pair's tiles to the dE / dC items that wait for them
+        // publish the quad's halves to the dE / dC items that wait for them
         if (leader && ok) {
           bulk_wait_group0();
           fence_proxy_async_global();
-          red_release_add(A.counters + A.ctr_g_b + it.chunk * A.nb + b, ntiles);
-          red_release_add(A.counters + A.ctr_g_t + it.begin, 1);
-          if (it.end >= 0) red_release_add(A.counters + A.ctr_g_t + it.end, 1);
+          red_release_add(A.counters + A.ctr_g_b + it.chunk * A.nb + b, it.s);
+          for (int j = 0; j < it.s; ++j) red_release_add(A.counters + A.ctr_g_t + (quad_half(it, j) >> 1), 1);
         }
         __syncwarp();
         if (*abort_flag) ok = false;
@@ -653,7 +666,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         red_release_add(A.counters + A.ctr_b_done + it.chunk, 1);
       }
       if (de && !has) continue;  // nothing to add for this row block in this chunk
-      // After a pair every warp's earlier bulk stores must have read the whole region; between dE / dC
+      // After a quad every warp's earlier bulk stores must have read the whole region; between dE / dC
       // items each warp only reuses its own staging images, which next_image() guards.
       if (region_shared && !region_free()) break;
       region_shared = false;

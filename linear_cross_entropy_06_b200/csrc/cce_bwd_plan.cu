@@ -18,9 +18,9 @@
 //   halves << kSlotBits), vocabulary tiles ascending; hp_b counts the kept halves before each entry.
 // Flat work lists the backward kernel reads with one load per item:
 //   rb_range[c * nb + b]   the entries [lo, hi) of row block b inside vocabulary chunk c;
-//   pair_desc/pair_slot    the pairs of consecutive listed tiles of a row block inside a chunk,
-//                          by the vocabulary tile of their first tile (pstart_t[t] is the first
-//                          pair starting in tile t, so a chunk's pairs are contiguous).
+//   quad_b/quad_h/quad_s   the quads (up to four consecutive kept halves of a row block inside a chunk),
+//                          by the vocabulary tile of their first half (pstart_t[t] is the first quad
+//                          starting in tile t, so a chunk's quads are contiguous).
 #include <algorithm>
 
 #include "cce_device.cuh"
@@ -264,42 +264,68 @@ __device__ __forceinline__ int lower_bound_t(const int2* e, int lo, int hi, int 
   return lo;
 }
 
-// A listed tile (b, t) starts a pair when its position in row block b's list inside t's chunk is
-// even; the pair is (b, t) and b's next listed tile in the chunk, if any. Pairs are listed by the
-// vocabulary tile of their first tile (then row block), so that the recompute of concurrent pairs
-// shares C tiles in L2. One warp per vocabulary tile; pass 0 counts the pairs starting in tile t
-// (into cnt_t, whose tile counts are already scanned into offsets_t), pass 1 (after the scan of
-// those counts into pstart_t) writes them.
-__device__ void pair_list_warp(const PlanArgs& A, int t, int lane, int pass) {
+// The recompute's items are quads: up to four consecutive kept halves of one row block inside a chunk,
+// from one or several of its listed tiles. A kept half starts a quad when its position among the kept
+// halves of its row block in the chunk (hp_b, counted from the row block's first entry there) is a
+// multiple of four. Quads are listed by the vocabulary tile of their first half (then row block), so
+// that the recompute of concurrent quads shares C rows in L2. One warp per vocabulary tile; pass 0
+// counts the quads starting in tile t (into cnt_t, whose tile counts are already scanned into
+// offsets_t), pass 1 (after the scan of those counts into pstart_t) writes them.
+__device__ void quad_list_warp(const PlanArgs& A, int t, int lane, int pass) {
   const BwdPlan& P = A.P;
-  const int nb = P.nb, nt = P.nt;
+  const int nb = P.nb;
   const int c = P.chunk_of[t];
   const int slot_base = P.offsets_t[P.chunk_t[c]];
   const int i0 = P.offsets_t[t], i1 = P.offsets_t[t + 1];
   int k = 0;
   for (int base = i0; base < i1; base += 32) {
     const int i = base + lane;
-    bool start = false;
-    int b = 0, p = 0;
+    int b = 0, p = 0, hm = 0, hrel = 0, nstart = 0;
     int2 rr = make_int2(0, 0);
     if (i < i1) {
-      b = P.entries_t[i].x >> 4;
+      const int x = P.entries_t[i].x;
+      b = x >> 4;
+      hm = flag_halves(x & 15);
       p = P.pos_b[i];
       rr = P.rb_range[static_cast<int64_t>(c) * nb + b];
-      start = ((p - rr.x) & 1) == 0;
+      hrel = P.hp_b[p] - P.hp_b[rr.x];  // kept halves of b in the chunk before this tile
+      for (int q = 0; q < __popc(hm); ++q) nstart += ((hrel + q) & 3) == 0 ? 1 : 0;
     }
-    const unsigned mask = __ballot_sync(0xffffffffu, start);
-    if (pass == 1 && start) {
-      const int out = P.pstart_t[t] + k + __popc(mask & ((1u << lane) - 1u));
-      const bool two = p + 1 < rr.y;
-      const int t1 = two ? P.entries_b[p + 1].x : -1;
-      const int slot1 = two ? (P.entries_b[p + 1].y & kSlotMask) : i;
-      const uint8_t* row = P.flags + static_cast<int64_t>(b) * nt;
-      const int kept = flag_halves(row[t]) | (two ? flag_halves(row[t1]) << 2 : 0);
-      P.pair_desc[out] = make_int4(b, t, t1, kept);
-      P.pair_slot[out] = make_int2(i - slot_base, slot1 - slot_base);
+    int incl = nstart;  // inclusive scan of the quad starts over the lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    k += __popc(mask);
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (pass == 1 && nstart > 0) {
+      int out = P.pstart_t[t] + k + incl - nstart;
+      for (int q = 0; q < __popc(hm); ++q) {
+        if (((hrel + q) & 3) != 0) continue;
+        // this tile's q-th kept half and the row block's next kept halves in the chunk, up to four
+        int th[4] = {-1, -1, -1, -1}, sl[4] = {0, 0, 0, 0};
+        int n = 0, skip = q;
+        for (int pp = p; pp < rr.y && n < 4; ++pp) {
+          const int2 e = P.entries_b[pp];
+          const int m = e.y >> kSlotBits;
+          for (int h = 0; h < 2 && n < 4; ++h) {
+            if (!((m >> h) & 1)) continue;
+            if (skip > 0) {
+              --skip;
+              continue;
+            }
+            th[n] = 2 * e.x + h;
+            sl[n] = (e.y & kSlotMask) - slot_base;
+            ++n;
+          }
+        }
+        P.quad_b[out] = b;
+        P.quad_h[out] = make_int4(th[0], th[1], th[2], th[3]);
+        P.quad_s[out] = make_int4(sl[0], sl[1], sl[2], sl[3]);
+        ++out;
+      }
+    }
+    k += total;
   }
   if (pass == 0 && lane == 0) P.cnt_t[t] = k;
 }
@@ -310,8 +336,8 @@ __device__ void pair_list_warp(const PlanArgs& A, int t, int lane, int pass) {
 //    written by bwd_finalize_kernel); both ascending.
 //  - de_list: the row blocks with a listed tile in the chunk (they get dE items), ascending.
 //  - empty_list: the chunk's empty tiles, appended to one list for the whole vocabulary.
-//  - grp_size: pairs(c) and dE/dC(c), at their places in the queue order pairs(0), then pairs(c) and
-//    dE/dC(c - 1) for c = 1 .. n-1, then dE/dC(n - 1): pairs(c) is group 2c - 1 (0 for c = 0) and
+//  - grp_size: quads(c) and dE/dC(c), at their places in the queue order quads(0), then quads(c) and
+//    dE/dC(c - 1) for c = 1 .. n-1, then dE/dC(n - 1): quads(c) is group 2c - 1 (0 for c = 0) and
 //    dE/dC(c) group min(2c + 2, 2n - 1).
 __device__ void chunk_items_block(const PlanArgs& A, int c, int nchunks) {
   __shared__ int em_base;
@@ -368,7 +394,7 @@ __device__ void chunk_items_block(const PlanArgs& A, int c, int nchunks) {
 // gradient tiles fit one buffer (at most chunk_g_tiles listed tiles) and the C rows its tiles read
 // stay within kChunkCBytes (at most chunk_c_tiles vocabulary tiles with a listed tile), so that a
 // sparse stretch of the vocabulary forms one long chunk: fewer chunks mean fewer partial sums of dE
-// and longer groups of pairs ahead of each chunk's dE / dC items. A chunk of the fixed length
+// and longer groups of quads ahead of each chunk's dE / dC items. A chunk of the fixed length
 // chunk_vt always satisfies both limits, so there are never more than P.nchunks chunks.
 // Greedy, decided by warp 0 over 32 vocabulary tiles at a time (the prefix sums offsets_t staged in
 // shared memory by the block): each lane tests whether its tile still fits the open chunk, and the
@@ -449,9 +475,9 @@ __device__ __forceinline__ int chunk_containing(const int* chunk_t, int n, int t
 //  4  entries_t; row lists (entries_b, hp_b, pos_b); the rows whose target half is skipped, grouped
 //     by vocabulary tile; the vocabulary chunks (one block)
 //  5  row ranges per chunk; the chunk of every vocabulary tile
-//  6  pair counts per vocabulary tile
-//  7  scan of the pair counts (pstart_t)
-//  8  pairs; chunk work lists and queue group sizes
+//  6  quad counts per vocabulary tile
+//  7  scan of the quad counts (pstart_t)
+//  8  quads; chunk work lists and queue group sizes
 //  9  scan of the group sizes (grp_start); the skipped count: by the last block to finish phase 8
 __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_constant__ PlanArgs A) {
   const BwdPlan& P = A.P;
@@ -535,6 +561,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     halves = __reduce_add_sync(0xffffffffu, halves);
     if (lane == 0) {
       P.cnt_t[t] = listed;
+      P.cnt_ht[t] = halves;
       atomicAdd(P.kept_total, halves);
     }
   }
@@ -591,7 +618,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
   zero_part(round + 1);
 
   // 6
-  for (int t = gwarp; t < nt; t += gwarps) pair_list_warp(A, t, lane, 0);
+  for (int t = gwarp; t < nt; t += gwarps) quad_list_warp(A, t, lane, 0);
   if (!grid_barrier(ctl, ++round)) return;
   zero_part(round + 1);
 
@@ -601,7 +628,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
   zero_part(round + 1);
 
   // 8
-  for (int t = gwarp; t < nt; t += gwarps) pair_list_warp(A, t, lane, 1);
+  for (int t = gwarp; t < nt; t += gwarps) quad_list_warp(A, t, lane, 1);
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x) chunk_items_block(A, c, nchunks);
   zero_part(9);
 

@@ -126,11 +126,13 @@ struct BwdPlan {
   int64_t chunk_c_tiles;  // vocabulary tiles with a listed tile a chunk may hold (kChunkCBytes of C)
   int64_t chunk_g_tiles;  // listed tiles a chunk may hold (one gradient-tile buffer)
   int2* rb_range;   // [nchunks * nb]: entries [lo, hi) of each row block inside each chunk
-  int* pstart_t;    // [nt + 1]: first pair whose first tile is in vocabulary tile t
-  int4* pair_desc;  // [pair capacity]: (b, t0, t1 or -1, kept halves: t0's in bits 0-1, t1's in 2-3),
-                    // by t0 then b
-  int2* pair_slot;  // [pair capacity]: gradient-tile slots of t0 and t1, relative to the chunk
-  int* grp_size;    // [2 * nchunks]: work items of each queue group (pairs of chunk c, then its dE/dC)
+  int* pstart_t;    // [nt + 1]: first quad whose first half is in vocabulary tile t
+  int* quad_b;      // [quad capacity]: row block of each quad (up to four kept halves of one row block
+                    // in a chunk), by the tile of its first half then row block
+  int4* quad_h;     // [quad capacity]: its halves, each 2 t + h (-1 when absent)
+  int4* quad_s;     // [quad capacity]: their tiles' gradient slots, relative to the chunk
+  int* cnt_ht;      // [nt]: kept halves of each vocabulary tile (over its listed row blocks)
+  int* grp_size;    // [2 * nchunks]: work items of each queue group (quads of chunk c, then its dE/dC)
   int* grp_start;   // [2 * nchunks + 1]: their prefix sums
   int* vt_order;    // [nt]: chunk c's vocabulary tiles at [chunk_t[c], chunk_t[c + 1]): first the ndc[c]
                     // with a listed tile (dC items), ascending, then the empty ones, ascending
@@ -173,8 +175,10 @@ struct BwdArgs {
   const int* nde;
   const int* chunk_t;
   const int* pstart_t;
-  const int4* pair_desc;
-  const int2* pair_slot;
+  const int* quad_b;
+  const int4* quad_h;
+  const int4* quad_s;
+  const int* cnt_ht;
   const int2* rb_range;
   const int* offsets_t;
   const int2* entries_t;
@@ -183,7 +187,7 @@ struct BwdArgs {
   const void* zero_half;  // 8 KB of zeros: the gradient of a skipped half, as the dC MMAs read it
   uint8_t* gscratch;
   int* qctr;      // queue position, zero at launch
-  int* counters;  // zero at launch: [ctr_g_b] gradient tiles stored per (chunk, row block),
+  int* counters;  // zero at launch: [ctr_g_b] gradient halves stored per (chunk, row block),
                   // [ctr_g_t] per vocabulary tile, [ctr_b_done] dE / dC items finished per chunk
   int ctr_g_b, ctr_g_t, ctr_b_done;
   int* err;
