@@ -49,12 +49,12 @@ KERNEL_SOURCES = {  # the kernel and what sets up its work (maps, plan, chunking
 }
 TRAFFIC_BYTES = {
     "fwd_lse_kernel": {
-        (4096, 4096, 128256): ("88deeb025a0b2e01974e376c5d1e0a0f628c3c281c1b57310147076a4a529f48",
-                               1085084928 + 67180288),
+        (4096, 4096, 128256): ("158f928c17a7c4f2ac351672a16cf5ff0ae7e1a20c3bf18e5ec48c64b97201a8",
+                               1085087488 + 66741504),
     },
     "bwd_kernel": {
-        (4096, 4096, 128256): ("6526e827035f2ab17d905cc8499f4fa38b38ab4ae3e922ffbe2df9989fd1a433",
-                               4313867520 + 1672815360),
+        (4096, 4096, 128256): ("4d69a6968d52397bb3e0a213507b3126563dcb1e2658304f5c6020a8e94f6f25",
+                               4550376192 + 1674573568),
     },
 }
 
