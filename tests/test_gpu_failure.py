@@ -3,7 +3,7 @@
 Forward: the kernel's producer is told (through a test-only environment switch, read at call
 time) to issue no loads, so the MMA warp's wait on the first stage gives up after
 CCE_WAIT_TIMEOUT_MS. Backward: the dE items of the first vocabulary chunk are told to wait for
-one gradient tile more than the recompute stores, so their wait on a counter raised by other
+one gradient half more than the recompute stores, so their wait on a counter raised by other
 CTAs gives up; the other CTAs see the recorded error and stop too. Planning: one block of the
 cooperative planning launch leaves before the first grid barrier, so the other blocks' wait there
 gives up. In every case the kernel records CCE_ERR_DEVICE_TIMEOUT and exits cleanly; the test
