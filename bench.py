@@ -194,7 +194,8 @@ def algorithmic_flops(N: int, D: int, V: int, kept_tiles: int, tile: tuple) -> t
 
 
 def listed_tile_count(skip_map) -> int:
-    """128 x 128 tiles with a kept 128 x 64 unit: the tiles whose dC MMAs run (over both halves)."""
+    """Backward tiles (128 x 128) with a kept 128 x 64 unit: the tiles whose dC MMAs run (over both
+    halves)."""
     kept = (skip_map == 0)
     if kept.shape[1] % 2:
         kept = torch.nn.functional.pad(kept, (0, 1))

@@ -94,12 +94,12 @@ constexpr int64_t kChunkCBytes = int64_t(128) << 20;
 // vocabulary tile; a chunk is written while the one before it is read) fit in the scratch: 4 MiB
 // per 128-row block, at least 128 MiB. The scratch grows with N, not with V, so that a chunk keeps
 // the same number of vocabulary tiles as N grows: each chunk adds a full N x D fp32 partial into
-// dE. The backward's queue places the dE/dC items of chunk c - 2 before the pairs of chunk c, so
+// dE. The backward's queue places the dE/dC items of chunk c - 2 before the quads of chunk c, so
 // two buffers are the fewest that keep every wait pointing to an earlier item.
 constexpr int64_t kGradScratchPerRowBlock = int64_t(4) << 20;
 constexpr int64_t kGradScratchMin = int64_t(128) << 20;
 constexpr int kGradBuffers = 2;
-static_assert(kGradBuffers >= 2, "the pairs of chunk c reuse the buffer of chunk c - kGradBuffers");
+static_assert(kGradBuffers >= 2, "the quads of chunk c reuse the buffer of chunk c - kGradBuffers");
 
 struct BwdPlan {
   int nb, nt;
@@ -231,7 +231,7 @@ struct PlanArgs {
   uint64_t timeout_ns;
   int inject_stall;        // test hook: block 0 leaves before the first grid barrier, whose wait then runs out
 };
-// One cooperative launch: the row scales, the tile flags, both tile lists, the pair list, the
+// One cooperative launch: the row scales, the tile flags, both tile lists, the quad list, the
 // chunks' work lists and queue groups, the onehot-only rows, and the skipped count.
 cudaError_t launch_bwd_plan(const PlanArgs& A, int num_sms, cudaStream_t s);
 // after_kernel: the previous operation on s is a kernel (the planning launch or a column sum).
