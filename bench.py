@@ -49,12 +49,12 @@ KERNEL_SOURCES = {  # the kernel and what sets up its work (maps, plan, chunking
 }
 TRAFFIC_BYTES = {
     "fwd_lse_kernel": {
-        (4096, 4096, 128256): ("158f928c17a7c4f2ac351672a16cf5ff0ae7e1a20c3bf18e5ec48c64b97201a8",
-                               1085087488 + 66741504),
+        (4096, 4096, 128256): ("2ed61cfe1a1a6ec72e48cd6d2754b958037681af0ba13cc5ce0ada1deecb2e2f",
+                               1085621248 + 67207680),
     },
     "bwd_kernel": {
-        (4096, 4096, 128256): ("4d69a6968d52397bb3e0a213507b3126563dcb1e2658304f5c6020a8e94f6f25",
-                               4550376192 + 1674573568),
+        (4096, 4096, 128256): ("d17440dea28d61347ec4d2753c760768a083030d6a3fd051d876eebdf64ec76e",
+                               4559904512 + 1673345536),
     },
 }
 
